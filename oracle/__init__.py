@@ -1,0 +1,118 @@
+"""fp64 CPU oracle for the KDA forward pass.
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline leg are the only callers.  The CUDA library never
+imports, links or calls anything here, and nothing here imports the library.
+
+The arithmetic lives in ``kda_oracle.c`` (plain C, fp64, token-by-token
+recurrence).  It follows the Kimi K3 technical-report digest
+(discuss.pytorch.kr), section "Kimi Delta Attention: delta rule with a
+per-channel forget gate", state-update equation
+``S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T``,
+``o_t = S_t^T q_t``, with ``alpha_t = exp(g_t)`` from the "Bounded decay"
+section.  This module only marshals arrays: it converts inputs to fp64
+exactly (bf16 and fp32 values are representable in fp64) and calls C.
+
+Every function is pinned by ``tests/test_oracle_pins.py``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "kda_oracle.c")
+_LIB = os.path.join(_HERE, "libkda_oracle.so")
+_lib = None
+
+_dp = ctypes.POINTER(ctypes.c_double)
+_i64p = ctypes.POINTER(ctypes.c_int64)
+
+
+def build(force: bool = False) -> str:
+    """Compile the C oracle in place (gcc, -O3, portable x86-64 code)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O3", "-fPIC", "-shared", "-std=c11", "-o", tmp, _SRC, "-lm", "-lpthread"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB)
+        lib.kda_oracle_fwd.restype = ctypes.c_int
+        lib.kda_oracle_fwd.argtypes = [_dp] * 8 + [ctypes.c_int, _i64p] + [ctypes.c_int] * 4
+        lib.kda_oracle_decode_step.restype = None
+        lib.kda_oracle_decode_step.argtypes = [_dp] * 7 + [ctypes.c_int] * 4
+        _lib = lib
+    return _lib
+
+
+def _f64(x) -> np.ndarray:
+    if hasattr(x, "detach"):  # torch tensor: exact widening on the host
+        x = x.detach().to("cpu")
+        import torch
+        x = x.to(torch.float64).numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(_dp)
+
+
+def default_threads() -> int:
+    return len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
+
+
+def fwd(q, k, v, g, beta, init_state=None, cu_seqlens=None, nthreads: int | None = None,
+        want_out: bool = True):
+    """Token-by-token fp64 KDA forward.
+
+    Shapes follow the library's layout: q,k,g ``[B,T,H,dk]``, v ``[B,T,H,dv]``,
+    beta ``[B,T,H]``, init_state ``[N,H,dk,dv]`` or None (zeros).  With
+    ``cu_seqlens`` (N+1 offsets) the tensors are packed ``[1,T_total,H,*]``
+    and each sequence starts from its own ``init_state[n]``.
+
+    Returns ``(out [B,T,H,dv], final_state [N,H,dk,dv])`` as float64 arrays.
+    """
+    lib = _load()
+    q, k, v, g, beta = (_f64(x) for x in (q, k, v, g, beta))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if cu_seqlens is None:
+        offsets = np.arange(B + 1, dtype=np.int64) * T
+    else:
+        offsets = np.ascontiguousarray(np.asarray(
+            cu_seqlens.cpu() if hasattr(cu_seqlens, "cpu") else cu_seqlens, dtype=np.int64))
+        assert B == 1, "packed inputs have batch dimension 1"
+    N = len(offsets) - 1
+    init = None if init_state is None else _f64(init_state)
+    out = np.zeros((B, T, H, dv), np.float64) if want_out else None
+    fin = np.zeros((N, H, dk, dv), np.float64)
+    lib.kda_oracle_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(init), _ptr(out),
+                       _ptr(fin), N, offsets.ctypes.data_as(_i64p), H, dk, dv,
+                       int(nthreads or default_threads()))
+    return out, fin
+
+
+def decode_step(q, k, v, g, beta, state):
+    """One in-place decode step on an fp64 state ``[B,H,dk,dv]`` (modified).
+
+    q,k,g ``[B,H,dk]``, v ``[B,H,dv]``, beta ``[B,H]``.  Returns out ``[B,H,dv]``.
+    """
+    lib = _load()
+    assert state.dtype == np.float64 and state.flags.c_contiguous
+    q, k, v, g, beta = (_f64(x) for x in (q, k, v, g, beta))
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    out = np.zeros((B, H, dv), np.float64)
+    lib.kda_oracle_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state),
+                               _ptr(out), B, H, dk, dv)
+    return out
