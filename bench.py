@@ -1,0 +1,383 @@
+#!/usr/bin/env python
+"""Benchmark of the KDA forward pass on B200 through the C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...      # the fp64 CPU oracle arm
+
+Default workload: the model-shaped prefill B=1, H=96, T=65536, dk=dv=128,
+bf16 q/k/v/o with fp32 log-decay, beta and state (the 64K pretraining
+context with the model's 96 heads).  One step = one kda_fwd over that batch.
+The same run also times the B=512, H=96 single-token decode (one
+kda_decode_step per step, state updated in place) and reports it under
+"decode".  Inputs are synthetic (seeded), resident in HBM before the timed
+region, and far larger than the 126 MB L2, so no flush is needed.
+
+Metric: Mtoken-heads/s = tokens x heads / time / 1e6, plus the fraction of
+the HBM roofline (measured copy bandwidth from MEASURED_PEAKS.json).
+
+Multi-GPU (torchrun): every rank runs its own copy of the workload (the
+heads and sequences are independent chains, so no data-path collective);
+per-GPU work is fixed ("weak" scaling) and the value counts all ranks' work
+over the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "KDA fwd Mtoken-heads/s at H=96,d=128 (prefill & decode); % of roofline"
+UNIT = "Mtoken-heads/s"
+CHUNK = 64
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def prefill_bytes(tokens_heads, chains, dk, dv, io_bytes, with_init):
+    """Algorithmic HBM bytes of one forward: q,k,v,o in the I/O dtype, fp32
+    log-decay and beta, plus the fp32 final state (and initial state)."""
+    per_th = io_bytes * (2 * dk + 2 * dv) + 4 * dk + 4
+    return tokens_heads * per_th + chains * dk * dv * 4 * (2 if with_init else 1)
+
+
+def prefill_flops(tokens_heads, dk, dv, C=CHUNK):
+    """Chunk-method flops per token-head: state products (W S, Q S, K^T Delta)
+    6 dk dv, intra-chunk Gram/WY/output work C (6 dk + 4 dv), solve C^2/3."""
+    return tokens_heads * (6 * dk * dv + C * (6 * dk + 4 * dv) + C * C / 3)
+
+
+def decode_bytes(B, H, dk, dv, io_bytes):
+    return B * H * (2 * dk * dv * 4 + io_bytes * (2 * dk + 2 * dv) + 4 * dk + 4)
+
+
+def tc_kernel_sha():
+    src = os.path.join(ROOT, "gated_delta_rule_121_b200", "csrc", "kda_fwd_tc.cu")
+    return hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+
+
+def profiled_traffic(workload):
+    """DRAM bytes per launch of the tensor-core kernel from the committed ncu
+    summary, or None when it is missing or the kernel changed since."""
+    p = os.path.join(ROOT, "profiles", f"kda_fwd_tc_{workload}_traffic.txt")
+    if not os.path.exists(p):
+        return None
+    kv = {}
+    for line in open(p):
+        if "=" in line and not line.startswith("#"):
+            k, v = line.strip().split("=", 1)
+            kv[k.strip()] = v.strip()
+    if kv.get("kernel_source_sha256") != tc_kernel_sha():
+        return None
+    try:
+        return float(kv["traffic_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples while the timed region runs."""
+    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.hw_slowdown",
+              "clocks_event_reasons.hw_thermal_slowdown", "clocks_event_reasons.sw_thermal_slowdown",
+              "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, uuid):
+        self.uuid, self.proc, self.lines = uuid, None, []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.uuid, "--query-gpu=" + ",".join(self.FIELDS),
+                 "--format=csv,noheader,nounits", "-lms", "50"], stdout=subprocess.PIPE,
+                stderr=subprocess.DEVNULL, text=True)
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.1)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in self.lines:
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 7:
+                continue
+            try:
+                sm.append(float(f[0]))
+                mx.append(float(f[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def time_loop(fn, steps, warmup, stream, dist_ctx):
+    import torch
+    for _ in range(warmup):
+        fn()
+    dist_ctx.barrier()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(steps):
+        fn()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    dist_ctx.barrier()
+    return dist_ctx.max(t0.elapsed_time(t1) / 1000.0)
+
+
+class Dist:
+    def __init__(self):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+
+    def init(self, backend):
+        if self.world > 1:
+            import datetime
+            import torch.distributed as dist
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+            self.pg = dist
+
+    def barrier(self):
+        if self.pg is not None:
+            self.pg.barrier()
+
+    def max(self, x):
+        if self.pg is None:
+            return x
+        import torch
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg is not None:
+            self.pg.destroy_process_group()
+
+
+def workload_spec(name):
+    import synth
+    return {"prefill64k": synth.PRETRAIN, "mid": synth.MID, "varlen": synth.VARLEN,
+            "stress": synth.STRESS}[name]
+
+
+# ----------------------------------------------------------------- oracle arm
+def oracle_sample(spec, budget_s, threads):
+    """Oracle throughput on a bounded sample of the workload: the first H_s
+    heads and T_s tokens of one sequence, sized to ~budget_s seconds."""
+    import oracle
+    import synth
+    H_s = max(1, min(spec.H, threads))
+    cal = synth.make_prefill(spec, "cpu", T=256, B=1, H=1, lengths=[256] if spec.varlen else None)
+    t = time.perf_counter()
+    oracle.fwd(cal["q"], cal["k"], cal["v"], cal["g"], cal["beta"], None, cal["cu_seqlens"], nthreads=1)
+    per_tok = (time.perf_counter() - t) / 256
+    par = min(threads, H_s)
+    T_s = int(max(64, min(spec.T if not spec.varlen else 262144, budget_s * par / (H_s * per_tok))))
+    inp = synth.make_prefill(spec, "cpu", T=T_s, B=1, H=H_s, lengths=[T_s] if spec.varlen else None)
+    t = time.perf_counter()
+    oracle.fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["init_state"], inp["cu_seqlens"],
+               nthreads=threads)
+    el = time.perf_counter() - t
+    return dict(value=H_s * T_s / el / 1e6, unit=UNIT, cores=min(threads, H_s), kind="oracle",
+                sample=f"{H_s} heads x {T_s} tokens of one sequence ({spec.name}), fp64 C recurrence",
+                seconds=el)
+
+
+def run_reference(args, d):
+    import oracle
+    spec = workload_spec(args.workload)
+    if d.rank != 0:
+        return
+    threads = oracle.default_threads()
+    budget = max(1.0, min(8.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample(spec, budget, threads)
+    vals, secs = [], 0.0
+    last = None
+    for _ in range(args.steps):
+        last = oracle_sample(spec, budget, threads)
+        vals.append(last["value"])
+        secs += last["seconds"]
+    v = statistics.median(vals)
+    cb = dict(last)
+    cb["value"] = v
+    cb.pop("seconds", None)
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * secs / max(1, args.steps),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": spec.name, "sample": cb["sample"]},
+            "cpu_baseline": cb, "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0,
+                                        "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------- native arm
+def run_native(args, d):
+    import torch
+
+    import gated_delta_rule_121_b200 as kda
+    import synth
+
+    torch.cuda.set_device(d.local)
+    dev = torch.device("cuda", d.local)
+    d.init("nccl")
+    peaks, peak_src = load_peaks()
+    spec = workload_spec(args.workload)
+    stream = torch.cuda.current_stream(dev)
+
+    inp = synth.make_prefill(spec, dev)
+    q, k, v, g, beta, init, cu = (inp[n] for n in ("q", "k", "v", "g", "beta", "init_state", "cu_seqlens"))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    N = cu.numel() - 1 if cu is not None else B
+    tokens = B * T
+    th = tokens * H
+    out = torch.empty_like(v)
+    fin = torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev)
+    ws = kda.alloc_workspace(N, tokens, H, dk, dv, q.dtype, dev)
+    io_bytes = q.element_size()
+
+    def step():
+        kda.kda_fwd(q, k, v, g, beta, init, cu, out=out, final_state=fin, workspace=ws, stream=stream)
+
+    uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid).replace("GPU-", "")
+    with ClockSampler(uuid) as clk:
+        sec = time_loop(step, args.steps, args.warmup, stream, d)
+    status = kda.kda_workspace_status(ws, stream)
+    if status != kda.KDA_OK:
+        raise RuntimeError(f"device status {kda.kda_status_string(status)}")
+    per_step = sec / args.steps
+    value = d.world * th * args.steps / sec / 1e6
+    bytes_alg = prefill_bytes(th, N * H, dk, dv, io_bytes, init is not None)
+    flops_alg = prefill_flops(th, dk, dv)
+    achieved = bytes_alg / per_step / 1e9
+    peak = peaks["hbm_gbs"]
+    t_roof = max(bytes_alg / (peak * 1e9), flops_alg / (peaks["bf16_tflops"] * 1e12))
+    traffic = profiled_traffic(args.workload)
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": d.world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": per_step * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16" if q.dtype == torch.bfloat16 else "f32", "data": "synthetic",
+            "config": {"workload": spec.name, "B": B, "T": T, "H": H, "dk": dk, "dv": dv, "sequences": N,
+                       "chunk": CHUNK, "l2": "inputs larger than L2 (%.1f GB per step), no flush" %
+                       (bytes_alg / 1e9), "parallelism": f"dp{d.world} independent replicas, no collective"},
+            "pct_of_roofline": 100.0 * t_roof / per_step,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": traffic, "peak_source": peak_src,
+                         "bytes_per_launch": bytes_alg, "kernel": "kda_fwd_tc_kernel",
+                         "tensor_tflops": flops_alg / per_step / 1e12,
+                         "tensor_frac_of_bf16_peak": flops_alg / per_step / 1e12 / peaks["bf16_tflops"]},
+            "gpu_launches": args.steps, "clocks": clk.summary()}
+
+    if not args.no_decode:
+        line["decode"] = bench_decode(args, d, dev, stream, peaks, kda, synth)
+    if not args.no_e2e:
+        line["e2e"] = bench_e2e(args, d, dev, stream, inp, kda, th)
+    if d.world == 1 and d.rank == 0 and not args.no_cpu_baseline:
+        import oracle
+        line["cpu_baseline"] = {k: v for k, v in oracle_sample(spec, 12.0, oracle.default_threads()).items()
+                                if k != "seconds"}
+    if d.rank == 0:
+        print(json.dumps(line), flush=True)
+    d.close()
+
+
+def bench_decode(args, d, dev, stream, peaks, kda, synth):
+    import torch
+    spec = synth.DECODE
+    state = synth.make_decode_state(spec, dev)
+    n_in = args.warmup + args.steps
+    xs = [synth.make_decode_step(spec, s, dev) for s in range(n_in)]
+    out = torch.empty((spec.B, spec.H, spec.dv), dtype=spec.dtype, device=dev)
+    it = iter(range(10 ** 9))
+
+    def step():
+        x = xs[next(it) % n_in]
+        kda.kda_decode_step(x["q"], x["k"], x["v"], x["g"], x["beta"], state, out=out, stream=stream)
+
+    sec = time_loop(step, args.steps, args.warmup, stream, d)
+    per = sec / args.steps
+    nbytes = decode_bytes(spec.B, spec.H, spec.dk, spec.dv, 2)
+    ach = nbytes / per / 1e9
+    del xs, state
+    return {"workload": spec.name, "value": d.world * spec.B * spec.H * args.steps / sec / 1e6, "unit": UNIT,
+            "ms_per_step": per * 1e3, "gpu_launches": args.steps,
+            "roofline": {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": ach / peaks["hbm_gbs"], "traffic": None, "bytes_per_launch": nbytes,
+                         "kernel": "kda_decode_kernel<128,128,bf16>"}}
+
+
+def bench_e2e(args, d, dev, stream, inp, kda, th):
+    """Same metric through the public API from pinned host buffers: every
+    step copies the inputs host->device and the output and final state back."""
+    import torch
+    host = {n: (t.cpu().pin_memory() if t is not None else None) for n, t in inp.items()}
+    bufs = {}
+    steps = max(1, min(args.steps, 5))
+
+    def step():
+        o, f, _ = kda.kda_fwd_host(host["q"], host["k"], host["v"], host["g"], host["beta"], host["init_state"],
+                                   host["cu_seqlens"], device=dev, stream=stream, dev_buffers=bufs)
+
+    sec = time_loop(step, steps, 1, stream, d)
+    h2d = sum(t.numel() * t.element_size() for n, t in host.items() if t is not None)
+    d2h = bufs["out_h"].numel() * bufs["out_h"].element_size() + bufs["fin_h"].numel() * 4
+    return {"value": d.world * th * steps / sec / 1e6, "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": steps, "ms_per_step": sec / steps * 1e3}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--workload", choices=["prefill64k", "mid", "varlen", "stress"], default="prefill64k")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
+    d = Dist()
+    if args.impl == "reference":
+        run_reference(args, d)
+    else:
+        run_native(args, d)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,205 @@
+"""Python binding of libkda.so, the B200 (sm_100a) KDA forward library.
+
+Argument marshalling only: every step of the forward pass runs in the CUDA
+kernels behind the C ABI (include/kda.h).  PyTorch supplies device memory
+and streams.  There is no CPU fallback: if the shared library cannot be
+loaded, every call raises.
+
+Functions mirror the C entry points:
+  kda_fwd(q, k, v, log_alpha, beta, ...)        chunked prefill
+  kda_decode_step(q, k, v, log_alpha, beta, state, ...)   in-place decode
+  kda_fwd_workspace_size(...), kda_workspace_status(ws), kda_status_string(s)
+and ``kda_fwd_host`` runs kda_fwd on host (pinned) tensors, copying inputs in
+and outputs back on the given stream.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libkda.so")
+
+KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_WORKSPACE, KDA_ERR_CUDA, KDA_ERR_TIMEOUT = range(6)
+KDA_F32, KDA_BF16 = 0, 1
+_DT = {torch.float32: KDA_F32, torch.bfloat16: KDA_BF16}
+
+_lib = None
+_vp, _fp, _i32p = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p
+
+
+class KdaError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {kda_status_string(code)}")
+        self.code = code
+
+
+def lib() -> ctypes.CDLL:
+    """Load libkda.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: run `python -m gated_delta_rule_121_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        L.kda_version.restype = ctypes.c_int
+        L.kda_status_string.restype = ctypes.c_char_p
+        L.kda_status_string.argtypes = [ctypes.c_int]
+        L.kda_fwd_workspace_size.restype = ctypes.c_size_t
+        L.kda_fwd_workspace_size.argtypes = [ctypes.c_int, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
+                                             ctypes.c_int, ctypes.c_int]
+        fwd_args = [_vp, _vp, _vp, _fp, _fp, _fp, _vp, _fp, ctypes.c_int, ctypes.c_int64, ctypes.c_int,
+                    ctypes.c_int, ctypes.c_int, _i32p, _vp, ctypes.c_int, _vp, ctypes.c_size_t]
+        L.kda_fwd.restype = ctypes.c_int
+        L.kda_fwd.argtypes = fwd_args
+        L.kda_testing_fwd.restype = ctypes.c_int
+        L.kda_testing_fwd.argtypes = fwd_args + [_fp, ctypes.c_uint64]
+        L.kda_testing_debug_floats.restype = ctypes.c_int
+        L.kda_testing_fwd_path.restype = ctypes.c_int
+        L.kda_testing_fwd_path.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int]
+        L.kda_decode_step.restype = ctypes.c_int
+        L.kda_decode_step.argtypes = [_vp, _vp, _vp, _fp, _fp, _fp, _vp, ctypes.c_int, ctypes.c_int,
+                                      ctypes.c_int, ctypes.c_int, _vp, ctypes.c_int]
+        L.kda_workspace_status.restype = ctypes.c_int
+        L.kda_workspace_status.argtypes = [_vp, _vp]
+        _lib = L
+    return _lib
+
+
+def kda_status_string(code: int) -> str:
+    return lib().kda_status_string(int(code)).decode()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_ptr(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(code, what):
+    if code != KDA_OK:
+        raise KdaError(code, what)
+
+
+def kda_fwd_workspace_size(B, T, H, dk, dv, dtype=torch.bfloat16) -> int:
+    return int(lib().kda_fwd_workspace_size(B, T, H, dk, dv, _DT[dtype]))
+
+
+def alloc_workspace(B, T, H, dk, dv, dtype=torch.bfloat16, device="cuda") -> torch.Tensor:
+    n = kda_fwd_workspace_size(B, T, H, dk, dv, dtype)
+    return torch.empty(max(n, 16), dtype=torch.uint8, device=device)
+
+
+def kda_workspace_status(workspace: torch.Tensor, stream=None) -> int:
+    return int(lib().kda_workspace_status(_ptr(workspace), _stream_ptr(stream)))
+
+
+def _shapes(q, v, cu_seqlens):
+    if q.dim() != 4:
+        raise ValueError("q must be [B, T, H, dk]")
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if cu_seqlens is not None:
+        if B != 1:
+            raise ValueError("packed (cu_seqlens) inputs must have batch dimension 1")
+        N = cu_seqlens.numel() - 1
+    else:
+        N = B
+    return B, T, H, dk, dv, N
+
+
+def kda_fwd(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None, out=None, final_state=None,
+            output_final_state=True, workspace=None, stream=None, _debug=None, _wait_ns=None):
+    """KDA forward over whole sequences (see include/kda.h, kda_fwd).
+
+    q, k, log_alpha: [B,T,H,dk]; v: [B,T,H,dv]; beta: [B,T,H]; q/k/v share a
+    dtype (bf16 or fp32); log_alpha, beta and states are fp32.  Returns
+    ``(out, final_state)``; final_state is None when not requested.
+    """
+    B, T, H, dk, dv, N = _shapes(q, v, cu_seqlens)
+    dt = _DT[q.dtype]
+    for name, t, dtype in (("k", k, q.dtype), ("v", v, q.dtype), ("log_alpha", log_alpha, torch.float32),
+                           ("beta", beta, torch.float32)):
+        if t.dtype != dtype or not t.is_contiguous() or t.device != q.device:
+            raise ValueError(f"{name}: expected contiguous {dtype} on {q.device}")
+    if init_state is not None and (init_state.dtype != torch.float32 or not init_state.is_contiguous()
+                                   or tuple(init_state.shape) != (N, H, dk, dv)):
+        raise ValueError("init_state must be contiguous fp32 [N, H, dk, dv]")
+    if cu_seqlens is not None and cu_seqlens.dtype != torch.int32:
+        raise ValueError("cu_seqlens must be int32")
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    if final_state is None and output_final_state:
+        final_state = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = alloc_workspace(N, B * T, H, dk, dv, q.dtype, q.device)
+    Targ = T if cu_seqlens is None else T  # packed: T is the total token count
+    args = (_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(init_state), _ptr(out),
+            _ptr(final_state), N, Targ, H, dk, dv, _ptr(cu_seqlens), _stream_ptr(stream), dt,
+            _ptr(workspace), workspace.numel())
+    if _debug is None and _wait_ns is None:
+        code = lib().kda_fwd(*args)
+    else:
+        code = lib().kda_testing_fwd(*args, _ptr(_debug), int(_wait_ns if _wait_ns is not None else 2_000_000_000))
+    _check(code, "kda_fwd")
+    return out, final_state
+
+
+def kda_decode_step(q, k, v, log_alpha, beta, state, out=None, stream=None):
+    """One decode step; ``state`` [B,H,dk,dv] fp32 is updated in place.
+    q,k,log_alpha: [B,H,dk]; v: [B,H,dv]; beta: [B,H].  Returns out [B,H,dv]."""
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    if state.dtype != torch.float32 or not state.is_contiguous() or tuple(state.shape) != (B, H, dk, dv):
+        raise ValueError("state must be contiguous fp32 [B, H, dk, dv]")
+    for name, t in (("k", k), ("v", v), ("log_alpha", log_alpha), ("beta", beta)):
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    if out is None:
+        out = torch.empty((B, H, dv), dtype=q.dtype, device=q.device)
+    code = lib().kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(state), _ptr(out),
+                                 B, H, dk, dv, _stream_ptr(stream), _DT[q.dtype])
+    _check(code, "kda_decode_step")
+    return out
+
+
+def kda_fwd_host(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None, device="cuda", stream=None,
+                 dev_buffers=None):
+    """kda_fwd on host tensors (pinned for asynchronous copies): copies the
+    inputs to ``device``, runs the forward and copies ``out`` and the final
+    state back.  ``dev_buffers`` (a dict returned by a previous call) lets
+    repeated calls reuse device memory.  Returns (out_host, final_host,
+    dev_buffers)."""
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    if dev_buffers is None:
+        dev_buffers = {}
+    def dev(name, t):
+        if t is None:
+            return None
+        b = dev_buffers.get(name)
+        if b is None or b.shape != t.shape or b.dtype != t.dtype:
+            b = dev_buffers[name] = torch.empty(t.shape, dtype=t.dtype, device=device)
+        b.copy_(t, non_blocking=True)
+        return b
+    with torch.cuda.stream(s):
+        dq, dk_, dv_, dg, db = (dev(n, t) for n, t in (("q", q), ("k", k), ("v", v), ("g", log_alpha),
+                                                        ("beta", beta)))
+        di = dev("init", init_state)
+        dcu = dev("cu", cu_seqlens)
+        B, T, H, dk, dv, N = _shapes(q, v, cu_seqlens)
+        if "out" not in dev_buffers or dev_buffers["out"].shape != (B, T, H, dv):
+            dev_buffers["out"] = torch.empty((B, T, H, dv), dtype=q.dtype, device=device)
+            dev_buffers["fin"] = torch.empty((N, H, dk, dv), dtype=torch.float32, device=device)
+            dev_buffers["ws"] = alloc_workspace(N, B * T, H, dk, dv, q.dtype, device)
+        kda_fwd(dq, dk_, dv_, dg, db, di, dcu, out=dev_buffers["out"], final_state=dev_buffers["fin"],
+                workspace=dev_buffers["ws"], stream=s)
+        if "out_h" not in dev_buffers or dev_buffers["out_h"].shape != (B, T, H, dv):
+            dev_buffers["out_h"] = torch.empty((B, T, H, dv), dtype=q.dtype, pin_memory=True)
+            dev_buffers["fin_h"] = torch.empty((N, H, dk, dv), dtype=torch.float32, pin_memory=True)
+        dev_buffers["out_h"].copy_(dev_buffers["out"], non_blocking=True)
+        dev_buffers["fin_h"].copy_(dev_buffers["fin"], non_blocking=True)
+    return dev_buffers["out_h"], dev_buffers["fin_h"], dev_buffers

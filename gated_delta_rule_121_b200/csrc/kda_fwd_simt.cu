@@ -1,0 +1,146 @@
+// Token-serial KDA forward on CUDA cores, exact fp32 arithmetic.
+//
+// This path serves fp32 inputs (whose accuracy contract forbids rounding
+// operands to TF32 or bf16) and the (dk, dv) shapes that have no tensor-core
+// kernel.  It runs the recurrence of the Kimi K3 digest's "Kimi Delta
+// Attention" section token by token:
+//   S' = Diag(exp g_t) S;  u = S'^T k_t;  S = S' + beta_t k_t (v_t - u)^T;
+//   o_t = S^T q_t.
+//
+// Work split: one block per (sequence, head, 32-column block of dv).  Columns
+// of S evolve independently (each v-channel sees the same k, g, beta), so
+// the dv split needs no communication.  Within a block, a warp owns 8
+// columns; its 32 lanes are 8 columns x 4 row groups, and lane (rg, j) keeps
+// rows i = 4m + rg of column j in registers.  Both per-token reductions over
+// rows (u and o) are 4-lane shuffles inside the warp, so the token loop has
+// no block barrier; barriers appear only when a chunk of TOK tokens is
+// staged in shared memory.
+#include "kda_internal.cuh"
+
+namespace kda {
+namespace {
+
+constexpr int TOK = 16;  // tokens staged per shared-memory round
+
+template <int DK, int DVB, typename IO>
+__global__ void __launch_bounds__(DVB * 4)
+    kda_fwd_simt_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO* __restrict__ v,
+                        const float* __restrict__ g, const float* __restrict__ beta,
+                        const float* __restrict__ init, IO* __restrict__ out, float* __restrict__ fin,
+                        const int32_t* __restrict__ cu, int64_t Tper, int H, int dv) {
+  constexpr int R = DK / 4;  // rows per lane
+  constexpr int NT = DVB * 4;
+  __shared__ float s_k[TOK][DK], s_q[TOK][DK], s_a[TOK][DK];
+  __shared__ float s_v[TOK][DVB], s_b[TOK], s_o[TOK][DVB];
+
+  const int nblk = dv / DVB;
+  const int blk = blockIdx.x % nblk;
+  const int h = (blockIdx.x / nblk) % H;
+  const int n = blockIdx.x / (nblk * H);
+  int64_t t0, L;
+  if (cu) {
+    t0 = cu[n];
+    L = (int64_t)cu[n + 1] - t0;
+  } else {
+    t0 = (int64_t)n * Tper;
+    L = Tper;
+  }
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int rg = lane >> 3, jc = lane & 7;
+  const int jl = warp * 8 + jc;       // column within the block
+  const int j = blk * DVB + jl;       // column of S / v / o
+  const int64_t sbase = ((int64_t)n * H + h) * DK * dv;
+
+  float s[R];
+#pragma unroll
+  for (int m = 0; m < R; ++m) s[m] = init ? init[sbase + (int64_t)(4 * m + rg) * dv + j] : 0.f;
+
+  for (int64_t c0 = 0; c0 < L; c0 += TOK) {
+    const int nt = (int)((L - c0) < TOK ? (L - c0) : TOK);
+    __syncthreads();
+    for (int e = tid; e < TOK * DK; e += NT) {
+      const int r = e / DK, i = e % DK;
+      float kk = 0.f, qq = 0.f, aa = 1.f;
+      if (r < nt) {
+        const int64_t row = ((t0 + c0 + r) * H + h) * DK + i;
+        kk = to_f32(k[row]);
+        qq = to_f32(q[row]);
+        aa = __expf(g[row]);
+      }
+      s_k[r][i] = kk; s_q[r][i] = qq; s_a[r][i] = aa;
+    }
+    for (int e = tid; e < TOK * DVB; e += NT) {
+      const int r = e / DVB, c = e % DVB;
+      s_v[r][c] = r < nt ? to_f32(v[((t0 + c0 + r) * H + h) * dv + blk * DVB + c]) : 0.f;
+    }
+    if (tid < TOK) s_b[tid] = tid < nt ? beta[(t0 + c0 + tid) * H + h] : 0.f;
+    __syncthreads();
+
+    for (int r = 0; r < nt; ++r) {
+      float pu = 0.f;
+#pragma unroll
+      for (int m = 0; m < R; ++m) {
+        const int i = 4 * m + rg;
+        s[m] *= s_a[r][i];
+        pu += s[m] * s_k[r][i];
+      }
+      pu += __shfl_xor_sync(0xffffffffu, pu, 8);
+      pu += __shfl_xor_sync(0xffffffffu, pu, 16);
+      const float d = s_b[r] * (s_v[r][jl] - pu);
+      float po = 0.f;
+#pragma unroll
+      for (int m = 0; m < R; ++m) {
+        const int i = 4 * m + rg;
+        s[m] += s_k[r][i] * d;
+        po += s[m] * s_q[r][i];
+      }
+      po += __shfl_xor_sync(0xffffffffu, po, 8);
+      po += __shfl_xor_sync(0xffffffffu, po, 16);
+      if (rg == 0) s_o[r][jl] = po;
+    }
+    __syncthreads();
+    for (int e = tid; e < nt * DVB; e += NT) {
+      const int r = e / DVB, c = e % DVB;
+      out[((t0 + c0 + r) * H + h) * dv + blk * DVB + c] = from_f32<IO>(s_o[r][c]);
+    }
+  }
+  if (fin) {
+#pragma unroll
+    for (int m = 0; m < R; ++m) fin[sbase + (int64_t)(4 * m + rg) * dv + j] = s[m];
+  }
+}
+
+template <int DK, typename IO>
+cudaError_t launch_k(const FwdArgs& a, cudaStream_t st) {
+  const int DVB = a.dv < 32 ? a.dv : 32;
+  const unsigned blocks = (unsigned)((int64_t)a.N * a.H * (a.dv / DVB));
+  if (blocks == 0) return cudaSuccess;
+  const int64_t Tper = a.cu ? 0 : a.T;
+#define KDA_SIMT_LAUNCH(DVB_)                                                                            \
+  kda_fwd_simt_kernel<DK, DVB_, IO><<<blocks, DVB_ * 4, 0, st>>>(                                        \
+      (const IO*)a.q, (const IO*)a.k, (const IO*)a.v, a.g, a.beta, a.init, (IO*)a.out, a.fin, a.cu, Tper, \
+      a.H, a.dv)
+  if (DVB == 16) KDA_SIMT_LAUNCH(16);
+  else KDA_SIMT_LAUNCH(32);
+#undef KDA_SIMT_LAUNCH
+  return cudaGetLastError();
+}
+
+template <typename IO>
+cudaError_t launch_io(const FwdArgs& a, cudaStream_t s) {
+  switch (a.dk) {
+    case 16: return launch_k<16, IO>(a, s);
+    case 32: return launch_k<32, IO>(a, s);
+    case 64: return launch_k<64, IO>(a, s);
+    case 128: return launch_k<128, IO>(a, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+cudaError_t launch_fwd_simt(const FwdArgs& a, bool bf16, cudaStream_t s) {
+  return bf16 ? launch_io<__nv_bfloat16>(a, s) : launch_io<float>(a, s);
+}
+
+}  // namespace kda

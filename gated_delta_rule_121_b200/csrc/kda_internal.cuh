@@ -1,0 +1,59 @@
+// Internal declarations shared by the KDA CUDA sources (not part of the ABI).
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+#include "../../include/kda.h"
+
+namespace kda {
+
+// Status word at the start of every kda_fwd workspace.  Kernels record the
+// first device-side failure here (atomicCAS from KDA_OK).
+struct DeviceStatus {
+  int code;
+  int where;  // which wait gave up (kernel-specific id), for diagnostics
+  int pad[2];
+};
+
+__device__ __forceinline__ void record_error(DeviceStatus* st, int code, int where) {
+  if (st && atomicCAS(&st->code, KDA_OK, code) == KDA_OK) st->where = where;
+}
+
+template <typename T> __device__ __forceinline__ float to_f32(T x);
+template <> __device__ __forceinline__ float to_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) {
+  return __bfloat162float(x);
+}
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+// Arguments of one forward call after host-side validation.
+struct FwdArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* g;
+  const float* beta;
+  const float* init;
+  void* out;
+  float* fin;
+  const int32_t* cu;  // device offsets or nullptr
+  int N;              // number of sequences
+  int64_t T;          // tokens per sequence (cu == nullptr) or total tokens
+  int H, dk, dv;
+  DeviceStatus* status;
+  void* dbg;          // optional debug dump (test hook), may be nullptr
+};
+
+// Launchers (return a CUDA error code; launches are asynchronous).
+cudaError_t launch_decode(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                          float* state, void* out, int B, int H, int dk, int dv, bool bf16, cudaStream_t s);
+cudaError_t launch_fwd_simt(const FwdArgs& a, bool bf16, cudaStream_t s);
+bool fwd_tc_supported(int dk, int dv, bool bf16);
+cudaError_t launch_fwd_tc(const FwdArgs& a, cudaStream_t s);
+
+}  // namespace kda

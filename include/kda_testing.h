@@ -1,0 +1,46 @@
+/*
+ * kda_testing.h — test hooks exported by libkda.so.  Not part of the stable
+ * ABI in kda.h; used by the library's own tests to look inside a forward
+ * call.  These hooks compute nothing the public entry points do not.
+ */
+#ifndef KDA_TESTING_H_
+#define KDA_TESTING_H_
+
+#include "kda.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Number of floats kda_testing_fwd writes to debug_out. */
+KDA_API int kda_testing_debug_floats(void);
+
+/*
+ * Same as kda_fwd, plus:
+ *   debug_out  device fp32 buffer of kda_testing_debug_floats() floats or
+ *              NULL.  When set (tensor-core path only, else
+ *              KDA_ERR_UNSUPPORTED), the block of chain 0 writes the
+ *              intermediates of its first chunk: P, A, T', W, U, Delta, O,
+ *              the state after the chunk and the chunk-total log-decay.
+ *   wait_ns    bound for every device-side wait in nanoseconds (kda_fwd
+ *              uses 2e9).  A bound of 0 makes the first wait that is not
+ *              already satisfied give up, which exercises the timeout path
+ *              (status KDA_ERR_TIMEOUT in the workspace) without faulting or
+ *              hanging the GPU: the kernel then drains its own copies and
+ *              tensor-core work with the normal bound and exits.
+ */
+KDA_API kda_status_t kda_testing_fwd(const void *q, const void *k, const void *v,
+                             const float *log_alpha, const float *beta,
+                             const float *init_state, void *out, float *final_state,
+                             int B, int64_t T, int H, int dk, int dv,
+                             const int32_t *cu_seqlens, void *stream, kda_dtype_t dt,
+                             void *workspace, size_t workspace_bytes,
+                             float *debug_out, uint64_t wait_ns);
+
+/* 1 when kda_fwd uses the tensor-core kernel for this shape, else 0. */
+KDA_API int kda_testing_fwd_path(int dk, int dv, kda_dtype_t dt);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* KDA_TESTING_H_ */

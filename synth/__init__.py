@@ -91,6 +91,8 @@ def _randn(gen, shape, device):
 
 def _slabbed(gen, T, rest, device, fn):
     """Draw a [T, *rest] tensor slab by slab, applying fn to each fp32 slab."""
+    if T == 0:
+        return fn(_randn(gen, (0,) + tuple(rest), device))
     parts = []
     for t0 in range(0, T, SLAB):
         parts.append(fn(_randn(gen, (min(SLAB, T - t0),) + tuple(rest), device)))

@@ -1,0 +1,166 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on
+the same seeded inputs.  Sizes span several 64-token chunks and ragged
+tails; the full-size workloads are checked on sampled heads."""
+import numpy as np
+import pytest
+import torch
+
+import gated_delta_rule_121_b200 as kda
+import oracle
+import synth
+from parity import assert_close, errors
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def run_gpu(inp):
+    return kda.kda_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["init_state"],
+                       inp["cu_seqlens"])
+
+
+def run_oracle(inp, heads=None):
+    sel = (lambda t: t) if heads is None else (lambda t: t[:, :, heads])
+    init = inp["init_state"]
+    if init is not None and heads is not None:
+        init = init[:, heads]
+    return oracle.fwd(sel(inp["q"]), sel(inp["k"]), sel(inp["v"]), sel(inp["g"]), sel(inp["beta"]), init,
+                      inp["cu_seqlens"])
+
+
+def check(inp, dtype, heads=None, what=""):
+    out, fin = run_gpu(inp)
+    torch.cuda.synchronize()
+    o_ref, f_ref = run_oracle(inp, heads)
+    if heads is not None:
+        out, fin = out[:, :, heads], fin[:, heads]
+    eo = assert_close(out, o_ref, dtype, f"{what} out")
+    ef = assert_close(fin, f_ref, dtype, f"{what} final_state")
+    return eo, ef
+
+
+def test_tiny_fp32_exact_path():
+    inp = synth.make_prefill(synth.TINY, DEV)
+    check(inp, torch.float32, what="tiny fp32")
+
+
+@pytest.mark.parametrize("T", [64, 100, 257])
+def test_bf16_small_ragged(T):
+    inp = synth.make_prefill(synth.MID, DEV, T=T, B=2, H=3)
+    check(inp, torch.bfloat16, what=f"bf16 T={T}")
+
+
+def test_mid_prefill_full():
+    inp = synth.make_prefill(synth.MID, DEV)
+    eo, ef = check(inp, torch.bfloat16, what="mid B2 H16 T4096")
+    print("mid errors", eo, ef)
+
+
+def test_stress_model_range_decay():
+    """g = -5 sigmoid(z): chunk totals far below the factorisation floor."""
+    inp = synth.make_prefill(synth.STRESS, DEV)
+    assert float(inp["g"].min()) < -4.0
+    check(inp, torch.bfloat16, what="stress g>=-5")
+
+
+def test_mixed_decay_chunks():
+    """Alternate mild and model-range decay so both Gram paths meet in one chain."""
+    inp = synth.make_prefill(synth.MID, DEV, T=512, B=1, H=2)
+    g = inp["g"].clone()
+    for c in range(0, 512, 128):
+        g[:, c:c + 64] *= 64.0          # -5 * sigmoid(z) on every other chunk
+    inp["g"] = g.contiguous()
+    check(inp, torch.bfloat16, what="mixed decay")
+
+
+@pytest.mark.parametrize("lengths", [[1, 63, 64, 65, 130, 0, 200], [0], [5], [300, 0, 0, 64]])
+def test_varlen_ragged_and_empty(lengths):
+    inp = synth.make_prefill(synth.VARLEN, DEV, H=4, lengths=lengths)
+    check(inp, torch.bfloat16, what=f"varlen {lengths}")
+
+
+def test_varlen_fp32_small_dims():
+    spec = synth.PrefillSpec("v32", 1, 0, 3, 32, 64, torch.float32, 11, init=True)
+    inp = synth.make_prefill(spec, DEV, lengths=[17, 0, 64, 90])
+    check(inp, torch.float32, what="fp32 dk32 dv64 varlen")
+
+
+@pytest.mark.parametrize("dk,dv", [(16, 16), (64, 128), (128, 32), (64, 64)])
+def test_bf16_other_dims(dk, dv):
+    spec = synth.PrefillSpec("dims", 2, 0, 2, dk, dv, torch.bfloat16, 12, init=True)
+    inp = synth.make_prefill(spec, DEV, T=150)
+    check(inp, torch.bfloat16, what=f"bf16 dk{dk} dv{dv}")
+
+
+def test_no_final_state_and_zero_init():
+    inp = synth.make_prefill(synth.MID, DEV, T=200, B=1, H=2)
+    out, fin = kda.kda_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], None, None,
+                           output_final_state=False)
+    assert fin is None
+    o_ref, _ = oracle.fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], None)
+    assert_close(out, o_ref, torch.bfloat16, "zero init")
+
+
+def test_chained_calls_equal_single_call():
+    """Chunked-prefill resume: [0,T1) then [T1,T) from the returned state."""
+    inp = synth.make_prefill(synth.MID, DEV, T=640, B=1, H=4)
+    o_full, f_full = run_gpu(inp)
+    T1 = 320
+    part = lambda t, s: t[:, s].contiguous()
+    a = {k: (part(v, slice(0, T1)) if k in ("q", "k", "v", "g", "beta") else v) for k, v in inp.items()}
+    o1, mid = run_gpu(a)
+    b = {k: (part(v, slice(T1, None)) if k in ("q", "k", "v", "g", "beta") else v) for k, v in inp.items()}
+    b["init_state"] = mid
+    o2, f2 = run_gpu(b)
+    e = errors(torch.cat([o1, o2], 1), o_full)
+    assert e["rel_fro"] < 1e-2
+    assert errors(f2, f_full)["rel_fro"] < 1e-2
+
+
+def test_model_shaped_prefill_sampled_heads():
+    """B=1, H=96, T=65536 (the 64K pretraining shape), heads 0 and 95 checked."""
+    inp = synth.make_prefill(synth.PRETRAIN, DEV)
+    eo, ef = check(inp, torch.bfloat16, heads=[0, 95], what="prefill H96 T65536")
+    print("pretrain errors", eo, ef)
+
+
+def test_debug_intermediates_match_chunk_model():
+    from chunk_model import chunk_forward
+    inp = synth.make_prefill(synth.MID, DEV, T=64, B=1, H=1)
+    dbg = torch.zeros(kda.lib().kda_testing_debug_floats(), dtype=torch.float32, device=DEV)
+    out, fin = kda.kda_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["init_state"], _debug=dbg)
+    torch.cuda.synchronize()
+    f = lambda t: t[0, :, 0].cpu().double().numpy()
+    O, S, it = chunk_forward(f(inp["q"]), f(inp["k"]), f(inp["v"]), f(inp["g"]), f(inp["beta"]),
+                             inp["init_state"][0, 0].cpu().double().numpy(), C=64, keep=True)
+    d = dbg.cpu().double().numpy()
+    it = it[0]
+    checks = [("P", d[0:4096].reshape(64, 64), it["P"]),
+              ("A", d[4096:8192].reshape(64, 64), it["A"]),
+              ("T'", d[8192:12288].reshape(64, 64), it["T"] * f(inp["beta"])[None, :]),
+              ("W", d[12288:20480].reshape(64, 128), it["W"]),
+              ("U", d[20480:28672].reshape(64, 128), it["U"]),
+              ("Delta", d[28672:36864].reshape(64, 128), it["Delta"]),
+              ("O", d[36864:45056].reshape(64, 128), O),
+              ("S", d[45056:61440].reshape(128, 128), S),
+              ("G_C", d[61440:61568], it["G"][-1])]
+    bad = []
+    for name, got, ref in checks:
+        e = errors(got, ref)
+        if not e["rel_fro"] < 2e-2:
+            bad.append((name, e))
+    assert not bad, bad
+
+
+def test_timeout_path_reports_status_and_context_survives():
+    inp = synth.make_prefill(synth.MID, DEV, T=256, B=1, H=2)
+    ws = kda.alloc_workspace(1, 256, 2, 128, 128)
+    kda.kda_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["init_state"], workspace=ws,
+                _wait_ns=0)
+    assert kda.kda_workspace_status(ws) == kda.KDA_ERR_TIMEOUT
+    # the context is still usable and a normal call succeeds
+    out, fin = kda.kda_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["init_state"],
+                           workspace=ws)
+    assert kda.kda_workspace_status(ws) == kda.KDA_OK
+    o_ref, f_ref = run_oracle(inp)
+    assert_close(out, o_ref, torch.bfloat16, "after timeout")
