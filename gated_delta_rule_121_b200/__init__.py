@@ -22,7 +22,8 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libkda.so")
 
-KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_WORKSPACE, KDA_ERR_CUDA, KDA_ERR_TIMEOUT = range(6)
+(KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_WORKSPACE, KDA_ERR_CUDA, KDA_ERR_TIMEOUT,
+ KDA_ERR_RANGE) = range(7)
 KDA_F32, KDA_BF16 = 0, 1
 _DT = {torch.float32: KDA_F32, torch.bfloat16: KDA_BF16}
 
@@ -54,7 +55,7 @@ def lib() -> ctypes.CDLL:
         L.kda_fwd.restype = ctypes.c_int
         L.kda_fwd.argtypes = fwd_args
         L.kda_testing_fwd.restype = ctypes.c_int
-        L.kda_testing_fwd.argtypes = fwd_args + [_fp, ctypes.c_uint64]
+        L.kda_testing_fwd.argtypes = fwd_args + [_fp, ctypes.c_uint64, ctypes.c_int]
         L.kda_testing_debug_floats.restype = ctypes.c_int
         L.kda_testing_fwd_path.restype = ctypes.c_int
         L.kda_testing_fwd_path.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int]
@@ -113,7 +114,7 @@ def _shapes(q, v, cu_seqlens):
 
 
 def kda_fwd(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None, out=None, final_state=None,
-            output_final_state=True, workspace=None, stream=None, _debug=None, _wait_ns=None):
+            output_final_state=True, workspace=None, stream=None, _debug=None, _wait_ns=None, _inject_stuck=False):
     """KDA forward over whole sequences (see include/kda.h, kda_fwd).
 
     q, k, log_alpha: [B,T,H,dk]; v: [B,T,H,dv]; beta: [B,T,H]; q/k/v share a
@@ -141,10 +142,11 @@ def kda_fwd(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None, out=None
     args = (_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(init_state), _ptr(out),
             _ptr(final_state), N, Targ, H, dk, dv, _ptr(cu_seqlens), _stream_ptr(stream), dt,
             _ptr(workspace), workspace.numel())
-    if _debug is None and _wait_ns is None:
+    if _debug is None and _wait_ns is None and not _inject_stuck:
         code = lib().kda_fwd(*args)
     else:
-        code = lib().kda_testing_fwd(*args, _ptr(_debug), int(_wait_ns if _wait_ns is not None else 2_000_000_000))
+        code = lib().kda_testing_fwd(*args, _ptr(_debug), int(_wait_ns if _wait_ns is not None else 2_000_000_000),
+                                     int(bool(_inject_stuck)))
     _check(code, "kda_fwd")
     return out, final_state
 

@@ -9,7 +9,8 @@
 #include "kda_internal.cuh"
 
 namespace kda {
-cudaError_t launch_fwd_tc_impl(const FwdArgs& a, cudaStream_t s, uint64_t wait_ns);
+cudaError_t launch_fwd_tc_impl(const FwdArgs& a, cudaStream_t s, uint64_t wait_ns, int inject_stuck,
+                               int32_t* order_ws);
 int fwd_tc_debug_floats();
 }  // namespace kda
 
@@ -50,20 +51,22 @@ const char* kda_status_string(kda_status_t s) {
     case KDA_ERR_WORKSPACE: return "KDA_ERR_WORKSPACE: workspace missing or too small";
     case KDA_ERR_CUDA: return "KDA_ERR_CUDA: a CUDA call or kernel launch failed";
     case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT: a device-side bounded wait gave up";
+    case KDA_ERR_RANGE: return "KDA_ERR_RANGE: a tensor-core operand exceeded fp16 range";
   }
   return "KDA_ERR_UNKNOWN";
 }
 
 size_t kda_fwd_workspace_size(int B, int64_t T, int H, int dk, int dv, kda_dtype_t dt) {
-  (void)B; (void)T; (void)H; (void)dk; (void)dv; (void)dt;
-  return kStatusBytes;
+  (void)T; (void)H; (void)dk; (void)dv; (void)dt;
+  const size_t order = B > 0 ? (size_t)B * sizeof(int32_t) : 0;
+  return kStatusBytes + ((order + 255) / 256) * 256;
 }
 
 static kda_status_t fwd_impl(const void* q, const void* k, const void* v, const float* log_alpha,
                              const float* beta, const float* init_state, void* out, float* final_state, int B,
                              int64_t T, int H, int dk, int dv, const int32_t* cu_seqlens, void* stream,
                              kda_dtype_t dt, void* workspace, size_t workspace_bytes, float* dbg,
-                             uint64_t wait_ns) {
+                             uint64_t wait_ns, int inject_stuck) {
   kda_status_t st = validate_fwd(q, k, v, log_alpha, beta, init_state, out, final_state, B, T, H, dk, dv, dt);
   if (st != KDA_OK) return st;
   if (cu_seqlens && !aligned16(cu_seqlens)) return KDA_ERR_INVALID_ARG;
@@ -78,8 +81,9 @@ static kda_status_t fwd_impl(const void* q, const void* k, const void* v, const 
   cudaError_t e;
   const int64_t tokens = cu_seqlens ? T : (int64_t)B * T;
   if (kda::fwd_tc_supported(dk, dv, bf16) && tokens > 0)
-    e = kda::launch_fwd_tc_impl(a, s, wait_ns);
-  else if (dbg)
+    e = kda::launch_fwd_tc_impl(a, s, wait_ns, inject_stuck,
+                                reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + kStatusBytes));
+  else if (dbg || inject_stuck)
     return KDA_ERR_UNSUPPORTED;
   else
     e = kda::launch_fwd_simt(a, bf16, s);
@@ -91,7 +95,7 @@ kda_status_t kda_fwd(const void* q, const void* k, const void* v, const float* l
                      int dv, const int32_t* cu_seqlens, void* stream, kda_dtype_t dt, void* workspace,
                      size_t workspace_bytes) {
   return fwd_impl(q, k, v, log_alpha, beta, init_state, out, final_state, B, T, H, dk, dv, cu_seqlens, stream,
-                  dt, workspace, workspace_bytes, nullptr, 2000000000ull);
+                  dt, workspace, workspace_bytes, nullptr, 2000000000ull, 0);
 }
 
 kda_status_t kda_decode_step(const void* q, const void* k, const void* v, const float* log_alpha,
@@ -126,9 +130,9 @@ kda_status_t kda_testing_fwd(const void* q, const void* k, const void* v, const 
                              const float* beta, const float* init_state, void* out, float* final_state, int B,
                              int64_t T, int H, int dk, int dv, const int32_t* cu_seqlens, void* stream,
                              kda_dtype_t dt, void* workspace, size_t workspace_bytes, float* debug_out,
-                             uint64_t wait_ns) {
+                             uint64_t wait_ns, int inject_stuck) {
   return fwd_impl(q, k, v, log_alpha, beta, init_state, out, final_state, B, T, H, dk, dv, cu_seqlens, stream,
-                  dt, workspace, workspace_bytes, debug_out, wait_ns);
+                  dt, workspace, workspace_bytes, debug_out, wait_ns, inject_stuck);
 }
 
 int kda_testing_fwd_path(int dk, int dv, kda_dtype_t dt) {

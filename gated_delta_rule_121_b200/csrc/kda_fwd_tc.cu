@@ -1,41 +1,45 @@
-// Chunked KDA forward on the sm_100a tensor cores (tcgen05 / TMEM / TMA),
-// bf16 q, k, v, out with dk = dv = 128, fp32 state, chunk length C = 64.
+// Chunked KDA forward on the sm_100a tensor cores (tcgen05 / TMEM / TMA).
+// bf16 q, k, v, out with dk = dv = 128, fp32 decay, beta and state; chunk
+// length C = 64.
 //
-// What it computes (Kimi K3 digest, "Kimi Delta Attention" section, chunkwise
-// form: chunk output = inter-chunk term (Gamma ⊙ Q) S + intra-chunk term
-// A Ṽ), written out per chunk with in-chunk cumulative log-decay
-// G_r = sum_{s<=r} g_s (per key channel):
-//   A_rs  = beta_r sum_c k_rc k_sc exp(G_rc - G_sc)   (s < r)       "A_kk"
-//   P_rs  = sum_c q_rc k_sc exp(G_rc - G_sc)          (s <= r)
-//   T     = (I + A)^-1,  T' = T diag(beta)
-//   W     = T' (K ⊙ Γ),   U = T' V                    (WY / UT transform)
-//   Δ     = U - W S                                    (Ṽ of the digest)
-//   O     = (Q ⊙ Γ) S + P Δ
-//   S    <- Diag(Γ_C) S + (K ⊙ exp(G_C - G))^T Δ
-// (Γ = exp(G); Γ_C its last row.)  Unrolling the recurrence of the same
-// section over a chunk gives exactly these identities.
+// What it computes (Kimi K3 digest, "Kimi Delta Attention" section: chunk
+// output = inter-chunk term (Gamma ⊙ Q) S + intra-chunk term A Ṽ), written
+// out per chunk with the in-chunk cumulative log-decay G_r = sum_{s<=r} g_s
+// (per key channel) and its chunk total G_C:
+//   A_rs = beta_r sum_c k_rc k_sc exp(G_rc - G_sc)    (s < r)
+//   P_rs = sum_c q_rc k_sc exp(G_rc - G_sc)           (s <= r)
+//   T    = (I + A)^-1,   T' = T diag(beta)
+//   S'   = Diag(exp G_C) S                     (state decayed to chunk end)
+//   QE   = Q ⊙ exp(G - G_C),  KE = K ⊙ exp(G - G_C),  KH = K ⊙ exp(G_C - G)
+//   W'   = T' KE,   U = T' V,   Δ = U - W' S'
+//   O    = QE S' + P Δ
+//   S   <- S' + KH^T Δ
+// which is the same section's recurrence unrolled over a chunk (QE S' =
+// (Q ⊙ e^G) S and W' S' = T' (K ⊙ e^G) S).  The factors exp(G - G_C) grow
+// up to exp(-G_C): with the digest's bounded decay ("Bounded decay" section,
+// g >= -5) every tile is a dense matmul as long as a chunk's total decay is
+// moderate.  A chunk whose total decay in some channel is below 2^-10 takes
+// the general variant: its Gram matrices P, A come from CUDA cores using the
+// exact differences G_r - G_s, the operands use the chunk START as reference
+// (QE = Q e^G, KE = K e^G), and the scan decays S only after D1.
 //
-// Bounded decay ("Bounded decay" section: g >= g_min = -5): the pairwise
-// decay exp(G_rc - G_sc) is factorised as exp(G_rc) * exp(-G_sc) so that the
-// Gram matrices become dense bf16 matmuls.  The factor exp(-G) stays finite
-// only while the chunk's total decay is moderate; a chunk whose total
-// log-decay in some channel is below -64 takes the general path, which forms
-// the two Gram matrices on CUDA cores from the exact differences G_r - G_s.
-// Everything after the Gram matrices is shared by both paths.
+// Operands are fp16 (10-bit mantissa) with fp32 accumulation: the fp32
+// state and every product stay accurate to well inside the bf16 output's own
+// rounding.  Values that would not fit fp16 set KDA_ERR_RANGE.
 //
-// Layout of the work: one CTA per (sequence, head) chain, chunks in order.
-// All UMMAs are M = 128 with the state kept TRANSPOSED in TMEM (lane j =
-// value channel, column c = key channel), so the tensor-core "rows" are the
-// 128 value channels:
-//   G1  [P ; A_raw](lanes r, 64+r)  = [QΓ ; KΓ] · K̃^T       (K̃ = K ⊙ e^{-G})
-//   G2  W^T (lane c)                = (KΓ)^T · T'^T
-//   G3  U^T (lane j)                = V^T · T'^T
-//   D1  O^T = S^T (QΓ)^T,  (WS)^T = S^T W^T
-//   D2  S^T += Δ^T K̂,  O^T += Δ^T P^T                    (K̂ = K ⊙ e^{G_C-G})
-// Δ^T = U^T - (WS)^T is formed lane-wise in registers.  S^T lives in TMEM
-// (fp32) for the whole chain; a bf16 copy in shared memory is the A operand
-// of D1.  Q, K, V tiles arrive by TMA with 128-byte swizzle, two chunks
-// ahead; Q and K are rescaled in place into QΓ and KΓ.
+// Work split (one CTA per (sequence, head) chain, chunks in order):
+//   warps 4-7, "prologue" group (PG): for chunk c+1 — cumulative decay,
+//     operand scaling, G1 Gram UMMA, the triangular solve on CUDA cores,
+//     G2/G3 UMMAs for W'^T and U^T, and the W'^T store;
+//   warps 0-3, "scan" group (SG): for chunk c — the state recurrence:
+//     decay S^T, D1 = { O^T = S'^T QE^T ;  Δ^T = U^T - S'^T W'^T }, Δ^T to
+//     fp16, D2 = { S^T += Δ^T KH ;  O^T += Δ^T P^T }, output store.
+// The state is kept TRANSPOSED in TMEM (lane j = value channel, column c =
+// key channel) so that every UMMA has M = 128: the value channels.  S'^T and
+// Δ^T are the A operands of D1/D2 straight from TMEM (fp16 pairs per
+// column); every other operand is a 128-byte-swizzled fp16 tile in shared
+// memory.  Q, K, V arrive by TMA two chunks ahead.  Each group has one
+// elected thread that issues its UMMAs; mbarriers carry the hand-offs.
 #include <cuda.h>
 
 #include "kda_internal.cuh"
@@ -44,495 +48,658 @@
 namespace kda {
 namespace {
 
-constexpr int CH = 64;    // chunk length
-constexpr int D = 128;    // dk = dv
-constexpr int NTHR = 128;
+constexpr int CH = 64;  // chunk length
+constexpr int D = 128;  // dk = dv
+constexpr int NTHR = 256;
 constexpr float LOG2E = 1.4426950408889634f;
-constexpr float FAST_MIN_LOG2 = -92.0f;  // chunk-total decay floor for the factorised Gram (~e^-64)
+constexpr float FAST_MIN_LOG2 = -10.0f;  // chunk-total decay floor (log2) for the tensor-core Gram
+constexpr float F16_SAFE = 60000.0f;     // |x| above this would overflow fp16 operands
 constexpr uint64_t WAIT_NS = 2000000000ull;
 
-// Shared memory map (bytes from a 1024-aligned base).
-constexpr uint32_t STAGE_BYTES = 49152;      // [Q;K] 32 KB + V 16 KB
+// ---- shared memory map (bytes from a 1024-aligned base)
+constexpr uint32_t STAGE_BYTES = 49152;  // [Q;K] 32 KB (per 64-channel half: Q rows, then K rows) + V 16 KB
 constexpr uint32_t OFF_QK = 0, OFF_V = 32768;
-constexpr uint32_t SM_G = 2 * STAGE_BYTES;   // g tile, fp32 [64][128]       32 KB
-constexpr uint32_t SM_KT = SM_G + 32768;     // K̃ (bf16) -> A (fp32) -> T'   16 KB
-constexpr uint32_t SM_KH = SM_KT + 16384;    // K̂ (bf16)                     16 KB
-constexpr uint32_t SM_P = SM_KH + 16384;     // P (bf16)                      8 KB
-constexpr uint32_t SM_WD = SM_P + 8192;      // W, then Δ^T (bf16)           16 KB
-constexpr uint32_t SM_SB = SM_WD + 16384;    // S^T bf16                     32 KB
-constexpr uint32_t SM_MISC = SM_SB + 32768;
-constexpr uint32_t MISC_BYTES = 3072;
-constexpr uint32_t SMEM_BYTES = SM_MISC + MISC_BYTES + 1024;  // + alignment slack
+constexpr uint32_t SM_KX = 2 * STAGE_BYTES;  // KH fp16 [s][c], x2          32 KB
+constexpr uint32_t SM_P = SM_KX + 32768;     // P fp16 [r][s], x2            16 KB
+constexpr uint32_t SM_WT = SM_P + 16384;     // W'^T fp16 [c][r]             16 KB
+constexpr uint32_t SM_A = SM_WT + 16384;     // A fp32 [64][64] -> T' fp16   16 KB
+constexpr uint32_t SM_DG = SM_A + 16384;     // D_0, D_1 fp32 [32][32]        8 KB
+constexpr uint32_t SM_X = SM_DG + 8192;      // X fp32 [32][32]               4 KB
+constexpr uint32_t SM_MISC = SM_X + 4096;
+constexpr uint32_t MISC_BYTES = 4096;
+constexpr uint32_t SMEM_BYTES = SM_MISC + MISC_BYTES + 1024;
 
-// TMEM columns (fp32 accumulators, 128 lanes each).
-constexpr uint32_t TM_S = 0, TM_O = 128, TM_WS = 192, TM_GRAM = 256, TM_W = 320, TM_U = 384;
+// misc layout
+enum Bar {
+  B_FULL0 = 0, B_FULL1, B_G1, B_G23, B_D1, B_D2, B_GC0, B_GC1, B_PRO0, B_PRO1, B_BUF0, B_BUF1,
+  B_DFREE, B_WFREE, B_DRAIN_PG, B_DRAIN_SG, B_NEVER, NUM_BARS
+};
+constexpr uint32_t MS_TMEM = 160, MS_ABORT = 164, MS_FAST = 168, MS_CNT = 176;  // MS_CNT: int[4]
+constexpr uint32_t MS_BETA = 256;    // [2][64] fp32
+constexpr uint32_t MS_GC = 768;      // [2][128] fp32: exp(G_C)
+constexpr uint32_t MS_RED = 1792;    // [4][128] fp32
+constexpr uint32_t MS_END = 3840;
+static_assert(NUM_BARS * 8 <= MS_TMEM, "barrier area");
+static_assert(MS_END <= MISC_BYTES, "misc area");
+
+// ---- TMEM columns
+constexpr uint32_t TM_S = 0;        // S^T fp32, 128 cols
+constexpr uint32_t TM_O = 128;      // O^T fp32, 2 x 64 cols
+constexpr uint32_t TM_DELTA = 256;  // U^T, then Δ^T, fp32, 64 cols
+constexpr uint32_t TM_GW = 320;     // Gram, then W'^T, fp32, 64 cols
+constexpr uint32_t TM_SB = 384;     // S'^T fp16 pairs (A operand), 64 cols
+constexpr uint32_t TM_DT = 448;     // Δ^T fp16 pairs (A operand), 32 cols
 constexpr uint32_t TMEM_COLS = 512;
 
-// Debug dump offsets (floats) for chain 0, chunk 0.
+// ---- debug dump (floats) for chain 0, chunk 0
 constexpr int DBG_P = 0, DBG_A = 4096, DBG_T = 8192, DBG_W = 12288, DBG_U = 20480, DBG_DELTA = 28672,
               DBG_O = 36864, DBG_S = 45056, DBG_GC = 61440, DBG_FLOATS = 61568;
 
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+// ------------------------------------------------------------------ helpers
+__device__ __forceinline__ void st_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
                : "memory");
 }
-__device__ __forceinline__ void st_shared_v2(uint32_t addr, uint32_t a, uint32_t b) {
+__device__ __forceinline__ void st_v2(uint32_t addr, uint32_t a, uint32_t b) {
   asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(addr), "r"(a), "r"(b) : "memory");
-}
-__device__ __forceinline__ void st_shared_b16(uint32_t addr, float x) {
-  __nv_bfloat16 h = __float2bfloat16_rn(x);
-  asm volatile("st.shared.b16 [%0], %1;" ::"r"(addr), "h"(*reinterpret_cast<uint16_t*>(&h)) : "memory");
 }
 __device__ __forceinline__ float4 ld_bf16x4(uint32_t addr) {
   uint32_t a, b;
   asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(a), "=r"(b) : "r"(addr));
-  __nv_bfloat162 x = *reinterpret_cast<__nv_bfloat162*>(&a), y = *reinterpret_cast<__nv_bfloat162*>(&b);
-  float2 fx = __bfloat1622float2(x), fy = __bfloat1622float2(y);
-  return make_float4(fx.x, fx.y, fy.x, fy.y);
+  const float2 x = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&a));
+  const float2 y = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&b));
+  return make_float4(x.x, x.y, y.x, y.y);
 }
 __device__ __forceinline__ float ld_bf16(uint32_t addr) {
   uint16_t u;
   asm volatile("ld.shared.b16 %0, [%1];" : "=h"(u) : "r"(addr));
   return __bfloat162float(*reinterpret_cast<__nv_bfloat16*>(&u));
 }
-__device__ __forceinline__ void st_bf16x4(uint32_t addr, float4 v) {
-  st_shared_v2(addr, pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
+__device__ __forceinline__ void st_f16x4(uint32_t addr, float4 v) {
+  st_v2(addr, pack_f16x2(v.x, v.y), pack_f16x2(v.z, v.w));
 }
-// Eight consecutive fp32 values -> one 16-byte chunk of bf16.
-__device__ __forceinline__ void st_bf16x8(uint32_t addr, const float* v) {
-  st_shared_v4(addr, pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
-               pack_bf16x2(v[6], v[7]));
+__device__ __forceinline__ void st_f16x8(uint32_t addr, const float* v) {
+  st_v4(addr, pack_f16x2(v[0], v[1]), pack_f16x2(v[2], v[3]), pack_f16x2(v[4], v[5]), pack_f16x2(v[6], v[7]));
 }
-// fp32 [64][64] matrix with 16-byte units XOR-swizzled by row (conflict-free
-// row writes and broadcast reads).
+__device__ __forceinline__ float4 mul4(float4 a, float4 b) {
+  return make_float4(a.x * b.x, a.y * b.y, a.z * b.z, a.w * b.w);
+}
+__device__ __forceinline__ float4 ex2_4(float4 a) { return make_float4(ex2(a.x), ex2(a.y), ex2(a.z), ex2(a.w)); }
+__device__ __forceinline__ float amax4(float4 a) {
+  return fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(a.z), fabsf(a.w)));
+}
+// fp32 [64][64] with 16-byte units XOR-swizzled by row.
 __device__ __forceinline__ uint32_t a_off(uint32_t r, uint32_t s) {
   return r * 256u + ((s >> 2) ^ (r & 7u)) * 16u + (s & 3u) * 4u;
 }
+// fp32 [32][32] with 16-byte units XOR-swizzled by row.
+__device__ __forceinline__ uint32_t b_off(uint32_t r, uint32_t s) {
+  return r * 128u + ((s >> 2) ^ (r & 7u)) * 16u + (s & 3u) * 4u;
+}
+// Bounded wait that also gives up when the other group has aborted.
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, uint64_t ns, volatile int* abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > ns) return false;
+  }
+  return true;
+}
 
-__global__ void __launch_bounds__(NTHR, 1)
-    kda_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
-                      const float* __restrict__ beta, const float* __restrict__ init,
-                      __nv_bfloat16* __restrict__ out, float* __restrict__ fin, const int32_t* __restrict__ cu,
-                      int64_t Tper, int H, DeviceStatus* status, float* __restrict__ dbg, uint64_t wait_ns) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const uint32_t sb = smem_u32(sm);
-  uint64_t* bar_stage = reinterpret_cast<uint64_t*>(sm + SM_MISC);  // [2]
-  uint64_t* bar_g = bar_stage + 2;
-  uint64_t* bar_mma = bar_stage + 3;
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + SM_MISC + 64);
-  volatile int* s_abort = reinterpret_cast<volatile int*>(sm + SM_MISC + 68);
-  float* s_beta = reinterpret_cast<float*>(sm + SM_MISC + 128);  // [64]
-  float* s_gc = reinterpret_cast<float*>(sm + SM_MISC + 384);    // [128] exp(G_C)
-  float* s_red = reinterpret_cast<float*>(sm + SM_MISC + 896);   // [4][128]
-
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int chain = blockIdx.x;
-  const int n = chain / H, h = chain % H;
+struct Ctx {
+  uint8_t* sm;
+  uint32_t sb;  // shared-window address of sm
+  uint64_t* bars;
+  volatile int* abort;
+  uint32_t tmem;
+  int h, H, nchunks;
   int64_t t0, L;
-  if (cu) {
-    t0 = cu[n];
-    L = (int64_t)cu[n + 1] - t0;
-  } else {
-    t0 = (int64_t)n * Tper;
-    L = Tper;
-  }
-  const int nchunks = (int)((L + CH - 1) / CH);
-  const bool dump = (dbg != nullptr) && chain == 0;
+  DeviceStatus* status;
+  uint64_t wait_ns;
+  float* dbg;  // chain-0 debug dump or nullptr
+};
 
-  if (tid == 0) {
-    mbar_init(&bar_stage[0], 1);
-    mbar_init(&bar_stage[1], 1);
-    mbar_init(bar_g, 1);
-    mbar_init(bar_mma, 1);
-    fence_mbar_init();
-    *s_abort = 0;
-    prefetch_tmap(&tm_q);
-    prefetch_tmap(&tm_k);
-    prefetch_tmap(&tm_v);
-    prefetch_tmap(&tm_g);
-  }
-  if (warp == 0) {
-    tmem_alloc(s_tmem, TMEM_COLS);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *s_tmem;
-  const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);  // this warp's TMEM lane quarter
+__device__ __forceinline__ bool cwait(const Ctx& x, int bar, uint32_t parity, int where) {
+  if (wait_bar(&x.bars[bar], parity, x.wait_ns, x.abort)) return true;
+  if (!*x.abort) record_error(x.status, KDA_ERR_TIMEOUT, where);
+  *x.abort = 1;
+  return false;
+}
 
-  // Async-op bookkeeping: thread 0 issues every TMA and UMMA; all threads
-  // wait on the same phases in the same order, so the waited counts agree.
-  int stage_issued[2] = {0, 0}, stage_waited[2] = {0, 0}, g_issued = 0, g_waited = 0;
-  int mma_issued = 0, mma_waited = 0;
+// Group-uniform bounded wait: every thread of named-barrier group `grp` (128
+// threads) polls, then the group agrees on the outcome, so no thread can
+// leave a loop while the others wait at a barrier or a .sync.aligned op.
+__device__ __forceinline__ bool gwait(const Ctx& x, int bar, uint32_t parity, int where, int grp) {
+  bool ok = wait_bar(&x.bars[bar], parity, x.wait_ns, x.abort);
+  if (!ok) {
+    if (!*x.abort) record_error(x.status, KDA_ERR_TIMEOUT, where);
+    *x.abort = 1;
+  }
+  return named_sync_and(grp, 128, ok);
+}
+
+__device__ __forceinline__ int chunk_valid(const Ctx& x, int c) {
+  const int64_t rem = x.L - (int64_t)c * CH;
+  return rem < CH ? (int)rem : CH;
+}
+
+// ======================================================== prologue group
+__device__ void prologue_group(const Ctx& x, const float* __restrict__ g, const float* __restrict__ beta,
+                               int (&consumed)[2]) {
+  const int p = threadIdx.x - 128;  // 0..127, also the TMEM lane
+  const int rq = p >> 5, cq = p & 31;  // rows 16 rq.., channels 4 cq..
+  const int ch0 = 4 * cq, hh = ch0 >> 6, cc = ch0 & 63;
+  const uint32_t tl = x.tmem + ((uint32_t)(rq * 32) << 16);
+  uint8_t* sm = x.sm;
+  const uint32_t sb = x.sb;
+  float* s_red = reinterpret_cast<float*>(sm + SM_MISC + MS_RED);
+  const int H = x.H;
+
+  // Register prefetch of this thread's g rows and of beta for chunk c.
+  auto load_g = [&](int c, float4(&gv)[16], float& bv) {
+    const int valid = c < x.nchunks ? chunk_valid(x, c) : 0;
+    const int64_t tok0 = x.t0 + (int64_t)c * CH;
+#pragma unroll
+    for (int m = 0; m < 16; ++m) {
+      const int r = 16 * rq + m;
+      gv[m] = r < valid ? __ldg(reinterpret_cast<const float4*>(g + ((tok0 + r) * H + x.h) * D + ch0))
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    bv = (p < CH && p < valid) ? __ldg(beta + (tok0 + p) * H + x.h) : 0.f;
+  };
+
+  float4 gv[16];
+  float bv;
+  load_g(0, gv, bv);
+  int g1_ph = 0, g23_ph = 0;
+
+  for (int c = 0; c < x.nchunks; ++c) {
+    const int b2 = c & 1;
+    const int valid = chunk_valid(x, c);
+    const bool dmp = x.dbg && c == 0;
+    const uint32_t stg = sb + b2 * STAGE_BYTES;
+    float* s_gc = reinterpret_cast<float*>(sm + SM_MISC + MS_GC) + b2 * 128;
+    float* s_beta = reinterpret_cast<float*>(sm + SM_MISC + MS_BETA) + b2 * 64;
+    volatile int* s_fast = reinterpret_cast<volatile int*>(sm + SM_MISC + MS_FAST) + b2;
+
+    // Buffers [b2] were last used by the scan of chunk c-2.
+    if (c >= 2 && !gwait(x, B_BUF0 + b2, ((c >> 1) - 1) & 1, 11, 1)) break;
+    if (!gwait(x, B_FULL0 + b2, (c >> 1) & 1, 12, 1)) break;
+    ++consumed[b2];
+
+    // ---- (a1) cumulative decay in log2 units
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int m = 0; m < 16; ++m) {
+      acc.x += gv[m].x * LOG2E; acc.y += gv[m].y * LOG2E; acc.z += gv[m].z * LOG2E; acc.w += gv[m].w * LOG2E;
+      gv[m] = acc;  // gv now holds the local inclusive prefix
+    }
+    *reinterpret_cast<float4*>(s_red + rq * 128 + ch0) = acc;
+    named_sync(1, 128);
+    float4 tot = make_float4(0.f, 0.f, 0.f, 0.f), off = tot;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float4 v = *reinterpret_cast<const float4*>(s_red + q * 128 + ch0);
+      if (q < rq) { off.x += v.x; off.y += v.y; off.z += v.z; off.w += v.w; }
+      tot.x += v.x; tot.y += v.y; tot.z += v.z; tot.w += v.w;
+    }
+#pragma unroll
+    for (int m = 0; m < 16; ++m) {
+      gv[m].x += off.x; gv[m].y += off.y; gv[m].z += off.z; gv[m].w += off.w;  // G (log2)
+    }
+    const bool fast = named_sync_and(1, 128, fminf(fminf(tot.x, tot.y), fminf(tot.z, tot.w)) >= FAST_MIN_LOG2);
+    if (rq == 0) *reinterpret_cast<float4*>(s_gc + ch0) = ex2_4(tot);
+    if (p == 0) *s_fast = fast ? 1 : 0;
+    if (p < CH) s_beta[p] = bv;
+    if (dmp && rq == 0) {
+      const float LN2 = 0.6931471805599453f;
+      x.dbg[DBG_GC + ch0] = tot.x * LN2; x.dbg[DBG_GC + ch0 + 1] = tot.y * LN2;
+      x.dbg[DBG_GC + ch0 + 2] = tot.z * LN2; x.dbg[DBG_GC + ch0 + 3] = tot.w * LN2;
+    }
+    named_sync(1, 128);
+    if (p == 0) mbar_arrive(&x.bars[B_GC0 + b2]);
+
+    const uint32_t qb = stg + OFF_QK + hh * 16384, kb = qb + 8192;
+    const uint32_t vb = stg + OFF_V + hh * 8192;
+    const uint32_t khb = sb + SM_KX + b2 * 16384 + hh * 8192;
+    const float4 ref = fast ? tot : make_float4(0.f, 0.f, 0.f, 0.f);
+    bool bad = false;
+
+    if (!fast) {
+      // ---- general variant: Gram matrices on CUDA cores from exact decay
+      // differences.  G is staged through the W'^T tile in two channel
+      // halves (fp32 [64][64]); that tile is free once D1 of chunk c-1 is done.
+      if (c >= 1 && !gwait(x, B_WFREE, (c - 1) & 1, 13, 1)) break;
+      const int r = p & 63, s0 = (p >> 6) * 32;
+      float pa[32], aa[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) pa[i] = aa[i] = 0.f;
+      for (int half = 0; half < 2; ++half) {
+        named_sync(1, 128);
+        if (hh == half) {
+#pragma unroll
+          for (int m = 0; m < 16; ++m)
+            *reinterpret_cast<float4*>(sm + SM_WT + (16 * rq + m) * 256 + cc * 4) = gv[m];
+        }
+        named_sync(1, 128);
+        if (r < valid) {
+          for (int ch = 0; ch < 64; ++ch) {
+            const uint32_t off_r = half * 16384 + sw128_off(r, ch);
+            const float gr = *reinterpret_cast<const float*>(sm + SM_WT + r * 256 + ch * 4);
+            const float qr = ld_bf16(stg + OFF_QK + off_r), kr = ld_bf16(stg + OFF_QK + 8192 + off_r);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const int s = s0 + i;
+              if (s <= r) {
+                const float gs = *reinterpret_cast<const float*>(sm + SM_WT + s * 256 + ch * 4);
+                const float ks = ld_bf16(stg + OFF_QK + 8192 + half * 16384 + sw128_off(s, ch));
+                const float e = ex2(gr - gs) * ks;
+                pa[i] += qr * e;
+                aa[i] += kr * e;
+              }
+            }
+          }
+        }
+      }
+      const float br = s_beta[r];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int s = s0 + i;
+        aa[i] = s < r ? br * aa[i] : 0.f;
+        if (!(s <= r)) pa[i] = 0.f;
+      }
+#pragma unroll
+      for (int q8 = 0; q8 < 4; ++q8) {
+        const int s = s0 + 8 * q8;
+        st_f16x8(sb + SM_P + b2 * 8192 + r * 128 + ((((s >> 3) ^ r) & 7) << 4), pa + 8 * q8);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        *reinterpret_cast<float4*>(sm + SM_A + a_off(r, s0 + 4 * u)) =
+            make_float4(aa[4 * u], aa[4 * u + 1], aa[4 * u + 2], aa[4 * u + 3]);
+      if (dmp) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          x.dbg[DBG_P + r * 64 + s0 + i] = pa[i];
+          x.dbg[DBG_A + r * 64 + s0 + i] = aa[i];
+        }
+      }
+      named_sync(1, 128);  // raw Q/K reads are done before they are rescaled in place
+    }
+
+    // ---- (a2) operand scaling: QE, KE in place, KH into KX[b2], V -> fp16.
+#pragma unroll
+    for (int m = 0; m < 16; ++m) {
+      const int r = 16 * rq + m;
+      const uint32_t o = sw128_off(r, cc);
+      float4 q4 = ld_bf16x4(qb + o), k4 = ld_bf16x4(kb + o), v4 = ld_bf16x4(vb + o);
+      if (r >= valid) q4 = k4 = v4 = make_float4(0.f, 0.f, 0.f, 0.f);
+      const float4 e = ex2_4(make_float4(gv[m].x - ref.x, gv[m].y - ref.y, gv[m].z - ref.z, gv[m].w - ref.w));
+      const float4 hcoef =
+          ex2_4(make_float4(tot.x - gv[m].x, tot.y - gv[m].y, tot.z - gv[m].z, tot.w - gv[m].w));
+      bad |= amax4(v4) > F16_SAFE;
+      st_f16x4(qb + o, mul4(q4, e));
+      st_f16x4(kb + o, mul4(k4, e));
+      st_f16x4(vb + o, v4);
+      st_f16x4(khb + o, mul4(k4, hcoef));
+    }
+    if (bad) record_error(x.status, KDA_ERR_RANGE, 20);
+    fence_proxy_async_smem();
+    named_sync(1, 128);
+
+    if (fast) {
+      // ---- G1: [P ; A_raw] = [QE ; KE] . KH^T   (M=128, N=64, K=128)
+      if (p == 0) {
+        tc_fence_after();
+        const uint32_t id = idesc_f16_f32(128, 64, 0, 0);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const uint64_t da = sdesc_sw128(stg + OFF_QK + (i >> 2) * 16384 + (i & 3) * 32, 16, 1024);
+          const uint64_t db = sdesc_sw128(sb + SM_KX + b2 * 16384 + (i >> 2) * 8192 + (i & 3) * 32, 16, 1024);
+          umma_ss(x.tmem + TM_GW, da, db, id, i > 0);
+        }
+        umma_commit(&x.bars[B_G1]);
+      }
+      if (!gwait(x, B_G1, g1_ph, 14, 1)) break;
+      g1_ph ^= 1;
+      tc_fence_after();
+      float r0[32], r1[32];
+      tmem_ld32(tl + TM_GW, r0);
+      tmem_ld32(tl + TM_GW + 32, r1);
+      if (p < CH) {  // P row p, lower triangle including the diagonal
+#pragma unroll
+        for (int s = 0; s < 32; ++s) {
+          if (s > p) r0[s] = 0.f;
+          if (s + 32 > p) r1[s] = 0.f;
+        }
+#pragma unroll
+        for (int q8 = 0; q8 < 8; ++q8)
+          st_f16x8(sb + SM_P + b2 * 8192 + p * 128 + (((q8 ^ p) & 7) << 4),
+                   q8 < 4 ? r0 + 8 * q8 : r1 + 8 * (q8 - 4));
+        if (dmp) {
+#pragma unroll
+          for (int s = 0; s < 64; ++s) x.dbg[DBG_P + p * 64 + s] = s < 32 ? r0[s] : r1[s - 32];
+        }
+      } else {  // A row r = beta_r (KE KH^T)_rs, strictly lower
+        const int r = p - CH;
+        const float b = s_beta[r];
+#pragma unroll
+        for (int s = 0; s < 32; ++s) {
+          r0[s] = s < r ? b * r0[s] : 0.f;
+          r1[s] = s + 32 < r ? b * r1[s] : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const float* v = u < 8 ? r0 + 4 * u : r1 + 4 * (u - 8);
+          *reinterpret_cast<float4*>(sm + SM_A + a_off(r, 4 * u)) = make_float4(v[0], v[1], v[2], v[3]);
+        }
+        if (dmp) {
+#pragma unroll
+          for (int s = 0; s < 64; ++s) x.dbg[DBG_A + r * 64 + s] = s < 32 ? r0[s] : r1[s - 32];
+        }
+      }
+      tc_fence_before();
+      named_sync(1, 128);
+    }
+
+    // ---- (a3) T = (I + A)^-1 in 2 x 2 blocks of 32:
+    //   D_b = (I + A_bb)^-1 by forward substitution (one column per thread),
+    //   T_10 = -D_1 (A_10 D_0);  T' = T diag(beta) as fp16 [r][s].
+    if (p < 64) {
+      const int bk = p >> 5, jj = p & 31;
+      float xs[32];
+#pragma unroll
+      for (int r = 0; r < 32; ++r) xs[r] = 0.f;
+#pragma unroll
+      for (int r = 0; r < 32; ++r) {
+        float a0 = (r == jj) ? 1.f : 0.f, a1 = 0.f;
+#pragma unroll
+        for (int u = 0; u < (r + 3) / 4; ++u) {
+          const float4 a4 = *reinterpret_cast<const float4*>(sm + SM_A + a_off(32 * bk + r, 32 * bk + 4 * u));
+          a0 -= a4.x * xs[4 * u] + a4.z * xs[4 * u + 2];
+          a1 -= a4.y * xs[4 * u + 1] + a4.w * xs[4 * u + 3];
+        }
+        xs[r] = a0 + a1;
+      }
+#pragma unroll
+      for (int r = 0; r < 32; ++r) *reinterpret_cast<float*>(sm + SM_DG + bk * 4096 + b_off(r, jj)) = xs[r];
+    }
+    named_sync(1, 128);
+    const int rr = p >> 2, q8 = p & 3;  // output row rr, columns 8 q8 .. 8 q8 + 7 of a 32x32 block
+    {
+      float o8[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) o8[i] = 0.f;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {  // X = A_10 D_0
+        const float4 a4 = *reinterpret_cast<const float4*>(sm + SM_A + a_off(32 + rr, 4 * u));
+        const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const int s = 4 * u + t;
+          const float4 d0 = *reinterpret_cast<const float4*>(sm + SM_DG + b_off(s, 8 * q8));
+          const float4 d1 = *reinterpret_cast<const float4*>(sm + SM_DG + b_off(s, 8 * q8 + 4));
+          o8[0] += av[t] * d0.x; o8[1] += av[t] * d0.y; o8[2] += av[t] * d0.z; o8[3] += av[t] * d0.w;
+          o8[4] += av[t] * d1.x; o8[5] += av[t] * d1.y; o8[6] += av[t] * d1.z; o8[7] += av[t] * d1.w;
+        }
+      }
+      *reinterpret_cast<float4*>(sm + SM_X + b_off(rr, 8 * q8)) = make_float4(o8[0], o8[1], o8[2], o8[3]);
+      *reinterpret_cast<float4*>(sm + SM_X + b_off(rr, 8 * q8 + 4)) = make_float4(o8[4], o8[5], o8[6], o8[7]);
+    }
+    named_sync(1, 128);
+    {
+      float o8[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) o8[i] = 0.f;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {  // T_10 = -D_1 X
+        const float4 a4 = *reinterpret_cast<const float4*>(sm + SM_DG + 4096 + b_off(rr, 4 * u));
+        const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const int s = 4 * u + t;
+          const float4 d0 = *reinterpret_cast<const float4*>(sm + SM_X + b_off(s, 8 * q8));
+          const float4 d1 = *reinterpret_cast<const float4*>(sm + SM_X + b_off(s, 8 * q8 + 4));
+          o8[0] -= av[t] * d0.x; o8[1] -= av[t] * d0.y; o8[2] -= av[t] * d0.z; o8[3] -= av[t] * d0.w;
+          o8[4] -= av[t] * d1.x; o8[5] -= av[t] * d1.y; o8[6] -= av[t] * d1.z; o8[7] -= av[t] * d1.w;
+        }
+      }
+      float d0v[8], d1v[8], z8[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float bl = s_beta[8 * q8 + i], bh = s_beta[32 + 8 * q8 + i];
+        d0v[i] = *reinterpret_cast<const float*>(sm + SM_DG + b_off(rr, 8 * q8 + i)) * bl;
+        d1v[i] = *reinterpret_cast<const float*>(sm + SM_DG + 4096 + b_off(rr, 8 * q8 + i)) * bh;
+        o8[i] *= bl;
+        z8[i] = 0.f;
+      }
+      named_sync(1, 128);  // every read of A is done before T' overwrites its first half
+      // T' rows rr and 32+rr, 16-byte chunks at columns 8 q8 and 32 + 8 q8.
+      st_f16x8(sb + SM_A + sw128_off(rr, 8 * q8), d0v);
+      st_f16x8(sb + SM_A + sw128_off(rr, 32 + 8 * q8), z8);
+      st_f16x8(sb + SM_A + sw128_off(32 + rr, 8 * q8), o8);
+      st_f16x8(sb + SM_A + sw128_off(32 + rr, 32 + 8 * q8), d1v);
+      if (dmp) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          x.dbg[DBG_T + rr * 64 + 8 * q8 + i] = d0v[i];
+          x.dbg[DBG_T + rr * 64 + 32 + 8 * q8 + i] = 0.f;
+          x.dbg[DBG_T + (32 + rr) * 64 + 8 * q8 + i] = o8[i];
+          x.dbg[DBG_T + (32 + rr) * 64 + 32 + 8 * q8 + i] = d1v[i];
+        }
+      }
+    }
+    fence_proxy_async_smem();
+    named_sync(1, 128);
+
+    // ---- (a4) G2: W'^T = KE^T T'^T -> TM_GW;  G3: U^T = V^T T'^T -> TM_DELTA
+    if (p == 0) {
+      bool ok = true;
+      if (c >= 1) ok = cwait(x, B_DFREE, (c - 1) & 1, 15);  // scan has read Δ of chunk c-1
+      if (ok) {
+        tc_fence_after();
+        const uint32_t id = idesc_f16_f32(128, 64, 1, 0);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint64_t da = sdesc_sw128(stg + OFF_QK + 8192 + i * 2048, 16384, 1024);
+          const uint64_t db = sdesc_sw128(sb + SM_A + i * 32, 16, 1024);
+          umma_ss(x.tmem + TM_GW, da, db, id, i > 0);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint64_t da = sdesc_sw128(stg + OFF_V + i * 2048, 8192, 1024);
+          const uint64_t db = sdesc_sw128(sb + SM_A + i * 32, 16, 1024);
+          umma_ss(x.tmem + TM_DELTA, da, db, id, i > 0);
+        }
+        umma_commit(&x.bars[B_G23]);
+      }
+    }
+    // Prefetch next chunk's decay and beta while the UMMAs run.
+    float4 gn[16];
+    float bn;
+    load_g(c + 1, gn, bn);
+    if (!gwait(x, B_G23, g23_ph, 16, 1)) break;
+    g23_ph ^= 1;
+    tc_fence_after();
+    if (fast && c >= 1 && !gwait(x, B_WFREE, (c - 1) & 1, 17, 1)) break;
+    {  // lane c holds W'^T[c][r]: store row c of the MN-major B operand of D1
+      float w0[32], w1[32];
+      tmem_ld32(tl + TM_GW, w0);
+      tmem_ld32(tl + TM_GW + 32, w1);
+      float mx = 0.f;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) mx = fmaxf(mx, fmaxf(fabsf(w0[i]), fabsf(w1[i])));
+      if (!(mx <= F16_SAFE)) record_error(x.status, KDA_ERR_RANGE, 21);
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        st_f16x8(sb + SM_WT + p * 128 + (((q ^ p) & 7) << 4), q < 4 ? w0 + 8 * q : w1 + 8 * (q - 4));
+      if (dmp) {
+        float u0[32], u1[32];
+        tmem_ld32(tl + TM_DELTA, u0);
+        tmem_ld32(tl + TM_DELTA + 32, u1);
+#pragma unroll
+        for (int r = 0; r < 64; ++r) {
+          x.dbg[DBG_W + r * 128 + p] = r < 32 ? w0[r] : w1[r - 32];
+          x.dbg[DBG_U + r * 128 + p] = r < 32 ? u0[r] : u1[r - 32];
+        }
+      }
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    named_sync(1, 128);
+    if (p == 0) mbar_arrive(&x.bars[B_PRO0 + b2]);
+#pragma unroll
+    for (int m = 0; m < 16; ++m) gv[m] = gn[m];
+    bv = bn;
+  }
+}
+
+// ============================================================ scan group
+__device__ void scan_group(const Ctx& x, const void* tmq, const void* tmk, const void* tmv,
+                           const float* __restrict__ init, __nv_bfloat16* __restrict__ out,
+                           float* __restrict__ fin, int64_t sbase, bool inject_stuck, int (&issued)[2]) {
+  const int j = threadIdx.x;  // 0..127: TMEM lane = value channel
+  const uint32_t tl = x.tmem + ((uint32_t)((j >> 5) * 32) << 16);
+  uint8_t* sm = x.sm;
+  const uint32_t sb = x.sb;
+  const int H = x.H;
+
   auto issue_stage = [&](int c) {
     const int st = c & 1;
-    const int tok = (int)(t0 + (int64_t)c * CH);
+    const int tok = (int)(x.t0 + (int64_t)c * CH);
     uint8_t* dst = sm + st * STAGE_BYTES;
-    mbar_arrive_expect_tx(&bar_stage[st], STAGE_BYTES);
+    uint64_t* bar = &x.bars[B_FULL0 + st];
+    mbar_arrive_expect_tx(bar, STAGE_BYTES);
+#pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
-      tma_load_3d(dst + OFF_QK + hh * 16384, &tm_q, &bar_stage[st], 64 * hh, h, tok);
-      tma_load_3d(dst + OFF_QK + hh * 16384 + 8192, &tm_k, &bar_stage[st], 64 * hh, h, tok);
-      tma_load_3d(dst + OFF_V + hh * 8192, &tm_v, &bar_stage[st], 64 * hh, h, tok);
+      tma_load_3d(dst + OFF_QK + hh * 16384, tmq, bar, 64 * hh, x.h, tok);
+      tma_load_3d(dst + OFF_QK + hh * 16384 + 8192, tmk, bar, 64 * hh, x.h, tok);
+      tma_load_3d(dst + OFF_V + hh * 8192, tmv, bar, 64 * hh, x.h, tok);
     }
-    ++stage_issued[st];
   };
-  auto issue_g = [&](int c) {
-    mbar_arrive_expect_tx(bar_g, 32768);
-    tma_load_3d(sm + SM_G, &tm_g, bar_g, 0, h, (int)(t0 + (int64_t)c * CH));
-    ++g_issued;
-  };
-  auto wait_mma = [&](int where) {
-    // Only a completed phase counts as waited; the error path drains the rest.
-    if (mbar_wait(bar_mma, mma_waited & 1, wait_ns)) {
-      ++mma_waited;
-    } else {
-      record_error(status, KDA_ERR_TIMEOUT, where);
-      *s_abort = 1;
+  if (j == 0) {
+    if (x.nchunks > 0) {
+      issue_stage(0);
+      ++issued[0];
     }
-    tc_fence_after();
-  };
-  // Barrier that also reports whether any thread gave up on a wait.
-  auto sync_abort = [&]() -> bool {
-    __syncthreads();
-    return *s_abort != 0;
-  };
-
-  if (tid == 0 && nchunks > 0) {
-    issue_stage(0);
-    issue_g(0);
-    if (nchunks > 1) issue_stage(1);
+    if (x.nchunks > 1) {
+      issue_stage(1);
+      ++issued[1];
+    }
   }
-
-  const int64_t sbase = ((int64_t)n * H + h) * D * D;
-  const int j = tid;  // TMEM lane = value channel in the transposed-state phases
-  // ---- initial state: S^T into TMEM, bf16 copy into SB.
+  // S^T <- initial state (zeros without one).
 #pragma unroll
   for (int cb = 0; cb < 4; ++cb) {
     float r[32];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) r[i] = init ? init[sbase + (int64_t)(cb * 32 + i) * D + j] : 0.f;
+    for (int i = 0; i < 32; ++i) r[i] = init ? __ldg(init + sbase + (int64_t)(cb * 32 + i) * D + j) : 0.f;
     tmem_st32(tl + TM_S + cb * 32, r);
-#pragma unroll
-    for (int q8 = 0; q8 < 4; ++q8) {
-      const int c = cb * 32 + q8 * 8;
-      st_bf16x8(sb + SM_SB + (c >> 6) * 16384 + sw128_off(j, c & 63), r + q8 * 8);
-    }
   }
   tmem_wait_st();
-  fence_proxy_async_smem();
-  tc_fence_before();
-  __syncthreads();
 
-  const uint32_t ID_K64 = idesc_bf16_f32(128, 64, 0, 0);
-  const uint32_t ID_MN64 = idesc_bf16_f32(128, 64, 1, 0);
-  const uint32_t ID_S = idesc_bf16_f32(128, 128, 0, 1);
-
-  for (int c = 0; c < nchunks; ++c) {
-    const int st = c & 1;
-    const uint32_t stg = sb + st * STAGE_BYTES;
-    const int64_t tok0 = t0 + (int64_t)c * CH;
-    const int valid = (int)((L - (int64_t)c * CH) < CH ? (L - (int64_t)c * CH) : CH);
-    const bool dmp = dump && c == 0;
-
-    if (tid < CH) s_beta[tid] = tid < valid ? beta[(tok0 + tid) * H + h] : 0.f;
-    if (mbar_wait(bar_g, g_waited & 1, wait_ns)) {
-      ++g_waited;
-    } else {
-      record_error(status, KDA_ERR_TIMEOUT, 1);
-      *s_abort = 1;
-    }
-    if (mbar_wait(&bar_stage[st], stage_waited[st] & 1, wait_ns)) {
-      ++stage_waited[st];
-    } else {
-      record_error(status, KDA_ERR_TIMEOUT, 2);
-      *s_abort = 1;
-    }
-
-    // ---- (a1) in-chunk cumulative decay, log2 units.  Thread (rq = warp,
-    // cq = lane): rows 16 rq .. 16 rq + 15, channels 4 cq .. 4 cq + 3.
-    const int rq = warp;
-    const int ch0 = 4 * lane, hh = ch0 >> 6, cc = ch0 & 63;
-    float4 G[16];
-    {
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  auto store_out = [&](int c) {
+    const int valid = chunk_valid(x, c);
+    const int64_t tok0 = x.t0 + (int64_t)c * CH;
+    float o[32];
 #pragma unroll
-      for (int m = 0; m < 16; ++m) {
-        const int r = 16 * rq + m;
-        float4 gv = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (r < valid) gv = *reinterpret_cast<const float4*>(sm + SM_G + r * 512 + ch0 * 4);
-        acc.x += gv.x * LOG2E; acc.y += gv.y * LOG2E; acc.z += gv.z * LOG2E; acc.w += gv.w * LOG2E;
-        G[m] = acc;
+    for (int half = 0; half < 2; ++half) {
+      tmem_ld32(tl + TM_O + (c & 1) * 64 + half * 32, o);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int r = half * 32 + i;
+        if (r < valid) out[((tok0 + r) * H + x.h) * D + j] = __float2bfloat16_rn(o[i]);
+        if (x.dbg && c == 0) x.dbg[DBG_O + r * 128 + j] = o[i];
       }
-      *reinterpret_cast<float4*>(s_red + rq * 128 + ch0) = acc;
     }
-    if (sync_abort()) break;
-    float4 tot = make_float4(0.f, 0.f, 0.f, 0.f);
-    {
-      float4 off = tot;
+  };
+
+  int d1_ph = 0, d2_ph = 0;
+  bool ok = true;
+  for (int c = 0; c < x.nchunks && ok; ++c) {
+    const int b2 = c & 1;
+    const uint32_t stg = sb + b2 * STAGE_BYTES;
+    const float* s_gc = reinterpret_cast<const float*>(sm + SM_MISC + MS_GC) + b2 * 128;
+    if (inject_stuck && c == 0 && !gwait(x, B_NEVER, 0, 99, 2)) {
+      ok = false;
+      break;
+    }
+    // ---- S pass: S^T (decayed to the chunk end when this chunk is "fast")
+    // -> S'^T as fp16 pairs, the A operand of D1.
+    if (c >= 1) {
+      if (!gwait(x, B_D2, d2_ph, 31, 2)) {
+        ok = false;
+        break;
+      }
+      d2_ph ^= 1;
+      tc_fence_after();
+    }
+    if (!gwait(x, B_GC0 + b2, (c >> 1) & 1, 32, 2)) {
+      ok = false;
+      break;
+    }
+    const bool fast = *reinterpret_cast<volatile int*>(sm + SM_MISC + MS_FAST + 4 * b2) != 0;
+    float mx = 0.f;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float4 v = *reinterpret_cast<const float4*>(s_red + q * 128 + ch0);
-        if (q < rq) { off.x += v.x; off.y += v.y; off.z += v.z; off.w += v.w; }
-        tot.x += v.x; tot.y += v.y; tot.z += v.z; tot.w += v.w;
+    for (int cb = 0; cb < 4; ++cb) {
+      float s[32];
+      uint32_t pk[16];
+      tmem_ld32(tl + TM_S + cb * 32, s);
+      if (fast) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) s[i] *= s_gc[cb * 32 + i];
+        tmem_st32(tl + TM_S + cb * 32, s);
       }
 #pragma unroll
-      for (int m = 0; m < 16; ++m) {
-        G[m].x += off.x; G[m].y += off.y; G[m].z += off.z; G[m].w += off.w;
+      for (int i = 0; i < 16; ++i) {
+        pk[i] = pack_f16x2(s[2 * i], s[2 * i + 1]);
+        mx = fmaxf(mx, fmaxf(fabsf(s[2 * i]), fabsf(s[2 * i + 1])));
       }
+      tmem_st16(tl + TM_SB + cb * 16, pk);
     }
-    const float4 egc = make_float4(ex2(tot.x), ex2(tot.y), ex2(tot.z), ex2(tot.w));
-    if (rq == 0) {
-      *reinterpret_cast<float4*>(s_gc + ch0) = egc;
-      if (dmp) {
-        const float LN2 = 0.6931471805599453f;
-        dbg[DBG_GC + ch0 + 0] = tot.x * LN2; dbg[DBG_GC + ch0 + 1] = tot.y * LN2;
-        dbg[DBG_GC + ch0 + 2] = tot.z * LN2; dbg[DBG_GC + ch0 + 3] = tot.w * LN2;
-      }
+    if (!(mx <= F16_SAFE)) record_error(x.status, KDA_ERR_RANGE, 30);
+    tmem_wait_st();
+    tc_fence_before();
+    if (!named_sync_and(2, 128, !*x.abort)) {
+      ok = false;
+      break;
     }
-    const bool ok_fast = fminf(fminf(tot.x, tot.y), fminf(tot.z, tot.w)) >= FAST_MIN_LOG2;
-    const bool fast = __syncthreads_and(ok_fast) != 0;
 
-    const uint32_t qb = stg + OFF_QK + hh * 16384;  // Q rows of this thread's channel half
-    const uint32_t kb = qb + 8192;                  // K rows
-    const uint32_t ktb = sb + SM_KT + hh * 8192;
-    const uint32_t khb = sb + SM_KH + hh * 8192;
-
-    if (fast) {
-      // ---- (a2, fast) QΓ, KΓ in place; K̃ = K e^{-G}; K̂ = K e^{G_C - G}.
-#pragma unroll
-      for (int m = 0; m < 16; ++m) {
-        const int r = 16 * rq + m;
-        const uint32_t o = sw128_off(r, cc);
-        float4 q4 = ld_bf16x4(qb + o), k4 = ld_bf16x4(kb + o);
-        if (r >= valid) q4 = k4 = make_float4(0.f, 0.f, 0.f, 0.f);
-        const float4 e = make_float4(ex2(G[m].x), ex2(G[m].y), ex2(G[m].z), ex2(G[m].w));
-        const float4 ie = make_float4(ex2(-G[m].x), ex2(-G[m].y), ex2(-G[m].z), ex2(-G[m].w));
-        st_bf16x4(qb + o, make_float4(q4.x * e.x, q4.y * e.y, q4.z * e.z, q4.w * e.w));
-        st_bf16x4(kb + o, make_float4(k4.x * e.x, k4.y * e.y, k4.z * e.z, k4.w * e.w));
-        st_bf16x4(ktb + o, make_float4(k4.x * ie.x, k4.y * ie.y, k4.z * ie.z, k4.w * ie.w));
-        st_bf16x4(khb + o, make_float4(k4.x * (egc.x * ie.x), k4.y * (egc.y * ie.y), k4.z * (egc.z * ie.z),
-                                       k4.w * (egc.w * ie.w)));
-      }
-      fence_proxy_async_smem();
-      if (sync_abort()) break;
-      // ---- (a2) G1: [P ; A_raw] = [QΓ ; KΓ] · K̃^T   (M=128, N=64, K=128)
-      if (tid == 0) {
+    // ---- D1: O^T = S'^T QE^T ;  Δ^T = U^T - S'^T W'^T    (A = S'^T from TMEM)
+    if (j == 0) {
+      if (cwait(x, B_PRO0 + b2, (c >> 1) & 1, 33)) {
         tc_fence_after();
+        const uint32_t idq = idesc_f16_f32(128, 64, 0, 0);
+        const uint32_t idw = idesc_f16_f32(128, 64, 0, 1, 1);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          const uint64_t da = sdesc_sw128(stg + OFF_QK + (i >> 2) * 16384 + (i & 3) * 32, 16, 1024);
-          const uint64_t db = sdesc_sw128(sb + SM_KT + (i >> 2) * 8192 + (i & 3) * 32, 16, 1024);
-          umma_bf16(tmem + TM_GRAM, da, db, ID_K64, i > 0);
+          const uint64_t dq = sdesc_sw128(stg + OFF_QK + (i >> 2) * 16384 + (i & 3) * 32, 16, 1024);
+          umma_tmem_a(x.tmem + TM_O + b2 * 64, x.tmem + TM_SB + i * 8, dq, idq, i > 0);
         }
-        umma_commit(bar_mma);
-        ++mma_issued;
-      }
-      wait_mma(3);
-      if (sync_abort()) break;
-      {
-        float r0[32], r1[32];
-        tmem_ld32(tl + TM_GRAM, r0);
-        tmem_ld32(tl + TM_GRAM + 32, r1);
-        if (tid < CH) {  // lanes 0..63: P row r, lower triangle incl. diagonal
-          const int r = tid;
 #pragma unroll
-          for (int s = 0; s < 32; ++s) {
-            if (s > r) r0[s] = 0.f;
-            if (s + 32 > r) r1[s] = 0.f;
-          }
-#pragma unroll
-          for (int q8 = 0; q8 < 8; ++q8)
-            st_bf16x8(sb + SM_P + r * 128 + (((q8 ^ r) & 7) << 4), q8 < 4 ? r0 + q8 * 8 : r1 + (q8 - 4) * 8);
-          if (dmp)
-#pragma unroll
-            for (int s = 0; s < 64; ++s) dbg[DBG_P + r * 64 + s] = s < 32 ? r0[s] : r1[s - 32];
-        } else {  // lanes 64..127: A row r = beta_r * (KΓ K̃^T)_rs, strictly lower
-          const int r = tid - CH;
-          const float b = s_beta[r];
-#pragma unroll
-          for (int s = 0; s < 32; ++s) {
-            r0[s] = s < r ? b * r0[s] : 0.f;
-            r1[s] = s + 32 < r ? b * r1[s] : 0.f;
-          }
-#pragma unroll
-          for (int u = 0; u < 16; ++u) {
-            const float* v = u < 8 ? r0 + 4 * u : r1 + 4 * (u - 8);
-            *reinterpret_cast<float4*>(sm + SM_KT + a_off(r, 4 * u)) = make_float4(v[0], v[1], v[2], v[3]);
-          }
-          if (dmp)
-#pragma unroll
-            for (int s = 0; s < 64; ++s) dbg[DBG_A + r * 64 + s] = s < 32 ? r0[s] : r1[s - 32];
+        for (int i = 0; i < 8; ++i) {
+          const uint64_t dw = sdesc_sw128(sb + SM_WT + i * 2048, 8192, 1024);
+          umma_tmem_a(x.tmem + TM_DELTA, x.tmem + TM_SB + i * 8, dw, idw, 1);
         }
-      }
-    } else {
-      // ---- (a2, general) G over the g tile; P and A on CUDA cores from the
-      // exact differences G_r - G_s; then QΓ, KΓ in place and K̂.
-#pragma unroll
-      for (int m = 0; m < 16; ++m)
-        *reinterpret_cast<float4*>(sm + SM_G + (16 * rq + m) * 512 + ch0 * 4) = G[m];
-      if (sync_abort()) break;
-      {
-        const int r = tid & 63, s0 = (tid >> 6) * 32;
-        const uint32_t qrow = stg + OFF_QK, krow = stg + OFF_QK + 8192;
-        const float br = s_beta[r];
-        for (int s = s0; s < s0 + 32; ++s) {
-          float p = 0.f, a = 0.f;
-          if (s <= r && r < valid) {
-            for (int ch = 0; ch < D; ++ch) {
-              const uint32_t o_r = (ch >> 6) * 16384 + sw128_off(r, ch & 63);
-              const uint32_t o_s = (ch >> 6) * 16384 + sw128_off(s, ch & 63);
-              const float gr = *reinterpret_cast<const float*>(sm + SM_G + r * 512 + ch * 4);
-              const float gs = *reinterpret_cast<const float*>(sm + SM_G + s * 512 + ch * 4);
-              const float e = ex2(gr - gs);
-              const float ks = ld_bf16(krow + o_s);
-              p += ld_bf16(qrow + o_r) * ks * e;
-              a += ld_bf16(krow + o_r) * ks * e;
-            }
-          }
-          a = (s < r) ? br * a : 0.f;
-          st_shared_b16(sb + SM_P + sw128_off(r, s), p);
-          *reinterpret_cast<float*>(sm + SM_KT + a_off(r, s)) = a;
-          if (dmp) {
-            dbg[DBG_P + r * 64 + s] = p;
-            dbg[DBG_A + r * 64 + s] = a;
-          }
-        }
-      }
-      if (sync_abort()) break;
-#pragma unroll
-      for (int m = 0; m < 16; ++m) {
-        const int r = 16 * rq + m;
-        const uint32_t o = sw128_off(r, cc);
-        float4 q4 = ld_bf16x4(qb + o), k4 = ld_bf16x4(kb + o);
-        if (r >= valid) q4 = k4 = make_float4(0.f, 0.f, 0.f, 0.f);
-        const float4 e = make_float4(ex2(G[m].x), ex2(G[m].y), ex2(G[m].z), ex2(G[m].w));
-        const float4 eh = make_float4(ex2(tot.x - G[m].x), ex2(tot.y - G[m].y), ex2(tot.z - G[m].z),
-                                      ex2(tot.w - G[m].w));
-        st_bf16x4(qb + o, make_float4(q4.x * e.x, q4.y * e.y, q4.z * e.z, q4.w * e.w));
-        st_bf16x4(kb + o, make_float4(k4.x * e.x, k4.y * e.y, k4.z * e.z, k4.w * e.w));
-        st_bf16x4(khb + o, make_float4(k4.x * eh.x, k4.y * eh.y, k4.z * eh.z, k4.w * eh.w));
+        umma_commit(&x.bars[B_D1]);
+        umma_commit(&x.bars[B_WFREE]);
       }
     }
-    fence_proxy_async_smem();
-    if (sync_abort()) break;
+    if (c >= 1) store_out(c - 1);
+    if (!gwait(x, B_D1, d1_ph, 34, 2)) {
+      ok = false;
+      break;
+    }
+    d1_ph ^= 1;
+    tc_fence_after();
+    // The stage of chunk c is no longer read: fetch chunk c+2 into it.
+    if (j == 0 && c + 2 < x.nchunks) {
+      issue_stage(c + 2);
+      ++issued[b2];
+    }
 
-    // ---- (a3) T = (I + A)^-1 by forward substitution, one column per
-    // thread (threads 0..63); T' = T diag(beta) stored as bf16 [r][s].
-    {
-      float x[CH];
-      if (tid < CH) {
-#pragma unroll
-        for (int r = 0; r < CH; ++r) x[r] = 0.f;
-#pragma unroll
-        for (int r = 0; r < CH; ++r) {
-          float acc = (r == j) ? 1.f : 0.f;
-#pragma unroll
-          for (int u = 0; u < (r + 3) / 4; ++u) {
-            const float4 a4 = *reinterpret_cast<const float4*>(sm + SM_KT + a_off(r, 4 * u));
-            acc -= a4.x * x[4 * u] + a4.y * x[4 * u + 1] + a4.z * x[4 * u + 2] + a4.w * x[4 * u + 3];
-          }
-          x[r] = acc;
-        }
-      }
-      __syncthreads();  // every read of A is done before T' overwrites it
-      if (tid < CH) {
-        const float bj = s_beta[j];
-#pragma unroll
-        for (int r = 0; r < CH; ++r) {
-          st_shared_b16(sb + SM_KT + sw128_off(r, j), x[r] * bj);
-          if (dmp) dbg[DBG_T + r * 64 + j] = x[r] * bj;
-        }
-      }
-    }
-    fence_proxy_async_smem();
-    if (sync_abort()) break;
-
-    // ---- (a4) G2: W^T = (KΓ)^T T'^T;  G3: U^T = V^T T'^T   (M=128, N=64, K=64)
-    if (tid == 0) {
-      tc_fence_after();
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint64_t da = sdesc_sw128(stg + OFF_QK + 8192 + i * 2048, 16384, 1024);
-        const uint64_t db = sdesc_sw128(sb + SM_KT + i * 32, 16, 1024);
-        umma_bf16(tmem + TM_W, da, db, ID_MN64, i > 0);
-      }
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint64_t da = sdesc_sw128(stg + OFF_V + i * 2048, 8192, 1024);
-        const uint64_t db = sdesc_sw128(sb + SM_KT + i * 32, 16, 1024);
-        umma_bf16(tmem + TM_U, da, db, ID_MN64, i > 0);
-      }
-      umma_commit(bar_mma);
-      ++mma_issued;
-      if (c + 1 < nchunks) issue_g(c + 1);  // g tile is free: every read of it is behind us
-    }
-    wait_mma(4);
-    if (sync_abort()) break;
-    {  // lane c holds W^T[c][r]; store W[r][c] (K-major B operand of D1)
-      float w0[32], w1[32];
-      tmem_ld32(tl + TM_W, w0);
-      tmem_ld32(tl + TM_W + 32, w1);
-      const uint32_t wb = sb + SM_WD + (j >> 6) * 8192;
-#pragma unroll
-      for (int r = 0; r < 32; ++r) {
-        st_shared_b16(wb + sw128_off(r, j & 63), w0[r]);
-        st_shared_b16(wb + sw128_off(r + 32, j & 63), w1[r]);
-      }
-      if (dmp) {
-        float u0[32], u1[32];
-        tmem_ld32(tl + TM_U, u0);
-        tmem_ld32(tl + TM_U + 32, u1);
-#pragma unroll
-        for (int r = 0; r < 64; ++r) {
-          dbg[DBG_W + r * 128 + j] = r < 32 ? w0[r] : w1[r - 32];
-          dbg[DBG_U + r * 128 + j] = r < 32 ? u0[r] : u1[r - 32];
-        }
-      }
-    }
-    fence_proxy_async_smem();
-    if (sync_abort()) break;
-
-    // ---- (a5/a6) D1: O^T = S^T (QΓ)^T,  (WS)^T = S^T W^T   (M=128, N=64, K=128)
-    if (tid == 0) {
-      tc_fence_after();
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const uint64_t da = sdesc_sw128(sb + SM_SB + (i >> 2) * 16384 + (i & 3) * 32, 16, 1024);
-        const uint64_t dq = sdesc_sw128(stg + OFF_QK + (i >> 2) * 16384 + (i & 3) * 32, 16, 1024);
-        umma_bf16(tmem + TM_O, da, dq, ID_K64, i > 0);
-      }
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const uint64_t da = sdesc_sw128(sb + SM_SB + (i >> 2) * 16384 + (i & 3) * 32, 16, 1024);
-        const uint64_t dw = sdesc_sw128(sb + SM_WD + (i >> 2) * 8192 + (i & 3) * 32, 16, 1024);
-        umma_bf16(tmem + TM_WS, da, dw, ID_K64, i > 0);
-      }
-      umma_commit(bar_mma);
-      ++mma_issued;
-    }
-    wait_mma(5);
-    // The stage's QΓ, KΓ and V have all been consumed: prefetch chunk c+2.
-    if (tid == 0 && c + 2 < nchunks && !*s_abort) issue_stage(c + 2);
-    {
-      // Δ^T[j][r] = U^T - (WS)^T, bf16 row j of the K-major A operand of D2.
-      float u[32], w[32], d[64];
-      tmem_ld32(tl + TM_U, u);
-      tmem_ld32(tl + TM_WS, w);
-#pragma unroll
-      for (int r = 0; r < 32; ++r) d[r] = u[r] - w[r];
-      tmem_ld32(tl + TM_U + 32, u);
-      tmem_ld32(tl + TM_WS + 32, w);
-#pragma unroll
-      for (int r = 0; r < 32; ++r) d[32 + r] = u[r] - w[r];
-#pragma unroll
-      for (int q8 = 0; q8 < 8; ++q8) st_bf16x8(sb + SM_WD + j * 128 + (((q8 ^ j) & 7) << 4), d + q8 * 8);
-      if (dmp)
-#pragma unroll
-        for (int r = 0; r < 64; ++r) dbg[DBG_DELTA + r * 128 + j] = d[r];
-      // S^T <- S^T Diag(Γ_C)  (decay of key channel c = TMEM column c)
+    // ---- Δ^T -> fp16 pairs (A operand of D2); general chunks decay S^T here.
+    if (!fast) {
 #pragma unroll
       for (int cb = 0; cb < 4; ++cb) {
         float s[32];
@@ -541,90 +708,184 @@ __global__ void __launch_bounds__(NTHR, 1)
         for (int i = 0; i < 32; ++i) s[i] *= s_gc[cb * 32 + i];
         tmem_st32(tl + TM_S + cb * 32, s);
       }
-      tmem_wait_st();
     }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    if (sync_abort()) break;
-
-    // ---- (a5/a6) D2: S^T += Δ^T K̂ (N=128);  O^T += Δ^T P^T (N=64);  K=64
-    if (tid == 0) {
-      tc_fence_after();
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint64_t da = sdesc_sw128(sb + SM_WD + i * 32, 16, 1024);
-        const uint64_t dk = sdesc_sw128(sb + SM_KH + i * 2048, 8192, 1024);
-        umma_bf16(tmem + TM_S, da, dk, ID_S, 1);
-      }
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint64_t da = sdesc_sw128(sb + SM_WD + i * 32, 16, 1024);
-        const uint64_t dp = sdesc_sw128(sb + SM_P + i * 32, 16, 1024);
-        umma_bf16(tmem + TM_O, da, dp, ID_K64, 1);
-      }
-      umma_commit(bar_mma);
-      ++mma_issued;
-    }
-    wait_mma(6);
-    if (sync_abort()) break;
     {
-      // New S^T -> bf16 copy for the next chunk's D1.
+      float d[32];
+      uint32_t pk[16];
+      float dm = 0.f;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        tmem_ld32(tl + TM_DELTA + half * 32, d);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          pk[i] = pack_f16x2(d[2 * i], d[2 * i + 1]);
+          dm = fmaxf(dm, fmaxf(fabsf(d[2 * i]), fabsf(d[2 * i + 1])));
+        }
+        tmem_st16(tl + TM_DT + half * 16, pk);
+        if (x.dbg && c == 0) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) x.dbg[DBG_DELTA + (half * 32 + i) * 128 + j] = d[i];
+        }
+      }
+      if (!(dm <= F16_SAFE)) record_error(x.status, KDA_ERR_RANGE, 31);
+    }
+    tmem_wait_st();
+    tc_fence_before();
+    named_sync(2, 128);
+
+    // ---- D2: S^T += Δ^T KH ;  O^T += Δ^T P^T      (A = Δ^T from TMEM)
+    if (j == 0) {
+      mbar_arrive(&x.bars[B_DFREE]);
+      tc_fence_after();
+      const uint32_t ids = idesc_f16_f32(128, 128, 0, 1);
+      const uint32_t idp = idesc_f16_f32(128, 64, 0, 0);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint64_t dk = sdesc_sw128(sb + SM_KX + b2 * 16384 + i * 2048, 8192, 1024);
+        umma_tmem_a(x.tmem + TM_S, x.tmem + TM_DT + i * 8, dk, ids, 1);
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint64_t dp = sdesc_sw128(sb + SM_P + b2 * 8192 + i * 32, 16, 1024);
+        umma_tmem_a(x.tmem + TM_O + b2 * 64, x.tmem + TM_DT + i * 8, dp, idp, 1);
+      }
+      umma_commit(&x.bars[B_D2]);
+      umma_commit(&x.bars[B_BUF0 + b2]);
+    }
+  }
+  if (named_sync_and(2, 128, ok && !*x.abort) && x.nchunks > 0) {
+    if (gwait(x, B_D2, d2_ph, 35, 2)) {
+      tc_fence_after();
+      store_out(x.nchunks - 1);
+    }
+  }
+  if (named_sync_and(2, 128, !*x.abort)) {
+    if (x.dbg && x.nchunks > 0) {
 #pragma unroll
       for (int cb = 0; cb < 4; ++cb) {
         float s[32];
         tmem_ld32(tl + TM_S + cb * 32, s);
 #pragma unroll
-        for (int q8 = 0; q8 < 4; ++q8) {
-          const int ch = cb * 32 + q8 * 8;
-          st_bf16x8(sb + SM_SB + (ch >> 6) * 16384 + sw128_off(j, ch & 63), s + q8 * 8);
-        }
-        if (dmp)
-#pragma unroll
-          for (int i = 0; i < 32; ++i) dbg[DBG_S + (cb * 32 + i) * 128 + j] = s[i];
-      }
-      // O^T lane j -> out[token r][h][j]
-      float o[32];
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        tmem_ld32(tl + TM_O + half * 32, o);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int r = half * 32 + i;
-          if (r < valid) out[((tok0 + r) * H + h) * D + j] = __float2bfloat16_rn(o[i]);
-          if (dmp) dbg[DBG_O + r * 128 + j] = o[i];
-        }
+        for (int i = 0; i < 32; ++i) x.dbg[DBG_S + (cb * 32 + i) * 128 + j] = s[i];
       }
     }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    if (sync_abort()) break;
+    if (fin) {
+#pragma unroll
+      for (int cb = 0; cb < 4; ++cb) {
+        float s[32];
+        tmem_ld32(tl + TM_S + cb * 32, s);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) fin[sbase + (int64_t)(cb * 32 + i) * D + j] = s[i];
+      }
+    }
+  }
+}
+
+__global__ void __launch_bounds__(NTHR, 1)
+    kda_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ g,
+                      const float* __restrict__ beta, const float* __restrict__ init,
+                      __nv_bfloat16* __restrict__ out, float* __restrict__ fin, const int32_t* __restrict__ cu,
+                      const int32_t* __restrict__ order, int64_t Tper, int H, DeviceStatus* status,
+                      float* __restrict__ dbg, uint64_t wait_ns, int inject_stuck) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Ctx x;
+  x.sm = sm;
+  x.sb = smem_u32(sm);
+  x.bars = reinterpret_cast<uint64_t*>(sm + SM_MISC);
+  x.abort = reinterpret_cast<volatile int*>(sm + SM_MISC + MS_ABORT);
+  x.status = status;
+  x.wait_ns = wait_ns;
+  const int tid = threadIdx.x, warp = tid >> 5;
+  // Work item: with packed batches the blocks follow `order`, so that the
+  // longest sequences start first.
+  const int n0 = blockIdx.x / H;
+  const int n = order ? order[n0] : n0;
+  x.h = blockIdx.x % H;
+  x.H = H;
+  if (cu) {
+    x.t0 = cu[n];
+    x.L = (int64_t)cu[n + 1] - x.t0;
+  } else {
+    x.t0 = (int64_t)n * Tper;
+    x.L = Tper;
+  }
+  x.nchunks = (int)((x.L + CH - 1) / CH);
+  x.dbg = (dbg && n == 0 && x.h == 0) ? dbg : nullptr;
+
+  if (tid == 0) {
+    for (int i = 0; i < NUM_BARS; ++i) mbar_init(&x.bars[i], 1);
+    fence_mbar_init();
+    *x.abort = 0;
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+  }
+  if (warp == 0) {
+    tmem_alloc(reinterpret_cast<uint32_t*>(sm + SM_MISC + MS_TMEM), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  x.tmem = *reinterpret_cast<volatile uint32_t*>(sm + SM_MISC + MS_TMEM);
+  const int64_t sbase = ((int64_t)n * H + x.h) * D * D;
+
+  int cnt[2] = {0, 0};  // TMA stages issued (scan group) / consumed (prologue group)
+  int* s_cnt = reinterpret_cast<int*>(sm + SM_MISC + MS_CNT);
+  if (warp < 4) {
+    scan_group(x, &tm_q, &tm_k, &tm_v, init, out, fin, sbase, inject_stuck != 0, cnt);
+    if (tid == 0) { s_cnt[0] = cnt[0]; s_cnt[1] = cnt[1]; }
+  } else {
+    prologue_group(x, g, beta, cnt);
+    if (tid == 128) { s_cnt[2] = cnt[0]; s_cnt[3] = cnt[1]; }
   }
 
-  if (*s_abort) {
-    // Error path: let every copy and UMMA this CTA issued finish (bounded)
-    // before the tensor memory is released.
-    if (tid == 0) {
-      for (int st = 0; st < 2; ++st)
-        for (; stage_waited[st] < stage_issued[st]; ++stage_waited[st])
-          mbar_wait(&bar_stage[st], stage_waited[st] & 1, WAIT_NS);
-      for (; g_waited < g_issued; ++g_waited) mbar_wait(bar_g, g_waited & 1, WAIT_NS);
-      for (; mma_waited < mma_issued; ++mma_waited) mbar_wait(bar_mma, mma_waited & 1, WAIT_NS);
-    }
-  } else if (fin) {
-#pragma unroll
-    for (int cb = 0; cb < 4; ++cb) {
-      float s[32];
-      tmem_ld32(tl + TM_S + cb * 32, s);
-#pragma unroll
-      for (int i = 0; i < 32; ++i) fin[sbase + (int64_t)(cb * 32 + i) * D + j] = s[i];
-    }
+  // Drain: every UMMA issued by a group's elected thread has completed, and
+  // (on the error path) every TMA load in flight has landed, before TMEM is
+  // released and the block exits.
+  if (tid == 0 || tid == 128) {
+    uint64_t* db = &x.bars[tid == 0 ? B_DRAIN_SG : B_DRAIN_PG];
+    umma_commit(db);
+    mbar_wait(db, 0, WAIT_NS);
+  }
+  __syncthreads();
+  if (tid == 0) {
+    // Wait (bounded) for any TMA load that was issued but never consumed.
+    for (int st = 0; st < 2; ++st)
+      for (int k = s_cnt[2 + st]; k < s_cnt[st]; ++k) mbar_wait(&x.bars[B_FULL0 + st], k & 1, WAIT_NS);
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, TMEM_COLS);
+    tmem_dealloc(x.tmem, TMEM_COLS);
   }
+}
+
+// Packed batches: order sequences by decreasing length (bucketed by
+// floor(log2(length))) so the longest chains are scheduled first.
+__global__ void kda_order_kernel(const int32_t* __restrict__ cu, int N, int32_t* __restrict__ order) {
+  __shared__ int cnt[33], base[33];
+  const int tid = threadIdx.x;
+  if (tid < 33) cnt[tid] = 0;
+  __syncthreads();
+  auto bucket = [&](int n) {
+    const int L = cu[n + 1] - cu[n];
+    return L <= 0 ? 32 : __clz(L);  // longer sequences -> smaller bucket index
+  };
+  for (int n = tid; n < N; n += blockDim.x) atomicAdd(&cnt[bucket(n)], 1);
+  __syncthreads();
+  if (tid == 0) {
+    int acc = 0;
+    for (int b = 0; b < 33; ++b) {
+      base[b] = acc;
+      acc += cnt[b];
+    }
+  }
+  __syncthreads();
+  for (int n = tid; n < N; n += blockDim.x) order[atomicAdd(&base[bucket(n)], 1)] = n;
 }
 
 // ------------------------------------------------------------------ host
@@ -644,46 +905,45 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// Tensor [T_total][H][d] as a 3-D map (d innermost), box {box_d, 1, 64 tokens}.
-bool make_map(CUtensorMap* m, CUtensorMapDataType dt, uint32_t esz, const void* ptr, int d, int H, int64_t Ttot,
-              uint32_t box_d, CUtensorMapSwizzle sw) {
+// bf16 tensor [T_total][H][128] as a 3-D map, box {64 channels, 1 head, 64 tokens}, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* ptr, int H, int64_t Ttot) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
-  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)Ttot};
-  cuuint64_t strides[2] = {(cuuint64_t)d * esz, (cuuint64_t)H * d * esz};
-  cuuint32_t box[3] = {box_d, 1, (cuuint32_t)CH};
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)Ttot};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
+  cuuint32_t box[3] = {64, 1, (cuuint32_t)CH};
   cuuint32_t es[3] = {1, 1, 1};
-  return enc(m, dt, 3, const_cast<void*>(ptr), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
 
 bool fwd_tc_supported(int dk, int dv, bool bf16) { return bf16 && dk == D && dv == D; }
 
-cudaError_t launch_fwd_tc_impl(const FwdArgs& a, cudaStream_t s, uint64_t wait_ns) {
+cudaError_t launch_fwd_tc_impl(const FwdArgs& a, cudaStream_t s, uint64_t wait_ns, int inject_stuck,
+                               int32_t* order_ws) {
   const int64_t Ttot = a.cu ? a.T : (int64_t)a.N * a.T;
   const unsigned blocks = (unsigned)((int64_t)a.N * a.H);
   if (blocks == 0) return cudaSuccess;
-  CUtensorMap mq, mk, mv, mg;
-  // A map needs at least one token row; an all-empty batch still runs the
-  // kernel (to copy init -> final) with maps that are never read.
+  CUtensorMap mq, mk, mv;
   const int64_t Tmap = Ttot > 0 ? Ttot : 1;
-  if (!make_map(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.q, D, a.H, Tmap, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map(&mk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.k, D, a.H, Tmap, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map(&mv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.v, D, a.H, Tmap, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map(&mg, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.g, D, a.H, Tmap, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
+  if (!make_map(&mq, a.q, a.H, Tmap) || !make_map(&mk, a.k, a.H, Tmap) || !make_map(&mv, a.v, a.H, Tmap))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(kda_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)SMEM_BYTES);
+  const int32_t* order = nullptr;
+  if (a.cu && order_ws && a.N > 1) {
+    kda_order_kernel<<<1, 1024, 0, s>>>(a.cu, a.N, order_ws);
+    order = order_ws;
+  }
+  cudaError_t e =
+      cudaFuncSetAttribute(kda_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  kda_fwd_tc_kernel<<<blocks, NTHR, SMEM_BYTES, s>>>(mq, mk, mv, mg, a.beta, a.init, (__nv_bfloat16*)a.out,
-                                                     a.fin, a.cu, a.cu ? 0 : a.T, a.H, a.status, (float*)a.dbg,
-                                                     wait_ns);
+  kda_fwd_tc_kernel<<<blocks, NTHR, SMEM_BYTES, s>>>(mq, mk, mv, a.g, a.beta, a.init, (__nv_bfloat16*)a.out,
+                                                     a.fin, a.cu, order, a.cu ? 0 : a.T, a.H, a.status,
+                                                     (float*)a.dbg, wait_ns, inject_stuck);
   return cudaGetLastError();
 }
-
-cudaError_t launch_fwd_tc(const FwdArgs& a, cudaStream_t s) { return launch_fwd_tc_impl(a, s, WAIT_NS); }
 
 int fwd_tc_debug_floats() { return DBG_FLOATS; }
 

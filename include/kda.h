@@ -63,19 +63,22 @@ typedef enum {
     KDA_ERR_UNSUPPORTED = 2,  /* dk/dv/dtype combination not built */
     KDA_ERR_WORKSPACE = 3,    /* workspace missing or smaller than required */
     KDA_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed */
-    KDA_ERR_TIMEOUT = 5       /* a device-side bounded wait gave up */
+    KDA_ERR_TIMEOUT = 5,      /* a device-side bounded wait gave up */
+    KDA_ERR_RANGE = 6         /* a tensor-core operand exceeded fp16 range (see kda_fwd) */
 } kda_status_t;
 
 /* Element type of q, k, v and out.  log_alpha, beta and states are always
- * fp32.  KDA_F32 inputs are computed without rounding operands to TF32 or
- * bf16; KDA_BF16 inputs use bf16 tensor-core operands with fp32
- * accumulation and an fp32 state. */
+ * fp32.  KDA_F32 inputs are computed in fp32 on CUDA cores, without rounding
+ * operands to TF32 or bf16.  KDA_BF16 inputs with dk = dv = 128 run on the
+ * tensor cores with fp16 operands (10-bit mantissa), fp32 accumulation and an
+ * fp32 state; other bf16 shapes run in fp32 on CUDA cores. */
 typedef enum { KDA_F32 = 0, KDA_BF16 = 1 } kda_dtype_t;
 
 /*
- * Bytes of device workspace kda_fwd needs for these sizes (0 is possible
- * only if the call would do no work).  With cu_seqlens, pass B = N (number
- * of sequences) and T = total packed tokens.
+ * Bytes of device workspace kda_fwd needs for these sizes: a 256-byte
+ * status word plus, for packed batches, N int32 slots of scratch in which
+ * the longest-first order of the sequences is built.  With cu_seqlens, pass
+ * B = N (number of sequences) and T = total packed tokens.
  */
 KDA_API size_t kda_fwd_workspace_size(int B, int64_t T, int H, int dk, int dv, kda_dtype_t dt);
 
@@ -102,6 +105,11 @@ KDA_API size_t kda_fwd_workspace_size(int B, int64_t T, int H, int dk, int dv, k
  *   workspace  device scratch of at least kda_fwd_workspace_size(...) bytes,
  *              16-byte aligned; its contents on entry do not matter.  It must
  *              not be shared by calls that may run concurrently.
+ * Range (tensor-core path): v, the state and the intermediate values W, U,
+ * Delta are rounded to fp16 operands, so their magnitudes must stay below
+ * 6e4 (|v| and |S| of order 1e3 or less are safe).  A value beyond that is
+ * reported as KDA_ERR_RANGE through kda_workspace_status(); outputs are then
+ * not meaningful.
  */
 KDA_API kda_status_t kda_fwd(const void *q, const void *k, const void *v,
                      const float *log_alpha, const float *beta,
@@ -132,7 +140,8 @@ KDA_API kda_status_t kda_decode_step(const void *q, const void *k, const void *v
  * Read back the device status word of a workspace used by kda_fwd.
  * Synchronises `stream` (it is the one call that does) and returns KDA_OK or
  * the first device-side error recorded since the workspace was last passed
- * to kda_fwd (KDA_ERR_TIMEOUT when a bounded wait expired).
+ * to kda_fwd (KDA_ERR_TIMEOUT when a bounded wait expired, KDA_ERR_RANGE
+ * when an fp16 operand overflowed).
  */
 KDA_API kda_status_t kda_workspace_status(const void *workspace, void *stream);
 

@@ -23,11 +23,13 @@ KDA_API int kda_testing_debug_floats(void);
  *              intermediates of its first chunk: P, A, T', W, U, Delta, O,
  *              the state after the chunk and the chunk-total log-decay.
  *   wait_ns    bound for every device-side wait in nanoseconds (kda_fwd
- *              uses 2e9).  A bound of 0 makes the first wait that is not
- *              already satisfied give up, which exercises the timeout path
- *              (status KDA_ERR_TIMEOUT in the workspace) without faulting or
- *              hanging the GPU: the kernel then drains its own copies and
- *              tensor-core work with the normal bound and exits.
+ *              uses 2e9).
+ *   inject_stuck  when nonzero (tensor-core path), the scan warps of every
+ *              block first wait on a barrier that nothing ever signals.  The
+ *              wait gives up after wait_ns, records KDA_ERR_TIMEOUT in the
+ *              workspace status word and the block unwinds: it drains its own
+ *              copies and tensor-core work and releases its tensor memory, so
+ *              the GPU context stays usable.  Nothing faults or hangs.
  */
 KDA_API kda_status_t kda_testing_fwd(const void *q, const void *k, const void *v,
                              const float *log_alpha, const float *beta,
@@ -35,7 +37,7 @@ KDA_API kda_status_t kda_testing_fwd(const void *q, const void *k, const void *v
                              int B, int64_t T, int H, int dk, int dv,
                              const int32_t *cu_seqlens, void *stream, kda_dtype_t dt,
                              void *workspace, size_t workspace_bytes,
-                             float *debug_out, uint64_t wait_ns);
+                             float *debug_out, uint64_t wait_ns, int inject_stuck);
 
 /* 1 when kda_fwd uses the tensor-core kernel for this shape, else 0. */
 KDA_API int kda_testing_fwd_path(int dk, int dv, kda_dtype_t dt);

@@ -37,7 +37,7 @@ def test_every_declared_symbol_is_exported():
 
 
 def test_status_strings():
-    for code in range(6):
+    for code in range(7):
         s = kda.kda_status_string(code)
         assert s.startswith("KDA_")
     assert "UNKNOWN" in kda.kda_status_string(99)

@@ -138,7 +138,8 @@ def test_debug_intermediates_match_chunk_model():
     checks = [("P", d[0:4096].reshape(64, 64), it["P"]),
               ("A", d[4096:8192].reshape(64, 64), it["A"]),
               ("T'", d[8192:12288].reshape(64, 64), it["T"] * f(inp["beta"])[None, :]),
-              ("W", d[12288:20480].reshape(64, 128), it["W"]),
+              # the kernel stores W' = W Diag(exp(-G_C)) (operands referenced to the chunk end)
+              ("W'", d[12288:20480].reshape(64, 128), it["W"] * np.exp(-it["G"][-1])[None, :]),
               ("U", d[20480:28672].reshape(64, 128), it["U"]),
               ("Delta", d[28672:36864].reshape(64, 128), it["Delta"]),
               ("O", d[36864:45056].reshape(64, 128), O),
@@ -153,10 +154,12 @@ def test_debug_intermediates_match_chunk_model():
 
 
 def test_timeout_path_reports_status_and_context_survives():
+    """A wait on a barrier nothing signals gives up after 1 ms, the status
+    word says so, and the next call on the same context succeeds."""
     inp = synth.make_prefill(synth.MID, DEV, T=256, B=1, H=2)
     ws = kda.alloc_workspace(1, 256, 2, 128, 128)
     kda.kda_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["init_state"], workspace=ws,
-                _wait_ns=0)
+                _wait_ns=1_000_000, _inject_stuck=True)
     assert kda.kda_workspace_status(ws) == kda.KDA_ERR_TIMEOUT
     # the context is still usable and a normal call succeeds
     out, fin = kda.kda_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["init_state"],
