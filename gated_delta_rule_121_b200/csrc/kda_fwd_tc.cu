@@ -75,6 +75,7 @@ enum Bar {
   B_DFREE, B_WFREE, B_DRAIN_PG, B_DRAIN_SG, B_NEVER, NUM_BARS
 };
 constexpr uint32_t MS_TMEM = 160, MS_ABORT = 164, MS_FAST = 168, MS_CNT = 176;  // MS_CNT: int[4]
+constexpr uint32_t MS_T0 = 192;  // int64: clock at block start (timing dump)
 constexpr uint32_t MS_BETA = 256;    // [2][64] fp32
 constexpr uint32_t MS_GC = 768;      // [2][128] fp32: exp(G_C)
 constexpr uint32_t MS_RED = 1792;    // [4][128] fp32
@@ -93,7 +94,10 @@ constexpr uint32_t TMEM_COLS = 512;
 
 // ---- debug dump (floats) for chain 0, chunk 0
 constexpr int DBG_P = 0, DBG_A = 4096, DBG_T = 8192, DBG_W = 12288, DBG_U = 20480, DBG_DELTA = 28672,
-              DBG_O = 36864, DBG_S = 45056, DBG_GC = 61440, DBG_FLOATS = 61568;
+              DBG_O = 36864, DBG_S = 45056, DBG_GC = 61440, DBG_TIME = 61568, DBG_FLOATS = 63616;
+// DBG_TIME: int64 [64 chunks][16 events] of SM clock cycles since block start
+// (events 0-7 prologue group, 8-15 scan group), chain 0 only.
+constexpr int TIME_CHUNKS = 64;
 
 // ------------------------------------------------------------------ helpers
 __device__ __forceinline__ void st_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
@@ -158,7 +162,14 @@ struct Ctx {
   DeviceStatus* status;
   uint64_t wait_ns;
   float* dbg;  // chain-0 debug dump or nullptr
+  long long* tdbg;  // chain-0 phase timestamps or nullptr
+  long long tstart;
 };
+
+// Phase timestamp (elected thread only) for the timing dump.
+__device__ __forceinline__ void tmark(const Ctx& x, int c, int ev) {
+  if (x.tdbg && c < TIME_CHUNKS) x.tdbg[c * 16 + ev] = clock64() - x.tstart;
+}
 
 __device__ __forceinline__ bool cwait(const Ctx& x, int bar, uint32_t parity, int where) {
   if (wait_bar(&x.bars[bar], parity, x.wait_ns, x.abort)) return true;
@@ -223,10 +234,12 @@ __device__ void prologue_group(const Ctx& x, const float* __restrict__ g, const 
     float* s_beta = reinterpret_cast<float*>(sm + SM_MISC + MS_BETA) + b2 * 64;
     volatile int* s_fast = reinterpret_cast<volatile int*>(sm + SM_MISC + MS_FAST) + b2;
 
+    if (p == 0) tmark(x, c, 0);
     // Buffers [b2] were last used by the scan of chunk c-2.
     if (c >= 2 && !gwait(x, B_BUF0 + b2, ((c >> 1) - 1) & 1, 11, 1)) break;
     if (!gwait(x, B_FULL0 + b2, (c >> 1) & 1, 12, 1)) break;
     ++consumed[b2];
+    if (p == 0) tmark(x, c, 1);
 
     // ---- (a1) cumulative decay in log2 units
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -258,7 +271,10 @@ __device__ void prologue_group(const Ctx& x, const float* __restrict__ g, const 
       x.dbg[DBG_GC + ch0 + 2] = tot.z * LN2; x.dbg[DBG_GC + ch0 + 3] = tot.w * LN2;
     }
     named_sync(1, 128);
-    if (p == 0) mbar_arrive(&x.bars[B_GC0 + b2]);
+    if (p == 0) {
+      mbar_arrive(&x.bars[B_GC0 + b2]);
+      tmark(x, c, 2);
+    }
 
     const uint32_t qb = stg + OFF_QK + hh * 16384, kb = qb + 8192;
     const uint32_t vb = stg + OFF_V + hh * 8192;
@@ -347,6 +363,7 @@ __device__ void prologue_group(const Ctx& x, const float* __restrict__ g, const 
     if (bad) record_error(x.status, KDA_ERR_RANGE, 20);
     fence_proxy_async_smem();
     named_sync(1, 128);
+    if (p == 0) tmark(x, c, 3);
 
     if (fast) {
       // ---- G1: [P ; A_raw] = [QE ; KE] . KH^T   (M=128, N=64, K=128)
@@ -403,6 +420,7 @@ __device__ void prologue_group(const Ctx& x, const float* __restrict__ g, const 
       named_sync(1, 128);
     }
 
+    if (p == 0) tmark(x, c, 4);
     // ---- (a3) T = (I + A)^-1 in 2 x 2 blocks of 32:
     //   D_b = (I + A_bb)^-1 by forward substitution (one column per thread),
     //   T_10 = -D_1 (A_10 D_0);  T' = T diag(beta) as fp16 [r][s].
@@ -494,6 +512,7 @@ __device__ void prologue_group(const Ctx& x, const float* __restrict__ g, const 
     named_sync(1, 128);
 
     // ---- (a4) G2: W'^T = KE^T T'^T -> TM_GW;  G3: U^T = V^T T'^T -> TM_DELTA
+    if (p == 0) tmark(x, c, 5);
     if (p == 0) {
       bool ok = true;
       if (c >= 1) ok = cwait(x, B_DFREE, (c - 1) & 1, 15);  // scan has read Δ of chunk c-1
@@ -521,6 +540,7 @@ __device__ void prologue_group(const Ctx& x, const float* __restrict__ g, const 
     load_g(c + 1, gn, bn);
     if (!gwait(x, B_G23, g23_ph, 16, 1)) break;
     g23_ph ^= 1;
+    if (p == 0) tmark(x, c, 6);
     tc_fence_after();
     if (fast && c >= 1 && !gwait(x, B_WFREE, (c - 1) & 1, 17, 1)) break;
     {  // lane c holds W'^T[c][r]: store row c of the MN-major B operand of D1
@@ -548,7 +568,10 @@ __device__ void prologue_group(const Ctx& x, const float* __restrict__ g, const 
     fence_proxy_async_smem();
     tc_fence_before();
     named_sync(1, 128);
-    if (p == 0) mbar_arrive(&x.bars[B_PRO0 + b2]);
+    if (p == 0) {
+      mbar_arrive(&x.bars[B_PRO0 + b2]);
+      tmark(x, c, 7);
+    }
 #pragma unroll
     for (int m = 0; m < 16; ++m) gv[m] = gn[m];
     bv = bn;
@@ -620,6 +643,7 @@ __device__ void scan_group(const Ctx& x, const void* tmq, const void* tmk, const
     const int b2 = c & 1;
     const uint32_t stg = sb + b2 * STAGE_BYTES;
     const float* s_gc = reinterpret_cast<const float*>(sm + SM_MISC + MS_GC) + b2 * 128;
+    if (j == 0) tmark(x, c, 8);
     if (inject_stuck && c == 0 && !gwait(x, B_NEVER, 0, 99, 2)) {
       ok = false;
       break;
@@ -634,6 +658,7 @@ __device__ void scan_group(const Ctx& x, const void* tmq, const void* tmk, const
       d2_ph ^= 1;
       tc_fence_after();
     }
+    if (j == 0) tmark(x, c, 9);
     if (!gwait(x, B_GC0 + b2, (c >> 1) & 1, 32, 2)) {
       ok = false;
       break;
@@ -664,6 +689,7 @@ __device__ void scan_group(const Ctx& x, const void* tmq, const void* tmk, const
       ok = false;
       break;
     }
+    if (j == 0) tmark(x, c, 10);
 
     // ---- D1: O^T = S'^T QE^T ;  Δ^T = U^T - S'^T W'^T    (A = S'^T from TMEM)
     if (j == 0) {
@@ -684,13 +710,16 @@ __device__ void scan_group(const Ctx& x, const void* tmq, const void* tmk, const
         umma_commit(&x.bars[B_D1]);
         umma_commit(&x.bars[B_WFREE]);
       }
+      tmark(x, c, 11);
     }
     if (c >= 1) store_out(c - 1);
+    if (j == 0) tmark(x, c, 12);
     if (!gwait(x, B_D1, d1_ph, 34, 2)) {
       ok = false;
       break;
     }
     d1_ph ^= 1;
+    if (j == 0) tmark(x, c, 13);
     tc_fence_after();
     // The stage of chunk c is no longer read: fetch chunk c+2 into it.
     if (j == 0 && c + 2 < x.nchunks) {
@@ -734,6 +763,7 @@ __device__ void scan_group(const Ctx& x, const void* tmq, const void* tmk, const
     named_sync(2, 128);
 
     // ---- D2: S^T += Δ^T KH ;  O^T += Δ^T P^T      (A = Δ^T from TMEM)
+    if (j == 0) tmark(x, c, 14);
     if (j == 0) {
       mbar_arrive(&x.bars[B_DFREE]);
       tc_fence_after();
@@ -751,6 +781,7 @@ __device__ void scan_group(const Ctx& x, const void* tmq, const void* tmk, const
       }
       umma_commit(&x.bars[B_D2]);
       umma_commit(&x.bars[B_BUF0 + b2]);
+      tmark(x, c, 15);
     }
   }
   if (named_sync_and(2, 128, ok && !*x.abort) && x.nchunks > 0) {
@@ -813,8 +844,11 @@ __global__ void __launch_bounds__(NTHR, 1)
   }
   x.nchunks = (int)((x.L + CH - 1) / CH);
   x.dbg = (dbg && n == 0 && x.h == 0) ? dbg : nullptr;
+  x.tdbg = x.dbg ? reinterpret_cast<long long*>(x.dbg + DBG_TIME) : nullptr;
+  long long* s_t0 = reinterpret_cast<long long*>(sm + SM_MISC + MS_T0);
 
   if (tid == 0) {
+    *s_t0 = clock64();
     for (int i = 0; i < NUM_BARS; ++i) mbar_init(&x.bars[i], 1);
     fence_mbar_init();
     *x.abort = 0;
@@ -830,6 +864,7 @@ __global__ void __launch_bounds__(NTHR, 1)
   __syncthreads();
   tc_fence_after();
   x.tmem = *reinterpret_cast<volatile uint32_t*>(sm + SM_MISC + MS_TMEM);
+  x.tstart = *s_t0;
   const int64_t sbase = ((int64_t)n * H + x.h) * D * D;
 
   int cnt[2] = {0, 0};  // TMA stages issued (scan group) / consumed (prologue group)
