@@ -50,7 +50,7 @@ namespace {
 
 constexpr int CH = 64;  // chunk length
 constexpr int D = 128;  // dk = dv
-constexpr int NTHR = 256;
+constexpr int NTHR = 384;  // 4 scan warps + 8 prologue warps
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float FAST_MIN_LOG2 = -10.0f;  // chunk-total decay floor (log2) for the tensor-core Gram
 constexpr float F16_SAFE = 60000.0f;     // |x| above this would overflow fp16 operands
@@ -64,9 +64,10 @@ constexpr uint32_t SM_P = SM_KX + 32768;     // P fp16 [r][s], x2            16 
 constexpr uint32_t SM_WT = SM_P + 16384;     // W'^T fp16 [c][r]             16 KB
 constexpr uint32_t SM_A = SM_WT + 16384;     // A fp32 [64][64] -> T' fp16   16 KB
 constexpr uint32_t SM_DG = SM_A + 16384;     // D_0, D_1 fp32 [32][32]        8 KB
-constexpr uint32_t SM_X = SM_DG + 8192;      // X fp32 [32][32]               4 KB
-constexpr uint32_t SM_MISC = SM_X + 4096;
-constexpr uint32_t MISC_BYTES = 4096;
+constexpr uint32_t SM_X = SM_DG + 8192;      // X fp32 [32][32] (Y before)    4 KB
+constexpr uint32_t SM_OST = SM_X + 4096;     // O staging bf16 [64][128]     16 KB
+constexpr uint32_t SM_MISC = SM_OST + 16384;
+constexpr uint32_t MISC_BYTES = 10240;
 constexpr uint32_t SMEM_BYTES = SM_MISC + MISC_BYTES + 1024;
 
 // misc layout
@@ -78,8 +79,9 @@ constexpr uint32_t MS_TMEM = 160, MS_ABORT = 164, MS_FAST = 168, MS_CNT = 176;  
 constexpr uint32_t MS_T0 = 192;  // int64: clock at block start (timing dump)
 constexpr uint32_t MS_BETA = 256;    // [2][64] fp32
 constexpr uint32_t MS_GC = 768;      // [2][128] fp32: exp(G_C)
-constexpr uint32_t MS_RED = 1792;    // [4][128] fp32
-constexpr uint32_t MS_END = 3840;
+constexpr uint32_t MS_RED = 1792;    // [8][128] fp32 log2 sums
+constexpr uint32_t MS_PRD = 5888;    // [8][128] fp32 products
+constexpr uint32_t MS_END = 9984;
 static_assert(NUM_BARS * 8 <= MS_TMEM, "barrier area");
 static_assert(MS_END <= MISC_BYTES, "misc area");
 
@@ -178,16 +180,16 @@ __device__ __forceinline__ bool cwait(const Ctx& x, int bar, uint32_t parity, in
   return false;
 }
 
-// Group-uniform bounded wait: every thread of named-barrier group `grp` (128
-// threads) polls, then the group agrees on the outcome, so no thread can
+// Group-uniform bounded wait: every thread of named-barrier group `grp`
+// (nthr threads) polls, then the group agrees on the outcome, so no thread can
 // leave a loop while the others wait at a barrier or a .sync.aligned op.
-__device__ __forceinline__ bool gwait(const Ctx& x, int bar, uint32_t parity, int where, int grp) {
+__device__ __forceinline__ bool gwait(const Ctx& x, int bar, uint32_t parity, int where, int grp, int nthr) {
   bool ok = wait_bar(&x.bars[bar], parity, x.wait_ns, x.abort);
   if (!ok) {
     if (!*x.abort) record_error(x.status, KDA_ERR_TIMEOUT, where);
     *x.abort = 1;
   }
-  return named_sync_and(grp, 128, ok);
+  return named_sync_and(grp, nthr, ok);
 }
 
 __device__ __forceinline__ int chunk_valid(const Ctx& x, int c) {
@@ -196,31 +198,135 @@ __device__ __forceinline__ int chunk_valid(const Ctx& x, int c) {
 }
 
 // ======================================================== prologue group
+// 8 warps (256 threads).  Row-wise work: thread (rg = warp 0..7, lane) owns
+// rows 8 rg .. 8 rg + 7 and channels 4 lane .. 4 lane + 3.  TMEM work: warp
+// rg reads lane quarter rg % 4 and column half rg / 4.
+constexpr int PG_THREADS = 256;
+
+// General chunks: P and A on CUDA cores from the exact decay differences
+// G_r - G_s (log2 units), staged through the W'^T tile in two channel halves.
+__device__ __forceinline__ void general_gram(const Ctx& x, uint32_t stg, int b2, int valid, const float4 (&G)[8]) {
+  const int p = threadIdx.x - 128;
+  const int rg = p >> 5, lane = p & 31;
+  const int ch0 = 4 * lane, hh = ch0 >> 6, cc = ch0 & 63;
+  uint8_t* sm = x.sm;
+  const float* s_beta = reinterpret_cast<const float*>(sm + SM_MISC + MS_BETA) + b2 * 64;
+  const int r = p & 63, s0 = (p >> 6) * 16;
+  float pa[16], aa[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) pa[i] = aa[i] = 0.f;
+  for (int half = 0; half < 2; ++half) {
+    named_sync(1, PG_THREADS);
+    if (hh == half) {
+#pragma unroll
+      for (int m = 0; m < 8; ++m) *reinterpret_cast<float4*>(sm + SM_WT + (8 * rg + m) * 256 + cc * 4) = G[m];
+    }
+    named_sync(1, PG_THREADS);
+    if (r < valid && s0 <= r) {
+#pragma unroll 1
+      for (int ch = 0; ch < 64; ++ch) {
+        const uint32_t off_r = half * 16384 + sw128_off(r, ch);
+        const float gr = *reinterpret_cast<const float*>(sm + SM_WT + r * 256 + ch * 4);
+        const float qr = ld_bf16(stg + OFF_QK + off_r), kr = ld_bf16(stg + OFF_QK + 8192 + off_r);
+#pragma unroll 4
+        for (int i = 0; i < 16; ++i) {
+          const int s = s0 + i;
+          if (s <= r) {
+            const float gs = *reinterpret_cast<const float*>(sm + SM_WT + s * 256 + ch * 4);
+            const float ks = ld_bf16(stg + OFF_QK + 8192 + half * 16384 + sw128_off(s, ch));
+            const float e = ex2(gr - gs) * ks;
+            pa[i] += qr * e;
+            aa[i] += kr * e;
+          }
+        }
+      }
+    }
+  }
+  const float br = s_beta[r];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int s = s0 + i;
+    aa[i] = s < r ? br * aa[i] : 0.f;
+    if (!(s <= r)) pa[i] = 0.f;
+  }
+#pragma unroll
+  for (int q8 = 0; q8 < 2; ++q8) {
+    const int s = s0 + 8 * q8;
+    st_f16x8(x.sb + SM_P + b2 * 8192 + r * 128 + ((((s >> 3) ^ r) & 7) << 4), pa + 8 * q8);
+  }
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+    *reinterpret_cast<float4*>(sm + SM_A + a_off(r, s0 + 4 * u)) =
+        make_float4(aa[4 * u], aa[4 * u + 1], aa[4 * u + 2], aa[4 * u + 3]);
+  named_sync(1, PG_THREADS);  // raw Q/K reads are done before they are rescaled in place
+}
+
+// Debug dump of P (fp16 tile) and A (fp32 tile) for chunk 0 of chain 0.
+__device__ __noinline__ void dump_pa(float* dbg, const uint8_t* sm, int b2) {
+  const int p = threadIdx.x - 128;
+  for (int e = p; e < 4096; e += PG_THREADS) {
+    const int r = e >> 6, s = e & 63;
+    const uint16_t u = *reinterpret_cast<const uint16_t*>(sm + SM_P + b2 * 8192 + sw128_off(r, s));
+    dbg[DBG_P + e] = __half2float(*reinterpret_cast<const __half*>(&u));
+    dbg[DBG_A + e] = *reinterpret_cast<const float*>(sm + SM_A + a_off(r, s));
+  }
+}
+// Debug dump of T' (fp16 tile).
+__device__ __noinline__ void dump_t(float* dbg, const uint8_t* sm) {
+  const int p = threadIdx.x - 128;
+  for (int e = p; e < 4096; e += PG_THREADS) {
+    const uint16_t u = *reinterpret_cast<const uint16_t*>(sm + SM_A + sw128_off(e >> 6, e & 63));
+    dbg[DBG_T + e] = __half2float(*reinterpret_cast<const __half*>(&u));
+  }
+}
+// Debug dump of W' (from the fp16 W'^T tile) and U (TMEM, before D1).
+__device__ __noinline__ void dump_wu(float* dbg, const uint8_t* sm, uint32_t tmem) {
+  const int p = threadIdx.x - 128;
+  for (int e = p; e < 8192; e += PG_THREADS) {
+    const int r = e >> 7, c = e & 127;  // W'[r][c] = W'^T[c][r]
+    const uint16_t u = *reinterpret_cast<const uint16_t*>(sm + SM_WT + sw128_off(c, r));
+    dbg[DBG_W + e] = __half2float(*reinterpret_cast<const __half*>(&u));
+  }
+  const int rg = p >> 5;
+  if (rg < 4) {  // warps 4..7 read lane quarter rg of U^T
+    const uint32_t tl = tmem + ((uint32_t)(rg * 32) << 16);
+    const int j = rg * 32 + (p & 31);
+    float u0[32];
+    for (int half = 0; half < 2; ++half) {
+      tmem_ld32(tl + TM_DELTA + half * 32, u0);
+      for (int i = 0; i < 32; ++i) dbg[DBG_U + (half * 32 + i) * 128 + j] = u0[i];
+    }
+  }
+}
+
 __device__ void prologue_group(const Ctx& x, const float* __restrict__ g, const float* __restrict__ beta,
                                int (&consumed)[2]) {
-  const int p = threadIdx.x - 128;  // 0..127, also the TMEM lane
-  const int rq = p >> 5, cq = p & 31;  // rows 16 rq.., channels 4 cq..
-  const int ch0 = 4 * cq, hh = ch0 >> 6, cc = ch0 & 63;
-  const uint32_t tl = x.tmem + ((uint32_t)(rq * 32) << 16);
+  const int p = threadIdx.x - 128;  // 0..255
+  const int rg = p >> 5, lane = p & 31;
+  const int ch0 = 4 * lane, hh = ch0 >> 6, cc = ch0 & 63;
+  const int lq = rg & 3, chalf = rg >> 2;  // TMEM lane quarter, column half
+  const uint32_t tl = x.tmem + ((uint32_t)(lq * 32) << 16);
+  const int ti = lq * 32 + lane;  // this thread's TMEM lane
   uint8_t* sm = x.sm;
   const uint32_t sb = x.sb;
-  float* s_red = reinterpret_cast<float*>(sm + SM_MISC + MS_RED);
+  float* s_red = reinterpret_cast<float*>(sm + SM_MISC + MS_RED);   // [8][128] log2 sums
+  float* s_prd = reinterpret_cast<float*>(sm + SM_MISC + MS_PRD);   // [8][128] products
   const int H = x.H;
 
-  // Register prefetch of this thread's g rows and of beta for chunk c.
-  auto load_g = [&](int c, float4(&gv)[16], float& bv) {
+  // Register prefetch of this thread's g rows (8 x float4) and of beta.
+  auto load_g = [&](int c, float4(&gv)[8], float& bv) {
     const int valid = c < x.nchunks ? chunk_valid(x, c) : 0;
     const int64_t tok0 = x.t0 + (int64_t)c * CH;
 #pragma unroll
-    for (int m = 0; m < 16; ++m) {
-      const int r = 16 * rq + m;
+    for (int m = 0; m < 8; ++m) {
+      const int r = 8 * rg + m;
       gv[m] = r < valid ? __ldg(reinterpret_cast<const float4*>(g + ((tok0 + r) * H + x.h) * D + ch0))
                         : make_float4(0.f, 0.f, 0.f, 0.f);
     }
     bv = (p < CH && p < valid) ? __ldg(beta + (tok0 + p) * H + x.h) : 0.f;
   };
 
-  float4 gv[16];
+  float4 gv[8];
   float bv;
   load_g(0, gv, bv);
   int g1_ph = 0, g23_ph = 0;
@@ -236,133 +342,107 @@ __device__ void prologue_group(const Ctx& x, const float* __restrict__ g, const 
 
     if (p == 0) tmark(x, c, 0);
     // Buffers [b2] were last used by the scan of chunk c-2.
-    if (c >= 2 && !gwait(x, B_BUF0 + b2, ((c >> 1) - 1) & 1, 11, 1)) break;
-    if (!gwait(x, B_FULL0 + b2, (c >> 1) & 1, 12, 1)) break;
+    if (c >= 2 && !gwait(x, B_BUF0 + b2, ((c >> 1) - 1) & 1, 11, 1, PG_THREADS)) break;
+    if (!gwait(x, B_FULL0 + b2, (c >> 1) & 1, 12, 1, PG_THREADS)) break;
     ++consumed[b2];
     if (p == 0) tmark(x, c, 1);
 
-    // ---- (a1) cumulative decay in log2 units
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    // ---- (a1) decay factors.  alpha = e^g (one MUFU op per element); the
+    // cumulative products give e^{G_r} and e^{G_C - G_r}, and the log2 sums
+    // give G for the range test and the general variant.
+    float4 fw[8], bw[8];
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f), pr = make_float4(1.f, 1.f, 1.f, 1.f);
 #pragma unroll
-    for (int m = 0; m < 16; ++m) {
-      acc.x += gv[m].x * LOG2E; acc.y += gv[m].y * LOG2E; acc.z += gv[m].z * LOG2E; acc.w += gv[m].w * LOG2E;
-      gv[m] = acc;  // gv now holds the local inclusive prefix
+    for (int m = 0; m < 8; ++m) {
+      const float4 l = make_float4(gv[m].x * LOG2E, gv[m].y * LOG2E, gv[m].z * LOG2E, gv[m].w * LOG2E);
+      bw[m] = ex2_4(l);  // alpha of row m (kept for the suffix products)
+      acc.x += l.x; acc.y += l.y; acc.z += l.z; acc.w += l.w;
+      pr = mul4(pr, bw[m]);
+      gv[m] = acc;  // local inclusive log2 prefix
+      fw[m] = pr;   // local inclusive product
     }
-    *reinterpret_cast<float4*>(s_red + rq * 128 + ch0) = acc;
-    named_sync(1, 128);
-    float4 tot = make_float4(0.f, 0.f, 0.f, 0.f), off = tot;
+    {
+      float4 sp = make_float4(1.f, 1.f, 1.f, 1.f);  // suffix products within the 8 rows
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
+      for (int m = 7; m >= 0; --m) {
+        const float4 a = bw[m];
+        bw[m] = sp;
+        sp = mul4(sp, a);
+      }
+    }
+    *reinterpret_cast<float4*>(s_red + rg * 128 + ch0) = acc;
+    *reinterpret_cast<float4*>(s_prd + rg * 128 + ch0) = pr;
+    named_sync(1, PG_THREADS);
+    float4 tot = make_float4(0.f, 0.f, 0.f, 0.f), off = tot;
+    float4 fo = make_float4(1.f, 1.f, 1.f, 1.f), bo = fo;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
       const float4 v = *reinterpret_cast<const float4*>(s_red + q * 128 + ch0);
-      if (q < rq) { off.x += v.x; off.y += v.y; off.z += v.z; off.w += v.w; }
+      const float4 w = *reinterpret_cast<const float4*>(s_prd + q * 128 + ch0);
+      if (q < rg) {
+        off.x += v.x; off.y += v.y; off.z += v.z; off.w += v.w;
+        fo = mul4(fo, w);
+      }
+      if (q > rg) bo = mul4(bo, w);
       tot.x += v.x; tot.y += v.y; tot.z += v.z; tot.w += v.w;
     }
 #pragma unroll
-    for (int m = 0; m < 16; ++m) {
+    for (int m = 0; m < 8; ++m) {
       gv[m].x += off.x; gv[m].y += off.y; gv[m].z += off.z; gv[m].w += off.w;  // G (log2)
     }
-    const bool fast = named_sync_and(1, 128, fminf(fminf(tot.x, tot.y), fminf(tot.z, tot.w)) >= FAST_MIN_LOG2);
-    if (rq == 0) *reinterpret_cast<float4*>(s_gc + ch0) = ex2_4(tot);
+    const bool fast =
+        named_sync_and(1, PG_THREADS, fminf(fminf(tot.x, tot.y), fminf(tot.z, tot.w)) >= FAST_MIN_LOG2);
+    if (rg == 0) *reinterpret_cast<float4*>(s_gc + ch0) = ex2_4(tot);
     if (p == 0) *s_fast = fast ? 1 : 0;
     if (p < CH) s_beta[p] = bv;
-    if (dmp && rq == 0) {
+    if (dmp && rg == 0) {
       const float LN2 = 0.6931471805599453f;
       x.dbg[DBG_GC + ch0] = tot.x * LN2; x.dbg[DBG_GC + ch0 + 1] = tot.y * LN2;
       x.dbg[DBG_GC + ch0 + 2] = tot.z * LN2; x.dbg[DBG_GC + ch0 + 3] = tot.w * LN2;
     }
-    named_sync(1, 128);
+    named_sync(1, PG_THREADS);
     if (p == 0) {
       mbar_arrive(&x.bars[B_GC0 + b2]);
       tmark(x, c, 2);
     }
-
-    const uint32_t qb = stg + OFF_QK + hh * 16384, kb = qb + 8192;
-    const uint32_t vb = stg + OFF_V + hh * 8192;
-    const uint32_t khb = sb + SM_KX + b2 * 16384 + hh * 8192;
-    const float4 ref = fast ? tot : make_float4(0.f, 0.f, 0.f, 0.f);
-    bool bad = false;
+    // Row factors: E = e^{G_r - ref} (ref = G_C on fast chunks, 0 otherwise), H = e^{G_C - G_r}.
+    {
+      float4 ef = fo;
+      if (fast) ef = mul4(ef, ex2_4(make_float4(-tot.x, -tot.y, -tot.z, -tot.w)));
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        fw[m] = mul4(fw[m], ef);
+        bw[m] = mul4(bw[m], bo);
+      }
+    }
 
     if (!fast) {
-      // ---- general variant: Gram matrices on CUDA cores from exact decay
-      // differences.  G is staged through the W'^T tile in two channel
-      // halves (fp32 [64][64]); that tile is free once D1 of chunk c-1 is done.
-      if (c >= 1 && !gwait(x, B_WFREE, (c - 1) & 1, 13, 1)) break;
-      const int r = p & 63, s0 = (p >> 6) * 32;
-      float pa[32], aa[32];
-#pragma unroll
-      for (int i = 0; i < 32; ++i) pa[i] = aa[i] = 0.f;
-      for (int half = 0; half < 2; ++half) {
-        named_sync(1, 128);
-        if (hh == half) {
-#pragma unroll
-          for (int m = 0; m < 16; ++m)
-            *reinterpret_cast<float4*>(sm + SM_WT + (16 * rq + m) * 256 + cc * 4) = gv[m];
-        }
-        named_sync(1, 128);
-        if (r < valid) {
-          for (int ch = 0; ch < 64; ++ch) {
-            const uint32_t off_r = half * 16384 + sw128_off(r, ch);
-            const float gr = *reinterpret_cast<const float*>(sm + SM_WT + r * 256 + ch * 4);
-            const float qr = ld_bf16(stg + OFF_QK + off_r), kr = ld_bf16(stg + OFF_QK + 8192 + off_r);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const int s = s0 + i;
-              if (s <= r) {
-                const float gs = *reinterpret_cast<const float*>(sm + SM_WT + s * 256 + ch * 4);
-                const float ks = ld_bf16(stg + OFF_QK + 8192 + half * 16384 + sw128_off(s, ch));
-                const float e = ex2(gr - gs) * ks;
-                pa[i] += qr * e;
-                aa[i] += kr * e;
-              }
-            }
-          }
-        }
-      }
-      const float br = s_beta[r];
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const int s = s0 + i;
-        aa[i] = s < r ? br * aa[i] : 0.f;
-        if (!(s <= r)) pa[i] = 0.f;
-      }
-#pragma unroll
-      for (int q8 = 0; q8 < 4; ++q8) {
-        const int s = s0 + 8 * q8;
-        st_f16x8(sb + SM_P + b2 * 8192 + r * 128 + ((((s >> 3) ^ r) & 7) << 4), pa + 8 * q8);
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u)
-        *reinterpret_cast<float4*>(sm + SM_A + a_off(r, s0 + 4 * u)) =
-            make_float4(aa[4 * u], aa[4 * u + 1], aa[4 * u + 2], aa[4 * u + 3]);
-      if (dmp) {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          x.dbg[DBG_P + r * 64 + s0 + i] = pa[i];
-          x.dbg[DBG_A + r * 64 + s0 + i] = aa[i];
-        }
-      }
-      named_sync(1, 128);  // raw Q/K reads are done before they are rescaled in place
+      if (c >= 1 && !gwait(x, B_WFREE, (c - 1) & 1, 13, 1, PG_THREADS)) break;
+      general_gram(x, stg, b2, valid, gv);
     }
 
     // ---- (a2) operand scaling: QE, KE in place, KH into KX[b2], V -> fp16.
+    {
+      const uint32_t qb = stg + OFF_QK + hh * 16384, kb = qb + 8192;
+      const uint32_t vb = stg + OFF_V + hh * 8192;
+      const uint32_t khb = sb + SM_KX + b2 * 16384 + hh * 8192;
+      bool bad = false;
 #pragma unroll
-    for (int m = 0; m < 16; ++m) {
-      const int r = 16 * rq + m;
-      const uint32_t o = sw128_off(r, cc);
-      float4 q4 = ld_bf16x4(qb + o), k4 = ld_bf16x4(kb + o), v4 = ld_bf16x4(vb + o);
-      if (r >= valid) q4 = k4 = v4 = make_float4(0.f, 0.f, 0.f, 0.f);
-      const float4 e = ex2_4(make_float4(gv[m].x - ref.x, gv[m].y - ref.y, gv[m].z - ref.z, gv[m].w - ref.w));
-      const float4 hcoef =
-          ex2_4(make_float4(tot.x - gv[m].x, tot.y - gv[m].y, tot.z - gv[m].z, tot.w - gv[m].w));
-      bad |= amax4(v4) > F16_SAFE;
-      st_f16x4(qb + o, mul4(q4, e));
-      st_f16x4(kb + o, mul4(k4, e));
-      st_f16x4(vb + o, v4);
-      st_f16x4(khb + o, mul4(k4, hcoef));
+      for (int m = 0; m < 8; ++m) {
+        const int r = 8 * rg + m;
+        const uint32_t o = sw128_off(r, cc);
+        float4 q4 = ld_bf16x4(qb + o), k4 = ld_bf16x4(kb + o), v4 = ld_bf16x4(vb + o);
+        if (r >= valid) q4 = k4 = v4 = make_float4(0.f, 0.f, 0.f, 0.f);
+        bad |= amax4(v4) > F16_SAFE;
+        st_f16x4(qb + o, mul4(q4, fw[m]));
+        st_f16x4(kb + o, mul4(k4, fw[m]));
+        st_f16x4(vb + o, v4);
+        st_f16x4(khb + o, mul4(k4, bw[m]));
+      }
+      if (bad) record_error(x.status, KDA_ERR_RANGE, 20);
     }
-    if (bad) record_error(x.status, KDA_ERR_RANGE, 20);
     fence_proxy_async_smem();
-    named_sync(1, 128);
+    named_sync(1, PG_THREADS);
     if (p == 0) tmark(x, c, 3);
 
     if (fast) {
@@ -378,142 +458,154 @@ __device__ void prologue_group(const Ctx& x, const float* __restrict__ g, const 
         }
         umma_commit(&x.bars[B_G1]);
       }
-      if (!gwait(x, B_G1, g1_ph, 14, 1)) break;
+      if (!gwait(x, B_G1, g1_ph, 14, 1, PG_THREADS)) break;
       g1_ph ^= 1;
       tc_fence_after();
-      float r0[32], r1[32];
-      tmem_ld32(tl + TM_GW, r0);
-      tmem_ld32(tl + TM_GW + 32, r1);
-      if (p < CH) {  // P row p, lower triangle including the diagonal
+      float r0[32];
+      tmem_ld32(tl + TM_GW + chalf * 32, r0);  // row ti, columns 32 chalf .. +31
+      if (ti < CH) {  // P row, lower triangle including the diagonal
 #pragma unroll
-        for (int s = 0; s < 32; ++s) {
-          if (s > p) r0[s] = 0.f;
-          if (s + 32 > p) r1[s] = 0.f;
-        }
+        for (int s = 0; s < 32; ++s)
+          if (chalf * 32 + s > ti) r0[s] = 0.f;
 #pragma unroll
-        for (int q8 = 0; q8 < 8; ++q8)
-          st_f16x8(sb + SM_P + b2 * 8192 + p * 128 + (((q8 ^ p) & 7) << 4),
-                   q8 < 4 ? r0 + 8 * q8 : r1 + 8 * (q8 - 4));
-        if (dmp) {
-#pragma unroll
-          for (int s = 0; s < 64; ++s) x.dbg[DBG_P + p * 64 + s] = s < 32 ? r0[s] : r1[s - 32];
+        for (int k = 0; k < 4; ++k) {
+          const int q8 = chalf * 4 + k;
+          st_f16x8(sb + SM_P + b2 * 8192 + ti * 128 + (((q8 ^ ti) & 7) << 4), r0 + 8 * k);
         }
       } else {  // A row r = beta_r (KE KH^T)_rs, strictly lower
-        const int r = p - CH;
+        const int r = ti - CH;
         const float b = s_beta[r];
 #pragma unroll
-        for (int s = 0; s < 32; ++s) {
-          r0[s] = s < r ? b * r0[s] : 0.f;
-          r1[s] = s + 32 < r ? b * r1[s] : 0.f;
-        }
+        for (int s = 0; s < 32; ++s) r0[s] = (chalf * 32 + s < r) ? b * r0[s] : 0.f;
 #pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          const float* v = u < 8 ? r0 + 4 * u : r1 + 4 * (u - 8);
-          *reinterpret_cast<float4*>(sm + SM_A + a_off(r, 4 * u)) = make_float4(v[0], v[1], v[2], v[3]);
-        }
-        if (dmp) {
-#pragma unroll
-          for (int s = 0; s < 64; ++s) x.dbg[DBG_A + r * 64 + s] = s < 32 ? r0[s] : r1[s - 32];
-        }
+        for (int u = 0; u < 8; ++u)
+          *reinterpret_cast<float4*>(sm + SM_A + a_off(r, chalf * 32 + 4 * u)) =
+              make_float4(r0[4 * u], r0[4 * u + 1], r0[4 * u + 2], r0[4 * u + 3]);
       }
       tc_fence_before();
-      named_sync(1, 128);
+      named_sync(1, PG_THREADS);
     }
-
+    if (dmp) {
+      dump_pa(x.dbg, sm, b2);
+      named_sync(1, PG_THREADS);
+    }
     if (p == 0) tmark(x, c, 4);
-    // ---- (a3) T = (I + A)^-1 in 2 x 2 blocks of 32:
-    //   D_b = (I + A_bb)^-1 by forward substitution (one column per thread),
-    //   T_10 = -D_1 (A_10 D_0);  T' = T diag(beta) as fp16 [r][s].
+
+    // ---- (a3) T = (I + A)^-1 by blocks.  16x16 diagonal inverses E_a by
+    // forward substitution; D_b = [[E_2b, 0], [-E_2b+1 A'_b E_2b, E_2b+1]] are
+    // the 32x32 diagonal inverses; T_10 = -D_1 (A_10 D_0).
+    // T' = T diag(beta) as fp16 [r][s] over the A tile.
     if (p < 64) {
-      const int bk = p >> 5, jj = p & 31;
-      float xs[32];
+      const int a = p >> 4, jj = p & 15;
+      float xs[16];
 #pragma unroll
-      for (int r = 0; r < 32; ++r) xs[r] = 0.f;
+      for (int r = 0; r < 16; ++r) xs[r] = 0.f;
 #pragma unroll
-      for (int r = 0; r < 32; ++r) {
+      for (int r = 0; r < 16; ++r) {
         float a0 = (r == jj) ? 1.f : 0.f, a1 = 0.f;
 #pragma unroll
         for (int u = 0; u < (r + 3) / 4; ++u) {
-          const float4 a4 = *reinterpret_cast<const float4*>(sm + SM_A + a_off(32 * bk + r, 32 * bk + 4 * u));
+          const float4 a4 = *reinterpret_cast<const float4*>(sm + SM_A + a_off(16 * a + r, 16 * a + 4 * u));
           a0 -= a4.x * xs[4 * u] + a4.z * xs[4 * u + 2];
           a1 -= a4.y * xs[4 * u + 1] + a4.w * xs[4 * u + 3];
         }
         xs[r] = a0 + a1;
       }
+      // E_a -> diagonal 16x16 block of D_{a/2}
+      const uint32_t db = SM_DG + (a >> 1) * 4096;
+      const int o = (a & 1) * 16;
 #pragma unroll
-      for (int r = 0; r < 32; ++r) *reinterpret_cast<float*>(sm + SM_DG + bk * 4096 + b_off(r, jj)) = xs[r];
+      for (int r = 0; r < 16; ++r) *reinterpret_cast<float*>(sm + db + b_off(o + r, o + jj)) = xs[r];
+    } else if (p < 128) {  // zero the upper-right 16x16 block of D_0 and D_1
+      const int t = p - 64, b = t >> 5, rr = (t & 31) >> 1, cb = 16 + (t & 1) * 8;
+#pragma unroll
+      for (int i = 0; i < 8; i += 4)
+        *reinterpret_cast<float4*>(sm + SM_DG + b * 4096 + b_off(rr, cb + i)) = make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    named_sync(1, 128);
-    const int rr = p >> 2, q8 = p & 3;  // output row rr, columns 8 q8 .. 8 q8 + 7 of a 32x32 block
-    {
-      float o8[8];
+    named_sync(1, PG_THREADS);
+    {  // Y_b = A'_b E_2b  (A'_b = A[32b+16 .. +16][32b .. +16]) -> X tile as [2][16][16]
+      const int b = p >> 7, o = p & 127, r = o >> 3, c0 = 2 * (o & 7);
+      float y0 = 0.f, y1 = 0.f;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) o8[i] = 0.f;
+      for (int u = 0; u < 4; ++u) {
+        const float4 a4 = *reinterpret_cast<const float4*>(sm + SM_A + a_off(32 * b + 16 + r, 32 * b + 4 * u));
+        const float av[4] = {a4.x, a4.y, a4.z, a4.w};
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {  // X = A_10 D_0
+        for (int t = 0; t < 4; ++t) {
+          const int s = 4 * u + t;
+          const float2 e = *reinterpret_cast<const float2*>(sm + SM_DG + b * 4096 + b_off(s, c0));
+          y0 += av[t] * e.x;
+          y1 += av[t] * e.y;
+        }
+      }
+      *reinterpret_cast<float2*>(sm + SM_X + b * 1024 + r * 64 + c0 * 4) = make_float2(y0, y1);
+    }
+    named_sync(1, PG_THREADS);
+    {  // F_b = -E_2b+1 Y_b -> lower-left 16x16 block of D_b
+      const int b = p >> 7, o = p & 127, r = o >> 3, c0 = 2 * (o & 7);
+      float f0 = 0.f, f1 = 0.f;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float4 e4 = *reinterpret_cast<const float4*>(sm + SM_DG + b * 4096 + b_off(16 + r, 16 + 4 * u));
+        const float ev[4] = {e4.x, e4.y, e4.z, e4.w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const int s = 4 * u + t;
+          const float2 y = *reinterpret_cast<const float2*>(sm + SM_X + b * 1024 + s * 64 + c0 * 4);
+          f0 -= ev[t] * y.x;
+          f1 -= ev[t] * y.y;
+        }
+      }
+      *reinterpret_cast<float2*>(sm + SM_DG + b * 4096 + b_off(16 + r, c0)) = make_float2(f0, f1);
+    }
+    named_sync(1, PG_THREADS);
+    const int rr = p >> 3, c4 = 4 * (p & 7);  // 32x32 output row rr, columns c4 .. c4+3
+    {  // X = A_10 D_0
+      float4 o4 = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
         const float4 a4 = *reinterpret_cast<const float4*>(sm + SM_A + a_off(32 + rr, 4 * u));
         const float av[4] = {a4.x, a4.y, a4.z, a4.w};
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
-          const int s = 4 * u + t;
-          const float4 d0 = *reinterpret_cast<const float4*>(sm + SM_DG + b_off(s, 8 * q8));
-          const float4 d1 = *reinterpret_cast<const float4*>(sm + SM_DG + b_off(s, 8 * q8 + 4));
-          o8[0] += av[t] * d0.x; o8[1] += av[t] * d0.y; o8[2] += av[t] * d0.z; o8[3] += av[t] * d0.w;
-          o8[4] += av[t] * d1.x; o8[5] += av[t] * d1.y; o8[6] += av[t] * d1.z; o8[7] += av[t] * d1.w;
+          const float4 d = *reinterpret_cast<const float4*>(sm + SM_DG + b_off(4 * u + t, c4));
+          o4.x += av[t] * d.x; o4.y += av[t] * d.y; o4.z += av[t] * d.z; o4.w += av[t] * d.w;
         }
       }
-      *reinterpret_cast<float4*>(sm + SM_X + b_off(rr, 8 * q8)) = make_float4(o8[0], o8[1], o8[2], o8[3]);
-      *reinterpret_cast<float4*>(sm + SM_X + b_off(rr, 8 * q8 + 4)) = make_float4(o8[4], o8[5], o8[6], o8[7]);
+      *reinterpret_cast<float4*>(sm + SM_X + b_off(rr, c4)) = o4;
     }
-    named_sync(1, 128);
-    {
-      float o8[8];
+    named_sync(1, PG_THREADS);
+    {  // T_10 = -D_1 X, then T' = T diag(beta) as fp16
+      float4 o4 = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) o8[i] = 0.f;
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {  // T_10 = -D_1 X
+      for (int u = 0; u < 8; ++u) {
         const float4 a4 = *reinterpret_cast<const float4*>(sm + SM_DG + 4096 + b_off(rr, 4 * u));
         const float av[4] = {a4.x, a4.y, a4.z, a4.w};
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
-          const int s = 4 * u + t;
-          const float4 d0 = *reinterpret_cast<const float4*>(sm + SM_X + b_off(s, 8 * q8));
-          const float4 d1 = *reinterpret_cast<const float4*>(sm + SM_X + b_off(s, 8 * q8 + 4));
-          o8[0] -= av[t] * d0.x; o8[1] -= av[t] * d0.y; o8[2] -= av[t] * d0.z; o8[3] -= av[t] * d0.w;
-          o8[4] -= av[t] * d1.x; o8[5] -= av[t] * d1.y; o8[6] -= av[t] * d1.z; o8[7] -= av[t] * d1.w;
+          const float4 d = *reinterpret_cast<const float4*>(sm + SM_X + b_off(4 * u + t, c4));
+          o4.x -= av[t] * d.x; o4.y -= av[t] * d.y; o4.z -= av[t] * d.z; o4.w -= av[t] * d.w;
         }
       }
-      float d0v[8], d1v[8], z8[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float bl = s_beta[8 * q8 + i], bh = s_beta[32 + 8 * q8 + i];
-        d0v[i] = *reinterpret_cast<const float*>(sm + SM_DG + b_off(rr, 8 * q8 + i)) * bl;
-        d1v[i] = *reinterpret_cast<const float*>(sm + SM_DG + 4096 + b_off(rr, 8 * q8 + i)) * bh;
-        o8[i] *= bl;
-        z8[i] = 0.f;
-      }
-      named_sync(1, 128);  // every read of A is done before T' overwrites its first half
-      // T' rows rr and 32+rr, 16-byte chunks at columns 8 q8 and 32 + 8 q8.
-      st_f16x8(sb + SM_A + sw128_off(rr, 8 * q8), d0v);
-      st_f16x8(sb + SM_A + sw128_off(rr, 32 + 8 * q8), z8);
-      st_f16x8(sb + SM_A + sw128_off(32 + rr, 8 * q8), o8);
-      st_f16x8(sb + SM_A + sw128_off(32 + rr, 32 + 8 * q8), d1v);
-      if (dmp) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          x.dbg[DBG_T + rr * 64 + 8 * q8 + i] = d0v[i];
-          x.dbg[DBG_T + rr * 64 + 32 + 8 * q8 + i] = 0.f;
-          x.dbg[DBG_T + (32 + rr) * 64 + 8 * q8 + i] = o8[i];
-          x.dbg[DBG_T + (32 + rr) * 64 + 32 + 8 * q8 + i] = d1v[i];
-        }
-      }
+      const float4 bl = *reinterpret_cast<const float4*>(s_beta + c4);
+      const float4 bh = *reinterpret_cast<const float4*>(s_beta + 32 + c4);
+      const float4 d0 = *reinterpret_cast<const float4*>(sm + SM_DG + b_off(rr, c4));
+      const float4 d1 = *reinterpret_cast<const float4*>(sm + SM_DG + 4096 + b_off(rr, c4));
+      st_f16x4(sb + SM_A + sw128_off(rr, c4), mul4(d0, bl));
+      st_f16x4(sb + SM_A + sw128_off(rr, 32 + c4), make_float4(0.f, 0.f, 0.f, 0.f));
+      st_f16x4(sb + SM_A + sw128_off(32 + rr, c4), mul4(o4, bl));
+      st_f16x4(sb + SM_A + sw128_off(32 + rr, 32 + c4), mul4(d1, bh));
     }
     fence_proxy_async_smem();
-    named_sync(1, 128);
+    named_sync(1, PG_THREADS);
+    if (dmp) {
+      dump_t(x.dbg, sm);
+      named_sync(1, PG_THREADS);
+    }
 
     // ---- (a4) G2: W'^T = KE^T T'^T -> TM_GW;  G3: U^T = V^T T'^T -> TM_DELTA
-    if (p == 0) tmark(x, c, 5);
     if (p == 0) {
+      tmark(x, c, 5);
       bool ok = true;
       if (c >= 1) ok = cwait(x, B_DFREE, (c - 1) & 1, 15);  // scan has read Δ of chunk c-1
       if (ok) {
@@ -535,51 +627,73 @@ __device__ void prologue_group(const Ctx& x, const float* __restrict__ g, const 
       }
     }
     // Prefetch next chunk's decay and beta while the UMMAs run.
-    float4 gn[16];
+    float4 gn[8];
     float bn;
     load_g(c + 1, gn, bn);
-    if (!gwait(x, B_G23, g23_ph, 16, 1)) break;
+    if (!gwait(x, B_G23, g23_ph, 16, 1, PG_THREADS)) break;
     g23_ph ^= 1;
-    if (p == 0) tmark(x, c, 6);
     tc_fence_after();
-    if (fast && c >= 1 && !gwait(x, B_WFREE, (c - 1) & 1, 17, 1)) break;
-    {  // lane c holds W'^T[c][r]: store row c of the MN-major B operand of D1
-      float w0[32], w1[32];
-      tmem_ld32(tl + TM_GW, w0);
-      tmem_ld32(tl + TM_GW + 32, w1);
+    if (p == 0) tmark(x, c, 6);
+    if (fast && c >= 1 && !gwait(x, B_WFREE, (c - 1) & 1, 17, 1, PG_THREADS)) break;
+    {  // lane ti holds W'^T[ti][r] for r in this warp's column half: row ti of the MN-major B operand of D1
+      float w0[32];
+      tmem_ld32(tl + TM_GW + chalf * 32, w0);
       float mx = 0.f;
 #pragma unroll
-      for (int i = 0; i < 32; ++i) mx = fmaxf(mx, fmaxf(fabsf(w0[i]), fabsf(w1[i])));
+      for (int i = 0; i < 32; ++i) mx = fmaxf(mx, fabsf(w0[i]));
       if (!(mx <= F16_SAFE)) record_error(x.status, KDA_ERR_RANGE, 21);
 #pragma unroll
-      for (int q = 0; q < 8; ++q)
-        st_f16x8(sb + SM_WT + p * 128 + (((q ^ p) & 7) << 4), q < 4 ? w0 + 8 * q : w1 + 8 * (q - 4));
-      if (dmp) {
-        float u0[32], u1[32];
-        tmem_ld32(tl + TM_DELTA, u0);
-        tmem_ld32(tl + TM_DELTA + 32, u1);
-#pragma unroll
-        for (int r = 0; r < 64; ++r) {
-          x.dbg[DBG_W + r * 128 + p] = r < 32 ? w0[r] : w1[r - 32];
-          x.dbg[DBG_U + r * 128 + p] = r < 32 ? u0[r] : u1[r - 32];
-        }
+      for (int k = 0; k < 4; ++k) {
+        const int q = chalf * 4 + k;
+        st_f16x8(sb + SM_WT + ti * 128 + (((q ^ ti) & 7) << 4), w0 + 8 * k);
       }
     }
     fence_proxy_async_smem();
     tc_fence_before();
-    named_sync(1, 128);
+    named_sync(1, PG_THREADS);
+    if (dmp) {
+      dump_wu(x.dbg, sm, x.tmem);
+      named_sync(1, PG_THREADS);
+    }
     if (p == 0) {
       mbar_arrive(&x.bars[B_PRO0 + b2]);
       tmark(x, c, 7);
     }
 #pragma unroll
-    for (int m = 0; m < 16; ++m) gv[m] = gn[m];
+    for (int m = 0; m < 8; ++m) gv[m] = gn[m];
     bv = bn;
   }
 }
 
+// Debug dumps from the scan group (TMEM / staging tile), chain 0.
+__device__ __noinline__ void dump_delta(float* dbg, uint32_t tmem) {
+  const int j = threadIdx.x;
+  const uint32_t tl = tmem + ((uint32_t)((j >> 5) * 32) << 16);
+  float d[32];
+  for (int half = 0; half < 2; ++half) {
+    tmem_ld32(tl + TM_DELTA + half * 32, d);
+    for (int i = 0; i < 32; ++i) dbg[DBG_DELTA + (half * 32 + i) * 128 + j] = d[i];
+  }
+}
+__device__ __noinline__ void dump_s(float* dbg, uint32_t tmem) {
+  const int j = threadIdx.x;
+  const uint32_t tl = tmem + ((uint32_t)((j >> 5) * 32) << 16);
+  float s[32];
+  for (int cb = 0; cb < 4; ++cb) {
+    tmem_ld32(tl + TM_S + cb * 32, s);
+    for (int i = 0; i < 32; ++i) dbg[DBG_S + (cb * 32 + i) * 128 + j] = s[i];
+  }
+}
+__device__ __noinline__ void dump_o(float* dbg, const uint8_t* sm) {
+  for (int e = threadIdx.x; e < 8192; e += 128) {
+    const int r = e >> 7, jj = e & 127;
+    const uint16_t u = *reinterpret_cast<const uint16_t*>(sm + SM_OST + (jj >> 6) * 8192 + sw128_off(r, jj & 63));
+    dbg[DBG_O + e] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(&u));
+  }
+}
+
 // ============================================================ scan group
-__device__ void scan_group(const Ctx& x, const void* tmq, const void* tmk, const void* tmv,
+__device__ void scan_group(const Ctx& x, const void* tmq, const void* tmk, const void* tmv, const void* tmo,
                            const float* __restrict__ init, __nv_bfloat16* __restrict__ out,
                            float* __restrict__ fin, int64_t sbase, bool inject_stuck, int (&issued)[2]) {
   const int j = threadIdx.x;  // 0..127: TMEM lane = value channel
@@ -621,6 +735,9 @@ __device__ void scan_group(const Ctx& x, const void* tmq, const void* tmk, const
   }
   tmem_wait_st();
 
+  // Output of chunk c: O^T (lane j) -> bf16 staging tile in the TMA box
+  // layout -> one TMA store per 64-channel half for a full chunk, or plain
+  // 16-byte stores of the valid rows for a sequence's last, partial chunk.
   auto store_out = [&](int c) {
     const int valid = chunk_valid(x, c);
     const int64_t tok0 = x.t0 + (int64_t)c * CH;
@@ -630,9 +747,28 @@ __device__ void scan_group(const Ctx& x, const void* tmq, const void* tmk, const
       tmem_ld32(tl + TM_O + (c & 1) * 64 + half * 32, o);
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
-        const int r = half * 32 + i;
-        if (r < valid) out[((tok0 + r) * H + x.h) * D + j] = __float2bfloat16_rn(o[i]);
-        if (x.dbg && c == 0) x.dbg[DBG_O + r * 128 + j] = o[i];
+        const __nv_bfloat16 hv = __float2bfloat16_rn(o[i]);
+        asm volatile("st.shared.b16 [%0], %1;" ::"r"(sb + SM_OST + (j >> 6) * 8192 + sw128_off(half * 32 + i, j & 63)),
+                     "h"(*reinterpret_cast<const uint16_t*>(&hv))
+                     : "memory");
+      }
+    }
+    fence_proxy_async_smem();
+    named_sync(2, 128);
+    if (x.dbg && c == 0) dump_o(x.dbg, sm);
+    if (valid == CH) {
+      if (j == 0) {
+        tma_store_3d(tmo, sm + SM_OST, 0, x.h, (int)tok0);
+        tma_store_3d(tmo, sm + SM_OST + 8192, 64, x.h, (int)tok0);
+        bulk_commit();
+      }
+    } else {
+      const int r = j >> 1, hf = j & 1;
+      if (r < valid) {
+        uint4* dst = reinterpret_cast<uint4*>(out + ((tok0 + r) * H + x.h) * D + hf * 64);
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          dst[q] = *reinterpret_cast<const uint4*>(sm + SM_OST + hf * 8192 + r * 128 + (((q ^ r) & 7) << 4));
       }
     }
   };
@@ -644,14 +780,14 @@ __device__ void scan_group(const Ctx& x, const void* tmq, const void* tmk, const
     const uint32_t stg = sb + b2 * STAGE_BYTES;
     const float* s_gc = reinterpret_cast<const float*>(sm + SM_MISC + MS_GC) + b2 * 128;
     if (j == 0) tmark(x, c, 8);
-    if (inject_stuck && c == 0 && !gwait(x, B_NEVER, 0, 99, 2)) {
+    if (inject_stuck && c == 0 && !gwait(x, B_NEVER, 0, 99, 2, 128)) {
       ok = false;
       break;
     }
     // ---- S pass: S^T (decayed to the chunk end when this chunk is "fast")
     // -> S'^T as fp16 pairs, the A operand of D1.
     if (c >= 1) {
-      if (!gwait(x, B_D2, d2_ph, 31, 2)) {
+      if (!gwait(x, B_D2, d2_ph, 31, 2, 128)) {
         ok = false;
         break;
       }
@@ -659,7 +795,7 @@ __device__ void scan_group(const Ctx& x, const void* tmq, const void* tmk, const
       tc_fence_after();
     }
     if (j == 0) tmark(x, c, 9);
-    if (!gwait(x, B_GC0 + b2, (c >> 1) & 1, 32, 2)) {
+    if (!gwait(x, B_GC0 + b2, (c >> 1) & 1, 32, 2, 128)) {
       ok = false;
       break;
     }
@@ -683,6 +819,7 @@ __device__ void scan_group(const Ctx& x, const void* tmq, const void* tmk, const
       tmem_st16(tl + TM_SB + cb * 16, pk);
     }
     if (!(mx <= F16_SAFE)) record_error(x.status, KDA_ERR_RANGE, 30);
+    if (j == 0) bulk_wait_read0();  // the staging tile is free again
     tmem_wait_st();
     tc_fence_before();
     if (!named_sync_and(2, 128, !*x.abort)) {
@@ -714,7 +851,7 @@ __device__ void scan_group(const Ctx& x, const void* tmq, const void* tmk, const
     }
     if (c >= 1) store_out(c - 1);
     if (j == 0) tmark(x, c, 12);
-    if (!gwait(x, B_D1, d1_ph, 34, 2)) {
+    if (!gwait(x, B_D1, d1_ph, 34, 2, 128)) {
       ok = false;
       break;
     }
@@ -751,13 +888,10 @@ __device__ void scan_group(const Ctx& x, const void* tmq, const void* tmk, const
           dm = fmaxf(dm, fmaxf(fabsf(d[2 * i]), fabsf(d[2 * i + 1])));
         }
         tmem_st16(tl + TM_DT + half * 16, pk);
-        if (x.dbg && c == 0) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) x.dbg[DBG_DELTA + (half * 32 + i) * 128 + j] = d[i];
-        }
       }
       if (!(dm <= F16_SAFE)) record_error(x.status, KDA_ERR_RANGE, 31);
     }
+    if (x.dbg && c == 0) dump_delta(x.dbg, x.tmem);
     tmem_wait_st();
     tc_fence_before();
     named_sync(2, 128);
@@ -785,21 +919,16 @@ __device__ void scan_group(const Ctx& x, const void* tmq, const void* tmk, const
     }
   }
   if (named_sync_and(2, 128, ok && !*x.abort) && x.nchunks > 0) {
-    if (gwait(x, B_D2, d2_ph, 35, 2)) {
+    if (gwait(x, B_D2, d2_ph, 35, 2, 128)) {
       tc_fence_after();
+      if (j == 0) bulk_wait_read0();
+      named_sync(2, 128);
       store_out(x.nchunks - 1);
     }
   }
+  if (j == 0) bulk_wait_all();  // every output store has completed
   if (named_sync_and(2, 128, !*x.abort)) {
-    if (x.dbg && x.nchunks > 0) {
-#pragma unroll
-      for (int cb = 0; cb < 4; ++cb) {
-        float s[32];
-        tmem_ld32(tl + TM_S + cb * 32, s);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) x.dbg[DBG_S + (cb * 32 + i) * 128 + j] = s[i];
-      }
-    }
+    if (x.dbg && x.nchunks > 0) dump_s(x.dbg, x.tmem);
     if (fin) {
 #pragma unroll
       for (int cb = 0; cb < 4; ++cb) {
@@ -814,7 +943,8 @@ __device__ void scan_group(const Ctx& x, const void* tmq, const void* tmk, const
 
 __global__ void __launch_bounds__(NTHR, 1)
     kda_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                      const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ g,
+                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                      const float* __restrict__ g,
                       const float* __restrict__ beta, const float* __restrict__ init,
                       __nv_bfloat16* __restrict__ out, float* __restrict__ fin, const int32_t* __restrict__ cu,
                       const int32_t* __restrict__ order, int64_t Tper, int H, DeviceStatus* status,
@@ -855,6 +985,7 @@ __global__ void __launch_bounds__(NTHR, 1)
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
+    prefetch_tmap(&tm_o);
   }
   if (warp == 0) {
     tmem_alloc(reinterpret_cast<uint32_t*>(sm + SM_MISC + MS_TMEM), TMEM_COLS);
@@ -870,7 +1001,7 @@ __global__ void __launch_bounds__(NTHR, 1)
   int cnt[2] = {0, 0};  // TMA stages issued (scan group) / consumed (prologue group)
   int* s_cnt = reinterpret_cast<int*>(sm + SM_MISC + MS_CNT);
   if (warp < 4) {
-    scan_group(x, &tm_q, &tm_k, &tm_v, init, out, fin, sbase, inject_stuck != 0, cnt);
+    scan_group(x, &tm_q, &tm_k, &tm_v, &tm_o, init, out, fin, sbase, inject_stuck != 0, cnt);
     if (tid == 0) { s_cnt[0] = cnt[0]; s_cnt[1] = cnt[1]; }
   } else {
     prologue_group(x, g, beta, cnt);
@@ -962,9 +1093,10 @@ cudaError_t launch_fwd_tc_impl(const FwdArgs& a, cudaStream_t s, uint64_t wait_n
   const int64_t Ttot = a.cu ? a.T : (int64_t)a.N * a.T;
   const unsigned blocks = (unsigned)((int64_t)a.N * a.H);
   if (blocks == 0) return cudaSuccess;
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mo;
   const int64_t Tmap = Ttot > 0 ? Ttot : 1;
-  if (!make_map(&mq, a.q, a.H, Tmap) || !make_map(&mk, a.k, a.H, Tmap) || !make_map(&mv, a.v, a.H, Tmap))
+  if (!make_map(&mq, a.q, a.H, Tmap) || !make_map(&mk, a.k, a.H, Tmap) || !make_map(&mv, a.v, a.H, Tmap) ||
+      !make_map(&mo, a.out, a.H, Tmap))
     return cudaErrorInvalidValue;
   const int32_t* order = nullptr;
   if (a.cu && order_ws && a.N > 1) {
@@ -974,7 +1106,7 @@ cudaError_t launch_fwd_tc_impl(const FwdArgs& a, cudaStream_t s, uint64_t wait_n
   cudaError_t e =
       cudaFuncSetAttribute(kda_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  kda_fwd_tc_kernel<<<blocks, NTHR, SMEM_BYTES, s>>>(mq, mk, mv, a.g, a.beta, a.init, (__nv_bfloat16*)a.out,
+  kda_fwd_tc_kernel<<<blocks, NTHR, SMEM_BYTES, s>>>(mq, mk, mv, mo, a.g, a.beta, a.init, (__nv_bfloat16*)a.out,
                                                      a.fin, a.cu, order, a.cu ? 0 : a.T, a.H, a.status,
                                                      (float*)a.dbg, wait_ns, inject_stuck);
   return cudaGetLastError();
