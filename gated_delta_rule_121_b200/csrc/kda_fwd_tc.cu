@@ -96,9 +96,9 @@ constexpr uint32_t TMEM_COLS = 512;
 
 // ---- debug dump (floats) for chain 0, chunk 0
 constexpr int DBG_P = 0, DBG_A = 4096, DBG_T = 8192, DBG_W = 12288, DBG_U = 20480, DBG_DELTA = 28672,
-              DBG_O = 36864, DBG_S = 45056, DBG_GC = 61440, DBG_TIME = 61568, DBG_FLOATS = 63616;
-// DBG_TIME: int64 [64 chunks][16 events] of SM clock cycles since block start
-// (events 0-7 prologue group, 8-15 scan group), chain 0 only.
+              DBG_O = 36864, DBG_S = 45056, DBG_GC = 61440, DBG_TIME = 61568, DBG_FLOATS = 65664;
+// DBG_TIME: int64 [64 chunks][32 events] of SM clock cycles since block start
+// (events 0-7 and 16-23 prologue group, 8-15 scan group), chain 0 only.
 constexpr int TIME_CHUNKS = 64;
 
 // ------------------------------------------------------------------ helpers
@@ -170,7 +170,7 @@ struct Ctx {
 
 // Phase timestamp (elected thread only) for the timing dump.
 __device__ __forceinline__ void tmark(const Ctx& x, int c, int ev) {
-  if (x.tdbg && c < TIME_CHUNKS) x.tdbg[c * 16 + ev] = clock64() - x.tstart;
+  if (x.tdbg && c < TIME_CHUNKS) x.tdbg[c * 32 + ev] = clock64() - x.tstart;
 }
 
 __device__ __forceinline__ bool cwait(const Ctx& x, int bar, uint32_t parity, int where) {
@@ -183,13 +183,27 @@ __device__ __forceinline__ bool cwait(const Ctx& x, int bar, uint32_t parity, in
 // Group-uniform bounded wait: every thread of named-barrier group `grp`
 // (nthr threads) polls, then the group agrees on the outcome, so no thread can
 // leave a loop while the others wait at a barrier or a .sync.aligned op.
+//
+// Only the group's first thread polls the mbarrier; the others block in the
+// hardware named barrier, so waiting warps take no issue slots or shared
+// memory bandwidth from the warps that are working.  The barrier (with the
+// tcgen05 / proxy fences the callers place after it) carries the observed
+// completion to the rest of the group.
 __device__ __forceinline__ bool gwait(const Ctx& x, int bar, uint32_t parity, int where, int grp, int nthr) {
-  bool ok = wait_bar(&x.bars[bar], parity, x.wait_ns, x.abort);
-  if (!ok) {
-    if (!*x.abort) record_error(x.status, KDA_ERR_TIMEOUT, where);
-    *x.abort = 1;
+  const bool elected = threadIdx.x == (grp == 2 ? 0u : 128u);
+  bool ok = true;
+  if (elected) {
+    ok = wait_bar(&x.bars[bar], parity, x.wait_ns, x.abort);
+    if (!ok) {
+      if (!*x.abort) record_error(x.status, KDA_ERR_TIMEOUT, where);
+      *x.abort = 1;
+    }
   }
-  return named_sync_and(grp, nthr, ok);
+  ok = named_sync_and(grp, nthr, ok);
+  // Each thread also observes the completed phase itself (an acquire that
+  // returns at once), so the data it guards is visible to every thread.
+  if (ok && !elected) mbar_try_wait(&x.bars[bar], parity);
+  return ok;
 }
 
 __device__ __forceinline__ int chunk_valid(const Ctx& x, int c) {
@@ -523,6 +537,7 @@ __device__ void prologue_group(const Ctx& x, const float* __restrict__ g, const 
         *reinterpret_cast<float4*>(sm + SM_DG + b * 4096 + b_off(rr, cb + i)) = make_float4(0.f, 0.f, 0.f, 0.f);
     }
     named_sync(1, PG_THREADS);
+    if (p == 0) tmark(x, c, 16);
     {  // Y_b = A'_b E_2b  (A'_b = A[32b+16 .. +16][32b .. +16]) -> X tile as [2][16][16]
       const int b = p >> 7, o = p & 127, r = o >> 3, c0 = 2 * (o & 7);
       float y0 = 0.f, y1 = 0.f;
@@ -541,6 +556,7 @@ __device__ void prologue_group(const Ctx& x, const float* __restrict__ g, const 
       *reinterpret_cast<float2*>(sm + SM_X + b * 1024 + r * 64 + c0 * 4) = make_float2(y0, y1);
     }
     named_sync(1, PG_THREADS);
+    if (p == 0) tmark(x, c, 17);
     {  // F_b = -E_2b+1 Y_b -> lower-left 16x16 block of D_b
       const int b = p >> 7, o = p & 127, r = o >> 3, c0 = 2 * (o & 7);
       float f0 = 0.f, f1 = 0.f;
@@ -559,6 +575,7 @@ __device__ void prologue_group(const Ctx& x, const float* __restrict__ g, const 
       *reinterpret_cast<float2*>(sm + SM_DG + b * 4096 + b_off(16 + r, c0)) = make_float2(f0, f1);
     }
     named_sync(1, PG_THREADS);
+    if (p == 0) tmark(x, c, 18);
     const int rr = p >> 3, c4 = 4 * (p & 7);  // 32x32 output row rr, columns c4 .. c4+3
     {  // X = A_10 D_0
       float4 o4 = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -575,6 +592,7 @@ __device__ void prologue_group(const Ctx& x, const float* __restrict__ g, const 
       *reinterpret_cast<float4*>(sm + SM_X + b_off(rr, c4)) = o4;
     }
     named_sync(1, PG_THREADS);
+    if (p == 0) tmark(x, c, 19);
     {  // T_10 = -D_1 X, then T' = T diag(beta) as fp16
       float4 o4 = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
@@ -950,7 +968,9 @@ __global__ void __launch_bounds__(NTHR, 1)
                       const int32_t* __restrict__ order, int64_t Tper, int H, DeviceStatus* status,
                       float* __restrict__ dbg, uint64_t wait_ns, int inject_stuck) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // Align to 1024 bytes by offsetting from the shared array itself, so the
+  // compiler keeps treating every access through `sm` as a shared-memory one.
+  uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   Ctx x;
   x.sm = sm;
   x.sb = smem_u32(sm);
