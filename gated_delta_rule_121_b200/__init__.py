@@ -7,6 +7,7 @@ loaded, every call raises.
 
 Functions mirror the C entry points:
   kda_fwd(q, k, v, log_alpha, beta, ...)        chunked prefill
+  kda_fwd_noalloc(...)                           the same, scratch in a fixed library array
   kda_decode_step(q, k, v, log_alpha, beta, state, ...)   in-place decode
   kda_fwd_workspace_size(...), kda_workspace_status(ws), kda_status_string(s)
 and ``kda_fwd_host`` runs kda_fwd on host (pinned) tensors, copying inputs in
@@ -59,6 +60,8 @@ def lib() -> ctypes.CDLL:
         L.kda_testing_debug_floats.restype = ctypes.c_int
         L.kda_testing_fwd_path.restype = ctypes.c_int
         L.kda_testing_fwd_path.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int]
+        L.kda_fwd_noalloc.restype = ctypes.c_int
+        L.kda_fwd_noalloc.argtypes = fwd_args[:-2]
         L.kda_decode_step.restype = ctypes.c_int
         L.kda_decode_step.argtypes = [_vp, _vp, _vp, _fp, _fp, _fp, _vp, ctypes.c_int, ctypes.c_int,
                                       ctypes.c_int, ctypes.c_int, _vp, ctypes.c_int]
@@ -148,6 +151,23 @@ def kda_fwd(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None, out=None
         code = lib().kda_testing_fwd(*args, _ptr(_debug), int(_wait_ns if _wait_ns is not None else 2_000_000_000),
                                      int(bool(_inject_stuck)))
     _check(code, "kda_fwd")
+    return out, final_state
+
+
+def kda_fwd_noalloc(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None, out=None, final_state=None,
+                    stream=None):
+    """kda_fwd without a caller workspace (see include/kda.h, kda_fwd_noalloc):
+    the library's fixed device array serves as scratch, nothing is allocated
+    by the library.  Returns ``(out, final_state)``."""
+    B, T, H, dk, dv, N = _shapes(q, v, cu_seqlens)
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    if final_state is None:
+        final_state = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
+    code = lib().kda_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(init_state),
+                                 _ptr(out), _ptr(final_state), N, T, H, dk, dv, _ptr(cu_seqlens),
+                                 _stream_ptr(stream), _DT[q.dtype])
+    _check(code, "kda_fwd_noalloc")
     return out, final_state
 
 

@@ -119,6 +119,36 @@ KDA_API kda_status_t kda_fwd(const void *q, const void *k, const void *v,
                      void *workspace, size_t workspace_bytes);
 
 /*
+ * kda_fwd for callers that cannot allocate device memory (for example a
+ * hosting runtime that owns all device memory, or a serving loop that must
+ * not call cudaMalloc/cudaFree because they can synchronize the device).
+ * The pages describe no such interface; it exists for callers of this
+ * library.
+ *
+ * Same arguments and results as kda_fwd, without the workspace: the call
+ * uses a fixed device array owned by the library (256 bytes plus 4 bytes per
+ * sequence, for at most KDA_NOALLOC_MAX_SEQUENCES sequences; every GPU that
+ * loads the library holds it until the process exits) and allocates nothing.
+ *   - B (the number of sequences) above KDA_NOALLOC_MAX_SEQUENCES returns
+ *     KDA_ERR_WORKSPACE before any device work.
+ *   - The first call on each device looks up the array's device address
+ *     (with that device current); make that first call before any stream
+ *     capture.
+ *   - Every call on a device shares the one array.  Calls that may overlap on
+ *     the GPU (different streams, or other host threads) race on it; issue
+ *     them in order on one stream.
+ *   - The device status word lives in that array, so device-side errors
+ *     (KDA_ERR_TIMEOUT, KDA_ERR_RANGE) of this entry point cannot be read
+ *     back; use kda_fwd with a workspace when they must be checked.
+ */
+#define KDA_NOALLOC_MAX_SEQUENCES 8192
+KDA_API kda_status_t kda_fwd_noalloc(const void *q, const void *k, const void *v,
+                                     const float *log_alpha, const float *beta,
+                                     const float *init_state, void *out, float *final_state,
+                                     int B, int64_t T, int H, int dk, int dv,
+                                     const int32_t *cu_seqlens, void *stream, kda_dtype_t dt);
+
+/*
  * One decode step: one new token per sequence, state updated in place (the
  * digest's serving section, "speculative decoding and KDA state rewind":
  * the recurrent state is updated in place at every decode step).
