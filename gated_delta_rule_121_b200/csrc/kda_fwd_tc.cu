@@ -65,7 +65,8 @@ constexpr uint32_t SM_WT = SM_P + 16384;     // W'^T fp16 [c][r]             16 
 constexpr uint32_t SM_A = SM_WT + 16384;     // A fp32 [64][64] -> T' fp16   16 KB
 constexpr uint32_t SM_DG = SM_A + 16384;     // D_0, D_1 fp32 [32][32]        8 KB
 constexpr uint32_t SM_X = SM_DG + 8192;      // X fp32 [32][32] (Y before)    4 KB
-constexpr uint32_t SM_OST = SM_X + 4096;     // O staging bf16 [64][128]     16 KB
+constexpr uint32_t SM_T10 = SM_X + 4096;     // T_10 fp32 [32][32]            4 KB
+constexpr uint32_t SM_OST = SM_T10 + 4096 + 4096;  // O staging bf16 [64][128] 16 KB (1024-aligned)
 constexpr uint32_t SM_MISC = SM_OST + 16384;
 constexpr uint32_t MISC_BYTES = 10240;
 constexpr uint32_t SMEM_BYTES = SM_MISC + MISC_BYTES + 1024;
@@ -102,30 +103,29 @@ constexpr int DBG_P = 0, DBG_A = 4096, DBG_T = 8192, DBG_W = 12288, DBG_U = 2048
 constexpr int TIME_CHUNKS = 64;
 
 // ------------------------------------------------------------------ helpers
-__device__ __forceinline__ void st_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
-               : "memory");
-}
-__device__ __forceinline__ void st_v2(uint32_t addr, uint32_t a, uint32_t b) {
-  asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(addr), "r"(a), "r"(b) : "memory");
-}
-__device__ __forceinline__ float4 ld_bf16x4(uint32_t addr) {
-  uint32_t a, b;
-  asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(a), "=r"(b) : "r"(addr));
-  const float2 x = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&a));
-  const float2 y = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&b));
+// Shared-memory accesses are plain C++ through pointers derived from the
+// shared array (so they compile to shared loads/stores and the compiler may
+// schedule them freely between barriers).
+__device__ __forceinline__ float4 ld_bf16x4(const uint8_t* p) {
+  const uint2 u = *reinterpret_cast<const uint2*>(p);
+  const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+  const float2 y = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
   return make_float4(x.x, x.y, y.x, y.y);
 }
-__device__ __forceinline__ float ld_bf16(uint32_t addr) {
-  uint16_t u;
-  asm volatile("ld.shared.b16 %0, [%1];" : "=h"(u) : "r"(addr));
-  return __bfloat162float(*reinterpret_cast<__nv_bfloat16*>(&u));
+__device__ __forceinline__ float4 bf16x4_to_f32(uint2 u) {
+  const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+  const float2 y = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+  return make_float4(x.x, x.y, y.x, y.y);
 }
-__device__ __forceinline__ void st_f16x4(uint32_t addr, float4 v) {
-  st_v2(addr, pack_f16x2(v.x, v.y), pack_f16x2(v.z, v.w));
+__device__ __forceinline__ float ld_bf16(const uint8_t* p) {
+  return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(p));
 }
-__device__ __forceinline__ void st_f16x8(uint32_t addr, const float* v) {
-  st_v4(addr, pack_f16x2(v[0], v[1]), pack_f16x2(v[2], v[3]), pack_f16x2(v[4], v[5]), pack_f16x2(v[6], v[7]));
+__device__ __forceinline__ void st_f16x4(uint8_t* p, float4 v) {
+  *reinterpret_cast<uint2*>(p) = make_uint2(pack_f16x2(v.x, v.y), pack_f16x2(v.z, v.w));
+}
+__device__ __forceinline__ void st_f16x8(uint8_t* p, const float* v) {
+  *reinterpret_cast<uint4*>(p) = make_uint4(pack_f16x2(v[0], v[1]), pack_f16x2(v[2], v[3]), pack_f16x2(v[4], v[5]),
+                                            pack_f16x2(v[6], v[7]));
 }
 __device__ __forceinline__ float4 mul4(float4 a, float4 b) {
   return make_float4(a.x * b.x, a.y * b.y, a.z * b.z, a.w * b.w);
@@ -142,6 +142,44 @@ __device__ __forceinline__ uint32_t a_off(uint32_t r, uint32_t s) {
 __device__ __forceinline__ uint32_t b_off(uint32_t r, uint32_t s) {
   return r * 128u + ((s >> 2) ^ (r & 7u)) * 16u + (s & 3u) * 4u;
 }
+// One 16x8 tile of D = sign * A B with fp32 operands held in shared memory,
+// K = 8 * KSTEPS, computed on the warp-level tensor path as three tf32
+// products (hi*hi + hi*lo + lo*hi), which keeps close to fp32 accuracy.
+// fa(r, k) / fb(k, n) return the operand element addresses.
+template <int KSTEPS, typename FA, typename FB>
+__device__ __forceinline__ void warp_gemm_tf32x3(float (&d)[4], FA fa, FB fb) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  d[0] = d[1] = d[2] = d[3] = 0.f;
+  float av[KSTEPS][4], bv[KSTEPS][2];
+#pragma unroll
+  for (int ks = 0; ks < KSTEPS; ++ks) {  // every fragment load first: one shared-memory latency
+    const int k0 = 8 * ks;
+    av[ks][0] = *fa(g, k0 + t);
+    av[ks][1] = *fa(g + 8, k0 + t);
+    av[ks][2] = *fa(g, k0 + t + 4);
+    av[ks][3] = *fa(g + 8, k0 + t + 4);
+    bv[ks][0] = *fb(k0 + t, g);
+    bv[ks][1] = *fb(k0 + t + 4, g);
+  }
+#pragma unroll
+  for (int ks = 0; ks < KSTEPS; ++ks) {
+    uint32_t ah[4], al[4], bh[2], bl[2];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      ah[i] = to_tf32(av[ks][i]);
+      al[i] = to_tf32(av[ks][i] - __uint_as_float(ah[i]));
+    }
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      bh[i] = to_tf32(bv[ks][i]);
+      bl[i] = to_tf32(bv[ks][i] - __uint_as_float(bh[i]));
+    }
+    mma_tf32_16x8x8(d, al, bh);
+    mma_tf32_16x8x8(d, ah, bl);
+    mma_tf32_16x8x8(d, ah, bh);
+  }
+}
+
 // Bounded wait that also gives up when the other group has aborted.
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, uint64_t ns, volatile int* abort) {
   if (mbar_try_wait(bar, parity)) return true;
@@ -226,6 +264,8 @@ __device__ __forceinline__ void general_gram(const Ctx& x, uint32_t stg, int b2,
   uint8_t* sm = x.sm;
   const float* s_beta = reinterpret_cast<const float*>(sm + SM_MISC + MS_BETA) + b2 * 64;
   const int r = p & 63, s0 = (p >> 6) * 16;
+  const uint8_t* stp = sm + b2 * STAGE_BYTES;
+  (void)stg;
   float pa[16], aa[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) pa[i] = aa[i] = 0.f;
@@ -241,13 +281,13 @@ __device__ __forceinline__ void general_gram(const Ctx& x, uint32_t stg, int b2,
       for (int ch = 0; ch < 64; ++ch) {
         const uint32_t off_r = half * 16384 + sw128_off(r, ch);
         const float gr = *reinterpret_cast<const float*>(sm + SM_WT + r * 256 + ch * 4);
-        const float qr = ld_bf16(stg + OFF_QK + off_r), kr = ld_bf16(stg + OFF_QK + 8192 + off_r);
+        const float qr = ld_bf16(stp + OFF_QK + off_r), kr = ld_bf16(stp + OFF_QK + 8192 + off_r);
 #pragma unroll 4
         for (int i = 0; i < 16; ++i) {
           const int s = s0 + i;
           if (s <= r) {
             const float gs = *reinterpret_cast<const float*>(sm + SM_WT + s * 256 + ch * 4);
-            const float ks = ld_bf16(stg + OFF_QK + 8192 + half * 16384 + sw128_off(s, ch));
+            const float ks = ld_bf16(stp + OFF_QK + 8192 + half * 16384 + sw128_off(s, ch));
             const float e = ex2(gr - gs) * ks;
             pa[i] += qr * e;
             aa[i] += kr * e;
@@ -266,7 +306,7 @@ __device__ __forceinline__ void general_gram(const Ctx& x, uint32_t stg, int b2,
 #pragma unroll
   for (int q8 = 0; q8 < 2; ++q8) {
     const int s = s0 + 8 * q8;
-    st_f16x8(x.sb + SM_P + b2 * 8192 + r * 128 + ((((s >> 3) ^ r) & 7) << 4), pa + 8 * q8);
+    st_f16x8(sm + SM_P + b2 * 8192 + r * 128 + ((((s >> 3) ^ r) & 7) << 4), pa + 8 * q8);
   }
 #pragma unroll
   for (int u = 0; u < 4; ++u)
@@ -437,15 +477,24 @@ __device__ void prologue_group(const Ctx& x, const float* __restrict__ g, const 
 
     // ---- (a2) operand scaling: QE, KE in place, KH into KX[b2], V -> fp16.
     {
-      const uint32_t qb = stg + OFF_QK + hh * 16384, kb = qb + 8192;
-      const uint32_t vb = stg + OFF_V + hh * 8192;
-      const uint32_t khb = sb + SM_KX + b2 * 16384 + hh * 8192;
+      uint8_t* qb = sm + b2 * STAGE_BYTES + OFF_QK + hh * 16384;
+      uint8_t* kb = qb + 8192;
+      uint8_t* vb = sm + b2 * STAGE_BYTES + OFF_V + hh * 8192;
+      uint8_t* khb = sm + SM_KX + b2 * 16384 + hh * 8192;
+      uint2 qr[8], kr[8], vr[8];
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {  // all loads first, then the in-place stores
+        const uint32_t o = sw128_off(8 * rg + m, cc);
+        qr[m] = *reinterpret_cast<const uint2*>(qb + o);
+        kr[m] = *reinterpret_cast<const uint2*>(kb + o);
+        vr[m] = *reinterpret_cast<const uint2*>(vb + o);
+      }
       bool bad = false;
 #pragma unroll
       for (int m = 0; m < 8; ++m) {
         const int r = 8 * rg + m;
         const uint32_t o = sw128_off(r, cc);
-        float4 q4 = ld_bf16x4(qb + o), k4 = ld_bf16x4(kb + o), v4 = ld_bf16x4(vb + o);
+        float4 q4 = bf16x4_to_f32(qr[m]), k4 = bf16x4_to_f32(kr[m]), v4 = bf16x4_to_f32(vr[m]);
         if (r >= valid) q4 = k4 = v4 = make_float4(0.f, 0.f, 0.f, 0.f);
         bad |= amax4(v4) > F16_SAFE;
         st_f16x4(qb + o, mul4(q4, fw[m]));
@@ -471,9 +520,11 @@ __device__ void prologue_group(const Ctx& x, const float* __restrict__ g, const 
           umma_ss(x.tmem + TM_GW, da, db, id, i > 0);
         }
         umma_commit(&x.bars[B_G1]);
+        tmark(x, c, 20);
       }
       if (!gwait(x, B_G1, g1_ph, 14, 1, PG_THREADS)) break;
       g1_ph ^= 1;
+      if (p == 0) tmark(x, c, 21);
       tc_fence_after();
       float r0[32];
       tmem_ld32(tl + TM_GW + chalf * 32, r0);  // row ti, columns 32 chalf .. +31
@@ -484,7 +535,7 @@ __device__ void prologue_group(const Ctx& x, const float* __restrict__ g, const 
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           const int q8 = chalf * 4 + k;
-          st_f16x8(sb + SM_P + b2 * 8192 + ti * 128 + (((q8 ^ ti) & 7) << 4), r0 + 8 * k);
+          st_f16x8(sm + SM_P + b2 * 8192 + ti * 128 + (((q8 ^ ti) & 7) << 4), r0 + 8 * k);
         }
       } else {  // A row r = beta_r (KE KH^T)_rs, strictly lower
         const int r = ti - CH;
@@ -510,20 +561,27 @@ __device__ void prologue_group(const Ctx& x, const float* __restrict__ g, const 
     // the 32x32 diagonal inverses; T_10 = -D_1 (A_10 D_0).
     // T' = T diag(beta) as fp16 [r][s] over the A tile.
     if (p < 64) {
+      // Column sweep: once x[s] is final it updates every later row.  The
+      // loads do not depend on x, so the dependency chain is one FMA per
+      // column; column s+1 is fetched while column s is applied.
       const int a = p >> 4, jj = p & 15;
-      float xs[16];
-#pragma unroll
-      for (int r = 0; r < 16; ++r) xs[r] = 0.f;
+      auto ael = [&](int r, int c) { return *reinterpret_cast<const float*>(sm + SM_A + a_off(16 * a + r, 16 * a + c)); };
+      float xs[16], col[16], nxt[16];
 #pragma unroll
       for (int r = 0; r < 16; ++r) {
-        float a0 = (r == jj) ? 1.f : 0.f, a1 = 0.f;
+        xs[r] = (r == jj) ? 1.f : 0.f;
+        col[r] = r >= 1 ? ael(r, 0) : 0.f;
+      }
 #pragma unroll
-        for (int u = 0; u < (r + 3) / 4; ++u) {
-          const float4 a4 = *reinterpret_cast<const float4*>(sm + SM_A + a_off(16 * a + r, 16 * a + 4 * u));
-          a0 -= a4.x * xs[4 * u] + a4.z * xs[4 * u + 2];
-          a1 -= a4.y * xs[4 * u + 1] + a4.w * xs[4 * u + 3];
-        }
-        xs[r] = a0 + a1;
+      for (int sc = 0; sc < 15; ++sc) {
+#pragma unroll
+        for (int r = 0; r < 16; ++r) nxt[r] = (sc + 1 < 15 && r >= sc + 2) ? ael(r, sc + 1) : 0.f;
+        const float xsc = xs[sc];
+#pragma unroll
+        for (int r = 0; r < 16; ++r)
+          if (r > sc) xs[r] -= col[r] * xsc;
+#pragma unroll
+        for (int r = 0; r < 16; ++r) col[r] = nxt[r];
       }
       // E_a -> diagonal 16x16 block of D_{a/2}
       const uint32_t db = SM_DG + (a >> 1) * 4096;
@@ -538,81 +596,63 @@ __device__ void prologue_group(const Ctx& x, const float* __restrict__ g, const 
     }
     named_sync(1, PG_THREADS);
     if (p == 0) tmark(x, c, 16);
-    {  // Y_b = A'_b E_2b  (A'_b = A[32b+16 .. +16][32b .. +16]) -> X tile as [2][16][16]
-      const int b = p >> 7, o = p & 127, r = o >> 3, c0 = 2 * (o & 7);
-      float y0 = 0.f, y1 = 0.f;
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const float4 a4 = *reinterpret_cast<const float4*>(sm + SM_A + a_off(32 * b + 16 + r, 32 * b + 4 * u));
-        const float av[4] = {a4.x, a4.y, a4.z, a4.w};
-#pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          const int s = 4 * u + t;
-          const float2 e = *reinterpret_cast<const float2*>(sm + SM_DG + b * 4096 + b_off(s, c0));
-          y0 += av[t] * e.x;
-          y1 += av[t] * e.y;
-        }
-      }
-      *reinterpret_cast<float2*>(sm + SM_X + b * 1024 + r * 64 + c0 * 4) = make_float2(y0, y1);
+    const int pw = p >> 5, lg = lane >> 2, lt = lane & 3;  // warp in group; mma fragment coordinates
+    if (pw < 4) {  // Y_b = A'_b E_2b  (A'_b = A[32b+16 .. +16][32b .. +16]) -> X tile as [2][16][16]
+      const int b = pw >> 1, nt = pw & 1;
+      float d[4];
+      warp_gemm_tf32x3<2>(
+          d, [&](int r, int k) { return reinterpret_cast<const float*>(sm + SM_A + a_off(32 * b + 16 + r, 32 * b + k)); },
+          [&](int k, int n) { return reinterpret_cast<const float*>(sm + SM_DG + b * 4096 + b_off(k, 8 * nt + n)); });
+      float* y = reinterpret_cast<float*>(sm + SM_X + b * 1024);
+      *reinterpret_cast<float2*>(y + lg * 16 + 8 * nt + 2 * lt) = make_float2(d[0], d[1]);
+      *reinterpret_cast<float2*>(y + (lg + 8) * 16 + 8 * nt + 2 * lt) = make_float2(d[2], d[3]);
     }
     named_sync(1, PG_THREADS);
     if (p == 0) tmark(x, c, 17);
-    {  // F_b = -E_2b+1 Y_b -> lower-left 16x16 block of D_b
-      const int b = p >> 7, o = p & 127, r = o >> 3, c0 = 2 * (o & 7);
-      float f0 = 0.f, f1 = 0.f;
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const float4 e4 = *reinterpret_cast<const float4*>(sm + SM_DG + b * 4096 + b_off(16 + r, 16 + 4 * u));
-        const float ev[4] = {e4.x, e4.y, e4.z, e4.w};
-#pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          const int s = 4 * u + t;
-          const float2 y = *reinterpret_cast<const float2*>(sm + SM_X + b * 1024 + s * 64 + c0 * 4);
-          f0 -= ev[t] * y.x;
-          f1 -= ev[t] * y.y;
-        }
-      }
-      *reinterpret_cast<float2*>(sm + SM_DG + b * 4096 + b_off(16 + r, c0)) = make_float2(f0, f1);
+    if (pw < 4) {  // F_b = -E_2b+1 Y_b -> lower-left 16x16 block of D_b
+      const int b = pw >> 1, nt = pw & 1;
+      float d[4];
+      warp_gemm_tf32x3<2>(
+          d, [&](int r, int k) { return reinterpret_cast<const float*>(sm + SM_DG + b * 4096 + b_off(16 + r, 16 + k)); },
+          [&](int k, int n) { return reinterpret_cast<const float*>(sm + SM_X + b * 1024 + (k * 16 + 8 * nt + n) * 4); });
+      uint8_t* db = sm + SM_DG + b * 4096;
+      *reinterpret_cast<float2*>(db + b_off(16 + lg, 8 * nt + 2 * lt)) = make_float2(-d[0], -d[1]);
+      *reinterpret_cast<float2*>(db + b_off(24 + lg, 8 * nt + 2 * lt)) = make_float2(-d[2], -d[3]);
     }
     named_sync(1, PG_THREADS);
     if (p == 0) tmark(x, c, 18);
-    const int rr = p >> 3, c4 = 4 * (p & 7);  // 32x32 output row rr, columns c4 .. c4+3
-    {  // X = A_10 D_0
-      float4 o4 = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const float4 a4 = *reinterpret_cast<const float4*>(sm + SM_A + a_off(32 + rr, 4 * u));
-        const float av[4] = {a4.x, a4.y, a4.z, a4.w};
-#pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          const float4 d = *reinterpret_cast<const float4*>(sm + SM_DG + b_off(4 * u + t, c4));
-          o4.x += av[t] * d.x; o4.y += av[t] * d.y; o4.z += av[t] * d.z; o4.w += av[t] * d.w;
-        }
-      }
-      *reinterpret_cast<float4*>(sm + SM_X + b_off(rr, c4)) = o4;
+    {  // X = A_10 D_0  (32x32x32, one 16x8 tile per warp)
+      const int mt = pw >> 2, nt = pw & 3;
+      float d[4];
+      warp_gemm_tf32x3<4>(
+          d, [&](int r, int k) { return reinterpret_cast<const float*>(sm + SM_A + a_off(32 + 16 * mt + r, k)); },
+          [&](int k, int n) { return reinterpret_cast<const float*>(sm + SM_DG + b_off(k, 8 * nt + n)); });
+      *reinterpret_cast<float2*>(sm + SM_X + b_off(16 * mt + lg, 8 * nt + 2 * lt)) = make_float2(d[0], d[1]);
+      *reinterpret_cast<float2*>(sm + SM_X + b_off(16 * mt + lg + 8, 8 * nt + 2 * lt)) = make_float2(d[2], d[3]);
     }
     named_sync(1, PG_THREADS);
     if (p == 0) tmark(x, c, 19);
-    {  // T_10 = -D_1 X, then T' = T diag(beta) as fp16
-      float4 o4 = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const float4 a4 = *reinterpret_cast<const float4*>(sm + SM_DG + 4096 + b_off(rr, 4 * u));
-        const float av[4] = {a4.x, a4.y, a4.z, a4.w};
-#pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          const float4 d = *reinterpret_cast<const float4*>(sm + SM_X + b_off(4 * u + t, c4));
-          o4.x -= av[t] * d.x; o4.y -= av[t] * d.y; o4.z -= av[t] * d.z; o4.w -= av[t] * d.w;
-        }
-      }
+    {  // T_10 = -D_1 X
+      const int mt = pw >> 2, nt = pw & 3;
+      float d[4];
+      warp_gemm_tf32x3<4>(
+          d, [&](int r, int k) { return reinterpret_cast<const float*>(sm + SM_DG + 4096 + b_off(16 * mt + r, k)); },
+          [&](int k, int n) { return reinterpret_cast<const float*>(sm + SM_X + b_off(k, 8 * nt + n)); });
+      *reinterpret_cast<float2*>(sm + SM_T10 + b_off(16 * mt + lg, 8 * nt + 2 * lt)) = make_float2(-d[0], -d[1]);
+      *reinterpret_cast<float2*>(sm + SM_T10 + b_off(16 * mt + lg + 8, 8 * nt + 2 * lt)) = make_float2(-d[2], -d[3]);
+    }
+    named_sync(1, PG_THREADS);
+    {  // T' = T diag(beta) as fp16 [r][s]: rows rr and 32 + rr, columns c4 .. c4+3 and 32 + c4 ..
+      const int rr = p >> 3, c4 = 4 * (p & 7);
       const float4 bl = *reinterpret_cast<const float4*>(s_beta + c4);
       const float4 bh = *reinterpret_cast<const float4*>(s_beta + 32 + c4);
       const float4 d0 = *reinterpret_cast<const float4*>(sm + SM_DG + b_off(rr, c4));
       const float4 d1 = *reinterpret_cast<const float4*>(sm + SM_DG + 4096 + b_off(rr, c4));
-      st_f16x4(sb + SM_A + sw128_off(rr, c4), mul4(d0, bl));
-      st_f16x4(sb + SM_A + sw128_off(rr, 32 + c4), make_float4(0.f, 0.f, 0.f, 0.f));
-      st_f16x4(sb + SM_A + sw128_off(32 + rr, c4), mul4(o4, bl));
-      st_f16x4(sb + SM_A + sw128_off(32 + rr, 32 + c4), mul4(d1, bh));
+      const float4 t10 = *reinterpret_cast<const float4*>(sm + SM_T10 + b_off(rr, c4));
+      st_f16x4(sm + SM_A + sw128_off(rr, c4), mul4(d0, bl));
+      st_f16x4(sm + SM_A + sw128_off(rr, 32 + c4), make_float4(0.f, 0.f, 0.f, 0.f));
+      st_f16x4(sm + SM_A + sw128_off(32 + rr, c4), mul4(t10, bl));
+      st_f16x4(sm + SM_A + sw128_off(32 + rr, 32 + c4), mul4(d1, bh));
     }
     fence_proxy_async_smem();
     named_sync(1, PG_THREADS);
@@ -642,6 +682,7 @@ __device__ void prologue_group(const Ctx& x, const float* __restrict__ g, const 
           umma_ss(x.tmem + TM_DELTA, da, db, id, i > 0);
         }
         umma_commit(&x.bars[B_G23]);
+        tmark(x, c, 22);
       }
     }
     // Prefetch next chunk's decay and beta while the UMMAs run.
@@ -663,7 +704,7 @@ __device__ void prologue_group(const Ctx& x, const float* __restrict__ g, const 
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         const int q = chalf * 4 + k;
-        st_f16x8(sb + SM_WT + ti * 128 + (((q ^ ti) & 7) << 4), w0 + 8 * k);
+        st_f16x8(sm + SM_WT + ti * 128 + (((q ^ ti) & 7) << 4), w0 + 8 * k);
       }
     }
     fence_proxy_async_smem();
@@ -759,17 +800,14 @@ __device__ void scan_group(const Ctx& x, const void* tmq, const void* tmk, const
   auto store_out = [&](int c) {
     const int valid = chunk_valid(x, c);
     const int64_t tok0 = x.t0 + (int64_t)c * CH;
-    float o[32];
+    float o0[32], o1[32];
+    tmem_ld32x2(tl + TM_O + (c & 1) * 64, tl + TM_O + (c & 1) * 64 + 32, o0, o1);
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      tmem_ld32(tl + TM_O + (c & 1) * 64 + half * 32, o);
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const __nv_bfloat16 hv = __float2bfloat16_rn(o[i]);
-        asm volatile("st.shared.b16 [%0], %1;" ::"r"(sb + SM_OST + (j >> 6) * 8192 + sw128_off(half * 32 + i, j & 63)),
-                     "h"(*reinterpret_cast<const uint16_t*>(&hv))
-                     : "memory");
-      }
+    for (int i = 0; i < 32; ++i) {
+      *reinterpret_cast<__nv_bfloat16*>(sm + SM_OST + (j >> 6) * 8192 + sw128_off(i, j & 63)) =
+          __float2bfloat16_rn(o0[i]);
+      *reinterpret_cast<__nv_bfloat16*>(sm + SM_OST + (j >> 6) * 8192 + sw128_off(32 + i, j & 63)) =
+          __float2bfloat16_rn(o1[i]);
     }
     fence_proxy_async_smem();
     named_sync(2, 128);
@@ -820,21 +858,31 @@ __device__ void scan_group(const Ctx& x, const void* tmq, const void* tmk, const
     const bool fast = *reinterpret_cast<volatile int*>(sm + SM_MISC + MS_FAST + 4 * b2) != 0;
     float mx = 0.f;
 #pragma unroll
-    for (int cb = 0; cb < 4; ++cb) {
-      float s[32];
+    for (int cp = 0; cp < 2; ++cp) {
+      float s0[32], s1[32];
       uint32_t pk[16];
-      tmem_ld32(tl + TM_S + cb * 32, s);
+      tmem_ld32x2(tl + TM_S + cp * 64, tl + TM_S + cp * 64 + 32, s0, s1);
       if (fast) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) s[i] *= s_gc[cb * 32 + i];
-        tmem_st32(tl + TM_S + cb * 32, s);
+        for (int i = 0; i < 32; ++i) {
+          s0[i] *= s_gc[cp * 64 + i];
+          s1[i] *= s_gc[cp * 64 + 32 + i];
+        }
+        tmem_st32(tl + TM_S + cp * 64, s0);
+        tmem_st32(tl + TM_S + cp * 64 + 32, s1);
       }
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        pk[i] = pack_f16x2(s[2 * i], s[2 * i + 1]);
-        mx = fmaxf(mx, fmaxf(fabsf(s[2 * i]), fabsf(s[2 * i + 1])));
+        pk[i] = pack_f16x2(s0[2 * i], s0[2 * i + 1]);
+        mx = fmaxf(mx, fmaxf(fabsf(s0[2 * i]), fabsf(s0[2 * i + 1])));
       }
-      tmem_st16(tl + TM_SB + cb * 16, pk);
+      tmem_st16(tl + TM_SB + cp * 32, pk);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        pk[i] = pack_f16x2(s1[2 * i], s1[2 * i + 1]);
+        mx = fmaxf(mx, fmaxf(fabsf(s1[2 * i]), fabsf(s1[2 * i + 1])));
+      }
+      tmem_st16(tl + TM_SB + cp * 32 + 16, pk);
     }
     if (!(mx <= F16_SAFE)) record_error(x.status, KDA_ERR_RANGE, 30);
     if (j == 0) bulk_wait_read0();  // the staging tile is free again
@@ -849,6 +897,7 @@ __device__ void scan_group(const Ctx& x, const void* tmq, const void* tmk, const
     // ---- D1: O^T = S'^T QE^T ;  Δ^T = U^T - S'^T W'^T    (A = S'^T from TMEM)
     if (j == 0) {
       if (cwait(x, B_PRO0 + b2, (c >> 1) & 1, 33)) {
+        tmark(x, c, 24);
         tc_fence_after();
         const uint32_t idq = idesc_f16_f32(128, 64, 0, 0);
         const uint32_t idw = idesc_f16_f32(128, 64, 0, 1, 1);
@@ -894,19 +943,22 @@ __device__ void scan_group(const Ctx& x, const void* tmq, const void* tmk, const
       }
     }
     {
-      float d[32];
+      float d0[32], d1[32];
       uint32_t pk[16];
       float dm = 0.f;
+      tmem_ld32x2(tl + TM_DELTA, tl + TM_DELTA + 32, d0, d1);
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        tmem_ld32(tl + TM_DELTA + half * 32, d);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          pk[i] = pack_f16x2(d[2 * i], d[2 * i + 1]);
-          dm = fmaxf(dm, fmaxf(fabsf(d[2 * i]), fabsf(d[2 * i + 1])));
-        }
-        tmem_st16(tl + TM_DT + half * 16, pk);
+      for (int i = 0; i < 16; ++i) {
+        pk[i] = pack_f16x2(d0[2 * i], d0[2 * i + 1]);
+        dm = fmaxf(dm, fmaxf(fabsf(d0[2 * i]), fabsf(d0[2 * i + 1])));
       }
+      tmem_st16(tl + TM_DT, pk);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        pk[i] = pack_f16x2(d1[2 * i], d1[2 * i + 1]);
+        dm = fmaxf(dm, fmaxf(fabsf(d1[2 * i]), fabsf(d1[2 * i + 1])));
+      }
+      tmem_st16(tl + TM_DT + 16, pk);
       if (!(dm <= F16_SAFE)) record_error(x.status, KDA_ERR_RANGE, 31);
     }
     if (x.dbg && c == 0) dump_delta(x.dbg, x.tmem);
