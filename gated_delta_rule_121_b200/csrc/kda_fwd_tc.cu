@@ -27,10 +27,12 @@
 // state and every product stay accurate to well inside the bf16 output's own
 // rounding.  Values that would not fit fp16 set KDA_ERR_RANGE.
 //
-// Work split (one CTA per (sequence, head) chain, chunks in order):
-//   warps 4-7, "prologue" group (PG): for chunk c+1 — cumulative decay,
-//     operand scaling, G1 Gram UMMA, the triangular solve on CUDA cores,
-//     G2/G3 UMMAs for W'^T and U^T, and the W'^T store;
+// Work split (one CTA per (sequence, head) chain, chunks in order), three
+// groups of four warps:
+//   warps 4-7, "front" group: for chunk c+2 — cumulative decay fused with
+//     the operand scaling, the G1 Gram UMMA, and the P / A tiles;
+//   warps 8-11, "back" group: for chunk c+1 — the triangular solve on CUDA
+//     cores, G2/G3 UMMAs for W'^T and U^T, and the W'^T store;
 //   warps 0-3, "scan" group (SG): for chunk c — the state recurrence:
 //     decay S^T, D1 = { O^T = S'^T QE^T ;  Δ^T = U^T - S'^T W'^T }, Δ^T to
 //     fp16, D2 = { S^T += Δ^T KH ;  O^T += Δ^T P^T }, output store.
@@ -50,7 +52,7 @@ namespace {
 
 constexpr int CH = 64;  // chunk length
 constexpr int D = 128;  // dk = dv
-constexpr int NTHR = 384;  // 4 scan warps + 8 prologue warps
+constexpr int NTHR = 384;  // scan, front and back groups of 4 warps
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float FAST_MIN_LOG2 = -10.0f;  // chunk-total decay floor (log2) for the tensor-core Gram
 constexpr float F16_SAFE = 60000.0f;     // |x| above this would overflow fp16 operands
@@ -62,44 +64,50 @@ constexpr uint32_t OFF_QK = 0, OFF_V = 32768;
 constexpr uint32_t SM_KX = 2 * STAGE_BYTES;  // KH fp16 [s][c], x2          32 KB
 constexpr uint32_t SM_P = SM_KX + 32768;     // P fp16 [r][s], x2            16 KB
 constexpr uint32_t SM_WT = SM_P + 16384;     // W'^T fp16 [c][r]             16 KB
-constexpr uint32_t SM_A = SM_WT + 16384;     // A fp32 [64][64] -> T' fp16   16 KB
+constexpr uint32_t SM_A = SM_WT + 16384;     // A fp32 [64][64]              16 KB
 constexpr uint32_t SM_DG = SM_A + 16384;     // D_0, D_1 fp32 [32][32]        8 KB
 constexpr uint32_t SM_X = SM_DG + 8192;      // X fp32 [32][32] (Y before)    4 KB
 constexpr uint32_t SM_T10 = SM_X + 4096;     // T_10 fp32 [32][32]            4 KB
+constexpr uint32_t SM_TP = SM_X;             // T' fp16 [64][64] over X, T_10  8 KB
 constexpr uint32_t SM_OST = SM_T10 + 4096 + 4096;  // O staging bf16 [64][128] 16 KB (1024-aligned)
 constexpr uint32_t SM_MISC = SM_OST + 16384;
-constexpr uint32_t MISC_BYTES = 10240;
+constexpr uint32_t MISC_BYTES = 4096;
 constexpr uint32_t SMEM_BYTES = SM_MISC + MISC_BYTES + 1024;
 
 // misc layout
+// Hand-offs: FULL (TMA -> front), GC (front -> scan: decay totals), FR
+// (front -> back: A tile and operands), AFREE (back -> front: A tile
+// released), PRO (back -> scan: W'^T, U^T), G1 / G23 / D1 / D2 (UMMA
+// completions), BUF (stage and KX/P buffers free), DFREE (Δ^T columns free
+// for the next U^T), WFREE (W'^T tile free).
 enum Bar {
-  B_FULL0 = 0, B_FULL1, B_G1, B_G23, B_D1, B_D2, B_GC0, B_GC1, B_PRO0, B_PRO1, B_BUF0, B_BUF1,
-  B_DFREE, B_WFREE, B_DRAIN_PG, B_DRAIN_SG, B_NEVER, NUM_BARS
+  B_FULL0 = 0, B_FULL1, B_G1, B_G23, B_D1, B_D2, B_GC0, B_GC1, B_FR0, B_FR1, B_AFREE, B_PRO0, B_PRO1,
+  B_BUF0, B_BUF1, B_DFREE, B_WFREE, B_DRAIN_F, B_DRAIN_B, B_DRAIN_SG, B_NEVER, NUM_BARS
 };
-constexpr uint32_t MS_TMEM = 160, MS_ABORT = 164, MS_FAST = 168, MS_CNT = 176;  // MS_CNT: int[4]
-constexpr uint32_t MS_T0 = 192;  // int64: clock at block start (timing dump)
+constexpr uint32_t MS_TMEM = 192, MS_ABORT = 196, MS_FAST = 200, MS_CNT = 208;  // MS_CNT: int[4]
+constexpr uint32_t MS_T0 = 224;  // int64: clock at block start (timing dump)
 constexpr uint32_t MS_BETA = 256;    // [2][64] fp32
 constexpr uint32_t MS_GC = 768;      // [2][128] fp32: exp(G_C)
-constexpr uint32_t MS_RED = 1792;    // [8][128] fp32 log2 sums
-constexpr uint32_t MS_PRD = 5888;    // [8][128] fp32 products
-constexpr uint32_t MS_END = 9984;
+constexpr uint32_t MS_RED = 1792;    // [4][128] fp32 log2 sums
+constexpr uint32_t MS_END = 3840;
 static_assert(NUM_BARS * 8 <= MS_TMEM, "barrier area");
 static_assert(MS_END <= MISC_BYTES, "misc area");
 
 // ---- TMEM columns
 constexpr uint32_t TM_S = 0;        // S^T fp32, 128 cols
 constexpr uint32_t TM_O = 128;      // O^T fp32, 2 x 64 cols
-constexpr uint32_t TM_DELTA = 256;  // U^T, then Δ^T, fp32, 64 cols
-constexpr uint32_t TM_GW = 320;     // Gram, then W'^T, fp32, 64 cols
+constexpr uint32_t TM_DELTA = 256;  // U^T, then Δ^T fp32; then Δ^T fp16 pairs (A operand) in its first 32 cols
+constexpr uint32_t TM_G = 320;      // Gram [P ; A_raw], fp32, 64 cols
 constexpr uint32_t TM_SB = 384;     // S'^T fp16 pairs (A operand), 64 cols
-constexpr uint32_t TM_DT = 448;     // Δ^T fp16 pairs (A operand), 32 cols
+constexpr uint32_t TM_W = 448;      // W'^T fp32, 64 cols
 constexpr uint32_t TMEM_COLS = 512;
 
 // ---- debug dump (floats) for chain 0, chunk 0
 constexpr int DBG_P = 0, DBG_A = 4096, DBG_T = 8192, DBG_W = 12288, DBG_U = 20480, DBG_DELTA = 28672,
               DBG_O = 36864, DBG_S = 45056, DBG_GC = 61440, DBG_TIME = 61568, DBG_FLOATS = 65664;
 // DBG_TIME: int64 [64 chunks][32 events] of SM clock cycles since block start
-// (events 0-7 and 16-23 prologue group, 8-15 scan group), chain 0 only.
+// (events 0-6 front group, 16-23 and 25 back group, 8-15 and 24 scan group),
+// chain 0 only.
 constexpr int TIME_CHUNKS = 64;
 
 // ------------------------------------------------------------------ helpers
@@ -218,8 +226,14 @@ __device__ __forceinline__ bool cwait(const Ctx& x, int bar, uint32_t parity, in
   return false;
 }
 
+// Named-barrier ids of the three 128-thread groups, and each group's first thread.
+constexpr int GRP_FRONT = 1, GRP_SG = 2, GRP_BACK = 3;
+__device__ __forceinline__ unsigned grp_leader(int grp) {
+  return grp == GRP_SG ? 0u : (grp == GRP_FRONT ? 128u : 256u);
+}
+
 // Group-uniform bounded wait: every thread of named-barrier group `grp`
-// (nthr threads) polls, then the group agrees on the outcome, so no thread can
+// (128 threads) polls, then the group agrees on the outcome, so no thread can
 // leave a loop while the others wait at a barrier or a .sync.aligned op.
 //
 // Only the group's first thread polls the mbarrier; the others block in the
@@ -227,8 +241,8 @@ __device__ __forceinline__ bool cwait(const Ctx& x, int bar, uint32_t parity, in
 // memory bandwidth from the warps that are working.  The barrier (with the
 // tcgen05 / proxy fences the callers place after it) carries the observed
 // completion to the rest of the group.
-__device__ __forceinline__ bool gwait(const Ctx& x, int bar, uint32_t parity, int where, int grp, int nthr) {
-  const bool elected = threadIdx.x == (grp == 2 ? 0u : 128u);
+__device__ __forceinline__ bool gwait(const Ctx& x, int bar, uint32_t parity, int where, int grp) {
+  const bool elected = threadIdx.x == grp_leader(grp);
   bool ok = true;
   if (elected) {
     ok = wait_bar(&x.bars[bar], parity, x.wait_ns, x.abort);
@@ -237,7 +251,7 @@ __device__ __forceinline__ bool gwait(const Ctx& x, int bar, uint32_t parity, in
       *x.abort = 1;
     }
   }
-  ok = named_sync_and(grp, nthr, ok);
+  ok = named_sync_and(grp, 128, ok);
   // Each thread also observes the completed phase itself (an acquire that
   // returns at once), so the data it guards is visible to every thread.
   if (ok && !elected) mbar_try_wait(&x.bars[bar], parity);
@@ -249,141 +263,156 @@ __device__ __forceinline__ int chunk_valid(const Ctx& x, int c) {
   return rem < CH ? (int)rem : CH;
 }
 
-// ======================================================== prologue group
-// 8 warps (256 threads).  Row-wise work: thread (rg = warp 0..7, lane) owns
-// rows 8 rg .. 8 rg + 7 and channels 4 lane .. 4 lane + 3.  TMEM work: warp
-// rg reads lane quarter rg % 4 and column half rg / 4.
-constexpr int PG_THREADS = 256;
+// ============================================== front and back groups
+// Two 128-thread groups share the chunk prologue and run one chunk apart:
+// while the back group finishes chunk c, the front group starts chunk c+1.
+//   front (warps 4-7): decay prefix fused with operand scaling, the G1 Gram
+//     UMMA, and the P / A tiles;
+//   back (warps 8-11): the triangular solve, T', the G2/G3 UMMAs and W'^T.
+// Row-wise front work: thread f (warp wq = f / 32, lane) owns rows
+// 16 wq .. 16 wq + 15 and channels 4 lane .. 4 lane + 3.  TMEM work: a warp
+// reads the lane quarter (warp index mod 4) it is allowed to access.
+constexpr int GRP = 128;  // threads per group
 
 // General chunks: P and A on CUDA cores from the exact decay differences
-// G_r - G_s (log2 units), staged through the W'^T tile in two channel halves.
-__device__ __forceinline__ void general_gram(const Ctx& x, uint32_t stg, int b2, int valid, const float4 (&G)[8]) {
-  const int p = threadIdx.x - 128;
-  const int rg = p >> 5, lane = p & 31;
+// G_r - G_s (log2 units), G staged through the A tile one channel half at a
+// time (the back group has released the A tile).  Raw Q and K are read from
+// the stage before they are rescaled in place.
+__device__ __forceinline__ void general_gram(const Ctx& x, int b2, int valid, const float4 (&gv)[16], float4 off) {
+  const int f = threadIdx.x - 128;
+  const int wq = f >> 5, lane = f & 31;
   const int ch0 = 4 * lane, hh = ch0 >> 6, cc = ch0 & 63;
   uint8_t* sm = x.sm;
   const float* s_beta = reinterpret_cast<const float*>(sm + SM_MISC + MS_BETA) + b2 * 64;
-  const int r = p & 63, s0 = (p >> 6) * 16;
+  const int r = f & 63;
   const uint8_t* stp = sm + b2 * STAGE_BYTES;
-  (void)stg;
-  float pa[16], aa[16];
+  uint32_t pk[2][8];
+  float ak[2][16];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) pa[i] = aa[i] = 0.f;
-  for (int half = 0; half < 2; ++half) {
-    named_sync(1, PG_THREADS);
-    if (hh == half) {
+  for (int j = 0; j < 2; ++j) {
+    const int s0 = (f >> 6) * 32 + 16 * j;
+    float pa[16], aa[16];
 #pragma unroll
-      for (int m = 0; m < 8; ++m) *reinterpret_cast<float4*>(sm + SM_WT + (8 * rg + m) * 256 + cc * 4) = G[m];
-    }
-    named_sync(1, PG_THREADS);
-    if (r < valid && s0 <= r) {
+    for (int i = 0; i < 16; ++i) pa[i] = aa[i] = 0.f;
+    for (int half = 0; half < 2; ++half) {
+      named_sync(GRP_FRONT, GRP);  // earlier readers of the staging tile are done
+      if (hh == half) {
+        float4 gr = off;
+#pragma unroll
+        for (int m = 0; m < 16; ++m) {
+          gr.x += gv[m].x; gr.y += gv[m].y; gr.z += gv[m].z; gr.w += gv[m].w;
+          *reinterpret_cast<float4*>(sm + SM_A + (16 * wq + m) * 256 + cc * 4) = gr;
+        }
+      }
+      named_sync(GRP_FRONT, GRP);
+      if (r < valid && s0 <= r) {
 #pragma unroll 1
-      for (int ch = 0; ch < 64; ++ch) {
-        const uint32_t off_r = half * 16384 + sw128_off(r, ch);
-        const float gr = *reinterpret_cast<const float*>(sm + SM_WT + r * 256 + ch * 4);
-        const float qr = ld_bf16(stp + OFF_QK + off_r), kr = ld_bf16(stp + OFF_QK + 8192 + off_r);
+        for (int ch = 0; ch < 64; ++ch) {
+          const uint32_t off_r = half * 16384 + sw128_off(r, ch);
+          const float gr = *reinterpret_cast<const float*>(sm + SM_A + r * 256 + ch * 4);
+          const float qr = ld_bf16(stp + OFF_QK + off_r), kr = ld_bf16(stp + OFF_QK + 8192 + off_r);
 #pragma unroll 4
-        for (int i = 0; i < 16; ++i) {
-          const int s = s0 + i;
-          if (s <= r) {
-            const float gs = *reinterpret_cast<const float*>(sm + SM_WT + s * 256 + ch * 4);
-            const float ks = ld_bf16(stp + OFF_QK + 8192 + half * 16384 + sw128_off(s, ch));
-            const float e = ex2(gr - gs) * ks;
-            pa[i] += qr * e;
-            aa[i] += kr * e;
+          for (int i = 0; i < 16; ++i) {
+            const int s = s0 + i;
+            if (s <= r) {
+              const float gs = *reinterpret_cast<const float*>(sm + SM_A + s * 256 + ch * 4);
+              const float ks = ld_bf16(stp + OFF_QK + 8192 + half * 16384 + sw128_off(s, ch));
+              const float e = ex2(gr - gs) * ks;
+              pa[i] += qr * e;
+              aa[i] += kr * e;
+            }
           }
         }
       }
     }
-  }
-  const float br = s_beta[r];
+    const float br = s_beta[r];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const int s = s0 + i;
-    aa[i] = s < r ? br * aa[i] : 0.f;
-    if (!(s <= r)) pa[i] = 0.f;
-  }
+    for (int i = 0; i < 16; ++i) {
+      const int s = s0 + i;
+      ak[j][i] = s < r ? br * aa[i] : 0.f;
+      if (!(s <= r)) pa[i] = 0.f;
+    }
 #pragma unroll
-  for (int q8 = 0; q8 < 2; ++q8) {
-    const int s = s0 + 8 * q8;
-    st_f16x8(sm + SM_P + b2 * 8192 + r * 128 + ((((s >> 3) ^ r) & 7) << 4), pa + 8 * q8);
+    for (int i = 0; i < 8; ++i) pk[j][i] = pack_f16x2(pa[2 * i], pa[2 * i + 1]);
   }
+  named_sync(GRP_FRONT, GRP);  // every staged G read is done before A overwrites the tile
 #pragma unroll
-  for (int u = 0; u < 4; ++u)
-    *reinterpret_cast<float4*>(sm + SM_A + a_off(r, s0 + 4 * u)) =
-        make_float4(aa[4 * u], aa[4 * u + 1], aa[4 * u + 2], aa[4 * u + 3]);
-  named_sync(1, PG_THREADS);  // raw Q/K reads are done before they are rescaled in place
+  for (int j = 0; j < 2; ++j) {
+    const int s0 = (f >> 6) * 32 + 16 * j;
+#pragma unroll
+    for (int q8 = 0; q8 < 2; ++q8) {
+      const int s = s0 + 8 * q8;
+      *reinterpret_cast<uint4*>(sm + SM_P + b2 * 8192 + r * 128 + ((((s >> 3) ^ r) & 7) << 4)) =
+          make_uint4(pk[j][4 * q8], pk[j][4 * q8 + 1], pk[j][4 * q8 + 2], pk[j][4 * q8 + 3]);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      *reinterpret_cast<float4*>(sm + SM_A + a_off(r, s0 + 4 * u)) =
+          make_float4(ak[j][4 * u], ak[j][4 * u + 1], ak[j][4 * u + 2], ak[j][4 * u + 3]);
+  }
+  named_sync(GRP_FRONT, GRP);  // raw Q/K reads are done before they are rescaled in place
 }
 
-// Debug dump of P (fp16 tile) and A (fp32 tile) for chunk 0 of chain 0.
-__device__ __noinline__ void dump_pa(float* dbg, const uint8_t* sm, int b2) {
-  const int p = threadIdx.x - 128;
-  for (int e = p; e < 4096; e += PG_THREADS) {
+// Debug dumps (chain 0, chunk 0): P (fp16 tile) and A (fp32 tile); T'; W'
+// (from the fp16 W'^T tile) and U (TMEM, before D1).
+__device__ __noinline__ void dump_pa(float* dbg, const uint8_t* sm, int b2, int p) {
+  for (int e = p; e < 4096; e += GRP) {
     const int r = e >> 6, s = e & 63;
     const uint16_t u = *reinterpret_cast<const uint16_t*>(sm + SM_P + b2 * 8192 + sw128_off(r, s));
     dbg[DBG_P + e] = __half2float(*reinterpret_cast<const __half*>(&u));
     dbg[DBG_A + e] = *reinterpret_cast<const float*>(sm + SM_A + a_off(r, s));
   }
 }
-// Debug dump of T' (fp16 tile).
-__device__ __noinline__ void dump_t(float* dbg, const uint8_t* sm) {
-  const int p = threadIdx.x - 128;
-  for (int e = p; e < 4096; e += PG_THREADS) {
-    const uint16_t u = *reinterpret_cast<const uint16_t*>(sm + SM_A + sw128_off(e >> 6, e & 63));
+__device__ __noinline__ void dump_t(float* dbg, const uint8_t* sm, int p) {
+  for (int e = p; e < 4096; e += GRP) {
+    const uint16_t u = *reinterpret_cast<const uint16_t*>(sm + SM_TP + sw128_off(e >> 6, e & 63));
     dbg[DBG_T + e] = __half2float(*reinterpret_cast<const __half*>(&u));
   }
 }
-// Debug dump of W' (from the fp16 W'^T tile) and U (TMEM, before D1).
-__device__ __noinline__ void dump_wu(float* dbg, const uint8_t* sm, uint32_t tmem) {
-  const int p = threadIdx.x - 128;
-  for (int e = p; e < 8192; e += PG_THREADS) {
+__device__ __noinline__ void dump_wu(float* dbg, const uint8_t* sm, uint32_t tmem, int p) {
+  for (int e = p; e < 8192; e += GRP) {
     const int r = e >> 7, c = e & 127;  // W'[r][c] = W'^T[c][r]
     const uint16_t u = *reinterpret_cast<const uint16_t*>(sm + SM_WT + sw128_off(c, r));
     dbg[DBG_W + e] = __half2float(*reinterpret_cast<const __half*>(&u));
   }
-  const int rg = p >> 5;
-  if (rg < 4) {  // warps 4..7 read lane quarter rg of U^T
-    const uint32_t tl = tmem + ((uint32_t)(rg * 32) << 16);
-    const int j = rg * 32 + (p & 31);
-    float u0[32];
-    for (int half = 0; half < 2; ++half) {
-      tmem_ld32(tl + TM_DELTA + half * 32, u0);
-      for (int i = 0; i < 32; ++i) dbg[DBG_U + (half * 32 + i) * 128 + j] = u0[i];
-    }
+  const int lq = p >> 5;  // lane quarter of this warp
+  const uint32_t tl = tmem + ((uint32_t)(lq * 32) << 16);
+  const int j = lq * 32 + (p & 31);
+  float u0[32];
+  for (int half = 0; half < 2; ++half) {
+    tmem_ld32(tl + TM_DELTA + half * 32, u0);
+    for (int i = 0; i < 32; ++i) dbg[DBG_U + (half * 32 + i) * 128 + j] = u0[i];
   }
 }
 
-__device__ void prologue_group(const Ctx& x, const float* __restrict__ g, const float* __restrict__ beta,
-                               int (&consumed)[2]) {
-  const int p = threadIdx.x - 128;  // 0..255
-  const int rg = p >> 5, lane = p & 31;
+__device__ void front_group(const Ctx& x, const float* __restrict__ g, const float* __restrict__ beta,
+                            int (&consumed)[2]) {
+  const int f = threadIdx.x - 128;  // 0..127
+  const int wq = f >> 5, lane = f & 31;
   const int ch0 = 4 * lane, hh = ch0 >> 6, cc = ch0 & 63;
-  const int lq = rg & 3, chalf = rg >> 2;  // TMEM lane quarter, column half
-  const uint32_t tl = x.tmem + ((uint32_t)(lq * 32) << 16);
-  const int ti = lq * 32 + lane;  // this thread's TMEM lane
+  const uint32_t tl = x.tmem + ((uint32_t)(wq * 32) << 16);
   uint8_t* sm = x.sm;
   const uint32_t sb = x.sb;
-  float* s_red = reinterpret_cast<float*>(sm + SM_MISC + MS_RED);   // [8][128] log2 sums
-  float* s_prd = reinterpret_cast<float*>(sm + SM_MISC + MS_PRD);   // [8][128] products
+  float* s_red = reinterpret_cast<float*>(sm + SM_MISC + MS_RED);  // [4][128] log2 sums
   const int H = x.H;
 
-  // Register prefetch of this thread's g rows (8 x float4) and of beta.
-  auto load_g = [&](int c, float4(&gv)[8], float& bv) {
+  // Register prefetch of this thread's g rows (16 x float4) and of beta.
+  auto load_g = [&](int c, float4(&gv)[16], float& bv) {
     const int valid = c < x.nchunks ? chunk_valid(x, c) : 0;
     const int64_t tok0 = x.t0 + (int64_t)c * CH;
 #pragma unroll
-    for (int m = 0; m < 8; ++m) {
-      const int r = 8 * rg + m;
+    for (int m = 0; m < 16; ++m) {
+      const int r = 16 * wq + m;
       gv[m] = r < valid ? __ldg(reinterpret_cast<const float4*>(g + ((tok0 + r) * H + x.h) * D + ch0))
                         : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    bv = (p < CH && p < valid) ? __ldg(beta + (tok0 + p) * H + x.h) : 0.f;
+    bv = (f < CH && f < valid) ? __ldg(beta + (tok0 + f) * H + x.h) : 0.f;
   };
 
-  float4 gv[8];
+  float4 gv[16];
   float bv;
   load_g(0, gv, bv);
-  int g1_ph = 0, g23_ph = 0;
+  int g1_ph = 0;
 
   for (int c = 0; c < x.nchunks; ++c) {
     const int b2 = c & 1;
@@ -394,178 +423,188 @@ __device__ void prologue_group(const Ctx& x, const float* __restrict__ g, const 
     float* s_beta = reinterpret_cast<float*>(sm + SM_MISC + MS_BETA) + b2 * 64;
     volatile int* s_fast = reinterpret_cast<volatile int*>(sm + SM_MISC + MS_FAST) + b2;
 
-    if (p == 0) tmark(x, c, 0);
+    if (f == 0) tmark(x, c, 0);
     // Buffers [b2] were last used by the scan of chunk c-2.
-    if (c >= 2 && !gwait(x, B_BUF0 + b2, ((c >> 1) - 1) & 1, 11, 1, PG_THREADS)) break;
-    if (!gwait(x, B_FULL0 + b2, (c >> 1) & 1, 12, 1, PG_THREADS)) break;
+    if (c >= 2 && !gwait(x, B_BUF0 + b2, ((c >> 1) - 1) & 1, 11, GRP_FRONT)) break;
+    if (!gwait(x, B_FULL0 + b2, (c >> 1) & 1, 12, GRP_FRONT)) break;
     ++consumed[b2];
-    if (p == 0) tmark(x, c, 1);
+    if (f == 0) tmark(x, c, 1);
 
-    // ---- (a1) decay factors.  alpha = e^g (one MUFU op per element); the
-    // cumulative products give e^{G_r} and e^{G_C - G_r}, and the log2 sums
-    // give G for the range test and the general variant.
-    float4 fw[8], bw[8];
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f), pr = make_float4(1.f, 1.f, 1.f, 1.f);
+    // ---- (a1) decay prefix in log2 units: this thread's 16-row sums, then
+    // the offsets of the earlier row groups and the chunk total G_C.
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int m = 0; m < 8; ++m) {
-      const float4 l = make_float4(gv[m].x * LOG2E, gv[m].y * LOG2E, gv[m].z * LOG2E, gv[m].w * LOG2E);
-      bw[m] = ex2_4(l);  // alpha of row m (kept for the suffix products)
-      acc.x += l.x; acc.y += l.y; acc.z += l.z; acc.w += l.w;
-      pr = mul4(pr, bw[m]);
-      gv[m] = acc;  // local inclusive log2 prefix
-      fw[m] = pr;   // local inclusive product
+    for (int m = 0; m < 16; ++m) {
+      gv[m] = make_float4(gv[m].x * LOG2E, gv[m].y * LOG2E, gv[m].z * LOG2E, gv[m].w * LOG2E);
+      acc.x += gv[m].x; acc.y += gv[m].y; acc.z += gv[m].z; acc.w += gv[m].w;
     }
-    {
-      float4 sp = make_float4(1.f, 1.f, 1.f, 1.f);  // suffix products within the 8 rows
-#pragma unroll
-      for (int m = 7; m >= 0; --m) {
-        const float4 a = bw[m];
-        bw[m] = sp;
-        sp = mul4(sp, a);
-      }
-    }
-    *reinterpret_cast<float4*>(s_red + rg * 128 + ch0) = acc;
-    *reinterpret_cast<float4*>(s_prd + rg * 128 + ch0) = pr;
-    named_sync(1, PG_THREADS);
+    *reinterpret_cast<float4*>(s_red + wq * 128 + ch0) = acc;
+    named_sync(GRP_FRONT, GRP);
     float4 tot = make_float4(0.f, 0.f, 0.f, 0.f), off = tot;
-    float4 fo = make_float4(1.f, 1.f, 1.f, 1.f), bo = fo;
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
+    for (int q = 0; q < 4; ++q) {
       const float4 v = *reinterpret_cast<const float4*>(s_red + q * 128 + ch0);
-      const float4 w = *reinterpret_cast<const float4*>(s_prd + q * 128 + ch0);
-      if (q < rg) {
-        off.x += v.x; off.y += v.y; off.z += v.z; off.w += v.w;
-        fo = mul4(fo, w);
-      }
-      if (q > rg) bo = mul4(bo, w);
+      if (q < wq) { off.x += v.x; off.y += v.y; off.z += v.z; off.w += v.w; }
       tot.x += v.x; tot.y += v.y; tot.z += v.z; tot.w += v.w;
     }
-#pragma unroll
-    for (int m = 0; m < 8; ++m) {
-      gv[m].x += off.x; gv[m].y += off.y; gv[m].z += off.z; gv[m].w += off.w;  // G (log2)
-    }
     const bool fast =
-        named_sync_and(1, PG_THREADS, fminf(fminf(tot.x, tot.y), fminf(tot.z, tot.w)) >= FAST_MIN_LOG2);
-    if (rg == 0) *reinterpret_cast<float4*>(s_gc + ch0) = ex2_4(tot);
-    if (p == 0) *s_fast = fast ? 1 : 0;
-    if (p < CH) s_beta[p] = bv;
-    if (dmp && rg == 0) {
+        named_sync_and(GRP_FRONT, GRP, fminf(fminf(tot.x, tot.y), fminf(tot.z, tot.w)) >= FAST_MIN_LOG2);
+    if (wq == 0) *reinterpret_cast<float4*>(s_gc + ch0) = ex2_4(tot);
+    if (f == 0) *s_fast = fast ? 1 : 0;
+    if (f < CH) s_beta[f] = bv;
+    if (dmp && wq == 0) {
       const float LN2 = 0.6931471805599453f;
       x.dbg[DBG_GC + ch0] = tot.x * LN2; x.dbg[DBG_GC + ch0 + 1] = tot.y * LN2;
       x.dbg[DBG_GC + ch0 + 2] = tot.z * LN2; x.dbg[DBG_GC + ch0 + 3] = tot.w * LN2;
     }
-    named_sync(1, PG_THREADS);
-    if (p == 0) {
-      mbar_arrive(&x.bars[B_GC0 + b2]);
-      tmark(x, c, 2);
-    }
-    // Row factors: E = e^{G_r - ref} (ref = G_C on fast chunks, 0 otherwise), H = e^{G_C - G_r}.
-    {
-      float4 ef = fo;
-      if (fast) ef = mul4(ef, ex2_4(make_float4(-tot.x, -tot.y, -tot.z, -tot.w)));
-#pragma unroll
-      for (int m = 0; m < 8; ++m) {
-        fw[m] = mul4(fw[m], ef);
-        bw[m] = mul4(bw[m], bo);
-      }
-    }
+    mbar_arrive(&x.bars[B_GC0 + b2]);  // one arrival per thread, after its own writes
+    if (f == 0) tmark(x, c, 2);
 
     if (!fast) {
-      if (c >= 1 && !gwait(x, B_WFREE, (c - 1) & 1, 13, 1, PG_THREADS)) break;
-      general_gram(x, stg, b2, valid, gv);
+      if (c >= 1 && !gwait(x, B_AFREE, (c - 1) & 1, 13, GRP_FRONT)) break;
+      general_gram(x, b2, valid, gv, off);
     }
 
-    // ---- (a2) operand scaling: QE, KE in place, KH into KX[b2], V -> fp16.
+    // ---- (a2) operand scaling, row by row: E = e^{G_r - ref} (ref = G_C on
+    // fast chunks, 0 otherwise), H = e^{G_C - G_r};  QE, KE, V (fp16) in
+    // place, KH into KX[b2].
     {
+      const float4 ref = fast ? tot : make_float4(0.f, 0.f, 0.f, 0.f);
+      float4 gr = off;
       uint8_t* qb = sm + b2 * STAGE_BYTES + OFF_QK + hh * 16384;
       uint8_t* kb = qb + 8192;
       uint8_t* vb = sm + b2 * STAGE_BYTES + OFF_V + hh * 8192;
       uint8_t* khb = sm + SM_KX + b2 * 16384 + hh * 8192;
-      uint2 qr[8], kr[8], vr[8];
-#pragma unroll
-      for (int m = 0; m < 8; ++m) {  // all loads first, then the in-place stores
-        const uint32_t o = sw128_off(8 * rg + m, cc);
-        qr[m] = *reinterpret_cast<const uint2*>(qb + o);
-        kr[m] = *reinterpret_cast<const uint2*>(kb + o);
-        vr[m] = *reinterpret_cast<const uint2*>(vb + o);
-      }
       bool bad = false;
 #pragma unroll
-      for (int m = 0; m < 8; ++m) {
-        const int r = 8 * rg + m;
-        const uint32_t o = sw128_off(r, cc);
-        float4 q4 = bf16x4_to_f32(qr[m]), k4 = bf16x4_to_f32(kr[m]), v4 = bf16x4_to_f32(vr[m]);
-        if (r >= valid) q4 = k4 = v4 = make_float4(0.f, 0.f, 0.f, 0.f);
-        bad |= amax4(v4) > F16_SAFE;
-        st_f16x4(qb + o, mul4(q4, fw[m]));
-        st_f16x4(kb + o, mul4(k4, fw[m]));
-        st_f16x4(vb + o, v4);
-        st_f16x4(khb + o, mul4(k4, bw[m]));
+      for (int mb = 0; mb < 16; mb += 4) {
+        uint2 qr[4], kr[4], vr[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {  // this batch's loads first, then the in-place stores
+          const uint32_t o = sw128_off(16 * wq + mb + i, cc);
+          qr[i] = *reinterpret_cast<const uint2*>(qb + o);
+          kr[i] = *reinterpret_cast<const uint2*>(kb + o);
+          vr[i] = *reinterpret_cast<const uint2*>(vb + o);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int m = mb + i, r = 16 * wq + m;
+          const uint32_t o = sw128_off(r, cc);
+          gr.x += gv[m].x; gr.y += gv[m].y; gr.z += gv[m].z; gr.w += gv[m].w;
+          const float4 fw = ex2_4(make_float4(gr.x - ref.x, gr.y - ref.y, gr.z - ref.z, gr.w - ref.w));
+          const float4 bw = ex2_4(make_float4(tot.x - gr.x, tot.y - gr.y, tot.z - gr.z, tot.w - gr.w));
+          float4 q4 = bf16x4_to_f32(qr[i]), k4 = bf16x4_to_f32(kr[i]), v4 = bf16x4_to_f32(vr[i]);
+          if (r >= valid) q4 = k4 = v4 = make_float4(0.f, 0.f, 0.f, 0.f);
+          bad |= amax4(v4) > F16_SAFE;
+          st_f16x4(qb + o, mul4(q4, fw));
+          st_f16x4(kb + o, mul4(k4, fw));
+          st_f16x4(vb + o, v4);
+          st_f16x4(khb + o, mul4(k4, bw));
+        }
       }
       if (bad) record_error(x.status, KDA_ERR_RANGE, 20);
     }
     fence_proxy_async_smem();
-    named_sync(1, PG_THREADS);
-    if (p == 0) tmark(x, c, 3);
+    named_sync(GRP_FRONT, GRP);
+    if (f == 0) tmark(x, c, 3);
 
     if (fast) {
       // ---- G1: [P ; A_raw] = [QE ; KE] . KH^T   (M=128, N=64, K=128)
-      if (p == 0) {
-        tc_fence_after();
-        const uint32_t id = idesc_f16_f32(128, 64, 0, 0);
+      if (f == 0) {
+        bool ok = true;
+        if (c >= 1) ok = cwait(x, B_AFREE, (c - 1) & 1, 14);  // the back group is done with A of c-1
+        if (ok) {
+          tc_fence_after();
+          const uint32_t id = idesc_f16_f32(128, 64, 0, 0);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const uint64_t da = sdesc_sw128(stg + OFF_QK + (i >> 2) * 16384 + (i & 3) * 32, 16, 1024);
-          const uint64_t db = sdesc_sw128(sb + SM_KX + b2 * 16384 + (i >> 2) * 8192 + (i & 3) * 32, 16, 1024);
-          umma_ss(x.tmem + TM_GW, da, db, id, i > 0);
+          for (int i = 0; i < 8; ++i) {
+            const uint64_t da = sdesc_sw128(stg + OFF_QK + (i >> 2) * 16384 + (i & 3) * 32, 16, 1024);
+            const uint64_t db = sdesc_sw128(sb + SM_KX + b2 * 16384 + (i >> 2) * 8192 + (i & 3) * 32, 16, 1024);
+            umma_ss(x.tmem + TM_G, da, db, id, i > 0);
+          }
+          umma_commit(&x.bars[B_G1]);
         }
-        umma_commit(&x.bars[B_G1]);
-        tmark(x, c, 20);
+        tmark(x, c, 4);
       }
-      if (!gwait(x, B_G1, g1_ph, 14, 1, PG_THREADS)) break;
+      if (!gwait(x, B_G1, g1_ph, 15, GRP_FRONT)) break;
       g1_ph ^= 1;
-      if (p == 0) tmark(x, c, 21);
       tc_fence_after();
-      float r0[32];
-      tmem_ld32(tl + TM_GW + chalf * 32, r0);  // row ti, columns 32 chalf .. +31
-      if (ti < CH) {  // P row, lower triangle including the diagonal
+      if (f == 0) tmark(x, c, 5);
+      float r0[32], r1[32];
+      tmem_ld32x2(tl + TM_G, tl + TM_G + 32, r0, r1);  // TMEM lane f: row f of [P ; A_raw]
+      if (wq < 2) {  // P row f, lower triangle including the diagonal
+        const int r = f;
 #pragma unroll
-        for (int s = 0; s < 32; ++s)
-          if (chalf * 32 + s > ti) r0[s] = 0.f;
+        for (int s = 0; s < 32; ++s) {
+          if (s > r) r0[s] = 0.f;
+          if (32 + s > r) r1[s] = 0.f;
+        }
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const int q8 = chalf * 4 + k;
-          st_f16x8(sm + SM_P + b2 * 8192 + ti * 128 + (((q8 ^ ti) & 7) << 4), r0 + 8 * k);
+          st_f16x8(sm + SM_P + b2 * 8192 + r * 128 + (((k ^ r) & 7) << 4), r0 + 8 * k);
+          st_f16x8(sm + SM_P + b2 * 8192 + r * 128 + ((((4 + k) ^ r) & 7) << 4), r1 + 8 * k);
         }
       } else {  // A row r = beta_r (KE KH^T)_rs, strictly lower
-        const int r = ti - CH;
+        const int r = f - CH;
         const float b = s_beta[r];
 #pragma unroll
-        for (int s = 0; s < 32; ++s) r0[s] = (chalf * 32 + s < r) ? b * r0[s] : 0.f;
+        for (int s = 0; s < 32; ++s) {
+          r0[s] = s < r ? b * r0[s] : 0.f;
+          r1[s] = 32 + s < r ? b * r1[s] : 0.f;
+        }
 #pragma unroll
-        for (int u = 0; u < 8; ++u)
-          *reinterpret_cast<float4*>(sm + SM_A + a_off(r, chalf * 32 + 4 * u)) =
+        for (int u = 0; u < 8; ++u) {
+          *reinterpret_cast<float4*>(sm + SM_A + a_off(r, 4 * u)) =
               make_float4(r0[4 * u], r0[4 * u + 1], r0[4 * u + 2], r0[4 * u + 3]);
+          *reinterpret_cast<float4*>(sm + SM_A + a_off(r, 32 + 4 * u)) =
+              make_float4(r1[4 * u], r1[4 * u + 1], r1[4 * u + 2], r1[4 * u + 3]);
+        }
       }
       tc_fence_before();
-      named_sync(1, PG_THREADS);
     }
+    fence_proxy_async_smem();  // P is read by the D2 UMMA
     if (dmp) {
-      dump_pa(x.dbg, sm, b2);
-      named_sync(1, PG_THREADS);
+      named_sync(GRP_FRONT, GRP);
+      dump_pa(x.dbg, sm, b2, f);
     }
-    if (p == 0) tmark(x, c, 4);
+    named_sync(GRP_FRONT, GRP);  // the front's TMEM reads are done before the next G1
+    mbar_arrive(&x.bars[B_FR0 + b2]);
+    if (f == 0) tmark(x, c, 6);
+    load_g(c + 1, gv, bv);
+  }
+}
+
+__device__ void back_group(const Ctx& x) {
+  const int k = threadIdx.x - 256;  // 0..127
+  const int bw = k >> 5, lane = k & 31;
+  const uint32_t tl = x.tmem + ((uint32_t)(bw * 32) << 16);
+  const int ti = bw * 32 + lane;  // this thread's TMEM lane
+  uint8_t* sm = x.sm;
+  const uint32_t sb = x.sb;
+  int g23_ph = 0;
+
+  for (int c = 0; c < x.nchunks; ++c) {
+    const int b2 = c & 1;
+    const bool dmp = x.dbg && c == 0;
+    const uint32_t stg = sb + b2 * STAGE_BYTES;
+    const float* s_beta = reinterpret_cast<const float*>(sm + SM_MISC + MS_BETA) + b2 * 64;
+
+    if (k == 0) tmark(x, c, 16);
+    if (!gwait(x, B_FR0 + b2, (c >> 1) & 1, 21, GRP_BACK)) break;
+    if (k == 0) tmark(x, c, 17);
 
     // ---- (a3) T = (I + A)^-1 by blocks.  16x16 diagonal inverses E_a by
     // forward substitution; D_b = [[E_2b, 0], [-E_2b+1 A'_b E_2b, E_2b+1]] are
     // the 32x32 diagonal inverses; T_10 = -D_1 (A_10 D_0).
-    // T' = T diag(beta) as fp16 [r][s] over the A tile.
-    if (p < 64) {
+    // T' = T diag(beta) as fp16 [r][s] in the TP tile.
+    if (k < 64) {
       // Column sweep: once x[s] is final it updates every later row.  The
       // loads do not depend on x, so the dependency chain is one FMA per
       // column; column s+1 is fetched while column s is applied.
-      const int a = p >> 4, jj = p & 15;
-      auto ael = [&](int r, int c) { return *reinterpret_cast<const float*>(sm + SM_A + a_off(16 * a + r, 16 * a + c)); };
+      const int a = k >> 4, jj = k & 15;
+      auto ael = [&](int r, int cl) {
+        return *reinterpret_cast<const float*>(sm + SM_A + a_off(16 * a + r, 16 * a + cl));
+      };
       float xs[16], col[16], nxt[16];
 #pragma unroll
       for (int r = 0; r < 16; ++r) {
@@ -588,139 +627,146 @@ __device__ void prologue_group(const Ctx& x, const float* __restrict__ g, const 
       const int o = (a & 1) * 16;
 #pragma unroll
       for (int r = 0; r < 16; ++r) *reinterpret_cast<float*>(sm + db + b_off(o + r, o + jj)) = xs[r];
-    } else if (p < 128) {  // zero the upper-right 16x16 block of D_0 and D_1
-      const int t = p - 64, b = t >> 5, rr = (t & 31) >> 1, cb = 16 + (t & 1) * 8;
+    } else {  // zero the upper-right 16x16 block of D_0 and D_1
+      const int t = k - 64, b = t >> 5, rr = (t & 31) >> 1, cb = 16 + (t & 1) * 8;
 #pragma unroll
       for (int i = 0; i < 8; i += 4)
         *reinterpret_cast<float4*>(sm + SM_DG + b * 4096 + b_off(rr, cb + i)) = make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    named_sync(1, PG_THREADS);
-    if (p == 0) tmark(x, c, 16);
-    const int pw = p >> 5, lg = lane >> 2, lt = lane & 3;  // warp in group; mma fragment coordinates
-    if (pw < 4) {  // Y_b = A'_b E_2b  (A'_b = A[32b+16 .. +16][32b .. +16]) -> X tile as [2][16][16]
-      const int b = pw >> 1, nt = pw & 1;
+    named_sync(GRP_BACK, GRP);
+    if (k == 0) tmark(x, c, 18);
+    const int lg = lane >> 2, lt = lane & 3;  // mma fragment coordinates
+    {  // Y_b = A'_b E_2b (A'_b = A[32b+16 .. +16][32b .. +16]), then F_b = -E_2b+1 Y_b
+      const int b = bw >> 1, nt = bw & 1;
       float d[4];
       warp_gemm_tf32x3<2>(
-          d, [&](int r, int k) { return reinterpret_cast<const float*>(sm + SM_A + a_off(32 * b + 16 + r, 32 * b + k)); },
-          [&](int k, int n) { return reinterpret_cast<const float*>(sm + SM_DG + b * 4096 + b_off(k, 8 * nt + n)); });
+          d, [&](int r, int kk) { return reinterpret_cast<const float*>(sm + SM_A + a_off(32 * b + 16 + r, 32 * b + kk)); },
+          [&](int kk, int n) { return reinterpret_cast<const float*>(sm + SM_DG + b * 4096 + b_off(kk, 8 * nt + n)); });
       float* y = reinterpret_cast<float*>(sm + SM_X + b * 1024);
       *reinterpret_cast<float2*>(y + lg * 16 + 8 * nt + 2 * lt) = make_float2(d[0], d[1]);
       *reinterpret_cast<float2*>(y + (lg + 8) * 16 + 8 * nt + 2 * lt) = make_float2(d[2], d[3]);
     }
-    named_sync(1, PG_THREADS);
-    if (p == 0) tmark(x, c, 17);
-    if (pw < 4) {  // F_b = -E_2b+1 Y_b -> lower-left 16x16 block of D_b
-      const int b = pw >> 1, nt = pw & 1;
+    named_sync(GRP_BACK, GRP);
+    {
+      const int b = bw >> 1, nt = bw & 1;
       float d[4];
       warp_gemm_tf32x3<2>(
-          d, [&](int r, int k) { return reinterpret_cast<const float*>(sm + SM_DG + b * 4096 + b_off(16 + r, 16 + k)); },
-          [&](int k, int n) { return reinterpret_cast<const float*>(sm + SM_X + b * 1024 + (k * 16 + 8 * nt + n) * 4); });
+          d, [&](int r, int kk) { return reinterpret_cast<const float*>(sm + SM_DG + b * 4096 + b_off(16 + r, 16 + kk)); },
+          [&](int kk, int n) { return reinterpret_cast<const float*>(sm + SM_X + b * 1024 + (kk * 16 + 8 * nt + n) * 4); });
       uint8_t* db = sm + SM_DG + b * 4096;
       *reinterpret_cast<float2*>(db + b_off(16 + lg, 8 * nt + 2 * lt)) = make_float2(-d[0], -d[1]);
       *reinterpret_cast<float2*>(db + b_off(24 + lg, 8 * nt + 2 * lt)) = make_float2(-d[2], -d[3]);
     }
-    named_sync(1, PG_THREADS);
-    if (p == 0) tmark(x, c, 18);
-    {  // X = A_10 D_0  (32x32x32, one 16x8 tile per warp)
-      const int mt = pw >> 2, nt = pw & 3;
+    named_sync(GRP_BACK, GRP);
+    if (k == 0) tmark(x, c, 19);
+#pragma unroll
+    for (int t = bw; t < 8; t += 4) {  // X = A_10 D_0  (32x32x32, 16x8 tiles)
+      const int mt = t >> 2, nt = t & 3;
       float d[4];
       warp_gemm_tf32x3<4>(
-          d, [&](int r, int k) { return reinterpret_cast<const float*>(sm + SM_A + a_off(32 + 16 * mt + r, k)); },
-          [&](int k, int n) { return reinterpret_cast<const float*>(sm + SM_DG + b_off(k, 8 * nt + n)); });
+          d, [&](int r, int kk) { return reinterpret_cast<const float*>(sm + SM_A + a_off(32 + 16 * mt + r, kk)); },
+          [&](int kk, int n) { return reinterpret_cast<const float*>(sm + SM_DG + b_off(kk, 8 * nt + n)); });
       *reinterpret_cast<float2*>(sm + SM_X + b_off(16 * mt + lg, 8 * nt + 2 * lt)) = make_float2(d[0], d[1]);
       *reinterpret_cast<float2*>(sm + SM_X + b_off(16 * mt + lg + 8, 8 * nt + 2 * lt)) = make_float2(d[2], d[3]);
     }
-    named_sync(1, PG_THREADS);
-    if (p == 0) tmark(x, c, 19);
-    {  // T_10 = -D_1 X
-      const int mt = pw >> 2, nt = pw & 3;
+    named_sync(GRP_BACK, GRP);
+    if (k == 0) {
+      mbar_arrive(&x.bars[B_AFREE]);  // A is no longer read
+      tmark(x, c, 20);
+    }
+#pragma unroll
+    for (int t = bw; t < 8; t += 4) {  // T_10 = -D_1 X
+      const int mt = t >> 2, nt = t & 3;
       float d[4];
       warp_gemm_tf32x3<4>(
-          d, [&](int r, int k) { return reinterpret_cast<const float*>(sm + SM_DG + 4096 + b_off(16 * mt + r, k)); },
-          [&](int k, int n) { return reinterpret_cast<const float*>(sm + SM_X + b_off(k, 8 * nt + n)); });
+          d, [&](int r, int kk) { return reinterpret_cast<const float*>(sm + SM_DG + 4096 + b_off(16 * mt + r, kk)); },
+          [&](int kk, int n) { return reinterpret_cast<const float*>(sm + SM_X + b_off(kk, 8 * nt + n)); });
       *reinterpret_cast<float2*>(sm + SM_T10 + b_off(16 * mt + lg, 8 * nt + 2 * lt)) = make_float2(-d[0], -d[1]);
       *reinterpret_cast<float2*>(sm + SM_T10 + b_off(16 * mt + lg + 8, 8 * nt + 2 * lt)) = make_float2(-d[2], -d[3]);
     }
-    named_sync(1, PG_THREADS);
-    {  // T' = T diag(beta) as fp16 [r][s]: rows rr and 32 + rr, columns c4 .. c4+3 and 32 + c4 ..
-      const int rr = p >> 3, c4 = 4 * (p & 7);
-      const float4 bl = *reinterpret_cast<const float4*>(s_beta + c4);
-      const float4 bh = *reinterpret_cast<const float4*>(s_beta + 32 + c4);
-      const float4 d0 = *reinterpret_cast<const float4*>(sm + SM_DG + b_off(rr, c4));
-      const float4 d1 = *reinterpret_cast<const float4*>(sm + SM_DG + 4096 + b_off(rr, c4));
-      const float4 t10 = *reinterpret_cast<const float4*>(sm + SM_T10 + b_off(rr, c4));
-      st_f16x4(sm + SM_A + sw128_off(rr, c4), mul4(d0, bl));
-      st_f16x4(sm + SM_A + sw128_off(rr, 32 + c4), make_float4(0.f, 0.f, 0.f, 0.f));
-      st_f16x4(sm + SM_A + sw128_off(32 + rr, c4), mul4(t10, bl));
-      st_f16x4(sm + SM_A + sw128_off(32 + rr, 32 + c4), mul4(d1, bh));
+    named_sync(GRP_BACK, GRP);
+    {  // T' = T diag(beta) as fp16 [r][s]: rows rr and 32 + rr, columns c8 .. c8+7 and 32 + c8 ..
+      const int rr = k >> 2, c8 = 8 * (k & 3);
+      float4 t00[2], t10[2], t11[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int c4 = c8 + 4 * h;
+        const float4 bl = *reinterpret_cast<const float4*>(s_beta + c4);
+        const float4 bh = *reinterpret_cast<const float4*>(s_beta + 32 + c4);
+        t00[h] = mul4(*reinterpret_cast<const float4*>(sm + SM_DG + b_off(rr, c4)), bl);
+        t11[h] = mul4(*reinterpret_cast<const float4*>(sm + SM_DG + 4096 + b_off(rr, c4)), bh);
+        t10[h] = mul4(*reinterpret_cast<const float4*>(sm + SM_T10 + b_off(rr, c4)), bl);
+      }
+      named_sync(GRP_BACK, GRP);  // the TP tile overlays X and T_10
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int c4 = c8 + 4 * h;
+        st_f16x4(sm + SM_TP + sw128_off(rr, c4), t00[h]);
+        st_f16x4(sm + SM_TP + sw128_off(rr, 32 + c4), make_float4(0.f, 0.f, 0.f, 0.f));
+        st_f16x4(sm + SM_TP + sw128_off(32 + rr, c4), t10[h]);
+        st_f16x4(sm + SM_TP + sw128_off(32 + rr, 32 + c4), t11[h]);
+      }
     }
     fence_proxy_async_smem();
-    named_sync(1, PG_THREADS);
+    named_sync(GRP_BACK, GRP);
     if (dmp) {
-      dump_t(x.dbg, sm);
-      named_sync(1, PG_THREADS);
+      dump_t(x.dbg, sm, k);
+      named_sync(GRP_BACK, GRP);
     }
 
-    // ---- (a4) G2: W'^T = KE^T T'^T -> TM_GW;  G3: U^T = V^T T'^T -> TM_DELTA
-    if (p == 0) {
-      tmark(x, c, 5);
+    // ---- (a4) G2: W'^T = KE^T T'^T -> TM_W;  G3: U^T = V^T T'^T -> TM_DELTA
+    if (k == 0) {
+      tmark(x, c, 21);
       bool ok = true;
-      if (c >= 1) ok = cwait(x, B_DFREE, (c - 1) & 1, 15);  // scan has read Δ of chunk c-1
+      if (c >= 1) ok = cwait(x, B_DFREE, (c - 1) & 1, 22);  // D2 of chunk c-1 has read Δ
       if (ok) {
         tc_fence_after();
         const uint32_t id = idesc_f16_f32(128, 64, 1, 0);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const uint64_t da = sdesc_sw128(stg + OFF_QK + 8192 + i * 2048, 16384, 1024);
-          const uint64_t db = sdesc_sw128(sb + SM_A + i * 32, 16, 1024);
-          umma_ss(x.tmem + TM_GW, da, db, id, i > 0);
+          const uint64_t db = sdesc_sw128(sb + SM_TP + i * 32, 16, 1024);
+          umma_ss(x.tmem + TM_W, da, db, id, i > 0);
         }
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const uint64_t da = sdesc_sw128(stg + OFF_V + i * 2048, 8192, 1024);
-          const uint64_t db = sdesc_sw128(sb + SM_A + i * 32, 16, 1024);
+          const uint64_t db = sdesc_sw128(sb + SM_TP + i * 32, 16, 1024);
           umma_ss(x.tmem + TM_DELTA, da, db, id, i > 0);
         }
         umma_commit(&x.bars[B_G23]);
-        tmark(x, c, 22);
       }
+      tmark(x, c, 22);
     }
-    // Prefetch next chunk's decay and beta while the UMMAs run.
-    float4 gn[8];
-    float bn;
-    load_g(c + 1, gn, bn);
-    if (!gwait(x, B_G23, g23_ph, 16, 1, PG_THREADS)) break;
+    if (!gwait(x, B_G23, g23_ph, 23, GRP_BACK)) break;
     g23_ph ^= 1;
     tc_fence_after();
-    if (p == 0) tmark(x, c, 6);
-    if (fast && c >= 1 && !gwait(x, B_WFREE, (c - 1) & 1, 17, 1, PG_THREADS)) break;
-    {  // lane ti holds W'^T[ti][r] for r in this warp's column half: row ti of the MN-major B operand of D1
-      float w0[32];
-      tmem_ld32(tl + TM_GW + chalf * 32, w0);
+    if (k == 0) tmark(x, c, 23);
+    if (c >= 1 && !gwait(x, B_WFREE, (c - 1) & 1, 24, GRP_BACK)) break;
+    {  // lane ti holds W'^T[ti][r]: row ti of the MN-major B operand of D1
+      float w0[32], w1[32];
+      tmem_ld32x2(tl + TM_W, tl + TM_W + 32, w0, w1);
       float mx = 0.f;
 #pragma unroll
-      for (int i = 0; i < 32; ++i) mx = fmaxf(mx, fabsf(w0[i]));
+      for (int i = 0; i < 32; ++i) mx = fmaxf(mx, fmaxf(fabsf(w0[i]), fabsf(w1[i])));
       if (!(mx <= F16_SAFE)) record_error(x.status, KDA_ERR_RANGE, 21);
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int q = chalf * 4 + k;
-        st_f16x8(sm + SM_WT + ti * 128 + (((q ^ ti) & 7) << 4), w0 + 8 * k);
+      for (int q = 0; q < 4; ++q) {
+        st_f16x8(sm + SM_WT + ti * 128 + (((q ^ ti) & 7) << 4), w0 + 8 * q);
+        st_f16x8(sm + SM_WT + ti * 128 + ((((4 + q) ^ ti) & 7) << 4), w1 + 8 * q);
       }
     }
     fence_proxy_async_smem();
     tc_fence_before();
-    named_sync(1, PG_THREADS);
+    named_sync(GRP_BACK, GRP);
     if (dmp) {
-      dump_wu(x.dbg, sm, x.tmem);
-      named_sync(1, PG_THREADS);
+      dump_wu(x.dbg, sm, x.tmem, k);
+      named_sync(GRP_BACK, GRP);
     }
-    if (p == 0) {
+    if (k == 0) {
       mbar_arrive(&x.bars[B_PRO0 + b2]);
-      tmark(x, c, 7);
+      tmark(x, c, 25);
     }
-#pragma unroll
-    for (int m = 0; m < 8; ++m) gv[m] = gn[m];
-    bv = bn;
   }
 }
 
@@ -836,14 +882,14 @@ __device__ void scan_group(const Ctx& x, const void* tmq, const void* tmk, const
     const uint32_t stg = sb + b2 * STAGE_BYTES;
     const float* s_gc = reinterpret_cast<const float*>(sm + SM_MISC + MS_GC) + b2 * 128;
     if (j == 0) tmark(x, c, 8);
-    if (inject_stuck && c == 0 && !gwait(x, B_NEVER, 0, 99, 2, 128)) {
+    if (inject_stuck && c == 0 && !gwait(x, B_NEVER, 0, 99, GRP_SG)) {
       ok = false;
       break;
     }
     // ---- S pass: S^T (decayed to the chunk end when this chunk is "fast")
     // -> S'^T as fp16 pairs, the A operand of D1.
     if (c >= 1) {
-      if (!gwait(x, B_D2, d2_ph, 31, 2, 128)) {
+      if (!gwait(x, B_D2, d2_ph, 31, GRP_SG)) {
         ok = false;
         break;
       }
@@ -851,7 +897,7 @@ __device__ void scan_group(const Ctx& x, const void* tmq, const void* tmk, const
       tc_fence_after();
     }
     if (j == 0) tmark(x, c, 9);
-    if (!gwait(x, B_GC0 + b2, (c >> 1) & 1, 32, 2, 128)) {
+    if (!gwait(x, B_GC0 + b2, (c >> 1) & 1, 32, GRP_SG)) {
       ok = false;
       break;
     }
@@ -918,7 +964,7 @@ __device__ void scan_group(const Ctx& x, const void* tmq, const void* tmk, const
     }
     if (c >= 1) store_out(c - 1);
     if (j == 0) tmark(x, c, 12);
-    if (!gwait(x, B_D1, d1_ph, 34, 2, 128)) {
+    if (!gwait(x, B_D1, d1_ph, 34, GRP_SG)) {
       ok = false;
       break;
     }
@@ -942,6 +988,7 @@ __device__ void scan_group(const Ctx& x, const void* tmq, const void* tmk, const
         tmem_st32(tl + TM_S + cb * 32, s);
       }
     }
+    if (x.dbg && c == 0) dump_delta(x.dbg, x.tmem);  // before the fp16 pairs overwrite its first columns
     {
       float d0[32], d1[32];
       uint32_t pk[16];
@@ -952,16 +999,15 @@ __device__ void scan_group(const Ctx& x, const void* tmq, const void* tmk, const
         pk[i] = pack_f16x2(d0[2 * i], d0[2 * i + 1]);
         dm = fmaxf(dm, fmaxf(fabsf(d0[2 * i]), fabsf(d0[2 * i + 1])));
       }
-      tmem_st16(tl + TM_DT, pk);
+      tmem_st16(tl + TM_DELTA, pk);
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         pk[i] = pack_f16x2(d1[2 * i], d1[2 * i + 1]);
         dm = fmaxf(dm, fmaxf(fabsf(d1[2 * i]), fabsf(d1[2 * i + 1])));
       }
-      tmem_st16(tl + TM_DT + 16, pk);
+      tmem_st16(tl + TM_DELTA + 16, pk);
       if (!(dm <= F16_SAFE)) record_error(x.status, KDA_ERR_RANGE, 31);
     }
-    if (x.dbg && c == 0) dump_delta(x.dbg, x.tmem);
     tmem_wait_st();
     tc_fence_before();
     named_sync(2, 128);
@@ -969,27 +1015,27 @@ __device__ void scan_group(const Ctx& x, const void* tmq, const void* tmk, const
     // ---- D2: S^T += Δ^T KH ;  O^T += Δ^T P^T      (A = Δ^T from TMEM)
     if (j == 0) tmark(x, c, 14);
     if (j == 0) {
-      mbar_arrive(&x.bars[B_DFREE]);
       tc_fence_after();
       const uint32_t ids = idesc_f16_f32(128, 128, 0, 1);
       const uint32_t idp = idesc_f16_f32(128, 64, 0, 0);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const uint64_t dk = sdesc_sw128(sb + SM_KX + b2 * 16384 + i * 2048, 8192, 1024);
-        umma_tmem_a(x.tmem + TM_S, x.tmem + TM_DT + i * 8, dk, ids, 1);
+        umma_tmem_a(x.tmem + TM_S, x.tmem + TM_DELTA + i * 8, dk, ids, 1);
       }
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const uint64_t dp = sdesc_sw128(sb + SM_P + b2 * 8192 + i * 32, 16, 1024);
-        umma_tmem_a(x.tmem + TM_O + b2 * 64, x.tmem + TM_DT + i * 8, dp, idp, 1);
+        umma_tmem_a(x.tmem + TM_O + b2 * 64, x.tmem + TM_DELTA + i * 8, dp, idp, 1);
       }
       umma_commit(&x.bars[B_D2]);
       umma_commit(&x.bars[B_BUF0 + b2]);
+      umma_commit(&x.bars[B_DFREE]);  // Δ^T read: the next U^T may land
       tmark(x, c, 15);
     }
   }
   if (named_sync_and(2, 128, ok && !*x.abort) && x.nchunks > 0) {
-    if (gwait(x, B_D2, d2_ph, 35, 2, 128)) {
+    if (gwait(x, B_D2, d2_ph, 35, GRP_SG)) {
       tc_fence_after();
       if (j == 0) bulk_wait_read0();
       named_sync(2, 128);
@@ -1051,7 +1097,8 @@ __global__ void __launch_bounds__(NTHR, 1)
 
   if (tid == 0) {
     *s_t0 = clock64();
-    for (int i = 0; i < NUM_BARS; ++i) mbar_init(&x.bars[i], 1);
+    for (int i = 0; i < NUM_BARS; ++i)
+      mbar_init(&x.bars[i], (i == B_GC0 || i == B_GC1 || i == B_FR0 || i == B_FR1) ? GRP : 1);
     fence_mbar_init();
     *x.abort = 0;
     prefetch_tmap(&tm_q);
@@ -1070,21 +1117,23 @@ __global__ void __launch_bounds__(NTHR, 1)
   x.tstart = *s_t0;
   const int64_t sbase = ((int64_t)n * H + x.h) * D * D;
 
-  int cnt[2] = {0, 0};  // TMA stages issued (scan group) / consumed (prologue group)
+  int cnt[2] = {0, 0};  // TMA stages issued (scan group) / consumed (front group)
   int* s_cnt = reinterpret_cast<int*>(sm + SM_MISC + MS_CNT);
   if (warp < 4) {
     scan_group(x, &tm_q, &tm_k, &tm_v, &tm_o, init, out, fin, sbase, inject_stuck != 0, cnt);
     if (tid == 0) { s_cnt[0] = cnt[0]; s_cnt[1] = cnt[1]; }
-  } else {
-    prologue_group(x, g, beta, cnt);
+  } else if (warp < 8) {
+    front_group(x, g, beta, cnt);
     if (tid == 128) { s_cnt[2] = cnt[0]; s_cnt[3] = cnt[1]; }
+  } else {
+    back_group(x);
   }
 
   // Drain: every UMMA issued by a group's elected thread has completed, and
   // (on the error path) every TMA load in flight has landed, before TMEM is
   // released and the block exits.
-  if (tid == 0 || tid == 128) {
-    uint64_t* db = &x.bars[tid == 0 ? B_DRAIN_SG : B_DRAIN_PG];
+  if (tid == 0 || tid == 128 || tid == 256) {
+    uint64_t* db = &x.bars[tid == 0 ? B_DRAIN_SG : (tid == 128 ? B_DRAIN_F : B_DRAIN_B)];
     umma_commit(db);
     mbar_wait(db, 0, WAIT_NS);
   }
