@@ -75,14 +75,14 @@ constexpr uint32_t MISC_BYTES = 4096;
 constexpr uint32_t SMEM_BYTES = SM_MISC + MISC_BYTES + 1024;
 
 // misc layout
-// Hand-offs: FULL (TMA -> front), GC (front -> scan: decay totals), FR
-// (front -> back: A tile and operands), AFREE (back -> front: A tile
-// released), PRO (back -> scan: W'^T, U^T), G1 / G23 / D1 / D2 (UMMA
-// completions), BUF (stage and KX/P buffers free), DFREE (Δ^T columns free
+// Hand-offs: FULL (TMA -> front), GC (front -> scan: decay totals), OPS
+// (front -> scan: QE ready), FR (front -> back: A tile and operands), AFREE (back -> front: A tile
+// released), PRO (back -> scan: W'^T, U^T), G1 / G23 / D1A / D1 / D2
+// (UMMA completions), BUF (stage and KX/P buffers free), DFREE (Δ^T columns free
 // for the next U^T), WFREE (W'^T tile free).
 enum Bar {
-  B_FULL0 = 0, B_FULL1, B_G1, B_G23, B_D1, B_D2, B_GC0, B_GC1, B_FR0, B_FR1, B_AFREE, B_PRO0, B_PRO1,
-  B_BUF0, B_BUF1, B_DFREE, B_WFREE, B_DRAIN_F, B_DRAIN_B, B_DRAIN_SG, B_NEVER, NUM_BARS
+  B_FULL0 = 0, B_FULL1, B_G1, B_G23, B_D1A, B_D1, B_D2, B_GC0, B_GC1, B_OPS0, B_OPS1, B_FR0, B_FR1, B_AFREE,
+  B_PRO0, B_PRO1, B_BUF0, B_BUF1, B_DFREE, B_WFREE, B_DRAIN_F, B_DRAIN_B, B_DRAIN_SG, B_NEVER, NUM_BARS
 };
 constexpr uint32_t MS_TMEM = 192, MS_ABORT = 196, MS_FAST = 200, MS_CNT = 208;  // MS_CNT: int[4]
 constexpr uint32_t MS_T0 = 224;  // int64: clock at block start (timing dump)
@@ -157,7 +157,9 @@ __device__ __forceinline__ uint32_t b_off(uint32_t r, uint32_t s) {
 template <int KSTEPS, typename FA, typename FB>
 __device__ __forceinline__ void warp_gemm_tf32x3(float (&d)[4], FA fa, FB fb) {
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-  d[0] = d[1] = d[2] = d[3] = 0.f;
+  // Separate accumulators for the three products keep the dependent chains
+  // KSTEPS long; the small terms are added first.
+  float dhh[4] = {0.f, 0.f, 0.f, 0.f}, dhl[4] = {0.f, 0.f, 0.f, 0.f}, dlh[4] = {0.f, 0.f, 0.f, 0.f};
   float av[KSTEPS][4], bv[KSTEPS][2];
 #pragma unroll
   for (int ks = 0; ks < KSTEPS; ++ks) {  // every fragment load first: one shared-memory latency
@@ -182,10 +184,12 @@ __device__ __forceinline__ void warp_gemm_tf32x3(float (&d)[4], FA fa, FB fb) {
       bh[i] = to_tf32(bv[ks][i]);
       bl[i] = to_tf32(bv[ks][i] - __uint_as_float(bh[i]));
     }
-    mma_tf32_16x8x8(d, al, bh);
-    mma_tf32_16x8x8(d, ah, bl);
-    mma_tf32_16x8x8(d, ah, bh);
+    mma_tf32_16x8x8(dlh, al, bh);
+    mma_tf32_16x8x8(dhl, ah, bl);
+    mma_tf32_16x8x8(dhh, ah, bh);
   }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) d[i] = (dlh[i] + dhl[i]) + dhh[i];
 }
 
 // Bounded wait that also gives up when the other group has aborted.
@@ -424,14 +428,9 @@ __device__ void front_group(const Ctx& x, const float* __restrict__ g, const flo
     volatile int* s_fast = reinterpret_cast<volatile int*>(sm + SM_MISC + MS_FAST) + b2;
 
     if (f == 0) tmark(x, c, 0);
-    // Buffers [b2] were last used by the scan of chunk c-2.
-    if (c >= 2 && !gwait(x, B_BUF0 + b2, ((c >> 1) - 1) & 1, 11, GRP_FRONT)) break;
-    if (!gwait(x, B_FULL0 + b2, (c >> 1) & 1, 12, GRP_FRONT)) break;
-    ++consumed[b2];
-    if (f == 0) tmark(x, c, 1);
-
-    // ---- (a1) decay prefix in log2 units: this thread's 16-row sums, then
-    // the offsets of the earlier row groups and the chunk total G_C.
+    // ---- (a1) decay prefix in log2 units (registers only): this thread's
+    // 16-row sums, then the offsets of the earlier row groups and the chunk
+    // total G_C.
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int m = 0; m < 16; ++m) {
@@ -449,41 +448,50 @@ __device__ void front_group(const Ctx& x, const float* __restrict__ g, const flo
     }
     const bool fast =
         named_sync_and(GRP_FRONT, GRP, fminf(fminf(tot.x, tot.y), fminf(tot.z, tot.w)) >= FAST_MIN_LOG2);
-    if (wq == 0) *reinterpret_cast<float4*>(s_gc + ch0) = ex2_4(tot);
-    if (f == 0) *s_fast = fast ? 1 : 0;
-    if (f < CH) s_beta[f] = bv;
-    if (dmp && wq == 0) {
-      const float LN2 = 0.6931471805599453f;
-      x.dbg[DBG_GC + ch0] = tot.x * LN2; x.dbg[DBG_GC + ch0 + 1] = tot.y * LN2;
-      x.dbg[DBG_GC + ch0 + 2] = tot.z * LN2; x.dbg[DBG_GC + ch0 + 3] = tot.w * LN2;
-    }
-    mbar_arrive(&x.bars[B_GC0 + b2]);  // one arrival per thread, after its own writes
-    if (f == 0) tmark(x, c, 2);
-
-    if (!fast) {
+    if (f == 0) tmark(x, c, 1);
+    // Per-chunk values for the scan and back groups, in buffers [b2] that the
+    // scan of chunk c-2 has released.
+    auto publish = [&]() {
+      if (wq == 0) *reinterpret_cast<float4*>(s_gc + ch0) = ex2_4(tot);
+      if (f == 0) *s_fast = fast ? 1 : 0;
+      if (f < CH) s_beta[f] = bv;
+      if (dmp && wq == 0) {
+        const float LN2 = 0.6931471805599453f;
+        x.dbg[DBG_GC + ch0] = tot.x * LN2; x.dbg[DBG_GC + ch0 + 1] = tot.y * LN2;
+        x.dbg[DBG_GC + ch0 + 2] = tot.z * LN2; x.dbg[DBG_GC + ch0 + 3] = tot.w * LN2;
+      }
+      mbar_arrive(&x.bars[B_GC0 + b2]);  // one arrival per thread, after its own writes
+    };
+    if (!fast) {  // the general Gram writes P[b2] and stages G through the A tile first
+      if (c >= 2 && !gwait(x, B_BUF0 + b2, ((c >> 1) - 1) & 1, 11, GRP_FRONT)) break;
+      publish();
       if (c >= 1 && !gwait(x, B_AFREE, (c - 1) & 1, 13, GRP_FRONT)) break;
-      general_gram(x, b2, valid, gv, off);
     }
+    if (!gwait(x, B_FULL0 + b2, (c >> 1) & 1, 12, GRP_FRONT)) break;
+    ++consumed[b2];
+    if (f == 0) tmark(x, c, 2);
+    if (!fast) general_gram(x, b2, valid, gv, off);
 
     // ---- (a2) operand scaling, row by row: E = e^{G_r - ref} (ref = G_C on
-    // fast chunks, 0 otherwise), H = e^{G_C - G_r};  QE, KE, V (fp16) in
-    // place, KH into KX[b2].
+    // fast chunks, 0 otherwise), H = e^{G_C - G_r}.  QE, KE and V (fp16) go
+    // in place; KH goes to KX[b2] once the scan of chunk c-2 has released it.
+    const float4 ref = fast ? tot : make_float4(0.f, 0.f, 0.f, 0.f);
+    uint8_t* qb = sm + b2 * STAGE_BYTES + OFF_QK + hh * 16384;
+    uint8_t* kb = qb + 8192;
+    uint8_t* vb = sm + b2 * STAGE_BYTES + OFF_V + hh * 8192;
+    uint8_t* khb = sm + SM_KX + b2 * 16384 + hh * 8192;
+    uint2 kraw[16];  // raw K rows, kept for KH
     {
-      const float4 ref = fast ? tot : make_float4(0.f, 0.f, 0.f, 0.f);
       float4 gr = off;
-      uint8_t* qb = sm + b2 * STAGE_BYTES + OFF_QK + hh * 16384;
-      uint8_t* kb = qb + 8192;
-      uint8_t* vb = sm + b2 * STAGE_BYTES + OFF_V + hh * 8192;
-      uint8_t* khb = sm + SM_KX + b2 * 16384 + hh * 8192;
       bool bad = false;
 #pragma unroll
       for (int mb = 0; mb < 16; mb += 4) {
-        uint2 qr[4], kr[4], vr[4];
+        uint2 qr[4], vr[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {  // this batch's loads first, then the in-place stores
           const uint32_t o = sw128_off(16 * wq + mb + i, cc);
           qr[i] = *reinterpret_cast<const uint2*>(qb + o);
-          kr[i] = *reinterpret_cast<const uint2*>(kb + o);
+          kraw[mb + i] = *reinterpret_cast<const uint2*>(kb + o);
           vr[i] = *reinterpret_cast<const uint2*>(vb + o);
         }
 #pragma unroll
@@ -492,21 +500,40 @@ __device__ void front_group(const Ctx& x, const float* __restrict__ g, const flo
           const uint32_t o = sw128_off(r, cc);
           gr.x += gv[m].x; gr.y += gv[m].y; gr.z += gv[m].z; gr.w += gv[m].w;
           const float4 fw = ex2_4(make_float4(gr.x - ref.x, gr.y - ref.y, gr.z - ref.z, gr.w - ref.w));
-          const float4 bw = ex2_4(make_float4(tot.x - gr.x, tot.y - gr.y, tot.z - gr.z, tot.w - gr.w));
-          float4 q4 = bf16x4_to_f32(qr[i]), k4 = bf16x4_to_f32(kr[i]), v4 = bf16x4_to_f32(vr[i]);
-          if (r >= valid) q4 = k4 = v4 = make_float4(0.f, 0.f, 0.f, 0.f);
+          float4 q4 = bf16x4_to_f32(qr[i]), k4 = bf16x4_to_f32(kraw[m]), v4 = bf16x4_to_f32(vr[i]);
+          if (r >= valid) {
+            q4 = k4 = v4 = make_float4(0.f, 0.f, 0.f, 0.f);
+            kraw[m] = make_uint2(0u, 0u);
+          }
           bad |= amax4(v4) > F16_SAFE;
           st_f16x4(qb + o, mul4(q4, fw));
           st_f16x4(kb + o, mul4(k4, fw));
           st_f16x4(vb + o, v4);
-          st_f16x4(khb + o, mul4(k4, bw));
         }
       }
       if (bad) record_error(x.status, KDA_ERR_RANGE, 20);
     }
     fence_proxy_async_smem();
-    named_sync(GRP_FRONT, GRP);
+    mbar_arrive(&x.bars[B_OPS0 + b2]);  // QE is ready for the scan's D1a
     if (f == 0) tmark(x, c, 3);
+    if (fast) {
+      if (c >= 2 && !gwait(x, B_BUF0 + b2, ((c >> 1) - 1) & 1, 11, GRP_FRONT)) break;
+      publish();
+    }
+    if (f == 0) tmark(x, c, 4);
+    {
+      float4 gr = off;
+#pragma unroll
+      for (int m = 0; m < 16; ++m) {
+        const uint32_t o = sw128_off(16 * wq + m, cc);
+        gr.x += gv[m].x; gr.y += gv[m].y; gr.z += gv[m].z; gr.w += gv[m].w;
+        const float4 bw = ex2_4(make_float4(tot.x - gr.x, tot.y - gr.y, tot.z - gr.z, tot.w - gr.w));
+        st_f16x4(khb + o, mul4(bf16x4_to_f32(kraw[m]), bw));
+      }
+    }
+    fence_proxy_async_smem();
+    named_sync(GRP_FRONT, GRP);
+    if (f == 0) tmark(x, c, 5);
 
     if (fast) {
       // ---- G1: [P ; A_raw] = [QE ; KE] . KH^T   (M=128, N=64, K=128)
@@ -524,12 +551,12 @@ __device__ void front_group(const Ctx& x, const float* __restrict__ g, const flo
           }
           umma_commit(&x.bars[B_G1]);
         }
-        tmark(x, c, 4);
+        tmark(x, c, 6);
       }
       if (!gwait(x, B_G1, g1_ph, 15, GRP_FRONT)) break;
       g1_ph ^= 1;
       tc_fence_after();
-      if (f == 0) tmark(x, c, 5);
+      if (f == 0) tmark(x, c, 7);
       float r0[32], r1[32];
       tmem_ld32x2(tl + TM_G, tl + TM_G + 32, r0, r1);  // TMEM lane f: row f of [P ; A_raw]
       if (wq < 2) {  // P row f, lower triangle including the diagonal
@@ -569,7 +596,7 @@ __device__ void front_group(const Ctx& x, const float* __restrict__ g, const flo
     }
     named_sync(GRP_FRONT, GRP);  // the front's TMEM reads are done before the next G1
     mbar_arrive(&x.bars[B_FR0 + b2]);
-    if (f == 0) tmark(x, c, 6);
+    if (f == 0) tmark(x, c, 26);
     load_g(c + 1, gv, bv);
   }
 }
@@ -940,18 +967,26 @@ __device__ void scan_group(const Ctx& x, const void* tmq, const void* tmk, const
     }
     if (j == 0) tmark(x, c, 10);
 
-    // ---- D1: O^T = S'^T QE^T ;  Δ^T = U^T - S'^T W'^T    (A = S'^T from TMEM)
+    // ---- D1a: O^T = S'^T QE^T as soon as QE is ready;  D1b: Δ^T = U^T -
+    // S'^T W'^T once the back group has W'^T and U^T.  (A = S'^T from TMEM)
     if (j == 0) {
-      if (cwait(x, B_PRO0 + b2, (c >> 1) & 1, 33)) {
-        tmark(x, c, 24);
+      bool okj = cwait(x, B_OPS0 + b2, (c >> 1) & 1, 36);
+      if (okj) {
         tc_fence_after();
         const uint32_t idq = idesc_f16_f32(128, 64, 0, 0);
-        const uint32_t idw = idesc_f16_f32(128, 64, 0, 1, 1);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const uint64_t dq = sdesc_sw128(stg + OFF_QK + (i >> 2) * 16384 + (i & 3) * 32, 16, 1024);
           umma_tmem_a(x.tmem + TM_O + b2 * 64, x.tmem + TM_SB + i * 8, dq, idq, i > 0);
         }
+        umma_commit(&x.bars[B_D1A]);
+        tmark(x, c, 27);
+      }
+      okj = okj && cwait(x, B_PRO0 + b2, (c >> 1) & 1, 33);
+      if (okj) {
+        tmark(x, c, 24);
+        tc_fence_after();
+        const uint32_t idw = idesc_f16_f32(128, 64, 0, 1, 1);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const uint64_t dw = sdesc_sw128(sb + SM_WT + i * 2048, 8192, 1024);
@@ -961,6 +996,14 @@ __device__ void scan_group(const Ctx& x, const void* tmq, const void* tmk, const
         umma_commit(&x.bars[B_WFREE]);
       }
       tmark(x, c, 11);
+      // Once D1a has read QE, nothing reads the stage of chunk c any more
+      // (G1, G2 and G3 finished before PRO): fetch chunk c+2 into it.
+      okj = okj && cwait(x, B_D1A, c & 1, 37);
+      if (okj && c + 2 < x.nchunks) {
+        issue_stage(c + 2);
+        ++issued[b2];
+      }
+      tmark(x, c, 28);
     }
     if (c >= 1) store_out(c - 1);
     if (j == 0) tmark(x, c, 12);
@@ -971,11 +1014,6 @@ __device__ void scan_group(const Ctx& x, const void* tmq, const void* tmk, const
     d1_ph ^= 1;
     if (j == 0) tmark(x, c, 13);
     tc_fence_after();
-    // The stage of chunk c is no longer read: fetch chunk c+2 into it.
-    if (j == 0 && c + 2 < x.nchunks) {
-      issue_stage(c + 2);
-      ++issued[b2];
-    }
 
     // ---- Δ^T -> fp16 pairs (A operand of D2); general chunks decay S^T here.
     if (!fast) {
@@ -1098,7 +1136,7 @@ __global__ void __launch_bounds__(NTHR, 1)
   if (tid == 0) {
     *s_t0 = clock64();
     for (int i = 0; i < NUM_BARS; ++i)
-      mbar_init(&x.bars[i], (i == B_GC0 || i == B_GC1 || i == B_FR0 || i == B_FR1) ? GRP : 1);
+      mbar_init(&x.bars[i], (i == B_GC0 || i == B_GC1 || i == B_OPS0 || i == B_OPS1 || i == B_FR0 || i == B_FR1) ? GRP : 1);
     fence_mbar_init();
     *x.abort = 0;
     prefetch_tmap(&tm_q);
