@@ -155,38 +155,56 @@ def time_loop(fn, steps, warmup, stream, dist_ctx):
     t1.record(stream)
     torch.cuda.synchronize()
     dist_ctx.barrier()
-    return dist_ctx.max(t0.elapsed_time(t1) / 1000.0)
+    return t0.elapsed_time(t1) / 1000.0
 
 
 class Dist:
+    """One process per GPU (torchrun env).  The only collectives are the
+    timing barrier and the reductions of the per-rank results: every rank
+    runs its own independent chains, so the data path has no exchange."""
+
     def __init__(self):
         self.world = int(os.environ.get("WORLD_SIZE", "1"))
         self.rank = int(os.environ.get("RANK", "0"))
         self.local = int(os.environ.get("LOCAL_RANK", "0"))
         self.pg = None
+        self.device = "cpu"
 
-    def init(self, backend):
+    def init(self, backend, timeout_s=120):
         if self.world > 1:
             import datetime
             import torch.distributed as dist
-            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s))
             self.pg = dist
+            self.device = "cuda" if backend == "nccl" else "cpu"
 
     def barrier(self):
         if self.pg is not None:
             self.pg.barrier()
 
-    def max(self, x):
+    def _reduce(self, x, op):
         if self.pg is None:
             return x
         import torch
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
-        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        t = torch.tensor([x], dtype=torch.float64, device=self.device)
+        self.pg.all_reduce(t, op=op)
         return float(t.item())
+
+    def max(self, x):
+        return self._reduce(x, self.pg.ReduceOp.MAX if self.pg is not None else None)
+
+    def sum(self, x):
+        return self._reduce(x, self.pg.ReduceOp.SUM if self.pg is not None else None)
 
     def close(self):
         if self.pg is not None:
             self.pg.destroy_process_group()
+
+
+def job_throughput(d, units, seconds):
+    """Whole-job rate: the units every rank processed over the slowest
+    rank's time (seconds is this rank's own device time)."""
+    return d.sum(units) / d.max(seconds)
 
 
 def workload_spec(name):
@@ -281,8 +299,8 @@ def run_native(args, d):
     status = kda.kda_workspace_status(ws, stream)
     if status != kda.KDA_OK:
         raise RuntimeError(f"device status {kda.kda_status_string(status)}")
-    per_step = sec / args.steps
-    value = d.world * th * args.steps / sec / 1e6
+    value = job_throughput(d, th * args.steps, sec) / 1e6
+    per_step = d.max(sec) / args.steps
     bytes_alg = prefill_bytes(th, N * H, dk, dv, io_bytes, init is not None)
     flops_alg = prefill_flops(th, dk, dv)
     achieved = bytes_alg / per_step / 1e9
@@ -301,7 +319,7 @@ def run_native(args, d):
                          "bytes_per_launch": bytes_alg, "kernel": "kda_fwd_tc_kernel",
                          "tensor_tflops": flops_alg / per_step / 1e12,
                          "tensor_frac_of_bf16_peak": flops_alg / per_step / 1e12 / peaks["bf16_tflops"]},
-            "gpu_launches": args.steps, "clocks": clk.summary()}
+            "gpu_launches": args.steps * (2 if (cu is not None and N > 1) else 1), "clocks": clk.summary()}
 
     if not args.no_decode:
         line["decode"] = bench_decode(args, d, dev, stream, peaks, kda, synth)
@@ -330,11 +348,12 @@ def bench_decode(args, d, dev, stream, peaks, kda, synth):
         kda.kda_decode_step(x["q"], x["k"], x["v"], x["g"], x["beta"], state, out=out, stream=stream)
 
     sec = time_loop(step, args.steps, args.warmup, stream, d)
-    per = sec / args.steps
+    value = job_throughput(d, spec.B * spec.H * args.steps, sec) / 1e6
+    per = d.max(sec) / args.steps
     nbytes = decode_bytes(spec.B, spec.H, spec.dk, spec.dv, 2)
     ach = nbytes / per / 1e9
     del xs, state
-    return {"workload": spec.name, "value": d.world * spec.B * spec.H * args.steps / sec / 1e6, "unit": UNIT,
+    return {"workload": spec.name, "value": value, "unit": UNIT,
             "ms_per_step": per * 1e3, "gpu_launches": args.steps,
             "roofline": {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": ach / peaks["hbm_gbs"], "traffic": None, "bytes_per_launch": nbytes,
@@ -353,11 +372,12 @@ def bench_e2e(args, d, dev, stream, inp, kda, th):
         o, f, _ = kda.kda_fwd_host(host["q"], host["k"], host["v"], host["g"], host["beta"], host["init_state"],
                                    host["cu_seqlens"], device=dev, stream=stream, dev_buffers=bufs)
 
-    sec = time_loop(step, steps, 1, stream, d)
+    sec = time_loop(step, steps, args.warmup, stream, d)
     h2d = sum(t.numel() * t.element_size() for n, t in host.items() if t is not None)
     d2h = bufs["out_h"].numel() * bufs["out_h"].element_size() + bufs["fin_h"].numel() * 4
-    return {"value": d.world * th * steps / sec / 1e6, "unit": UNIT, "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "steps": steps, "ms_per_step": sec / steps * 1e3}
+    value = job_throughput(d, th * steps, sec) / 1e6
+    return {"value": value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": steps, "ms_per_step": d.max(sec) / steps * 1e3}
 
 
 def main():
