@@ -25,7 +25,9 @@
 //
 // Operands are fp16 (10-bit mantissa) with fp32 accumulation: the fp32
 // state and every product stay accurate to well inside the bf16 output's own
-// rounding.  Values that would not fit fp16 set KDA_ERR_RANGE.
+// rounding.  Values that would not fit fp16 set KDA_ERR_RANGE: every
+// operand overflow (V, S', W', the Gram tiles) reaches Δ as inf or NaN, so
+// the range test is made once, on Δ, with a NaN-propagating maximum.
 //
 // Work split (one CTA per (sequence, head) chain, chunks in order), three
 // groups of four warps:
@@ -114,16 +116,11 @@ constexpr int TIME_CHUNKS = 64;
 // Shared-memory accesses are plain C++ through pointers derived from the
 // shared array (so they compile to shared loads/stores and the compiler may
 // schedule them freely between barriers).
-__device__ __forceinline__ float4 ld_bf16x4(const uint8_t* p) {
-  const uint2 u = *reinterpret_cast<const uint2*>(p);
-  const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
-  const float2 y = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
-  return make_float4(x.x, x.y, y.x, y.y);
-}
+// Four bf16 (two packed words, element 0 in the low half) to fp32: a bf16 is
+// the upper half of the fp32 with the same value.
 __device__ __forceinline__ float4 bf16x4_to_f32(uint2 u) {
-  const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
-  const float2 y = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
-  return make_float4(x.x, x.y, y.x, y.y);
+  return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u),
+                     __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xffff0000u));
 }
 __device__ __forceinline__ float ld_bf16(const uint8_t* p) {
   return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(p));
@@ -135,13 +132,28 @@ __device__ __forceinline__ void st_f16x8(uint8_t* p, const float* v) {
   *reinterpret_cast<uint4*>(p) = make_uint4(pack_f16x2(v[0], v[1]), pack_f16x2(v[2], v[3]), pack_f16x2(v[4], v[5]),
                                             pack_f16x2(v[6], v[7]));
 }
+// Elementwise float4 arithmetic on the paired fp32 pipe (two lanes per instruction).
 __device__ __forceinline__ float4 mul4(float4 a, float4 b) {
-  return make_float4(a.x * b.x, a.y * b.y, a.z * b.z, a.w * b.w);
+  const float2 lo = __fmul2_rn(make_float2(a.x, a.y), make_float2(b.x, b.y));
+  const float2 hi = __fmul2_rn(make_float2(a.z, a.w), make_float2(b.z, b.w));
+  return make_float4(lo.x, lo.y, hi.x, hi.y);
+}
+__device__ __forceinline__ float4 add4(float4 a, float4 b) {
+  const float2 lo = __fadd2_rn(make_float2(a.x, a.y), make_float2(b.x, b.y));
+  const float2 hi = __fadd2_rn(make_float2(a.z, a.w), make_float2(b.z, b.w));
+  return make_float4(lo.x, lo.y, hi.x, hi.y);
+}
+__device__ __forceinline__ float4 sub4(float4 a, float4 b) {
+  return add4(a, make_float4(-b.x, -b.y, -b.z, -b.w));
+}
+// max(|m|, |x|), propagating NaN (the sign of the result is not meaningful):
+// the fp16 range test of a tensor-core operand, one instruction per element.
+__device__ __forceinline__ float amax_nan(float m, float x) {
+  float r;
+  asm("max.NaN.xorsign.abs.f32 %0, %1, %2;" : "=f"(r) : "f"(m), "f"(x));
+  return r;
 }
 __device__ __forceinline__ float4 ex2_4(float4 a) { return make_float4(ex2(a.x), ex2(a.y), ex2(a.z), ex2(a.w)); }
-__device__ __forceinline__ float amax4(float4 a) {
-  return fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(a.z), fabsf(a.w)));
-}
 // fp32 [64][64] with 16-byte units XOR-swizzled by row.
 __device__ __forceinline__ uint32_t a_off(uint32_t r, uint32_t s) {
   return r * 256u + ((s >> 2) ^ (r & 7u)) * 16u + (s & 3u) * 4u;
@@ -480,10 +492,25 @@ __device__ void front_group(const Ctx& x, const float* __restrict__ g, const flo
     uint8_t* kb = qb + 8192;
     uint8_t* vb = sm + b2 * STAGE_BYTES + OFF_V + hh * 8192;
     uint8_t* khb = sm + SM_KX + b2 * 16384 + hh * 8192;
+    if (valid < CH) {
+      // Rows past the end of a sequence's last chunk hold other data: zero
+      // this thread's rows and channels of the raw tiles, so the scaling
+      // pass below needs no per-row mask.
+#pragma unroll 1
+      for (int m = 0; m < 16; ++m) {
+        const int r = 16 * wq + m;
+        if (r >= valid) {
+          const uint32_t o = sw128_off(r, cc);
+          *reinterpret_cast<uint2*>(qb + o) = make_uint2(0u, 0u);
+          *reinterpret_cast<uint2*>(kb + o) = make_uint2(0u, 0u);
+          *reinterpret_cast<uint2*>(vb + o) = make_uint2(0u, 0u);
+        }
+      }
+    }
     uint2 kraw[16];  // raw K rows, kept for KH
     {
+      const float4 nref = fast ? make_float4(-tot.x, -tot.y, -tot.z, -tot.w) : make_float4(0.f, 0.f, 0.f, 0.f);
       float4 gr = off;
-      bool bad = false;
 #pragma unroll
       for (int mb = 0; mb < 16; mb += 4) {
         uint2 qr[4], vr[4];
@@ -496,22 +523,15 @@ __device__ void front_group(const Ctx& x, const float* __restrict__ g, const flo
         }
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const int m = mb + i, r = 16 * wq + m;
-          const uint32_t o = sw128_off(r, cc);
-          gr.x += gv[m].x; gr.y += gv[m].y; gr.z += gv[m].z; gr.w += gv[m].w;
-          const float4 fw = ex2_4(make_float4(gr.x - ref.x, gr.y - ref.y, gr.z - ref.z, gr.w - ref.w));
-          float4 q4 = bf16x4_to_f32(qr[i]), k4 = bf16x4_to_f32(kraw[m]), v4 = bf16x4_to_f32(vr[i]);
-          if (r >= valid) {
-            q4 = k4 = v4 = make_float4(0.f, 0.f, 0.f, 0.f);
-            kraw[m] = make_uint2(0u, 0u);
-          }
-          bad |= amax4(v4) > F16_SAFE;
-          st_f16x4(qb + o, mul4(q4, fw));
-          st_f16x4(kb + o, mul4(k4, fw));
-          st_f16x4(vb + o, v4);
+          const int m = mb + i;
+          const uint32_t o = sw128_off(16 * wq + m, cc);
+          gr = add4(gr, gv[m]);
+          const float4 fw = ex2_4(add4(gr, nref));
+          st_f16x4(qb + o, mul4(bf16x4_to_f32(qr[i]), fw));
+          st_f16x4(kb + o, mul4(bf16x4_to_f32(kraw[m]), fw));
+          st_f16x4(vb + o, bf16x4_to_f32(vr[i]));
         }
       }
-      if (bad) record_error(x.status, KDA_ERR_RANGE, 20);
     }
     fence_proxy_async_smem();
     mbar_arrive(&x.bars[B_OPS0 + b2]);  // QE is ready for the scan's D1a
@@ -526,9 +546,8 @@ __device__ void front_group(const Ctx& x, const float* __restrict__ g, const flo
 #pragma unroll
       for (int m = 0; m < 16; ++m) {
         const uint32_t o = sw128_off(16 * wq + m, cc);
-        gr.x += gv[m].x; gr.y += gv[m].y; gr.z += gv[m].z; gr.w += gv[m].w;
-        const float4 bw = ex2_4(make_float4(tot.x - gr.x, tot.y - gr.y, tot.z - gr.z, tot.w - gr.w));
-        st_f16x4(khb + o, mul4(bf16x4_to_f32(kraw[m]), bw));
+        gr = add4(gr, gv[m]);
+        st_f16x4(khb + o, mul4(bf16x4_to_f32(kraw[m]), ex2_4(sub4(tot, gr))));
       }
     }
     fence_proxy_async_smem();
@@ -773,10 +792,6 @@ __device__ void back_group(const Ctx& x) {
     {  // lane ti holds W'^T[ti][r]: row ti of the MN-major B operand of D1
       float w0[32], w1[32];
       tmem_ld32x2(tl + TM_W, tl + TM_W + 32, w0, w1);
-      float mx = 0.f;
-#pragma unroll
-      for (int i = 0; i < 32; ++i) mx = fmaxf(mx, fmaxf(fabsf(w0[i]), fabsf(w1[i])));
-      if (!(mx <= F16_SAFE)) record_error(x.status, KDA_ERR_RANGE, 21);
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         st_f16x8(sm + SM_WT + ti * 128 + (((q ^ ti) & 7) << 4), w0 + 8 * q);
@@ -929,7 +944,6 @@ __device__ void scan_group(const Ctx& x, const void* tmq, const void* tmk, const
       break;
     }
     const bool fast = *reinterpret_cast<volatile int*>(sm + SM_MISC + MS_FAST + 4 * b2) != 0;
-    float mx = 0.f;
 #pragma unroll
     for (int cp = 0; cp < 2; ++cp) {
       float s0[32], s1[32];
@@ -937,27 +951,24 @@ __device__ void scan_group(const Ctx& x, const void* tmq, const void* tmk, const
       tmem_ld32x2(tl + TM_S + cp * 64, tl + TM_S + cp * 64 + 32, s0, s1);
       if (fast) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          s0[i] *= s_gc[cp * 64 + i];
-          s1[i] *= s_gc[cp * 64 + 32 + i];
+        for (int i = 0; i < 32; i += 4) {
+          const float4 g0 = *reinterpret_cast<const float4*>(s_gc + cp * 64 + i);
+          const float4 g1 = *reinterpret_cast<const float4*>(s_gc + cp * 64 + 32 + i);
+          const float4 a = mul4(make_float4(s0[i], s0[i + 1], s0[i + 2], s0[i + 3]), g0);
+          const float4 b = mul4(make_float4(s1[i], s1[i + 1], s1[i + 2], s1[i + 3]), g1);
+          s0[i] = a.x; s0[i + 1] = a.y; s0[i + 2] = a.z; s0[i + 3] = a.w;
+          s1[i] = b.x; s1[i + 1] = b.y; s1[i + 2] = b.z; s1[i + 3] = b.w;
         }
         tmem_st32(tl + TM_S + cp * 64, s0);
         tmem_st32(tl + TM_S + cp * 64 + 32, s1);
       }
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        pk[i] = pack_f16x2(s0[2 * i], s0[2 * i + 1]);
-        mx = fmaxf(mx, fmaxf(fabsf(s0[2 * i]), fabsf(s0[2 * i + 1])));
-      }
+      for (int i = 0; i < 16; ++i) pk[i] = pack_f16x2(s0[2 * i], s0[2 * i + 1]);
       tmem_st16(tl + TM_SB + cp * 32, pk);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        pk[i] = pack_f16x2(s1[2 * i], s1[2 * i + 1]);
-        mx = fmaxf(mx, fmaxf(fabsf(s1[2 * i]), fabsf(s1[2 * i + 1])));
-      }
+      for (int i = 0; i < 16; ++i) pk[i] = pack_f16x2(s1[2 * i], s1[2 * i + 1]);
       tmem_st16(tl + TM_SB + cp * 32 + 16, pk);
     }
-    if (!(mx <= F16_SAFE)) record_error(x.status, KDA_ERR_RANGE, 30);
     if (j == 0) bulk_wait_read0();  // the staging tile is free again
     tmem_wait_st();
     tc_fence_before();
@@ -1035,16 +1046,16 @@ __device__ void scan_group(const Ctx& x, const void* tmq, const void* tmk, const
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         pk[i] = pack_f16x2(d0[2 * i], d0[2 * i + 1]);
-        dm = fmaxf(dm, fmaxf(fabsf(d0[2 * i]), fabsf(d0[2 * i + 1])));
+        dm = amax_nan(amax_nan(dm, d0[2 * i]), d0[2 * i + 1]);
       }
       tmem_st16(tl + TM_DELTA, pk);
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         pk[i] = pack_f16x2(d1[2 * i], d1[2 * i + 1]);
-        dm = fmaxf(dm, fmaxf(fabsf(d1[2 * i]), fabsf(d1[2 * i + 1])));
+        dm = amax_nan(amax_nan(dm, d1[2 * i]), d1[2 * i + 1]);
       }
       tmem_st16(tl + TM_DELTA + 16, pk);
-      if (!(dm <= F16_SAFE)) record_error(x.status, KDA_ERR_RANGE, 31);
+      if (!(fabsf(dm) <= F16_SAFE)) record_error(x.status, KDA_ERR_RANGE, 31);
     }
     tmem_wait_st();
     tc_fence_before();

@@ -167,3 +167,21 @@ def test_timeout_path_reports_status_and_context_survives():
     assert kda.kda_workspace_status(ws) == kda.KDA_OK
     o_ref, f_ref = run_oracle(inp)
     assert_close(out, o_ref, torch.bfloat16, "after timeout")
+
+
+@pytest.mark.parametrize("what", ["v", "state"])
+def test_fp16_range_overflow_is_reported(what):
+    """Values beyond the fp16 range of the tensor-core operands (a huge v, or
+    a huge initial state) are reported as KDA_ERR_RANGE in the status word;
+    the next call on the same workspace starts clean."""
+    inp = synth.make_prefill(synth.MID, DEV, T=192, B=1, H=2)
+    ws = kda.alloc_workspace(1, 192, 2, 128, 128)
+    args = {k: v for k, v in inp.items()}
+    if what == "v":
+        args["v"] = (inp["v"].float() * 1e6).to(torch.bfloat16)
+    else:
+        args["init_state"] = inp["init_state"] * 1e9
+    kda.kda_fwd(args["q"], args["k"], args["v"], args["g"], args["beta"], args["init_state"], workspace=ws)
+    assert kda.kda_workspace_status(ws) == kda.KDA_ERR_RANGE
+    kda.kda_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["init_state"], workspace=ws)
+    assert kda.kda_workspace_status(ws) == kda.KDA_OK
