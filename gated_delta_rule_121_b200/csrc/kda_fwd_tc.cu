@@ -164,7 +164,10 @@ __device__ __forceinline__ uint32_t b_off(uint32_t r, uint32_t s) {
 }
 // One 16x8 tile of D = sign * A B with fp32 operands held in shared memory,
 // K = 8 * KSTEPS, computed on the warp-level tensor path as three tf32
-// products (hi*hi + hi*lo + lo*hi), which keeps close to fp32 accuracy.
+// products (hi*hi + hi*lo + lo*hi), which keeps close to fp32 accuracy.  hi
+// is x with its low 13 mantissa bits cleared (exactly a tf32 value); lo = x -
+// hi is exact in fp32 and the MMA reads its leading 10 mantissa bits, so the
+// dropped part is below 2^-21 |x|.
 // fa(r, k) / fb(k, n) return the operand element addresses.
 template <int KSTEPS, typename FA, typename FB>
 __device__ __forceinline__ void warp_gemm_tf32x3(float (&d)[4], FA fa, FB fb) {
@@ -188,13 +191,13 @@ __device__ __forceinline__ void warp_gemm_tf32x3(float (&d)[4], FA fa, FB fb) {
     uint32_t ah[4], al[4], bh[2], bl[2];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      ah[i] = to_tf32(av[ks][i]);
-      al[i] = to_tf32(av[ks][i] - __uint_as_float(ah[i]));
+      ah[i] = __float_as_uint(av[ks][i]) & 0xffffe000u;
+      al[i] = __float_as_uint(av[ks][i] - __uint_as_float(ah[i]));
     }
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
-      bh[i] = to_tf32(bv[ks][i]);
-      bl[i] = to_tf32(bv[ks][i] - __uint_as_float(bh[i]));
+      bh[i] = __float_as_uint(bv[ks][i]) & 0xffffe000u;
+      bl[i] = __float_as_uint(bv[ks][i] - __uint_as_float(bh[i]));
     }
     mma_tf32_16x8x8(dlh, al, bh);
     mma_tf32_16x8x8(dhl, ah, bl);
@@ -376,7 +379,7 @@ __device__ __noinline__ void dump_pa(float* dbg, const uint8_t* sm, int b2, int 
     const int r = e >> 6, s = e & 63;
     const uint16_t u = *reinterpret_cast<const uint16_t*>(sm + SM_P + b2 * 8192 + sw128_off(r, s));
     dbg[DBG_P + e] = __half2float(*reinterpret_cast<const __half*>(&u));
-    dbg[DBG_A + e] = *reinterpret_cast<const float*>(sm + SM_A + a_off(r, s));
+    dbg[DBG_A + e] = s < r ? *reinterpret_cast<const float*>(sm + SM_A + a_off(r, s)) : 0.f;
   }
 }
 __device__ __noinline__ void dump_t(float* dbg, const uint8_t* sm, int p) {
@@ -444,10 +447,11 @@ __device__ void front_group(const Ctx& x, const float* __restrict__ g, const flo
     // 16-row sums, then the offsets of the earlier row groups and the chunk
     // total G_C.
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    const float4 l2e = make_float4(LOG2E, LOG2E, LOG2E, LOG2E);
 #pragma unroll
     for (int m = 0; m < 16; ++m) {
-      gv[m] = make_float4(gv[m].x * LOG2E, gv[m].y * LOG2E, gv[m].z * LOG2E, gv[m].w * LOG2E);
-      acc.x += gv[m].x; acc.y += gv[m].y; acc.z += gv[m].z; acc.w += gv[m].w;
+      gv[m] = mul4(gv[m], l2e);
+      acc = add4(acc, gv[m]);
     }
     *reinterpret_cast<float4*>(s_red + wq * 128 + ch0) = acc;
     named_sync(GRP_FRONT, GRP);
@@ -590,20 +594,15 @@ __device__ void front_group(const Ctx& x, const float* __restrict__ g, const flo
           st_f16x8(sm + SM_P + b2 * 8192 + r * 128 + (((k ^ r) & 7) << 4), r0 + 8 * k);
           st_f16x8(sm + SM_P + b2 * 8192 + r * 128 + ((((4 + k) ^ r) & 7) << 4), r1 + 8 * k);
         }
-      } else {  // A row r = beta_r (KE KH^T)_rs, strictly lower
+      } else {  // A row r = beta_r (KE KH^T)_rs; the solve reads only its strictly lower part
         const int r = f - CH;
-        const float b = s_beta[r];
-#pragma unroll
-        for (int s = 0; s < 32; ++s) {
-          r0[s] = s < r ? b * r0[s] : 0.f;
-          r1[s] = 32 + s < r ? b * r1[s] : 0.f;
-        }
+        const float4 b = make_float4(s_beta[r], s_beta[r], s_beta[r], s_beta[r]);
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
           *reinterpret_cast<float4*>(sm + SM_A + a_off(r, 4 * u)) =
-              make_float4(r0[4 * u], r0[4 * u + 1], r0[4 * u + 2], r0[4 * u + 3]);
+              mul4(make_float4(r0[4 * u], r0[4 * u + 1], r0[4 * u + 2], r0[4 * u + 3]), b);
           *reinterpret_cast<float4*>(sm + SM_A + a_off(r, 32 + 4 * u)) =
-              make_float4(r1[4 * u], r1[4 * u + 1], r1[4 * u + 2], r1[4 * u + 3]);
+              mul4(make_float4(r1[4 * u], r1[4 * u + 1], r1[4 * u + 2], r1[4 * u + 3]), b);
         }
       }
       tc_fence_before();
@@ -644,29 +643,24 @@ __device__ void back_group(const Ctx& x) {
     // the 32x32 diagonal inverses; T_10 = -D_1 (A_10 D_0).
     // T' = T diag(beta) as fp16 [r][s] in the TP tile.
     if (k < 64) {
-      // Column sweep: once x[s] is final it updates every later row.  The
-      // loads do not depend on x, so the dependency chain is one FMA per
-      // column; column s+1 is fetched while column s is applied.
+      // Forward substitution down the rows of diagonal block a (thread:
+      // column jj of its inverse): x[r] = [r == jj] - sum_{s<r} A[r][s] x[s].
+      // The A rows are float4 loads that do not depend on x; only the
+      // strictly lower entries are read.
       const int a = k >> 4, jj = k & 15;
-      auto ael = [&](int r, int cl) {
-        return *reinterpret_cast<const float*>(sm + SM_A + a_off(16 * a + r, 16 * a + cl));
-      };
-      float xs[16], col[16], nxt[16];
+      float xs[16];
 #pragma unroll
       for (int r = 0; r < 16; ++r) {
-        xs[r] = (r == jj) ? 1.f : 0.f;
-        col[r] = r >= 1 ? ael(r, 0) : 0.f;
-      }
+        float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
-      for (int sc = 0; sc < 15; ++sc) {
-#pragma unroll
-        for (int r = 0; r < 16; ++r) nxt[r] = (sc + 1 < 15 && r >= sc + 2) ? ael(r, sc + 1) : 0.f;
-        const float xsc = xs[sc];
-#pragma unroll
-        for (int r = 0; r < 16; ++r)
-          if (r > sc) xs[r] -= col[r] * xsc;
-#pragma unroll
-        for (int r = 0; r < 16; ++r) col[r] = nxt[r];
+        for (int u = 0; u < (r + 3) / 4; ++u) {
+          const float4 a4 = *reinterpret_cast<const float4*>(sm + SM_A + a_off(16 * a + r, 16 * a + 4 * u));
+          acc0 = fmaf(a4.x, xs[4 * u], acc0);
+          if (4 * u + 1 < r) acc1 = fmaf(a4.y, xs[4 * u + 1], acc1);
+          if (4 * u + 2 < r) acc0 = fmaf(a4.z, xs[4 * u + 2], acc0);
+          if (4 * u + 3 < r) acc1 = fmaf(a4.w, xs[4 * u + 3], acc1);
+        }
+        xs[r] = ((r == jj) ? 1.f : 0.f) - (acc0 + acc1);
       }
       // E_a -> diagonal 16x16 block of D_{a/2}
       const uint32_t db = SM_DG + (a >> 1) * 4096;
@@ -890,12 +884,19 @@ __device__ void scan_group(const Ctx& x, const void* tmq, const void* tmk, const
     const int64_t tok0 = x.t0 + (int64_t)c * CH;
     float o0[32], o1[32];
     tmem_ld32x2(tl + TM_O + (c & 1) * 64, tl + TM_O + (c & 1) * 64 + 32, o0, o1);
+    // Lanes j and j^1 hold channels jc, jc+1 of every token; they swap one
+    // value per token pair so that each writes both channels of one token
+    // (the even lane the even token) as one 4-byte word.
+    const int odd = j & 1, jc = j & ~1;
+    uint8_t* ost = sm + SM_OST + (jc >> 6) * 8192;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      *reinterpret_cast<__nv_bfloat16*>(sm + SM_OST + (j >> 6) * 8192 + sw128_off(i, j & 63)) =
-          __float2bfloat16_rn(o0[i]);
-      *reinterpret_cast<__nv_bfloat16*>(sm + SM_OST + (j >> 6) * 8192 + sw128_off(32 + i, j & 63)) =
-          __float2bfloat16_rn(o1[i]);
+    for (int t = 0; t < 16; ++t) {
+      const float s0 = odd ? o0[2 * t] : o0[2 * t + 1], s1 = odd ? o1[2 * t] : o1[2 * t + 1];
+      const float r0 = __shfl_xor_sync(0xffffffffu, s0, 1), r1 = __shfl_xor_sync(0xffffffffu, s1, 1);
+      const uint32_t w0 = odd ? pack_bf16x2(r0, o0[2 * t + 1]) : pack_bf16x2(o0[2 * t], r0);
+      const uint32_t w1 = odd ? pack_bf16x2(r1, o1[2 * t + 1]) : pack_bf16x2(o1[2 * t], r1);
+      *reinterpret_cast<uint32_t*>(ost + sw128_off(2 * t + odd, jc & 63)) = w0;
+      *reinterpret_cast<uint32_t*>(ost + sw128_off(32 + 2 * t + odd, jc & 63)) = w1;
     }
     fence_proxy_async_smem();
     named_sync(2, 128);

@@ -255,12 +255,6 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// fp32 -> tf32 (round to nearest, ties away), returned as the fp32 bit pattern.
-__device__ __forceinline__ uint32_t to_tf32(float x) {
-  uint32_t r;
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-  return r;
-}
 // Warp-level D(16x8) += A(16x8) * B(8x8), tf32 inputs, fp32 accumulators
 // (mma.sync m16n8k8).  Fragment ownership (g = lane/4, t = lane%4):
 // a = {A[g][t], A[g+8][t], A[g][t+4], A[g+8][t+4]}, b = {B[t][g], B[t+4][g]},
