@@ -73,7 +73,7 @@ constexpr uint32_t SM_T10 = SM_X + 4096;     // T_10 fp32 [32][32]            4 
 constexpr uint32_t SM_TP = SM_X;             // T' fp16 [64][64] over X, T_10  8 KB
 constexpr uint32_t SM_OST = SM_T10 + 4096 + 4096;  // O staging bf16 [64][128] 16 KB (1024-aligned)
 constexpr uint32_t SM_MISC = SM_OST + 16384;
-constexpr uint32_t MISC_BYTES = 4096;
+constexpr uint32_t MISC_BYTES = 8192;
 constexpr uint32_t SMEM_BYTES = SM_MISC + MISC_BYTES + 1024;
 
 // misc layout
@@ -90,8 +90,8 @@ constexpr uint32_t MS_TMEM = 192, MS_ABORT = 196, MS_FAST = 200, MS_CNT = 208;  
 constexpr uint32_t MS_T0 = 224;  // int64: clock at block start (timing dump)
 constexpr uint32_t MS_BETA = 256;    // [2][64] fp32
 constexpr uint32_t MS_GC = 768;      // [2][128] fp32: exp(G_C)
-constexpr uint32_t MS_RED = 1792;    // [4][128] fp32 log2 sums
-constexpr uint32_t MS_END = 3840;
+constexpr uint32_t MS_RED = 1792;    // [8][128] fp32 log2 sums
+constexpr uint32_t MS_END = 5888;
 static_assert(NUM_BARS * 8 <= MS_TMEM, "barrier area");
 static_assert(MS_END <= MISC_BYTES, "misc area");
 
@@ -154,6 +154,40 @@ __device__ __forceinline__ float amax_nan(float m, float x) {
   return r;
 }
 __device__ __forceinline__ float4 ex2_4(float4 a) { return make_float4(ex2(a.x), ex2(a.y), ex2(a.z), ex2(a.w)); }
+// Eight consecutive channels of one row (the front group's unit of work).
+struct F8 {
+  float4 a, b;
+};
+__device__ __forceinline__ F8 f8(float v) { return {make_float4(v, v, v, v), make_float4(v, v, v, v)}; }
+__device__ __forceinline__ F8 add8(F8 x, F8 y) { return {add4(x.a, y.a), add4(x.b, y.b)}; }
+__device__ __forceinline__ F8 sub8(F8 x, F8 y) { return {sub4(x.a, y.a), sub4(x.b, y.b)}; }
+__device__ __forceinline__ F8 mul8(F8 x, F8 y) { return {mul4(x.a, y.a), mul4(x.b, y.b)}; }
+__device__ __forceinline__ F8 ex2_8(F8 x) { return {ex2_4(x.a), ex2_4(x.b)}; }
+__device__ __forceinline__ F8 bf16x8_to_f32(uint4 u) {
+  return {bf16x4_to_f32(make_uint2(u.x, u.y)), bf16x4_to_f32(make_uint2(u.z, u.w))};
+}
+__device__ __forceinline__ void st_f16x8(uint8_t* p, F8 v) {
+  *reinterpret_cast<uint4*>(p) = make_uint4(pack_f16x2(v.a.x, v.a.y), pack_f16x2(v.a.z, v.a.w),
+                                            pack_f16x2(v.b.x, v.b.y), pack_f16x2(v.b.z, v.b.w));
+}
+__device__ __forceinline__ float min8(F8 x) {
+  return fminf(fminf(fminf(x.a.x, x.a.y), fminf(x.a.z, x.a.w)), fminf(fminf(x.b.x, x.b.y), fminf(x.b.z, x.b.w)));
+}
+// 32 bytes of read-only global data: one 256-bit load when the address is
+// 32-byte aligned, else two 128-bit loads.
+__device__ __forceinline__ F8 ldg8(const float* p, bool v8) {
+  F8 r;
+  if (v8) {
+    asm volatile("ld.global.nc.v8.f32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=f"(r.a.x), "=f"(r.a.y), "=f"(r.a.z), "=f"(r.a.w), "=f"(r.b.x), "=f"(r.b.y), "=f"(r.b.z),
+                   "=f"(r.b.w)
+                 : "l"(p));
+  } else {
+    r.a = __ldg(reinterpret_cast<const float4*>(p));
+    r.b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  }
+  return r;
+}
 // fp32 [64][64] with 16-byte units XOR-swizzled by row.
 __device__ __forceinline__ uint32_t a_off(uint32_t r, uint32_t s) {
   return r * 256u + ((s >> 2) ^ (r & 7u)) * 16u + (s & 3u) * 4u;
@@ -288,19 +322,18 @@ __device__ __forceinline__ int chunk_valid(const Ctx& x, int c) {
 //   front (warps 4-7): decay prefix fused with operand scaling, the G1 Gram
 //     UMMA, and the P / A tiles;
 //   back (warps 8-11): the triangular solve, T', the G2/G3 UMMAs and W'^T.
-// Row-wise front work: thread f (warp wq = f / 32, lane) owns rows
-// 16 wq .. 16 wq + 15 and channels 4 lane .. 4 lane + 3.  TMEM work: a warp
-// reads the lane quarter (warp index mod 4) it is allowed to access.
+// Row-wise front work: thread f owns rows 8 (f / 16) .. + 7 and channels
+// 8 (f % 16) .. + 7, so every tile access is 16 bytes wide.  TMEM work: a
+// warp reads the lane quarter (warp index mod 4) it is allowed to access.
 constexpr int GRP = 128;  // threads per group
 
 // General chunks: P and A on CUDA cores from the exact decay differences
 // G_r - G_s (log2 units), G staged through the A tile one channel half at a
 // time (the back group has released the A tile).  Raw Q and K are read from
 // the stage before they are rescaled in place.
-__device__ __forceinline__ void general_gram(const Ctx& x, int b2, int valid, const float4 (&gv)[16], float4 off) {
+__device__ __forceinline__ void general_gram(const Ctx& x, int b2, int valid, const F8 (&gv)[8]) {
   const int f = threadIdx.x - 128;
-  const int wq = f >> 5, lane = f & 31;
-  const int ch0 = 4 * lane, hh = ch0 >> 6, cc = ch0 & 63;
+  const int rg = f >> 4, ch0 = 8 * (f & 15), hh = ch0 >> 6, cc = ch0 & 63;
   uint8_t* sm = x.sm;
   const float* s_beta = reinterpret_cast<const float*>(sm + SM_MISC + MS_BETA) + b2 * 64;
   const int r = f & 63;
@@ -316,11 +349,12 @@ __device__ __forceinline__ void general_gram(const Ctx& x, int b2, int valid, co
     for (int half = 0; half < 2; ++half) {
       named_sync(GRP_FRONT, GRP);  // earlier readers of the staging tile are done
       if (hh == half) {
-        float4 gr = off;
+        F8 gr = f8(0.f);
 #pragma unroll
-        for (int m = 0; m < 16; ++m) {
-          gr.x += gv[m].x; gr.y += gv[m].y; gr.z += gv[m].z; gr.w += gv[m].w;
-          *reinterpret_cast<float4*>(sm + SM_A + (16 * wq + m) * 256 + cc * 4) = gr;
+        for (int m = 0; m < 8; ++m) {
+          gr = add8(gr, gv[m]);
+          *reinterpret_cast<float4*>(sm + SM_A + (8 * rg + m) * 256 + cc * 4) = gr.a;
+          *reinterpret_cast<float4*>(sm + SM_A + (8 * rg + m) * 256 + cc * 4 + 16) = gr.b;
         }
       }
       named_sync(GRP_FRONT, GRP);
@@ -405,30 +439,36 @@ __device__ __noinline__ void dump_wu(float* dbg, const uint8_t* sm, uint32_t tme
 }
 
 __device__ void front_group(const Ctx& x, const float* __restrict__ g, const float* __restrict__ beta,
-                            int (&consumed)[2]) {
+                            const void* tmg, int (&consumed)[2]) {
   const int f = threadIdx.x - 128;  // 0..127
-  const int wq = f >> 5, lane = f & 31;
-  const int ch0 = 4 * lane, hh = ch0 >> 6, cc = ch0 & 63;
+  const int wq = f >> 5;                                    // warp: TMEM lane quarter
+  const int rg = f >> 4, ch0 = 8 * (f & 15), hh = ch0 >> 6, cc = ch0 & 63;
   const uint32_t tl = x.tmem + ((uint32_t)(wq * 32) << 16);
   uint8_t* sm = x.sm;
   const uint32_t sb = x.sb;
-  float* s_red = reinterpret_cast<float*>(sm + SM_MISC + MS_RED);  // [4][128] log2 sums
+  float* s_red = reinterpret_cast<float*>(sm + SM_MISC + MS_RED);  // [8][128] log2 sums
   const int H = x.H;
+  const bool g32 = (reinterpret_cast<uintptr_t>(g) & 31u) == 0;
 
-  // Register prefetch of this thread's g rows (16 x float4) and of beta.
-  auto load_g = [&](int c, float4(&gv)[16], float& bv) {
+  // Register prefetch of this thread's g rows (8 rows x 8 channels) and of beta.
+  auto load_g = [&](int c, F8(&gv)[8], float& bv) {
     const int valid = c < x.nchunks ? chunk_valid(x, c) : 0;
     const int64_t tok0 = x.t0 + (int64_t)c * CH;
 #pragma unroll
-    for (int m = 0; m < 16; ++m) {
-      const int r = 16 * wq + m;
-      gv[m] = r < valid ? __ldg(reinterpret_cast<const float4*>(g + ((tok0 + r) * H + x.h) * D + ch0))
-                        : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int m = 0; m < 8; ++m) {
+      const int r = 8 * rg + m;
+      gv[m] = r < valid ? ldg8(g + ((tok0 + r) * H + x.h) * D + ch0, g32) : f8(0.f);
     }
     bv = (f < CH && f < valid) ? __ldg(beta + (tok0 + f) * H + x.h) : 0.f;
   };
 
-  float4 gv[16];
+  // The decay rows of a chunk are read with per-thread loads; an L2 prefetch
+  // of the chunk's [64 x 128] fp32 tile two chunks ahead keeps those loads
+  // short.
+  if (f == 0) {
+    for (int c = 0; c < 2 && c < x.nchunks; ++c) tma_prefetch_l2_3d(tmg, 0, x.h, (int)(x.t0 + (int64_t)c * CH));
+  }
+  F8 gv[8];
   float bv;
   load_g(0, gv, bv);
   int g1_ph = 0;
@@ -442,39 +482,49 @@ __device__ void front_group(const Ctx& x, const float* __restrict__ g, const flo
     float* s_beta = reinterpret_cast<float*>(sm + SM_MISC + MS_BETA) + b2 * 64;
     volatile int* s_fast = reinterpret_cast<volatile int*>(sm + SM_MISC + MS_FAST) + b2;
 
-    if (f == 0) tmark(x, c, 0);
+    if (f == 0) {
+      tmark(x, c, 0);
+      if (c + 2 < x.nchunks) tma_prefetch_l2_3d(tmg, 0, x.h, (int)(x.t0 + (int64_t)(c + 2) * CH));
+    }
     // ---- (a1) decay prefix in log2 units (registers only): this thread's
-    // 16-row sums, then the offsets of the earlier row groups and the chunk
+    // 8-row sums, then the offsets of the earlier row groups and the chunk
     // total G_C.
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    const float4 l2e = make_float4(LOG2E, LOG2E, LOG2E, LOG2E);
+    F8 acc = f8(0.f);
+    const F8 l2e = f8(LOG2E);
 #pragma unroll
-    for (int m = 0; m < 16; ++m) {
-      gv[m] = mul4(gv[m], l2e);
-      acc = add4(acc, gv[m]);
+    for (int m = 0; m < 8; ++m) {
+      gv[m] = mul8(gv[m], l2e);
+      acc = add8(acc, gv[m]);
     }
-    *reinterpret_cast<float4*>(s_red + wq * 128 + ch0) = acc;
+    *reinterpret_cast<float4*>(s_red + rg * 128 + ch0) = acc.a;
+    *reinterpret_cast<float4*>(s_red + rg * 128 + ch0 + 4) = acc.b;
     named_sync(GRP_FRONT, GRP);
-    float4 tot = make_float4(0.f, 0.f, 0.f, 0.f), off = tot;
+    F8 tot = f8(0.f), off = tot;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const float4 v = *reinterpret_cast<const float4*>(s_red + q * 128 + ch0);
-      if (q < wq) { off.x += v.x; off.y += v.y; off.z += v.z; off.w += v.w; }
-      tot.x += v.x; tot.y += v.y; tot.z += v.z; tot.w += v.w;
+    for (int q = 0; q < 8; ++q) {
+      const F8 v = {*reinterpret_cast<const float4*>(s_red + q * 128 + ch0),
+                    *reinterpret_cast<const float4*>(s_red + q * 128 + ch0 + 4)};
+      if (q < rg) off = add8(off, v);
+      tot = add8(tot, v);
     }
-    const bool fast =
-        named_sync_and(GRP_FRONT, GRP, fminf(fminf(tot.x, tot.y), fminf(tot.z, tot.w)) >= FAST_MIN_LOG2);
+    const bool fast = named_sync_and(GRP_FRONT, GRP, min8(tot) >= FAST_MIN_LOG2);
+    gv[0] = add8(gv[0], off);  // from here the running sum of gv[0..m] is G of row 8 rg + m
     if (f == 0) tmark(x, c, 1);
     // Per-chunk values for the scan and back groups, in buffers [b2] that the
     // scan of chunk c-2 has released.
     auto publish = [&]() {
-      if (wq == 0) *reinterpret_cast<float4*>(s_gc + ch0) = ex2_4(tot);
+      if (rg == 0) {
+        const F8 e = ex2_8(tot);
+        *reinterpret_cast<float4*>(s_gc + ch0) = e.a;
+        *reinterpret_cast<float4*>(s_gc + ch0 + 4) = e.b;
+      }
       if (f == 0) *s_fast = fast ? 1 : 0;
       if (f < CH) s_beta[f] = bv;
-      if (dmp && wq == 0) {
+      if (dmp && rg == 0) {
         const float LN2 = 0.6931471805599453f;
-        x.dbg[DBG_GC + ch0] = tot.x * LN2; x.dbg[DBG_GC + ch0 + 1] = tot.y * LN2;
-        x.dbg[DBG_GC + ch0 + 2] = tot.z * LN2; x.dbg[DBG_GC + ch0 + 3] = tot.w * LN2;
+        const float tv[8] = {tot.a.x, tot.a.y, tot.a.z, tot.a.w, tot.b.x, tot.b.y, tot.b.z, tot.b.w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) x.dbg[DBG_GC + ch0 + i] = tv[i] * LN2;
       }
       mbar_arrive(&x.bars[B_GC0 + b2]);  // one arrival per thread, after its own writes
     };
@@ -486,12 +536,11 @@ __device__ void front_group(const Ctx& x, const float* __restrict__ g, const flo
     if (!gwait(x, B_FULL0 + b2, (c >> 1) & 1, 12, GRP_FRONT)) break;
     ++consumed[b2];
     if (f == 0) tmark(x, c, 2);
-    if (!fast) general_gram(x, b2, valid, gv, off);
+    if (!fast) general_gram(x, b2, valid, gv);
 
     // ---- (a2) operand scaling, row by row: E = e^{G_r - ref} (ref = G_C on
     // fast chunks, 0 otherwise), H = e^{G_C - G_r}.  QE, KE and V (fp16) go
     // in place; KH goes to KX[b2] once the scan of chunk c-2 has released it.
-    const float4 ref = fast ? tot : make_float4(0.f, 0.f, 0.f, 0.f);
     uint8_t* qb = sm + b2 * STAGE_BYTES + OFF_QK + hh * 16384;
     uint8_t* kb = qb + 8192;
     uint8_t* vb = sm + b2 * STAGE_BYTES + OFF_V + hh * 8192;
@@ -501,39 +550,38 @@ __device__ void front_group(const Ctx& x, const float* __restrict__ g, const flo
       // this thread's rows and channels of the raw tiles, so the scaling
       // pass below needs no per-row mask.
 #pragma unroll 1
-      for (int m = 0; m < 16; ++m) {
-        const int r = 16 * wq + m;
+      for (int m = 0; m < 8; ++m) {
+        const int r = 8 * rg + m;
         if (r >= valid) {
           const uint32_t o = sw128_off(r, cc);
-          *reinterpret_cast<uint2*>(qb + o) = make_uint2(0u, 0u);
-          *reinterpret_cast<uint2*>(kb + o) = make_uint2(0u, 0u);
-          *reinterpret_cast<uint2*>(vb + o) = make_uint2(0u, 0u);
+          *reinterpret_cast<uint4*>(qb + o) = make_uint4(0u, 0u, 0u, 0u);
+          *reinterpret_cast<uint4*>(kb + o) = make_uint4(0u, 0u, 0u, 0u);
+          *reinterpret_cast<uint4*>(vb + o) = make_uint4(0u, 0u, 0u, 0u);
         }
       }
     }
-    uint2 kraw[16];  // raw K rows, kept for KH
+    uint4 kraw[8];  // raw K rows, kept for KH
     {
-      const float4 nref = fast ? make_float4(-tot.x, -tot.y, -tot.z, -tot.w) : make_float4(0.f, 0.f, 0.f, 0.f);
-      float4 gr = off;
+      F8 gr = f8(0.f);
 #pragma unroll
-      for (int mb = 0; mb < 16; mb += 4) {
-        uint2 qr[4], vr[4];
+      for (int mb = 0; mb < 8; mb += 2) {
+        uint4 qr[2], vr[2];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {  // this batch's loads first, then the in-place stores
-          const uint32_t o = sw128_off(16 * wq + mb + i, cc);
-          qr[i] = *reinterpret_cast<const uint2*>(qb + o);
-          kraw[mb + i] = *reinterpret_cast<const uint2*>(kb + o);
-          vr[i] = *reinterpret_cast<const uint2*>(vb + o);
+        for (int i = 0; i < 2; ++i) {  // this batch's loads first, then the in-place stores
+          const uint32_t o = sw128_off(8 * rg + mb + i, cc);
+          qr[i] = *reinterpret_cast<const uint4*>(qb + o);
+          kraw[mb + i] = *reinterpret_cast<const uint4*>(kb + o);
+          vr[i] = *reinterpret_cast<const uint4*>(vb + o);
         }
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < 2; ++i) {
           const int m = mb + i;
-          const uint32_t o = sw128_off(16 * wq + m, cc);
-          gr = add4(gr, gv[m]);
-          const float4 fw = ex2_4(add4(gr, nref));
-          st_f16x4(qb + o, mul4(bf16x4_to_f32(qr[i]), fw));
-          st_f16x4(kb + o, mul4(bf16x4_to_f32(kraw[m]), fw));
-          st_f16x4(vb + o, bf16x4_to_f32(vr[i]));
+          const uint32_t o = sw128_off(8 * rg + m, cc);
+          gr = add8(gr, gv[m]);
+          const F8 fw = ex2_8(fast ? sub8(gr, tot) : gr);
+          st_f16x8(qb + o, mul8(bf16x8_to_f32(qr[i]), fw));
+          st_f16x8(kb + o, mul8(bf16x8_to_f32(kraw[m]), fw));
+          st_f16x8(vb + o, bf16x8_to_f32(vr[i]));
         }
       }
     }
@@ -546,12 +594,12 @@ __device__ void front_group(const Ctx& x, const float* __restrict__ g, const flo
     }
     if (f == 0) tmark(x, c, 4);
     {
-      float4 gr = off;
+      F8 gr = f8(0.f);
 #pragma unroll
-      for (int m = 0; m < 16; ++m) {
-        const uint32_t o = sw128_off(16 * wq + m, cc);
-        gr = add4(gr, gv[m]);
-        st_f16x4(khb + o, mul4(bf16x4_to_f32(kraw[m]), ex2_4(sub4(tot, gr))));
+      for (int m = 0; m < 8; ++m) {
+        const uint32_t o = sw128_off(8 * rg + m, cc);
+        gr = add8(gr, gv[m]);
+        st_f16x8(khb + o, mul8(bf16x8_to_f32(kraw[m]), ex2_8(sub8(tot, gr))));
       }
     }
     fence_proxy_async_smem();
@@ -1110,6 +1158,7 @@ __device__ void scan_group(const Ctx& x, const void* tmq, const void* tmk, const
 __global__ void __launch_bounds__(NTHR, 1)
     kda_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                      const __grid_constant__ CUtensorMap tm_g,
                       const float* __restrict__ g,
                       const float* __restrict__ beta, const float* __restrict__ init,
                       __nv_bfloat16* __restrict__ out, float* __restrict__ fin, const int32_t* __restrict__ cu,
@@ -1155,6 +1204,7 @@ __global__ void __launch_bounds__(NTHR, 1)
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
     prefetch_tmap(&tm_o);
+    prefetch_tmap(&tm_g);
   }
   if (warp == 0) {
     tmem_alloc(reinterpret_cast<uint32_t*>(sm + SM_MISC + MS_TMEM), TMEM_COLS);
@@ -1173,7 +1223,7 @@ __global__ void __launch_bounds__(NTHR, 1)
     scan_group(x, &tm_q, &tm_k, &tm_v, &tm_o, init, out, fin, sbase, inject_stuck != 0, cnt);
     if (tid == 0) { s_cnt[0] = cnt[0]; s_cnt[1] = cnt[1]; }
   } else if (warp < 8) {
-    front_group(x, g, beta, cnt);
+    front_group(x, g, beta, &tm_g, cnt);
     if (tid == 128) { s_cnt[2] = cnt[0]; s_cnt[3] = cnt[1]; }
   } else {
     back_group(x);
@@ -1255,6 +1305,20 @@ bool make_map(CUtensorMap* m, const void* ptr, int H, int64_t Ttot) {
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// fp32 log-decay [T_total][H][128] as a 3-D map, box {128 channels, 1 head, 64 tokens}
+// (used for L2 prefetches only).
+bool make_map_g(CUtensorMap* m, const float* ptr, int H, int64_t Ttot) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)Ttot};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 4, (cuuint64_t)H * D * 4};
+  cuuint32_t box[3] = {(cuuint32_t)D, 1, (cuuint32_t)CH};
+  cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(ptr), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 bool fwd_tc_supported(int dk, int dv, bool bf16) { return bf16 && dk == D && dv == D; }
@@ -1264,10 +1328,10 @@ cudaError_t launch_fwd_tc_impl(const FwdArgs& a, cudaStream_t s, uint64_t wait_n
   const int64_t Ttot = a.cu ? a.T : (int64_t)a.N * a.T;
   const unsigned blocks = (unsigned)((int64_t)a.N * a.H);
   if (blocks == 0) return cudaSuccess;
-  CUtensorMap mq, mk, mv, mo;
+  CUtensorMap mq, mk, mv, mo, mg;
   const int64_t Tmap = Ttot > 0 ? Ttot : 1;
   if (!make_map(&mq, a.q, a.H, Tmap) || !make_map(&mk, a.k, a.H, Tmap) || !make_map(&mv, a.v, a.H, Tmap) ||
-      !make_map(&mo, a.out, a.H, Tmap))
+      !make_map(&mo, a.out, a.H, Tmap) || !make_map_g(&mg, a.g, a.H, Tmap))
     return cudaErrorInvalidValue;
   const int32_t* order = nullptr;
   if (a.cu && order_ws && a.N > 1) {
@@ -1277,7 +1341,7 @@ cudaError_t launch_fwd_tc_impl(const FwdArgs& a, cudaStream_t s, uint64_t wait_n
   cudaError_t e =
       cudaFuncSetAttribute(kda_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  kda_fwd_tc_kernel<<<blocks, NTHR, SMEM_BYTES, s>>>(mq, mk, mv, mo, a.g, a.beta, a.init, (__nv_bfloat16*)a.out,
+  kda_fwd_tc_kernel<<<blocks, NTHR, SMEM_BYTES, s>>>(mq, mk, mv, mo, mg, a.g, a.beta, a.init, (__nv_bfloat16*)a.out,
                                                      a.fin, a.cu, order, a.cu ? 0 : a.T, a.H, a.status,
                                                      (float*)a.dbg, wait_ns, inject_stuck);
   return cudaGetLastError();
