@@ -210,13 +210,16 @@ __device__ __forceinline__ void warp_gemm_tf32x3(float (&d)[4], FA fa, FB fb) {
   // KSTEPS long; the small terms are added first.
   float dhh[4] = {0.f, 0.f, 0.f, 0.f}, dhl[4] = {0.f, 0.f, 0.f, 0.f}, dlh[4] = {0.f, 0.f, 0.f, 0.f};
   float av[KSTEPS][4], bv[KSTEPS][2];
+  // ldmatrix row address of this lane: tile lane/8 = (rows 8 (tile & 1)..,
+  // words 4 (tile >> 1)..) of the 16x8 A block.
+  const int arow = (lane & 7) + 8 * ((lane >> 3) & 1), akof = 4 * (lane >> 4);
 #pragma unroll
   for (int ks = 0; ks < KSTEPS; ++ks) {  // every fragment load first: one shared-memory latency
     const int k0 = 8 * ks;
-    av[ks][0] = *fa(g, k0 + t);
-    av[ks][1] = *fa(g + 8, k0 + t);
-    av[ks][2] = *fa(g, k0 + t + 4);
-    av[ks][3] = *fa(g + 8, k0 + t + 4);
+    uint32_t a4[4];
+    ldsm_x4(smem_u32(fa(arow, k0 + akof)), a4);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) av[ks][i] = __uint_as_float(a4[i]);
     bv[ks][0] = *fb(k0 + t, g);
     bv[ks][1] = *fb(k0 + t + 4, g);
   }

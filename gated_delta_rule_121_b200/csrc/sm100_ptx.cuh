@@ -280,6 +280,17 @@ __device__ __forceinline__ uint32_t sw128_off(uint32_t row, uint32_t col) {
   return row * 128u + ((((col >> 3) ^ row) & 7u) << 4) + ((col & 7u) << 1);
 }
 
+// Four 8x8 b16 tiles from shared memory (lane l supplies the row address of
+// tile l / 8, row l % 8); lane l receives the 32-bit word l % 4 of row l / 4
+// of each tile.  With 32-bit data an 8x8 b16 tile is 8 rows x 4 words, so
+// this is also the A-fragment layout of a tf32 m16n8k8 MMA.
+__device__ __forceinline__ void ldsm_x4(uint32_t saddr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(saddr)
+               : "memory");
+}
+
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   __half2 h = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
