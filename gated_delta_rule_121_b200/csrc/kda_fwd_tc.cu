@@ -1068,8 +1068,6 @@ __device__ void scan_group(const Ctx& x, const void* tmq, const void* tmk, const
       }
       tmark(x, c, 28);
     }
-    if (c >= 1) store_out(c - 1);
-    if (j == 0) tmark(x, c, 12);
     if (!gwait(x, B_D1, d1_ph, 34, GRP_SG)) {
       ok = false;
       break;
@@ -1134,6 +1132,10 @@ __device__ void scan_group(const Ctx& x, const void* tmq, const void* tmk, const
       umma_commit(&x.bars[B_DFREE]);  // Δ^T read: the next U^T may land
       tmark(x, c, 15);
     }
+    // The output of chunk c-1 (final since D2 of c-1), off the path from
+    // D1b to D2 that the next chunks' front and back wait on.
+    if (c >= 1) store_out(c - 1);
+    if (j == 0) tmark(x, c, 12);
   }
   if (named_sync_and(2, 128, ok && !*x.abort) && x.nchunks > 0) {
     if (gwait(x, B_D2, d2_ph, 35, GRP_SG)) {
