@@ -124,6 +124,17 @@ def test_model_shaped_prefill_sampled_heads():
     print("pretrain errors", eo, ef)
 
 
+def test_packed_varlen_full_size_sampled_heads():
+    """The packed long-context workload at full size: H=32, 1,048,576 tokens in
+    sequences of log-uniform length in [1024, 262144], each with its own
+    initial state; heads 0 and 31 of every sequence checked."""
+    inp = synth.make_prefill(synth.VARLEN, DEV)
+    cu = inp["cu_seqlens"].cpu()
+    assert int(cu[-1]) == 1 << 20 and cu.numel() - 1 >= 3
+    eo, ef = check(inp, torch.bfloat16, heads=[0, 31], what="varlen H32 T1M")
+    print("varlen errors", cu.numel() - 1, "sequences", eo, ef)
+
+
 def test_debug_intermediates_match_chunk_model():
     from chunk_model import chunk_forward
     inp = synth.make_prefill(synth.MID, DEV, T=64, B=1, H=1)
