@@ -54,7 +54,7 @@ namespace {
 
 constexpr int CH = 64;  // chunk length
 constexpr int D = 128;  // dk = dv
-constexpr int NTHR = 384;  // scan, front and back groups of 4 warps
+constexpr int NTHR = 512;  // scan (4 warps), front (8 warps) and back (4 warps) groups
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float FAST_MIN_LOG2 = -10.0f;  // chunk-total decay floor (log2) for the tensor-core Gram
 constexpr float F16_SAFE = 60000.0f;     // |x| above this would overflow fp16 operands
@@ -282,14 +282,18 @@ __device__ __forceinline__ bool cwait(const Ctx& x, int bar, uint32_t parity, in
   return false;
 }
 
-// Named-barrier ids of the three 128-thread groups, and each group's first thread.
+// Named-barrier ids of the three groups, their first threads and sizes:
+// scan = warps 0-3, front = warps 4-11, back = warps 12-15.
 constexpr int GRP_FRONT = 1, GRP_SG = 2, GRP_BACK = 3;
+constexpr int FRONT_T = 256, BACK_T = 128, SG_T = 128;
+constexpr unsigned FRONT0 = 128, BACK0 = 384;
 __device__ __forceinline__ unsigned grp_leader(int grp) {
-  return grp == GRP_SG ? 0u : (grp == GRP_FRONT ? 128u : 256u);
+  return grp == GRP_SG ? 0u : (grp == GRP_FRONT ? FRONT0 : BACK0);
 }
+__device__ __forceinline__ int grp_size(int grp) { return grp == GRP_FRONT ? FRONT_T : 128; }
 
 // Group-uniform bounded wait: every thread of named-barrier group `grp`
-// (128 threads) polls, then the group agrees on the outcome, so no thread can
+// (all its threads) polls, then the group agrees on the outcome, so no thread can
 // leave a loop while the others wait at a barrier or a .sync.aligned op.
 //
 // Only the group's first thread polls the mbarrier; the others block in the
@@ -307,7 +311,7 @@ __device__ __forceinline__ bool gwait(const Ctx& x, int bar, uint32_t parity, in
       *x.abort = 1;
     }
   }
-  ok = named_sync_and(grp, 128, ok);
+  ok = named_sync_and(grp, grp_size(grp), ok);
   // Each thread also observes the completed phase itself (an acquire that
   // returns at once), so the data it guards is visible to every thread.
   if (ok && !elected) mbar_try_wait(&x.bars[bar], parity);
@@ -328,91 +332,78 @@ __device__ __forceinline__ int chunk_valid(const Ctx& x, int c) {
 // Row-wise front work: thread f owns rows 8 (f / 16) .. + 7 and channels
 // 8 (f % 16) .. + 7, so every tile access is 16 bytes wide.  TMEM work: a
 // warp reads the lane quarter (warp index mod 4) it is allowed to access.
-constexpr int GRP = 128;  // threads per group
+constexpr int GRP = 128;  // threads of the scan and back groups
 
 // General chunks: P and A on CUDA cores from the exact decay differences
 // G_r - G_s (log2 units), G staged through the A tile one channel half at a
 // time (the back group has released the A tile).  Raw Q and K are read from
 // the stage before they are rescaled in place.
-__device__ __forceinline__ void general_gram(const Ctx& x, int b2, int valid, const F8 (&gv)[8]) {
-  const int f = threadIdx.x - 128;
+__device__ __forceinline__ void general_gram(const Ctx& x, int b2, int valid, const F8 (&gv)[4]) {
+  const int f = threadIdx.x - FRONT0;
   const int rg = f >> 4, ch0 = 8 * (f & 15), hh = ch0 >> 6, cc = ch0 & 63;
   uint8_t* sm = x.sm;
   const float* s_beta = reinterpret_cast<const float*>(sm + SM_MISC + MS_BETA) + b2 * 64;
-  const int r = f & 63;
+  const int r = f & 63, s0 = (f >> 6) * 16;  // row r, columns s0 .. s0 + 15
   const uint8_t* stp = sm + b2 * STAGE_BYTES;
-  uint32_t pk[2][8];
-  float ak[2][16];
+  float pa[16], aa[16];
 #pragma unroll
-  for (int j = 0; j < 2; ++j) {
-    const int s0 = (f >> 6) * 32 + 16 * j;
-    float pa[16], aa[16];
+  for (int i = 0; i < 16; ++i) pa[i] = aa[i] = 0.f;
+  for (int half = 0; half < 2; ++half) {
+    named_sync(GRP_FRONT, FRONT_T);  // earlier readers of the staging tile are done
+    if (hh == half) {
+      F8 gr = f8(0.f);
 #pragma unroll
-    for (int i = 0; i < 16; ++i) pa[i] = aa[i] = 0.f;
-    for (int half = 0; half < 2; ++half) {
-      named_sync(GRP_FRONT, GRP);  // earlier readers of the staging tile are done
-      if (hh == half) {
-        F8 gr = f8(0.f);
-#pragma unroll
-        for (int m = 0; m < 8; ++m) {
-          gr = add8(gr, gv[m]);
-          *reinterpret_cast<float4*>(sm + SM_A + (8 * rg + m) * 256 + cc * 4) = gr.a;
-          *reinterpret_cast<float4*>(sm + SM_A + (8 * rg + m) * 256 + cc * 4 + 16) = gr.b;
-        }
+      for (int m = 0; m < 4; ++m) {
+        gr = add8(gr, gv[m]);
+        *reinterpret_cast<float4*>(sm + SM_A + (4 * rg + m) * 256 + cc * 4) = gr.a;
+        *reinterpret_cast<float4*>(sm + SM_A + (4 * rg + m) * 256 + cc * 4 + 16) = gr.b;
       }
-      named_sync(GRP_FRONT, GRP);
-      if (r < valid && s0 <= r) {
+    }
+    named_sync(GRP_FRONT, FRONT_T);
+    if (r < valid && s0 <= r) {
 #pragma unroll 1
-        for (int ch = 0; ch < 64; ++ch) {
-          const uint32_t off_r = half * 16384 + sw128_off(r, ch);
-          const float gr = *reinterpret_cast<const float*>(sm + SM_A + r * 256 + ch * 4);
-          const float qr = ld_bf16(stp + OFF_QK + off_r), kr = ld_bf16(stp + OFF_QK + 8192 + off_r);
+      for (int ch = 0; ch < 64; ++ch) {
+        const uint32_t off_r = half * 16384 + sw128_off(r, ch);
+        const float gr = *reinterpret_cast<const float*>(sm + SM_A + r * 256 + ch * 4);
+        const float qr = ld_bf16(stp + OFF_QK + off_r), kr = ld_bf16(stp + OFF_QK + 8192 + off_r);
 #pragma unroll 4
-          for (int i = 0; i < 16; ++i) {
-            const int s = s0 + i;
-            if (s <= r) {
-              const float gs = *reinterpret_cast<const float*>(sm + SM_A + s * 256 + ch * 4);
-              const float ks = ld_bf16(stp + OFF_QK + 8192 + half * 16384 + sw128_off(s, ch));
-              const float e = ex2(gr - gs) * ks;
-              pa[i] += qr * e;
-              aa[i] += kr * e;
-            }
+        for (int i = 0; i < 16; ++i) {
+          const int s = s0 + i;
+          if (s <= r) {
+            const float gs = *reinterpret_cast<const float*>(sm + SM_A + s * 256 + ch * 4);
+            const float ks = ld_bf16(stp + OFF_QK + 8192 + half * 16384 + sw128_off(s, ch));
+            const float e = ex2(gr - gs) * ks;
+            pa[i] += qr * e;
+            aa[i] += kr * e;
           }
         }
       }
     }
-    const float br = s_beta[r];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int s = s0 + i;
-      ak[j][i] = s < r ? br * aa[i] : 0.f;
-      if (!(s <= r)) pa[i] = 0.f;
-    }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) pk[j][i] = pack_f16x2(pa[2 * i], pa[2 * i + 1]);
   }
-  named_sync(GRP_FRONT, GRP);  // every staged G read is done before A overwrites the tile
+  const float br = s_beta[r];
 #pragma unroll
-  for (int j = 0; j < 2; ++j) {
-    const int s0 = (f >> 6) * 32 + 16 * j;
-#pragma unroll
-    for (int q8 = 0; q8 < 2; ++q8) {
-      const int s = s0 + 8 * q8;
-      *reinterpret_cast<uint4*>(sm + SM_P + b2 * 8192 + r * 128 + ((((s >> 3) ^ r) & 7) << 4)) =
-          make_uint4(pk[j][4 * q8], pk[j][4 * q8 + 1], pk[j][4 * q8 + 2], pk[j][4 * q8 + 3]);
-    }
-#pragma unroll
-    for (int u = 0; u < 4; ++u)
-      *reinterpret_cast<float4*>(sm + SM_A + a_off(r, s0 + 4 * u)) =
-          make_float4(ak[j][4 * u], ak[j][4 * u + 1], ak[j][4 * u + 2], ak[j][4 * u + 3]);
+  for (int i = 0; i < 16; ++i) {
+    const int s = s0 + i;
+    aa[i] = s < r ? br * aa[i] : 0.f;
+    if (!(s <= r)) pa[i] = 0.f;
   }
-  named_sync(GRP_FRONT, GRP);  // raw Q/K reads are done before they are rescaled in place
+  named_sync(GRP_FRONT, FRONT_T);  // every staged G read is done before A overwrites the tile
+#pragma unroll
+  for (int q8 = 0; q8 < 2; ++q8) {
+    const int s = s0 + 8 * q8;
+    st_f16x8(sm + SM_P + b2 * 8192 + r * 128 + ((((s >> 3) ^ r) & 7) << 4), pa + 8 * q8);
+  }
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+    *reinterpret_cast<float4*>(sm + SM_A + a_off(r, s0 + 4 * u)) =
+        make_float4(aa[4 * u], aa[4 * u + 1], aa[4 * u + 2], aa[4 * u + 3]);
+  named_sync(GRP_FRONT, FRONT_T);  // raw Q/K reads are done before they are rescaled in place
 }
 
 // Debug dumps (chain 0, chunk 0): P (fp16 tile) and A (fp32 tile); T'; W'
 // (from the fp16 W'^T tile) and U (TMEM, before D1).
 __device__ __noinline__ void dump_pa(float* dbg, const uint8_t* sm, int b2, int p) {
-  for (int e = p; e < 4096; e += GRP) {
+  for (int e = p; e < 4096; e += FRONT_T) {
     const int r = e >> 6, s = e & 63;
     const uint16_t u = *reinterpret_cast<const uint16_t*>(sm + SM_P + b2 * 8192 + sw128_off(r, s));
     dbg[DBG_P + e] = __half2float(*reinterpret_cast<const __half*>(&u));
@@ -443,23 +434,24 @@ __device__ __noinline__ void dump_wu(float* dbg, const uint8_t* sm, uint32_t tme
 
 __device__ void front_group(const Ctx& x, const float* __restrict__ g, const float* __restrict__ beta,
                             const void* tmg, int (&consumed)[2]) {
-  const int f = threadIdx.x - 128;  // 0..127
-  const int wq = f >> 5;                                    // warp: TMEM lane quarter
+  const int f = threadIdx.x - FRONT0;  // 0..255
+  const int wq = f >> 5, lane = f & 31;
+  const int lq = wq & 3, chh = wq >> 2;                      // TMEM lane quarter, column half
   const int rg = f >> 4, ch0 = 8 * (f & 15), hh = ch0 >> 6, cc = ch0 & 63;
-  const uint32_t tl = x.tmem + ((uint32_t)(wq * 32) << 16);
+  const uint32_t tl = x.tmem + ((uint32_t)(lq * 32) << 16);
   uint8_t* sm = x.sm;
   const uint32_t sb = x.sb;
-  float* s_red = reinterpret_cast<float*>(sm + SM_MISC + MS_RED);  // [8][128] log2 sums
+  float* s_red = reinterpret_cast<float*>(sm + SM_MISC + MS_RED);  // [8][128] log2 sums, one row per warp
   const int H = x.H;
   const bool g32 = (reinterpret_cast<uintptr_t>(g) & 31u) == 0;
 
-  // Register prefetch of this thread's g rows (8 rows x 8 channels) and of beta.
-  auto load_g = [&](int c, F8(&gv)[8], float& bv) {
+  // Register prefetch of this thread's g rows (4 rows x 8 channels) and of beta.
+  auto load_g = [&](int c, F8(&gv)[4], float& bv) {
     const int valid = c < x.nchunks ? chunk_valid(x, c) : 0;
     const int64_t tok0 = x.t0 + (int64_t)c * CH;
 #pragma unroll
-    for (int m = 0; m < 8; ++m) {
-      const int r = 8 * rg + m;
+    for (int m = 0; m < 4; ++m) {
+      const int r = 4 * rg + m;
       gv[m] = r < valid ? ldg8(g + ((tok0 + r) * H + x.h) * D + ch0, g32) : f8(0.f);
     }
     bv = (f < CH && f < valid) ? __ldg(beta + (tok0 + f) * H + x.h) : 0.f;
@@ -471,7 +463,7 @@ __device__ void front_group(const Ctx& x, const float* __restrict__ g, const flo
   if (f == 0) {
     for (int c = 0; c < 2 && c < x.nchunks; ++c) tma_prefetch_l2_3d(tmg, 0, x.h, (int)(x.t0 + (int64_t)c * CH));
   }
-  F8 gv[8];
+  F8 gv[4];
   float bv;
   load_g(0, gv, bv);
   int g1_ph = 0;
@@ -490,28 +482,37 @@ __device__ void front_group(const Ctx& x, const float* __restrict__ g, const flo
       if (c + 2 < x.nchunks) tma_prefetch_l2_3d(tmg, 0, x.h, (int)(x.t0 + (int64_t)(c + 2) * CH));
     }
     // ---- (a1) decay prefix in log2 units (registers only): this thread's
-    // 8-row sums, then the offsets of the earlier row groups and the chunk
-    // total G_C.
+    // 4-row sums; the two row groups of a warp combine by shuffle, the eight
+    // warps through shared memory; then the offsets of the earlier row
+    // groups and the chunk total G_C.
     F8 acc = f8(0.f);
     const F8 l2e = f8(LOG2E);
 #pragma unroll
-    for (int m = 0; m < 8; ++m) {
+    for (int m = 0; m < 4; ++m) {
       gv[m] = mul8(gv[m], l2e);
       acc = add8(acc, gv[m]);
     }
-    *reinterpret_cast<float4*>(s_red + rg * 128 + ch0) = acc.a;
-    *reinterpret_cast<float4*>(s_red + rg * 128 + ch0 + 4) = acc.b;
-    named_sync(GRP_FRONT, GRP);
-    F8 tot = f8(0.f), off = tot;
+    F8 other;  // the other row group of this warp (lane ^ 16)
+    other.a.x = __shfl_xor_sync(0xffffffffu, acc.a.x, 16); other.a.y = __shfl_xor_sync(0xffffffffu, acc.a.y, 16);
+    other.a.z = __shfl_xor_sync(0xffffffffu, acc.a.z, 16); other.a.w = __shfl_xor_sync(0xffffffffu, acc.a.w, 16);
+    other.b.x = __shfl_xor_sync(0xffffffffu, acc.b.x, 16); other.b.y = __shfl_xor_sync(0xffffffffu, acc.b.y, 16);
+    other.b.z = __shfl_xor_sync(0xffffffffu, acc.b.z, 16); other.b.w = __shfl_xor_sync(0xffffffffu, acc.b.w, 16);
+    const F8 wsum = add8(acc, other);
+    if (lane < 16) {
+      *reinterpret_cast<float4*>(s_red + wq * 128 + ch0) = wsum.a;
+      *reinterpret_cast<float4*>(s_red + wq * 128 + ch0 + 4) = wsum.b;
+    }
+    named_sync(GRP_FRONT, FRONT_T);
+    F8 tot = f8(0.f), off = (lane >= 16) ? other : f8(0.f);
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
       const F8 v = {*reinterpret_cast<const float4*>(s_red + q * 128 + ch0),
                     *reinterpret_cast<const float4*>(s_red + q * 128 + ch0 + 4)};
-      if (q < rg) off = add8(off, v);
+      if (q < wq) off = add8(off, v);
       tot = add8(tot, v);
     }
-    const bool fast = named_sync_and(GRP_FRONT, GRP, min8(tot) >= FAST_MIN_LOG2);
-    gv[0] = add8(gv[0], off);  // from here the running sum of gv[0..m] is G of row 8 rg + m
+    const bool fast = named_sync_and(GRP_FRONT, FRONT_T, min8(tot) >= FAST_MIN_LOG2);
+    gv[0] = add8(gv[0], off);  // from here the running sum of gv[0..m] is G of row 4 rg + m
     if (f == 0) tmark(x, c, 1);
     // Per-chunk values for the scan and back groups, in buffers [b2] that the
     // scan of chunk c-2 has released.
@@ -553,8 +554,8 @@ __device__ void front_group(const Ctx& x, const float* __restrict__ g, const flo
       // this thread's rows and channels of the raw tiles, so the scaling
       // pass below needs no per-row mask.
 #pragma unroll 1
-      for (int m = 0; m < 8; ++m) {
-        const int r = 8 * rg + m;
+      for (int m = 0; m < 4; ++m) {
+        const int r = 4 * rg + m;
         if (r >= valid) {
           const uint32_t o = sw128_off(r, cc);
           *reinterpret_cast<uint4*>(qb + o) = make_uint4(0u, 0u, 0u, 0u);
@@ -563,15 +564,15 @@ __device__ void front_group(const Ctx& x, const float* __restrict__ g, const flo
         }
       }
     }
-    uint4 kraw[8];  // raw K rows, kept for KH
+    uint4 kraw[4];  // raw K rows, kept for KH
     {
       F8 gr = f8(0.f);
 #pragma unroll
-      for (int mb = 0; mb < 8; mb += 2) {
+      for (int mb = 0; mb < 4; mb += 2) {
         uint4 qr[2], vr[2];
 #pragma unroll
         for (int i = 0; i < 2; ++i) {  // this batch's loads first, then the in-place stores
-          const uint32_t o = sw128_off(8 * rg + mb + i, cc);
+          const uint32_t o = sw128_off(4 * rg + mb + i, cc);
           qr[i] = *reinterpret_cast<const uint4*>(qb + o);
           kraw[mb + i] = *reinterpret_cast<const uint4*>(kb + o);
           vr[i] = *reinterpret_cast<const uint4*>(vb + o);
@@ -579,7 +580,7 @@ __device__ void front_group(const Ctx& x, const float* __restrict__ g, const flo
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
           const int m = mb + i;
-          const uint32_t o = sw128_off(8 * rg + m, cc);
+          const uint32_t o = sw128_off(4 * rg + m, cc);
           gr = add8(gr, gv[m]);
           const F8 fw = ex2_8(fast ? sub8(gr, tot) : gr);
           st_f16x8(qb + o, mul8(bf16x8_to_f32(qr[i]), fw));
@@ -599,14 +600,14 @@ __device__ void front_group(const Ctx& x, const float* __restrict__ g, const flo
     {
       F8 gr = f8(0.f);
 #pragma unroll
-      for (int m = 0; m < 8; ++m) {
-        const uint32_t o = sw128_off(8 * rg + m, cc);
+      for (int m = 0; m < 4; ++m) {
+        const uint32_t o = sw128_off(4 * rg + m, cc);
         gr = add8(gr, gv[m]);
         st_f16x8(khb + o, mul8(bf16x8_to_f32(kraw[m]), ex2_8(sub8(tot, gr))));
       }
     }
     fence_proxy_async_smem();
-    named_sync(GRP_FRONT, GRP);
+    named_sync(GRP_FRONT, FRONT_T);
     if (f == 0) tmark(x, c, 5);
 
     if (fast) {
@@ -631,39 +632,35 @@ __device__ void front_group(const Ctx& x, const float* __restrict__ g, const flo
       g1_ph ^= 1;
       tc_fence_after();
       if (f == 0) tmark(x, c, 7);
-      float r0[32], r1[32];
-      tmem_ld32x2(tl + TM_G, tl + TM_G + 32, r0, r1);  // TMEM lane f: row f of [P ; A_raw]
-      if (wq < 2) {  // P row f, lower triangle including the diagonal
-        const int r = f;
+      // TMEM lane 32 lq + lane is row ti of [P ; A_raw]; this warp reads
+      // columns 32 chh .. 32 chh + 31.
+      const int ti = 32 * lq + lane;
+      float r0[32];
+      tmem_ld32(tl + TM_G + chh * 32, r0);
+      if (lq < 2) {  // P row ti, lower triangle including the diagonal
+        const int r = ti;
 #pragma unroll
-        for (int s = 0; s < 32; ++s) {
-          if (s > r) r0[s] = 0.f;
-          if (32 + s > r) r1[s] = 0.f;
-        }
+        for (int s = 0; s < 32; ++s)
+          if (chh * 32 + s > r) r0[s] = 0.f;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          st_f16x8(sm + SM_P + b2 * 8192 + r * 128 + (((k ^ r) & 7) << 4), r0 + 8 * k);
-          st_f16x8(sm + SM_P + b2 * 8192 + r * 128 + ((((4 + k) ^ r) & 7) << 4), r1 + 8 * k);
-        }
+        for (int k = 0; k < 4; ++k)
+          st_f16x8(sm + SM_P + b2 * 8192 + r * 128 + ((((4 * chh + k) ^ r) & 7) << 4), r0 + 8 * k);
       } else {  // A row r = beta_r (KE KH^T)_rs; the solve reads only its strictly lower part
-        const int r = f - CH;
+        const int r = ti - CH;
         const float4 b = make_float4(s_beta[r], s_beta[r], s_beta[r], s_beta[r]);
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          *reinterpret_cast<float4*>(sm + SM_A + a_off(r, 4 * u)) =
+        for (int u = 0; u < 8; ++u)
+          *reinterpret_cast<float4*>(sm + SM_A + a_off(r, 32 * chh + 4 * u)) =
               mul4(make_float4(r0[4 * u], r0[4 * u + 1], r0[4 * u + 2], r0[4 * u + 3]), b);
-          *reinterpret_cast<float4*>(sm + SM_A + a_off(r, 32 + 4 * u)) =
-              mul4(make_float4(r1[4 * u], r1[4 * u + 1], r1[4 * u + 2], r1[4 * u + 3]), b);
-        }
       }
       tc_fence_before();
     }
     fence_proxy_async_smem();  // P is read by the D2 UMMA
     if (dmp) {
-      named_sync(GRP_FRONT, GRP);
+      named_sync(GRP_FRONT, FRONT_T);
       dump_pa(x.dbg, sm, b2, f);
     }
-    named_sync(GRP_FRONT, GRP);  // the front's TMEM reads are done before the next G1
+    named_sync(GRP_FRONT, FRONT_T);  // the front's TMEM reads are done before the next G1
     mbar_arrive(&x.bars[B_FR0 + b2]);
     if (f == 0) tmark(x, c, 26);
     load_g(c + 1, gv, bv);
@@ -671,7 +668,7 @@ __device__ void front_group(const Ctx& x, const float* __restrict__ g, const flo
 }
 
 __device__ void back_group(const Ctx& x) {
-  const int k = threadIdx.x - 256;  // 0..127
+  const int k = threadIdx.x - BACK0;  // 0..127
   const int bw = k >> 5, lane = k & 31;
   const uint32_t tl = x.tmem + ((uint32_t)(bw * 32) << 16);
   const int ti = bw * 32 + lane;  // this thread's TMEM lane
@@ -1202,7 +1199,7 @@ __global__ void __launch_bounds__(NTHR, 1)
   if (tid == 0) {
     *s_t0 = clock64();
     for (int i = 0; i < NUM_BARS; ++i)
-      mbar_init(&x.bars[i], (i == B_GC0 || i == B_GC1 || i == B_OPS0 || i == B_OPS1 || i == B_FR0 || i == B_FR1) ? GRP : 1);
+      mbar_init(&x.bars[i], (i == B_GC0 || i == B_GC1 || i == B_OPS0 || i == B_OPS1 || i == B_FR0 || i == B_FR1) ? FRONT_T : 1);
     fence_mbar_init();
     *x.abort = 0;
     prefetch_tmap(&tm_q);
@@ -1227,9 +1224,9 @@ __global__ void __launch_bounds__(NTHR, 1)
   if (warp < 4) {
     scan_group(x, &tm_q, &tm_k, &tm_v, &tm_o, init, out, fin, sbase, inject_stuck != 0, cnt);
     if (tid == 0) { s_cnt[0] = cnt[0]; s_cnt[1] = cnt[1]; }
-  } else if (warp < 8) {
+  } else if (warp < 12) {
     front_group(x, g, beta, &tm_g, cnt);
-    if (tid == 128) { s_cnt[2] = cnt[0]; s_cnt[3] = cnt[1]; }
+    if (tid == (int)FRONT0) { s_cnt[2] = cnt[0]; s_cnt[3] = cnt[1]; }
   } else {
     back_group(x);
   }
@@ -1237,8 +1234,8 @@ __global__ void __launch_bounds__(NTHR, 1)
   // Drain: every UMMA issued by a group's elected thread has completed, and
   // (on the error path) every TMA load in flight has landed, before TMEM is
   // released and the block exits.
-  if (tid == 0 || tid == 128 || tid == 256) {
-    uint64_t* db = &x.bars[tid == 0 ? B_DRAIN_SG : (tid == 128 ? B_DRAIN_F : B_DRAIN_B)];
+  if (tid == 0 || tid == (int)FRONT0 || tid == (int)BACK0) {
+    uint64_t* db = &x.bars[tid == 0 ? B_DRAIN_SG : (tid == (int)FRONT0 ? B_DRAIN_F : B_DRAIN_B)];
     umma_commit(db);
     mbar_wait(db, 0, WAIT_NS);
   }
