@@ -29,12 +29,13 @@
 // operand overflow (V, S', W', the Gram tiles) reaches Δ as inf or NaN, so
 // the range test is made once, on Δ, with a NaN-propagating maximum.
 //
-// Work split (one CTA per (sequence, head) chain, chunks in order), three
-// groups of four warps:
-//   warps 4-7, "front" group: for chunk c+2 — cumulative decay fused with
+// Work split (one CTA of 16 warps per (sequence, head) chain, chunks in
+// order), three groups:
+//   warps 4-11, "front" group: for chunk c+2 — cumulative decay fused with
 //     the operand scaling, the G1 Gram UMMA, and the P / A tiles;
-//   warps 8-11, "back" group: for chunk c+1 — the triangular solve on CUDA
-//     cores, G2/G3 UMMAs for W'^T and U^T, and the W'^T store;
+//   warps 12-15, "back" group: for chunk c+1 — the triangular solve (CUDA
+//     cores and warp-level tf32 MMAs), G2/G3 UMMAs for W'^T and U^T, and the
+//     W'^T store;
 //   warps 0-3, "scan" group (SG): for chunk c — the state recurrence:
 //     decay S^T, D1 = { O^T = S'^T QE^T ;  Δ^T = U^T - S'^T W'^T }, Δ^T to
 //     fp16, D2 = { S^T += Δ^T KH ;  O^T += Δ^T P^T }, output store.
@@ -324,12 +325,13 @@ __device__ __forceinline__ int chunk_valid(const Ctx& x, int c) {
 }
 
 // ============================================== front and back groups
-// Two 128-thread groups share the chunk prologue and run one chunk apart:
-// while the back group finishes chunk c, the front group starts chunk c+1.
-//   front (warps 4-7): decay prefix fused with operand scaling, the G1 Gram
-//     UMMA, and the P / A tiles;
-//   back (warps 8-11): the triangular solve, T', the G2/G3 UMMAs and W'^T.
-// Row-wise front work: thread f owns rows 8 (f / 16) .. + 7 and channels
+// Two groups share the chunk prologue and run one chunk apart: while the
+// back group finishes chunk c, the front group starts chunk c+1.
+//   front (warps 4-11, 256 threads): decay prefix fused with operand
+//     scaling, the G1 Gram UMMA, and the P / A tiles;
+//   back (warps 12-15, 128 threads): the triangular solve, T', the G2/G3
+//     UMMAs and W'^T.
+// Row-wise front work: thread f owns rows 4 (f / 16) .. + 3 and channels
 // 8 (f % 16) .. + 7, so every tile access is 16 bytes wide.  TMEM work: a
 // warp reads the lane quarter (warp index mod 4) it is allowed to access.
 constexpr int GRP = 128;  // threads of the scan and back groups
