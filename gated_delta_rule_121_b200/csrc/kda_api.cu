@@ -72,6 +72,8 @@ static kda_status_t fwd_impl(const void* q, const void* k, const void* v, const 
   if (cu_seqlens && !aligned16(cu_seqlens)) return KDA_ERR_INVALID_ARG;
   if (!workspace || !aligned16(workspace) || workspace_bytes < kda_fwd_workspace_size(B, T, H, dk, dv, dt))
     return KDA_ERR_WORKSPACE;
+  // Token coordinates are 32-bit in the kernels (TMA tile coordinates).
+  if ((cu_seqlens ? T : (int64_t)B * T) > (int64_t)INT32_MAX) return KDA_ERR_UNSUPPORTED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   kda::DeviceStatus* status = reinterpret_cast<kda::DeviceStatus*>(workspace);
   if (cudaMemsetAsync(status, 0, sizeof(kda::DeviceStatus), s) != cudaSuccess) return KDA_ERR_CUDA;

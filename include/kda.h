@@ -38,6 +38,8 @@
  *     unit of transfer).
  *   - Alignment: every pointer must be 16-byte aligned (KDA_ERR_INVALID_ARG).
  *   - Sizes: dk, dv in {16, 32, 64, 128} (else KDA_ERR_UNSUPPORTED).
+ *   - The total token count (B*T, or T when packed) must be below 2^31
+ *     (else KDA_ERR_UNSUPPORTED).
  *   - Aliasing: out must not overlap any input.  final_state may alias
  *     init_state exactly (in-place chaining).
  */

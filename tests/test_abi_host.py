@@ -73,6 +73,12 @@ def test_fwd_rejects_invalid_arguments(kw, code):
     assert _fwd(**kw) == code
 
 
+def test_fwd_rejects_more_than_2_31_tokens():
+    """The batched token count B*T must fit the kernels' 32-bit token index."""
+    assert _fwd(B=3, T=1 << 30, ws=P(4096), wsb=1024) == kda.KDA_ERR_UNSUPPORTED
+    assert _fwd(B=1, T=(1 << 31), wsb=1024) == kda.KDA_ERR_UNSUPPORTED
+
+
 def test_decode_rejects_invalid_arguments():
     L = kda.lib()
     ok = [P(256), P(512), P(768), P(1024), P(1280), P(1536), P(2048)]
