@@ -92,6 +92,37 @@ def test_bf16_other_dims(dk, dv):
     check(inp, torch.bfloat16, what=f"bf16 dk{dk} dv{dv}")
 
 
+def test_final_state_may_alias_init_state():
+    """In-place chaining: final_state given as the init_state tensor itself."""
+    inp = synth.make_prefill(synth.MID, DEV, T=300, B=2, H=3)
+    ref_out, ref_fin = run_gpu(inp)
+    state = inp["init_state"].clone()
+    out, fin = kda.kda_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], state, None, final_state=state)
+    torch.cuda.synchronize()
+    assert fin.data_ptr() == state.data_ptr()
+    assert torch.equal(out, ref_out) and torch.equal(fin, ref_fin)
+
+
+def test_many_short_packed_sequences():
+    """200 packed sequences of 0..300 tokens: partial chunks everywhere and the
+    longest-first order over many length buckets."""
+    g = torch.Generator().manual_seed(77)
+    lengths = torch.randint(0, 301, (200,), generator=g).tolist()
+    lengths[3] = 0
+    lengths[7] = 1
+    inp = synth.make_prefill(synth.VARLEN, DEV, H=2, lengths=lengths)
+    check(inp, torch.bfloat16, what="200 short packed sequences")
+
+
+def test_batched_zero_tokens_returns_init_state():
+    inp = synth.make_prefill(synth.MID, DEV, T=64, B=2, H=2)
+    e = lambda t: t[:, :0].contiguous()
+    out, fin = kda.kda_fwd(e(inp["q"]), e(inp["k"]), e(inp["v"]), e(inp["g"]), e(inp["beta"]), inp["init_state"])
+    torch.cuda.synchronize()
+    assert out.shape[1] == 0
+    assert torch.equal(fin, inp["init_state"])
+
+
 def test_no_final_state_and_zero_init():
     inp = synth.make_prefill(synth.MID, DEV, T=200, B=1, H=2)
     out, fin = kda.kda_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], None, None,
