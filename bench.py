@@ -380,6 +380,44 @@ def bench_e2e(args, d, dev, stream, inp, kda, th):
             "d2h_bytes_per_step": d2h, "steps": steps, "ms_per_step": d.max(sec) / steps * 1e3}
 
 
+# Phase boundaries recorded by the tensor-core kernel's test hook (chain 0):
+# (name, from event, to event) per group; see include/kda_testing.h.
+PHASES = {
+    "front": [("decay_prefix", 0, 1), ("stage_wait", 1, 2), ("scale_q_k_v", 2, 3), ("buffer_wait", 3, 4),
+              ("kh", 4, 5), ("g1_issue", 5, 6), ("g1_wait", 6, 7), ("p_a_tiles", 7, 26)],
+    "back": [("front_wait", 16, 17), ("diag_inverses", 17, 18), ("y_f", 18, 19), ("x", 19, 20),
+             ("t10_tprime", 20, 21), ("g2_g3_issue", 21, 22), ("g2_g3_wait", 22, 23), ("w_tile", 23, 25)],
+    "scan": [("d2_wait", 8, 9), ("s_pass", 9, 10), ("d1a", 10, 27), ("back_wait", 27, 24), ("d1b", 24, 11),
+             ("tma", 11, 28), ("d1_wait", 28, 13), ("delta", 13, 14), ("d2_issue", 14, 15), ("output", 15, 12)],
+}
+
+
+def run_phases(args):
+    """Per-phase SM cycles of chain 0 (chunks 8..59), from the test hook."""
+    import numpy as np
+    import torch
+
+    import gated_delta_rule_121_b200 as kda
+    import synth
+    spec = workload_spec(args.workload)
+    inp = synth.make_prefill(spec, torch.device("cuda"))
+    dbg = torch.zeros(kda.lib().kda_testing_debug_floats(), dtype=torch.float32, device="cuda")
+    for _ in range(args.warmup):
+        kda.kda_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["init_state"], inp["cu_seqlens"],
+                    _debug=dbg)
+    torch.cuda.synchronize()
+    t = dbg[61568:].cpu().numpy().view(np.int64).reshape(64, 32)
+    cu = inp["cu_seqlens"]
+    n0 = int(cu[1] - cu[0]) if cu is not None else inp["q"].shape[1]
+    hi = min(60, (n0 + CHUNK - 1) // CHUNK)  # chunks of chain 0 with timestamps, skipping the ramp
+    lo = min(8, hi // 2)
+    res = {"workload": spec.name, "chunks": [lo, hi], "unit": "SM cycles per chunk (chain 0)"}
+    for grp, ph in PHASES.items():
+        res[grp] = {n: float(np.mean(t[lo:hi, b] - t[lo:hi, a])) for n, a, b in ph}
+    res["period"] = float(np.mean(np.diff(t[lo:hi, 0])))
+    print(json.dumps(res), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -390,10 +428,14 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--phases", action="store_true",
+                    help="print per-phase cycles of the tensor-core kernel (test hook) instead of timing")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
     d = Dist()
-    if args.impl == "reference":
+    if args.phases:
+        run_phases(args)
+    elif args.impl == "reference":
         run_reference(args, d)
     else:
         run_native(args, d)

@@ -19,9 +19,18 @@ KDA_API int kda_testing_debug_floats(void);
  * Same as kda_fwd, plus:
  *   debug_out  device fp32 buffer of kda_testing_debug_floats() floats or
  *              NULL.  When set (tensor-core path only, else
- *              KDA_ERR_UNSUPPORTED), the block of chain 0 writes the
- *              intermediates of its first chunk: P, A, T', W, U, Delta, O,
- *              the state after the chunk and the chunk-total log-decay.
+ *              KDA_ERR_UNSUPPORTED), the block of chain 0 (sequence 0, head 0)
+ *              writes the intermediates of its first chunk, row-major fp32
+ *              at these float offsets: P [64][64] at 0, A [64][64] at 4096
+ *              (strictly lower part), T' [64][64] at 8192, W' [64][128] at
+ *              12288 (W' = W Diag(exp(-G_C)), the chunk-end-referenced
+ *              pseudo-keys), U [64][128] at 20480, Delta [64][128] at 28672,
+ *              O [64][128] at 36864, the state after the chunk [128][128] at
+ *              45056, the chunk-total log-decay G_C [128] at 61440; and, as
+ *              int64 from float offset 61568, [64 chunks][32 events] of SM
+ *              clock cycles since the block started: phase boundaries of
+ *              the first 64 chunks (events 0-7 and 26: front group; 16-23
+ *              and 25: back group; 8-15, 24, 27, 28: scan group).
  *   wait_ns    bound for every device-side wait in nanoseconds (kda_fwd
  *              uses 2e9).
  *   inject_stuck  when nonzero (tensor-core path), the scan warps of every
