@@ -347,58 +347,58 @@ __device__ __forceinline__ void general_gram(const Ctx& x, int b2, int valid, co
   const float* s_beta = reinterpret_cast<const float*>(sm + SM_MISC + MS_BETA) + b2 * 64;
   const int r = f & 63, s0 = (f >> 6) * 16;  // row r, columns s0 .. s0 + 15
   const uint8_t* stp = sm + b2 * STAGE_BYTES;
-  float pa[16], aa[16];
+  const float br = s_beta[r];
+  float4 ak[4];  // A row r, columns s0 + 4 ib .. + 3 (the A tile holds the staged G until the end)
+  // Blocks of 4 columns, each over both channel halves: the 8 accumulators
+  // of a block have fixed indices and stay in registers.
 #pragma unroll
-  for (int i = 0; i < 16; ++i) pa[i] = aa[i] = 0.f;
-  for (int half = 0; half < 2; ++half) {
-    named_sync(GRP_FRONT, FRONT_T);  // earlier readers of the staging tile are done
-    if (hh == half) {
-      F8 gr = f8(0.f);
+  for (int ib = 0; ib < 4; ++ib) {
+    float p4[4] = {0.f, 0.f, 0.f, 0.f}, a4[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int half = 0; half < 2; ++half) {
+      named_sync(GRP_FRONT, FRONT_T);  // earlier readers of the staging tile are done
+      if (hh == half) {
+        F8 gr = f8(0.f);
 #pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        gr = add8(gr, gv[m]);
-        *reinterpret_cast<float4*>(sm + SM_A + (4 * rg + m) * 256 + cc * 4) = gr.a;
-        *reinterpret_cast<float4*>(sm + SM_A + (4 * rg + m) * 256 + cc * 4 + 16) = gr.b;
+        for (int m = 0; m < 4; ++m) {
+          gr = add8(gr, gv[m]);
+          *reinterpret_cast<float4*>(sm + SM_A + (4 * rg + m) * 256 + cc * 4) = gr.a;
+          *reinterpret_cast<float4*>(sm + SM_A + (4 * rg + m) * 256 + cc * 4 + 16) = gr.b;
+        }
       }
-    }
-    named_sync(GRP_FRONT, FRONT_T);
-    if (r < valid && s0 <= r) {
+      named_sync(GRP_FRONT, FRONT_T);
+      if (r < valid && s0 + 4 * ib <= r) {
 #pragma unroll 1
-      for (int ch = 0; ch < 64; ++ch) {
-        const uint32_t off_r = half * 16384 + sw128_off(r, ch);
-        const float gr = *reinterpret_cast<const float*>(sm + SM_A + r * 256 + ch * 4);
-        const float qr = ld_bf16(stp + OFF_QK + off_r), kr = ld_bf16(stp + OFF_QK + 8192 + off_r);
-#pragma unroll 4
-        for (int i = 0; i < 16; ++i) {
-          const int s = s0 + i;
-          if (s <= r) {
-            const float gs = *reinterpret_cast<const float*>(sm + SM_A + s * 256 + ch * 4);
-            const float ks = ld_bf16(stp + OFF_QK + 8192 + half * 16384 + sw128_off(s, ch));
-            const float e = ex2(gr - gs) * ks;
-            pa[i] += qr * e;
-            aa[i] += kr * e;
+        for (int ch = 0; ch < 64; ++ch) {
+          const uint32_t off_r = half * 16384 + sw128_off(r, ch);
+          const float gr = *reinterpret_cast<const float*>(sm + SM_A + r * 256 + ch * 4);
+          const float qr = ld_bf16(stp + OFF_QK + off_r), kr = ld_bf16(stp + OFF_QK + 8192 + off_r);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int s = s0 + 4 * ib + e;
+            if (s <= r) {
+              const float gs = *reinterpret_cast<const float*>(sm + SM_A + s * 256 + ch * 4);
+              const float ks = ld_bf16(stp + OFF_QK + 8192 + half * 16384 + sw128_off(s, ch));
+              const float ef = ex2(gr - gs) * ks;
+              p4[e] += qr * ef;
+              a4[e] += kr * ef;
+            }
           }
         }
       }
     }
-  }
-  const float br = s_beta[r];
+    // P row r, these 4 columns (lower triangle including the diagonal), as fp16.
+    const int s = s0 + 4 * ib;
+    float pv[4];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const int s = s0 + i;
-    aa[i] = s < r ? br * aa[i] : 0.f;
-    if (!(s <= r)) pa[i] = 0.f;
+    for (int e = 0; e < 4; ++e) pv[e] = (s + e <= r) ? p4[e] : 0.f;
+    *reinterpret_cast<uint2*>(sm + SM_P + b2 * 8192 + r * 128 + ((((s >> 3) ^ r) & 7) << 4) + (s & 7) * 2) =
+        make_uint2(pack_f16x2(pv[0], pv[1]), pack_f16x2(pv[2], pv[3]));
+    ak[ib] = make_float4(s < r ? br * a4[0] : 0.f, s + 1 < r ? br * a4[1] : 0.f, s + 2 < r ? br * a4[2] : 0.f,
+                         s + 3 < r ? br * a4[3] : 0.f);
   }
   named_sync(GRP_FRONT, FRONT_T);  // every staged G read is done before A overwrites the tile
 #pragma unroll
-  for (int q8 = 0; q8 < 2; ++q8) {
-    const int s = s0 + 8 * q8;
-    st_f16x8(sm + SM_P + b2 * 8192 + r * 128 + ((((s >> 3) ^ r) & 7) << 4), pa + 8 * q8);
-  }
-#pragma unroll
-  for (int u = 0; u < 4; ++u)
-    *reinterpret_cast<float4*>(sm + SM_A + a_off(r, s0 + 4 * u)) =
-        make_float4(aa[4 * u], aa[4 * u + 1], aa[4 * u + 2], aa[4 * u + 3]);
+  for (int ib = 0; ib < 4; ++ib) *reinterpret_cast<float4*>(sm + SM_A + a_off(r, s0 + 4 * ib)) = ak[ib];
   named_sync(GRP_FRONT, FRONT_T);  // raw Q/K reads are done before they are rescaled in place
 }
 
