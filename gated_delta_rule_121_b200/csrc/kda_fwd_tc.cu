@@ -340,6 +340,12 @@ constexpr int GRP = 128;  // threads of the scan and back groups
 // G_r - G_s (log2 units), G staged through the A tile one channel half at a
 // time (the back group has released the A tile).  Raw Q and K are read from
 // the stage before they are rescaled in place.
+// Staged G (one 64-channel half): row r, channel ch, with the 16-byte units of
+// each row rotated by the row so that a warp reading one channel of 32 rows
+// touches 16 different units.
+__device__ __forceinline__ uint32_t g_off(int r, int ch) {
+  return (uint32_t)r * 256u + ((((uint32_t)ch >> 2) + (uint32_t)r) & 15u) * 16u + ((uint32_t)ch & 3u) * 4u;
+}
 __device__ __forceinline__ void general_gram(const Ctx& x, int b2, int valid, const F8 (&gv)[4]) {
   const int f = threadIdx.x - FRONT0;
   const int rg = f >> 4, ch0 = 8 * (f & 15), hh = ch0 >> 6, cc = ch0 & 63;
@@ -361,22 +367,22 @@ __device__ __forceinline__ void general_gram(const Ctx& x, int b2, int valid, co
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
           gr = add8(gr, gv[m]);
-          *reinterpret_cast<float4*>(sm + SM_A + (4 * rg + m) * 256 + cc * 4) = gr.a;
-          *reinterpret_cast<float4*>(sm + SM_A + (4 * rg + m) * 256 + cc * 4 + 16) = gr.b;
+          *reinterpret_cast<float4*>(sm + SM_A + g_off(4 * rg + m, cc)) = gr.a;
+          *reinterpret_cast<float4*>(sm + SM_A + g_off(4 * rg + m, cc + 4)) = gr.b;
         }
       }
       named_sync(GRP_FRONT, FRONT_T);
       if (r < valid && s0 + 4 * ib <= r) {
-#pragma unroll 1
+#pragma unroll 2
         for (int ch = 0; ch < 64; ++ch) {
           const uint32_t off_r = half * 16384 + sw128_off(r, ch);
-          const float gr = *reinterpret_cast<const float*>(sm + SM_A + r * 256 + ch * 4);
+          const float gr = *reinterpret_cast<const float*>(sm + SM_A + g_off(r, ch));
           const float qr = ld_bf16(stp + OFF_QK + off_r), kr = ld_bf16(stp + OFF_QK + 8192 + off_r);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int s = s0 + 4 * ib + e;
             if (s <= r) {
-              const float gs = *reinterpret_cast<const float*>(sm + SM_A + s * 256 + ch * 4);
+              const float gs = *reinterpret_cast<const float*>(sm + SM_A + g_off(s, ch));
               const float ks = ld_bf16(stp + OFF_QK + 8192 + half * 16384 + sw128_off(s, ch));
               const float ef = ex2(gr - gs) * ks;
               p4[e] += qr * ef;
