@@ -176,10 +176,6 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       :: "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
       : "memory");
 }
-__device__ __forceinline__ void tmem_wait_ld() {
-  __syncwarp();
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
 __device__ __forceinline__ void tmem_wait_st() {
   __syncwarp();
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
@@ -199,17 +195,6 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
   return d;
 }
 
-// Instruction descriptor, kind::f16 with bf16 A/B and fp32 accumulation.
-// a_mn / b_mn select MN-major (1) or K-major (0) operands.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn, int b_mn) {
-  return (1u << 4)                      // D format: f32
-         | (1u << 7)                    // A format: bf16
-         | (1u << 10)                   // B format: bf16
-         | ((uint32_t)a_mn << 15)       // A major
-         | ((uint32_t)b_mn << 16)       // B major
-         | ((uint32_t)(N >> 3) << 17)   // N / 8
-         | ((uint32_t)(M >> 4) << 24);  // M / 16
-}
 
 // D[tmem] (+)= A[smem] * B[smem]^T, issued by one thread (operand types come
 // from the instruction descriptor).
