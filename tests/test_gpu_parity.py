@@ -56,6 +56,14 @@ def test_mid_prefill_full():
     print("mid errors", eo, ef)
 
 
+def test_mid_prefill_fp32():
+    """The mid shape with fp32 q/k/v (the CUDA-core path) at the 1e-4 bar."""
+    spec = synth.PrefillSpec("mid_fp32", 2, 4096, 16, 128, 128, torch.float32, 13, init=True)
+    inp = synth.make_prefill(spec, DEV)
+    eo, ef = check(inp, torch.float32, what="mid fp32")
+    print("mid fp32 errors", eo, ef)
+
+
 def test_stress_model_range_decay():
     """g = -5 sigmoid(z): chunk totals far below the factorisation floor."""
     inp = synth.make_prefill(synth.STRESS, DEV)
