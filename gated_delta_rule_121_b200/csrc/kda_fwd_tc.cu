@@ -19,9 +19,11 @@
 // up to exp(-G_C): with the digest's bounded decay ("Bounded decay" section,
 // g >= -5) every tile is a dense matmul as long as a chunk's total decay is
 // moderate.  A chunk whose total decay in some channel is below 2^-10 takes
-// the general variant: its Gram matrices P, A come from CUDA cores using the
-// exact differences G_r - G_s, the operands use the chunk START as reference
-// (QE = Q e^G, KE = K e^G), and the scan decays S only after D1.
+// the general variant: its Gram matrices P, A come from six tensor-core
+// Grams whose decay references sit at block boundaries between the two
+// tokens of every pair (so no operand factor exceeds 1), the operands use the
+// chunk START as reference (QE = Q e^G, KE = K e^G), and the scan decays S
+// only after D1.
 //
 // Operands are fp16 (10-bit mantissa) with fp32 accumulation: the fp32
 // state and every product stay accurate to well inside the bf16 output's own
@@ -92,7 +94,8 @@ constexpr uint32_t MS_T0 = 224;  // int64: clock at block start (timing dump)
 constexpr uint32_t MS_BETA = 256;    // [2][64] fp32
 constexpr uint32_t MS_GC = 768;      // [2][128] fp32: exp(G_C)
 constexpr uint32_t MS_RED = 1792;    // [8][128] fp32 log2 sums
-constexpr uint32_t MS_END = 5888;
+constexpr uint32_t MS_DIAG = 5888;   // [64] fp32: q_r . k_r (general chunks)
+constexpr uint32_t MS_END = 6144;
 static_assert(NUM_BARS * 8 <= MS_TMEM, "barrier area");
 static_assert(MS_END <= MISC_BYTES, "misc area");
 
@@ -336,76 +339,163 @@ __device__ __forceinline__ int chunk_valid(const Ctx& x, int c) {
 // warp reads the lane quarter (warp index mod 4) it is allowed to access.
 constexpr int GRP = 128;  // threads of the scan and back groups
 
-// General chunks: P and A on CUDA cores from the exact decay differences
-// G_r - G_s (log2 units), G staged through the A tile one channel half at a
-// time (the back group has released the A tile).  Raw Q and K are read from
-// the stage before they are rescaled in place.
-// Staged G (one 64-channel half): row r, channel ch, with the 16-byte units of
-// each row rotated by the row so that a warp reading one channel of 32 rows
-// touches 16 different units.
-__device__ __forceinline__ uint32_t g_off(int r, int ch) {
-  return (uint32_t)r * 256u + ((((uint32_t)ch >> 2) + (uint32_t)r) & 15u) * 16u + ((uint32_t)ch & 3u) * 4u;
+// P (fp16, lower triangle with the diagonal) and A (fp32, beta-scaled; the
+// solve reads only its strictly lower part) from one 32-column slice of
+// [P ; A_raw] per thread: TMEM lane ti (row ti of [P ; A_raw]), columns
+// 32 chh .. 32 chh + 31.
+__device__ __forceinline__ void store_pa(uint8_t* sm, int b2, int ti, int chh, const float* s_beta,
+                                         float (&r0)[32]) {
+  if (ti < CH) {  // P row ti
+    const int r = ti;
+#pragma unroll
+    for (int s = 0; s < 32; ++s)
+      if (chh * 32 + s > r) r0[s] = 0.f;
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      st_f16x8(sm + SM_P + b2 * 8192 + r * 128 + ((((4 * chh + k) ^ r) & 7) << 4), r0 + 8 * k);
+  } else {  // A row r = beta_r (row r of the decayed K K^T)
+    const int r = ti - CH;
+    const float4 b = make_float4(s_beta[r], s_beta[r], s_beta[r], s_beta[r]);
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      *reinterpret_cast<float4*>(sm + SM_A + a_off(r, 32 * chh + 4 * u)) =
+          mul4(make_float4(r0[4 * u], r0[4 * u + 1], r0[4 * u + 2], r0[4 * u + 3]), b);
+  }
 }
-__device__ __forceinline__ void general_gram(const Ctx& x, int b2, int valid, const F8 (&gv)[4]) {
+
+// General chunks (total decay of the chunk below the end-referenced range in
+// some channel): P and A on the tensor cores with the reference of every
+// decay factor placed between the two tokens it connects, so that no operand
+// is scaled by more than 1.  Level p = 64, 32, ..., 2 splits the rows into
+// aligned p-blocks with an earlier and a later half and takes as reference
+// R the cumulative decay G at the last row of the earlier half; it scales a
+// later row r by e^{G_r - R} and an earlier row by e^{R - G_r} (both <= 1 for
+// a non-positive log decay), so its Gram [Q ; K] K^T holds the products
+// q_r k_s e^{G_r - G_s} exactly for the pairs r > s that straddle one of its
+// boundaries: those whose highest differing index bit is p/2.  Levels run
+// from p = 64 down; each keeps the pairs with r and s in the same p-block,
+// so the finest level that contains a pair wins.  The diagonal of P (no
+// decay) is the plain q_r . k_r.  Q and K rows scaled for a level go to a
+// tile of the stage layout whose two 64-channel halves are the A tile and
+// KX[b2] (both released: AFREE and BUF were waited for); the row-group end
+// values of G (the references of levels 8..64) are staged in the P tile.
+__device__ __forceinline__ bool level_gram(const Ctx& x, int b2, const F8 (&gv)[4], int& g1_ph) {
   const int f = threadIdx.x - FRONT0;
+  const int wq = f >> 5, lane = f & 31, lq = wq & 3, chh = wq >> 2;
   const int rg = f >> 4, ch0 = 8 * (f & 15), hh = ch0 >> 6, cc = ch0 & 63;
   uint8_t* sm = x.sm;
+  const uint32_t sb = x.sb;
+  float* s_ref = reinterpret_cast<float*>(sm + SM_P + b2 * 8192);  // [16][128]: G at row 4 k + 3
+  float* s_diag = reinterpret_cast<float*>(sm + SM_MISC + MS_DIAG);
   const float* s_beta = reinterpret_cast<const float*>(sm + SM_MISC + MS_BETA) + b2 * 64;
-  const int r = f & 63, s0 = (f >> 6) * 16;  // row r, columns s0 .. s0 + 15
-  const uint8_t* stp = sm + b2 * STAGE_BYTES;
-  const float br = s_beta[r];
-  float4 ak[4];  // A row r, columns s0 + 4 ib .. + 3 (the A tile holds the staged G until the end)
-  // Blocks of 4 columns, each over both channel halves: the 8 accumulators
-  // of a block have fixed indices and stay in registers.
+  const uint8_t* qb = sm + b2 * STAGE_BYTES + OFF_QK + hh * 16384;
+  const uint8_t* kb = qb + 8192;
+  uint8_t* lt = sm + (hh ? SM_KX + b2 * 16384 : SM_A);  // this thread's channel half of the level tile
+  const uint32_t tl = x.tmem + ((uint32_t)(lq * 32) << 16);
+  const int ti = 32 * lq + lane, r = ti & 63;
+
+  {  // G at the end of this thread's row group, and the raw diagonal q_r . k_r
+    const F8 ge = add8(add8(add8(gv[0], gv[1]), gv[2]), gv[3]);
+    *reinterpret_cast<float4*>(s_ref + rg * 128 + ch0) = ge.a;
+    *reinterpret_cast<float4*>(s_ref + rg * 128 + ch0 + 4) = ge.b;
+    float d[4];
 #pragma unroll
-  for (int ib = 0; ib < 4; ++ib) {
-    float p4[4] = {0.f, 0.f, 0.f, 0.f}, a4[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int half = 0; half < 2; ++half) {
-      named_sync(GRP_FRONT, FRONT_T);  // earlier readers of the staging tile are done
-      if (hh == half) {
-        F8 gr = f8(0.f);
+    for (int m = 0; m < 4; ++m) {
+      const uint32_t o = sw128_off(4 * rg + m, cc);
+      const F8 qv = bf16x8_to_f32(*reinterpret_cast<const uint4*>(qb + o));
+      const F8 kv = bf16x8_to_f32(*reinterpret_cast<const uint4*>(kb + o));
+      const F8 pr = mul8(qv, kv);
+      d[m] = ((pr.a.x + pr.a.y) + (pr.a.z + pr.a.w)) + ((pr.b.x + pr.b.y) + (pr.b.z + pr.b.w));
+    }
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          gr = add8(gr, gv[m]);
-          *reinterpret_cast<float4*>(sm + SM_A + g_off(4 * rg + m, cc)) = gr.a;
-          *reinterpret_cast<float4*>(sm + SM_A + g_off(4 * rg + m, cc + 4)) = gr.b;
-        }
+    for (int o = 1; o < 16; o <<= 1)
+#pragma unroll
+      for (int m = 0; m < 4; ++m) d[m] += __shfl_xor_sync(0xffffffffu, d[m], o);
+    if ((f & 15) == 0) {
+#pragma unroll
+      for (int m = 0; m < 4; ++m) s_diag[4 * rg + m] = d[m];
+    }
+  }
+  named_sync(GRP_FRONT, FRONT_T);
+
+  float acc[32];
+#pragma unroll
+  for (int L = 6; L >= 1; --L) {
+    const int p = 1 << L;
+    // ---- this level's scaled rows: row 4 rg + m times 2^{x_m} (log2 units)
+    F8 dr = f8(0.f);  // G_r - R, running over this thread's rows
+    bool later = false;
+    if (L >= 3) {  // reference R: the end of row group kref (another thread's rows)
+      const int kref = (rg & ~(p / 4 - 1)) + p / 8 - 1;
+      const F8 R = {*reinterpret_cast<const float4*>(s_ref + kref * 128 + ch0),
+                    *reinterpret_cast<const float4*>(s_ref + kref * 128 + ch0 + 4)};
+      later = ((4 * rg) & (p / 2)) != 0;
+      dr = sub8(f8(0.f), R);
+    }
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const uint32_t o = sw128_off(4 * rg + m, cc);
+      F8 e;
+      if (L >= 3) {
+        dr = add8(dr, gv[m]);
+        e = ex2_8(later ? dr : sub8(f8(0.f), dr));
+      } else if (L == 2) {  // reference: row 4 rg + 1
+        e = m == 1 ? f8(1.f) : ex2_8(m == 0 ? gv[1] : (m == 2 ? gv[2] : add8(gv[2], gv[3])));
+      } else {  // references: rows 4 rg and 4 rg + 2
+        e = (m & 1) == 0 ? f8(1.f) : ex2_8(m == 1 ? gv[1] : gv[3]);
       }
-      named_sync(GRP_FRONT, FRONT_T);
-      if (r < valid && s0 + 4 * ib <= r) {
-#pragma unroll 2
-        for (int ch = 0; ch < 64; ++ch) {
-          const uint32_t off_r = half * 16384 + sw128_off(r, ch);
-          const float gr = *reinterpret_cast<const float*>(sm + SM_A + g_off(r, ch));
-          const float qr = ld_bf16(stp + OFF_QK + off_r), kr = ld_bf16(stp + OFF_QK + 8192 + off_r);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int s = s0 + 4 * ib + e;
-            if (s <= r) {
-              const float gs = *reinterpret_cast<const float*>(sm + SM_A + g_off(s, ch));
-              const float ks = ld_bf16(stp + OFF_QK + 8192 + half * 16384 + sw128_off(s, ch));
-              const float ef = ex2(gr - gs) * ks;
-              p4[e] += qr * ef;
-              a4[e] += kr * ef;
-            }
-          }
-        }
+      for (int hq = 0; hq < 2; ++hq) {  // 4 channels at a time
+        const float4 eh = hq ? e.b : e.a;
+        const uint2 qh = *reinterpret_cast<const uint2*>(qb + o + 8 * hq);
+        const uint2 kh = *reinterpret_cast<const uint2*>(kb + o + 8 * hq);
+        st_f16x4(lt + o + 8 * hq, mul4(bf16x4_to_f32(qh), eh));
+        st_f16x4(lt + 8192 + o + 8 * hq, mul4(bf16x4_to_f32(kh), eh));
       }
     }
-    // P row r, these 4 columns (lower triangle including the diagonal), as fp16.
-    const int s = s0 + 4 * ib;
-    float pv[4];
+    fence_proxy_async_smem();
+    tc_fence_before();
+    named_sync(GRP_FRONT, FRONT_T);  // tile written; the previous level's TMEM reads are done
+    // ---- [Q ; K] K^T of the level tile (M=128, N=64, K=128) -> TM_G
+    if (f == 0) {
+      tc_fence_after();
+      const uint32_t id = idesc_f16_f32(128, 64, 0, 0);
 #pragma unroll
-    for (int e = 0; e < 4; ++e) pv[e] = (s + e <= r) ? p4[e] : 0.f;
-    *reinterpret_cast<uint2*>(sm + SM_P + b2 * 8192 + r * 128 + ((((s >> 3) ^ r) & 7) << 4) + (s & 7) * 2) =
-        make_uint2(pack_f16x2(pv[0], pv[1]), pack_f16x2(pv[2], pv[3]));
-    ak[ib] = make_float4(s < r ? br * a4[0] : 0.f, s + 1 < r ? br * a4[1] : 0.f, s + 2 < r ? br * a4[2] : 0.f,
-                         s + 3 < r ? br * a4[3] : 0.f);
+      for (int i = 0; i < 8; ++i) {
+        const uint32_t base = (i >> 2) ? sb + SM_KX + b2 * 16384 : sb + SM_A;
+        const uint64_t da = sdesc_sw128(base + (i & 3) * 32, 16, 1024);
+        const uint64_t db = sdesc_sw128(base + 8192 + (i & 3) * 32, 16, 1024);
+        umma_ss(x.tmem + TM_G, da, db, id, i > 0);
+      }
+      umma_commit(&x.bars[B_G1]);
+    }
+    if (!gwait(x, B_G1, g1_ph, 16, GRP_FRONT)) return false;
+    g1_ph ^= 1;
+    tc_fence_after();
+    if (L == 6) {
+      tmem_ld32(tl + TM_G + chh * 32, acc);
+    } else if ((lq & 1) == chh) {  // (warp-uniform) a warp whose rows and columns share a 32-block
+#pragma unroll
+      for (int hv = 0; hv < 4; ++hv) {
+        float val[8];
+        tmem_ld8(tl + TM_G + chh * 32 + hv * 8, val);
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          if ((r >> L) == ((32 * chh + 8 * hv + u) >> L)) acc[8 * hv + u] = val[u];
+      }
+    }
   }
-  named_sync(GRP_FRONT, FRONT_T);  // every staged G read is done before A overwrites the tile
-#pragma unroll
-  for (int ib = 0; ib < 4; ++ib) *reinterpret_cast<float4*>(sm + SM_A + a_off(r, s0 + 4 * ib)) = ak[ib];
-  named_sync(GRP_FRONT, FRONT_T);  // raw Q/K reads are done before they are rescaled in place
+  // Every level's UMMA has completed and every thread is past the last
+  // level's tile barrier, so the P tile (reference table) and the A tile
+  // (level tile half) may be overwritten.
+  store_pa(sm, b2, ti, chh, s_beta, acc);
+  if (ti < CH && (r >> 5) == chh) {  // the diagonal of P
+    const __half h = __float2half_rn(s_diag[r]);
+    *reinterpret_cast<__half*>(sm + SM_P + b2 * 8192 + sw128_off(r, r)) = h;
+  }
+  tc_fence_before();
+  named_sync(GRP_FRONT, FRONT_T);  // TMEM reads done before the next G1; tiles complete before the raw-row rescaling
+  return true;
 }
 
 // Debug dumps (chain 0, chunk 0): P (fp16 tile) and A (fp32 tile); T'; W'
@@ -511,7 +601,7 @@ __device__ void front_group(const Ctx& x, const float* __restrict__ g, const flo
       *reinterpret_cast<float4*>(s_red + wq * 128 + ch0 + 4) = wsum.b;
     }
     named_sync(GRP_FRONT, FRONT_T);
-    F8 tot = f8(0.f), off = (lane >= 16) ? other : f8(0.f);
+    F8 tot = f8(0.f), off = (lane >= 16) ? other : f8(0.f);  // tot: G_C
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
       const F8 v = {*reinterpret_cast<const float4*>(s_red + q * 128 + ch0),
@@ -540,7 +630,7 @@ __device__ void front_group(const Ctx& x, const float* __restrict__ g, const flo
       }
       mbar_arrive(&x.bars[B_GC0 + b2]);  // one arrival per thread, after its own writes
     };
-    if (!fast) {  // the general Gram writes P[b2] and stages G through the A tile first
+    if (!fast) {  // the general Gram works in P[b2], KX[b2] and the A tile
       if (c >= 2 && !gwait(x, B_BUF0 + b2, ((c >> 1) - 1) & 1, 11, GRP_FRONT)) break;
       publish();
       if (c >= 1 && !gwait(x, B_AFREE, (c - 1) & 1, 13, GRP_FRONT)) break;
@@ -548,11 +638,6 @@ __device__ void front_group(const Ctx& x, const float* __restrict__ g, const flo
     if (!gwait(x, B_FULL0 + b2, (c >> 1) & 1, 12, GRP_FRONT)) break;
     ++consumed[b2];
     if (f == 0) tmark(x, c, 2);
-    if (!fast) general_gram(x, b2, valid, gv);
-
-    // ---- (a2) operand scaling, row by row: E = e^{G_r - ref} (ref = G_C on
-    // fast chunks, 0 otherwise), H = e^{G_C - G_r}.  QE, KE and V (fp16) go
-    // in place; KH goes to KX[b2] once the scan of chunk c-2 has released it.
     uint8_t* qb = sm + b2 * STAGE_BYTES + OFF_QK + hh * 16384;
     uint8_t* kb = qb + 8192;
     uint8_t* vb = sm + b2 * STAGE_BYTES + OFF_V + hh * 8192;
@@ -560,7 +645,7 @@ __device__ void front_group(const Ctx& x, const float* __restrict__ g, const flo
     if (valid < CH) {
       // Rows past the end of a sequence's last chunk hold other data: zero
       // this thread's rows and channels of the raw tiles, so the scaling
-      // pass below needs no per-row mask.
+      // pass (and the general Gram) needs no per-row mask.
 #pragma unroll 1
       for (int m = 0; m < 4; ++m) {
         const int r = 4 * rg + m;
@@ -572,6 +657,20 @@ __device__ void front_group(const Ctx& x, const float* __restrict__ g, const flo
         }
       }
     }
+    if (!fast) {
+      if (!level_gram(x, b2, gv, g1_ph)) break;
+      // G_C again from the warp sums (the same additions in the same order),
+      // so that it is not held in registers across the Gram.
+      tot = f8(0.f);
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        tot = add8(tot, F8{*reinterpret_cast<const float4*>(s_red + q * 128 + ch0),
+                           *reinterpret_cast<const float4*>(s_red + q * 128 + ch0 + 4)});
+    }
+
+    // ---- (a2) operand scaling, row by row: E = e^{G_r - ref} (ref = G_C on
+    // fast chunks, 0 otherwise), H = e^{G_C - G_r}.  QE, KE and V (fp16) go
+    // in place; KH goes to KX[b2] once the scan of chunk c-2 has released it.
     uint4 kraw[4];  // raw K rows, kept for KH
     {
       F8 gr = f8(0.f);
@@ -642,25 +741,9 @@ __device__ void front_group(const Ctx& x, const float* __restrict__ g, const flo
       if (f == 0) tmark(x, c, 7);
       // TMEM lane 32 lq + lane is row ti of [P ; A_raw]; this warp reads
       // columns 32 chh .. 32 chh + 31.
-      const int ti = 32 * lq + lane;
       float r0[32];
       tmem_ld32(tl + TM_G + chh * 32, r0);
-      if (lq < 2) {  // P row ti, lower triangle including the diagonal
-        const int r = ti;
-#pragma unroll
-        for (int s = 0; s < 32; ++s)
-          if (chh * 32 + s > r) r0[s] = 0.f;
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          st_f16x8(sm + SM_P + b2 * 8192 + r * 128 + ((((4 * chh + k) ^ r) & 7) << 4), r0 + 8 * k);
-      } else {  // A row r = beta_r (KE KH^T)_rs; the solve reads only its strictly lower part
-        const int r = ti - CH;
-        const float4 b = make_float4(s_beta[r], s_beta[r], s_beta[r], s_beta[r]);
-#pragma unroll
-        for (int u = 0; u < 8; ++u)
-          *reinterpret_cast<float4*>(sm + SM_A + a_off(r, 32 * chh + 4 * u)) =
-              mul4(make_float4(r0[4 * u], r0[4 * u + 1], r0[4 * u + 2], r0[4 * u + 3]), b);
-      }
+      store_pa(sm, b2, 32 * lq + lane, chh, s_beta, r0);
       tc_fence_before();
     }
     fence_proxy_async_smem();  // P is read by the D2 UMMA

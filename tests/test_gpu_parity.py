@@ -174,9 +174,16 @@ def test_packed_varlen_full_size_sampled_heads():
     print("varlen errors", cu.numel() - 1, "sequences", eo, ef)
 
 
-def test_debug_intermediates_match_chunk_model():
+@pytest.mark.parametrize("decay", ["mild", "model_range"])
+def test_debug_intermediates_match_chunk_model(decay):
+    """One chunk's P, A, T', W', U, Δ, O and S against the fp64 chunk model:
+    with mild decay the chunk takes the end-referenced Gram, with model-range
+    decay (g down to -5) the level Gram and start-referenced operands."""
     from chunk_model import chunk_forward
     inp = synth.make_prefill(synth.MID, DEV, T=64, B=1, H=1)
+    if decay == "model_range":
+        inp["g"] = (inp["g"] * 64.0).contiguous()  # -5 sigmoid(z)
+        assert float(inp["g"].sum(1).min()) < -7.0  # chunk total below the end-referenced floor
     dbg = torch.zeros(kda.lib().kda_testing_debug_floats(), dtype=torch.float32, device=DEV)
     out, fin = kda.kda_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["init_state"], _debug=dbg)
     torch.cuda.synchronize()
@@ -188,8 +195,10 @@ def test_debug_intermediates_match_chunk_model():
     checks = [("P", d[0:4096].reshape(64, 64), it["P"]),
               ("A", d[4096:8192].reshape(64, 64), it["A"]),
               ("T'", d[8192:12288].reshape(64, 64), it["T"] * f(inp["beta"])[None, :]),
-              # the kernel stores W' = W Diag(exp(-G_C)) (operands referenced to the chunk end)
-              ("W'", d[12288:20480].reshape(64, 128), it["W"] * np.exp(-it["G"][-1])[None, :]),
+              # fast chunks store W' = W Diag(exp(-G_C)) (operands referenced to the chunk
+              # end), general chunks W' = W (referenced to the chunk start)
+              ("W'", d[12288:20480].reshape(64, 128),
+               it["W"] * (np.exp(-it["G"][-1])[None, :] if decay == "mild" else 1.0)),
               ("U", d[20480:28672].reshape(64, 128), it["U"]),
               ("Delta", d[28672:36864].reshape(64, 128), it["Delta"]),
               ("O", d[36864:45056].reshape(64, 128), O),
