@@ -94,8 +94,8 @@ constexpr uint32_t MS_T0 = 224;  // int64: clock at block start (timing dump)
 constexpr uint32_t MS_BETA = 256;    // [2][64] fp32
 constexpr uint32_t MS_GC = 768;      // [2][128] fp32: exp(G_C)
 constexpr uint32_t MS_RED = 1792;    // [8][128] fp32 log2 sums
-constexpr uint32_t MS_DIAG = 5888;   // [64] fp32: q_r . k_r (general chunks)
-constexpr uint32_t MS_END = 6144;
+constexpr uint32_t MS_PAIRS = 5888;  // [64][8] fp32: P, A of the pairs inside 4-row groups (general chunks)
+constexpr uint32_t MS_END = 7936;
 static_assert(NUM_BARS * 8 <= MS_TMEM, "barrier area");
 static_assert(MS_END <= MISC_BYTES, "misc area");
 
@@ -112,7 +112,7 @@ constexpr uint32_t TMEM_COLS = 512;
 constexpr int DBG_P = 0, DBG_A = 4096, DBG_T = 8192, DBG_W = 12288, DBG_U = 20480, DBG_DELTA = 28672,
               DBG_O = 36864, DBG_S = 45056, DBG_GC = 61440, DBG_TIME = 61568, DBG_FLOATS = 65664;
 // DBG_TIME: int64 [64 chunks][32 events] of SM clock cycles since block start
-// (events 0-6 front group, 16-23 and 25 back group, 8-15 and 24 scan group),
+// (events 0-7, 26, 29, 30 front group, 16-23 and 25 back group, 8-15, 24, 27, 28 scan group),
 // chain 0 only.
 constexpr int TIME_CHUNKS = 64;
 
@@ -366,7 +366,7 @@ __device__ __forceinline__ void store_pa(uint8_t* sm, int b2, int ti, int chh, c
 // General chunks (total decay of the chunk below the end-referenced range in
 // some channel): P and A on the tensor cores with the reference of every
 // decay factor placed between the two tokens it connects, so that no operand
-// is scaled by more than 1.  Level p = 64, 32, ..., 2 splits the rows into
+// is scaled by more than 1.  Level p = 64, 32, 16, 8 splits the rows into
 // aligned p-blocks with an earlier and a later half and takes as reference
 // R the cumulative decay G at the last row of the earlier half; it scales a
 // later row r by e^{G_r - R} and an earlier row by e^{R - G_r} (both <= 1 for
@@ -374,19 +374,21 @@ __device__ __forceinline__ void store_pa(uint8_t* sm, int b2, int ti, int chh, c
 // q_r k_s e^{G_r - G_s} exactly for the pairs r > s that straddle one of its
 // boundaries: those whose highest differing index bit is p/2.  Levels run
 // from p = 64 down; each keeps the pairs with r and s in the same p-block,
-// so the finest level that contains a pair wins.  The diagonal of P (no
-// decay) is the plain q_r . k_r.  Q and K rows scaled for a level go to a
-// tile of the stage layout whose two 64-channel halves are the A tile and
-// KX[b2] (both released: AFREE and BUF were waited for); the row-group end
-// values of G (the references of levels 8..64) are staged in the P tile.
-__device__ __forceinline__ bool level_gram(const Ctx& x, int b2, const F8 (&gv)[4], int& g1_ph) {
+// so the finest level that contains a pair wins.  The pairs inside one
+// 4-row group (and the diagonal of P) are one thread's own rows: they are
+// summed exactly on CUDA cores from the per-token ratios e^{g}.  Q and K
+// rows scaled for a level go to a tile of the stage layout whose two
+// 64-channel halves are the A tile and KX[b2] (both released: AFREE and BUF
+// were waited for); the row-group end values of G (the references) are
+// staged in the P tile.
+__device__ __forceinline__ bool level_gram(const Ctx& x, int c, int b2, const F8 (&gv)[4], int& g1_ph) {
   const int f = threadIdx.x - FRONT0;
   const int wq = f >> 5, lane = f & 31, lq = wq & 3, chh = wq >> 2;
   const int rg = f >> 4, ch0 = 8 * (f & 15), hh = ch0 >> 6, cc = ch0 & 63;
   uint8_t* sm = x.sm;
   const uint32_t sb = x.sb;
   float* s_ref = reinterpret_cast<float*>(sm + SM_P + b2 * 8192);  // [16][128]: G at row 4 k + 3
-  float* s_diag = reinterpret_cast<float*>(sm + SM_MISC + MS_DIAG);
+  float* s_pairs = reinterpret_cast<float*>(sm + SM_MISC + MS_PAIRS);
   const float* s_beta = reinterpret_cast<const float*>(sm + SM_MISC + MS_BETA) + b2 * 64;
   const uint8_t* qb = sm + b2 * STAGE_BYTES + OFF_QK + hh * 16384;
   const uint8_t* kb = qb + 8192;
@@ -394,69 +396,37 @@ __device__ __forceinline__ bool level_gram(const Ctx& x, int b2, const F8 (&gv)[
   const uint32_t tl = x.tmem + ((uint32_t)(lq * 32) << 16);
   const int ti = 32 * lq + lane, r = ti & 63;
 
-  {  // G at the end of this thread's row group, and the raw diagonal q_r . k_r
+  {  // G at the end of this thread's row group (a reference of the levels)
     const F8 ge = add8(add8(add8(gv[0], gv[1]), gv[2]), gv[3]);
     *reinterpret_cast<float4*>(s_ref + rg * 128 + ch0) = ge.a;
     *reinterpret_cast<float4*>(s_ref + rg * 128 + ch0 + 4) = ge.b;
-    float d[4];
-#pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      const uint32_t o = sw128_off(4 * rg + m, cc);
-      const F8 qv = bf16x8_to_f32(*reinterpret_cast<const uint4*>(qb + o));
-      const F8 kv = bf16x8_to_f32(*reinterpret_cast<const uint4*>(kb + o));
-      const F8 pr = mul8(qv, kv);
-      d[m] = ((pr.a.x + pr.a.y) + (pr.a.z + pr.a.w)) + ((pr.b.x + pr.b.y) + (pr.b.z + pr.b.w));
-    }
-#pragma unroll
-    for (int o = 1; o < 16; o <<= 1)
-#pragma unroll
-      for (int m = 0; m < 4; ++m) d[m] += __shfl_xor_sync(0xffffffffu, d[m], o);
-    if ((f & 15) == 0) {
-#pragma unroll
-      for (int m = 0; m < 4; ++m) s_diag[4 * rg + m] = d[m];
-    }
   }
-  named_sync(GRP_FRONT, FRONT_T);
+  named_sync(GRP_FRONT, FRONT_T);  // references staged
 
-  float acc[32];
-#pragma unroll
-  for (int L = 6; L >= 1; --L) {
+  // Level L: scale this thread's Q and K rows into the level tile.
+  auto write_tile = [&](int L) {
     const int p = 1 << L;
-    // ---- this level's scaled rows: row 4 rg + m times 2^{x_m} (log2 units)
-    F8 dr = f8(0.f);  // G_r - R, running over this thread's rows
-    bool later = false;
-    if (L >= 3) {  // reference R: the end of row group kref (another thread's rows)
-      const int kref = (rg & ~(p / 4 - 1)) + p / 8 - 1;
-      const F8 R = {*reinterpret_cast<const float4*>(s_ref + kref * 128 + ch0),
-                    *reinterpret_cast<const float4*>(s_ref + kref * 128 + ch0 + 4)};
-      later = ((4 * rg) & (p / 2)) != 0;
-      dr = sub8(f8(0.f), R);
-    }
+    // row 4 rg + m times 2^{x_m} (log2 units); reference R: the end of row
+    // group kref (another thread's rows)
+    const int kref = (rg & ~(p / 4 - 1)) + p / 8 - 1;
+    const bool later = ((4 * rg) & (p / 2)) != 0;
+    F8 dr = sub8(f8(0.f), F8{*reinterpret_cast<const float4*>(s_ref + kref * 128 + ch0),
+                             *reinterpret_cast<const float4*>(s_ref + kref * 128 + ch0 + 4)});  // G_r - R
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
       const uint32_t o = sw128_off(4 * rg + m, cc);
-      F8 e;
-      if (L >= 3) {
-        dr = add8(dr, gv[m]);
-        e = ex2_8(later ? dr : sub8(f8(0.f), dr));
-      } else if (L == 2) {  // reference: row 4 rg + 1
-        e = m == 1 ? f8(1.f) : ex2_8(m == 0 ? gv[1] : (m == 2 ? gv[2] : add8(gv[2], gv[3])));
-      } else {  // references: rows 4 rg and 4 rg + 2
-        e = (m & 1) == 0 ? f8(1.f) : ex2_8(m == 1 ? gv[1] : gv[3]);
-      }
-#pragma unroll
-      for (int hq = 0; hq < 2; ++hq) {  // 4 channels at a time
-        const float4 eh = hq ? e.b : e.a;
-        const uint2 qh = *reinterpret_cast<const uint2*>(qb + o + 8 * hq);
-        const uint2 kh = *reinterpret_cast<const uint2*>(kb + o + 8 * hq);
-        st_f16x4(lt + o + 8 * hq, mul4(bf16x4_to_f32(qh), eh));
-        st_f16x4(lt + 8192 + o + 8 * hq, mul4(bf16x4_to_f32(kh), eh));
-      }
+      dr = add8(dr, gv[m]);
+      const F8 e = ex2_8(later ? dr : sub8(f8(0.f), dr));
+      st_f16x8(lt + o, mul8(bf16x8_to_f32(*reinterpret_cast<const uint4*>(qb + o)), e));
+      st_f16x8(lt + 8192 + o, mul8(bf16x8_to_f32(*reinterpret_cast<const uint4*>(kb + o)), e));
     }
     fence_proxy_async_smem();
+  };
+  // [Q ; K] K^T of the level tile (M=128, N=64, K=128) -> TM_G, once every
+  // thread has written its rows and finished reading the previous level.
+  auto issue = [&]() {
     tc_fence_before();
-    named_sync(GRP_FRONT, FRONT_T);  // tile written; the previous level's TMEM reads are done
-    // ---- [Q ; K] K^T of the level tile (M=128, N=64, K=128) -> TM_G
+    named_sync(GRP_FRONT, FRONT_T);
     if (f == 0) {
       tc_fence_after();
       const uint32_t id = idesc_f16_f32(128, 64, 0, 0);
@@ -469,9 +439,73 @@ __device__ __forceinline__ bool level_gram(const Ctx& x, int b2, const F8 (&gv)[
       }
       umma_commit(&x.bars[B_G1]);
     }
+  };
+  write_tile(6);
+  issue();
+  if (f == 0) tmark(x, c, 29);
+
+  {  // While the first level runs: the pairs s <= r inside this thread's rows
+     // 4 rg .. 4 rg + 3 over its 8 channels, pv[] = P (10 pairs with the
+     // diagonal), av[] = A (6 pairs); e^{G_r - G_s} is the running product of
+     // the ratios e^{g_t}, s < t <= r.
+    float pv[10] = {}, av[6] = {};
+#pragma unroll
+    for (int hq = 0; hq < 2; ++hq) {  // 4 channels at a time
+      const float4 al[4] = {make_float4(1.f, 1.f, 1.f, 1.f), ex2_4(hq ? gv[1].b : gv[1].a),
+                            ex2_4(hq ? gv[2].b : gv[2].a), ex2_4(hq ? gv[3].b : gv[3].a)};
+      int ip = 0, ia = 0;
+#pragma unroll
+      for (int s = 0; s < 4; ++s) {
+        const float4 ks = bf16x4_to_f32(*reinterpret_cast<const uint2*>(kb + sw128_off(4 * rg + s, cc) + 8 * hq));
+        float4 e = make_float4(1.f, 1.f, 1.f, 1.f);
+#pragma unroll
+        for (int rr = s; rr < 4; ++rr) {
+          if (rr > s) e = mul4(e, al[rr]);
+          const uint32_t o = sw128_off(4 * rg + rr, cc) + 8 * hq;
+          const float4 ke = mul4(ks, e);
+          const float4 pq = mul4(bf16x4_to_f32(*reinterpret_cast<const uint2*>(qb + o)), ke);
+          pv[ip++] += (pq.x + pq.y) + (pq.z + pq.w);
+          if (rr > s) {
+            const float4 pk = mul4(bf16x4_to_f32(*reinterpret_cast<const uint2*>(kb + o)), ke);
+            av[ia++] += (pk.x + pk.y) + (pk.z + pk.w);
+          }
+        }
+      }
+    }
+    // Sum over the 16 threads of the row group (lanes differing in bits 0-3).
+#pragma unroll
+    for (int o = 1; o < 16; o <<= 1) {
+#pragma unroll
+      for (int i = 0; i < 10; ++i) pv[i] += __shfl_xor_sync(0xffffffffu, pv[i], o);
+#pragma unroll
+      for (int i = 0; i < 6; ++i) av[i] += __shfl_xor_sync(0xffffffffu, av[i], o);
+    }
+    if ((f & 15) == 0) {  // [r][0..3]: P_{r, 4 rg + j};  [r][4..7]: A_{r, 4 rg + j} (j < r - 4 rg)
+      int ip = 0, ia = 0;
+      float tp[4][4] = {}, ta[4][4] = {};
+#pragma unroll
+      for (int s = 0; s < 4; ++s)
+#pragma unroll
+        for (int rr = s; rr < 4; ++rr) {
+          tp[rr][s] = pv[ip++];
+          if (rr > s) ta[rr][s] = av[ia++];
+        }
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        float* row = s_pairs + (4 * rg + m) * 8;
+        *reinterpret_cast<float4*>(row) = make_float4(tp[m][0], tp[m][1], tp[m][2], tp[m][3]);
+        *reinterpret_cast<float4*>(row + 4) = make_float4(ta[m][0], ta[m][1], ta[m][2], ta[m][3]);
+      }
+    }
+  }
+
+  float acc[32];
+#pragma unroll
+  for (int L = 6; L >= 3; --L) {
     if (!gwait(x, B_G1, g1_ph, 16, GRP_FRONT)) return false;
     g1_ph ^= 1;
     tc_fence_after();
+    if (L > 3) write_tile(L - 1);  // the tile is free again; TM_G still holds level L
     if (L == 6) {
       tmem_ld32(tl + TM_G + chh * 32, acc);
     } else if ((lq & 1) == chh) {  // (warp-uniform) a warp whose rows and columns share a 32-block
@@ -484,17 +518,22 @@ __device__ __forceinline__ bool level_gram(const Ctx& x, int b2, const F8 (&gv)[
           if ((r >> L) == ((32 * chh + 8 * hv + u) >> L)) acc[8 * hv + u] = val[u];
       }
     }
+    if (L > 3) issue();
+  }
+  if (f == 0) tmark(x, c, 30);
+  if ((lq & 1) == chh) {  // the pairs inside 4-row groups
+    const float4 t = *reinterpret_cast<const float4*>(s_pairs + r * 8 + (ti < CH ? 0 : 4));
+    const float tv[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+    for (int u = 0; u < 32; ++u)
+      if ((r >> 2) == ((32 * chh + u) >> 2)) acc[u] = tv[u & 3];
   }
   // Every level's UMMA has completed and every thread is past the last
   // level's tile barrier, so the P tile (reference table) and the A tile
   // (level tile half) may be overwritten.
   store_pa(sm, b2, ti, chh, s_beta, acc);
-  if (ti < CH && (r >> 5) == chh) {  // the diagonal of P
-    const __half h = __float2half_rn(s_diag[r]);
-    *reinterpret_cast<__half*>(sm + SM_P + b2 * 8192 + sw128_off(r, r)) = h;
-  }
   tc_fence_before();
-  named_sync(GRP_FRONT, FRONT_T);  // TMEM reads done before the next G1; tiles complete before the raw-row rescaling
+  named_sync(GRP_FRONT, FRONT_T);  // TMEM reads done before the next G1
   return true;
 }
 
@@ -658,7 +697,7 @@ __device__ void front_group(const Ctx& x, const float* __restrict__ g, const flo
       }
     }
     if (!fast) {
-      if (!level_gram(x, b2, gv, g1_ph)) break;
+      if (!level_gram(x, c, b2, gv, g1_ph)) break;
       // G_C again from the warp sums (the same additions in the same order),
       // so that it is not held in registers across the Gram.
       tot = f8(0.f);

@@ -24,12 +24,16 @@ KDA_API int kda_testing_debug_floats(void);
  *              at these float offsets: P [64][64] at 0, A [64][64] at 4096
  *              (strictly lower part), T' [64][64] at 8192, W' [64][128] at
  *              12288 (W' = W Diag(exp(-G_C)), the chunk-end-referenced
- *              pseudo-keys), U [64][128] at 20480, Delta [64][128] at 28672,
- *              O [64][128] at 36864, the state after the chunk [128][128] at
- *              45056, the chunk-total log-decay G_C [128] at 61440; and, as
+ *              pseudo-keys, on chunks whose total decay keeps the
+ *              end-referenced operands in fp16 range; W' = W on the others,
+ *              which are referenced to the chunk start), U [64][128] at
+ *              20480, Delta [64][128] at 28672, O [64][128] at 36864, the
+ *              state after the chunk [128][128] at 45056, the chunk-total
+ *              log-decay G_C [128] at 61440; and, as
  *              int64 from float offset 61568, [64 chunks][32 events] of SM
  *              clock cycles since the block started: phase boundaries of
- *              the first 64 chunks (events 0-7 and 26: front group; 16-23
+ *              the first 64 chunks (events 0-7 and 26: front group, with
+ *              29 and 30 inside the Gram of strongly decaying chunks; 16-23
  *              and 25: back group; 8-15, 24, 27, 28: scan group).
  *   wait_ns    bound for every device-side wait in nanoseconds (kda_fwd
  *              uses 2e9).
