@@ -418,6 +418,49 @@ def run_phases(args):
     print(json.dumps(res), flush=True)
 
 
+def run_chains(args):
+    """Prefill over H independent heads (one chain each, B=1) for each H in
+    --chains: kernel time per 64-token chunk (median of --steps launches) and
+    chain 0's own chunk period in SM cycles (test hook).  The two diverge when
+    some chains run slower than chain 0."""
+    import numpy as np
+    import torch
+
+    import gated_delta_rule_121_b200 as kda
+    import synth
+    T = args.chain_tokens
+    for H in (int(h) for h in args.chains.split(",")):
+        spec = synth.PrefillSpec(f"chains_H{H}_T{T}", 1, T, H, 128, 128, torch.bfloat16, 2)
+        inp = synth.make_prefill(spec, torch.device("cuda"))
+        call = (inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["init_state"], inp["cu_seqlens"])
+        out = torch.empty_like(inp["q"])
+        fin = torch.empty(1, H, 128, 128, device="cuda")
+        ws = kda.alloc_workspace(1, T, H, 128, 128)
+        for _ in range(args.warmup):
+            kda.kda_fwd(*call, out=out, final_state=fin, workspace=ws)
+        torch.cuda.synchronize()
+        ms = []
+        for _ in range(args.steps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            kda.kda_fwd(*call, out=out, final_state=fin, workspace=ws)
+            e1.record()
+            torch.cuda.synchronize()
+            ms.append(e0.elapsed_time(e1))
+        med = float(np.median(ms))
+        res = {"chains": H, "tokens": T, "ms": med, "us_per_chunk": med * 1e3 / (T // CHUNK)}
+        if not args.no_period:
+            dbg = torch.zeros(kda.lib().kda_testing_debug_floats(), dtype=torch.float32, device="cuda")
+            kda.kda_fwd(*call, out=out, final_state=fin, workspace=ws, _debug=dbg)
+            torch.cuda.synchronize()
+            t = dbg[61568:].cpu().numpy().view(np.int64).reshape(64, 32)
+            hi = min(60, T // CHUNK)
+            res["chain0_period_cycles"] = float(np.mean(np.diff(t[min(8, hi // 2):hi, 0])))
+        print(json.dumps(res), flush=True)
+        del inp, out, fin, ws
+        torch.cuda.empty_cache()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -430,11 +473,17 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--phases", action="store_true",
                     help="print per-phase cycles of the tensor-core kernel (test hook) instead of timing")
+    ap.add_argument("--chains", default=None,
+                    help="comma-separated head counts: time B=1 prefills with that many chains instead")
+    ap.add_argument("--chain-tokens", type=int, default=16384)
+    ap.add_argument("--no-period", action="store_true", help="with --chains: skip the test-hook launch")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
     d = Dist()
     if args.phases:
         run_phases(args)
+    elif args.chains:
+        run_chains(args)
     elif args.impl == "reference":
         run_reference(args, d)
     else:

@@ -16,7 +16,10 @@ extern "C" {
 KDA_API int kda_testing_debug_floats(void);
 
 /*
- * Same as kda_fwd, plus:
+ * Same as kda_fwd, plus the hooks below.  A call that sets debug_out or
+ * inject_stuck runs the instrumented build of the tensor-core kernel (same
+ * source, with the dumps, timestamps and injection compiled in); other calls
+ * run the production build, which has none of them.
  *   debug_out  device fp32 buffer of kda_testing_debug_floats() floats or
  *              NULL.  When set (tensor-core path only, else
  *              KDA_ERR_UNSUPPORTED), the block of chain 0 (sequence 0, head 0)
