@@ -497,22 +497,28 @@ __device__ __forceinline__ bool level_gram(const Ctx& x, int c, int b2, const F8
   }
 
   float acc[32];
-#pragma unroll
-  for (int L = 6; L >= 3; --L) {
+  // Level 64 fills acc; levels 32, 16, 8 overwrite the pairs inside their blocks.
+  if (!gwait(x, B_G1, g1_ph, 16, GRP_FRONT)) return false;
+  g1_ph ^= 1;
+  tc_fence_after();
+  write_tile(5);  // the tile is free again; TM_G still holds level 64
+  tmem_ld32(tl + TM_G + chh * 32, acc);
+  issue();
+#pragma unroll 1
+  for (int L = 5; L >= 3; --L) {
     if (!gwait(x, B_G1, g1_ph, 16, GRP_FRONT)) return false;
     g1_ph ^= 1;
     tc_fence_after();
-    if (L > 3) write_tile(L - 1);  // the tile is free again; TM_G still holds level L
-    if (L == 6) {
-      tmem_ld32(tl + TM_G + chh * 32, acc);
-    } else if ((lq & 1) == chh) {  // (warp-uniform) a warp whose rows and columns share a 32-block
+    if (L > 3) write_tile(L - 1);
+    if ((lq & 1) == chh) {  // (warp-uniform) a warp whose rows and columns share a 32-block
+      const int rb = r >> L;
 #pragma unroll
       for (int hv = 0; hv < 4; ++hv) {
         float val[8];
         tmem_ld8(tl + TM_G + chh * 32 + hv * 8, val);
 #pragma unroll
         for (int u = 0; u < 8; ++u)
-          if ((r >> L) == ((32 * chh + 8 * hv + u) >> L)) acc[8 * hv + u] = val[u];
+          if (rb == ((32 * chh + 8 * hv + u) >> L)) acc[8 * hv + u] = val[u];
       }
     }
     if (L > 3) issue();
@@ -874,7 +880,7 @@ __device__ __forceinline__ void back_group(const Ctx& x) {
     }
     named_sync(GRP_BACK, GRP);
     if (k == 0) tmark(x, c, 19);
-#pragma unroll
+#pragma unroll 1
     for (int t = bw; t < 8; t += 4) {  // X = A_10 D_0  (32x32x32, 16x8 tiles)
       const int mt = t >> 2, nt = t & 3;
       float d[4];
@@ -889,7 +895,7 @@ __device__ __forceinline__ void back_group(const Ctx& x) {
       mbar_arrive(&x.bars[B_AFREE]);  // A is no longer read
       tmark(x, c, 20);
     }
-#pragma unroll
+#pragma unroll 1
     for (int t = bw; t < 8; t += 4) {  // T_10 = -D_1 X
       const int mt = t >> 2, nt = t & 3;
       float d[4];
@@ -1042,7 +1048,7 @@ __device__ __forceinline__ void scan_group(const Ctx& x, const void* tmq, const 
     }
   }
   // S^T <- initial state (zeros without one).
-#pragma unroll
+#pragma unroll 1
   for (int cb = 0; cb < 4; ++cb) {
     float r[32];
 #pragma unroll
@@ -1120,7 +1126,7 @@ __device__ __forceinline__ void scan_group(const Ctx& x, const void* tmq, const 
       break;
     }
     const bool fast = *reinterpret_cast<volatile int*>(sm + SM_MISC + MS_FAST + 4 * b2) != 0;
-#pragma unroll
+#pragma unroll 1
     for (int cp = 0; cp < 2; ++cp) {
       float s0[32], s1[32];
       uint32_t pk[16];
@@ -1202,7 +1208,7 @@ __device__ __forceinline__ void scan_group(const Ctx& x, const void* tmq, const 
 
     // ---- Δ^T -> fp16 pairs (A operand of D2); general chunks decay S^T here.
     if (!fast) {
-#pragma unroll
+#pragma unroll 1
       for (int cb = 0; cb < 4; ++cb) {
         float s[32];
         tmem_ld32(tl + TM_S + cb * 32, s);
@@ -1273,7 +1279,7 @@ __device__ __forceinline__ void scan_group(const Ctx& x, const void* tmq, const 
   if (named_sync_and(2, 128, !*x.abort)) {
     if (x.dbg && x.nchunks > 0) dump_s(x.dbg, x.tmem);
     if (fin) {
-#pragma unroll
+#pragma unroll 1
       for (int cb = 0; cb < 4; ++cb) {
         float s[32];
         tmem_ld32(tl + TM_S + cb * 32, s);
