@@ -437,19 +437,14 @@ __device__ __forceinline__ bool level_gram(const Ctx& x, int c, int b2, const F8
       umma_commit(&x.bars[B_G1]);
     }
   };
-  write_tile(6);
-  issue();
-  if (f == 0) tmark(x, c, 29);
-
+  auto pairs = [&]() {
   {  // While the first level runs: the pairs s <= r inside this thread's rows
      // 4 rg .. 4 rg + 3 over its 8 channels, pv[] = P (10 pairs with the
      // diagonal), av[] = A (6 pairs); e^{G_r - G_s} is the running product of
      // the ratios e^{g_t}, s < t <= r.
     float pv[10] = {}, av[6] = {};
-#pragma unroll
+#pragma unroll 1
     for (int hq = 0; hq < 2; ++hq) {  // 4 channels at a time
-      const float4 al[4] = {make_float4(1.f, 1.f, 1.f, 1.f), ex2_4(hq ? gv[1].b : gv[1].a),
-                            ex2_4(hq ? gv[2].b : gv[2].a), ex2_4(hq ? gv[3].b : gv[3].a)};
       int ip = 0, ia = 0;
 #pragma unroll
       for (int s = 0; s < 4; ++s) {
@@ -457,7 +452,7 @@ __device__ __forceinline__ bool level_gram(const Ctx& x, int c, int b2, const F8
         float4 e = make_float4(1.f, 1.f, 1.f, 1.f);
 #pragma unroll
         for (int rr = s; rr < 4; ++rr) {
-          if (rr > s) e = mul4(e, al[rr]);
+          if (rr > s) e = mul4(e, ex2_4(hq ? gv[rr].b : gv[rr].a));
           const uint32_t o = sw128_off(4 * rg + rr, cc) + 8 * hq;
           const float4 ke = mul4(ks, e);
           const float4 pq = mul4(bf16x4_to_f32(*reinterpret_cast<const uint2*>(qb + o)), ke);
@@ -496,21 +491,22 @@ __device__ __forceinline__ bool level_gram(const Ctx& x, int c, int b2, const F8
     }
   }
 
-  float acc[32];
+  };
+  float acc[32] = {};
+  // Pass L = 7 only starts level 64 (and, while it runs, the pairs inside
+  // 4-row groups); pass L takes level L's Gram and starts level L - 1.
   // Level 64 fills acc; levels 32, 16, 8 overwrite the pairs inside their blocks.
-  if (!gwait(x, B_G1, g1_ph, 16, GRP_FRONT)) return false;
-  g1_ph ^= 1;
-  tc_fence_after();
-  write_tile(5);  // the tile is free again; TM_G still holds level 64
-  tmem_ld32(tl + TM_G + chh * 32, acc);
-  issue();
 #pragma unroll 1
-  for (int L = 5; L >= 3; --L) {
-    if (!gwait(x, B_G1, g1_ph, 16, GRP_FRONT)) return false;
-    g1_ph ^= 1;
-    tc_fence_after();
-    if (L > 3) write_tile(L - 1);
-    if ((lq & 1) == chh) {  // (warp-uniform) a warp whose rows and columns share a 32-block
+  for (int L = 7; L >= 3; --L) {
+    if (L < 7) {
+      if (!gwait(x, B_G1, g1_ph, 16, GRP_FRONT)) return false;
+      g1_ph ^= 1;
+      tc_fence_after();
+    }
+    if (L > 3) write_tile(L - 1);  // the tile is free again; TM_G still holds level L
+    // (warp-uniform) below level 64, only a warp whose rows and columns share a
+    // 32-block has pairs to take
+    if (L == 6 || (L < 6 && (lq & 1) == chh)) {
       const int rb = r >> L;
 #pragma unroll
       for (int hv = 0; hv < 4; ++hv) {
@@ -522,6 +518,10 @@ __device__ __forceinline__ bool level_gram(const Ctx& x, int c, int b2, const F8
       }
     }
     if (L > 3) issue();
+    if (L == 7) {
+      if (f == 0) tmark(x, c, 29);
+      pairs();
+    }
   }
   if (f == 0) tmark(x, c, 30);
   if ((lq & 1) == chh) {  // the pairs inside 4-row groups
