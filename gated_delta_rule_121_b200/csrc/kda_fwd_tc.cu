@@ -197,52 +197,31 @@ __device__ __forceinline__ uint32_t a_off(uint32_t r, uint32_t s) {
 __device__ __forceinline__ uint32_t b_off(uint32_t r, uint32_t s) {
   return r * 128u + ((s >> 2) ^ (r & 7u)) * 16u + (s & 3u) * 4u;
 }
-// One 16x8 tile of D = sign * A B with fp32 operands held in shared memory,
-// K = 8 * KSTEPS, computed on the warp-level tensor path as three tf32
-// products (hi*hi + hi*lo + lo*hi), which keeps close to fp32 accuracy.  hi
-// is x with its low 13 mantissa bits cleared (exactly a tf32 value); lo = x -
-// hi is exact in fp32 and the MMA reads its leading 10 mantissa bits, so the
-// dropped part is below 2^-21 |x|.
-// fa(r, k) / fb(k, n) return the operand element addresses.
+// One 16x8 tile of D = A B with fp32 operands held in shared memory, K = 8 *
+// KSTEPS, on the warp-level tensor path in tf32 (the MMA reads the leading 10
+// mantissa bits of each operand).  The solve's inputs come from fp16 tensor-core
+// operands and its outputs are rounded to fp16, so tf32 block products leave the
+// end-to-end error unchanged (a CPU emulation of the kernel's rounding points:
+// output relative error 1.70e-3 with exact or tf32 block products, mild and
+// model-range decay alike).  fa(r, k) / fb(k, n) return the operand element
+// addresses.
 template <int KSTEPS, typename FA, typename FB>
-__device__ __forceinline__ void warp_gemm_tf32x3(float (&d)[4], FA fa, FB fb) {
+__device__ __forceinline__ void warp_gemm_tf32(float (&d)[4], FA fa, FB fb) {
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-  // Separate accumulators for the three products keep the dependent chains
-  // KSTEPS long; the small terms are added first.
-  float dhh[4] = {0.f, 0.f, 0.f, 0.f}, dhl[4] = {0.f, 0.f, 0.f, 0.f}, dlh[4] = {0.f, 0.f, 0.f, 0.f};
-  float av[KSTEPS][4], bv[KSTEPS][2];
+  d[0] = d[1] = d[2] = d[3] = 0.f;
+  uint32_t av[KSTEPS][4], bv[KSTEPS][2];
   // ldmatrix row address of this lane: tile lane/8 = (rows 8 (tile & 1)..,
   // words 4 (tile >> 1)..) of the 16x8 A block.
   const int arow = (lane & 7) + 8 * ((lane >> 3) & 1), akof = 4 * (lane >> 4);
 #pragma unroll
   for (int ks = 0; ks < KSTEPS; ++ks) {  // every fragment load first: one shared-memory latency
     const int k0 = 8 * ks;
-    uint32_t a4[4];
-    ldsm_x4(smem_u32(fa(arow, k0 + akof)), a4);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) av[ks][i] = __uint_as_float(a4[i]);
-    bv[ks][0] = *fb(k0 + t, g);
-    bv[ks][1] = *fb(k0 + t + 4, g);
+    ldsm_x4(smem_u32(fa(arow, k0 + akof)), av[ks]);
+    bv[ks][0] = __float_as_uint(*fb(k0 + t, g));
+    bv[ks][1] = __float_as_uint(*fb(k0 + t + 4, g));
   }
 #pragma unroll
-  for (int ks = 0; ks < KSTEPS; ++ks) {
-    uint32_t ah[4], al[4], bh[2], bl[2];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      ah[i] = __float_as_uint(av[ks][i]) & 0xffffe000u;
-      al[i] = __float_as_uint(av[ks][i] - __uint_as_float(ah[i]));
-    }
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      bh[i] = __float_as_uint(bv[ks][i]) & 0xffffe000u;
-      bl[i] = __float_as_uint(bv[ks][i] - __uint_as_float(bh[i]));
-    }
-    mma_tf32_16x8x8(dlh, al, bh);
-    mma_tf32_16x8x8(dhl, ah, bl);
-    mma_tf32_16x8x8(dhh, ah, bh);
-  }
-#pragma unroll
-  for (int i = 0; i < 4; ++i) d[i] = (dlh[i] + dhl[i]) + dhh[i];
+  for (int ks = 0; ks < KSTEPS; ++ks) mma_tf32_16x8x8(d, av[ks], bv[ks]);
 }
 
 // Bounded wait that also gives up when the other group has aborted.
@@ -860,7 +839,7 @@ __device__ __forceinline__ void back_group(const Ctx& x) {
     {  // Y_b = A'_b E_2b (A'_b = A[32b+16 .. +16][32b .. +16]), then F_b = -E_2b+1 Y_b
       const int b = bw >> 1, nt = bw & 1;
       float d[4];
-      warp_gemm_tf32x3<2>(
+      warp_gemm_tf32<2>(
           d, [&](int r, int kk) { return reinterpret_cast<const float*>(sm + SM_A + a_off(32 * b + 16 + r, 32 * b + kk)); },
           [&](int kk, int n) { return reinterpret_cast<const float*>(sm + SM_DG + b * 4096 + b_off(kk, 8 * nt + n)); });
       float* y = reinterpret_cast<float*>(sm + SM_X + b * 1024);
@@ -871,7 +850,7 @@ __device__ __forceinline__ void back_group(const Ctx& x) {
     {
       const int b = bw >> 1, nt = bw & 1;
       float d[4];
-      warp_gemm_tf32x3<2>(
+      warp_gemm_tf32<2>(
           d, [&](int r, int kk) { return reinterpret_cast<const float*>(sm + SM_DG + b * 4096 + b_off(16 + r, 16 + kk)); },
           [&](int kk, int n) { return reinterpret_cast<const float*>(sm + SM_X + b * 1024 + (kk * 16 + 8 * nt + n) * 4); });
       uint8_t* db = sm + SM_DG + b * 4096;
@@ -884,7 +863,7 @@ __device__ __forceinline__ void back_group(const Ctx& x) {
     for (int t = bw; t < 8; t += 4) {  // X = A_10 D_0  (32x32x32, 16x8 tiles)
       const int mt = t >> 2, nt = t & 3;
       float d[4];
-      warp_gemm_tf32x3<4>(
+      warp_gemm_tf32<4>(
           d, [&](int r, int kk) { return reinterpret_cast<const float*>(sm + SM_A + a_off(32 + 16 * mt + r, kk)); },
           [&](int kk, int n) { return reinterpret_cast<const float*>(sm + SM_DG + b_off(kk, 8 * nt + n)); });
       *reinterpret_cast<float2*>(sm + SM_X + b_off(16 * mt + lg, 8 * nt + 2 * lt)) = make_float2(d[0], d[1]);
@@ -899,7 +878,7 @@ __device__ __forceinline__ void back_group(const Ctx& x) {
     for (int t = bw; t < 8; t += 4) {  // T_10 = -D_1 X
       const int mt = t >> 2, nt = t & 3;
       float d[4];
-      warp_gemm_tf32x3<4>(
+      warp_gemm_tf32<4>(
           d, [&](int r, int kk) { return reinterpret_cast<const float*>(sm + SM_DG + 4096 + b_off(16 * mt + r, kk)); },
           [&](int kk, int n) { return reinterpret_cast<const float*>(sm + SM_X + b_off(kk, 8 * nt + n)); });
       *reinterpret_cast<float2*>(sm + SM_T10 + b_off(16 * mt + lg, 8 * nt + 2 * lt)) = make_float2(-d[0], -d[1]);
