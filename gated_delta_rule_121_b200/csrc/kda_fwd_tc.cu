@@ -19,11 +19,11 @@
 // up to exp(-G_C): with the digest's bounded decay ("Bounded decay" section,
 // g >= -5) every tile is a dense matmul as long as a chunk's total decay is
 // moderate.  A chunk whose total decay in some channel is below 2^-10 takes
-// the general variant: its Gram matrices P, A come from six tensor-core
+// the general variant: its Gram matrices P, A come from four tensor-core
 // Grams whose decay references sit at block boundaries between the two
-// tokens of every pair (so no operand factor exceeds 1), the operands use the
-// chunk START as reference (QE = Q e^G, KE = K e^G), and the scan decays S
-// only after D1.
+// tokens of every pair (so no operand factor exceeds 1) plus the pairs inside
+// 4-row groups on CUDA cores, the operands use the chunk START as reference
+// (QE = Q e^G, KE = K e^G), and the scan decays S only after D1.
 //
 // Operands are fp16 (10-bit mantissa) with fp32 accumulation: the fp32
 // state and every product stay accurate to well inside the bf16 output's own
