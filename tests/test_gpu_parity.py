@@ -81,6 +81,16 @@ def test_mixed_decay_chunks():
     check(inp, torch.bfloat16, what="mixed decay")
 
 
+def test_model_range_decay_ragged_packed():
+    """Strongly decaying chunks (level Gram) that end mid-chunk: packed
+    sequences of ragged lengths with g = -5 sigmoid(z), each with its own
+    initial state."""
+    inp = synth.make_prefill(synth.VARLEN, DEV, H=3, lengths=[1, 37, 64, 100, 130, 0, 257])
+    inp["g"] = (inp["g"] * 64.0).contiguous()
+    assert float(inp["g"].min()) < -4.0
+    check(inp, torch.bfloat16, what="varlen model-range decay")
+
+
 @pytest.mark.parametrize("lengths", [[1, 63, 64, 65, 130, 0, 200], [0], [5], [300, 0, 0, 64]])
 def test_varlen_ragged_and_empty(lengths):
     inp = synth.make_prefill(synth.VARLEN, DEV, H=4, lengths=lengths)
