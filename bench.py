@@ -3,6 +3,8 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
     python bench.py --impl reference ...      # the fp64 CPU oracle arm
+    python bench.py --phases [--workload NAME] # per-phase cycles (test-hook build)
+    python bench.py --chains 64,96,148        # time per chunk against concurrent chains
 
 Default workload: the model-shaped prefill B=1, H=96, T=65536, dk=dv=128,
 bf16 q/k/v/o with fp32 log-decay, beta and state (the 64K pretraining
