@@ -18,8 +18,11 @@
  * k are expected L2-normalised by the caller (the model does this before the
  * recurrence) but nothing relies on it.
  *
- * Precondition (documented, not checked): every g value lies in [-5, 0].
- * Results for g outside that range are not covered by the accuracy contract.
+ * Precondition (documented, not checked): every g value is finite and <= 0
+ * (alpha <= 1, a decay).  The model's range is [-5, 0]; the kernels do not
+ * rely on that lower bound (every decay factor they form is at most 1 for
+ * any g <= 0; the parity tests cover g down to -20).  Results for g > 0 are
+ * not covered by the accuracy contract.
  *
  * Conventions shared by every entry point:
  *   - Ownership: the caller allocates and owns every buffer.  The library
@@ -91,7 +94,7 @@ KDA_API size_t kda_fwd_workspace_size(int B, int64_t T, int H, int dk, int dv, k
  *
  *   q, k       [B, T, H, dk]  dtype dt, device
  *   v          [B, T, H, dv]  dtype dt, device
- *   log_alpha  [B, T, H, dk]  fp32, device; g = log(alpha) in [-5, 0]
+ *   log_alpha  [B, T, H, dk]  fp32, device; g = log(alpha) <= 0
  *   beta       [B, T, H]      fp32, device
  *   init_state [N, H, dk, dv] fp32, device, or NULL for a zero start
  *   out        [B, T, H, dv]  dtype dt, device, written (rounded to nearest

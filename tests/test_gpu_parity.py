@@ -91,6 +91,15 @@ def test_model_range_decay_ragged_packed():
     check(inp, torch.bfloat16, what="varlen model-range decay")
 
 
+def test_decay_beyond_the_model_bound():
+    """g = -20 sigmoid(z), four times past the model's bound g >= -5: every
+    factor of the strongly decaying path stays at most 1 for any g <= 0."""
+    inp = synth.make_prefill(synth.VARLEN, DEV, H=2, lengths=[257, 64, 3, 190])
+    inp["g"] = (inp["g"] * 256.0).contiguous()
+    assert float(inp["g"].min()) < -15.0
+    check(inp, torch.bfloat16, what="g >= -20")
+
+
 @pytest.mark.parametrize("lengths", [[1, 63, 64, 65, 130, 0, 200], [0], [5], [300, 0, 0, 64]])
 def test_varlen_ragged_and_empty(lengths):
     inp = synth.make_prefill(synth.VARLEN, DEV, H=4, lengths=lengths)
