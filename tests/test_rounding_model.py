@@ -5,7 +5,9 @@ numbers that anyone can reproduce without a GPU:
 * the triangular solve's 32x32 block products in plain tf32 give the same
   end-to-end error as exact products (the fp16 operands and the bf16 output
   set the error);
-* fp16 tensor-core operands are more accurate than bf16 ones.
+* fp16 tensor-core operands are more accurate than bf16 ones;
+* (for a planned tensor-core solve) the WY pseudo-values formed by blocked
+  substitution with fp16 operands keep the same error.
 
 The model follows the chunk form of the Kimi K3 digest ("Kimi Delta Attention"
 section; chunk output = inter-chunk (Gamma . Q) S + intra-chunk A V~) with the
@@ -117,3 +119,57 @@ def test_bf16_operands_are_less_accurate_than_fp16(case):
     eb = run(case, bf16, False)
     assert eb[0] > 2.0 * e16[0]  # output relative Frobenius error
     assert eb[2] > 2.0 * e16[2]  # final-state relative Frobenius error
+
+
+def model_blocked_wy(q, k, v, g, beta, s0, C=64):
+    """The same chunk form with [W' | U] = (I + A)^-1 diag(beta) [KE | V] by
+    blocked forward substitution over 16-row blocks, every product taking fp16
+    operands (A, the diagonal-block inverses, the right-hand sides and the
+    finished blocks) with fp32 accumulation; U stays fp32."""
+    T = q.shape[0]
+    S = s0.astype(np.float32).copy()
+    O = np.zeros((T, v.shape[1]), np.float32)
+    dk = q.shape[1]
+    for c0 in range(0, T, C):
+        sl = slice(c0, c0 + C)
+        Q, K, V, b = q[sl], k[sl], v[sl], beta[sl]
+        G = np.cumsum(g[sl].astype(np.float32), 0)
+        GC = G[-1]
+        S1 = np.exp(GC)[:, None] * S
+        QE, KE, KH = f16(Q * np.exp(G - GC)), f16(K * np.exp(G - GC)), f16(K * np.exp(GC - G))
+        P = f16(np.tril(QE @ KH.T))
+        A = np.tril(b[:, None] * (KE @ KH.T), -1).astype(np.float32)
+        rhs = np.concatenate([b[:, None] * KE, b[:, None] * V], 1).astype(np.float32)
+        X = np.zeros_like(rhs)
+        Xh = np.zeros_like(rhs)
+        for i in range(4):
+            r = slice(16 * i, 16 * i + 16)
+            Ei = np.linalg.inv(np.eye(16) + A[r, r].astype(np.float64)).astype(np.float32)
+            R = rhs[r] - f16(A[r, :16 * i]) @ Xh[:16 * i]
+            X[r] = f16(Ei) @ f16(R)
+            Xh[r] = f16(X[r])
+        W, U = Xh[:, :dk], X[:, dk:]
+        SS = f16(S1)
+        Delta = f16(U - W @ SS)
+        O[sl] = QE @ SS + P @ Delta
+        S = S1 + KH.T @ Delta
+    return bf16(O), S
+
+
+def test_blocked_substitution_with_fp16_operands_meets_the_bar(case):
+    inp, o_ref, f_ref = case
+    f = lambda t, h: t[0, :, h].float().numpy()
+    outs, fins = [], []
+    for h in range(2):
+        o, s = model_blocked_wy(f(inp["q"], h), f(inp["k"], h), f(inp["v"], h), f(inp["g"], h),
+                                inp["beta"][0, :, h].numpy(), inp["init_state"][0, h].numpy())
+        outs.append(o)
+        fins.append(s)
+    O = np.stack(outs, 1)[None]
+    e = errors(O, o_ref)
+    excess = float((np.abs(O - o_ref) - half_ulp_bf16(o_ref)).max()) / e["rms"]
+    srel = errors(np.stack(fins)[None], f_ref)["rel_fro"]
+    cur = run(case, f16, False)
+    assert e["rel_fro"] < 5e-3 and excess < 3e-2 and srel < 5e-3
+    # measured: 1.72e-3 / 2.45e-3 / 3.63e-4, against 1.72e-3 / 2.45e-3 / 3.93e-4 now
+    assert e["rel_fro"] <= 1.10 * cur[0] and srel <= 1.10 * cur[2]
