@@ -3,16 +3,20 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
     python bench.py --impl reference ...      # the fp64 CPU oracle arm
+    python bench.py --capture NAME            # a few launches of a small case, for ncu
     python bench.py --phases [--workload NAME] # per-phase cycles (test-hook build)
     python bench.py --chains 64,96,148        # time per chunk against concurrent chains
 
 Default workload: the model-shaped prefill B=1, H=96, T=65536, dk=dv=128,
 bf16 q/k/v/o with fp32 log-decay, beta and state (the 64K pretraining
 context with the model's 96 heads).  One step = one kda_fwd over that batch.
-The same run also times the B=512, H=96 single-token decode (one
-kda_decode_step per step, state updated in place) and reports it under
-"decode".  Inputs are synthetic (seeded), resident in HBM before the timed
-region, and far larger than the 126 MB L2, so no flush is needed.
+The same run also times, each under its own key: the B=512, H=96
+single-token decode ("decode": one kda_decode_step per step, state updated
+in place) and the other prefill workloads ("workloads": the mid batch
+B=2 H=16 T=4096, the packed 1M-token batch, and the model-range decay case).
+Inputs are synthetic (seeded) and resident in HBM before the timed region;
+workloads smaller than the 126 MB L2 (or close to it) get an L2 flush before
+every timed launch, the others are far larger than L2.
 
 Metric: Mtoken-heads/s = tokens x heads / time / 1e6, plus the fraction of
 the HBM roofline (measured copy bandwidth from MEASURED_PEAKS.json).
@@ -67,28 +71,38 @@ def decode_bytes(B, H, dk, dv, io_bytes):
     return B * H * (2 * dk * dv * 4 + io_bytes * (2 * dk + 2 * dv) + 4 * dk + 4)
 
 
-def tc_kernel_sha():
-    src = os.path.join(ROOT, "gated_delta_rule_121_b200", "csrc", "kda_fwd_tc.cu")
+def source_sha(name):
+    src = os.path.join(ROOT, "gated_delta_rule_121_b200", "csrc", name)
     return hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
 
 
-def profiled_traffic(workload):
-    """DRAM bytes per launch of the tensor-core kernel from the committed ncu
-    summary, or None when it is missing or the kernel changed since."""
-    p = os.path.join(ROOT, "profiles", f"kda_fwd_tc_{workload}_traffic.txt")
-    if not os.path.exists(p):
-        return None
+def read_kv(path):
     kv = {}
-    for line in open(p):
-        if "=" in line and not line.startswith("#"):
+    for line in open(path):
+        if "=" in line and not line.lstrip().startswith("#"):
             k, v = line.strip().split("=", 1)
             kv[k.strip()] = v.strip()
-    if kv.get("kernel_source_sha256") != tc_kernel_sha():
+    return kv
+
+
+def scaled_traffic(profile, source, units, fixed_bytes):
+    """DRAM bytes per launch of a kernel from a committed ncu capture of a
+    smaller case of the same kernel, scaled to this launch: the capture's
+    bytes beyond its fixed part (states) per unit (token-head or decoded
+    head), times this launch's units, plus this launch's fixed part.  None when
+    the capture is missing or the kernel source changed since it was taken."""
+    p = os.path.join(ROOT, "profiles", profile)
+    if not os.path.exists(p):
+        return None
+    kv = read_kv(p)
+    if kv.get("kernel_source_sha256") != source_sha(source):
         return None
     try:
-        return float(kv["traffic_bytes_per_launch"])
-    except (KeyError, ValueError):
+        measured = float(kv["dram_bytes_read"]) + float(kv["dram_bytes_write"])
+        per_unit = (measured - float(kv["capture_fixed_bytes"])) / float(kv["capture_units"])
+    except (KeyError, ValueError, ZeroDivisionError):
         return None
+    return per_unit * units + fixed_bytes
 
 
 class ClockSampler:
@@ -158,6 +172,29 @@ def time_loop(fn, steps, warmup, stream, dist_ctx):
     torch.cuda.synchronize()
     dist_ctx.barrier()
     return t0.elapsed_time(t1) / 1000.0
+
+
+def time_loop_flushed(fn, steps, warmup, stream, dist_ctx, flush_bytes=256 << 20):
+    """Device time of `steps` launches of fn, each after a write of a buffer
+    twice the size of L2 (so no launch finds its inputs in L2); only the
+    launches are inside the timed events."""
+    import torch
+    buf = torch.empty(flush_bytes, dtype=torch.uint8, device=torch.cuda.current_device())
+    for _ in range(warmup):
+        fn()
+    dist_ctx.barrier()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    with torch.cuda.stream(stream):
+        for e0, e1 in ev:
+            buf.fill_(1)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+    torch.cuda.synchronize()
+    dist_ctx.barrier()
+    del buf
+    return sum(e0.elapsed_time(e1) for e0, e1 in ev) / 1000.0
 
 
 class Dist:
@@ -267,6 +304,65 @@ def run_reference(args, d):
 
 
 # ----------------------------------------------------------------- native arm
+# ncu captures that give the DRAM traffic of a full launch (scaled by units):
+# (profile file, kernel source, unit) per kernel.
+TRAFFIC_PROFILES = {
+    "kda_fwd_tc_kernel": ("kda_fwd_tc_prefill_h96_t4096_traffic.txt", "kda_fwd_tc.cu"),
+    "kda_decode_kernel": ("kda_decode_b64_h96_traffic.txt", "kda_decode.cu"),
+}
+FLUSH = {"mid": True, "stress": True, "prefill64k": False, "varlen": False}
+
+
+def bench_prefill(name, d, dev, stream, peaks, kda, synth, steps, warmup, with_traffic=False):
+    """Time `steps` kda_fwd launches over one workload; returns its JSON object
+    and the inputs (for the end-to-end leg)."""
+    import torch
+    spec = workload_spec(name)
+    inp = synth.make_prefill(spec, dev)
+    q, k, v, g, beta, init, cu = (inp[n] for n in ("q", "k", "v", "g", "beta", "init_state", "cu_seqlens"))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    N = cu.numel() - 1 if cu is not None else B
+    th = B * T * H
+    out = torch.empty_like(v)
+    fin = torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev)
+    ws = kda.alloc_workspace(N, B * T, H, dk, dv, q.dtype, dev)
+
+    def step():
+        kda.kda_fwd(q, k, v, g, beta, init, cu, out=out, final_state=fin, workspace=ws, stream=stream)
+
+    flush = FLUSH[name]
+    sec = (time_loop_flushed if flush else time_loop)(step, steps, warmup, stream, d)
+    status = kda.kda_workspace_status(ws, stream)
+    if status != kda.KDA_OK:
+        raise RuntimeError(f"{name}: device status {kda.kda_status_string(status)}")
+    per_step = d.max(sec) / steps
+    bytes_alg = prefill_bytes(th, N * H, dk, dv, q.element_size(), init is not None)
+    flops_alg = prefill_flops(th, dk, dv)
+    achieved = bytes_alg / per_step / 1e9
+    peak = peaks["hbm_gbs"]
+    t_roof = max(bytes_alg / (peak * 1e9), flops_alg / (peaks["bf16_tflops"] * 1e12))
+    traffic = None
+    if with_traffic:
+        prof, src = TRAFFIC_PROFILES["kda_fwd_tc_kernel"]
+        fixed = N * H * dk * dv * 4 * (2 if init is not None else 1)
+        traffic = scaled_traffic(prof, src, th, fixed)
+    launches = 2 if (cu is not None and N > 1) else 1  # packed batches: the order kernel, then the forward
+    res = {"workload": spec.name, "value": job_throughput(d, th * steps, sec) / 1e6, "unit": UNIT,
+           "ms_per_step": per_step * 1e3, "steps": steps, "sequences": N, "token_heads": th,
+           "l2": ("flushed before every launch (256 MB write)" if flush else
+                  "inputs larger than L2 (%.1f GB per step), no flush" % (bytes_alg / 1e9)),
+           "pct_of_roofline": 100.0 * t_roof / per_step,
+           "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                        "frac": achieved / peak, "traffic": traffic, "bytes_per_launch": bytes_alg,
+                        "kernel": "kda_fwd_tc_kernel",
+                        "tensor_tflops": flops_alg / per_step / 1e12,
+                        "tensor_frac_of_bf16_peak": flops_alg / per_step / 1e12 / peaks["bf16_tflops"]},
+           "gpu_launches": steps * launches}
+    del out, fin, ws
+    return res, inp
+
+
 def run_native(args, d):
     import torch
 
@@ -277,56 +373,41 @@ def run_native(args, d):
     dev = torch.device("cuda", d.local)
     d.init("nccl")
     peaks, peak_src = load_peaks()
-    spec = workload_spec(args.workload)
     stream = torch.cuda.current_stream(dev)
-
-    inp = synth.make_prefill(spec, dev)
-    q, k, v, g, beta, init, cu = (inp[n] for n in ("q", "k", "v", "g", "beta", "init_state", "cu_seqlens"))
-    B, T, H, dk = q.shape
-    dv = v.shape[-1]
-    N = cu.numel() - 1 if cu is not None else B
-    tokens = B * T
-    th = tokens * H
-    out = torch.empty_like(v)
-    fin = torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev)
-    ws = kda.alloc_workspace(N, tokens, H, dk, dv, q.dtype, dev)
-    io_bytes = q.element_size()
-
-    def step():
-        kda.kda_fwd(q, k, v, g, beta, init, cu, out=out, final_state=fin, workspace=ws, stream=stream)
-
     uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid).replace("GPU-", "")
-    with ClockSampler(uuid) as clk:
-        sec = time_loop(step, args.steps, args.warmup, stream, d)
-    status = kda.kda_workspace_status(ws, stream)
-    if status != kda.KDA_OK:
-        raise RuntimeError(f"device status {kda.kda_status_string(status)}")
-    value = job_throughput(d, th * args.steps, sec) / 1e6
-    per_step = d.max(sec) / args.steps
-    bytes_alg = prefill_bytes(th, N * H, dk, dv, io_bytes, init is not None)
-    flops_alg = prefill_flops(th, dk, dv)
-    achieved = bytes_alg / per_step / 1e9
-    peak = peaks["hbm_gbs"]
-    t_roof = max(bytes_alg / (peak * 1e9), flops_alg / (peaks["bf16_tflops"] * 1e12))
-    traffic = profiled_traffic(args.workload)
-    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": d.world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": per_step * 1e3, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16" if q.dtype == torch.bfloat16 else "f32", "data": "synthetic",
-            "config": {"workload": spec.name, "B": B, "T": T, "H": H, "dk": dk, "dv": dv, "sequences": N,
-                       "chunk": CHUNK, "l2": "inputs larger than L2 (%.1f GB per step), no flush" %
-                       (bytes_alg / 1e9), "parallelism": f"dp{d.world} independent replicas, no collective"},
-            "pct_of_roofline": 100.0 * t_roof / per_step,
-            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": traffic, "peak_source": peak_src,
-                         "bytes_per_launch": bytes_alg, "kernel": "kda_fwd_tc_kernel",
-                         "tensor_tflops": flops_alg / per_step / 1e12,
-                         "tensor_frac_of_bf16_peak": flops_alg / per_step / 1e12 / peaks["bf16_tflops"]},
-            "gpu_launches": args.steps * (2 if (cu is not None and N > 1) else 1), "clocks": clk.summary()}
 
+    with ClockSampler(uuid) as clk:
+        main, inp = bench_prefill(args.workload, d, dev, stream, peaks, kda, synth, args.steps, args.warmup,
+                                  with_traffic=args.workload == "prefill64k")
+    q, v = inp["q"], inp["v"]
+    B, T, H, dk = q.shape
+    spec = workload_spec(args.workload)
+    main["roofline"]["peak_source"] = peak_src
+    line = {"metric": METRIC, "value": main["value"], "unit": UNIT, "n_gpus": d.world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": main["ms_per_step"], "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if q.dtype == torch.bfloat16 else "f32",
+            "data": "synthetic",
+            "config": {"workload": spec.name, "B": B, "T": T, "H": H, "dk": dk, "dv": v.shape[-1],
+                       "sequences": main["sequences"], "chunk": CHUNK, "l2": main["l2"],
+                       "parallelism": f"dp{d.world} independent replicas, no collective"},
+            "pct_of_roofline": main["pct_of_roofline"], "roofline": main["roofline"],
+            "gpu_launches": main["gpu_launches"], "clocks": clk.summary()}
+
+    if not args.no_e2e:
+        line["e2e"] = bench_e2e(args, d, dev, stream, inp, kda, B * T * H)
+    del inp
+    torch.cuda.empty_cache()
     if not args.no_decode:
         line["decode"] = bench_decode(args, d, dev, stream, peaks, kda, synth)
-    if not args.no_e2e:
-        line["e2e"] = bench_e2e(args, d, dev, stream, inp, kda, th)
+    if not args.no_workloads:
+        others = {}
+        for name, steps in (("mid", 50), ("varlen", 8), ("stress", 50)):
+            if name == args.workload:
+                continue
+            res, _ = bench_prefill(name, d, dev, stream, peaks, kda, synth, steps, args.warmup)
+            others[name] = res
+            torch.cuda.empty_cache()
+        line["workloads"] = others
     if d.world == 1 and d.rank == 0 and not args.no_cpu_baseline:
         import oracle
         line["cpu_baseline"] = {k: v for k, v in oracle_sample(spec, 12.0, oracle.default_threads()).items()
@@ -354,32 +435,70 @@ def bench_decode(args, d, dev, stream, peaks, kda, synth):
     per = d.max(sec) / args.steps
     nbytes = decode_bytes(spec.B, spec.H, spec.dk, spec.dv, 2)
     ach = nbytes / per / 1e9
+    prof, src = TRAFFIC_PROFILES["kda_decode_kernel"]
+    traffic = scaled_traffic(prof, src, spec.B * spec.H, 0.0)
     del xs, state
     return {"workload": spec.name, "value": value, "unit": UNIT,
             "ms_per_step": per * 1e3, "gpu_launches": args.steps,
+            "l2": "state 3.2 GB per step, far larger than L2, no flush",
             "roofline": {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": ach / peaks["hbm_gbs"], "traffic": None, "bytes_per_launch": nbytes,
+                         "frac": ach / peaks["hbm_gbs"], "traffic": traffic, "bytes_per_launch": nbytes,
                          "kernel": "kda_decode_kernel<128,128,bf16>"}}
 
 
 def bench_e2e(args, d, dev, stream, inp, kda, th):
-    """Same metric through the public API from pinned host buffers: every
-    step copies the inputs host->device and the output and final state back."""
+    """Same metric through the C entry point kda_fwd_host from pinned host
+    buffers: every step copies the inputs host->device and the output and
+    final state back, all enqueued by that one call."""
     import torch
     host = {n: (t.cpu().pin_memory() if t is not None else None) for n, t in inp.items()}
     bufs = {}
     steps = max(1, min(args.steps, 5))
 
     def step():
-        o, f, _ = kda.kda_fwd_host(host["q"], host["k"], host["v"], host["g"], host["beta"], host["init_state"],
-                                   host["cu_seqlens"], device=dev, stream=stream, dev_buffers=bufs)
+        kda.kda_fwd_host(host["q"], host["k"], host["v"], host["g"], host["beta"], host["init_state"],
+                         host["cu_seqlens"], device=dev, stream=stream, dev_buffers=bufs)
 
+    step()  # allocates the device buffers outside the timed region
     sec = time_loop(step, steps, args.warmup, stream, d)
     h2d = sum(t.numel() * t.element_size() for n, t in host.items() if t is not None)
     d2h = bufs["out_h"].numel() * bufs["out_h"].element_size() + bufs["fin_h"].numel() * 4
     value = job_throughput(d, th * steps, sec) / 1e6
-    return {"value": value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+    del bufs, host
+    return {"value": value, "unit": UNIT, "h2d_bytes_per_step": h2d, "entry_point": "kda_fwd_host",
             "d2h_bytes_per_step": d2h, "steps": steps, "ms_per_step": d.max(sec) / steps * 1e3}
+
+
+# Small cases for ncu counter captures (a few GB on the device at most,
+# inputs larger than L2); the traffic files under profiles/ name the case.
+CAPTURES = {
+    "prefill_h96_t4096": "B=1 H=96 T=4096 d=128 bf16 prefill (the 64K workload's heads, 1/16 of its tokens)",
+    "mid": "B=2 H=16 T=4096 d=128 bf16 prefill with initial states",
+    "decode_b64_h96": "B=64 H=96 d=128 bf16 decode step (1/8 of the decode workload's sequences)",
+}
+
+
+def run_capture(args):
+    """A few launches of one small case, nothing else: the command ncu wraps."""
+    import torch
+
+    import gated_delta_rule_121_b200 as kda
+    import synth
+    dev = torch.device("cuda")
+    n = max(1, args.steps)
+    if args.capture == "decode_b64_h96":
+        spec = synth.DECODE
+        state = synth.make_decode_state(spec, dev, B=64)
+        x = synth.make_decode_step(spec, 0, dev, B=64)
+        for _ in range(n):
+            kda.kda_decode_step(x["q"], x["k"], x["v"], x["g"], x["beta"], state)
+    else:
+        spec = synth.PRETRAIN if args.capture == "prefill_h96_t4096" else synth.MID
+        inp = synth.make_prefill(spec, dev, T=4096)
+        for _ in range(n):
+            kda.kda_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["init_state"], inp["cu_seqlens"])
+    torch.cuda.synchronize()
+    print(json.dumps({"capture": args.capture, "what": CAPTURES[args.capture], "launches": n}), flush=True)
 
 
 # Phase boundaries recorded by the tensor-core kernel's test hook (chain 0):
@@ -473,6 +592,9 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true", help="skip the mid, varlen and stress objects")
+    ap.add_argument("--capture", choices=sorted(CAPTURES), default=None,
+                    help="run --steps launches of a small case (for ncu), nothing else")
     ap.add_argument("--phases", action="store_true",
                     help="print per-phase cycles of the tensor-core kernel (test hook) instead of timing")
     ap.add_argument("--chains", default=None,
@@ -482,7 +604,9 @@ def main():
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
     d = Dist()
-    if args.phases:
+    if args.capture:
+        run_capture(args)
+    elif args.phases:
         run_phases(args)
     elif args.chains:
         run_chains(args)

@@ -10,8 +10,9 @@ Functions mirror the C entry points:
   kda_fwd_noalloc(...)                           the same, scratch in a fixed library array
   kda_decode_step(q, k, v, log_alpha, beta, state, ...)   in-place decode
   kda_fwd_workspace_size(...), kda_workspace_status(ws), kda_status_string(s)
-and ``kda_fwd_host`` runs kda_fwd on host (pinned) tensors, copying inputs in
-and outputs back on the given stream.
+and ``kda_fwd_host`` runs kda_fwd on host (pinned) tensors through the C
+entry point of the same name, which copies inputs in and outputs back on the
+given stream.
 """
 from __future__ import annotations
 
@@ -62,9 +63,14 @@ def lib() -> ctypes.CDLL:
         L.kda_testing_fwd_path.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int]
         L.kda_fwd_noalloc.restype = ctypes.c_int
         L.kda_fwd_noalloc.argtypes = fwd_args[:-2]
+        L.kda_fwd_noalloc_status.restype = ctypes.c_int
+        L.kda_fwd_noalloc_status.argtypes = [_vp]
         L.kda_decode_step.restype = ctypes.c_int
         L.kda_decode_step.argtypes = [_vp, _vp, _vp, _fp, _fp, _fp, _vp, ctypes.c_int, ctypes.c_int,
                                       ctypes.c_int, ctypes.c_int, _vp, ctypes.c_int]
+        L.kda_fwd_host.restype = ctypes.c_int
+        L.kda_fwd_host.argtypes = [_vp, _vp, ctypes.c_int, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                   _vp, ctypes.c_int, _vp, ctypes.c_size_t]
         L.kda_workspace_status.restype = ctypes.c_int
         L.kda_workspace_status.argtypes = [_vp, _vp]
         _lib = L
@@ -141,9 +147,9 @@ def kda_fwd(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None, out=None
         final_state = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
     if workspace is None:
         workspace = alloc_workspace(N, B * T, H, dk, dv, q.dtype, q.device)
-    Targ = T if cu_seqlens is None else T  # packed: T is the total token count
+    # packed: T is the total token count, the per-sequence length otherwise
     args = (_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(init_state), _ptr(out),
-            _ptr(final_state), N, Targ, H, dk, dv, _ptr(cu_seqlens), _stream_ptr(stream), dt,
+            _ptr(final_state), N, T, H, dk, dv, _ptr(cu_seqlens), _stream_ptr(stream), dt,
             _ptr(workspace), workspace.numel())
     if _debug is None and _wait_ns is None and not _inject_stuck:
         code = lib().kda_fwd(*args)
@@ -171,6 +177,12 @@ def kda_fwd_noalloc(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None, 
     return out, final_state
 
 
+def kda_fwd_noalloc_status(stream=None) -> int:
+    """Device status of the last kda_fwd_noalloc call on the current device
+    (synchronises the stream)."""
+    return int(lib().kda_fwd_noalloc_status(_stream_ptr(stream)))
+
+
 def kda_decode_step(q, k, v, log_alpha, beta, state, out=None, stream=None):
     """One decode step; ``state`` [B,H,dk,dv] fp32 is updated in place.
     q,k,log_alpha: [B,H,dk]; v: [B,H,dv]; beta: [B,H].  Returns out [B,H,dv]."""
@@ -189,39 +201,47 @@ def kda_decode_step(q, k, v, log_alpha, beta, state, out=None, stream=None):
     return out
 
 
+class _FwdTensors(ctypes.Structure):
+    """kda_fwd_tensors_t: the pointers of one kda_fwd call."""
+    _fields_ = [(n, ctypes.c_void_p) for n in ("q", "k", "v", "log_alpha", "beta", "init_state", "cu_seqlens",
+                                                 "out", "final_state")]
+
+
+def _tensors(d):
+    return _FwdTensors(*[None if d.get(n) is None else d[n].data_ptr() for n, _ in _FwdTensors._fields_])
+
+
 def kda_fwd_host(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None, device="cuda", stream=None,
                  dev_buffers=None):
-    """kda_fwd on host tensors (pinned for asynchronous copies): copies the
-    inputs to ``device``, runs the forward and copies ``out`` and the final
-    state back.  ``dev_buffers`` (a dict returned by a previous call) lets
-    repeated calls reuse device memory.  Returns (out_host, final_host,
-    dev_buffers)."""
+    """kda_fwd on host tensors through the C entry point kda_fwd_host: one call
+    enqueues the host-to-device copies of the inputs (pinned memory makes them
+    asynchronous), the forward, and the copies of ``out`` and the final state
+    back.  ``dev_buffers`` (a dict returned by a previous call) holds the
+    device buffers and the pinned host outputs for repeated calls.  Returns
+    (out_host, final_host, dev_buffers); synchronise the stream before reading
+    the host outputs."""
     s = stream if stream is not None else torch.cuda.current_stream(device)
+    B, T, H, dk, dv, N = _shapes(q, v, cu_seqlens)
+    host_in = dict(q=q, k=k, v=v, log_alpha=log_alpha, beta=beta, init_state=init_state, cu_seqlens=cu_seqlens)
     if dev_buffers is None:
         dev_buffers = {}
-    def dev(name, t):
-        if t is None:
-            return None
-        b = dev_buffers.get(name)
-        if b is None or b.shape != t.shape or b.dtype != t.dtype:
-            b = dev_buffers[name] = torch.empty(t.shape, dtype=t.dtype, device=device)
-        b.copy_(t, non_blocking=True)
-        return b
-    with torch.cuda.stream(s):
-        dq, dk_, dv_, dg, db = (dev(n, t) for n, t in (("q", q), ("k", k), ("v", v), ("g", log_alpha),
-                                                        ("beta", beta)))
-        di = dev("init", init_state)
-        dcu = dev("cu", cu_seqlens)
-        B, T, H, dk, dv, N = _shapes(q, v, cu_seqlens)
-        if "out" not in dev_buffers or dev_buffers["out"].shape != (B, T, H, dv):
-            dev_buffers["out"] = torch.empty((B, T, H, dv), dtype=q.dtype, device=device)
-            dev_buffers["fin"] = torch.empty((N, H, dk, dv), dtype=torch.float32, device=device)
-            dev_buffers["ws"] = alloc_workspace(N, B * T, H, dk, dv, q.dtype, device)
-        kda_fwd(dq, dk_, dv_, dg, db, di, dcu, out=dev_buffers["out"], final_state=dev_buffers["fin"],
-                workspace=dev_buffers["ws"], stream=s)
-        if "out_h" not in dev_buffers or dev_buffers["out_h"].shape != (B, T, H, dv):
-            dev_buffers["out_h"] = torch.empty((B, T, H, dv), dtype=q.dtype, pin_memory=True)
-            dev_buffers["fin_h"] = torch.empty((N, H, dk, dv), dtype=torch.float32, pin_memory=True)
-        dev_buffers["out_h"].copy_(dev_buffers["out"], non_blocking=True)
-        dev_buffers["fin_h"].copy_(dev_buffers["fin"], non_blocking=True)
+    if dev_buffers.get("_shape") != (B, T, H, dk, dv, N, q.dtype):
+        dev_buffers.clear()
+        dev_buffers["_shape"] = (B, T, H, dk, dv, N, q.dtype)
+        dev = {n: (None if t is None else torch.empty(t.shape, dtype=t.dtype, device=device))
+               for n, t in host_in.items()}
+        dev["out"] = torch.empty((B, T, H, dv), dtype=q.dtype, device=device)
+        dev["final_state"] = torch.empty((N, H, dk, dv), dtype=torch.float32, device=device)
+        dev_buffers["dev"] = dev
+        dev_buffers["ws"] = alloc_workspace(N, B * T, H, dk, dv, q.dtype, device)
+        dev_buffers["out_h"] = torch.empty((B, T, H, dv), dtype=q.dtype, pin_memory=True)
+        dev_buffers["fin_h"] = torch.empty((N, H, dk, dv), dtype=torch.float32, pin_memory=True)
+    host = dict(host_in, out=dev_buffers["out_h"], final_state=dev_buffers["fin_h"])
+    for n, t in host_in.items():
+        if t is not None and (t.device.type != "cpu" or not t.is_contiguous()):
+            raise ValueError(f"{n}: expected a contiguous host tensor")
+    ws = dev_buffers["ws"]
+    code = lib().kda_fwd_host(ctypes.byref(_tensors(host)), ctypes.byref(_tensors(dev_buffers["dev"])), N, T, H,
+                              dk, dv, ctypes.c_void_p(s.cuda_stream), _DT[q.dtype], _ptr(ws), ws.numel())
+    _check(code, "kda_fwd_host")
     return dev_buffers["out_h"], dev_buffers["fin_h"], dev_buffers

@@ -10,7 +10,13 @@
 
 namespace kda {
 cudaError_t launch_fwd_tc_impl(const FwdArgs& a, cudaStream_t s, uint64_t wait_ns, int inject_stuck,
-                               int32_t* order_ws);
+                               int32_t* order_ws, const ModeArgs& ma);
+cudaError_t launch_ckpt_base(const int32_t* cu, int N, int interval, int32_t* base, cudaStream_t s);
+cudaError_t launch_compose(const float* trans, const float* s0, const float* init, float* state_in, float* fin,
+                           int R, int N, int H, int dk, int dv, int rank_major, cudaStream_t s);
+cudaError_t launch_correct(const float* o32, const float* qhat, const float* s_in, void* out, const int32_t* cu,
+                           int P, int64_t Tper, int64_t Ttot, int H, int dk, int dv, bool bf16, cudaStream_t s);
+cudaError_t launch_segment_cu(const int32_t* cu, int64_t Tper, int N, int R, int32_t* seg_cu, cudaStream_t s);
 int fwd_tc_debug_floats();
 }  // namespace kda
 
@@ -66,8 +72,10 @@ static kda_status_t fwd_impl(const void* q, const void* k, const void* v, const 
                              const float* beta, const float* init_state, void* out, float* final_state, int B,
                              int64_t T, int H, int dk, int dv, const int32_t* cu_seqlens, void* stream,
                              kda_dtype_t dt, void* workspace, size_t workspace_bytes, float* dbg,
-                             uint64_t wait_ns, int inject_stuck) {
-  kda_status_t st = validate_fwd(q, k, v, log_alpha, beta, init_state, out, final_state, B, T, H, dk, dv, dt);
+                             uint64_t wait_ns, int inject_stuck, const kda::ModeArgs& ma = kda::ModeArgs()) {
+  // Segment runs write fp32 outputs to their own buffers (out may be NULL).
+  const void* out_chk = ma.mode == kda::MODE_SEG ? (const void*)ma.o32 : out;
+  kda_status_t st = validate_fwd(q, k, v, log_alpha, beta, init_state, out_chk, final_state, B, T, H, dk, dv, dt);
   if (st != KDA_OK) return st;
   if (cu_seqlens && !aligned16(cu_seqlens)) return KDA_ERR_INVALID_ARG;
   if (!workspace || !aligned16(workspace) || workspace_bytes < kda_fwd_workspace_size(B, T, H, dk, dv, dt))
@@ -84,11 +92,11 @@ static kda_status_t fwd_impl(const void* q, const void* k, const void* v, const 
   const int64_t tokens = cu_seqlens ? T : (int64_t)B * T;
   if (kda::fwd_tc_supported(dk, dv, bf16) && tokens > 0)
     e = kda::launch_fwd_tc_impl(a, s, wait_ns, inject_stuck,
-                                reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + kStatusBytes));
+                                reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + kStatusBytes), ma);
   else if (dbg || inject_stuck)
     return KDA_ERR_UNSUPPORTED;
   else
-    e = kda::launch_fwd_simt(a, bf16, s);
+    e = kda::launch_fwd_simt(a, bf16, s, ma);
   return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
@@ -98,6 +106,50 @@ kda_status_t kda_fwd(const void* q, const void* k, const void* v, const float* l
                      size_t workspace_bytes) {
   return fwd_impl(q, k, v, log_alpha, beta, init_state, out, final_state, B, T, H, dk, dv, cu_seqlens, stream,
                   dt, workspace, workspace_bytes, nullptr, 2000000000ull, 0);
+}
+
+kda_status_t kda_fwd_host(const kda_fwd_tensors_t* host, const kda_fwd_tensors_t* dev, int B, int64_t T, int H,
+                          int dk, int dv, void* stream, kda_dtype_t dt, void* workspace, size_t workspace_bytes) {
+  if (!host || !dev) return KDA_ERR_INVALID_ARG;
+  if ((host->init_state == nullptr) != (dev->init_state == nullptr) ||
+      (host->cu_seqlens == nullptr) != (dev->cu_seqlens == nullptr))
+    return KDA_ERR_INVALID_ARG;
+  if (B < 0 || T < 0 || H <= 0 || (dt != KDA_F32 && dt != KDA_BF16)) return KDA_ERR_INVALID_ARG;
+  const bool packed = dev->cu_seqlens != nullptr;
+  const int64_t tokens = packed ? T : (int64_t)B * T;
+  const size_t esz = dt == KDA_BF16 ? 2 : 4;
+  const size_t th = (size_t)tokens * H;
+  const size_t states = (size_t)B * H * dk * dv * sizeof(float);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  struct Copy {
+    void* dst;
+    const void* src;
+    size_t bytes;
+  };
+  const Copy in[] = {{const_cast<void*>(dev->q), host->q, th * dk * esz},
+                     {const_cast<void*>(dev->k), host->k, th * dk * esz},
+                     {const_cast<void*>(dev->v), host->v, th * dv * esz},
+                     {const_cast<float*>(dev->log_alpha), host->log_alpha, th * dk * sizeof(float)},
+                     {const_cast<float*>(dev->beta), host->beta, th * sizeof(float)},
+                     {const_cast<float*>(dev->init_state), host->init_state, dev->init_state ? states : 0},
+                     {const_cast<int32_t*>(dev->cu_seqlens), host->cu_seqlens,
+                      packed ? (size_t)(B + 1) * sizeof(int32_t) : 0}};
+  for (const Copy& c : in) {
+    if (c.bytes == 0) continue;
+    if (!c.dst || !c.src) return KDA_ERR_INVALID_ARG;
+    if (cudaMemcpyAsync(c.dst, c.src, c.bytes, cudaMemcpyHostToDevice, s) != cudaSuccess) return KDA_ERR_CUDA;
+  }
+  kda_status_t st = kda_fwd(dev->q, dev->k, dev->v, dev->log_alpha, dev->beta, dev->init_state, dev->out,
+                            dev->final_state, B, T, H, dk, dv, dev->cu_seqlens, stream, dt, workspace,
+                            workspace_bytes);
+  if (st != KDA_OK) return st;
+  if (host->out && th > 0 &&
+      cudaMemcpyAsync(host->out, dev->out, th * dv * esz, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return KDA_ERR_CUDA;
+  if (host->final_state && dev->final_state && states > 0 &&
+      cudaMemcpyAsync(host->final_state, dev->final_state, states, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return KDA_ERR_CUDA;
+  return KDA_OK;
 }
 
 kda_status_t kda_decode_step(const void* q, const void* k, const void* v, const float* log_alpha,
@@ -123,6 +175,186 @@ kda_status_t kda_workspace_status(const void* workspace, void* stream) {
   if (cudaMemcpyAsync(&h, workspace, sizeof(h), cudaMemcpyDeviceToHost, s) != cudaSuccess) return KDA_ERR_CUDA;
   if (cudaStreamSynchronize(s) != cudaSuccess) return KDA_ERR_CUDA;
   return static_cast<kda_status_t>(h.code);
+}
+
+// ---- interval checkpoints (prefix-cache states) ----
+static size_t order_bytes(int N) { return ((size_t)(N > 0 ? N : 0) * sizeof(int32_t) + 255) / 256 * 256; }
+
+size_t kda_fwd_checkpoints_workspace_size(int B, int64_t T, int H, int dk, int dv, kda_dtype_t dt) {
+  return kda_fwd_workspace_size(B, T, H, dk, dv, dt) + order_bytes(B);
+}
+
+kda_status_t kda_fwd_checkpoints(const void* q, const void* k, const void* v, const float* log_alpha,
+                                 const float* beta, const float* init_state, void* out, float* final_state, int B,
+                                 int64_t T, int H, int dk, int dv, const int32_t* cu_seqlens, void* stream,
+                                 kda_dtype_t dt, float* checkpoints, int interval, int64_t capacity,
+                                 void* workspace, size_t workspace_bytes) {
+  if (interval <= 0 || interval % 64 != 0) return KDA_ERR_UNSUPPORTED;
+  if (capacity < 0 || (capacity > 0 && (!checkpoints || !aligned16(checkpoints)))) return KDA_ERR_INVALID_ARG;
+  if (!workspace || !aligned16(workspace) ||
+      workspace_bytes < kda_fwd_checkpoints_workspace_size(B, T, H, dk, dv, dt))
+    return KDA_ERR_WORKSPACE;
+  if (!cu_seqlens && B > 0 && (int64_t)B * (T / interval) > capacity) return KDA_ERR_INVALID_ARG;
+  kda::ModeArgs ma;
+  ma.mode = kda::MODE_CKPT;
+  ma.ckpt = checkpoints;
+  ma.ckpt_interval = interval;
+  ma.ckpt_every = interval / 64;
+  ma.ckpt_capacity = capacity;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cu_seqlens && B > 0) {
+    if (!aligned16(cu_seqlens)) return KDA_ERR_INVALID_ARG;
+    int32_t* base = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) +
+                                               kda_fwd_workspace_size(B, T, H, dk, dv, dt));
+    if (kda::launch_ckpt_base(cu_seqlens, B, interval, base, s) != cudaSuccess) return KDA_ERR_CUDA;
+    ma.ckpt_base = base;
+  }
+  return fwd_impl(q, k, v, log_alpha, beta, init_state, out, final_state, B, T, H, dk, dv, cu_seqlens, stream, dt,
+                  workspace, workspace_bytes, nullptr, 2000000000ull, 0, ma);
+}
+
+// ---- segment pieces, composition, correction (context parallelism) ----
+kda_status_t kda_segment_fwd(const void* q, const void* k, const void* v, const float* log_alpha,
+                             const float* beta, float* out_zero, float* state_zero, float* qhat,
+                             float* transition, int B, int64_t T, int H, int dk, int dv,
+                             const int32_t* cu_seqlens, void* stream, kda_dtype_t dt, void* workspace,
+                             size_t workspace_bytes) {
+  if (dk != dv) return KDA_ERR_UNSUPPORTED;
+  const int64_t tokens = cu_seqlens ? T : (int64_t)B * T;
+  if (tokens > 0 && (!out_zero || !qhat)) return KDA_ERR_INVALID_ARG;
+  if (B > 0 && (!state_zero || !transition)) return KDA_ERR_INVALID_ARG;
+  for (const void* p : {(const void*)out_zero, (const void*)qhat, (const void*)state_zero, (const void*)transition})
+    if (!aligned16(p)) return KDA_ERR_INVALID_ARG;
+  kda::ModeArgs ma;
+  ma.mode = kda::MODE_SEG;
+  ma.o32 = out_zero;
+  ma.qhat32 = qhat;
+  ma.trans = transition;
+  return fwd_impl(q, k, v, log_alpha, beta, nullptr, nullptr, state_zero, B, T, H, dk, dv, cu_seqlens, stream, dt,
+                  workspace, workspace_bytes, nullptr, 2000000000ull, 0, ma);
+}
+
+kda_status_t kda_state_compose(const float* transition, const float* state_zero, const float* init_state,
+                               float* state_in, float* final_state, int R, int N, int H, int dk, int dv,
+                               int rank_major, void* stream) {
+  if (R < 0 || N < 0 || H <= 0) return KDA_ERR_INVALID_ARG;
+  if (!dim_ok(dk) || !dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
+  if (R > 0 && N > 0 && (!transition || !state_zero)) return KDA_ERR_INVALID_ARG;
+  for (const void* p : {(const void*)transition, (const void*)state_zero, (const void*)init_state,
+                        (const void*)state_in, (const void*)final_state})
+    if (!aligned16(p)) return KDA_ERR_INVALID_ARG;
+  if (N == 0) return KDA_OK;
+  cudaError_t e = kda::launch_compose(transition, state_zero, init_state, state_in, final_state, R, N, H, dk, dv,
+                                      rank_major ? 1 : 0, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+kda_status_t kda_output_correct(const float* out_zero, const float* qhat, const float* state_in, void* out, int B,
+                                int64_t T, int H, int dk, int dv, const int32_t* cu_seqlens, void* stream,
+                                kda_dtype_t dt) {
+  if (B < 0 || T < 0 || H <= 0 || (dt != KDA_F32 && dt != KDA_BF16)) return KDA_ERR_INVALID_ARG;
+  if (!dim_ok(dk) || !dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
+  const int64_t tokens = cu_seqlens ? T : (int64_t)B * T;
+  if (tokens > (int64_t)INT32_MAX) return KDA_ERR_UNSUPPORTED;
+  if (tokens > 0 && (!out_zero || !qhat || !state_in || !out)) return KDA_ERR_INVALID_ARG;
+  for (const void* p : {(const void*)out_zero, (const void*)qhat, (const void*)state_in, (const void*)out,
+                        (const void*)cu_seqlens})
+    if (!aligned16(p)) return KDA_ERR_INVALID_ARG;
+  if (tokens == 0 || B == 0) return KDA_OK;
+  cudaError_t e = kda::launch_correct(out_zero, qhat, state_in, out, cu_seqlens, B, cu_seqlens ? 0 : T, tokens, H,
+                                      dk, dv, dt == KDA_BF16, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+// ---- intra-device context parallelism ----
+namespace {
+struct CpLayout {
+  size_t seg_cu, order, o32, qhat, s0, trans, s_in, total;
+};
+CpLayout cp_layout(int B, int64_t T, int H, int dk, int dv, int n_seg) {
+  auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+  const int64_t tokens = T;  // caller passes the total token count (B*T for batched inputs)
+  const size_t P = (size_t)(B > 0 ? B : 0) * (size_t)(n_seg > 0 ? n_seg : 1);
+  CpLayout L;
+  size_t off = kStatusBytes;
+  L.seg_cu = off; off += up((P + 1) * sizeof(int32_t));
+  L.order = off; off += up(P * sizeof(int32_t));
+  L.o32 = off; off += up((size_t)tokens * H * dv * sizeof(float));
+  L.qhat = off; off += up((size_t)tokens * H * dk * sizeof(float));
+  L.s0 = off; off += up(P * H * (size_t)dk * dv * sizeof(float));
+  L.trans = off; off += up(P * H * (size_t)dk * dk * sizeof(float));
+  L.s_in = off; off += up(P * H * (size_t)dk * dv * sizeof(float));
+  L.total = off;
+  return L;
+}
+}  // namespace
+
+size_t kda_fwd_cp_workspace_size(int B, int64_t T, int H, int dk, int dv, kda_dtype_t dt, int n_seg) {
+  (void)dt;
+  return cp_layout(B, T, H, dk, dv, n_seg).total;
+}
+
+int kda_cp_segments(int N, int64_t tokens_per_sequence, int H, int sm_count) {
+  // Two blocks per (segment, head) (the zero-start run and the transition run)
+  // must fit one wave of blocks on the SMs; a segment should keep at least
+  // eight 64-token chunks so the pipeline fill stays small against its length.
+  const int64_t chains = (int64_t)N * H;
+  if (chains <= 0 || sm_count <= 0) return 1;
+  int best = 1;
+  for (int r = 2; r <= 64; ++r) {
+    if (2 * chains * r > sm_count) break;
+    if (tokens_per_sequence / r < 8 * 64) break;
+    best = r;
+  }
+  return best;
+}
+
+kda_status_t kda_fwd_cp(const void* q, const void* k, const void* v, const float* log_alpha, const float* beta,
+                        const float* init_state, void* out, float* final_state, int B, int64_t T, int H, int dk,
+                        int dv, const int32_t* cu_seqlens, void* stream, kda_dtype_t dt, int n_seg,
+                        void* workspace, size_t workspace_bytes) {
+  if (n_seg < 1 || n_seg > 4096) return KDA_ERR_INVALID_ARG;
+  if (dk != dv) return KDA_ERR_UNSUPPORTED;
+  kda_status_t st = validate_fwd(q, k, v, log_alpha, beta, init_state, out, final_state, B, T, H, dk, dv, dt);
+  if (st != KDA_OK) return st;
+  if (cu_seqlens && !aligned16(cu_seqlens)) return KDA_ERR_INVALID_ARG;
+  const int64_t tokens = cu_seqlens ? T : (int64_t)B * T;
+  if (tokens > (int64_t)INT32_MAX || (int64_t)B * n_seg > (int64_t)INT32_MAX / 4) return KDA_ERR_UNSUPPORTED;
+  const CpLayout L = cp_layout(B, tokens, H, dk, dv, n_seg);
+  if (!workspace || !aligned16(workspace) || workspace_bytes < L.total) return KDA_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  if (cudaMemsetAsync(ws, 0, sizeof(kda::DeviceStatus), s) != cudaSuccess) return KDA_ERR_CUDA;
+  if (B == 0) return KDA_OK;
+  const int P = B * n_seg;
+  int32_t* seg_cu = reinterpret_cast<int32_t*>(ws + L.seg_cu);
+  float* o32 = reinterpret_cast<float*>(ws + L.o32);
+  float* qhat = reinterpret_cast<float*>(ws + L.qhat);
+  float* s0 = reinterpret_cast<float*>(ws + L.s0);
+  float* tr = reinterpret_cast<float*>(ws + L.trans);
+  float* s_in = reinterpret_cast<float*>(ws + L.s_in);
+  if (kda::launch_segment_cu(cu_seqlens, cu_seqlens ? 0 : T, B, n_seg, seg_cu, s) != cudaSuccess)
+    return KDA_ERR_CUDA;
+  // Pieces of every segment: the segments form a packed batch of P sequences
+  // over the same token tensors.  The status word of the workspace is shared;
+  // the order scratch follows it (L.order == kStatusBytes + aligned seg_cu).
+  kda::ModeArgs ma;
+  ma.mode = kda::MODE_SEG;
+  ma.o32 = o32;
+  ma.qhat32 = qhat;
+  ma.trans = tr;
+  kda::FwdArgs a{q, k, v, log_alpha, beta, nullptr, nullptr, s0, seg_cu, P, tokens, H, dk, dv,
+                 reinterpret_cast<kda::DeviceStatus*>(ws), nullptr};
+  cudaError_t e;
+  if (kda::fwd_tc_supported(dk, dv, dt == KDA_BF16) && tokens > 0)
+    e = kda::launch_fwd_tc_impl(a, s, 2000000000ull, 0, reinterpret_cast<int32_t*>(ws + L.order), ma);
+  else
+    e = kda::launch_fwd_simt(a, dt == KDA_BF16, s, ma);
+  if (e != cudaSuccess) return KDA_ERR_CUDA;
+  e = kda::launch_compose(tr, s0, init_state, s_in, final_state, n_seg, B, H, dk, dv, 0, s);
+  if (e != cudaSuccess) return KDA_ERR_CUDA;
+  e = kda::launch_correct(o32, qhat, s_in, out, seg_cu, P, 0, tokens, H, dk, dv, dt == KDA_BF16, s);
+  return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
 // ---- test hooks (include/kda_testing.h) ----

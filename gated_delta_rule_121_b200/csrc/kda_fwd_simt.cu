@@ -22,21 +22,35 @@ namespace {
 
 constexpr int TOK = 16;  // tokens staged per shared-memory round
 
-template <int DK, int DVB, typename IO>
+// MODE (FwdMode): MODE_CKPT also writes the state every ma.ckpt_interval
+// tokens of each sequence; MODE_SEG runs every (sequence, head, column block)
+// twice, the second time (blocks from `units` on) as the transition run:
+// values taken as zero, identity start, outputs and final state to qhat32
+// and trans (dk == dv).
+template <int DK, int DVB, typename IO, int MODE>
 __global__ void __launch_bounds__(DVB * 4)
     kda_fwd_simt_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO* __restrict__ v,
                         const float* __restrict__ g, const float* __restrict__ beta,
                         const float* __restrict__ init, IO* __restrict__ out, float* __restrict__ fin,
-                        const int32_t* __restrict__ cu, int64_t Tper, int H, int dv) {
+                        const int32_t* __restrict__ cu, int64_t Tper, int H, int dv, const ModeArgs ma,
+                        int units, DeviceStatus* status) {
   constexpr int R = DK / 4;  // rows per lane
   constexpr int NT = DVB * 4;
   __shared__ float s_k[TOK][DK], s_q[TOK][DK], s_a[TOK][DK];
   __shared__ float s_v[TOK][DVB], s_b[TOK], s_o[TOK][DVB];
 
   const int nblk = dv / DVB;
-  const int blk = blockIdx.x % nblk;
-  const int h = (blockIdx.x / nblk) % H;
-  const int n = blockIdx.x / (nblk * H);
+  int bid = blockIdx.x;
+  bool trans = false;
+  if constexpr (MODE == MODE_SEG) {
+    trans = bid >= units;
+    if (trans) bid -= units;
+    init = nullptr;
+    if (trans) fin = ma.trans;
+  }
+  const int blk = bid % nblk;
+  const int h = (bid / nblk) % H;
+  const int n = bid / (nblk * H);
   int64_t t0, L;
   if (cu) {
     t0 = cu[n];
@@ -53,7 +67,13 @@ __global__ void __launch_bounds__(DVB * 4)
 
   float s[R];
 #pragma unroll
-  for (int m = 0; m < R; ++m) s[m] = init ? init[sbase + (int64_t)(4 * m + rg) * dv + j] : 0.f;
+  for (int m = 0; m < R; ++m) {
+    s[m] = init ? init[sbase + (int64_t)(4 * m + rg) * dv + j] : 0.f;
+    if constexpr (MODE == MODE_SEG) s[m] = (trans && 4 * m + rg == j) ? 1.f : 0.f;
+  }
+  int64_t ckpt0 = 0;
+  if constexpr (MODE == MODE_CKPT)
+    ckpt0 = ma.ckpt_base ? ma.ckpt_base[n] : (int64_t)n * (Tper / ma.ckpt_interval);
 
   for (int64_t c0 = 0; c0 < L; c0 += TOK) {
     const int nt = (int)((L - c0) < TOK ? (L - c0) : TOK);
@@ -71,7 +91,7 @@ __global__ void __launch_bounds__(DVB * 4)
     }
     for (int e = tid; e < TOK * DVB; e += NT) {
       const int r = e / DVB, c = e % DVB;
-      s_v[r][c] = r < nt ? to_f32(v[((t0 + c0 + r) * H + h) * dv + blk * DVB + c]) : 0.f;
+      s_v[r][c] = (r < nt && !trans) ? to_f32(v[((t0 + c0 + r) * H + h) * dv + blk * DVB + c]) : 0.f;
     }
     if (tid < TOK) s_b[tid] = tid < nt ? beta[(t0 + c0 + tid) * H + h] : 0.f;
     __syncthreads();
@@ -97,11 +117,28 @@ __global__ void __launch_bounds__(DVB * 4)
       po += __shfl_xor_sync(0xffffffffu, po, 8);
       po += __shfl_xor_sync(0xffffffffu, po, 16);
       if (rg == 0) s_o[r][jl] = po;
+      if constexpr (MODE == MODE_CKPT) {
+        const int64_t done = c0 + r + 1;  // tokens of this sequence processed so far
+        if (done % ma.ckpt_interval == 0) {
+          const int64_t slot = ckpt0 + done / ma.ckpt_interval - 1;
+          if (slot < ma.ckpt_capacity) {
+            float* dst = ma.ckpt + (slot * H + h) * DK * dv;
+#pragma unroll
+            for (int m = 0; m < R; ++m) dst[(int64_t)(4 * m + rg) * dv + j] = s[m];
+          } else if (status && rg == 0 && jl == 0) {
+            record_error(status, KDA_ERR_INVALID_ARG, 41);
+          }
+        }
+      }
     }
     __syncthreads();
     for (int e = tid; e < nt * DVB; e += NT) {
       const int r = e / DVB, c = e % DVB;
-      out[((t0 + c0 + r) * H + h) * dv + blk * DVB + c] = from_f32<IO>(s_o[r][c]);
+      const int64_t o = ((t0 + c0 + r) * H + h) * dv + blk * DVB + c;
+      if constexpr (MODE == MODE_SEG)
+        (trans ? ma.qhat32 : ma.o32)[o] = s_o[r][c];
+      else
+        out[o] = from_f32<IO>(s_o[r][c]);
     }
   }
   if (fin) {
@@ -110,37 +147,47 @@ __global__ void __launch_bounds__(DVB * 4)
   }
 }
 
-template <int DK, typename IO>
-cudaError_t launch_k(const FwdArgs& a, cudaStream_t st) {
+template <int DK, typename IO, int MODE>
+cudaError_t launch_k(const FwdArgs& a, cudaStream_t st, const ModeArgs& ma) {
   const int DVB = a.dv < 32 ? a.dv : 32;
-  const unsigned blocks = (unsigned)((int64_t)a.N * a.H * (a.dv / DVB));
+  const int units = (int)((int64_t)a.N * a.H * (a.dv / DVB));
+  const unsigned blocks = (unsigned)(MODE == MODE_SEG ? 2 * (int64_t)units : (int64_t)units);
   if (blocks == 0) return cudaSuccess;
   const int64_t Tper = a.cu ? 0 : a.T;
 #define KDA_SIMT_LAUNCH(DVB_)                                                                            \
-  kda_fwd_simt_kernel<DK, DVB_, IO><<<blocks, DVB_ * 4, 0, st>>>(                                        \
+  kda_fwd_simt_kernel<DK, DVB_, IO, MODE><<<blocks, DVB_ * 4, 0, st>>>(                                  \
       (const IO*)a.q, (const IO*)a.k, (const IO*)a.v, a.g, a.beta, a.init, (IO*)a.out, a.fin, a.cu, Tper, \
-      a.H, a.dv)
+      a.H, a.dv, ma, units, a.status)
   if (DVB == 16) KDA_SIMT_LAUNCH(16);
   else KDA_SIMT_LAUNCH(32);
 #undef KDA_SIMT_LAUNCH
   return cudaGetLastError();
 }
 
-template <typename IO>
-cudaError_t launch_io(const FwdArgs& a, cudaStream_t s) {
+template <typename IO, int MODE>
+cudaError_t launch_io(const FwdArgs& a, cudaStream_t s, const ModeArgs& ma) {
   switch (a.dk) {
-    case 16: return launch_k<16, IO>(a, s);
-    case 32: return launch_k<32, IO>(a, s);
-    case 64: return launch_k<64, IO>(a, s);
-    case 128: return launch_k<128, IO>(a, s);
+    case 16: return launch_k<16, IO, MODE>(a, s, ma);
+    case 32: return launch_k<32, IO, MODE>(a, s, ma);
+    case 64: return launch_k<64, IO, MODE>(a, s, ma);
+    case 128: return launch_k<128, IO, MODE>(a, s, ma);
   }
   return cudaErrorInvalidValue;
 }
 
+template <int MODE>
+cudaError_t launch_mode(const FwdArgs& a, bool bf16, cudaStream_t s, const ModeArgs& ma) {
+  return bf16 ? launch_io<__nv_bfloat16, MODE>(a, s, ma) : launch_io<float, MODE>(a, s, ma);
+}
+
 }  // namespace
 
-cudaError_t launch_fwd_simt(const FwdArgs& a, bool bf16, cudaStream_t s) {
-  return bf16 ? launch_io<__nv_bfloat16>(a, s) : launch_io<float>(a, s);
+cudaError_t launch_fwd_simt(const FwdArgs& a, bool bf16, cudaStream_t s, const ModeArgs& ma) {
+  switch (ma.mode) {
+    case MODE_CKPT: return launch_mode<MODE_CKPT>(a, bf16, s, ma);
+    case MODE_SEG: return launch_mode<MODE_SEG>(a, bf16, s, ma);
+    default: return launch_mode<MODE_PLAIN>(a, bf16, s, ma);
+  }
 }
 
 }  // namespace kda

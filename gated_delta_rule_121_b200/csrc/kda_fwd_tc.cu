@@ -248,6 +248,8 @@ struct Ctx {
   float* dbg;  // chain-0 debug dump or nullptr
   long long* tdbg;  // chain-0 phase timestamps or nullptr
   long long tstart;
+  bool trans;       // MODE_SEG: this block runs the transition (zero values, identity start)
+  int64_t ckpt0;    // MODE_CKPT: checkpoint slot of this sequence's first interval
 };
 
 // Phase timestamp (elected thread only) for the timing dump.
@@ -551,6 +553,7 @@ __device__ __noinline__ void dump_wu(float* dbg, const uint8_t* sm, uint32_t tme
   }
 }
 
+template <int MODE>
 __device__ __forceinline__ void front_group(const Ctx& x, const float* __restrict__ g, const float* __restrict__ beta,
                             const void* tmg, int (&consumed)[2]) {
   const int f = threadIdx.x - FRONT0;  // 0..255
@@ -713,7 +716,11 @@ __device__ __forceinline__ void front_group(const Ctx& x, const float* __restric
           const F8 fw = ex2_8(fast ? sub8(gr, tot) : gr);
           st_f16x8(qb + o, mul8(bf16x8_to_f32(qr[i]), fw));
           st_f16x8(kb + o, mul8(bf16x8_to_f32(kraw[m]), fw));
-          st_f16x8(vb + o, bf16x8_to_f32(vr[i]));
+          if constexpr (MODE == MODE_SEG) {  // a transition run takes every value as zero
+            st_f16x8(vb + o, x.trans ? f8(0.f) : bf16x8_to_f32(vr[i]));
+          } else {
+            st_f16x8(vb + o, bf16x8_to_f32(vr[i]));
+          }
         }
       }
     }
@@ -993,10 +1000,28 @@ __device__ __noinline__ void dump_o(float* dbg, const uint8_t* sm) {
   }
 }
 
+// One checkpoint: columns col0 .. col0+63 of S^T held by this lane (value
+// channel j), written as rows col0 .. col0+63 of the state [dk][dv] in slot
+// `slot`.  A slot beyond the caller's capacity is skipped and reported.
+__device__ __forceinline__ void store_ckpt(const Ctx& x, const ModeArgs& ma, int64_t slot, int col0,
+                                           const float (&s0)[32], const float (&s1)[32]) {
+  if (slot >= ma.ckpt_capacity) {
+    record_error(x.status, KDA_ERR_INVALID_ARG, 40);
+    return;
+  }
+  float* dst = ma.ckpt + ((slot * x.H + x.h) * D + col0) * D + (threadIdx.x & 127);
+#pragma unroll 8
+  for (int i = 0; i < 32; ++i) __stcs(dst + i * D, s0[i]);
+#pragma unroll 8
+  for (int i = 0; i < 32; ++i) __stcs(dst + (32 + i) * D, s1[i]);
+}
+
 // ============================================================ scan group
+template <int MODE>
 __device__ __forceinline__ void scan_group(const Ctx& x, const void* tmq, const void* tmk, const void* tmv, const void* tmo,
                            const float* __restrict__ init, __nv_bfloat16* __restrict__ out,
-                           float* __restrict__ fin, int64_t sbase, bool inject_stuck, int (&issued)[2]) {
+                           float* __restrict__ fin, int64_t sbase, bool inject_stuck, int (&issued)[2],
+                           const ModeArgs& ma) {
   const int j = threadIdx.x;  // 0..127: TMEM lane = value channel
   const uint32_t tl = x.tmem + ((uint32_t)((j >> 5) * 32) << 16);
   uint8_t* sm = x.sm;
@@ -1031,7 +1056,12 @@ __device__ __forceinline__ void scan_group(const Ctx& x, const void* tmq, const 
   for (int cb = 0; cb < 4; ++cb) {
     float r[32];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) r[i] = init ? __ldg(init + sbase + (int64_t)(cb * 32 + i) * D + j) : 0.f;
+    for (int i = 0; i < 32; ++i) {
+      if constexpr (MODE == MODE_SEG)  // zero start, or the identity for a transition run
+        r[i] = (x.trans && cb * 32 + i == j) ? 1.f : 0.f;
+      else
+        r[i] = init ? __ldg(init + sbase + (int64_t)(cb * 32 + i) * D + j) : 0.f;
+    }
     tmem_st32(tl + TM_S + cb * 32, r);
   }
   tmem_wait_st();
@@ -1044,6 +1074,19 @@ __device__ __forceinline__ void scan_group(const Ctx& x, const void* tmq, const 
     const int64_t tok0 = x.t0 + (int64_t)c * CH;
     float o0[32], o1[32];
     tmem_ld32x2(tl + TM_O + (c & 1) * 64, tl + TM_O + (c & 1) * 64 + 32, o0, o1);
+    if constexpr (MODE == MODE_SEG) {
+      // fp32 outputs straight from the registers: lane j writes channel j of
+      // every valid token (a warp stores 128 contiguous bytes per token).
+      float* dst = (x.trans ? ma.qhat32 : ma.o32) + (tok0 * H + x.h) * D + j;
+      const int64_t st = (int64_t)H * D;
+#pragma unroll
+      for (int t = 0; t < 32; ++t)
+        if (t < valid) __stcs(dst + t * st, o0[t]);
+#pragma unroll
+      for (int t = 0; t < 32; ++t)
+        if (32 + t < valid) __stcs(dst + (32 + t) * st, o1[t]);
+      return;
+    }
     // Lanes j and j^1 hold channels jc, jc+1 of every token; they swap one
     // value per token pair so that each writes both channels of one token
     // (the even lane the even token) as one 4-byte word.
@@ -1110,6 +1153,11 @@ __device__ __forceinline__ void scan_group(const Ctx& x, const void* tmq, const 
       float s0[32], s1[32];
       uint32_t pk[16];
       tmem_ld32x2(tl + TM_S + cp * 64, tl + TM_S + cp * 64 + 32, s0, s1);
+      if constexpr (MODE == MODE_CKPT) {
+        // The state after chunk c-1 (before this chunk's decay) is the
+        // checkpoint of the interval that ends there.
+        if (c % ma.ckpt_every == 0) store_ckpt(x, ma, x.ckpt0 + c / ma.ckpt_every - 1, cp * 64, s0, s1);
+      }
       if (fast) {
 #pragma unroll
         for (int i = 0; i < 32; i += 4) {
@@ -1266,12 +1314,26 @@ __device__ __forceinline__ void scan_group(const Ctx& x, const void* tmq, const 
         for (int i = 0; i < 32; ++i) fin[sbase + (int64_t)(cb * 32 + i) * D + j] = s[i];
       }
     }
+    if constexpr (MODE == MODE_CKPT) {
+      const int64_t every_tok = (int64_t)ma.ckpt_every * CH;
+      if (x.L > 0 && x.L % every_tok == 0) {
+#pragma unroll 1
+        for (int cp = 0; cp < 2; ++cp) {
+          float s0[32], s1[32];
+          tmem_ld32x2(tl + TM_S + cp * 64, tl + TM_S + cp * 64 + 32, s0, s1);
+          store_ckpt(x, ma, x.ckpt0 + x.L / every_tok - 1, cp * 64, s0, s1);
+        }
+      }
+    }
   }
 }
 
 // HOOKS: the test-hook build (intermediate dumps, phase timestamps, the
 // stuck-wait injection); without it those branches fold away at compile time.
-template <bool HOOKS>
+// MODE (FwdMode): MODE_PLAIN is the production forward; MODE_CKPT adds the
+// interval checkpoints; MODE_SEG runs two blocks per (sequence, head): the
+// first N*H blocks the zero-start runs, the next N*H the transition runs.
+template <bool HOOKS, int MODE>
 __global__ void __launch_bounds__(NTHR, 1)
     kda_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -1280,7 +1342,8 @@ __global__ void __launch_bounds__(NTHR, 1)
                       const float* __restrict__ beta, const float* __restrict__ init,
                       __nv_bfloat16* __restrict__ out, float* __restrict__ fin, const int32_t* __restrict__ cu,
                       const int32_t* __restrict__ order, int64_t Tper, int H, DeviceStatus* status,
-                      float* __restrict__ dbg, uint64_t wait_ns, int inject_stuck) {
+                      float* __restrict__ dbg, uint64_t wait_ns, int inject_stuck,
+                      const __grid_constant__ ModeArgs ma, int units) {
   extern __shared__ uint8_t smem_raw[];
   // Align to 1024 bytes by offsetting from the shared array itself, so the
   // compiler keeps treating every access through `sm` as a shared-memory one.
@@ -1295,9 +1358,16 @@ __global__ void __launch_bounds__(NTHR, 1)
   const int tid = threadIdx.x, warp = tid >> 5;
   // Work item: with packed batches the blocks follow `order`, so that the
   // longest sequences start first.
-  const int n0 = blockIdx.x / H;
+  int bid = blockIdx.x;
+  x.trans = false;
+  if constexpr (MODE == MODE_SEG) {
+    x.trans = bid >= units;
+    if (x.trans) bid -= units;
+    if (x.trans) fin = ma.trans;
+  }
+  const int n0 = bid / H;
   const int n = order ? order[n0] : n0;
-  x.h = blockIdx.x % H;
+  x.h = bid % H;
   x.H = H;
   if (cu) {
     x.t0 = cu[n];
@@ -1307,6 +1377,9 @@ __global__ void __launch_bounds__(NTHR, 1)
     x.L = Tper;
   }
   x.nchunks = (int)((x.L + CH - 1) / CH);
+  x.ckpt0 = 0;
+  if constexpr (MODE == MODE_CKPT)
+    x.ckpt0 = ma.ckpt_base ? ma.ckpt_base[n] : (int64_t)n * (Tper / ((int64_t)ma.ckpt_every * CH));
   x.dbg = (HOOKS && dbg && n == 0 && x.h == 0) ? dbg : nullptr;
   x.tdbg = x.dbg ? reinterpret_cast<long long*>(x.dbg + DBG_TIME) : nullptr;
   long long* s_t0 = reinterpret_cast<long long*>(sm + SM_MISC + MS_T0);
@@ -1337,10 +1410,10 @@ __global__ void __launch_bounds__(NTHR, 1)
   int cnt[2] = {0, 0};  // TMA stages issued (scan group) / consumed (front group)
   int* s_cnt = reinterpret_cast<int*>(sm + SM_MISC + MS_CNT);
   if (warp < 4) {
-    scan_group(x, &tm_q, &tm_k, &tm_v, &tm_o, init, out, fin, sbase, HOOKS && inject_stuck != 0, cnt);
+    scan_group<MODE>(x, &tm_q, &tm_k, &tm_v, &tm_o, init, out, fin, sbase, HOOKS && inject_stuck != 0, cnt, ma);
     if (tid == 0) { s_cnt[0] = cnt[0]; s_cnt[1] = cnt[1]; }
   } else if (warp < 12) {
-    front_group(x, g, beta, &tm_g, cnt);
+    front_group<MODE>(x, g, beta, &tm_g, cnt);
     if (tid == (int)FRONT0) { s_cnt[2] = cnt[0]; s_cnt[3] = cnt[1]; }
   } else {
     back_group(x);
@@ -1392,6 +1465,33 @@ __global__ void kda_order_kernel(const int32_t* __restrict__ cu, int N, int32_t*
   for (int n = tid; n < N; n += blockDim.x) order[atomicAdd(&base[bucket(n)], 1)] = n;
 }
 
+// Packed batches with checkpoints: slot of the first checkpoint of every
+// sequence = the number of whole intervals in the sequences before it
+// (one block; a running prefix over blocks of 1024 sequences).
+__global__ void kda_ckpt_base_kernel(const int32_t* __restrict__ cu, int N, int interval, int32_t* __restrict__ base) {
+  __shared__ int part[1024];
+  __shared__ int carry;
+  const int tid = threadIdx.x;
+  if (tid == 0) carry = 0;
+  __syncthreads();
+  for (int n0 = 0; n0 < N; n0 += 1024) {
+    const int n = n0 + tid;
+    const int cnt = n < N ? (cu[n + 1] - cu[n]) / interval : 0;
+    part[tid] = cnt;
+    __syncthreads();
+    for (int o = 1; o < 1024; o <<= 1) {  // inclusive scan
+      const int v = tid >= o ? part[tid - o] : 0;
+      __syncthreads();
+      part[tid] += v;
+      __syncthreads();
+    }
+    if (n < N) base[n] = carry + part[tid] - cnt;
+    __syncthreads();
+    if (tid == 1023) carry += part[1023];
+    __syncthreads();
+  }
+}
+
 // ------------------------------------------------------------------ host
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -1440,26 +1540,36 @@ bool make_map_g(CUtensorMap* m, const float* ptr, int H, int64_t Ttot) {
 
 bool fwd_tc_supported(int dk, int dv, bool bf16) { return bf16 && dk == D && dv == D; }
 
+cudaError_t launch_ckpt_base(const int32_t* cu, int N, int interval, int32_t* base, cudaStream_t s) {
+  kda_ckpt_base_kernel<<<1, 1024, 0, s>>>(cu, N, interval, base);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_fwd_tc_impl(const FwdArgs& a, cudaStream_t s, uint64_t wait_ns, int inject_stuck,
-                               int32_t* order_ws) {
+                               int32_t* order_ws, const ModeArgs& ma) {
   const int64_t Ttot = a.cu ? a.T : (int64_t)a.N * a.T;
-  const unsigned blocks = (unsigned)((int64_t)a.N * a.H);
+  const int units = (int)((int64_t)a.N * a.H);
+  const unsigned blocks = (unsigned)(ma.mode == MODE_SEG ? 2 * (int64_t)units : (int64_t)units);
   if (blocks == 0) return cudaSuccess;
   CUtensorMap mq, mk, mv, mo, mg;
   const int64_t Tmap = Ttot > 0 ? Ttot : 1;
   if (!make_map(&mq, a.q, a.H, Tmap) || !make_map(&mk, a.k, a.H, Tmap) || !make_map(&mv, a.v, a.H, Tmap) ||
-      !make_map(&mo, a.out, a.H, Tmap) || !make_map_g(&mg, a.g, a.H, Tmap))
+      !make_map(&mo, a.out ? a.out : a.q, a.H, Tmap) || !make_map_g(&mg, a.g, a.H, Tmap))
     return cudaErrorInvalidValue;
   const int32_t* order = nullptr;
   if (a.cu && order_ws && a.N > 1) {
     kda_order_kernel<<<1, 1024, 0, s>>>(a.cu, a.N, order_ws);
     order = order_ws;
   }
-  auto* kern = (a.dbg || inject_stuck) ? kda_fwd_tc_kernel<true> : kda_fwd_tc_kernel<false>;
+  auto* kern = (a.dbg || inject_stuck) ? kda_fwd_tc_kernel<true, MODE_PLAIN>
+               : ma.mode == MODE_CKPT  ? kda_fwd_tc_kernel<false, MODE_CKPT>
+               : ma.mode == MODE_SEG   ? kda_fwd_tc_kernel<false, MODE_SEG>
+                                       : kda_fwd_tc_kernel<false, MODE_PLAIN>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
   if (e != cudaSuccess) return e;
   kern<<<blocks, NTHR, SMEM_BYTES, s>>>(mq, mk, mv, mo, mg, a.g, a.beta, a.init, (__nv_bfloat16*)a.out, a.fin, a.cu,
-                                        order, a.cu ? 0 : a.T, a.H, a.status, (float*)a.dbg, wait_ns, inject_stuck);
+                                        order, a.cu ? 0 : a.T, a.H, a.status, (float*)a.dbg, wait_ns, inject_stuck,
+                                        ma, units);
   return cudaGetLastError();
 }
 

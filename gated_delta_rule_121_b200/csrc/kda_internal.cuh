@@ -49,10 +49,35 @@ struct FwdArgs {
   void* dbg;          // optional debug dump (test hook), may be nullptr
 };
 
+// What a forward launch produces besides out / final state.
+enum FwdMode {
+  MODE_PLAIN = 0,  // out and final state
+  MODE_CKPT = 1,   // plus the state every `ckpt_every` chunks of each sequence
+  MODE_SEG = 2,    // segment pieces: two runs per (sequence, head), both with
+                   // fp32 outputs and no init state: the zero-start run
+                   // (outputs o32, final state fin) and the transition run
+                   // (values taken as zero, identity start: outputs qhat32,
+                   // final state = the transition, written to trans)
+};
+
+struct ModeArgs {
+  int mode = MODE_PLAIN;
+  // MODE_CKPT
+  float* ckpt = nullptr;              // [capacity][H][dk][dv]
+  const int32_t* ckpt_base = nullptr; // first checkpoint slot of each sequence (packed batches)
+  int ckpt_every = 0;                 // interval in 64-token chunks (tensor-core path) ...
+  int ckpt_interval = 0;              // ... and in tokens
+  int64_t ckpt_capacity = 0;
+  // MODE_SEG
+  float* o32 = nullptr;     // [T_total][H][dv]
+  float* qhat32 = nullptr;  // [T_total][H][dk]
+  float* trans = nullptr;   // [N][H][dk][dk]
+};
+
 // Launchers (return a CUDA error code; launches are asynchronous).
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const float* g, const float* beta,
                           float* state, void* out, int B, int H, int dk, int dv, bool bf16, cudaStream_t s);
-cudaError_t launch_fwd_simt(const FwdArgs& a, bool bf16, cudaStream_t s);
+cudaError_t launch_fwd_simt(const FwdArgs& a, bool bf16, cudaStream_t s, const ModeArgs& m = ModeArgs());
 bool fwd_tc_supported(int dk, int dv, bool bf16);
 cudaError_t launch_fwd_tc(const FwdArgs& a, cudaStream_t s);
 

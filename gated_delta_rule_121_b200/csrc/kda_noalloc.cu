@@ -9,6 +9,7 @@
 // device.  This entry point takes the same inputs and outputs as kda_fwd and
 // uses, instead of a caller-provided workspace, a fixed array in device
 // memory that belongs to the library.  It allocates nothing.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -25,21 +26,58 @@ __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 256;
 std::mutex g_mu;
-void* g_scratch_addr[kMaxDevices];
+struct CachedAddr {
+  unsigned long long ctx_id;  // driver context the address belongs to (0: none yet)
+  void* addr;
+};
+CachedAddr g_cache[kMaxDevices];
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// Unique id of the thread's current driver context, or 0 when there is none
+// (for example right after cudaDeviceReset, before the runtime makes a new
+// one).  Ids are never reused within a process, so a cached address is
+// trusted only while the context that produced it is still the current one.
+unsigned long long current_ctx_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static bool looked_up = false;
+  if (!looked_up) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+    looked_up = true;
+  }
+  if (!get_current || !get_id) return 0;
+  CUcontext c = nullptr;
+  unsigned long long id = 0;
+  if (get_current(&c) != CUDA_SUCCESS || !c || get_id(c, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
 
 // Device address of the array for the current device.  In host code the
-// array's name is only a host-side stand-in, so the address is looked up
-// once per device (with that device current) and cached.
+// array's name is only a host-side stand-in, so the address is looked up with
+// that device current and cached per device; the cache is refreshed when the
+// device's context has changed since (cudaDeviceReset destroys the old one).
 void* scratch_for_current_device() {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
   std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_scratch_addr[dev]) {
+  const unsigned long long id = current_ctx_id();
+  if (id == 0 || g_cache[dev].ctx_id != id || !g_cache[dev].addr) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
-    g_scratch_addr[dev] = p;
+    g_cache[dev].addr = p;
+    g_cache[dev].ctx_id = current_ctx_id();  // the lookup makes a context current if there was none
   }
-  return g_scratch_addr[dev];
+  return g_cache[dev].addr;
 }
 
 }  // namespace
@@ -56,4 +94,10 @@ extern "C" kda_status_t kda_fwd_noalloc(const void* q, const void* k, const void
   // the order array, so nothing left by the previous call is read.
   return kda_fwd(q, k, v, log_alpha, beta, init_state, out, final_state, B, T, H, dk, dv, cu_seqlens, stream, dt,
                  scratch, kScratchBytes);
+}
+
+extern "C" kda_status_t kda_fwd_noalloc_status(void* stream) {
+  void* scratch = scratch_for_current_device();
+  if (!scratch) return KDA_ERR_CUDA;
+  return kda_workspace_status(scratch, stream);
 }

@@ -1,0 +1,271 @@
+// Segment decomposition of the KDA state scan: the kernels that compose
+// segment pieces and correct zero-start outputs (Kimi K3 digest, "KDA
+// algorithm-system co-design", paragraphs on intra-device context
+// parallelism and on KDA context parallelism, KCP).
+//
+// With the transition form of the recurrence, S_t = M_t S_{t-1} + beta_t
+// k_t v_t^T, M_t = (I - beta_t k_t k_t^T) Diag(alpha_t), the state after a
+// segment that starts from S_in is
+//     S_end = S~ + M S_in,
+// where S~ is the segment's state from a zero start and M = M_last ... M_first
+// its transition; both depend only on the segment's own tokens.  Inside the
+// segment the output of token t is, by the same linearity,
+//     o_t = o~_t + S_in^T qhat_t,   qhat_t = M_{t<-first}^T q_t,
+// with o~ the zero-start output.  The forward kernels produce (o~, S~) and
+// (qhat, M) per segment (MODE_SEG); this file holds
+//   - the composition S_in[r+1] = S~_r + M_r S_in[r] over the segments of a
+//     sequence (a sequential prefix, fp32 on CUDA cores, one block per
+//     (sequence, head, 32 value columns): the columns of S evolve
+//     independently), and
+//   - the correction o_t = o~_t + S_in^T qhat_t (dense 64-token x dv tiles on
+//     the warp-level tensor path with tf32 operands rounded to nearest; the
+//     zero-start output o~ stays fp32, so the result is rounded once).
+#include <cstdint>
+
+#include "../../include/kda.h"
+#include "kda_internal.cuh"
+#include "sm100_ptx.cuh"
+
+namespace kda {
+namespace {
+
+// ------------------------------------------------------------ composition
+// Pieces of sequence m: p = m * R + r (piece-major) or r * N + m (rank-major,
+// the order of an all-gather over ranks).  state_in[p] = the state entering
+// piece p; final_state[m] = the state after the last piece.
+template <int DK>
+__global__ void __launch_bounds__(256)
+    compose_kernel(const float* __restrict__ trans, const float* __restrict__ s0, const float* __restrict__ init,
+                   float* __restrict__ state_in, float* __restrict__ fin, int R, int N, int H, int dv,
+                   int rank_major) {
+  constexpr int RPT = DK / 8;  // rows per thread: warp w holds rows w, w + 8, ...
+  __shared__ float s_cur[DK][33];
+  const int ncb = (dv + 31) / 32;
+  const int cb = blockIdx.x % ncb;
+  const int h = (blockIdx.x / ncb) % H;
+  const int m = blockIdx.x / (ncb * H);
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int c = cb * 32 + lane;
+  const bool col = c < dv;
+  const int64_t sd = (int64_t)DK * dv, mm = (int64_t)DK * DK;
+
+  float cur[RPT];
+#pragma unroll
+  for (int u = 0; u < RPT; ++u) {
+    const int i = w + 8 * u;
+    cur[u] = (init && col) ? init[((int64_t)m * H + h) * sd + (int64_t)i * dv + c] : 0.f;
+  }
+  for (int r = 0; r < R; ++r) {
+    const int64_t p = rank_major ? (int64_t)r * N + m : (int64_t)m * R + r;
+    const int64_t ph = p * H + h;
+#pragma unroll
+    for (int u = 0; u < RPT; ++u) {
+      const int i = w + 8 * u;
+      if (col && state_in) state_in[ph * sd + (int64_t)i * dv + c] = cur[u];
+      s_cur[i][lane] = cur[u];
+    }
+    __syncthreads();
+    // next = S~_p + M_p cur: row i of M_p is read by every lane of the warp
+    // (one broadcast load per element), cur from shared memory.
+    const float* Mp = trans + ph * mm;
+    float acc[RPT];
+#pragma unroll
+    for (int u = 0; u < RPT; ++u) acc[u] = col ? s0[ph * sd + (int64_t)(w + 8 * u) * dv + c] : 0.f;
+#pragma unroll 4
+    for (int kk = 0; kk < DK; ++kk) {
+      const float sv = s_cur[kk][lane];
+#pragma unroll
+      for (int u = 0; u < RPT; ++u) acc[u] = fmaf(__ldg(Mp + (int64_t)(w + 8 * u) * DK + kk), sv, acc[u]);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int u = 0; u < RPT; ++u) cur[u] = acc[u];
+  }
+  if (fin && col) {
+#pragma unroll
+    for (int u = 0; u < RPT; ++u)
+      fin[((int64_t)m * H + h) * sd + (int64_t)(w + 8 * u) * dv + c] = cur[u];
+  }
+}
+
+// ------------------------------------------------------------ correction
+constexpr int CT = 64;        // tokens per tile
+constexpr int CPAD = 4;       // row padding (floats) of the shared tiles: conflict-free fragments
+
+__device__ __forceinline__ uint32_t tf32_rna(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
+
+// Piece that holds packed token t: the last p with cu[p] <= t.
+__device__ __forceinline__ int piece_of(const int32_t* cu, int P, int64_t t) {
+  int lo = 0, hi = P - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (cu[mid] <= t) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
+
+// One block: 64 consecutive tokens x all DV channels of one head.  Each of
+// the 4 warps owns 16 tokens; K = DK in steps of 8.  A tile that straddles
+// pieces is computed once per piece, each pass writing only its own rows.
+template <int DK, int DV, typename IO>
+__global__ void __launch_bounds__(128)
+    correct_kernel(const float* __restrict__ o32, const float* __restrict__ qhat, const float* __restrict__ s_in,
+                   IO* __restrict__ out, const int32_t* __restrict__ cu, int P, int64_t Tper, int64_t Ttot, int H) {
+  extern __shared__ float csm[];
+  float* s_q = csm;                        // [CT][DK + CPAD]
+  float* s_s = csm + CT * (DK + CPAD);     // [DK][DV + CPAD]
+  const int h = blockIdx.y;
+  const int64_t t0 = (int64_t)blockIdx.x * CT;
+  const int nt = (int)((Ttot - t0) < CT ? (Ttot - t0) : CT);
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, g = lane >> 2, tq = lane & 3;
+
+  // qhat rows of the tile (rows past the end are zero)
+  for (int e = tid; e < CT * (DK / 4); e += 128) {
+    const int r = e / (DK / 4), c4 = (e % (DK / 4)) * 4;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (r < nt) v = __ldcs(reinterpret_cast<const float4*>(qhat + ((t0 + r) * H + h) * DK + c4));
+    *reinterpret_cast<float4*>(s_q + r * (DK + CPAD) + c4) = v;
+  }
+  const int p_first = cu ? piece_of(cu, P, t0) : (int)(t0 / Tper);
+  const int p_last = cu ? piece_of(cu, P, t0 + nt - 1) : (int)((t0 + nt - 1) / Tper);
+  for (int p = p_first; p <= p_last; ++p) {
+    const int64_t lo = cu ? cu[p] : (int64_t)p * Tper, hi = cu ? cu[p + 1] : (int64_t)(p + 1) * Tper;
+    if (hi <= lo) continue;  // empty piece
+    __syncthreads();         // the previous pass is done with s_s
+    const float* S = s_in + ((int64_t)p * H + h) * DK * DV;
+    for (int e = tid; e < DK * (DV / 4); e += 128) {
+      const int r = e / (DV / 4), c4 = (e % (DV / 4)) * 4;
+      *reinterpret_cast<float4*>(s_s + r * (DV + CPAD) + c4) = __ldg(reinterpret_cast<const float4*>(S + r * DV + c4));
+    }
+    __syncthreads();
+    if (w * 16 >= nt) continue;
+    float d[DV / 8][4];
+#pragma unroll
+    for (int n = 0; n < DV / 8; ++n) d[n][0] = d[n][1] = d[n][2] = d[n][3] = 0.f;
+    const float* qa = s_q + (w * 16) * (DK + CPAD);
+#pragma unroll 2
+    for (int k0 = 0; k0 < DK; k0 += 8) {
+      uint32_t a[4];
+      a[0] = tf32_rna(qa[g * (DK + CPAD) + k0 + tq]);
+      a[1] = tf32_rna(qa[(g + 8) * (DK + CPAD) + k0 + tq]);
+      a[2] = tf32_rna(qa[g * (DK + CPAD) + k0 + tq + 4]);
+      a[3] = tf32_rna(qa[(g + 8) * (DK + CPAD) + k0 + tq + 4]);
+#pragma unroll
+      for (int n = 0; n < DV / 8; ++n) {
+        uint32_t b[2];
+        b[0] = tf32_rna(s_s[(k0 + tq) * (DV + CPAD) + n * 8 + g]);
+        b[1] = tf32_rna(s_s[(k0 + tq + 4) * (DV + CPAD) + n * 8 + g]);
+        mma_tf32_16x8x8(d[n], a, b);
+      }
+    }
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const int r = w * 16 + g + 8 * half;
+      const int64_t t = t0 + r;
+      if (r >= nt || t < lo || t >= hi) continue;
+      const int64_t base = (t * H + h) * DV;
+#pragma unroll
+      for (int n = 0; n < DV / 8; ++n) {
+        const int c = n * 8 + 2 * tq;
+        const float2 z = __ldcs(reinterpret_cast<const float2*>(o32 + base + c));
+        out[base + c] = from_f32<IO>(z.x + d[n][2 * half]);
+        out[base + c + 1] = from_f32<IO>(z.y + d[n][2 * half + 1]);
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------ segment layout
+// Segment offsets for the intra-device split: sequence m of length L is cut
+// into R segments at tokens c0 + floor(L r / R).  seg_cu[m R + r] is the start
+// of segment r; seg_cu[N R] = the total token count.
+__global__ void segment_cu_kernel(const int32_t* __restrict__ cu, int64_t Tper, int N, int R,
+                                  int32_t* __restrict__ seg_cu) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i > (int64_t)N * R) return;
+  if (i == (int64_t)N * R) {
+    seg_cu[i] = cu ? cu[N] : (int32_t)(Tper * N);
+    return;
+  }
+  const int m = (int)(i / R), r = (int)(i % R);
+  const int64_t c0 = cu ? cu[m] : Tper * m;
+  const int64_t L = cu ? (int64_t)cu[m + 1] - c0 : Tper;
+  seg_cu[i] = (int32_t)(c0 + (L * r) / R);
+}
+
+template <int DK>
+cudaError_t compose_dk(const float* trans, const float* s0, const float* init, float* state_in, float* fin, int R,
+                       int N, int H, int dv, int rank_major, cudaStream_t s) {
+  const int ncb = (dv + 31) / 32;
+  const int64_t blocks = (int64_t)N * H * ncb;
+  if (blocks == 0) return cudaSuccess;
+  compose_kernel<DK><<<(unsigned)blocks, 256, 0, s>>>(trans, s0, init, state_in, fin, R, N, H, dv, rank_major);
+  return cudaGetLastError();
+}
+
+template <int DK, int DV, typename IO>
+cudaError_t correct_t(const float* o32, const float* qhat, const float* s_in, void* out, const int32_t* cu, int P,
+                      int64_t Tper, int64_t Ttot, int H, cudaStream_t s) {
+  if (Ttot == 0) return cudaSuccess;
+  const size_t smem = sizeof(float) * ((size_t)CT * (DK + CPAD) + (size_t)DK * (DV + CPAD));
+  auto* kern = correct_kernel<DK, DV, IO>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((unsigned)((Ttot + CT - 1) / CT), (unsigned)H);
+  kern<<<grid, 128, smem, s>>>(o32, qhat, s_in, (IO*)out, cu, P, Tper, Ttot, H);
+  return cudaGetLastError();
+}
+
+template <int DK, typename IO>
+cudaError_t correct_dv(const float* o32, const float* qhat, const float* s_in, void* out, const int32_t* cu, int P,
+                       int64_t Tper, int64_t Ttot, int H, int dv, cudaStream_t s) {
+  switch (dv) {
+    case 16: return correct_t<DK, 16, IO>(o32, qhat, s_in, out, cu, P, Tper, Ttot, H, s);
+    case 32: return correct_t<DK, 32, IO>(o32, qhat, s_in, out, cu, P, Tper, Ttot, H, s);
+    case 64: return correct_t<DK, 64, IO>(o32, qhat, s_in, out, cu, P, Tper, Ttot, H, s);
+    case 128: return correct_t<DK, 128, IO>(o32, qhat, s_in, out, cu, P, Tper, Ttot, H, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+cudaError_t launch_compose(const float* trans, const float* s0, const float* init, float* state_in, float* fin,
+                           int R, int N, int H, int dk, int dv, int rank_major, cudaStream_t s) {
+  switch (dk) {
+    case 16: return compose_dk<16>(trans, s0, init, state_in, fin, R, N, H, dv, rank_major, s);
+    case 32: return compose_dk<32>(trans, s0, init, state_in, fin, R, N, H, dv, rank_major, s);
+    case 64: return compose_dk<64>(trans, s0, init, state_in, fin, R, N, H, dv, rank_major, s);
+    case 128: return compose_dk<128>(trans, s0, init, state_in, fin, R, N, H, dv, rank_major, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_correct(const float* o32, const float* qhat, const float* s_in, void* out, const int32_t* cu,
+                           int P, int64_t Tper, int64_t Ttot, int H, int dk, int dv, bool bf16, cudaStream_t s) {
+  switch (dk) {
+#define KDA_CORRECT_DK(DK_)                                                                                  \
+  case DK_:                                                                                                  \
+    return bf16 ? correct_dv<DK_, __nv_bfloat16>(o32, qhat, s_in, out, cu, P, Tper, Ttot, H, dv, s)          \
+                : correct_dv<DK_, float>(o32, qhat, s_in, out, cu, P, Tper, Ttot, H, dv, s);
+    KDA_CORRECT_DK(16)
+    KDA_CORRECT_DK(32)
+    KDA_CORRECT_DK(64)
+    KDA_CORRECT_DK(128)
+#undef KDA_CORRECT_DK
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_segment_cu(const int32_t* cu, int64_t Tper, int N, int R, int32_t* seg_cu, cudaStream_t s) {
+  const int64_t n = (int64_t)N * R + 1;
+  segment_cu_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(cu, Tper, N, R, seg_cu);
+  return cudaGetLastError();
+}
+
+}  // namespace kda

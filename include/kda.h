@@ -142,9 +142,12 @@ KDA_API kda_status_t kda_fwd(const void *q, const void *k, const void *v,
  *   - Every call on a device shares the one array.  Calls that may overlap on
  *     the GPU (different streams, or other host threads) race on it; issue
  *     them in order on one stream.
- *   - The device status word lives in that array, so device-side errors
- *     (KDA_ERR_TIMEOUT, KDA_ERR_RANGE) of this entry point cannot be read
- *     back; use kda_fwd with a workspace when they must be checked.
+ *   - The device status word lives in that array: read device-side errors
+ *     (KDA_ERR_TIMEOUT, KDA_ERR_RANGE) of the last call on the current
+ *     device with kda_fwd_noalloc_status().
+ *   - The array's address is cached per device together with the id of the
+ *     device's context; after cudaDeviceReset the next call looks it up
+ *     again.
  */
 #define KDA_NOALLOC_MAX_SEQUENCES 8192
 KDA_API kda_status_t kda_fwd_noalloc(const void *q, const void *k, const void *v,
@@ -152,6 +155,43 @@ KDA_API kda_status_t kda_fwd_noalloc(const void *q, const void *k, const void *v
                                      const float *init_state, void *out, float *final_state,
                                      int B, int64_t T, int H, int dk, int dv,
                                      const int32_t *cu_seqlens, void *stream, kda_dtype_t dt);
+
+/*
+ * Device status of the last kda_fwd_noalloc call on the current device, read
+ * from the library's fixed array: synchronises `stream` (pass the stream the
+ * call ran on) and returns KDA_OK, KDA_ERR_TIMEOUT or KDA_ERR_RANGE as
+ * kda_workspace_status does for a caller workspace.  Allocates nothing.
+ */
+KDA_API kda_status_t kda_fwd_noalloc_status(void *stream);
+
+/*
+ * The tensors of one kda_fwd call, as a set of pointers (all on the host, or
+ * all on the device).  init_state, cu_seqlens and final_state may be NULL with
+ * the meaning they have in kda_fwd.
+ */
+typedef struct kda_fwd_tensors {
+    const void *q, *k, *v;
+    const float *log_alpha, *beta, *init_state;
+    const int32_t *cu_seqlens;
+    void *out;
+    float *final_state;
+} kda_fwd_tensors_t;
+
+/*
+ * kda_fwd on host buffers: enqueues on `stream` the host-to-device copies of
+ * every input in `host` (q, k, v, log_alpha, beta, and init_state /
+ * cu_seqlens when set) into the caller's device buffers `dev`, the forward
+ * on `dev`, and the device-to-host copies of out (and final_state when both
+ * `host` and `dev` set it).  One cudaMemcpyAsync per tensor; page-locked host
+ * memory makes the copies asynchronous.  Sizes and the other arguments are
+ * those of kda_fwd; `host` and `dev` must set the same optional tensors.
+ * Returns at once; synchronise `stream` before reading the host outputs.
+ * This is the end-to-end path a serving process without its own device
+ * staging logic would call.
+ */
+KDA_API kda_status_t kda_fwd_host(const kda_fwd_tensors_t *host, const kda_fwd_tensors_t *dev,
+                                  int B, int64_t T, int H, int dk, int dv, void *stream,
+                                  kda_dtype_t dt, void *workspace, size_t workspace_bytes);
 
 /*
  * One decode step: one new token per sequence, state updated in place (the
@@ -170,6 +210,125 @@ KDA_API kda_status_t kda_decode_step(const void *q, const void *k, const void *v
                              const float *log_alpha, const float *beta,
                              float *state, void *out, int B, int H, int dk, int dv,
                              void *stream, kda_dtype_t dt);
+
+/*
+ * Interval checkpoints for prefix caching (the digest's serving section,
+ * "decoupling hash granularity from storage granularity": the KDA state is
+ * stored only at a sparse subset of the 512-token hash boundaries, so that a
+ * later request whose prefix matches up to such a boundary resumes prefill
+ * there instead of recomputing it).
+ *
+ * Same arguments and results as kda_fwd, plus
+ *   checkpoints [capacity, H, dk, dv] fp32, device: the state of every
+ *              sequence after each whole multiple of `interval` tokens from
+ *              its start (positions interval, 2 interval, ... <= its length;
+ *              a sequence whose length is a multiple of `interval` also gets
+ *              its final state as its last checkpoint).  Sequence n's
+ *              checkpoints are consecutive slots starting at
+ *              sum_{m<n} floor(L_m / interval).
+ *   interval   a positive multiple of 64 tokens (the chunk length), else
+ *              KDA_ERR_UNSUPPORTED.  The pages' hash block is 512.
+ *   capacity   number of slots in `checkpoints`.  Batched inputs need
+ *              B * floor(T / interval) slots (checked on the host); for packed
+ *              batches a slot beyond it is skipped and reported as
+ *              KDA_ERR_INVALID_ARG through kda_workspace_status().
+ *   workspace  at least kda_fwd_checkpoints_workspace_size(...) bytes.
+ * Extra HBM traffic: dk * dv * 4 bytes per head per checkpoint.
+ */
+KDA_API size_t kda_fwd_checkpoints_workspace_size(int B, int64_t T, int H, int dk, int dv, kda_dtype_t dt);
+KDA_API kda_status_t kda_fwd_checkpoints(const void *q, const void *k, const void *v,
+                                         const float *log_alpha, const float *beta,
+                                         const float *init_state, void *out, float *final_state,
+                                         int B, int64_t T, int H, int dk, int dv,
+                                         const int32_t *cu_seqlens, void *stream, kda_dtype_t dt,
+                                         float *checkpoints, int interval, int64_t capacity,
+                                         void *workspace, size_t workspace_bytes);
+
+/*
+ * Segment pieces (the digest's "KDA algorithm-system co-design" section,
+ * KCP paragraph: with M_t = (I - beta_t k_t k_t^T) Diag(alpha_t) the state
+ * after a segment is S~ + M S_in, where the transition M and the zero-start
+ * state S~ depend only on the segment's own tokens).  Every sequence of the
+ * batch is one segment; for each (sequence, head) this computes
+ *   out_zero   [B, T, H, dv] fp32: the outputs from a zero initial state
+ *   state_zero [N, H, dk, dv] fp32: the state after the segment from zero (S~)
+ *   qhat       [B, T, H, dk] fp32: qhat_t = M_{t<-first}^T q_t, the transition
+ *              from the segment start through token t applied to q_t, so that
+ *              the output from an initial state S_in is out_zero_t + S_in^T qhat_t
+ *   transition [N, H, dk, dk] fp32: M, the product of the segment's M_t
+ * Requires dk == dv (else KDA_ERR_UNSUPPORTED).  Other arguments, layouts
+ * and the workspace are those of kda_fwd (kda_fwd_workspace_size).
+ * Cost: two forward passes over the segment (the second with values taken as
+ * zero and an identity start), both with fp32 outputs.
+ */
+KDA_API kda_status_t kda_segment_fwd(const void *q, const void *k, const void *v,
+                                     const float *log_alpha, const float *beta,
+                                     float *out_zero, float *state_zero, float *qhat, float *transition,
+                                     int B, int64_t T, int H, int dk, int dv,
+                                     const int32_t *cu_seqlens, void *stream, kda_dtype_t dt,
+                                     void *workspace, size_t workspace_bytes);
+
+/*
+ * Prefix composition of segment pieces (same paragraph: the rank-level
+ * updates compose associatively, so every segment's incoming state follows
+ * from a prefix scan).  N sequences, each cut into R consecutive pieces
+ * r = 0..R-1; piece (m, r) is at index m*R + r (rank_major = 0) or r*N + m
+ * (rank_major = 1, the layout of an all-gather over R ranks).
+ *   transition [R*N, H, dk, dk], state_zero [R*N, H, dk, dv]  (from
+ *              kda_segment_fwd of every piece), fp32, device
+ *   init_state [N, H, dk, dv] or NULL (zeros): the state before piece 0
+ *   state_in   [R*N, H, dk, dv] or NULL: the state entering each piece,
+ *              S_in(m, 0) = init, S_in(m, r+1) = S~(m, r) + M(m, r) S_in(m, r)
+ *   final_state[N, H, dk, dv] or NULL: the state after the last piece
+ * fp32 arithmetic on CUDA cores.  Asynchronous on `stream`; no workspace.
+ */
+KDA_API kda_status_t kda_state_compose(const float *transition, const float *state_zero,
+                                       const float *init_state, float *state_in, float *final_state,
+                                       int R, int N, int H, int dk, int dv, int rank_major, void *stream);
+
+/*
+ * Outputs of segments whose incoming states are known:
+ *   out_t = out_zero_t + S_in^T qhat_t   (rounded once to dtype dt)
+ * with out_zero and qhat from kda_segment_fwd and S_in = state_in[n] for the
+ * sequence n that holds token t (cu_seqlens as in kda_fwd).
+ *   state_in [N, H, dk, dv] fp32; out [B, T, H, dv] in dtype dt.
+ * The product runs on the warp-level tensor path with tf32 operands
+ * (rounded to nearest) and fp32 accumulation.  No workspace.
+ */
+KDA_API kda_status_t kda_output_correct(const float *out_zero, const float *qhat, const float *state_in,
+                                        void *out, int B, int64_t T, int H, int dk, int dv,
+                                        const int32_t *cu_seqlens, void *stream, kda_dtype_t dt);
+
+/*
+ * Intra-device context parallelism (the digest's co-design section, the
+ * intra-device context-parallel paragraph: under tensor parallelism a rank
+ * holds few heads, so a long prefill leaves most SMs idle; the sequence is
+ * split over the SMs of one device, the segment transitions are evaluated in
+ * parallel and merged to recover each segment's exact initial state, with no
+ * inter-device traffic).
+ *
+ * Same arguments and results as kda_fwd, plus n_seg: every sequence is cut
+ * into n_seg segments of near-equal length (at tokens start + floor(L r /
+ * n_seg), anywhere inside a 64-token chunk).  One launch computes the pieces
+ * of all segments (kda_segment_fwd), then kda_state_compose gives every
+ * segment's incoming state and the final state, and kda_output_correct the
+ * outputs.  Requires dk == dv.  n_seg = 1 is valid (one segment).
+ *   workspace  at least kda_fwd_cp_workspace_size(B, T_total, ..., n_seg)
+ *              bytes, where T_total is the token count (B*T for batched
+ *              inputs, T when packed); it holds the fp32 pieces: about
+ *              T_total * H * (dk + dv) * 4 bytes plus 3 states per segment.
+ * Worth it when 2 * N * H * n_seg blocks fit one wave on the device and the
+ * chains are few (kda_cp_segments suggests n_seg).
+ */
+KDA_API size_t kda_fwd_cp_workspace_size(int B, int64_t T_total, int H, int dk, int dv, kda_dtype_t dt,
+                                         int n_seg);
+KDA_API int kda_cp_segments(int N, int64_t tokens_per_sequence, int H, int sm_count);
+KDA_API kda_status_t kda_fwd_cp(const void *q, const void *k, const void *v,
+                                const float *log_alpha, const float *beta,
+                                const float *init_state, void *out, float *final_state,
+                                int B, int64_t T, int H, int dk, int dv,
+                                const int32_t *cu_seqlens, void *stream, kda_dtype_t dt, int n_seg,
+                                void *workspace, size_t workspace_bytes);
 
 /*
  * Read back the device status word of a workspace used by kda_fwd.

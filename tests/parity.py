@@ -4,13 +4,18 @@ The contract: relative Frobenius error <= 1e-4 for fp32 inputs; <= 5e-3 with
 max-abs <= 3e-2 * RMS(reference) for bf16 inputs, on both the output and the
 final state.  The reference is the unrounded fp64 oracle result.
 
-Reading of the max-abs bound for bf16 OUTPUTS: the output tensor is stored
-in bf16 (round to nearest even), so every element carries up to half a bf16
-ulp of |reference| that no implementation can avoid.  On heavy-tailed
-outputs (the model-range decay case: max|o| ~ 17 RMS) that rounding alone
-reaches ~0.039 RMS, above 3e-2 RMS.  The bound is therefore applied to the
-error in excess of that half ulp: max_i(|o_i - ref_i| - ulp(ref_i)/2) <=
-3e-2 RMS.  States are fp32 outputs and get no allowance.
+The max-abs bound is applied literally (max_i |x_i - ref_i| <= 3e-2 RMS) on
+every workload whose exact result, rounded to bf16, stays inside it: the
+benchmark shapes (mid, the 64K prefill, the packed 1M-token batch, decode).
+
+Reading of the max-abs bound for bf16 OUTPUTS of strongly decaying inputs
+(g down to the model's bound -5 and beyond): the output tensor is stored in
+bf16 (round to nearest even), so every element carries up to half a bf16 ulp
+of |reference| that no implementation can avoid.  On those heavy-tailed
+outputs (max|o| ~ 17 RMS) that rounding alone reaches ~0.039 RMS, above
+3e-2 RMS.  For them (``literal=False``) the bound is applied to the error in
+excess of that half ulp: max_i(|o_i - ref_i| - ulp(ref_i)/2) <= 3e-2 RMS.
+States are fp32 outputs and never get the allowance.
 """
 import numpy as np
 import torch
@@ -45,17 +50,62 @@ def half_ulp_bf16(ref):
     return np.where(a > 0, np.ldexp(1.0, (ex - 8).astype(np.int64)), 0.0)
 
 
-def assert_close(x, ref, dtype, what=""):
+def assert_close(x, ref, dtype, what="", literal=True):
+    """Assert the contract's tolerances.  ``literal=False`` (strongly decaying
+    inputs only) subtracts the output's unavoidable half-ulp bf16 rounding
+    before the max-abs test."""
     e = errors(x, ref)
     t = TOL[dtype]
     xa, ra = to_f64(x), to_f64(ref)
     assert np.isfinite(xa).all(), f"{what}: non-finite values"
     assert e["rel_fro"] <= t["rel_fro"], f"{what}: rel_fro {e['rel_fro']:.3e} > {t['rel_fro']:.1e}"
     if t["max_abs_rms"] is not None:
-        allowance = half_ulp_bf16(ra) if (isinstance(x, torch.Tensor) and x.dtype == torch.bfloat16) else 0.0
-        excess = float((np.abs(xa - ra) - allowance).max()) if xa.size else 0.0
-        e["max_abs_excess"] = excess
-        assert excess <= t["max_abs_rms"] * e["rms"], (
-            f"{what}: max_abs {e['max_abs']:.3e} (beyond output rounding {excess:.3e}) > "
-            f"{t['max_abs_rms']} * rms {e['rms']:.3e}")
+        bound = t["max_abs_rms"] * e["rms"]
+        if literal:
+            assert e["max_abs"] <= bound, (
+                f"{what}: max_abs {e['max_abs']:.3e} > {t['max_abs_rms']} * rms {e['rms']:.3e}")
+        else:
+            rounded_out = isinstance(x, torch.Tensor) and x.dtype == torch.bfloat16
+            allowance = half_ulp_bf16(ra) if rounded_out else 0.0
+            excess = float((np.abs(xa - ra) - allowance).max()) if xa.size else 0.0
+            e["max_abs_excess"] = excess
+            assert excess <= bound, (
+                f"{what}: max_abs {e['max_abs']:.3e} (beyond output rounding {excess:.3e}) > "
+                f"{t['max_abs_rms']} * rms {e['rms']:.3e}")
+    e["max_abs_over_rms"] = e["max_abs"] / max(e["rms"], 1e-300)
     return e
+
+
+class ErrorAccumulator:
+    """The contract's measures over a tensor checked in pieces (e.g. a few
+    heads at a time, so the fp64 reference of a full-size workload never has
+    to sit in host memory at once).  ``check()`` applies the same bounds as
+    ``assert_close`` with ``literal=True``."""
+
+    def __init__(self, dtype, what=""):
+        self.dtype, self.what = dtype, what
+        self.sq_diff = self.sq_ref = 0.0
+        self.max_abs = 0.0
+        self.n = 0
+
+    def add(self, x, ref):
+        xa, ra = to_f64(x), to_f64(ref)
+        assert np.isfinite(xa).all(), f"{self.what}: non-finite values"
+        d = xa - ra
+        self.sq_diff += float((d * d).sum())
+        self.sq_ref += float((ra * ra).sum())
+        if d.size:
+            self.max_abs = max(self.max_abs, float(np.abs(d).max()))
+        self.n += ra.size
+
+    def check(self):
+        t = TOL[self.dtype]
+        rel = np.sqrt(self.sq_diff) / max(np.sqrt(self.sq_ref), 1e-300)
+        rms = np.sqrt(self.sq_ref / max(self.n, 1))
+        e = dict(rel_fro=float(rel), max_abs=self.max_abs, rms=float(rms),
+                 max_abs_over_rms=self.max_abs / max(rms, 1e-300))
+        assert rel <= t["rel_fro"], f"{self.what}: rel_fro {rel:.3e} > {t['rel_fro']:.1e}"
+        if t["max_abs_rms"] is not None:
+            assert self.max_abs <= t["max_abs_rms"] * rms, (
+                f"{self.what}: max_abs {self.max_abs:.3e} > {t['max_abs_rms']} * rms {rms:.3e}")
+        return e

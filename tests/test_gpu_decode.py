@@ -7,7 +7,7 @@ import torch
 import gated_delta_rule_121_b200 as kda
 import oracle
 import synth
-from parity import assert_close, errors
+from parity import ErrorAccumulator, assert_close, errors
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -34,21 +34,31 @@ def test_decode_steps_match_oracle(dtype, dk, dv):
     assert_close(state, ref, dtype, "decode state")
 
 
-def test_decode_full_shape_sampled():
-    """B=512, H=96, dk=dv=128, bf16: 3 steps; sequences/heads sampled for the oracle."""
+def test_decode_full_shape_256_steps_sampled():
+    """The decode workload as specified: B=512, H=96, dk=dv=128, bf16 inputs,
+    256 consecutive in-place steps on the resident fp32 state.  24 (sequence,
+    head) pairs are followed by the fp64 oracle: every step's output and the
+    state after the last step, at the literal bounds."""
     spec = synth.DECODE
+    assert spec.steps == 256
     state = synth.make_decode_state(spec, DEV)
-    bsel = torch.tensor([0, 1, 255, 511])
-    hsel = torch.tensor([0, 47, 95])
-    ref = state[bsel][:, hsel].cpu().double().numpy().copy()
-    for step in range(3):
+    bsel = torch.tensor([0, 1, 137, 255, 384, 511])
+    hsel = torch.tensor([0, 31, 64, 95])
+    pick = lambda t: t[bsel][:, hsel]
+    ref = pick(state).cpu().double().numpy().copy()
+    acc = ErrorAccumulator(torch.bfloat16, "decode outputs over 256 steps")
+    out = torch.empty((spec.B, spec.H, spec.dv), dtype=spec.dtype, device=DEV)
+    for step in range(spec.steps):
         x = synth.make_decode_step(spec, step, DEV)
-        out = kda.kda_decode_step(x["q"], x["k"], x["v"], x["g"], x["beta"], state)
-        pick = lambda t: t[bsel][:, hsel]
+        kda.kda_decode_step(x["q"], x["k"], x["v"], x["g"], x["beta"], state, out=out)
         o_ref = oracle.decode_step(pick(x["q"]), pick(x["k"]), pick(x["v"]), pick(x["g"]), pick(x["beta"]), ref)
-        assert_close(pick(out), o_ref, torch.bfloat16, f"decode full out step {step}")
+        o = pick(out)
+        assert_close(o, o_ref, torch.bfloat16, f"decode full out step {step}")
+        acc.add(o, o_ref)
     torch.cuda.synchronize()
-    assert_close(state[bsel][:, hsel], ref, torch.bfloat16, "decode full state")
+    acc.check()
+    e = assert_close(pick(state), ref, torch.bfloat16, "decode full state after 256 steps")
+    print("decode 256 steps: final state", e)
 
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])

@@ -8,7 +8,7 @@ import torch
 import gated_delta_rule_121_b200 as kda
 import oracle
 import synth
-from parity import assert_close, errors
+from parity import ErrorAccumulator, assert_close, errors
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -28,15 +28,34 @@ def run_oracle(inp, heads=None):
                       inp["cu_seqlens"])
 
 
-def check(inp, dtype, heads=None, what=""):
+def check(inp, dtype, heads=None, what="", literal=True):
     out, fin = run_gpu(inp)
     torch.cuda.synchronize()
-    o_ref, f_ref = run_oracle(inp, heads)
     if heads is not None:
-        out, fin = out[:, :, heads], fin[:, heads]
-    eo = assert_close(out, o_ref, dtype, f"{what} out")
-    ef = assert_close(fin, f_ref, dtype, f"{what} final_state")
+        return check_sampled(inp, out, fin, dtype, heads, what)
+    o_ref, f_ref = run_oracle(inp, heads)
+    eo = assert_close(out, o_ref, dtype, f"{what} out", literal=literal)
+    ef = assert_close(fin, f_ref, dtype, f"{what} final_state", literal=literal)
     return eo, ef
+
+
+def check_sampled(inp, out, fin, dtype, heads, what, per_call=2):
+    """The oracle on the sampled heads, a few at a time, with the errors
+    accumulated over all of them (literal bounds)."""
+    ao, af = ErrorAccumulator(dtype, f"{what} out"), ErrorAccumulator(dtype, f"{what} final_state")
+    for i in range(0, len(heads), per_call):
+        hs = list(heads[i:i + per_call])
+        o_ref, f_ref = run_oracle(inp, hs)
+        ao.add(out[:, :, hs], o_ref)
+        af.add(fin[:, hs], f_ref)
+        del o_ref, f_ref
+    return ao.check(), af.check()
+
+
+def sampled_heads(H, n=8, seed=0):
+    """n seeded heads, always including the first and the last."""
+    rest = np.random.default_rng(seed).choice(np.arange(1, H - 1), size=n - 2, replace=False)
+    return sorted({0, H - 1, *rest.tolist()})
 
 
 def test_tiny_fp32_exact_path():
@@ -68,7 +87,7 @@ def test_stress_model_range_decay():
     """g = -5 sigmoid(z): chunk totals far below the factorisation floor."""
     inp = synth.make_prefill(synth.STRESS, DEV)
     assert float(inp["g"].min()) < -4.0
-    check(inp, torch.bfloat16, what="stress g>=-5")
+    check(inp, torch.bfloat16, what="stress g>=-5", literal=False)
 
 
 def test_mixed_decay_chunks():
@@ -78,7 +97,7 @@ def test_mixed_decay_chunks():
     for c in range(0, 512, 128):
         g[:, c:c + 64] *= 64.0          # -5 * sigmoid(z) on every other chunk
     inp["g"] = g.contiguous()
-    check(inp, torch.bfloat16, what="mixed decay")
+    check(inp, torch.bfloat16, what="mixed decay", literal=False)
 
 
 def test_model_range_decay_ragged_packed():
@@ -88,7 +107,7 @@ def test_model_range_decay_ragged_packed():
     inp = synth.make_prefill(synth.VARLEN, DEV, H=3, lengths=[1, 37, 64, 100, 130, 0, 257])
     inp["g"] = (inp["g"] * 64.0).contiguous()
     assert float(inp["g"].min()) < -4.0
-    check(inp, torch.bfloat16, what="varlen model-range decay")
+    check(inp, torch.bfloat16, what="varlen model-range decay", literal=False)
 
 
 def test_decay_beyond_the_model_bound():
@@ -97,7 +116,7 @@ def test_decay_beyond_the_model_bound():
     inp = synth.make_prefill(synth.VARLEN, DEV, H=2, lengths=[257, 64, 3, 190])
     inp["g"] = (inp["g"] * 256.0).contiguous()
     assert float(inp["g"].min()) < -15.0
-    check(inp, torch.bfloat16, what="g >= -20")
+    check(inp, torch.bfloat16, what="g >= -20", literal=False)
 
 
 @pytest.mark.parametrize("lengths", [[1, 63, 64, 65, 130, 0, 200], [0], [5], [300, 0, 0, 64]])
@@ -170,26 +189,33 @@ def test_chained_calls_equal_single_call():
     b = {k: (part(v, slice(T1, None)) if k in ("q", "k", "v", "g", "beta") else v) for k, v in inp.items()}
     b["init_state"] = mid
     o2, f2 = run_gpu(b)
-    e = errors(torch.cat([o1, o2], 1), o_full)
-    assert e["rel_fro"] < 1e-2
-    assert errors(f2, f_full)["rel_fro"] < 1e-2
+    torch.cuda.synchronize()
+    o_ref, f_ref = run_oracle(inp)
+    assert_close(torch.cat([o1, o2], 1), o_ref, torch.bfloat16, "chained out")
+    assert_close(f2, f_ref, torch.bfloat16, "chained final_state")
+    assert_close(o_full, o_ref, torch.bfloat16, "single-call out")
+    # the two GPU paths agree with each other far inside the oracle tolerance
+    assert errors(torch.cat([o1, o2], 1), o_full)["rel_fro"] < 5e-3
+    assert errors(f2, f_full)["rel_fro"] < 5e-3
 
 
 def test_model_shaped_prefill_sampled_heads():
-    """B=1, H=96, T=65536 (the 64K pretraining shape), heads 0 and 95 checked."""
+    """B=1, H=96, T=65536 (the 64K pretraining shape), eight seeded heads
+    including 0 and 95, at the literal max-abs bound."""
     inp = synth.make_prefill(synth.PRETRAIN, DEV)
-    eo, ef = check(inp, torch.bfloat16, heads=[0, 95], what="prefill H96 T65536")
+    eo, ef = check(inp, torch.bfloat16, heads=sampled_heads(96, seed=2), what="prefill H96 T65536")
     print("pretrain errors", eo, ef)
 
 
 def test_packed_varlen_full_size_sampled_heads():
     """The packed long-context workload at full size: H=32, 1,048,576 tokens in
     sequences of log-uniform length in [1024, 262144], each with its own
-    initial state; heads 0 and 31 of every sequence checked."""
+    initial state; eight seeded heads (0 and 31 among them) of every sequence
+    checked at the literal max-abs bound."""
     inp = synth.make_prefill(synth.VARLEN, DEV)
     cu = inp["cu_seqlens"].cpu()
     assert int(cu[-1]) == 1 << 20 and cu.numel() - 1 >= 3
-    eo, ef = check(inp, torch.bfloat16, heads=[0, 31], what="varlen H32 T1M")
+    eo, ef = check(inp, torch.bfloat16, heads=sampled_heads(32, seed=3), what="varlen H32 T1M")
     print("varlen errors", cu.numel() - 1, "sequences", eo, ef)
 
 
@@ -263,3 +289,19 @@ def test_fp16_range_overflow_is_reported(what):
     assert kda.kda_workspace_status(ws) == kda.KDA_ERR_RANGE
     kda.kda_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["init_state"], workspace=ws)
     assert kda.kda_workspace_status(ws) == kda.KDA_OK
+
+
+@pytest.mark.parametrize("packed", [False, True])
+def test_host_buffer_entry_point_matches_device_call(packed):
+    """kda_fwd_host (host buffers, copies enqueued by the library) returns the
+    bits kda_fwd returns on device buffers."""
+    if packed:
+        inp = synth.make_prefill(synth.VARLEN, DEV, H=3, lengths=[70, 0, 129])
+    else:
+        inp = synth.make_prefill(synth.MID, DEV, T=200, B=2, H=3)
+    ref_out, ref_fin = run_gpu(inp)
+    host = {n: (None if t is None else t.cpu().pin_memory()) for n, t in inp.items()}
+    out_h, fin_h, _ = kda.kda_fwd_host(host["q"], host["k"], host["v"], host["g"], host["beta"],
+                                       host["init_state"], host["cu_seqlens"], device=DEV)
+    torch.cuda.synchronize()
+    assert torch.equal(out_h, ref_out.cpu()) and torch.equal(fin_h, ref_fin.cpu())

@@ -17,3 +17,27 @@ def test_half_ulp_bounds_bf16_rounding():
     assert (err > 0.9 * hu).any()
     assert half_ulp_bf16(np.array([1.0]))[0] == 2.0 ** -8
     assert half_ulp_bf16(np.array([0.0]))[0] == 0.0
+
+
+def test_error_accumulator_matches_one_shot_measures():
+    import pytest
+    from parity import ErrorAccumulator, assert_close, errors
+    rng = np.random.default_rng(1)
+    ref = rng.standard_normal((4, 50, 6))
+    x = ref + 1e-3 * rng.standard_normal(ref.shape)
+    acc = ErrorAccumulator(torch.bfloat16, "pieces")
+    for h in range(6):
+        acc.add(x[:, :, h], ref[:, :, h])
+    e = acc.check()
+    e1 = errors(x, ref)
+    assert abs(e["rel_fro"] - e1["rel_fro"]) < 1e-12 * e1["rel_fro"] + 1e-15
+    assert e["max_abs"] == e1["max_abs"] and abs(e["rms"] - e1["rms"]) < 1e-12
+    # the literal max-abs bound fails where one element is off by more than 3e-2 RMS
+    y = x.copy()
+    y[0, 0, 0] += 0.05
+    bad = ErrorAccumulator(torch.bfloat16, "pieces")
+    bad.add(y, ref)
+    with pytest.raises(AssertionError):
+        bad.check()
+    with pytest.raises(AssertionError):
+        assert_close(y, ref, torch.bfloat16, literal=True)
