@@ -313,9 +313,11 @@ TRAFFIC_PROFILES = {
 FLUSH = {"mid": True, "stress": True, "prefill64k": False, "varlen": False}
 
 
-def bench_prefill(name, d, dev, stream, peaks, kda, synth, steps, warmup, with_traffic=False):
-    """Time `steps` kda_fwd launches over one workload; returns its JSON object
-    and the inputs (for the end-to-end leg)."""
+def bench_prefill(name, d, dev, stream, peaks, kda, synth, steps, warmup, with_traffic=False, variant=None):
+    """Time `steps` forward calls over one workload; returns its JSON object
+    and the inputs (for the end-to-end leg).  variant: None (kda_fwd), "cp"
+    (kda_fwd_cp, every sequence split over the SMs) or "ckpt512" (kda_fwd_checkpoints,
+    the state every 512 tokens)."""
     import torch
     spec = workload_spec(name)
     inp = synth.make_prefill(spec, dev)
@@ -327,9 +329,33 @@ def bench_prefill(name, d, dev, stream, peaks, kda, synth, steps, warmup, with_t
     out = torch.empty_like(v)
     fin = torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev)
     ws = kda.alloc_workspace(N, B * T, H, dk, dv, q.dtype, dev)
+    extra = {}
+    launches = 2 if (cu is not None and N > 1) else 1  # packed batches: the order kernel, then the forward
+    ckpt_bytes = 0
+    if variant == "cp":
+        n_seg = kda.kda_cp_segments(N, (B * T) // N, H)
+        ws = kda.alloc_cp_workspace(N, B * T, H, dk, dv, n_seg, q.dtype, dev)
+        extra["n_seg"] = n_seg
+        launches = 5  # segment offsets, order, segment pieces, composition, correction
 
-    def step():
-        kda.kda_fwd(q, k, v, g, beta, init, cu, out=out, final_state=fin, workspace=ws, stream=stream)
+        def step():
+            kda.kda_fwd_cp(q, k, v, g, beta, init, cu, n_seg=n_seg, out=out, final_state=fin, workspace=ws,
+                           stream=stream)
+    elif variant == "ckpt512":
+        cap = N * (T // 512) if cu is None else int(((cu[1:] - cu[:-1]).cpu() // 512).sum())
+        ck = torch.empty((cap, H, dk, dv), dtype=torch.float32, device=dev)
+        n = kda.lib().kda_fwd_checkpoints_workspace_size(N, B * T, H, dk, dv, kda._DT[q.dtype])
+        ws = torch.empty(n, dtype=torch.uint8, device=dev)
+        extra.update(interval=512, checkpoints=cap)
+        ckpt_bytes = cap * H * dk * dv * 4
+        launches += 1 if cu is not None else 0
+
+        def step():
+            kda.kda_fwd_checkpoints(q, k, v, g, beta, init, cu, interval=512, capacity=cap, out=out,
+                                    final_state=fin, checkpoints=ck, workspace=ws, stream=stream)
+    else:
+        def step():
+            kda.kda_fwd(q, k, v, g, beta, init, cu, out=out, final_state=fin, workspace=ws, stream=stream)
 
     flush = FLUSH[name]
     sec = (time_loop_flushed if flush else time_loop)(step, steps, warmup, stream, d)
@@ -337,7 +363,7 @@ def bench_prefill(name, d, dev, stream, peaks, kda, synth, steps, warmup, with_t
     if status != kda.KDA_OK:
         raise RuntimeError(f"{name}: device status {kda.kda_status_string(status)}")
     per_step = d.max(sec) / steps
-    bytes_alg = prefill_bytes(th, N * H, dk, dv, q.element_size(), init is not None)
+    bytes_alg = prefill_bytes(th, N * H, dk, dv, q.element_size(), init is not None) + ckpt_bytes
     flops_alg = prefill_flops(th, dk, dv)
     achieved = bytes_alg / per_step / 1e9
     peak = peaks["hbm_gbs"]
@@ -347,8 +373,7 @@ def bench_prefill(name, d, dev, stream, peaks, kda, synth, steps, warmup, with_t
         prof, src = TRAFFIC_PROFILES["kda_fwd_tc_kernel"]
         fixed = N * H * dk * dv * 4 * (2 if init is not None else 1)
         traffic = scaled_traffic(prof, src, th, fixed)
-    launches = 2 if (cu is not None and N > 1) else 1  # packed batches: the order kernel, then the forward
-    res = {"workload": spec.name, "value": job_throughput(d, th * steps, sec) / 1e6, "unit": UNIT,
+    res = {"workload": spec.name + (f"_{variant}" if variant else ""), "value": job_throughput(d, th * steps, sec) / 1e6, "unit": UNIT,
            "ms_per_step": per_step * 1e3, "steps": steps, "sequences": N, "token_heads": th,
            "l2": ("flushed before every launch (256 MB write)" if flush else
                   "inputs larger than L2 (%.1f GB per step), no flush" % (bytes_alg / 1e9)),
@@ -358,7 +383,9 @@ def bench_prefill(name, d, dev, stream, peaks, kda, synth, steps, warmup, with_t
                         "kernel": "kda_fwd_tc_kernel",
                         "tensor_tflops": flops_alg / per_step / 1e12,
                         "tensor_frac_of_bf16_peak": flops_alg / per_step / 1e12 / peaks["bf16_tflops"]},
-           "gpu_launches": steps * launches}
+           "gpu_launches": steps * launches, **extra}
+    if variant == "cp":
+        res["roofline"]["kernel"] = "kda_fwd_tc_kernel (segment mode) + composition + correction"
     del out, fin, ws
     return res, inp
 
@@ -401,11 +428,13 @@ def run_native(args, d):
         line["decode"] = bench_decode(args, d, dev, stream, peaks, kda, synth)
     if not args.no_workloads:
         others = {}
-        for name, steps in (("mid", 50), ("varlen", 8), ("stress", 50)):
-            if name == args.workload:
+        for key, name, steps, variant in (("mid", "mid", 50, None), ("mid_cp", "mid", 50, "cp"),
+                                          ("varlen", "varlen", 8, None), ("stress", "stress", 50, None),
+                                          ("prefill64k_ckpt512", "prefill64k", 10, "ckpt512")):
+            if name == args.workload and variant is None:
                 continue
-            res, _ = bench_prefill(name, d, dev, stream, peaks, kda, synth, steps, args.warmup)
-            others[name] = res
+            res, _ = bench_prefill(name, d, dev, stream, peaks, kda, synth, steps, args.warmup, variant=variant)
+            others[key] = res
             torch.cuda.empty_cache()
         line["workloads"] = others
     if d.world == 1 and d.rank == 0 and not args.no_cpu_baseline:

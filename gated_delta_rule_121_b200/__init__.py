@@ -8,6 +8,10 @@ loaded, every call raises.
 Functions mirror the C entry points:
   kda_fwd(q, k, v, log_alpha, beta, ...)        chunked prefill
   kda_fwd_noalloc(...)                           the same, scratch in a fixed library array
+  kda_fwd_checkpoints(..., interval)             prefill plus the state every `interval` tokens
+  kda_segment_fwd(...)                           zero-start outputs/state and transition of segments
+  kda_state_compose(...), kda_output_correct(...)   prefix composition, output correction
+  kda_fwd_cp(..., n_seg)                         prefill with every sequence split over the SMs
   kda_decode_step(q, k, v, log_alpha, beta, state, ...)   in-place decode
   kda_fwd_workspace_size(...), kda_workspace_status(ws), kda_status_string(s)
 and ``kda_fwd_host`` runs kda_fwd on host (pinned) tensors through the C
@@ -71,6 +75,26 @@ def lib() -> ctypes.CDLL:
         L.kda_fwd_host.restype = ctypes.c_int
         L.kda_fwd_host.argtypes = [_vp, _vp, ctypes.c_int, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                    _vp, ctypes.c_int, _vp, ctypes.c_size_t]
+        L.kda_fwd_checkpoints_workspace_size.restype = ctypes.c_size_t
+        L.kda_fwd_checkpoints_workspace_size.argtypes = L.kda_fwd_workspace_size.argtypes
+        L.kda_fwd_checkpoints.restype = ctypes.c_int
+        L.kda_fwd_checkpoints.argtypes = fwd_args[:-2] + [_fp, ctypes.c_int, ctypes.c_int64, _vp, ctypes.c_size_t]
+        L.kda_segment_fwd.restype = ctypes.c_int
+        L.kda_segment_fwd.argtypes = [_vp, _vp, _vp, _fp, _fp, _fp, _fp, _fp, _fp, ctypes.c_int, ctypes.c_int64,
+                                      ctypes.c_int, ctypes.c_int, ctypes.c_int, _i32p, _vp, ctypes.c_int, _vp,
+                                      ctypes.c_size_t]
+        L.kda_state_compose.restype = ctypes.c_int
+        L.kda_state_compose.argtypes = [_fp, _fp, _fp, _fp, _fp] + [ctypes.c_int] * 6 + [_vp]
+        L.kda_output_correct.restype = ctypes.c_int
+        L.kda_output_correct.argtypes = [_fp, _fp, _fp, _vp, ctypes.c_int, ctypes.c_int64, ctypes.c_int,
+                                         ctypes.c_int, ctypes.c_int, _i32p, _vp, ctypes.c_int]
+        L.kda_fwd_cp_workspace_size.restype = ctypes.c_size_t
+        L.kda_fwd_cp_workspace_size.argtypes = [ctypes.c_int, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
+                                                ctypes.c_int, ctypes.c_int, ctypes.c_int]
+        L.kda_cp_segments.restype = ctypes.c_int
+        L.kda_cp_segments.argtypes = [ctypes.c_int, ctypes.c_int64, ctypes.c_int, ctypes.c_int]
+        L.kda_fwd_cp.restype = ctypes.c_int
+        L.kda_fwd_cp.argtypes = fwd_args[:-2] + [ctypes.c_int, _vp, ctypes.c_size_t]
         L.kda_workspace_status.restype = ctypes.c_int
         L.kda_workspace_status.argtypes = [_vp, _vp]
         _lib = L
@@ -158,6 +182,145 @@ def kda_fwd(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None, out=None
                                      int(bool(_inject_stuck)))
     _check(code, "kda_fwd")
     return out, final_state
+
+
+def _check_inputs(q, k, v, log_alpha, beta, init_state, cu_seqlens, N, H, dk, dv):
+    for name, t, dtype in (("k", k, q.dtype), ("v", v, q.dtype), ("log_alpha", log_alpha, torch.float32),
+                           ("beta", beta, torch.float32)):
+        if t.dtype != dtype or not t.is_contiguous() or t.device != q.device:
+            raise ValueError(f"{name}: expected contiguous {dtype} on {q.device}")
+    if init_state is not None and (init_state.dtype != torch.float32 or not init_state.is_contiguous()
+                                   or tuple(init_state.shape) != (N, H, dk, dv)):
+        raise ValueError("init_state must be contiguous fp32 [N, H, dk, dv]")
+    if cu_seqlens is not None and cu_seqlens.dtype != torch.int32:
+        raise ValueError("cu_seqlens must be int32")
+
+
+def kda_fwd_checkpoints(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None, interval=512, capacity=None,
+                        out=None, final_state=None, checkpoints=None, workspace=None, stream=None):
+    """kda_fwd plus the state after every whole multiple of ``interval`` tokens
+    of each sequence (include/kda.h, kda_fwd_checkpoints).  ``capacity`` (the
+    number of checkpoint slots) defaults to the exact count, which for packed
+    batches is computed from ``cu_seqlens`` on the host (one small copy).
+    Returns ``(out, final_state, checkpoints [capacity, H, dk, dv])``."""
+    B, T, H, dk, dv, N = _shapes(q, v, cu_seqlens)
+    _check_inputs(q, k, v, log_alpha, beta, init_state, cu_seqlens, N, H, dk, dv)
+    if capacity is None:
+        if cu_seqlens is None:
+            capacity = N * (T // interval)
+        else:
+            lens = (cu_seqlens[1:] - cu_seqlens[:-1]).cpu()
+            capacity = int((lens // interval).sum())
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    if final_state is None:
+        final_state = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
+    if checkpoints is None:
+        checkpoints = torch.empty((max(capacity, 0), H, dk, dv), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        n = int(lib().kda_fwd_checkpoints_workspace_size(N, B * T, H, dk, dv, _DT[q.dtype]))
+        workspace = torch.empty(max(n, 16), dtype=torch.uint8, device=q.device)
+    code = lib().kda_fwd_checkpoints(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(init_state),
+                                     _ptr(out), _ptr(final_state), N, T, H, dk, dv, _ptr(cu_seqlens),
+                                     _stream_ptr(stream), _DT[q.dtype], _ptr(checkpoints), int(interval),
+                                     int(capacity), _ptr(workspace), workspace.numel())
+    _check(code, "kda_fwd_checkpoints")
+    return out, final_state, checkpoints
+
+
+def kda_segment_fwd(q, k, v, log_alpha, beta, cu_seqlens=None, workspace=None, stream=None):
+    """Pieces of every sequence taken as one segment (include/kda.h,
+    kda_segment_fwd).  Returns ``(out_zero, state_zero, qhat, transition)``,
+    all fp32: zero-start outputs [B,T,H,dv] and final states [N,H,dk,dv], and
+    qhat [B,T,H,dk] with the segment transitions [N,H,dk,dk]."""
+    B, T, H, dk, dv, N = _shapes(q, v, cu_seqlens)
+    _check_inputs(q, k, v, log_alpha, beta, None, cu_seqlens, N, H, dk, dv)
+    dev = q.device
+    out_zero = torch.empty((B, T, H, dv), dtype=torch.float32, device=dev)
+    qhat = torch.empty((B, T, H, dk), dtype=torch.float32, device=dev)
+    state_zero = torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev)
+    transition = torch.empty((N, H, dk, dk), dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = alloc_workspace(N, B * T, H, dk, dv, q.dtype, dev)
+    code = lib().kda_segment_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(out_zero),
+                                 _ptr(state_zero), _ptr(qhat), _ptr(transition), N, T, H, dk, dv,
+                                 _ptr(cu_seqlens), _stream_ptr(stream), _DT[q.dtype], _ptr(workspace),
+                                 workspace.numel())
+    _check(code, "kda_segment_fwd")
+    return out_zero, state_zero, qhat, transition
+
+
+def kda_state_compose(transition, state_zero, R, init_state=None, rank_major=False, state_in=None,
+                      final_state=None, stream=None):
+    """Incoming state of every piece and the final state of N sequences cut
+    into R pieces (include/kda.h, kda_state_compose).  transition
+    [R*N,H,dk,dk] and state_zero [R*N,H,dk,dv] fp32 on the device.  Returns
+    ``(state_in [R*N,H,dk,dv], final_state [N,H,dk,dv])``."""
+    P, H, dk, dv = state_zero.shape
+    if P % R:
+        raise ValueError("the piece count must be a multiple of R")
+    N = P // R
+    for t in (transition, state_zero, init_state):
+        if t is not None and (t.dtype != torch.float32 or not t.is_contiguous()):
+            raise ValueError("states must be contiguous fp32")
+    if state_in is None:
+        state_in = torch.empty_like(state_zero)
+    if final_state is None:
+        final_state = torch.empty((N, H, dk, dv), dtype=torch.float32, device=state_zero.device)
+    code = lib().kda_state_compose(_ptr(transition), _ptr(state_zero), _ptr(init_state), _ptr(state_in),
+                                   _ptr(final_state), R, N, H, dk, dv, int(bool(rank_major)), _stream_ptr(stream))
+    _check(code, "kda_state_compose")
+    return state_in, final_state
+
+
+def kda_output_correct(out_zero, qhat, state_in, cu_seqlens=None, dtype=torch.bfloat16, out=None, stream=None):
+    """out_t = out_zero_t + S_in^T qhat_t with S_in = state_in[sequence of t]
+    (include/kda.h, kda_output_correct).  Returns ``out`` in ``dtype``."""
+    B, T, H, dv = out_zero.shape
+    dk = qhat.shape[-1]
+    N = cu_seqlens.numel() - 1 if cu_seqlens is not None else B
+    if tuple(state_in.shape) != (N, H, dk, dv):
+        raise ValueError("state_in must be [N, H, dk, dv]")
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=dtype, device=out_zero.device)
+    code = lib().kda_output_correct(_ptr(out_zero), _ptr(qhat), _ptr(state_in), _ptr(out), N, T, H, dk, dv,
+                                    _ptr(cu_seqlens), _stream_ptr(stream), _DT[out.dtype])
+    _check(code, "kda_output_correct")
+    return out
+
+
+def kda_cp_segments(N, tokens_per_sequence, H, sm_count=None) -> int:
+    """Segments per sequence suggested for kda_fwd_cp on this device."""
+    if sm_count is None:
+        sm_count = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    return int(lib().kda_cp_segments(N, tokens_per_sequence, H, sm_count))
+
+
+def kda_fwd_cp(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None, n_seg=None, out=None,
+               final_state=None, workspace=None, stream=None):
+    """kda_fwd with every sequence split into ``n_seg`` segments that run on
+    separate SMs (include/kda.h, kda_fwd_cp).  ``n_seg`` defaults to
+    kda_cp_segments(...).  Returns ``(out, final_state)``."""
+    B, T, H, dk, dv, N = _shapes(q, v, cu_seqlens)
+    _check_inputs(q, k, v, log_alpha, beta, init_state, cu_seqlens, N, H, dk, dv)
+    if n_seg is None:
+        n_seg = kda_cp_segments(N, (B * T) // max(N, 1), H)
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    if final_state is None:
+        final_state = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = alloc_cp_workspace(N, B * T, H, dk, dv, n_seg, q.dtype, q.device)
+    code = lib().kda_fwd_cp(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(init_state), _ptr(out),
+                            _ptr(final_state), N, T, H, dk, dv, _ptr(cu_seqlens), _stream_ptr(stream),
+                            _DT[q.dtype], int(n_seg), _ptr(workspace), workspace.numel())
+    _check(code, "kda_fwd_cp")
+    return out, final_state
+
+
+def alloc_cp_workspace(N, T_total, H, dk, dv, n_seg, dtype=torch.bfloat16, device="cuda"):
+    n = int(lib().kda_fwd_cp_workspace_size(N, T_total, H, dk, dv, _DT[dtype], n_seg))
+    return torch.empty(max(n, 16), dtype=torch.uint8, device=device)
 
 
 def kda_fwd_noalloc(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None, out=None, final_state=None,

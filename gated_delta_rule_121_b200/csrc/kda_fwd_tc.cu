@@ -1156,7 +1156,7 @@ __device__ __forceinline__ void scan_group(const Ctx& x, const void* tmq, const 
       if constexpr (MODE == MODE_CKPT) {
         // The state after chunk c-1 (before this chunk's decay) is the
         // checkpoint of the interval that ends there.
-        if (c % ma.ckpt_every == 0) store_ckpt(x, ma, x.ckpt0 + c / ma.ckpt_every - 1, cp * 64, s0, s1);
+        if (c > 0 && c % ma.ckpt_every == 0) store_ckpt(x, ma, x.ckpt0 + c / ma.ckpt_every - 1, cp * 64, s0, s1);
       }
       if (fast) {
 #pragma unroll

@@ -19,7 +19,10 @@
 //     independently), and
 //   - the correction o_t = o~_t + S_in^T qhat_t (dense 64-token x dv tiles on
 //     the warp-level tensor path with tf32 operands rounded to nearest; the
-//     zero-start output o~ stays fp32, so the result is rounded once).
+//     zero-start output o~ stays fp32, so the result is rounded once).  For
+//     fp32 outputs, whose contract allows no tf32 rounding, every product is
+//     split into three tf32 products (hi*hi + hi*lo + lo*hi), accurate to
+//     about fp32.
 #include <cstdint>
 
 #include "../../include/kda.h"
@@ -148,19 +151,27 @@ __global__ void __launch_bounds__(128)
 #pragma unroll
     for (int n = 0; n < DV / 8; ++n) d[n][0] = d[n][1] = d[n][2] = d[n][3] = 0.f;
     const float* qa = s_q + (w * 16) * (DK + CPAD);
+    constexpr bool SPLIT = sizeof(IO) == 4;  // fp32 outputs: three-term tf32 products
 #pragma unroll 2
     for (int k0 = 0; k0 < DK; k0 += 8) {
-      uint32_t a[4];
-      a[0] = tf32_rna(qa[g * (DK + CPAD) + k0 + tq]);
-      a[1] = tf32_rna(qa[(g + 8) * (DK + CPAD) + k0 + tq]);
-      a[2] = tf32_rna(qa[g * (DK + CPAD) + k0 + tq + 4]);
-      a[3] = tf32_rna(qa[(g + 8) * (DK + CPAD) + k0 + tq + 4]);
+      const float af[4] = {qa[g * (DK + CPAD) + k0 + tq], qa[(g + 8) * (DK + CPAD) + k0 + tq],
+                           qa[g * (DK + CPAD) + k0 + tq + 4], qa[(g + 8) * (DK + CPAD) + k0 + tq + 4]};
+      uint32_t a[4], al[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        a[i] = tf32_rna(af[i]);
+        if (SPLIT) al[i] = tf32_rna(af[i] - __uint_as_float(a[i]));
+      }
 #pragma unroll
       for (int n = 0; n < DV / 8; ++n) {
-        uint32_t b[2];
-        b[0] = tf32_rna(s_s[(k0 + tq) * (DV + CPAD) + n * 8 + g]);
-        b[1] = tf32_rna(s_s[(k0 + tq + 4) * (DV + CPAD) + n * 8 + g]);
+        const float bf[2] = {s_s[(k0 + tq) * (DV + CPAD) + n * 8 + g], s_s[(k0 + tq + 4) * (DV + CPAD) + n * 8 + g]};
+        uint32_t b[2] = {tf32_rna(bf[0]), tf32_rna(bf[1])};
         mma_tf32_16x8x8(d[n], a, b);
+        if (SPLIT) {
+          const uint32_t bl[2] = {tf32_rna(bf[0] - __uint_as_float(b[0])), tf32_rna(bf[1] - __uint_as_float(b[1]))};
+          mma_tf32_16x8x8(d[n], a, bl);
+          mma_tf32_16x8x8(d[n], al, b);
+        }
       }
     }
 #pragma unroll

@@ -116,3 +116,24 @@ def decode_step(q, k, v, g, beta, state):
     lib.kda_oracle_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state),
                                _ptr(out), B, H, dk, dv)
     return out
+
+
+def transition(q, k, g, beta, cu_seqlens=None, nthreads: int | None = None):
+    """Segment transition of every (sequence, head) and the transformed queries.
+
+    The KCP paragraph of the digest's co-design section writes the recurrence
+    as ``S_t = M_t S_{t-1} + beta_t k_t v_t^T`` with
+    ``M_t = (I - beta_t k_t k_t^T) Diag(alpha_t)``; the transition of a
+    segment is ``M = M_last ... M_first``.  With every value zero the
+    recurrence is ``S_t = M_t S_{t-1}``, so starting from ``S_0 = I`` it gives
+    ``S_t = M_t ... M_first`` and reads ``o_t = S_t^T q_t``.  Returns
+    ``(qhat [B,T,H,dk], M [N,H,dk,dk])`` as float64 arrays, where qhat_t is
+    that read: the transition through token t applied to q_t.
+    """
+    q64 = _f64(q)
+    B, T, H, dk = q64.shape
+    N = B if cu_seqlens is None else (len(cu_seqlens) - 1 if not hasattr(cu_seqlens, "numel")
+                                       else cu_seqlens.numel() - 1)
+    zeros_v = np.zeros((B, T, H, dk), np.float64)
+    eye = np.broadcast_to(np.eye(dk), (N, H, dk, dk)).copy()
+    return fwd(q64, k, zeros_v, g, beta, eye, cu_seqlens, nthreads=nthreads)

@@ -110,3 +110,42 @@ def test_no_cpu_fallback_in_product_path():
     src = open(os.path.join(ROOT, "gated_delta_rule_121_b200", "__init__.py")).read()
     assert "oracle" not in src
     assert "numpy" not in src
+
+
+def test_new_entry_points_reject_invalid_arguments_on_the_host():
+    L = kda.lib()
+    fwd = [P(256), P(512), P(768), P(1024), P(1280), None, P(1536), P(2048), 1, 64, 2, 128, 128, None, None,
+           kda.KDA_BF16]
+    # checkpoints: interval must be a positive multiple of 64; a batched call needs B*floor(T/interval) slots
+    assert L.kda_fwd_checkpoints(*fwd, P(4096), 100, 8, P(8192), 1 << 20) == kda.KDA_ERR_UNSUPPORTED
+    assert L.kda_fwd_checkpoints(*fwd, P(4096), 0, 8, P(8192), 1 << 20) == kda.KDA_ERR_UNSUPPORTED
+    assert L.kda_fwd_checkpoints(*fwd, P(4096), 64, 0, P(8192), 1 << 20) == kda.KDA_ERR_INVALID_ARG
+    assert L.kda_fwd_checkpoints(*fwd, P(4100), 64, 8, P(8192), 1 << 20) == kda.KDA_ERR_INVALID_ARG
+    assert L.kda_fwd_checkpoints(*fwd, P(4096), 64, 8, None, 0) == kda.KDA_ERR_WORKSPACE
+    # segment pieces need square states
+    seg = [P(256), P(512), P(768), P(1024), P(1280), P(1536), P(2048), P(2560), P(3072)]
+    assert L.kda_segment_fwd(*seg, 1, 64, 2, 128, 64, None, None, kda.KDA_BF16, P(8192), 1024) == \
+        kda.KDA_ERR_UNSUPPORTED
+    assert L.kda_segment_fwd(*seg[:5], None, *seg[6:], 1, 64, 2, 128, 128, None, None, kda.KDA_BF16, P(8192),
+                             1024) == kda.KDA_ERR_INVALID_ARG
+    # composition and correction
+    assert L.kda_state_compose(P(256), P(512), None, None, None, 2, 1, 1, 96, 128, 0, None) == kda.KDA_ERR_UNSUPPORTED
+    assert L.kda_state_compose(None, None, None, None, None, 2, 1, 1, 128, 128, 0, None) == kda.KDA_ERR_INVALID_ARG
+    assert L.kda_state_compose(None, None, None, None, None, 2, 0, 1, 128, 128, 0, None) == kda.KDA_OK
+    assert L.kda_output_correct(P(256), P(512), P(768), P(1032), 1, 64, 2, 128, 128, None, None,
+                                kda.KDA_BF16) == kda.KDA_ERR_INVALID_ARG
+    assert L.kda_output_correct(P(256), P(512), P(768), P(1024), 1, 0, 2, 128, 128, None, None,
+                                kda.KDA_BF16) == kda.KDA_OK
+    # context parallelism: n_seg >= 1, square states, a large enough workspace
+    cp = fwd + [2]
+    assert L.kda_fwd_cp(*fwd, 0, P(8192), 1 << 30) == kda.KDA_ERR_INVALID_ARG
+    assert L.kda_fwd_cp(*cp, P(8192), 64) == kda.KDA_ERR_WORKSPACE
+    need = L.kda_fwd_cp_workspace_size(1, 64, 2, 128, 128, kda.KDA_BF16, 2)
+    assert need >= 64 * 2 * 256 * 4
+    assert L.kda_cp_segments(2, 4096, 16, 148) == 2
+    assert L.kda_cp_segments(1, 65536, 96, 148) == 1
+
+
+def test_kcp_module_has_no_oracle_or_cpu_path():
+    src = open(os.path.join(ROOT, "gated_delta_rule_121_b200", "kcp.py")).read()
+    assert "oracle" not in src.replace("oracle_ops", "") and "numpy" not in src

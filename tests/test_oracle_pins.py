@@ -243,3 +243,47 @@ def test_chunk_form_matches_oracle(T, C, g_scale):
     O, S = chunk_forward(q, k, v, g, beta, s0, C=C)
     np.testing.assert_allclose(O, out, rtol=1e-10, atol=1e-10)
     np.testing.assert_allclose(S, fin, rtol=1e-10, atol=1e-10)
+
+
+# -- segment transition and transformed queries (KCP paragraph) -------------
+@pytest.mark.parametrize("T,dk", [(1, 2), (5, 3), (8, 4)])
+def test_transition_is_the_product_of_token_transitions(T, dk):
+    """oracle.transition against explicit products of M_t = (I - b k k^T) Diag(e^g):
+    M = M_T ... M_1 and qhat_t = (M_t ... M_1)^T q_t."""
+    rng = np.random.default_rng(10 * T + dk)
+    q, k, _, g, beta, _ = _rand_chain(T, dk, dk, rng, unit=False)
+    qhat, M = oracle.transition(q[None, :, None], k[None, :, None], g[None, :, None], beta[None, :, None])
+    P = np.eye(dk)
+    for t in range(T):
+        P = (np.eye(dk) - beta[t] * np.outer(k[t], k[t])) @ np.diag(np.exp(g[t])) @ P
+        np.testing.assert_allclose(qhat[0, t, 0], P.T @ q[t], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(M[0, 0], P, rtol=1e-12, atol=1e-12)
+
+
+def test_segment_outputs_are_zero_start_plus_transformed_query_read():
+    """Within a segment entered with state S_in: o_t = o~_t + S_in^T qhat_t and
+    S_end = S~ + M S_in (linearity of the recurrence in the incoming state)."""
+    rng = np.random.default_rng(99)
+    T, dk = 37, 6
+    q, k, v, g, beta, s0 = _rand_chain(T, dk, dk, rng)
+    o_full, s_full = run_chain(q, k, v, g, beta, s0)
+    o_zero, s_zero = run_chain(q, k, v, g, beta, None)
+    qhat, M = oracle.transition(q[None, :, None], k[None, :, None], g[None, :, None], beta[None, :, None])
+    np.testing.assert_allclose(o_zero + qhat[0, :, 0] @ s0, o_full, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(s_zero + M[0, 0] @ s0, s_full, rtol=1e-11, atol=1e-12)
+
+
+def test_composition_over_many_segments():
+    """A sequence cut into 4 pieces: the prefix composition of the pieces'
+    (M, S~) reproduces the states at every cut and the final state."""
+    rng = np.random.default_rng(5)
+    T, dk = 60, 4
+    q, k, v, g, beta, s0 = _rand_chain(T, dk, dk, rng)
+    cuts = [0, 7, 20, 41, 60]
+    S = s0
+    for a, b in zip(cuts[:-1], cuts[1:]):
+        _, s_zero = run_chain(q[a:b], k[a:b], v[a:b], g[a:b], beta[a:b], None)
+        _, M = oracle.transition(q[None, a:b, None], k[None, a:b, None], g[None, a:b, None], beta[None, a:b, None])
+        S = s_zero + M[0, 0] @ S
+        _, s_ref = run_chain(q[:b], k[:b], v[:b], g[:b], beta[:b], s0)
+        np.testing.assert_allclose(S, s_ref, rtol=1e-10, atol=1e-12)
