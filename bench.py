@@ -316,11 +316,16 @@ FLUSH = {"mid": True, "stress": True, "prefill64k": False, "varlen": False}
 def bench_prefill(name, d, dev, stream, peaks, kda, synth, steps, warmup, with_traffic=False, variant=None):
     """Time `steps` forward calls over one workload; returns its JSON object
     and the inputs (for the end-to-end leg).  variant: None (kda_fwd), "cp"
-    (kda_fwd_cp, every sequence split over the SMs) or "ckpt512" (kda_fwd_checkpoints,
-    the state every 512 tokens)."""
+    (kda_fwd_cp, every sequence split over the SMs), "ckpt512" (kda_fwd_checkpoints,
+    the state every 512 tokens) or "gated" (kda_fwd_gated on the raw prologue
+    inputs)."""
     import torch
     spec = workload_spec(name)
-    inp = synth.make_prefill(spec, dev)
+    if variant == "gated":  # raw prologue inputs: unnormalised q, k and bf16 decay logits z (mild decay)
+        inp = synth.make_prologue_prefill(spec, dev)
+        inp["g"] = inp.pop("z")
+    else:
+        inp = synth.make_prefill(spec, dev)
     q, k, v, g, beta, init, cu = (inp[n] for n in ("q", "k", "v", "g", "beta", "init_state", "cu_seqlens"))
     B, T, H, dk = q.shape
     dv = v.shape[-1]
@@ -341,6 +346,11 @@ def bench_prefill(name, d, dev, stream, peaks, kda, synth, steps, warmup, with_t
         def step():
             kda.kda_fwd_cp(q, k, v, g, beta, init, cu, n_seg=n_seg, out=out, final_state=fin, workspace=ws,
                            stream=stream)
+    elif variant == "gated":
+        A_log = inp["A_log"]
+
+        def step():
+            kda.kda_fwd_gated(q, k, v, g, A_log, beta, init, cu, out=out, final_state=fin, workspace=ws, stream=stream)
     elif variant == "ckpt512":
         cap = N * (T // 512) if cu is None else int(((cu[1:] - cu[:-1]).cpu() // 512).sum())
         ck = torch.empty((cap, H, dk, dv), dtype=torch.float32, device=dev)
@@ -364,6 +374,8 @@ def bench_prefill(name, d, dev, stream, peaks, kda, synth, steps, warmup, with_t
         raise RuntimeError(f"{name}: device status {kda.kda_status_string(status)}")
     per_step = d.max(sec) / steps
     bytes_alg = prefill_bytes(th, N * H, dk, dv, q.element_size(), init is not None) + ckpt_bytes
+    if variant == "gated":  # the decay logits are bf16 (2 B) where the log-decays are fp32 (4 B)
+        bytes_alg -= th * dk * (4 - g.element_size())
     flops_alg = prefill_flops(th, dk, dv)
     achieved = bytes_alg / per_step / 1e9
     peak = peaks["hbm_gbs"]
@@ -430,7 +442,8 @@ def run_native(args, d):
         others = {}
         for key, name, steps, variant in (("mid", "mid", 50, None), ("mid_cp", "mid", 50, "cp"),
                                           ("varlen", "varlen", 8, None), ("stress", "stress", 50, None),
-                                          ("prefill64k_ckpt512", "prefill64k", 10, "ckpt512")):
+                                          ("prefill64k_ckpt512", "prefill64k", 10, "ckpt512"),
+                                          ("prefill64k_gated", "prefill64k", 10, "gated")):
             if name == args.workload and variant is None:
                 continue
             res, _ = bench_prefill(name, d, dev, stream, peaks, kda, synth, steps, args.warmup, variant=variant)

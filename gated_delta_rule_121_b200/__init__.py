@@ -13,6 +13,8 @@ Functions mirror the C entry points:
   kda_state_compose(...), kda_output_correct(...)   prefix composition, output correction
   kda_fwd_cp(..., n_seg)                         prefill with every sequence split over the SMs
   kda_decode_step(q, k, v, log_alpha, beta, state, ...)   in-place decode
+  kda_decode_step_gated(q, k, v, z, A_log, beta, state, ...)   the same with the input prologue
+  kda_decode_spec(prev, n_accepted, cur, state, ...)   speculative verification with state replay
   kda_fwd_workspace_size(...), kda_workspace_status(ws), kda_status_string(s)
 and ``kda_fwd_host`` runs kda_fwd on host (pinned) tensors through the C
 entry point of the same name, which copies inputs in and outputs back on the
@@ -95,6 +97,17 @@ def lib() -> ctypes.CDLL:
         L.kda_cp_segments.argtypes = [ctypes.c_int, ctypes.c_int64, ctypes.c_int, ctypes.c_int]
         L.kda_fwd_cp.restype = ctypes.c_int
         L.kda_fwd_cp.argtypes = fwd_args[:-2] + [ctypes.c_int, _vp, ctypes.c_size_t]
+        L.kda_fwd_gated.restype = ctypes.c_int
+        L.kda_fwd_gated.argtypes = [_vp, _vp, _vp, _vp, _fp, ctypes.c_float] + fwd_args[4:]
+        L.kda_decode_step_gated.restype = ctypes.c_int
+        L.kda_decode_step_gated.argtypes = [_vp, _vp, _vp, _vp, _fp, ctypes.c_float, _fp, _fp, _vp, ctypes.c_int,
+                                            ctypes.c_int, ctypes.c_int, ctypes.c_int, _vp, ctypes.c_int]
+        spec = [_vp] * 5 + [_i32p] + [_vp] * 5
+        tail = [_fp, _vp] + [ctypes.c_int] * 6 + [_vp, ctypes.c_int]
+        L.kda_decode_spec.restype = ctypes.c_int
+        L.kda_decode_spec.argtypes = spec + tail
+        L.kda_decode_spec_gated.restype = ctypes.c_int
+        L.kda_decode_spec_gated.argtypes = spec + [_fp, ctypes.c_float] + tail
         L.kda_workspace_status.restype = ctypes.c_int
         L.kda_workspace_status.argtypes = [_vp, _vp]
         _lib = L
@@ -372,6 +385,86 @@ class _FwdTensors(ctypes.Structure):
 
 def _tensors(d):
     return _FwdTensors(*[None if d.get(n) is None else d[n].data_ptr() for n, _ in _FwdTensors._fields_])
+
+
+G_MIN = -5.0  # the model's lower bound of the log decay
+
+
+def kda_fwd_gated(q, k, v, z, A_log, beta, init_state=None, cu_seqlens=None, g_min=G_MIN, out=None,
+                  final_state=None, workspace=None, stream=None):
+    """kda_fwd on the model's raw prologue inputs (include/kda.h,
+    kda_fwd_gated): q, k unnormalised [B,T,H,dk], z the decay logits (dtype of
+    q), A_log [H] fp32.  Returns ``(out, final_state)``."""
+    B, T, H, dk, dv, N = _shapes(q, v, cu_seqlens)
+    for name, t, dtype in (("k", k, q.dtype), ("v", v, q.dtype), ("z", z, q.dtype), ("beta", beta, torch.float32)):
+        if t.dtype != dtype or not t.is_contiguous() or t.device != q.device:
+            raise ValueError(f"{name}: expected contiguous {dtype} on {q.device}")
+    if tuple(z.shape) != tuple(q.shape):
+        raise ValueError("z must be shaped like q")
+    if init_state is not None and (init_state.dtype != torch.float32 or not init_state.is_contiguous()
+                                   or tuple(init_state.shape) != (N, H, dk, dv)):
+        raise ValueError("init_state must be contiguous fp32 [N, H, dk, dv]")
+    if A_log.dtype != torch.float32 or tuple(A_log.shape) != (H,):
+        raise ValueError("A_log must be fp32 [H]")
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    if final_state is None:
+        final_state = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = alloc_workspace(N, B * T, H, dk, dv, q.dtype, q.device)
+    code = lib().kda_fwd_gated(_ptr(q), _ptr(k), _ptr(v), _ptr(z), _ptr(A_log), float(g_min), _ptr(beta),
+                               _ptr(init_state), _ptr(out), _ptr(final_state), N, T, H, dk, dv, _ptr(cu_seqlens),
+                               _stream_ptr(stream), _DT[q.dtype], _ptr(workspace), workspace.numel())
+    _check(code, "kda_fwd_gated")
+    return out, final_state
+
+
+def kda_decode_step_gated(q, k, v, z, A_log, beta, state, g_min=G_MIN, out=None, stream=None):
+    """One decode step on raw prologue inputs (include/kda.h,
+    kda_decode_step_gated): q, k unnormalised, z the decay logits [B,H,dk]
+    (dtype of q), A_log [H] fp32.  ``state`` is updated in place."""
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    if state.dtype != torch.float32 or not state.is_contiguous() or tuple(state.shape) != (B, H, dk, dv):
+        raise ValueError("state must be contiguous fp32 [B, H, dk, dv]")
+    if out is None:
+        out = torch.empty((B, H, dv), dtype=q.dtype, device=q.device)
+    code = lib().kda_decode_step_gated(_ptr(q), _ptr(k), _ptr(v), _ptr(z), _ptr(A_log), float(g_min), _ptr(beta),
+                                       _ptr(state), _ptr(out), B, H, dk, dv, _stream_ptr(stream), _DT[q.dtype])
+    _check(code, "kda_decode_step_gated")
+    return out
+
+
+def kda_decode_spec(prev, n_accepted, cur, state, A_log=None, g_min=G_MIN, out=None, stream=None):
+    """Speculative verification with state replay (include/kda.h,
+    kda_decode_spec): ``prev`` (or None) and ``cur`` are dicts of q, k, v, g,
+    beta shaped [B, W, H, *] (g = the log-decay, or the decay logits when
+    ``A_log`` is given: the gated variant, q and k then unnormalised);
+    ``n_accepted`` int32 [B] on the device.  ``state`` [B,H,dk,dv] is updated
+    to the state after the accepted drafts and the bonus token cur[:, 0].
+    Returns the outputs of ``cur`` [B, W, H, dv]."""
+    B, W, H, dk = cur["q"].shape
+    dv = cur["v"].shape[-1]
+    Wp = 0 if prev is None else prev["q"].shape[1]
+    if state.dtype != torch.float32 or not state.is_contiguous() or tuple(state.shape) != (B, H, dk, dv):
+        raise ValueError("state must be contiguous fp32 [B, H, dk, dv]")
+    for src in (prev, cur):
+        if src is not None:
+            for n in ("q", "k", "v", "g", "beta"):
+                if not src[n].is_contiguous():
+                    raise ValueError(f"{n} must be contiguous")
+    if out is None:
+        out = torch.empty((B, W, H, dv), dtype=cur["q"].dtype, device=cur["q"].device)
+    p = (lambda n: None) if prev is None else (lambda n: _ptr(prev[n]))
+    head = [p("q"), p("k"), p("v"), p("g"), p("beta"), _ptr(n_accepted) if Wp else None,
+            _ptr(cur["q"]), _ptr(cur["k"]), _ptr(cur["v"]), _ptr(cur["g"]), _ptr(cur["beta"])]
+    tail = [_ptr(state), _ptr(out), B, Wp, W, H, dk, dv, _stream_ptr(stream), _DT[cur["q"].dtype]]
+    if A_log is None:
+        code = lib().kda_decode_spec(*head, *tail)
+    else:
+        code = lib().kda_decode_spec_gated(*head, _ptr(A_log), float(g_min), *tail)
+    _check(code, "kda_decode_spec")
+    return out
 
 
 def kda_fwd_host(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None, device="cuda", stream=None,

@@ -13,9 +13,11 @@ cudaError_t launch_fwd_tc_impl(const FwdArgs& a, cudaStream_t s, uint64_t wait_n
                                int32_t* order_ws, const ModeArgs& ma);
 cudaError_t launch_ckpt_base(const int32_t* cu, int N, int interval, int32_t* base, cudaStream_t s);
 cudaError_t launch_compose(const float* trans, const float* s0, const float* init, float* state_in, float* fin,
-                           int R, int N, int H, int dk, int dv, int rank_major, cudaStream_t s);
+                           int R, int N, int H, int dk, int dv, int rank_major, int first_from_init,
+                           cudaStream_t s);
 cudaError_t launch_correct(const float* o32, const float* qhat, const float* s_in, void* out, const int32_t* cu,
-                           int P, int64_t Tper, int64_t Ttot, int H, int dk, int dv, bool bf16, cudaStream_t s);
+                           int P, int64_t Tper, int64_t Ttot, int H, int dk, int dv, bool bf16, int skip_every,
+                           cudaStream_t s);
 cudaError_t launch_segment_cu(const int32_t* cu, int64_t Tper, int N, int R, int32_t* seg_cu, cudaStream_t s);
 int fwd_tc_debug_floats();
 }  // namespace kda
@@ -168,6 +170,67 @@ kda_status_t kda_decode_step(const void* q, const void* k, const void* v, const 
   return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
+kda_status_t kda_decode_step_gated(const void* q, const void* k, const void* v, const void* z, const float* A_log,
+                                   float g_min, const float* beta, float* state, void* out, int B, int H, int dk,
+                                   int dv, void* stream, kda_dtype_t dt) {
+  if (B < 0 || H <= 0) return KDA_ERR_INVALID_ARG;
+  if (dt != KDA_F32 && dt != KDA_BF16) return KDA_ERR_INVALID_ARG;
+  if (!dim_ok(dk) || !dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
+  const void* req[] = {q, k, v, z, A_log, beta, state, out};
+  for (const void* p : req)
+    if (!p || !aligned16(p)) return KDA_ERR_INVALID_ARG;
+  if ((int64_t)B * H > (int64_t)INT32_MAX) return KDA_ERR_UNSUPPORTED;
+  if (B == 0) return KDA_OK;
+  cudaError_t e = kda::launch_decode_gated(q, k, v, z, A_log, g_min, beta, state, out, B, H, dk, dv,
+                                           dt == KDA_BF16, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+static kda_status_t spec_impl(const void* qp, const void* kp, const void* vp, const void* gp, const float* bp,
+                              const int32_t* n_accepted, const void* q, const void* k, const void* v, const void* g,
+                              const float* beta, const float* A_log, float g_min, float* state, void* out, int B,
+                              int Wp, int W, int H, int dk, int dv, void* stream, kda_dtype_t dt) {
+  if (B < 0 || H <= 0 || Wp < 0 || W < 0) return KDA_ERR_INVALID_ARG;
+  if (Wp + W > KDA_SPEC_MAX_TOKENS) return KDA_ERR_UNSUPPORTED;
+  if (dt != KDA_F32 && dt != KDA_BF16) return KDA_ERR_INVALID_ARG;
+  if (!dim_ok(dk) || !dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
+  if (!state || !aligned16(state)) return KDA_ERR_INVALID_ARG;
+  if (W > 0) {
+    const void* req[] = {q, k, v, g, beta, out};
+    for (const void* p : req)
+      if (!p || !aligned16(p)) return KDA_ERR_INVALID_ARG;
+  }
+  if (Wp > 0) {
+    const void* req[] = {qp, kp, vp, gp, bp, n_accepted};
+    for (const void* p : req)
+      if (!p || !aligned16(p)) return KDA_ERR_INVALID_ARG;
+  }
+  if ((int64_t)B * H > (int64_t)INT32_MAX) return KDA_ERR_UNSUPPORTED;
+  if (B == 0) return KDA_OK;
+  cudaError_t e = kda::launch_spec(qp, kp, vp, gp, bp, Wp > 0 ? n_accepted : nullptr, q, k, v, g, beta, state, out,
+                                   B, Wp, W, H, dk, dv, dt == KDA_BF16, A_log, g_min,
+                                   reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+kda_status_t kda_decode_spec(const void* q_prev, const void* k_prev, const void* v_prev, const float* log_alpha_prev,
+                             const float* beta_prev, const int32_t* n_accepted, const void* q, const void* k,
+                             const void* v, const float* log_alpha, const float* beta, float* state, void* out,
+                             int B, int Wp, int W, int H, int dk, int dv, void* stream, kda_dtype_t dt) {
+  return spec_impl(q_prev, k_prev, v_prev, log_alpha_prev, beta_prev, n_accepted, q, k, v, log_alpha, beta, nullptr,
+                   0.f, state, out, B, Wp, W, H, dk, dv, stream, dt);
+}
+
+kda_status_t kda_decode_spec_gated(const void* q_prev, const void* k_prev, const void* v_prev, const void* z_prev,
+                                   const float* beta_prev, const int32_t* n_accepted, const void* q, const void* k,
+                                   const void* v, const void* z, const float* beta, const float* A_log, float g_min,
+                                   float* state, void* out, int B, int Wp, int W, int H, int dk, int dv,
+                                   void* stream, kda_dtype_t dt) {
+  if (!A_log || !aligned16(A_log)) return KDA_ERR_INVALID_ARG;
+  return spec_impl(q_prev, k_prev, v_prev, z_prev, beta_prev, n_accepted, q, k, v, z, beta, A_log, g_min, state,
+                   out, B, Wp, W, H, dk, dv, stream, dt);
+}
+
 kda_status_t kda_workspace_status(const void* workspace, void* stream) {
   if (!workspace || !aligned16(workspace)) return KDA_ERR_INVALID_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -175,6 +238,22 @@ kda_status_t kda_workspace_status(const void* workspace, void* stream) {
   if (cudaMemcpyAsync(&h, workspace, sizeof(h), cudaMemcpyDeviceToHost, s) != cudaSuccess) return KDA_ERR_CUDA;
   if (cudaStreamSynchronize(s) != cudaSuccess) return KDA_ERR_CUDA;
   return static_cast<kda_status_t>(h.code);
+}
+
+// ---- the model's input prologue fused into the prefill ----
+kda_status_t kda_fwd_gated(const void* q, const void* k, const void* v, const void* z, const float* A_log,
+                           float g_min, const float* beta, const float* init_state, void* out, float* final_state,
+                           int B, int64_t T, int H, int dk, int dv, const int32_t* cu_seqlens, void* stream,
+                           kda_dtype_t dt, void* workspace, size_t workspace_bytes) {
+  if (!A_log || !aligned16(A_log)) return KDA_ERR_INVALID_ARG;
+  kda::ModeArgs ma;
+  ma.mode = kda::MODE_GATED;
+  ma.A_log = A_log;
+  ma.g_min = g_min;
+  // The decay logits travel in the log-decay slot; validation checks them
+  // as one more token tensor.
+  return fwd_impl(q, k, v, static_cast<const float*>(z), beta, init_state, out, final_state, B, T, H, dk, dv,
+                  cu_seqlens, stream, dt, workspace, workspace_bytes, nullptr, 2000000000ull, 0, ma);
 }
 
 // ---- interval checkpoints (prefix-cache states) ----
@@ -245,7 +324,7 @@ kda_status_t kda_state_compose(const float* transition, const float* state_zero,
     if (!aligned16(p)) return KDA_ERR_INVALID_ARG;
   if (N == 0) return KDA_OK;
   cudaError_t e = kda::launch_compose(transition, state_zero, init_state, state_in, final_state, R, N, H, dk, dv,
-                                      rank_major ? 1 : 0, reinterpret_cast<cudaStream_t>(stream));
+                                      rank_major ? 1 : 0, 0, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
@@ -262,7 +341,7 @@ kda_status_t kda_output_correct(const float* out_zero, const float* qhat, const 
     if (!aligned16(p)) return KDA_ERR_INVALID_ARG;
   if (tokens == 0 || B == 0) return KDA_OK;
   cudaError_t e = kda::launch_correct(out_zero, qhat, state_in, out, cu_seqlens, B, cu_seqlens ? 0 : T, tokens, H,
-                                      dk, dv, dt == KDA_BF16, reinterpret_cast<cudaStream_t>(stream));
+                                      dk, dv, dt == KDA_BF16, 0, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
@@ -343,7 +422,8 @@ kda_status_t kda_fwd_cp(const void* q, const void* k, const void* v, const float
   ma.o32 = o32;
   ma.qhat32 = qhat;
   ma.trans = tr;
-  kda::FwdArgs a{q, k, v, log_alpha, beta, nullptr, nullptr, s0, seg_cu, P, tokens, H, dk, dv,
+  ma.seg_per_seq = n_seg;  // first segments run from init_state into `out` directly
+  kda::FwdArgs a{q, k, v, log_alpha, beta, init_state, out, s0, seg_cu, P, tokens, H, dk, dv,
                  reinterpret_cast<kda::DeviceStatus*>(ws), nullptr};
   cudaError_t e;
   if (kda::fwd_tc_supported(dk, dv, dt == KDA_BF16) && tokens > 0)
@@ -351,9 +431,9 @@ kda_status_t kda_fwd_cp(const void* q, const void* k, const void* v, const float
   else
     e = kda::launch_fwd_simt(a, dt == KDA_BF16, s, ma);
   if (e != cudaSuccess) return KDA_ERR_CUDA;
-  e = kda::launch_compose(tr, s0, init_state, s_in, final_state, n_seg, B, H, dk, dv, 0, s);
+  e = kda::launch_compose(tr, s0, init_state, s_in, final_state, n_seg, B, H, dk, dv, 0, 1, s);
   if (e != cudaSuccess) return KDA_ERR_CUDA;
-  e = kda::launch_correct(o32, qhat, s_in, out, seg_cu, P, 0, tokens, H, dk, dv, dt == KDA_BF16, s);
+  e = kda::launch_correct(o32, qhat, s_in, out, seg_cu, P, 0, tokens, H, dk, dv, dt == KDA_BF16, n_seg, s);
   return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 

@@ -16,6 +16,11 @@
 // loads and stores use streaming cache hints, and the two cross-row
 // reductions go through shared memory.  The path is bound by HBM bandwidth:
 // 2 * dk * dv * 4 bytes of state traffic per head.
+//
+// GATED: the token's inputs are those of the model's prologue (q and k
+// L2-normalised here; the decay from the decay logits, g = g_min *
+// sigmoid(exp(A_h) z), see kda_gate.cuh).
+#include "kda_gate.cuh"
 #include "kda_internal.cuh"
 
 namespace kda {
@@ -29,11 +34,11 @@ struct DecodeShape {
   static constexpr int NT = COLQ * RG;                                   // threads per block
 };
 
-template <int DK, int DV, typename IO>
+template <int DK, int DV, typename IO, bool GATED>
 __global__ void __launch_bounds__(DecodeShape<DK, DV>::NT)
     kda_decode_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO* __restrict__ v,
-                      const float* __restrict__ g, const float* __restrict__ beta, float* __restrict__ state,
-                      IO* __restrict__ out) {
+                      const void* __restrict__ g, const float* __restrict__ beta, float* __restrict__ state,
+                      IO* __restrict__ out, const float* __restrict__ A_log, float g_min, int H) {
   using Sh = DecodeShape<DK, DV>;
   constexpr int COLQ = Sh::COLQ, RG = Sh::RG, ROWS = Sh::ROWS, NT = Sh::NT;
   __shared__ float s_k[DK], s_q[DK], s_a[DK];
@@ -53,9 +58,37 @@ __global__ void __launch_bounds__(DecodeShape<DK, DV>::NT)
   for (int i = tid; i < DK; i += NT) {
     s_k[i] = to_f32(k[bh * DK + i]);
     s_q[i] = to_f32(q[bh * DK + i]);
-    s_a[i] = __expf(g[bh * DK + i]);
+    if constexpr (GATED)
+      s_a[i] = __expf(gate_log_decay(to_f32(static_cast<const IO*>(g)[bh * DK + i]), A_log[bh % H], g_min));
+    else
+      s_a[i] = __expf(static_cast<const float*>(g)[bh * DK + i]);
   }
   __syncthreads();
+  if constexpr (GATED) {  // L2-normalise q and k in place (one warp), then the block uses them
+    __shared__ float s_sc[2];
+    if (tid < 32) {
+      float qq = 0.f, kk = 0.f;
+      for (int i = tid; i < DK; i += 32) {
+        qq += s_q[i] * s_q[i];
+        kk += s_k[i] * s_k[i];
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        qq += __shfl_xor_sync(0xffffffffu, qq, o);
+        kk += __shfl_xor_sync(0xffffffffu, kk, o);
+      }
+      if (tid == 0) {
+        s_sc[0] = l2norm_scale(qq);
+        s_sc[1] = l2norm_scale(kk);
+      }
+    }
+    __syncthreads();
+    for (int i = tid; i < DK; i += NT) {
+      s_q[i] *= s_sc[0];
+      s_k[i] *= s_sc[1];
+    }
+    __syncthreads();
+  }
   if (tid < 32) {
     float acc = 0.f;
     for (int i = tid; i < DK; i += 32) acc += s_q[i] * s_k[i];
@@ -106,30 +139,46 @@ __global__ void __launch_bounds__(DecodeShape<DK, DV>::NT)
   }
 }
 
-template <int DK, int DV>
-cudaError_t launch_dims(const void* q, const void* k, const void* v, const float* g, const float* beta,
-                        float* state, void* out, int B, int H, bool bf16, cudaStream_t s) {
+template <int DK, int DV, bool GATED>
+cudaError_t launch_dims(const void* q, const void* k, const void* v, const void* g, const float* beta,
+                        float* state, void* out, int B, int H, bool bf16, const float* A_log, float g_min,
+                        cudaStream_t s) {
   const unsigned blocks = (unsigned)((int64_t)B * H);
   constexpr int NT = DecodeShape<DK, DV>::NT;
   if (bf16) {
     using T = __nv_bfloat16;
-    kda_decode_kernel<DK, DV, T><<<blocks, NT, 0, s>>>((const T*)q, (const T*)k, (const T*)v, g, beta, state,
-                                                      (T*)out);
+    kda_decode_kernel<DK, DV, T, GATED><<<blocks, NT, 0, s>>>((const T*)q, (const T*)k, (const T*)v, g, beta,
+                                                             state, (T*)out, A_log, g_min, H);
   } else {
-    kda_decode_kernel<DK, DV, float><<<blocks, NT, 0, s>>>((const float*)q, (const float*)k, (const float*)v,
-                                                          g, beta, state, (float*)out);
+    kda_decode_kernel<DK, DV, float, GATED><<<blocks, NT, 0, s>>>((const float*)q, (const float*)k,
+                                                                 (const float*)v, g, beta, state, (float*)out,
+                                                                 A_log, g_min, H);
   }
   return cudaGetLastError();
 }
 
-template <int DK>
-cudaError_t launch_dv(const void* q, const void* k, const void* v, const float* g, const float* beta,
-                      float* state, void* out, int B, int H, int dv, bool bf16, cudaStream_t s) {
+template <int DK, bool GATED>
+cudaError_t launch_dv(const void* q, const void* k, const void* v, const void* g, const float* beta,
+                      float* state, void* out, int B, int H, int dv, bool bf16, const float* A_log, float g_min,
+                      cudaStream_t s) {
   switch (dv) {
-    case 16: return launch_dims<DK, 16>(q, k, v, g, beta, state, out, B, H, bf16, s);
-    case 32: return launch_dims<DK, 32>(q, k, v, g, beta, state, out, B, H, bf16, s);
-    case 64: return launch_dims<DK, 64>(q, k, v, g, beta, state, out, B, H, bf16, s);
-    case 128: return launch_dims<DK, 128>(q, k, v, g, beta, state, out, B, H, bf16, s);
+    case 16: return launch_dims<DK, 16, GATED>(q, k, v, g, beta, state, out, B, H, bf16, A_log, g_min, s);
+    case 32: return launch_dims<DK, 32, GATED>(q, k, v, g, beta, state, out, B, H, bf16, A_log, g_min, s);
+    case 64: return launch_dims<DK, 64, GATED>(q, k, v, g, beta, state, out, B, H, bf16, A_log, g_min, s);
+    case 128: return launch_dims<DK, 128, GATED>(q, k, v, g, beta, state, out, B, H, bf16, A_log, g_min, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+template <bool GATED>
+cudaError_t launch_decode_g(const void* q, const void* k, const void* v, const void* g, const float* beta,
+                            float* state, void* out, int B, int H, int dk, int dv, bool bf16, const float* A_log,
+                            float g_min, cudaStream_t s) {
+  switch (dk) {
+    case 16: return launch_dv<16, GATED>(q, k, v, g, beta, state, out, B, H, dv, bf16, A_log, g_min, s);
+    case 32: return launch_dv<32, GATED>(q, k, v, g, beta, state, out, B, H, dv, bf16, A_log, g_min, s);
+    case 64: return launch_dv<64, GATED>(q, k, v, g, beta, state, out, B, H, dv, bf16, A_log, g_min, s);
+    case 128: return launch_dv<128, GATED>(q, k, v, g, beta, state, out, B, H, dv, bf16, A_log, g_min, s);
   }
   return cudaErrorInvalidValue;
 }
@@ -138,13 +187,13 @@ cudaError_t launch_dv(const void* q, const void* k, const void* v, const float* 
 
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const float* g, const float* beta,
                           float* state, void* out, int B, int H, int dk, int dv, bool bf16, cudaStream_t s) {
-  switch (dk) {
-    case 16: return launch_dv<16>(q, k, v, g, beta, state, out, B, H, dv, bf16, s);
-    case 32: return launch_dv<32>(q, k, v, g, beta, state, out, B, H, dv, bf16, s);
-    case 64: return launch_dv<64>(q, k, v, g, beta, state, out, B, H, dv, bf16, s);
-    case 128: return launch_dv<128>(q, k, v, g, beta, state, out, B, H, dv, bf16, s);
-  }
-  return cudaErrorInvalidValue;
+  return launch_decode_g<false>(q, k, v, g, beta, state, out, B, H, dk, dv, bf16, nullptr, 0.f, s);
+}
+
+cudaError_t launch_decode_gated(const void* q, const void* k, const void* v, const void* z, const float* A_log,
+                                float g_min, const float* beta, float* state, void* out, int B, int H, int dk,
+                                int dv, bool bf16, cudaStream_t s) {
+  return launch_decode_g<true>(q, k, v, z, beta, state, out, B, H, dk, dv, bf16, A_log, g_min, s);
 }
 
 }  // namespace kda

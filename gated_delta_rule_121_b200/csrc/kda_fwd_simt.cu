@@ -15,6 +15,7 @@
 // rows (u and o) are 4-lane shuffles inside the warp, so the token loop has
 // no block barrier; barriers appear only when a chunk of TOK tokens is
 // staged in shared memory.
+#include "kda_gate.cuh"
 #include "kda_internal.cuh"
 
 namespace kda {
@@ -26,7 +27,8 @@ constexpr int TOK = 16;  // tokens staged per shared-memory round
 // tokens of each sequence; MODE_SEG runs every (sequence, head, column block)
 // twice, the second time (blocks from `units` on) as the transition run:
 // values taken as zero, identity start, outputs and final state to qhat32
-// and trans (dk == dv).
+// and trans (dk == dv); MODE_GATED takes the decay logits in `g` (dtype IO)
+// and normalises q and k per token (the model's prologue, kda_gate.cuh).
 template <int DK, int DVB, typename IO, int MODE>
 __global__ void __launch_bounds__(DVB * 4)
     kda_fwd_simt_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO* __restrict__ v,
@@ -45,12 +47,16 @@ __global__ void __launch_bounds__(DVB * 4)
   if constexpr (MODE == MODE_SEG) {
     trans = bid >= units;
     if (trans) bid -= units;
-    init = nullptr;
     if (trans) fin = ma.trans;
   }
   const int blk = bid % nblk;
   const int h = (bid / nblk) % H;
   const int n = bid / (nblk * H);
+  // MODE_SEG: a sequence's first segment runs from its initial state with
+  // ordinary outputs and needs no transition run.
+  const bool first = MODE == MODE_SEG && ma.seg_per_seq > 0 && n % ma.seg_per_seq == 0;
+  if (first && trans) return;
+  if (MODE == MODE_SEG && !first) init = nullptr;
   int64_t t0, L;
   if (cu) {
     t0 = cu[n];
@@ -64,12 +70,13 @@ __global__ void __launch_bounds__(DVB * 4)
   const int jl = warp * 8 + jc;       // column within the block
   const int j = blk * DVB + jl;       // column of S / v / o
   const int64_t sbase = ((int64_t)n * H + h) * DK * dv;
+  const int64_t ibase = first ? ((int64_t)(n / ma.seg_per_seq) * H + h) * DK * dv : sbase;
 
   float s[R];
 #pragma unroll
   for (int m = 0; m < R; ++m) {
-    s[m] = init ? init[sbase + (int64_t)(4 * m + rg) * dv + j] : 0.f;
-    if constexpr (MODE == MODE_SEG) s[m] = (trans && 4 * m + rg == j) ? 1.f : 0.f;
+    s[m] = init ? init[ibase + (int64_t)(4 * m + rg) * dv + j] : 0.f;
+    if (MODE == MODE_SEG && !first) s[m] = (trans && 4 * m + rg == j) ? 1.f : 0.f;
   }
   int64_t ckpt0 = 0;
   if constexpr (MODE == MODE_CKPT)
@@ -85,7 +92,10 @@ __global__ void __launch_bounds__(DVB * 4)
         const int64_t row = ((t0 + c0 + r) * H + h) * DK + i;
         kk = to_f32(k[row]);
         qq = to_f32(q[row]);
-        aa = __expf(g[row]);
+        if constexpr (MODE == MODE_GATED)
+          aa = __expf(gate_log_decay(to_f32(reinterpret_cast<const IO*>(g)[row]), ma.A_log[h], ma.g_min));
+        else
+          aa = __expf(g[row]);
       }
       s_k[r][i] = kk; s_q[r][i] = qq; s_a[r][i] = aa;
     }
@@ -95,6 +105,26 @@ __global__ void __launch_bounds__(DVB * 4)
     }
     if (tid < TOK) s_b[tid] = tid < nt ? beta[(t0 + c0 + tid) * H + h] : 0.f;
     __syncthreads();
+    if constexpr (MODE == MODE_GATED) {  // L2-normalise the staged q and k rows, one warp per token
+      for (int r = warp; r < nt; r += NT / 32) {
+        float sq = 0.f, sk = 0.f;
+        for (int i = lane; i < DK; i += 32) {
+          sq += s_q[r][i] * s_q[r][i];
+          sk += s_k[r][i] * s_k[r][i];
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          sq += __shfl_xor_sync(0xffffffffu, sq, o);
+          sk += __shfl_xor_sync(0xffffffffu, sk, o);
+        }
+        const float fq = l2norm_scale(sq), fk = l2norm_scale(sk);
+        for (int i = lane; i < DK; i += 32) {
+          s_q[r][i] *= fq;
+          s_k[r][i] *= fk;
+        }
+      }
+      __syncthreads();
+    }
 
     for (int r = 0; r < nt; ++r) {
       float pu = 0.f;
@@ -135,7 +165,7 @@ __global__ void __launch_bounds__(DVB * 4)
     for (int e = tid; e < nt * DVB; e += NT) {
       const int r = e / DVB, c = e % DVB;
       const int64_t o = ((t0 + c0 + r) * H + h) * dv + blk * DVB + c;
-      if constexpr (MODE == MODE_SEG)
+      if (MODE == MODE_SEG && !first)
         (trans ? ma.qhat32 : ma.o32)[o] = s_o[r][c];
       else
         out[o] = from_f32<IO>(s_o[r][c]);
@@ -186,6 +216,7 @@ cudaError_t launch_fwd_simt(const FwdArgs& a, bool bf16, cudaStream_t s, const M
   switch (ma.mode) {
     case MODE_CKPT: return launch_mode<MODE_CKPT>(a, bf16, s, ma);
     case MODE_SEG: return launch_mode<MODE_SEG>(a, bf16, s, ma);
+    case MODE_GATED: return launch_mode<MODE_GATED>(a, bf16, s, ma);
     default: return launch_mode<MODE_PLAIN>(a, bf16, s, ma);
   }
 }

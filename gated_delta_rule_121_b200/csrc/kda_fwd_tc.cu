@@ -47,8 +47,16 @@
 // column); every other operand is a 128-byte-swizzled fp16 tile in shared
 // memory.  Q, K, V arrive by TMA two chunks ahead.  Each group has one
 // elected thread that issues its UMMAs; mbarriers carry the hand-offs.
+//
+// MODE_GATED takes the model's raw prologue inputs instead (Kimi K3 digest,
+// "Kimi Delta Attention" section: q, k L2-normalised, decay logits with a
+// per-head scale; "Bounded decay" section: g = g_min sigmoid(exp(A_h) z)).
+// The front group maps z to g while it forms the decay prefix and folds the
+// per-row normalisation factors 1/|q_r|, 1/|k_r| into the operand scaling
+// (fp32, before the fp16 rounding), so no normalised copy of q or k exists.
 #include <cuda.h>
 
+#include "kda_gate.cuh"
 #include "kda_internal.cuh"
 #include "sm100_ptx.cuh"
 
@@ -62,6 +70,13 @@ constexpr float LOG2E = 1.4426950408889634f;
 constexpr float FAST_MIN_LOG2 = -10.0f;  // chunk-total decay floor (log2) for the tensor-core Gram
 constexpr float F16_SAFE = 60000.0f;     // |x| above this would overflow fp16 operands
 constexpr uint64_t WAIT_NS = 2000000000ull;
+// Start value of a transition run (MODE_SEG): the identity times 2^12.  The
+// run is linear in its start (its values are zero), so its outputs and final
+// state are scaled back by 2^-12 exactly; meanwhile the fp16 operand copies
+// of the decaying state (entries of the transition, at most 1 in magnitude
+// for normalised keys) stay clear of the fp16 subnormal range down to ~1e-8.
+constexpr float TRANS_SCALE = 4096.0f;
+constexpr float TRANS_UNSCALE = 1.0f / 4096.0f;
 
 // ---- shared memory map (bytes from a 1024-aligned base)
 constexpr uint32_t STAGE_BYTES = 49152;  // [Q;K] 32 KB (per 64-channel half: Q rows, then K rows) + V 16 KB
@@ -76,7 +91,7 @@ constexpr uint32_t SM_T10 = SM_X + 4096;     // T_10 fp32 [32][32]            4 
 constexpr uint32_t SM_TP = SM_X;             // T' fp16 [64][64] over X, T_10  8 KB
 constexpr uint32_t SM_OST = SM_T10 + 4096 + 4096;  // O staging bf16 [64][128] 16 KB (1024-aligned)
 constexpr uint32_t SM_MISC = SM_OST + 16384;
-constexpr uint32_t MISC_BYTES = 8192;
+constexpr uint32_t MISC_BYTES = 8704;
 constexpr uint32_t SMEM_BYTES = SM_MISC + MISC_BYTES + 1024;
 
 // misc layout
@@ -95,7 +110,9 @@ constexpr uint32_t MS_BETA = 256;    // [2][64] fp32
 constexpr uint32_t MS_GC = 768;      // [2][128] fp32: exp(G_C)
 constexpr uint32_t MS_RED = 1792;    // [8][128] fp32 log2 sums
 constexpr uint32_t MS_PAIRS = 5888;  // [64][8] fp32: P, A of the pairs inside 4-row groups (general chunks)
-constexpr uint32_t MS_END = 7936;
+constexpr uint32_t MS_RQK = 7936;    // [16][8] fp32: 1/|q_r|, 1/|k_r| of each row group's 4 rows (MODE_GATED)
+constexpr uint32_t MS_GATE = 8448;   // [2] fp32: -exp(A_h) log2(e), g_min log2(e) (MODE_GATED)
+constexpr uint32_t MS_END = 8464;
 static_assert(NUM_BARS * 8 <= MS_TMEM, "barrier area");
 static_assert(MS_END <= MISC_BYTES, "misc area");
 
@@ -249,8 +266,63 @@ struct Ctx {
   long long* tdbg;  // chain-0 phase timestamps or nullptr
   long long tstart;
   bool trans;       // MODE_SEG: this block runs the transition (zero values, identity start)
+  bool first;       // MODE_SEG: first segment of a sequence, run from its initial state
   int64_t ckpt0;    // MODE_CKPT: checkpoint slot of this sequence's first interval
 };
+
+// MODE_GATED: per-token log2-decays of 8 channels from their bf16 decay
+// logits: g log2(e) = g_min log2(e) / (1 + 2^(-exp(A_h) log2(e) z)).
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ F8 gate_log2_8(uint4 u, float gz, float gmin2) {
+  F8 z = bf16x8_to_f32(u);
+  float* e = &z.a.x;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) e[i] = gmin2 * rcp_approx(1.f + ex2(gz * e[i]));
+  return z;
+}
+// MODE_GATED: 1/|x_r| for this thread's 4 rows of the raw q and k tiles (its 8
+// channels, summed over the 16 threads of the row group), stored in the row
+// group's entry of `tab` ([rg][0..3] = q, [rg][4..7] = k) for the group's
+// threads to read where they scale the rows (the values do not stay in
+// registers across the Gram).
+__device__ __forceinline__ void row_norms(const uint8_t* qb, const uint8_t* kb, int rg, int cc, float* tab) {
+  float rq[4], rk[4];
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    const uint32_t o = sw128_off(4 * rg + m, cc);
+    const F8 a = bf16x8_to_f32(*reinterpret_cast<const uint4*>(qb + o));
+    const F8 b = bf16x8_to_f32(*reinterpret_cast<const uint4*>(kb + o));
+    const F8 a2 = mul8(a, a), b2 = mul8(b, b);
+    rq[m] = ((a2.a.x + a2.a.y) + (a2.a.z + a2.a.w)) + ((a2.b.x + a2.b.y) + (a2.b.z + a2.b.w));
+    rk[m] = ((b2.a.x + b2.a.y) + (b2.a.z + b2.a.w)) + ((b2.b.x + b2.b.y) + (b2.b.z + b2.b.w));
+  }
+#pragma unroll
+  for (int o = 1; o < 16; o <<= 1) {
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      rq[m] += __shfl_xor_sync(0xffffffffu, rq[m], o);
+      rk[m] += __shfl_xor_sync(0xffffffffu, rk[m], o);
+    }
+  }
+  if ((threadIdx.x & 15) == 0) {
+    *reinterpret_cast<float4*>(tab + rg * 8) =
+        make_float4(l2norm_scale(rq[0]), l2norm_scale(rq[1]), l2norm_scale(rq[2]), l2norm_scale(rq[3]));
+    *reinterpret_cast<float4*>(tab + rg * 8 + 4) =
+        make_float4(l2norm_scale(rk[0]), l2norm_scale(rk[1]), l2norm_scale(rk[2]), l2norm_scale(rk[3]));
+  }
+  __syncwarp();  // a row group is half a warp
+}
+// This row group's factors from the table.
+__device__ __forceinline__ void row_factors(const uint8_t* sm, int rg, float (&rq)[4], float (&rk)[4]) {
+  const float* tab = reinterpret_cast<const float*>(sm + SM_MISC + MS_RQK) + rg * 8;
+  const float4 a = *reinterpret_cast<const float4*>(tab), b = *reinterpret_cast<const float4*>(tab + 4);
+  rq[0] = a.x; rq[1] = a.y; rq[2] = a.z; rq[3] = a.w;
+  rk[0] = b.x; rk[1] = b.y; rk[2] = b.z; rk[3] = b.w;
+}
 
 // Phase timestamp (elected thread only) for the timing dump.
 __device__ __forceinline__ void tmark(const Ctx& x, int c, int ev) {
@@ -359,6 +431,7 @@ __device__ __forceinline__ void store_pa(uint8_t* sm, int b2, int ti, int chh, c
 // 64-channel halves are the A tile and KX[b2] (both released: AFREE and BUF
 // were waited for); the row-group end values of G (the references) are
 // staged in the P tile.
+template <int MODE>
 __device__ __forceinline__ bool level_gram(const Ctx& x, int c, int b2, const F8 (&gv)[4], int& g1_ph) {
   const int f = threadIdx.x - FRONT0;
   const int wq = f >> 5, lane = f & 31, lq = wq & 3, chh = wq >> 2;
@@ -395,8 +468,14 @@ __device__ __forceinline__ bool level_gram(const Ctx& x, int c, int b2, const F8
       const uint32_t o = sw128_off(4 * rg + m, cc);
       dr = add8(dr, gv[m]);
       const F8 e = ex2_8(later ? dr : sub8(f8(0.f), dr));
-      st_f16x8(lt + o, mul8(bf16x8_to_f32(*reinterpret_cast<const uint4*>(qb + o)), e));
-      st_f16x8(lt + 8192 + o, mul8(bf16x8_to_f32(*reinterpret_cast<const uint4*>(kb + o)), e));
+      if constexpr (MODE == MODE_GATED) {  // with the row's normalisation factors
+        const float* tab = reinterpret_cast<const float*>(sm + SM_MISC + MS_RQK) + rg * 8;
+        st_f16x8(lt + o, mul8(bf16x8_to_f32(*reinterpret_cast<const uint4*>(qb + o)), mul8(e, f8(tab[m]))));
+        st_f16x8(lt + 8192 + o, mul8(bf16x8_to_f32(*reinterpret_cast<const uint4*>(kb + o)), mul8(e, f8(tab[4 + m]))));
+      } else {
+        st_f16x8(lt + o, mul8(bf16x8_to_f32(*reinterpret_cast<const uint4*>(qb + o)), e));
+        st_f16x8(lt + 8192 + o, mul8(bf16x8_to_f32(*reinterpret_cast<const uint4*>(kb + o)), e));
+      }
     }
     fence_proxy_async_smem();
   };
@@ -444,6 +523,18 @@ __device__ __forceinline__ bool level_gram(const Ctx& x, int c, int b2, const F8
           }
         }
       }
+    }
+    if constexpr (MODE == MODE_GATED) {  // the pairs' normalisation factors
+      float rq[4], rk[4];
+      row_factors(sm, rg, rq, rk);
+      int ip = 0, ia = 0;
+#pragma unroll
+      for (int s = 0; s < 4; ++s)
+#pragma unroll
+        for (int rr = s; rr < 4; ++rr) {
+          pv[ip++] *= rq[rr] * rk[s];
+          if (rr > s) av[ia++] *= rk[rr] * rk[s];
+        }
     }
     // Sum over the 16 threads of the row group (lanes differing in bits 0-3).
 #pragma unroll
@@ -574,7 +665,17 @@ __device__ __forceinline__ void front_group(const Ctx& x, const float* __restric
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
       const int r = 4 * rg + m;
-      gv[m] = r < valid ? ldg8(g + ((tok0 + r) * H + x.h) * D + ch0, g32) : f8(0.f);
+      if constexpr (MODE == MODE_GATED) {
+        // bf16 decay logits mapped to log2-decays at once; rows past the end
+        // get -inf, whose gate is exactly 0
+        const uint4 u = r < valid ? __ldg(reinterpret_cast<const uint4*>(
+                                        reinterpret_cast<const __nv_bfloat16*>(g) + ((tok0 + r) * H + x.h) * D + ch0))
+                                  : make_uint4(0xFF80FF80u, 0xFF80FF80u, 0xFF80FF80u, 0xFF80FF80u);
+        const float* gc = reinterpret_cast<const float*>(x.sm + SM_MISC + MS_GATE);
+        gv[m] = gate_log2_8(u, gc[0], gc[1]);
+      } else {
+        gv[m] = r < valid ? ldg8(g + ((tok0 + r) * H + x.h) * D + ch0, g32) : f8(0.f);
+      }
     }
     bv = (f < CH && f < valid) ? __ldg(beta + (tok0 + f) * H + x.h) : 0.f;
   };
@@ -611,7 +712,7 @@ __device__ __forceinline__ void front_group(const Ctx& x, const float* __restric
     const F8 l2e = f8(LOG2E);
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
-      gv[m] = mul8(gv[m], l2e);
+      if constexpr (MODE != MODE_GATED) gv[m] = mul8(gv[m], l2e);  // gated rows are in log2 units already
       acc = add8(acc, gv[m]);
     }
     F8 other;  // the other row group of this warp (lane ^ 16)
@@ -681,8 +782,9 @@ __device__ __forceinline__ void front_group(const Ctx& x, const float* __restric
         }
       }
     }
+    if constexpr (MODE == MODE_GATED) row_norms(qb, kb, rg, cc, reinterpret_cast<float*>(sm + SM_MISC + MS_RQK));
     if (!fast) {
-      if (!level_gram(x, c, b2, gv, g1_ph)) break;
+      if (!level_gram<MODE>(x, c, b2, gv, g1_ph)) break;
       // G_C again from the warp sums (the same additions in the same order),
       // so that it is not held in registers across the Gram.
       tot = f8(0.f);
@@ -696,6 +798,8 @@ __device__ __forceinline__ void front_group(const Ctx& x, const float* __restric
     // fast chunks, 0 otherwise), H = e^{G_C - G_r}.  QE, KE and V (fp16) go
     // in place; KH goes to KX[b2] once the scan of chunk c-2 has released it.
     uint4 kraw[4];  // raw K rows, kept for KH
+    float rq[4] = {1.f, 1.f, 1.f, 1.f}, rk[4] = {1.f, 1.f, 1.f, 1.f};
+    if constexpr (MODE == MODE_GATED) row_factors(sm, rg, rq, rk);
     {
       F8 gr = f8(0.f);
 #pragma unroll
@@ -714,8 +818,13 @@ __device__ __forceinline__ void front_group(const Ctx& x, const float* __restric
           const uint32_t o = sw128_off(4 * rg + m, cc);
           gr = add8(gr, gv[m]);
           const F8 fw = ex2_8(fast ? sub8(gr, tot) : gr);
-          st_f16x8(qb + o, mul8(bf16x8_to_f32(qr[i]), fw));
-          st_f16x8(kb + o, mul8(bf16x8_to_f32(kraw[m]), fw));
+          if constexpr (MODE == MODE_GATED) {
+            st_f16x8(qb + o, mul8(bf16x8_to_f32(qr[i]), mul8(fw, f8(rq[m]))));
+            st_f16x8(kb + o, mul8(bf16x8_to_f32(kraw[m]), mul8(fw, f8(rk[m]))));
+          } else {
+            st_f16x8(qb + o, mul8(bf16x8_to_f32(qr[i]), fw));
+            st_f16x8(kb + o, mul8(bf16x8_to_f32(kraw[m]), fw));
+          }
           if constexpr (MODE == MODE_SEG) {  // a transition run takes every value as zero
             st_f16x8(vb + o, x.trans ? f8(0.f) : bf16x8_to_f32(vr[i]));
           } else {
@@ -738,7 +847,10 @@ __device__ __forceinline__ void front_group(const Ctx& x, const float* __restric
       for (int m = 0; m < 4; ++m) {
         const uint32_t o = sw128_off(4 * rg + m, cc);
         gr = add8(gr, gv[m]);
-        st_f16x8(khb + o, mul8(bf16x8_to_f32(kraw[m]), ex2_8(sub8(tot, gr))));
+        if constexpr (MODE == MODE_GATED)
+          st_f16x8(khb + o, mul8(bf16x8_to_f32(kraw[m]), mul8(ex2_8(sub8(tot, gr)), f8(rk[m]))));
+        else
+          st_f16x8(khb + o, mul8(bf16x8_to_f32(kraw[m]), ex2_8(sub8(tot, gr))));
       }
     }
     fence_proxy_async_smem();
@@ -1010,9 +1122,9 @@ __device__ __forceinline__ void store_ckpt(const Ctx& x, const ModeArgs& ma, int
     return;
   }
   float* dst = ma.ckpt + ((slot * x.H + x.h) * D + col0) * D + (threadIdx.x & 127);
-#pragma unroll 8
+#pragma unroll
   for (int i = 0; i < 32; ++i) __stcs(dst + i * D, s0[i]);
-#pragma unroll 8
+#pragma unroll
   for (int i = 0; i < 32; ++i) __stcs(dst + (32 + i) * D, s1[i]);
 }
 
@@ -1020,8 +1132,8 @@ __device__ __forceinline__ void store_ckpt(const Ctx& x, const ModeArgs& ma, int
 template <int MODE>
 __device__ __forceinline__ void scan_group(const Ctx& x, const void* tmq, const void* tmk, const void* tmv, const void* tmo,
                            const float* __restrict__ init, __nv_bfloat16* __restrict__ out,
-                           float* __restrict__ fin, int64_t sbase, bool inject_stuck, int (&issued)[2],
-                           const ModeArgs& ma) {
+                           float* __restrict__ fin, int64_t sbase, int64_t ibase, bool inject_stuck,
+                           int (&issued)[2], const ModeArgs& ma) {
   const int j = threadIdx.x;  // 0..127: TMEM lane = value channel
   const uint32_t tl = x.tmem + ((uint32_t)((j >> 5) * 32) << 16);
   uint8_t* sm = x.sm;
@@ -1057,10 +1169,14 @@ __device__ __forceinline__ void scan_group(const Ctx& x, const void* tmq, const 
     float r[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
-      if constexpr (MODE == MODE_SEG)  // zero start, or the identity for a transition run
-        r[i] = (x.trans && cb * 32 + i == j) ? 1.f : 0.f;
-      else
-        r[i] = init ? __ldg(init + sbase + (int64_t)(cb * 32 + i) * D + j) : 0.f;
+      if constexpr (MODE == MODE_SEG) {  // zero start, the (scaled) identity, or a first segment's init
+        if (x.first)
+          r[i] = init ? __ldg(init + ibase + (int64_t)(cb * 32 + i) * D + j) : 0.f;
+        else
+          r[i] = (x.trans && cb * 32 + i == j) ? TRANS_SCALE : 0.f;
+      } else {
+        r[i] = init ? __ldg(init + ibase + (int64_t)(cb * 32 + i) * D + j) : 0.f;
+      }
     }
     tmem_st32(tl + TM_S + cb * 32, r);
   }
@@ -1074,17 +1190,18 @@ __device__ __forceinline__ void scan_group(const Ctx& x, const void* tmq, const 
     const int64_t tok0 = x.t0 + (int64_t)c * CH;
     float o0[32], o1[32];
     tmem_ld32x2(tl + TM_O + (c & 1) * 64, tl + TM_O + (c & 1) * 64 + 32, o0, o1);
-    if constexpr (MODE == MODE_SEG) {
+    if (MODE == MODE_SEG && !x.first) {
       // fp32 outputs straight from the registers: lane j writes channel j of
       // every valid token (a warp stores 128 contiguous bytes per token).
       float* dst = (x.trans ? ma.qhat32 : ma.o32) + (tok0 * H + x.h) * D + j;
       const int64_t st = (int64_t)H * D;
+      const float sc = x.trans ? TRANS_UNSCALE : 1.f;
 #pragma unroll
       for (int t = 0; t < 32; ++t)
-        if (t < valid) __stcs(dst + t * st, o0[t]);
+        if (t < valid) __stcs(dst + t * st, o0[t] * sc);
 #pragma unroll
       for (int t = 0; t < 32; ++t)
-        if (32 + t < valid) __stcs(dst + (32 + t) * st, o1[t]);
+        if (32 + t < valid) __stcs(dst + (32 + t) * st, o1[t] * sc);
       return;
     }
     // Lanes j and j^1 hold channels jc, jc+1 of every token; they swap one
@@ -1306,12 +1423,13 @@ __device__ __forceinline__ void scan_group(const Ctx& x, const void* tmq, const 
   if (named_sync_and(2, 128, !*x.abort)) {
     if (x.dbg && x.nchunks > 0) dump_s(x.dbg, x.tmem);
     if (fin) {
+      const float sc = (MODE == MODE_SEG && x.trans) ? TRANS_UNSCALE : 1.f;
 #pragma unroll 1
       for (int cb = 0; cb < 4; ++cb) {
         float s[32];
         tmem_ld32(tl + TM_S + cb * 32, s);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) fin[sbase + (int64_t)(cb * 32 + i) * D + j] = s[i];
+        for (int i = 0; i < 32; ++i) fin[sbase + (int64_t)(cb * 32 + i) * D + j] = MODE == MODE_SEG ? s[i] * sc : s[i];
       }
     }
     if constexpr (MODE == MODE_CKPT) {
@@ -1369,6 +1487,13 @@ __global__ void __launch_bounds__(NTHR, 1)
   const int n = order ? order[n0] : n0;
   x.h = bid % H;
   x.H = H;
+  x.first = false;
+  int64_t ibase = ((int64_t)n * H + x.h) * D * D;  // initial state of this chain
+  if constexpr (MODE == MODE_SEG) {
+    x.first = ma.seg_per_seq > 0 && n % ma.seg_per_seq == 0;
+    if (x.first && x.trans) return;  // a first segment needs no transition (the whole block leaves)
+    if (x.first) ibase = ((int64_t)(n / ma.seg_per_seq) * H + x.h) * D * D;
+  }
   if (cu) {
     x.t0 = cu[n];
     x.L = (int64_t)cu[n + 1] - x.t0;
@@ -1378,6 +1503,13 @@ __global__ void __launch_bounds__(NTHR, 1)
   }
   x.nchunks = (int)((x.L + CH - 1) / CH);
   x.ckpt0 = 0;
+  if constexpr (MODE == MODE_GATED) {
+    if (threadIdx.x == 0) {
+      float* gc = reinterpret_cast<float*>(sm + SM_MISC + MS_GATE);
+      gc[0] = -__expf(ma.A_log[x.h]) * LOG2E;
+      gc[1] = ma.g_min * LOG2E;
+    }
+  }
   if constexpr (MODE == MODE_CKPT)
     x.ckpt0 = ma.ckpt_base ? ma.ckpt_base[n] : (int64_t)n * (Tper / ((int64_t)ma.ckpt_every * CH));
   x.dbg = (HOOKS && dbg && n == 0 && x.h == 0) ? dbg : nullptr;
@@ -1410,7 +1542,8 @@ __global__ void __launch_bounds__(NTHR, 1)
   int cnt[2] = {0, 0};  // TMA stages issued (scan group) / consumed (front group)
   int* s_cnt = reinterpret_cast<int*>(sm + SM_MISC + MS_CNT);
   if (warp < 4) {
-    scan_group<MODE>(x, &tm_q, &tm_k, &tm_v, &tm_o, init, out, fin, sbase, HOOKS && inject_stuck != 0, cnt, ma);
+    scan_group<MODE>(x, &tm_q, &tm_k, &tm_v, &tm_o, init, out, fin, sbase, ibase, HOOKS && inject_stuck != 0, cnt,
+                     ma);
     if (tid == 0) { s_cnt[0] = cnt[0]; s_cnt[1] = cnt[1]; }
   } else if (warp < 12) {
     front_group<MODE>(x, g, beta, &tm_g, cnt);
@@ -1522,18 +1655,20 @@ bool make_map(CUtensorMap* m, const void* ptr, int H, int64_t Ttot) {
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// fp32 log-decay [T_total][H][128] as a 3-D map, box {128 channels, 1 head, 64 tokens}
-// (used for L2 prefetches only).
-bool make_map_g(CUtensorMap* m, const float* ptr, int H, int64_t Ttot) {
+// Decay rows [T_total][H][128] as a 3-D map, box {128 channels, 1 head, 64
+// tokens}: fp32 log-decays, or bf16 decay logits (MODE_GATED).  Used for L2
+// prefetches only.
+bool make_map_g(CUtensorMap* m, const void* ptr, int H, int64_t Ttot, bool bf16) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
+  const cuuint64_t es_bytes = bf16 ? 2 : 4;
   cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)Ttot};
-  cuuint64_t strides[2] = {(cuuint64_t)D * 4, (cuuint64_t)H * D * 4};
+  cuuint64_t strides[2] = {(cuuint64_t)D * es_bytes, (cuuint64_t)H * D * es_bytes};
   cuuint32_t box[3] = {(cuuint32_t)D, 1, (cuuint32_t)CH};
   cuuint32_t es[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(ptr), dims, strides, box, es,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(ptr),
+             dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
@@ -1554,7 +1689,7 @@ cudaError_t launch_fwd_tc_impl(const FwdArgs& a, cudaStream_t s, uint64_t wait_n
   CUtensorMap mq, mk, mv, mo, mg;
   const int64_t Tmap = Ttot > 0 ? Ttot : 1;
   if (!make_map(&mq, a.q, a.H, Tmap) || !make_map(&mk, a.k, a.H, Tmap) || !make_map(&mv, a.v, a.H, Tmap) ||
-      !make_map(&mo, a.out ? a.out : a.q, a.H, Tmap) || !make_map_g(&mg, a.g, a.H, Tmap))
+      !make_map(&mo, a.out ? a.out : a.q, a.H, Tmap) || !make_map_g(&mg, a.g, a.H, Tmap, ma.mode == MODE_GATED))
     return cudaErrorInvalidValue;
   const int32_t* order = nullptr;
   if (a.cu && order_ws && a.N > 1) {
@@ -1564,6 +1699,7 @@ cudaError_t launch_fwd_tc_impl(const FwdArgs& a, cudaStream_t s, uint64_t wait_n
   auto* kern = (a.dbg || inject_stuck) ? kda_fwd_tc_kernel<true, MODE_PLAIN>
                : ma.mode == MODE_CKPT  ? kda_fwd_tc_kernel<false, MODE_CKPT>
                : ma.mode == MODE_SEG   ? kda_fwd_tc_kernel<false, MODE_SEG>
+               : ma.mode == MODE_GATED ? kda_fwd_tc_kernel<false, MODE_GATED>
                                        : kda_fwd_tc_kernel<false, MODE_PLAIN>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
   if (e != cudaSuccess) return e;

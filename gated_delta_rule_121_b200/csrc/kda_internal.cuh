@@ -53,6 +53,9 @@ struct FwdArgs {
 enum FwdMode {
   MODE_PLAIN = 0,  // out and final state
   MODE_CKPT = 1,   // plus the state every `ckpt_every` chunks of each sequence
+  MODE_GATED = 3,  // the model's input prologue in the kernel: `g` holds the decay
+                   // logits z (dtype of q), g = g_min sigmoid(exp(A_h) z), and q, k
+                   // are L2-normalised per token and head
   MODE_SEG = 2,    // segment pieces: two runs per (sequence, head), both with
                    // fp32 outputs and no init state: the zero-start run
                    // (outputs o32, final state fin) and the transition run
@@ -72,11 +75,25 @@ struct ModeArgs {
   float* o32 = nullptr;     // [T_total][H][dv]
   float* qhat32 = nullptr;  // [T_total][H][dk]
   float* trans = nullptr;   // [N][H][dk][dk]
+  int seg_per_seq = 0;      // > 0: the batch is N/seg_per_seq sequences cut into that many
+                            // consecutive segments; the first segment of each runs from the
+                            // sequence's initial state with ordinary (dtype) outputs and no
+                            // transition run
+  // MODE_GATED
+  const float* A_log = nullptr;  // [H] per-head log scale of the decay logits
+  float g_min = -5.0f;           // lower bound of the log decay
 };
 
 // Launchers (return a CUDA error code; launches are asynchronous).
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const float* g, const float* beta,
                           float* state, void* out, int B, int H, int dk, int dv, bool bf16, cudaStream_t s);
+cudaError_t launch_decode_gated(const void* q, const void* k, const void* v, const void* z, const float* A_log,
+                                float g_min, const float* beta, float* state, void* out, int B, int H, int dk,
+                                int dv, bool bf16, cudaStream_t s);
+cudaError_t launch_spec(const void* qp, const void* kp, const void* vp, const void* gp, const float* bp,
+                        const int32_t* n_accepted, const void* q, const void* k, const void* v, const void* g,
+                        const float* beta, float* state, void* out, int B, int Wp, int W, int H, int dk, int dv,
+                        bool bf16, const float* A_log, float g_min, cudaStream_t s);
 cudaError_t launch_fwd_simt(const FwdArgs& a, bool bf16, cudaStream_t s, const ModeArgs& m = ModeArgs());
 bool fwd_tc_supported(int dk, int dv, bool bf16);
 cudaError_t launch_fwd_tc(const FwdArgs& a, cudaStream_t s);

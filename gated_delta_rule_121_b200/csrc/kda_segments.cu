@@ -17,7 +17,7 @@
 //     sequence (a sequential prefix, fp32 on CUDA cores, one block per
 //     (sequence, head, 32 value columns): the columns of S evolve
 //     independently), and
-//   - the correction o_t = o~_t + S_in^T qhat_t (dense 64-token x dv tiles on
+//   - the correction o_t = o~_t + S_in^T qhat_t (dense 128-token x dv tiles on
 //     the warp-level tensor path with tf32 operands rounded to nearest; the
 //     zero-start output o~ stays fp32, so the result is rounded once).  For
 //     fp32 outputs, whose contract allows no tf32 rounding, every product is
@@ -33,16 +33,29 @@ namespace kda {
 namespace {
 
 // ------------------------------------------------------------ composition
+// 16-byte asynchronous global->shared copies (zero-filled when src_bytes = 0).
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
 // Pieces of sequence m: p = m * R + r (piece-major) or r * N + m (rank-major,
 // the order of an all-gather over ranks).  state_in[p] = the state entering
-// piece p; final_state[m] = the state after the last piece.
+// piece p; final_state[m] = the state after the last piece.  Each step stages
+// the piece's transition M_p [DK][DK] in shared memory with asynchronous
+// copies, then every thread forms its rows of S~_p + M_p cur for its column.
 template <int DK>
 __global__ void __launch_bounds__(256)
     compose_kernel(const float* __restrict__ trans, const float* __restrict__ s0, const float* __restrict__ init,
                    float* __restrict__ state_in, float* __restrict__ fin, int R, int N, int H, int dv,
-                   int rank_major) {
+                   int rank_major, int first_from_init) {
   constexpr int RPT = DK / 8;  // rows per thread: warp w holds rows w, w + 8, ...
-  __shared__ float s_cur[DK][33];
+  extern __shared__ float cm[];
+  float* s_m = cm;                        // [DK][DK + 4]
+  float* s_cur = cm + DK * (DK + 4);      // [DK][33]
   const int ncb = (dv + 31) / 32;
   const int cb = blockIdx.x % ncb;
   const int h = (blockIdx.x / ncb) % H;
@@ -61,24 +74,31 @@ __global__ void __launch_bounds__(256)
   for (int r = 0; r < R; ++r) {
     const int64_t p = rank_major ? (int64_t)r * N + m : (int64_t)m * R + r;
     const int64_t ph = p * H + h;
+    // first_from_init: piece 0 already ran from the initial state, so its
+    // "zero-start" state is the state after it and it has no transition.
+    const bool skip_m = first_from_init && r == 0;
+    const float* Mp = trans + ph * mm;
+    if (!skip_m) {
+      for (int e = threadIdx.x; e < DK * DK / 4; e += 256) {
+        const int i = e / (DK / 4), k4 = (e % (DK / 4)) * 4;
+        cp_async16(s_m + i * (DK + 4) + k4, Mp + (int64_t)i * DK + k4, 16);
+      }
+    }
+    float acc[RPT];
 #pragma unroll
     for (int u = 0; u < RPT; ++u) {
       const int i = w + 8 * u;
       if (col && state_in) state_in[ph * sd + (int64_t)i * dv + c] = cur[u];
-      s_cur[i][lane] = cur[u];
+      s_cur[i * 33 + lane] = cur[u];
+      acc[u] = col ? __ldg(s0 + ph * sd + (int64_t)i * dv + c) : 0.f;
     }
+    cp_async_wait_all();
     __syncthreads();
-    // next = S~_p + M_p cur: row i of M_p is read by every lane of the warp
-    // (one broadcast load per element), cur from shared memory.
-    const float* Mp = trans + ph * mm;
-    float acc[RPT];
-#pragma unroll
-    for (int u = 0; u < RPT; ++u) acc[u] = col ? s0[ph * sd + (int64_t)(w + 8 * u) * dv + c] : 0.f;
 #pragma unroll 4
-    for (int kk = 0; kk < DK; ++kk) {
-      const float sv = s_cur[kk][lane];
+    for (int kk = 0; kk < (skip_m ? 0 : DK); ++kk) {
+      const float sv = s_cur[kk * 33 + lane];
 #pragma unroll
-      for (int u = 0; u < RPT; ++u) acc[u] = fmaf(__ldg(Mp + (int64_t)(w + 8 * u) * DK + kk), sv, acc[u]);
+      for (int u = 0; u < RPT; ++u) acc[u] = fmaf(s_m[(w + 8 * u) * (DK + 4) + kk], sv, acc[u]);
     }
     __syncthreads();
 #pragma unroll
@@ -92,7 +112,7 @@ __global__ void __launch_bounds__(256)
 }
 
 // ------------------------------------------------------------ correction
-constexpr int CT = 64;        // tokens per tile
+constexpr int CT = 128;       // tokens per block (8 warps x 16 tokens)
 constexpr int CPAD = 4;       // row padding (floats) of the shared tiles: conflict-free fragments
 
 __device__ __forceinline__ uint32_t tf32_rna(float x) {
@@ -112,39 +132,52 @@ __device__ __forceinline__ int piece_of(const int32_t* cu, int P, int64_t t) {
   return lo;
 }
 
-// One block: 64 consecutive tokens x all DV channels of one head.  Each of
-// the 4 warps owns 16 tokens; K = DK in steps of 8.  A tile that straddles
-// pieces is computed once per piece, each pass writing only its own rows.
+// One block: 128 consecutive tokens x all DV channels of one head.  The
+// tile's qhat rows and zero-start outputs and the piece's incoming state
+// S_in are staged in shared memory with asynchronous copies (one wait), so
+// every global read is in flight at once; each of the 8 warps then owns 16
+// tokens, K = DK in steps of 8.  A tile that straddles pieces is computed once
+// per piece, each pass writing only its own rows.
 template <int DK, int DV, typename IO>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(256)
     correct_kernel(const float* __restrict__ o32, const float* __restrict__ qhat, const float* __restrict__ s_in,
-                   IO* __restrict__ out, const int32_t* __restrict__ cu, int P, int64_t Tper, int64_t Ttot, int H) {
+                   IO* __restrict__ out, const int32_t* __restrict__ cu, int P, int64_t Tper, int64_t Ttot, int H,
+                   int skip_every) {
   extern __shared__ float csm[];
   float* s_q = csm;                        // [CT][DK + CPAD]
-  float* s_s = csm + CT * (DK + CPAD);     // [DK][DV + CPAD]
+  float* s_o = s_q + CT * (DK + CPAD);     // [CT][DV + CPAD]
+  float* s_s = s_o + CT * (DV + CPAD);     // [DK][DV + CPAD]
   const int h = blockIdx.y;
   const int64_t t0 = (int64_t)blockIdx.x * CT;
   const int nt = (int)((Ttot - t0) < CT ? (Ttot - t0) : CT);
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, g = lane >> 2, tq = lane & 3;
 
-  // qhat rows of the tile (rows past the end are zero)
-  for (int e = tid; e < CT * (DK / 4); e += 128) {
-    const int r = e / (DK / 4), c4 = (e % (DK / 4)) * 4;
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (r < nt) v = __ldcs(reinterpret_cast<const float4*>(qhat + ((t0 + r) * H + h) * DK + c4));
-    *reinterpret_cast<float4*>(s_q + r * (DK + CPAD) + c4) = v;
-  }
   const int p_first = cu ? piece_of(cu, P, t0) : (int)(t0 / Tper);
   const int p_last = cu ? piece_of(cu, P, t0 + nt - 1) : (int)((t0 + nt - 1) / Tper);
+  // skip_every > 0: pieces p with p % skip_every == 0 already hold their
+  // outputs (first segments run from the initial state)
+  if (skip_every > 0 && p_first == p_last && p_first % skip_every == 0) return;
+  // the tile's qhat rows and zero-start outputs (rows past the end zero-filled)
+  for (int e = tid; e < CT * (DK / 4); e += 256) {
+    const int r = e / (DK / 4), c4 = (e % (DK / 4)) * 4;
+    const int64_t t = t0 + (r < nt ? r : 0);
+    cp_async16(s_q + r * (DK + CPAD) + c4, qhat + (t * H + h) * DK + c4, r < nt ? 16u : 0u);
+  }
+  for (int e = tid; e < CT * (DV / 4); e += 256) {
+    const int r = e / (DV / 4), c4 = (e % (DV / 4)) * 4;
+    const int64_t t = t0 + (r < nt ? r : 0);
+    cp_async16(s_o + r * (DV + CPAD) + c4, o32 + (t * H + h) * DV + c4, r < nt ? 16u : 0u);
+  }
   for (int p = p_first; p <= p_last; ++p) {
     const int64_t lo = cu ? cu[p] : (int64_t)p * Tper, hi = cu ? cu[p + 1] : (int64_t)(p + 1) * Tper;
-    if (hi <= lo) continue;  // empty piece
+    if (hi <= lo || (skip_every > 0 && p % skip_every == 0)) continue;  // empty, or needs no correction
     __syncthreads();         // the previous pass is done with s_s
     const float* S = s_in + ((int64_t)p * H + h) * DK * DV;
-    for (int e = tid; e < DK * (DV / 4); e += 128) {
+    for (int e = tid; e < DK * (DV / 4); e += 256) {
       const int r = e / (DV / 4), c4 = (e % (DV / 4)) * 4;
-      *reinterpret_cast<float4*>(s_s + r * (DV + CPAD) + c4) = __ldg(reinterpret_cast<const float4*>(S + r * DV + c4));
+      cp_async16(s_s + r * (DV + CPAD) + c4, S + r * DV + c4, 16u);
     }
+    cp_async_wait_all();  // also completes the tile's rows on the first pass
     __syncthreads();
     if (w * 16 >= nt) continue;
     float d[DV / 8][4];
@@ -180,15 +213,16 @@ __global__ void __launch_bounds__(128)
       const int64_t t = t0 + r;
       if (r >= nt || t < lo || t >= hi) continue;
       const int64_t base = (t * H + h) * DV;
+      const float* zo = s_o + r * (DV + CPAD);
 #pragma unroll
       for (int n = 0; n < DV / 8; ++n) {
         const int c = n * 8 + 2 * tq;
-        const float2 z = __ldcs(reinterpret_cast<const float2*>(o32 + base + c));
-        out[base + c] = from_f32<IO>(z.x + d[n][2 * half]);
-        out[base + c + 1] = from_f32<IO>(z.y + d[n][2 * half + 1]);
+        out[base + c] = from_f32<IO>(zo[c] + d[n][2 * half]);
+        out[base + c + 1] = from_f32<IO>(zo[c + 1] + d[n][2 * half + 1]);
       }
     }
   }
+  cp_async_wait_all();  // no copy may still be landing when the block leaves
 }
 
 // ------------------------------------------------------------ segment layout
@@ -211,35 +245,40 @@ __global__ void segment_cu_kernel(const int32_t* __restrict__ cu, int64_t Tper, 
 
 template <int DK>
 cudaError_t compose_dk(const float* trans, const float* s0, const float* init, float* state_in, float* fin, int R,
-                       int N, int H, int dv, int rank_major, cudaStream_t s) {
+                       int N, int H, int dv, int rank_major, int first_from_init, cudaStream_t s) {
   const int ncb = (dv + 31) / 32;
   const int64_t blocks = (int64_t)N * H * ncb;
   if (blocks == 0) return cudaSuccess;
-  compose_kernel<DK><<<(unsigned)blocks, 256, 0, s>>>(trans, s0, init, state_in, fin, R, N, H, dv, rank_major);
+  const size_t smem = sizeof(float) * ((size_t)DK * (DK + 4) + (size_t)DK * 33);
+  cudaError_t e = cudaFuncSetAttribute(compose_kernel<DK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  compose_kernel<DK><<<(unsigned)blocks, 256, smem, s>>>(trans, s0, init, state_in, fin, R, N, H, dv, rank_major,
+                                                          first_from_init);
   return cudaGetLastError();
 }
 
 template <int DK, int DV, typename IO>
 cudaError_t correct_t(const float* o32, const float* qhat, const float* s_in, void* out, const int32_t* cu, int P,
-                      int64_t Tper, int64_t Ttot, int H, cudaStream_t s) {
+                      int64_t Tper, int64_t Ttot, int H, int skip_every, cudaStream_t s) {
   if (Ttot == 0) return cudaSuccess;
-  const size_t smem = sizeof(float) * ((size_t)CT * (DK + CPAD) + (size_t)DK * (DV + CPAD));
+  const size_t smem =
+      sizeof(float) * ((size_t)CT * (DK + CPAD) + (size_t)CT * (DV + CPAD) + (size_t)DK * (DV + CPAD));
   auto* kern = correct_kernel<DK, DV, IO>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)((Ttot + CT - 1) / CT), (unsigned)H);
-  kern<<<grid, 128, smem, s>>>(o32, qhat, s_in, (IO*)out, cu, P, Tper, Ttot, H);
+  kern<<<grid, 256, smem, s>>>(o32, qhat, s_in, (IO*)out, cu, P, Tper, Ttot, H, skip_every);
   return cudaGetLastError();
 }
 
 template <int DK, typename IO>
 cudaError_t correct_dv(const float* o32, const float* qhat, const float* s_in, void* out, const int32_t* cu, int P,
-                       int64_t Tper, int64_t Ttot, int H, int dv, cudaStream_t s) {
+                       int64_t Tper, int64_t Ttot, int H, int dv, int skip_every, cudaStream_t s) {
   switch (dv) {
-    case 16: return correct_t<DK, 16, IO>(o32, qhat, s_in, out, cu, P, Tper, Ttot, H, s);
-    case 32: return correct_t<DK, 32, IO>(o32, qhat, s_in, out, cu, P, Tper, Ttot, H, s);
-    case 64: return correct_t<DK, 64, IO>(o32, qhat, s_in, out, cu, P, Tper, Ttot, H, s);
-    case 128: return correct_t<DK, 128, IO>(o32, qhat, s_in, out, cu, P, Tper, Ttot, H, s);
+    case 16: return correct_t<DK, 16, IO>(o32, qhat, s_in, out, cu, P, Tper, Ttot, H, skip_every, s);
+    case 32: return correct_t<DK, 32, IO>(o32, qhat, s_in, out, cu, P, Tper, Ttot, H, skip_every, s);
+    case 64: return correct_t<DK, 64, IO>(o32, qhat, s_in, out, cu, P, Tper, Ttot, H, skip_every, s);
+    case 128: return correct_t<DK, 128, IO>(o32, qhat, s_in, out, cu, P, Tper, Ttot, H, skip_every, s);
   }
   return cudaErrorInvalidValue;
 }
@@ -247,23 +286,25 @@ cudaError_t correct_dv(const float* o32, const float* qhat, const float* s_in, v
 }  // namespace
 
 cudaError_t launch_compose(const float* trans, const float* s0, const float* init, float* state_in, float* fin,
-                           int R, int N, int H, int dk, int dv, int rank_major, cudaStream_t s) {
+                           int R, int N, int H, int dk, int dv, int rank_major, int first_from_init,
+                           cudaStream_t s) {
   switch (dk) {
-    case 16: return compose_dk<16>(trans, s0, init, state_in, fin, R, N, H, dv, rank_major, s);
-    case 32: return compose_dk<32>(trans, s0, init, state_in, fin, R, N, H, dv, rank_major, s);
-    case 64: return compose_dk<64>(trans, s0, init, state_in, fin, R, N, H, dv, rank_major, s);
-    case 128: return compose_dk<128>(trans, s0, init, state_in, fin, R, N, H, dv, rank_major, s);
+    case 16: return compose_dk<16>(trans, s0, init, state_in, fin, R, N, H, dv, rank_major, first_from_init, s);
+    case 32: return compose_dk<32>(trans, s0, init, state_in, fin, R, N, H, dv, rank_major, first_from_init, s);
+    case 64: return compose_dk<64>(trans, s0, init, state_in, fin, R, N, H, dv, rank_major, first_from_init, s);
+    case 128: return compose_dk<128>(trans, s0, init, state_in, fin, R, N, H, dv, rank_major, first_from_init, s);
   }
   return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_correct(const float* o32, const float* qhat, const float* s_in, void* out, const int32_t* cu,
-                           int P, int64_t Tper, int64_t Ttot, int H, int dk, int dv, bool bf16, cudaStream_t s) {
+                           int P, int64_t Tper, int64_t Ttot, int H, int dk, int dv, bool bf16, int skip_every,
+                           cudaStream_t s) {
   switch (dk) {
 #define KDA_CORRECT_DK(DK_)                                                                                  \
   case DK_:                                                                                                  \
-    return bf16 ? correct_dv<DK_, __nv_bfloat16>(o32, qhat, s_in, out, cu, P, Tper, Ttot, H, dv, s)          \
-                : correct_dv<DK_, float>(o32, qhat, s_in, out, cu, P, Tper, Ttot, H, dv, s);
+    return bf16 ? correct_dv<DK_, __nv_bfloat16>(o32, qhat, s_in, out, cu, P, Tper, Ttot, H, dv, skip_every, s) \
+                : correct_dv<DK_, float>(o32, qhat, s_in, out, cu, P, Tper, Ttot, H, dv, skip_every, s);
     KDA_CORRECT_DK(16)
     KDA_CORRECT_DK(32)
     KDA_CORRECT_DK(64)

@@ -212,6 +212,27 @@ KDA_API kda_status_t kda_decode_step(const void *q, const void *k, const void *v
                              void *stream, kda_dtype_t dt);
 
 /*
+ * kda_fwd with the model's input prologue fused in (the digest's "Kimi Delta
+ * Attention" section: q and k are L2-normalised, and the decay logits z get a
+ * per-head scale; "Bounded decay" section: g = g_min * sigmoid(exp(A_h) * z),
+ * alpha = exp(g), with g_min = -5 in the model's configuration):
+ *   q, k       [B, T, H, dk]  dtype dt, NOT normalised: the kernel uses
+ *              x / sqrt(|x|^2 + 1e-6) per (token, head), in fp32, folded into
+ *              its operand scaling (no normalised copy is written)
+ *   z          [B, T, H, dk]  dtype dt: the decay logits, in place of log_alpha
+ *   A_log      [H] fp32, device: the per-head log scale A_h
+ *   g_min      the lower bound of the log decay
+ * Everything else as kda_fwd (same workspace).  HBM traffic per token-head
+ * drops from 1540 to 1284 bytes for bf16 (z is bf16 where log_alpha is fp32).
+ */
+KDA_API kda_status_t kda_fwd_gated(const void *q, const void *k, const void *v, const void *z,
+                                   const float *A_log, float g_min, const float *beta,
+                                   const float *init_state, void *out, float *final_state,
+                                   int B, int64_t T, int H, int dk, int dv,
+                                   const int32_t *cu_seqlens, void *stream, kda_dtype_t dt,
+                                   void *workspace, size_t workspace_bytes);
+
+/*
  * Interval checkpoints for prefix caching (the digest's serving section,
  * "decoupling hash granularity from storage granularity": the KDA state is
  * stored only at a sparse subset of the 512-token hash boundaries, so that a
@@ -329,6 +350,68 @@ KDA_API kda_status_t kda_fwd_cp(const void *q, const void *k, const void *v,
                                 int B, int64_t T, int H, int dk, int dv,
                                 const int32_t *cu_seqlens, void *stream, kda_dtype_t dt, int n_seg,
                                 void *workspace, size_t workspace_bytes);
+
+/*
+ * The decode step with the model's input prologue fused in (the digest's KDA
+ * section: q and k are L2-normalised, the decay logits get a per-head
+ * scale; "Bounded decay" section: g = g_min * sigmoid(exp(A_h) * z)):
+ *   q, k       [B, H, dk]  dtype dt, NOT normalised; the kernel uses
+ *              x / sqrt(|x|^2 + 1e-6) per (sequence, head)
+ *   z          [B, H, dk]  dtype dt: the decay logits
+ *   A_log      [H] fp32: the per-head log scale A_h
+ *   g_min      the lower bound of the log decay (-5 in the model)
+ * Everything else as kda_decode_step.
+ */
+KDA_API kda_status_t kda_decode_step_gated(const void *q, const void *k, const void *v, const void *z,
+                                           const float *A_log, float g_min, const float *beta,
+                                           float *state, void *out, int B, int H, int dk, int dv,
+                                           void *stream, kda_dtype_t dt);
+
+/*
+ * Speculative-decode verification with state replay (the digest's serving
+ * section, "speculative decoding and KDA state rewind": the state after the
+ * accepted draft prefix is fully determined by the drafts' projected inputs,
+ * which are much smaller than the state; so only those inputs are kept, the
+ * accepted tokens' states are rebuilt on chip, and only the committed state
+ * is written back).
+ *
+ * One call per decode step, for B sequences:
+ *   *_prev     [B, Wp, H, d]: the previous call's window (its projected
+ *              inputs, kept by the caller); may be NULL when Wp = 0
+ *   n_accepted [B] int32, device: how many of those Wp draft tokens
+ *              verification accepted (clamped to [0, Wp])
+ *   q, k, v, log_alpha, beta  [B, W, H, d]: the new window; token 0 is the
+ *              bonus token (certain), tokens 1..W-1 the next drafts
+ *   state      [B, H, dk, dv] fp32: the committed state, read once, and
+ *              overwritten once with the state after the accepted tokens and
+ *              the bonus token
+ *   out        [B, W, H, dv]: the outputs of the W new tokens (each read with
+ *              the state after that token)
+ * The rejected drafts of the previous window are never applied; the new
+ * drafts' states stay on chip.  Wp + W <= KDA_SPEC_MAX_TOKENS.  W = 0 only
+ * replays.  No workspace.
+ */
+#define KDA_SPEC_MAX_TOKENS 64
+KDA_API kda_status_t kda_decode_spec(const void *q_prev, const void *k_prev, const void *v_prev,
+                                     const float *log_alpha_prev, const float *beta_prev,
+                                     const int32_t *n_accepted,
+                                     const void *q, const void *k, const void *v,
+                                     const float *log_alpha, const float *beta,
+                                     float *state, void *out, int B, int Wp, int W, int H, int dk, int dv,
+                                     void *stream, kda_dtype_t dt);
+
+/*
+ * kda_decode_spec with the input prologue fused in, as kda_decode_step_gated:
+ * z_prev / z are the decay logits (dtype dt) in place of the log-decays, and
+ * q, k are normalised by the kernel; A_log [H] and g_min as there.
+ */
+KDA_API kda_status_t kda_decode_spec_gated(const void *q_prev, const void *k_prev, const void *v_prev,
+                                           const void *z_prev, const float *beta_prev,
+                                           const int32_t *n_accepted,
+                                           const void *q, const void *k, const void *v, const void *z,
+                                           const float *beta, const float *A_log, float g_min,
+                                           float *state, void *out, int B, int Wp, int W, int H, int dk, int dv,
+                                           void *stream, kda_dtype_t dt);
 
 /*
  * Read back the device status word of a workspace used by kda_fwd.

@@ -137,3 +137,66 @@ def transition(q, k, g, beta, cu_seqlens=None, nthreads: int | None = None):
     zeros_v = np.zeros((B, T, H, dk), np.float64)
     eye = np.broadcast_to(np.eye(dk), (N, H, dk, dk)).copy()
     return fwd(q64, k, zeros_v, g, beta, eye, cu_seqlens, nthreads=nthreads)
+
+
+# -- the model's input prologue (digest: "Kimi Delta Attention" section, q and
+#    k L2-normalised, decay logits with a per-head bias/scale; "Bounded decay"
+#    section, g = g_min * sigmoid(exp(A_h) * z) with g_min = -5) ---------------
+G_MIN = -5.0
+L2NORM_EPS = 1e-6
+
+
+def gate(z, A_log, g_min=G_MIN):
+    """Log-decay from decay logits z [..., H, dk] and per-head log scales A_log
+    [H]: g = g_min * sigmoid(exp(A_h) * z), in fp64."""
+    z = _f64(z)
+    a = np.exp(_f64(A_log))[:, None]          # [H, 1], broadcast over the key channels
+    return g_min / (1.0 + np.exp(-a * z))
+
+
+def l2norm(x, eps=L2NORM_EPS):
+    """x / sqrt(|x|^2 + eps) over the last axis, in fp64."""
+    x = _f64(x)
+    return x / np.sqrt((x * x).sum(-1, keepdims=True) + eps)
+
+
+def fwd_gated(q, k, v, z, A_log, beta, init_state=None, cu_seqlens=None, g_min=G_MIN, nthreads=None):
+    """The forward with the prologue: normalise q and k, map z to g, then the
+    token-by-token recurrence (``fwd``)."""
+    return fwd(l2norm(q), l2norm(k), v, gate(z, A_log, g_min), beta, init_state, cu_seqlens, nthreads=nthreads)
+
+
+def decode_step_gated(q, k, v, z, A_log, beta, state, g_min=G_MIN):
+    """``decode_step`` with the prologue applied to the token's raw inputs."""
+    return decode_step(l2norm(q), l2norm(k), v, gate(z, A_log, g_min), beta, state)
+
+
+def spec_decode(prev, n_accepted, cur, state):
+    """Speculative-decode verification with state replay (digest, serving
+    section, "speculative decoding and KDA state rewind"), as a plain loop of
+    decode steps.  ``prev`` and ``cur`` are dicts of q, k, v, g, beta shaped
+    [B, W, H, *] (``prev`` may be None when nothing was drafted);
+    ``n_accepted`` [B].  For every sequence b: the first n_accepted[b] tokens
+    of ``prev`` are applied to the state (no outputs), then every token of
+    ``cur`` with its output; the state kept is the one after ``cur``'s first
+    token (or after the replay when ``cur`` is empty).  ``state`` (fp64
+    [B, H, dk, dv]) is updated in place to that kept state.  Returns the
+    outputs [B, W, H, dv]."""
+    B, W, H = cur["q"].shape[:3]
+    dv = state.shape[-1]
+    out = np.zeros((B, W, H, dv), np.float64)
+    na = np.asarray(_f64(n_accepted)).astype(np.int64) if n_accepted is not None else np.zeros(B, np.int64)
+    for b in range(B):
+        S = np.ascontiguousarray(state[b:b + 1])
+        one = lambda src, t: {n: _f64(src[n])[b:b + 1, t] for n in ("q", "k", "v", "g", "beta")}
+        for t in range(int(na[b]) if prev is not None else 0):
+            x = one(prev, t)
+            decode_step(x["q"], x["k"], x["v"], x["g"], x["beta"], S)
+        keep = S.copy()
+        for t in range(W):
+            x = one(cur, t)
+            out[b, t] = decode_step(x["q"], x["k"], x["v"], x["g"], x["beta"], S)[0]
+            if t == 0:
+                keep = S.copy()
+        state[b] = keep[0]
+    return out

@@ -156,3 +156,64 @@ def make_decode_step(spec: DecodeSpec, step: int, device="cpu", B: int | None = 
     B, H = B or spec.B, H or spec.H
     q, k, v, g, beta = draw_tokens(gen, B, H, spec.dk, spec.dv, spec.dtype, spec.g_scale, device)
     return dict(q=q, k=k, v=v, g=g, beta=beta)
+
+
+# -- raw inputs of the model's prologue (for the fused-prologue entry points) --
+def draw_prologue_tokens(gen, T, H, dk, dv, io_dtype, z_shift, device):
+    """Unnormalised q, k ~ N(0,1) (scaled per token by a factor in [0.5, 2) so
+    the normalisation matters), v ~ N(0,1), decay logits z ~ N(z_shift, 1) in
+    the I/O dtype, beta = sigmoid(N(0,1)); all token-major [T,H,*]."""
+    def scaled(x):
+        s = torch.rand(x.shape[:-1] + (1,), generator=gen, device=device) * 1.5 + 0.5
+        return (x * s).to(io_dtype)
+    q = _slabbed(gen, T, (H, dk), device, scaled)
+    k = _slabbed(gen, T, (H, dk), device, scaled)
+    v = _slabbed(gen, T, (H, dv), device, lambda x: x.to(io_dtype))
+    z = _slabbed(gen, T, (H, dk), device, lambda x: (x + z_shift).to(io_dtype))
+    beta = _slabbed(gen, T, (H,), device, torch.sigmoid)
+    return q, k, v, z, beta
+
+
+def make_prologue_prefill(spec: PrefillSpec, device="cpu", T: int | None = None, B: int | None = None,
+                          H: int | None = None, lengths: list[int] | None = None, z_shift: float = -5.0):
+    """Raw prologue inputs for one prefill call: q, k, v, z (decay logits), beta,
+    A_log [H] ~ N(0, 0.25) (standard deviation 0.5), init_state, cu_seqlens.
+    With A_log near 0, z_shift = -5 gives per-token log-decays g = -5
+    sigmoid(e^A z) of a few hundredths (the mild regime of the benchmark
+    generators); z_shift = 0 gives the model's full range down to -5."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(spec.seed + 1000)
+    H = H or spec.H
+    if lengths is not None or spec.varlen is not None:
+        if lengths is None:
+            total, lo, hi = spec.varlen
+            lengths = varlen_lengths(T or total, lo, hi, spec.seed)
+        Ttot = int(sum(lengths))
+        cu = torch.tensor(np.concatenate([[0], np.cumsum(lengths)]), dtype=torch.int32, device=device)
+        N, Bx, Tx = len(lengths), 1, Ttot
+    else:
+        B = B or spec.B
+        T = T if T is not None else spec.T
+        cu, N, Bx, Tx, Ttot = None, B, B, T, B * T
+    q, k, v, z, beta = draw_prologue_tokens(gen, Ttot, H, spec.dk, spec.dv, spec.dtype, z_shift, device)
+    A_log = (_randn(gen, (H,), device) * 0.5).contiguous()
+    init = (_randn(gen, (N, H, spec.dk, spec.dv), device) * 0.1).contiguous() if spec.init else None
+    shp = lambda x, d: x.reshape(Bx, Tx, H, d) if d else x.reshape(Bx, Tx, H)
+    return dict(q=shp(q, spec.dk), k=shp(k, spec.dk), v=shp(v, spec.dv), z=shp(z, spec.dk), beta=shp(beta, 0),
+                A_log=A_log, init_state=init, cu_seqlens=cu)
+
+
+def make_spec_window(spec: DecodeSpec, step: int, W: int, device="cpu", B: int | None = None,
+                     H: int | None = None, prologue: bool = False, z_shift: float = -5.0):
+    """One window of W tokens per sequence for speculative decoding, shaped
+    [B, W, H, *]: q, k, v, g (log-decay) and beta, or with ``prologue`` the
+    raw q, k and the decay logits z (as key "g") of the prologue."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(spec.seed * 1_000_003 + 7919 * (step + 1) + W)
+    B, H = B or spec.B, H or spec.H
+    if prologue:
+        q, k, v, g, beta = draw_prologue_tokens(gen, B * W, H, spec.dk, spec.dv, spec.dtype, z_shift, device)
+    else:
+        q, k, v, g, beta = draw_tokens(gen, B * W, H, spec.dk, spec.dv, spec.dtype, spec.g_scale, device)
+    r = lambda x: x.reshape((B, W) + tuple(x.shape[1:])).contiguous()
+    return dict(q=r(q), k=r(k), v=r(v), g=r(g), beta=r(beta))

@@ -50,13 +50,31 @@ def half_ulp_bf16(ref):
     return np.where(a > 0, np.ldexp(1.0, (ex - 8).astype(np.int64)), 0.0)
 
 
+def rounding_alone(ref):
+    """max |bf16(ref) - ref| / RMS(ref): what storing the exact result in bf16
+    costs by itself against the max-abs bound."""
+    ra = to_f64(ref)
+    if ra.size == 0:
+        return 0.0
+    rb = torch.from_numpy(ra).to(torch.bfloat16).double().numpy()
+    rms = np.linalg.norm(ra) / np.sqrt(ra.size)
+    return float(np.abs(rb - ra).max() / max(rms, 1e-300))
+
+
 def assert_close(x, ref, dtype, what="", literal=True):
     """Assert the contract's tolerances.  ``literal=False`` (strongly decaying
     inputs only) subtracts the output's unavoidable half-ulp bf16 rounding
-    before the max-abs test."""
+    before the max-abs test.  ``literal="auto"`` applies the literal bound
+    unless rounding the exact result to bf16 alone already takes more than
+    three quarters of it (then the excess reading, recorded in the result)."""
     e = errors(x, ref)
     t = TOL[dtype]
     xa, ra = to_f64(x), to_f64(ref)
+    if literal == "auto":
+        rounded_out = isinstance(x, torch.Tensor) and x.dtype == torch.bfloat16
+        e["rounding_alone"] = rounding_alone(ra) if rounded_out else 0.0
+        literal = t["max_abs_rms"] is None or e["rounding_alone"] <= 0.75 * t["max_abs_rms"]
+    e["literal"] = bool(literal)
     assert np.isfinite(xa).all(), f"{what}: non-finite values"
     assert e["rel_fro"] <= t["rel_fro"], f"{what}: rel_fro {e['rel_fro']:.3e} > {t['rel_fro']:.1e}"
     if t["max_abs_rms"] is not None:

@@ -51,7 +51,14 @@ def test_segment_pieces_match_oracle(case):
     assert_close(o0, o_ref, dtype, f"{case} zero-start out", literal=literal)
     assert_close(s0, s_ref, dtype, f"{case} zero-start state", literal=literal)
     assert_close(qh, qh_ref, dtype, f"{case} qhat", literal=literal)
-    assert_close(M, M_ref, dtype, f"{case} transition", literal=literal)
+    # The transition is dimensionless with the identity as its scale: it acts
+    # on an incoming state, so its error is measured per (sequence, head)
+    # against max(|M|_F, 1e-2) (a strongly decaying segment's M is ~0).
+    Mg, Mr = M.double().cpu().numpy(), np.asarray(M_ref)
+    err = np.linalg.norm((Mg - Mr).reshape(Mr.shape[0], Mr.shape[1], -1), axis=-1)
+    scale = np.maximum(np.linalg.norm(Mr.reshape(Mr.shape[0], Mr.shape[1], -1), axis=-1), 1e-2)
+    tol = 1e-4 if dtype == torch.float32 else 5e-3
+    assert (err / scale).max() <= tol, f"{case} transition: {(err / scale).max():.3e}"
 
 
 def _compose_ref(M, S0, init, R, rank_major):

@@ -287,3 +287,75 @@ def test_composition_over_many_segments():
         S = s_zero + M[0, 0] @ S
         _, s_ref = run_chain(q[:b], k[:b], v[:b], g[:b], beta[:b], s0)
         np.testing.assert_allclose(S, s_ref, rtol=1e-10, atol=1e-12)
+
+
+# -- the input prologue (KDA section: L2 norm of q, k; Bounded decay: the gate) --
+def test_gate_closed_forms():
+    """g = g_min sigmoid(e^A z): g(0) = g_min / 2; g -> g_min for z -> +inf and
+    -> 0 for z -> -inf; e^A scales z; always inside (g_min, 0)."""
+    H, d = 3, 5
+    A = np.array([0.0, np.log(2.0), -1.0])
+    z0 = np.zeros((4, H, d))
+    np.testing.assert_allclose(oracle.gate(z0, A), -2.5, rtol=0, atol=0)
+    assert np.all(oracle.gate(z0 + 200.0, A) < -5.0 + 1e-12)
+    assert np.all(oracle.gate(z0 - 200.0, A) > -1e-12)
+    rng = np.random.default_rng(3)
+    z = rng.standard_normal((4, H, d))
+    g = oracle.gate(z, A)
+    assert np.all((g > -5.0) & (g < 0.0))
+    np.testing.assert_allclose(g[:, 1], oracle.gate(2.0 * z, np.zeros(H))[:, 1], rtol=1e-15)
+    np.testing.assert_allclose(oracle.gate(z, A, g_min=-3.0), g * 0.6, rtol=1e-15)
+    # monotone decreasing in z (a larger logit decays more)
+    zs = np.sort(rng.standard_normal(50))
+    gs = oracle.gate(zs[:, None, None] * np.ones((1, H, d)), A)[:, 0, 0]
+    assert np.all(np.diff(gs) < 0)
+
+
+def test_l2norm_unit_rows_and_direction():
+    rng = np.random.default_rng(4)
+    x = rng.standard_normal((7, 3, 16)) * rng.uniform(0.1, 10.0, (7, 3, 1))
+    y = oracle.l2norm(x)
+    np.testing.assert_allclose(np.linalg.norm(y, axis=-1), 1.0, rtol=0, atol=1e-6)
+    cos = (x * y).sum(-1) / np.linalg.norm(x, axis=-1) / np.linalg.norm(y, axis=-1)
+    np.testing.assert_allclose(cos, 1.0, rtol=0, atol=1e-14)
+
+
+def test_gated_forward_ignores_the_scale_of_q_and_k():
+    """Normalising q and k makes the output blind to their per-token scale."""
+    rng = np.random.default_rng(8)
+    B, T, H, d = 1, 20, 2, 8
+    q = rng.standard_normal((B, T, H, d))
+    k = rng.standard_normal((B, T, H, d))
+    v = rng.standard_normal((B, T, H, d))
+    z = rng.standard_normal((B, T, H, d))
+    beta = rng.random((B, T, H))
+    A = np.array([0.3, -0.2])
+    o1, s1 = oracle.fwd_gated(q, k, v, z, A, beta)
+    o2, s2 = oracle.fwd_gated(q * rng.uniform(0.5, 3.0, (B, T, H, 1)), k * rng.uniform(0.5, 3.0, (B, T, H, 1)),
+                              v, z, A, beta)
+    np.testing.assert_allclose(o2, o1, rtol=1e-5, atol=1e-7)
+    np.testing.assert_allclose(s2, s1, rtol=1e-5, atol=1e-7)
+
+
+# -- speculative verification with state replay (serving section) -----------
+def test_spec_decode_equals_forward_over_the_accepted_tokens():
+    """Outputs of the new window = outputs of a forward over the accepted
+    drafts followed by the new window; the kept state = that forward's state
+    after the bonus token; rejected drafts leave no trace."""
+    rng = np.random.default_rng(12)
+    B, Wp, W, H, d = 4, 3, 4, 2, 6
+    mk = lambda n: dict(q=rng.standard_normal((B, n, H, d)), k=rng.standard_normal((B, n, H, d)),
+                        v=rng.standard_normal((B, n, H, d)), g=-0.3 * rng.random((B, n, H, d)),
+                        beta=rng.random((B, n, H)))
+    prev, cur = mk(Wp), mk(W)
+    s0 = 0.2 * rng.standard_normal((B, H, d, d))
+    na = np.array([0, 1, 3, 2])
+    st = s0.copy()
+    out = oracle.spec_decode(prev, na, cur, st)
+    for b in range(B):
+        cat = {n: np.concatenate([prev[n][b:b + 1, :na[b]], cur[n][b:b + 1]], 1) for n in prev}
+        o_ref, _ = oracle.fwd(cat["q"], cat["k"], cat["v"], cat["g"], cat["beta"], s0[b:b + 1])
+        np.testing.assert_allclose(out[b], o_ref[0, na[b]:], rtol=1e-12, atol=1e-12)
+        upto = {n: v[:, :na[b] + 1] for n, v in cat.items()}
+        _, s_ref = oracle.fwd(upto["q"], upto["k"], upto["v"], upto["g"], upto["beta"], s0[b:b + 1])
+        np.testing.assert_allclose(st[b], s_ref[0], rtol=1e-12, atol=1e-12)

@@ -41,3 +41,16 @@ def test_error_accumulator_matches_one_shot_measures():
         bad.check()
     with pytest.raises(AssertionError):
         assert_close(y, ref, torch.bfloat16, literal=True)
+
+
+def test_auto_reading_follows_the_rounding_of_the_exact_result():
+    from parity import assert_close, rounding_alone
+    rng = np.random.default_rng(2)
+    calm = rng.standard_normal(4000)                       # max ~ 3.7 RMS: rounding alone ~0.007 RMS
+    assert rounding_alone(calm) < 0.02
+    e = assert_close(torch.from_numpy(calm).to(torch.bfloat16), calm, torch.bfloat16, literal="auto")
+    assert e["literal"]
+    heavy = np.concatenate([rng.standard_normal(4000) * 0.05, [7.9, -7.9]])  # max ~ 50 RMS
+    assert rounding_alone(heavy) > 0.03
+    e = assert_close(torch.from_numpy(heavy).to(torch.bfloat16), heavy, torch.bfloat16, literal="auto")
+    assert not e["literal"]
