@@ -322,7 +322,7 @@ def bench_prefill(name, d, dev, stream, peaks, kda, synth, steps, warmup, with_t
     import torch
     spec = workload_spec(name)
     if variant == "gated":  # raw prologue inputs: unnormalised q, k and bf16 decay logits z (mild decay)
-        inp = synth.make_prologue_prefill(spec, dev)
+        inp = synth.make_prologue_prefill(spec, dev, a_std=0.0)
         inp["g"] = inp.pop("z")
     else:
         inp = synth.make_prefill(spec, dev)
@@ -438,6 +438,8 @@ def run_native(args, d):
     torch.cuda.empty_cache()
     if not args.no_decode:
         line["decode"] = bench_decode(args, d, dev, stream, peaks, kda, synth)
+        line["decode_gated"] = bench_decode(args, d, dev, stream, peaks, kda, synth, gated=True)
+        line["decode_spec"] = bench_spec(args, d, dev, stream, peaks, kda, synth)
     if not args.no_workloads:
         others = {}
         for key, name, steps, variant in (("mid", "mid", 50, None), ("mid_cp", "mid", 50, "cp"),
@@ -459,33 +461,90 @@ def run_native(args, d):
     d.close()
 
 
-def bench_decode(args, d, dev, stream, peaks, kda, synth):
+def bench_decode(args, d, dev, stream, peaks, kda, synth, gated=False):
+    """One decode step per timed step over the B=512, H=96 workload; gated:
+    kda_decode_step_gated on the raw prologue inputs (bf16 decay logits)."""
     import torch
     spec = synth.DECODE
     state = synth.make_decode_state(spec, dev)
     n_in = args.warmup + args.steps
-    xs = [synth.make_decode_step(spec, s, dev) for s in range(n_in)]
+    if gated:
+        xs = [{n: t[:, 0].contiguous() for n, t in synth.make_spec_window(spec, s, 1, dev, prologue=True).items()}
+              for s in range(n_in)]
+        A_log = torch.zeros(spec.H, dtype=torch.float32, device=dev)
+    else:
+        xs = [synth.make_decode_step(spec, s, dev) for s in range(n_in)]
     out = torch.empty((spec.B, spec.H, spec.dv), dtype=spec.dtype, device=dev)
     it = iter(range(10 ** 9))
 
     def step():
         x = xs[next(it) % n_in]
-        kda.kda_decode_step(x["q"], x["k"], x["v"], x["g"], x["beta"], state, out=out, stream=stream)
+        if gated:
+            kda.kda_decode_step_gated(x["q"], x["k"], x["v"], x["g"], A_log, x["beta"], state, out=out,
+                                      stream=stream)
+        else:
+            kda.kda_decode_step(x["q"], x["k"], x["v"], x["g"], x["beta"], state, out=out, stream=stream)
 
     sec = time_loop(step, args.steps, args.warmup, stream, d)
     value = job_throughput(d, spec.B * spec.H * args.steps, sec) / 1e6
     per = d.max(sec) / args.steps
     nbytes = decode_bytes(spec.B, spec.H, spec.dk, spec.dv, 2)
+    if gated:
+        nbytes -= spec.B * spec.H * spec.dk * 2  # bf16 decay logits in place of fp32 log-decays
     ach = nbytes / per / 1e9
     prof, src = TRAFFIC_PROFILES["kda_decode_kernel"]
-    traffic = scaled_traffic(prof, src, spec.B * spec.H, 0.0)
+    traffic = None if gated else scaled_traffic(prof, src, spec.B * spec.H, 0.0)
     del xs, state
-    return {"workload": spec.name, "value": value, "unit": UNIT,
+    return {"workload": spec.name + ("_gated" if gated else ""), "value": value, "unit": UNIT,
             "ms_per_step": per * 1e3, "gpu_launches": args.steps,
             "l2": "state 3.2 GB per step, far larger than L2, no flush",
             "roofline": {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": ach / peaks["hbm_gbs"], "traffic": traffic, "bytes_per_launch": nbytes,
                          "kernel": "kda_decode_kernel<128,128,bf16>"}}
+
+
+def bench_spec(args, d, dev, stream, peaks, kda, synth, W=4, sweep=(1, 2, 4, 8)):
+    """Speculative verification with state replay at B=512, H=96: every step
+    replays the accepted drafts of the previous window (accept counts drawn
+    uniformly in 0..W-1, seeded), runs the bonus token and W-1 new drafts, and
+    writes the state once.  value = new-window tokens x heads per second;
+    the roofline counts the state read and write plus the token bytes read.
+    Also the step time for windows of 1, 2, 4 and 8 tokens (the verification
+    cost against the number of tokens it covers)."""
+    import numpy as np
+    import torch
+    spec = synth.DECODE
+    B, H, dk, dv = spec.B, spec.H, spec.dk, spec.dv
+    rng = np.random.default_rng(9)
+    res = {"workload": f"spec_decode_bf16_B{B}_H{H}_d128_W{W}"}
+    times = {}
+    for w in sorted(set(sweep) | {W}):
+        state = synth.make_decode_state(spec, dev)
+        n_in = args.warmup + args.steps + 1
+        wins = [synth.make_spec_window(spec, s, w, dev) for s in range(n_in)]
+        accs = [torch.tensor(rng.integers(0, w, B), dtype=torch.int32, device=dev) for _ in range(n_in)]
+        out = torch.empty((B, w, H, dv), dtype=spec.dtype, device=dev)
+        it = iter(range(10 ** 9))
+
+        def step():
+            i = next(it) % (n_in - 1)
+            kda.kda_decode_spec(wins[i], accs[i], wins[i + 1], state, out=out, stream=stream)
+
+        sec = time_loop(step, args.steps, args.warmup, stream, d)
+        times[w] = d.max(sec) / args.steps
+        if w == W:
+            mean_acc = float(torch.stack(accs).float().mean())
+            nbytes = B * H * (2 * dk * dv * 4 + (w + mean_acc) * (2 * (2 * dk + dv) + 4 * dk + 4) + w * 2 * dv)
+            ach = nbytes / times[w] / 1e9
+            res.update(value=job_throughput(d, B * H * w * args.steps, sec) / 1e6, unit=UNIT,
+                       ms_per_step=times[w] * 1e3, mean_accepted=mean_acc, gpu_launches=args.steps,
+                       roofline={"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                 "frac": ach / peaks["hbm_gbs"], "traffic": None, "bytes_per_launch": nbytes,
+                                 "kernel": "kda_spec_kernel<128,128,bf16>"})
+        del wins, accs, state, out
+        torch.cuda.empty_cache()
+    res["ms_per_step_by_window"] = {str(w): t * 1e3 for w, t in sorted(times.items())}
+    return res
 
 
 def bench_e2e(args, d, dev, stream, inp, kda, th):

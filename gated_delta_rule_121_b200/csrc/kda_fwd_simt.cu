@@ -165,7 +165,7 @@ __global__ void __launch_bounds__(DVB * 4)
     for (int e = tid; e < nt * DVB; e += NT) {
       const int r = e / DVB, c = e % DVB;
       const int64_t o = ((t0 + c0 + r) * H + h) * dv + blk * DVB + c;
-      if (MODE == MODE_SEG && !first)
+      if (MODE == MODE_SEG)
         (trans ? ma.qhat32 : ma.o32)[o] = s_o[r][c];
       else
         out[o] = from_f32<IO>(s_o[r][c]);

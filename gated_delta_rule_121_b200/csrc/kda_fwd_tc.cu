@@ -1190,7 +1190,7 @@ __device__ __forceinline__ void scan_group(const Ctx& x, const void* tmq, const 
     const int64_t tok0 = x.t0 + (int64_t)c * CH;
     float o0[32], o1[32];
     tmem_ld32x2(tl + TM_O + (c & 1) * 64, tl + TM_O + (c & 1) * 64 + 32, o0, o1);
-    if (MODE == MODE_SEG && !x.first) {
+    if constexpr (MODE == MODE_SEG) {
       // fp32 outputs straight from the registers: lane j writes channel j of
       // every valid token (a warp stores 128 contiguous bytes per token).
       float* dst = (x.trans ? ma.qhat32 : ma.o32) + (tok0 * H + x.h) * D + j;

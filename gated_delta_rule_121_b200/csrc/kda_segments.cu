@@ -17,7 +17,7 @@
 //     sequence (a sequential prefix, fp32 on CUDA cores, one block per
 //     (sequence, head, 32 value columns): the columns of S evolve
 //     independently), and
-//   - the correction o_t = o~_t + S_in^T qhat_t (dense 128-token x dv tiles on
+//   - the correction o_t = o~_t + S_in^T qhat_t (dense 64-token x dv tiles on
 //     the warp-level tensor path with tf32 operands rounded to nearest; the
 //     zero-start output o~ stays fp32, so the result is rounded once).  For
 //     fp32 outputs, whose contract allows no tf32 rounding, every product is
@@ -112,7 +112,6 @@ __global__ void __launch_bounds__(256)
 }
 
 // ------------------------------------------------------------ correction
-constexpr int CT = 128;       // tokens per block (8 warps x 16 tokens)
 constexpr int CPAD = 4;       // row padding (floats) of the shared tiles: conflict-free fragments
 
 __device__ __forceinline__ uint32_t tf32_rna(float x) {
@@ -132,95 +131,148 @@ __device__ __forceinline__ int piece_of(const int32_t* cu, int P, int64_t t) {
   return lo;
 }
 
-// One block: 128 consecutive tokens x all DV channels of one head.  The
-// tile's qhat rows and zero-start outputs and the piece's incoming state
-// S_in are staged in shared memory with asynchronous copies (one wait), so
-// every global read is in flight at once; each of the 8 warps then owns 16
-// tokens, K = DK in steps of 8.  A tile that straddles pieces is computed once
-// per piece, each pass writing only its own rows.
-template <int DK, int DV, typename IO>
-__global__ void __launch_bounds__(256)
-    correct_kernel(const float* __restrict__ o32, const float* __restrict__ qhat, const float* __restrict__ s_in,
-                   IO* __restrict__ out, const int32_t* __restrict__ cu, int P, int64_t Tper, int64_t Ttot, int H,
-                   int skip_every) {
-  extern __shared__ float csm[];
-  float* s_q = csm;                        // [CT][DK + CPAD]
-  float* s_o = s_q + CT * (DK + CPAD);     // [CT][DV + CPAD]
-  float* s_s = s_o + CT * (DV + CPAD);     // [DK][DV + CPAD]
-  const int h = blockIdx.y;
-  const int64_t t0 = (int64_t)blockIdx.x * CT;
-  const int nt = (int)((Ttot - t0) < CT ? (Ttot - t0) : CT);
-  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, g = lane >> 2, tq = lane & 3;
+// Persistent blocks walk 64-token tiles of one head at a time (tile index
+// i = head * ntiles + tile, strided by the grid), with a two-stage pipeline:
+// while a tile is computed, the next tile's qhat rows and zero-start outputs
+// are already landing in shared memory (asynchronous copies).  The incoming
+// state S_in of a piece is staged once and kept while consecutive tiles stay
+// in that piece.  Each of the 4 warps owns 16 tokens of a tile; K = DK in
+// steps of 8.  A tile that straddles pieces is computed once per piece, each
+// pass writing only its own rows; pieces p with p % skip_every == 0 ran from
+// their initial state, so their (fp32) outputs are only rounded to IO.
+constexpr int TT = 64;  // tokens per tile
 
-  const int p_first = cu ? piece_of(cu, P, t0) : (int)(t0 / Tper);
-  const int p_last = cu ? piece_of(cu, P, t0 + nt - 1) : (int)((t0 + nt - 1) / Tper);
-  // skip_every > 0: pieces p with p % skip_every == 0 already hold their
-  // outputs (first segments run from the initial state)
-  if (skip_every > 0 && p_first == p_last && p_first % skip_every == 0) return;
-  // the tile's qhat rows and zero-start outputs (rows past the end zero-filled)
-  for (int e = tid; e < CT * (DK / 4); e += 256) {
+template <int DK, int DV>
+__device__ __forceinline__ void stage_tile(float* s_q, float* s_o, const float* qhat, const float* o32, int64_t t0,
+                                           int nt, int h, int H) {
+  for (int e = threadIdx.x; e < TT * (DK / 4); e += 128) {
     const int r = e / (DK / 4), c4 = (e % (DK / 4)) * 4;
     const int64_t t = t0 + (r < nt ? r : 0);
     cp_async16(s_q + r * (DK + CPAD) + c4, qhat + (t * H + h) * DK + c4, r < nt ? 16u : 0u);
   }
-  for (int e = tid; e < CT * (DV / 4); e += 256) {
+  for (int e = threadIdx.x; e < TT * (DV / 4); e += 128) {
     const int r = e / (DV / 4), c4 = (e % (DV / 4)) * 4;
     const int64_t t = t0 + (r < nt ? r : 0);
     cp_async16(s_o + r * (DV + CPAD) + c4, o32 + (t * H + h) * DV + c4, r < nt ? 16u : 0u);
   }
-  for (int p = p_first; p <= p_last; ++p) {
-    const int64_t lo = cu ? cu[p] : (int64_t)p * Tper, hi = cu ? cu[p + 1] : (int64_t)(p + 1) * Tper;
-    if (hi <= lo || (skip_every > 0 && p % skip_every == 0)) continue;  // empty, or needs no correction
-    __syncthreads();         // the previous pass is done with s_s
-    const float* S = s_in + ((int64_t)p * H + h) * DK * DV;
-    for (int e = tid; e < DK * (DV / 4); e += 256) {
-      const int r = e / (DV / 4), c4 = (e % (DV / 4)) * 4;
-      cp_async16(s_s + r * (DV + CPAD) + c4, S + r * DV + c4, 16u);
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+template <int DK, int DV, typename IO>
+__global__ void __launch_bounds__(128)
+    correct_kernel(const float* __restrict__ o32, const float* __restrict__ qhat, const float* __restrict__ s_in,
+                   IO* __restrict__ out, const int32_t* __restrict__ cu, int P, int64_t Tper, int64_t Ttot, int H,
+                   int skip_every) {
+  extern __shared__ float csm[];
+  float* s_s = csm;                          // [DK][DV + CPAD]   S_in of the current piece
+  float* s_q0 = s_s + DK * (DV + CPAD);      // [2][TT][DK + CPAD]
+  float* s_o0 = s_q0 + 2 * TT * (DK + CPAD);  // [2][TT][DV + CPAD]
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, g = lane >> 2, tq = lane & 3;
+  const int64_t ntiles = (Ttot + TT - 1) / TT;
+  const int64_t total = ntiles * H;
+  int64_t i = blockIdx.x;
+  if (i >= total) return;
+  int cur_p = -1, cur_h = -1;  // piece/head whose S_in is staged
+  int buf = 0;
+  {
+    const int h = (int)(i / ntiles);
+    const int64_t t0 = (i % ntiles) * TT;
+    stage_tile<DK, DV>(s_q0, s_o0, qhat, o32, t0, (int)((Ttot - t0) < TT ? (Ttot - t0) : TT), h, H);
+  }
+  for (; i < total; i += gridDim.x, buf ^= 1) {
+    const int h = (int)(i / ntiles);
+    const int64_t t0 = (i % ntiles) * TT;
+    const int nt = (int)((Ttot - t0) < TT ? (Ttot - t0) : TT);
+    float* s_q = s_q0 + buf * TT * (DK + CPAD);
+    float* s_o = s_o0 + buf * TT * (DV + CPAD);
+    // prefetch the next tile into the other buffer (its previous reader
+    // finished at the barrier that ended the last iteration)
+    const int64_t inext = i + gridDim.x;
+    if (inext < total) {
+      const int hn = (int)(inext / ntiles);
+      const int64_t tn = (inext % ntiles) * TT;
+      stage_tile<DK, DV>(s_q0 + (buf ^ 1) * TT * (DK + CPAD), s_o0 + (buf ^ 1) * TT * (DV + CPAD), qhat, o32, tn,
+                         (int)((Ttot - tn) < TT ? (Ttot - tn) : TT), hn, H);
+      asm volatile("cp.async.wait_group 1;" ::: "memory");  // this tile's copies have landed
+    } else {
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
     }
-    cp_async_wait_all();  // also completes the tile's rows on the first pass
     __syncthreads();
-    if (w * 16 >= nt) continue;
-    float d[DV / 8][4];
+    const int p_first = cu ? piece_of(cu, P, t0) : (int)(t0 / Tper);
+    const int p_last = cu ? piece_of(cu, P, t0 + nt - 1) : (int)((t0 + nt - 1) / Tper);
+    for (int p = p_first; p <= p_last; ++p) {
+      const int64_t lo = cu ? cu[p] : (int64_t)p * Tper, hi = cu ? cu[p + 1] : (int64_t)(p + 1) * Tper;
+      if (hi <= lo) continue;  // empty piece
+      if (skip_every > 0 && p % skip_every == 0) {  // outputs final: round this piece's rows
+        for (int e = tid; e < nt * (DV / 4); e += 128) {
+          const int r = e / (DV / 4), c4 = (e % (DV / 4)) * 4;
+          const int64_t t = t0 + r;
+          if (t < lo || t >= hi) continue;
+          const float* zo = s_o + r * (DV + CPAD) + c4;
+          const int64_t base = (t * H + h) * DV + c4;
+          out[base] = from_f32<IO>(zo[0]);
+          out[base + 1] = from_f32<IO>(zo[1]);
+          out[base + 2] = from_f32<IO>(zo[2]);
+          out[base + 3] = from_f32<IO>(zo[3]);
+        }
+        continue;
+      }
+      if (p != cur_p || h != cur_h) {  // stage this piece's S_in (kept for the next tiles)
+        __syncthreads();               // every warp is done with the previous S_in
+        const float* S = s_in + ((int64_t)p * H + h) * DK * DV;
+        for (int e = tid; e < DK * (DV / 4); e += 128) {
+          const int r = e / (DV / 4), c4 = (e % (DV / 4)) * 4;
+          *reinterpret_cast<float4*>(s_s + r * (DV + CPAD) + c4) = __ldg(reinterpret_cast<const float4*>(S + r * DV + c4));
+        }
+        __syncthreads();
+        cur_p = p;
+        cur_h = h;
+      }
+      if (w * 16 >= nt) continue;
+      float d[DV / 8][4];
 #pragma unroll
-    for (int n = 0; n < DV / 8; ++n) d[n][0] = d[n][1] = d[n][2] = d[n][3] = 0.f;
-    const float* qa = s_q + (w * 16) * (DK + CPAD);
-    constexpr bool SPLIT = sizeof(IO) == 4;  // fp32 outputs: three-term tf32 products
+      for (int n = 0; n < DV / 8; ++n) d[n][0] = d[n][1] = d[n][2] = d[n][3] = 0.f;
+      const float* qa = s_q + (w * 16) * (DK + CPAD);
+      constexpr bool SPLIT = sizeof(IO) == 4;  // fp32 outputs: three-term tf32 products
 #pragma unroll 2
-    for (int k0 = 0; k0 < DK; k0 += 8) {
-      const float af[4] = {qa[g * (DK + CPAD) + k0 + tq], qa[(g + 8) * (DK + CPAD) + k0 + tq],
-                           qa[g * (DK + CPAD) + k0 + tq + 4], qa[(g + 8) * (DK + CPAD) + k0 + tq + 4]};
-      uint32_t a[4], al[4];
+      for (int k0 = 0; k0 < DK; k0 += 8) {
+        const float af[4] = {qa[g * (DK + CPAD) + k0 + tq], qa[(g + 8) * (DK + CPAD) + k0 + tq],
+                             qa[g * (DK + CPAD) + k0 + tq + 4], qa[(g + 8) * (DK + CPAD) + k0 + tq + 4]};
+        uint32_t a[4], al[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        a[i] = tf32_rna(af[i]);
-        if (SPLIT) al[i] = tf32_rna(af[i] - __uint_as_float(a[i]));
+        for (int j = 0; j < 4; ++j) {
+          a[j] = tf32_rna(af[j]);
+          if (SPLIT) al[j] = tf32_rna(af[j] - __uint_as_float(a[j]));
+        }
+#pragma unroll
+        for (int n = 0; n < DV / 8; ++n) {
+          const float bf[2] = {s_s[(k0 + tq) * (DV + CPAD) + n * 8 + g],
+                               s_s[(k0 + tq + 4) * (DV + CPAD) + n * 8 + g]};
+          uint32_t bb[2] = {tf32_rna(bf[0]), tf32_rna(bf[1])};
+          mma_tf32_16x8x8(d[n], a, bb);
+          if (SPLIT) {
+            const uint32_t bl[2] = {tf32_rna(bf[0] - __uint_as_float(bb[0])), tf32_rna(bf[1] - __uint_as_float(bb[1]))};
+            mma_tf32_16x8x8(d[n], a, bl);
+            mma_tf32_16x8x8(d[n], al, bb);
+          }
+        }
       }
 #pragma unroll
-      for (int n = 0; n < DV / 8; ++n) {
-        const float bf[2] = {s_s[(k0 + tq) * (DV + CPAD) + n * 8 + g], s_s[(k0 + tq + 4) * (DV + CPAD) + n * 8 + g]};
-        uint32_t b[2] = {tf32_rna(bf[0]), tf32_rna(bf[1])};
-        mma_tf32_16x8x8(d[n], a, b);
-        if (SPLIT) {
-          const uint32_t bl[2] = {tf32_rna(bf[0] - __uint_as_float(b[0])), tf32_rna(bf[1] - __uint_as_float(b[1]))};
-          mma_tf32_16x8x8(d[n], a, bl);
-          mma_tf32_16x8x8(d[n], al, b);
+      for (int half = 0; half < 2; ++half) {
+        const int r = w * 16 + g + 8 * half;
+        const int64_t t = t0 + r;
+        if (r >= nt || t < lo || t >= hi) continue;
+        const int64_t base = (t * H + h) * DV;
+        const float* zo = s_o + r * (DV + CPAD);
+#pragma unroll
+        for (int n = 0; n < DV / 8; ++n) {
+          const int c = n * 8 + 2 * tq;
+          out[base + c] = from_f32<IO>(zo[c] + d[n][2 * half]);
+          out[base + c + 1] = from_f32<IO>(zo[c + 1] + d[n][2 * half + 1]);
         }
       }
     }
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      const int r = w * 16 + g + 8 * half;
-      const int64_t t = t0 + r;
-      if (r >= nt || t < lo || t >= hi) continue;
-      const int64_t base = (t * H + h) * DV;
-      const float* zo = s_o + r * (DV + CPAD);
-#pragma unroll
-      for (int n = 0; n < DV / 8; ++n) {
-        const int c = n * 8 + 2 * tq;
-        out[base + c] = from_f32<IO>(zo[c] + d[n][2 * half]);
-        out[base + c + 1] = from_f32<IO>(zo[c + 1] + d[n][2 * half + 1]);
-      }
-    }
+    __syncthreads();  // the buffer of this tile may be refilled next iteration
   }
   cp_async_wait_all();  // no copy may still be landing when the block leaves
 }
@@ -261,13 +313,16 @@ template <int DK, int DV, typename IO>
 cudaError_t correct_t(const float* o32, const float* qhat, const float* s_in, void* out, const int32_t* cu, int P,
                       int64_t Tper, int64_t Ttot, int H, int skip_every, cudaStream_t s) {
   if (Ttot == 0) return cudaSuccess;
-  const size_t smem =
-      sizeof(float) * ((size_t)CT * (DK + CPAD) + (size_t)CT * (DV + CPAD) + (size_t)DK * (DV + CPAD));
+  const size_t smem = sizeof(float) * ((size_t)DK * (DV + CPAD) + 2 * (size_t)TT * (DK + CPAD) +
+                                       2 * (size_t)TT * (DV + CPAD));
   auto* kern = correct_kernel<DK, DV, IO>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((unsigned)((Ttot + CT - 1) / CT), (unsigned)H);
-  kern<<<grid, 256, smem, s>>>(o32, qhat, s_in, (IO*)out, cu, P, Tper, Ttot, H, skip_every);
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t tiles = (Ttot + TT - 1) / TT * H;
+  const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);  // one persistent block per SM
+  kern<<<grid, 128, smem, s>>>(o32, qhat, s_in, (IO*)out, cu, P, Tper, Ttot, H, skip_every);
   return cudaGetLastError();
 }
 

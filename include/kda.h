@@ -388,10 +388,13 @@ KDA_API kda_status_t kda_decode_step_gated(const void *q, const void *k, const v
  *   out        [B, W, H, dv]: the outputs of the W new tokens (each read with
  *              the state after that token)
  * The rejected drafts of the previous window are never applied; the new
- * drafts' states stay on chip.  Wp + W <= KDA_SPEC_MAX_TOKENS.  W = 0 only
- * replays.  No workspace.
+ * drafts' states stay on chip.  The replayed and new tokens are taken as one
+ * chunk (the chunkwise form of the recurrence, fp32), so the state is read
+ * once and written once whatever the window.  Wp + W <= KDA_SPEC_MAX_TOKENS
+ * (else KDA_ERR_UNSUPPORTED).  W = 0 only replays (and keeps the state after
+ * the accepted drafts).  No workspace.
  */
-#define KDA_SPEC_MAX_TOKENS 64
+#define KDA_SPEC_MAX_TOKENS 16
 KDA_API kda_status_t kda_decode_spec(const void *q_prev, const void *k_prev, const void *v_prev,
                                      const float *log_alpha_prev, const float *beta_prev,
                                      const int32_t *n_accepted,
