@@ -249,7 +249,7 @@ def job_throughput(d, units, seconds):
 def workload_spec(name):
     import synth
     return {"prefill64k": synth.PRETRAIN, "mid": synth.MID, "varlen": synth.VARLEN,
-            "stress": synth.STRESS}[name]
+            "stress": synth.STRESS, "tp4": synth.TP4}[name]
 
 
 # ----------------------------------------------------------------- oracle arm
@@ -310,7 +310,7 @@ TRAFFIC_PROFILES = {
     "kda_fwd_tc_kernel": ("kda_fwd_tc_prefill_h96_t4096_traffic.txt", "kda_fwd_tc.cu"),
     "kda_decode_kernel": ("kda_decode_b64_h96_traffic.txt", "kda_decode.cu"),
 }
-FLUSH = {"mid": True, "stress": True, "prefill64k": False, "varlen": False}
+FLUSH = {"mid": True, "stress": True, "prefill64k": False, "varlen": False, "tp4": False}
 
 
 def bench_prefill(name, d, dev, stream, peaks, kda, synth, steps, warmup, with_traffic=False, variant=None):
@@ -341,7 +341,7 @@ def bench_prefill(name, d, dev, stream, peaks, kda, synth, steps, warmup, with_t
         n_seg = kda.kda_cp_segments(N, (B * T) // N, H)
         ws = kda.alloc_cp_workspace(N, B * T, H, dk, dv, n_seg, q.dtype, dev)
         extra["n_seg"] = n_seg
-        launches = 5  # segment offsets, order, segment pieces, composition, correction
+        launches = 6  # segment offsets, order, state pass, composition, order, forward
 
         def step():
             kda.kda_fwd_cp(q, k, v, g, beta, init, cu, n_seg=n_seg, out=out, final_state=fin, workspace=ws,
@@ -443,6 +443,7 @@ def run_native(args, d):
     if not args.no_workloads:
         others = {}
         for key, name, steps, variant in (("mid", "mid", 50, None), ("mid_cp", "mid", 50, "cp"),
+                                          ("tp4", "tp4", 10, None), ("tp4_cp", "tp4", 20, "cp"),
                                           ("varlen", "varlen", 8, None), ("stress", "stress", 50, None),
                                           ("prefill64k_ckpt512", "prefill64k", 10, "ckpt512"),
                                           ("prefill64k_gated", "prefill64k", 10, "gated")):
@@ -689,7 +690,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
-    ap.add_argument("--workload", choices=["prefill64k", "mid", "varlen", "stress"], default="prefill64k")
+    ap.add_argument("--workload", choices=["prefill64k", "mid", "varlen", "stress", "tp4"], default="prefill64k")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -13,7 +13,7 @@ cudaError_t launch_fwd_tc_impl(const FwdArgs& a, cudaStream_t s, uint64_t wait_n
                                int32_t* order_ws, const ModeArgs& ma);
 cudaError_t launch_ckpt_base(const int32_t* cu, int N, int interval, int32_t* base, cudaStream_t s);
 cudaError_t launch_compose(const float* trans, const float* s0, const float* init, float* state_in, float* fin,
-                           int R, int N, int H, int dk, int dv, int rank_major, int first_from_init,
+                           int R, int N, int H, int dk, int dv, int rank_major, int first_from_init, int apply_last,
                            cudaStream_t s);
 cudaError_t launch_correct(const float* o32, const float* qhat, const float* s_in, void* out, const int32_t* cu,
                            int P, int64_t Tper, int64_t Ttot, int H, int dk, int dv, bool bf16, int skip_every,
@@ -76,7 +76,7 @@ static kda_status_t fwd_impl(const void* q, const void* k, const void* v, const 
                              kda_dtype_t dt, void* workspace, size_t workspace_bytes, float* dbg,
                              uint64_t wait_ns, int inject_stuck, const kda::ModeArgs& ma = kda::ModeArgs()) {
   // Segment runs write fp32 outputs to their own buffers (out may be NULL).
-  const void* out_chk = ma.mode == kda::MODE_SEG ? (const void*)ma.o32 : out;
+  const void* out_chk = ma.mode == kda::MODE_SEG ? (const void*)(ma.o32 ? ma.o32 : final_state) : out;
   kda_status_t st = validate_fwd(q, k, v, log_alpha, beta, init_state, out_chk, final_state, B, T, H, dk, dv, dt);
   if (st != KDA_OK) return st;
   if (cu_seqlens && !aligned16(cu_seqlens)) return KDA_ERR_INVALID_ARG;
@@ -299,8 +299,8 @@ kda_status_t kda_segment_fwd(const void* q, const void* k, const void* v, const 
                              const int32_t* cu_seqlens, void* stream, kda_dtype_t dt, void* workspace,
                              size_t workspace_bytes) {
   if (dk != dv) return KDA_ERR_UNSUPPORTED;
-  const int64_t tokens = cu_seqlens ? T : (int64_t)B * T;
-  if (tokens > 0 && (!out_zero || !qhat)) return KDA_ERR_INVALID_ARG;
+  // out_zero and qhat are both set, or both NULL (states only)
+  if ((out_zero == nullptr) != (qhat == nullptr)) return KDA_ERR_INVALID_ARG;
   if (B > 0 && (!state_zero || !transition)) return KDA_ERR_INVALID_ARG;
   for (const void* p : {(const void*)out_zero, (const void*)qhat, (const void*)state_zero, (const void*)transition})
     if (!aligned16(p)) return KDA_ERR_INVALID_ARG;
@@ -324,7 +324,7 @@ kda_status_t kda_state_compose(const float* transition, const float* state_zero,
     if (!aligned16(p)) return KDA_ERR_INVALID_ARG;
   if (N == 0) return KDA_OK;
   cudaError_t e = kda::launch_compose(transition, state_zero, init_state, state_in, final_state, R, N, H, dk, dv,
-                                      rank_major ? 1 : 0, 0, reinterpret_cast<cudaStream_t>(stream));
+                                      rank_major ? 1 : 0, 0, 1, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
@@ -348,40 +348,42 @@ kda_status_t kda_output_correct(const float* out_zero, const float* qhat, const 
 // ---- intra-device context parallelism ----
 namespace {
 struct CpLayout {
-  size_t seg_cu, order, o32, qhat, s0, trans, s_in, total;
+  size_t seg_cu, order, s0, trans, s_in, fin, total;
 };
-CpLayout cp_layout(int B, int64_t T, int H, int dk, int dv, int n_seg) {
+CpLayout cp_layout(int B, int H, int dk, int dv, int n_seg) {
   auto up = [](size_t x) { return (x + 255) / 256 * 256; };
-  const int64_t tokens = T;  // caller passes the total token count (B*T for batched inputs)
   const size_t P = (size_t)(B > 0 ? B : 0) * (size_t)(n_seg > 0 ? n_seg : 1);
+  const size_t st = P * H * (size_t)dk * dv * sizeof(float);
   CpLayout L;
   size_t off = kStatusBytes;
   L.seg_cu = off; off += up((P + 1) * sizeof(int32_t));
   L.order = off; off += up(P * sizeof(int32_t));
-  L.o32 = off; off += up((size_t)tokens * H * dv * sizeof(float));
-  L.qhat = off; off += up((size_t)tokens * H * dk * sizeof(float));
-  L.s0 = off; off += up(P * H * (size_t)dk * dv * sizeof(float));
+  L.s0 = off; off += up(st);
   L.trans = off; off += up(P * H * (size_t)dk * dk * sizeof(float));
-  L.s_in = off; off += up(P * H * (size_t)dk * dv * sizeof(float));
+  L.s_in = off; off += up(st);
+  L.fin = off; off += up(st);
   L.total = off;
   return L;
 }
 }  // namespace
 
 size_t kda_fwd_cp_workspace_size(int B, int64_t T, int H, int dk, int dv, kda_dtype_t dt, int n_seg) {
-  (void)dt;
-  return cp_layout(B, T, H, dk, dv, n_seg).total;
+  (void)T; (void)dt;
+  return cp_layout(B, H, dk, dv, n_seg).total;
 }
 
 int kda_cp_segments(int N, int64_t tokens_per_sequence, int H, int sm_count) {
-  // Two blocks per (segment, head) (the zero-start run and the transition run)
-  // must fit one wave of blocks on the SMs; a segment should keep at least
-  // eight 64-token chunks so the pipeline fill stays small against its length.
+  // The state pass runs 2 n_seg - 3 blocks per (sequence, head) for n_seg >= 2
+  // (the first segment from its initial state, the middle ones as zero-start
+  // and transition runs, the last one not at all) and the output pass n_seg;
+  // both must fit one wave of blocks on the SMs.  A segment keeps at least
+  // eight 64-token chunks, and the split must shorten the serial depth:
+  // two passes of L / n_seg each against one of L.
   const int64_t chains = (int64_t)N * H;
   if (chains <= 0 || sm_count <= 0) return 1;
   int best = 1;
-  for (int r = 2; r <= 64; ++r) {
-    if (2 * chains * r > sm_count) break;
+  for (int r = 3; r <= 64; ++r) {
+    if (chains * (2 * r - 3) > sm_count || chains * r > sm_count) break;
     if (tokens_per_sequence / r < 8 * 64) break;
     best = r;
   }
@@ -399,7 +401,7 @@ kda_status_t kda_fwd_cp(const void* q, const void* k, const void* v, const float
   if (cu_seqlens && !aligned16(cu_seqlens)) return KDA_ERR_INVALID_ARG;
   const int64_t tokens = cu_seqlens ? T : (int64_t)B * T;
   if (tokens > (int64_t)INT32_MAX || (int64_t)B * n_seg > (int64_t)INT32_MAX / 4) return KDA_ERR_UNSUPPORTED;
-  const CpLayout L = cp_layout(B, tokens, H, dk, dv, n_seg);
+  const CpLayout L = cp_layout(B, H, dk, dv, n_seg);
   if (!workspace || !aligned16(workspace) || workspace_bytes < L.total) return KDA_ERR_WORKSPACE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
@@ -407,34 +409,47 @@ kda_status_t kda_fwd_cp(const void* q, const void* k, const void* v, const float
   if (B == 0) return KDA_OK;
   const int P = B * n_seg;
   int32_t* seg_cu = reinterpret_cast<int32_t*>(ws + L.seg_cu);
-  float* o32 = reinterpret_cast<float*>(ws + L.o32);
-  float* qhat = reinterpret_cast<float*>(ws + L.qhat);
+  int32_t* order = reinterpret_cast<int32_t*>(ws + L.order);
   float* s0 = reinterpret_cast<float*>(ws + L.s0);
   float* tr = reinterpret_cast<float*>(ws + L.trans);
   float* s_in = reinterpret_cast<float*>(ws + L.s_in);
+  float* fin_seg = reinterpret_cast<float*>(ws + L.fin);
+  kda::DeviceStatus* status = reinterpret_cast<kda::DeviceStatus*>(ws);
+  const bool tc = kda::fwd_tc_supported(dk, dv, dt == KDA_BF16) && tokens > 0;
+  const bool bf16 = dt == KDA_BF16;
   if (kda::launch_segment_cu(cu_seqlens, cu_seqlens ? 0 : T, B, n_seg, seg_cu, s) != cudaSuccess)
     return KDA_ERR_CUDA;
-  // Pieces of every segment: the segments form a packed batch of P sequences
-  // over the same token tensors.  The status word of the workspace is shared;
-  // the order scratch follows it (L.order == kStatusBytes + aligned seg_cu).
-  kda::ModeArgs ma;
-  ma.mode = kda::MODE_SEG;
-  ma.o32 = o32;
-  ma.qhat32 = qhat;
-  ma.trans = tr;
-  ma.seg_per_seq = n_seg;  // first segments run from init_state into `out` directly
-  kda::FwdArgs a{q, k, v, log_alpha, beta, init_state, out, s0, seg_cu, P, tokens, H, dk, dv,
-                 reinterpret_cast<kda::DeviceStatus*>(ws), nullptr};
-  cudaError_t e;
-  if (kda::fwd_tc_supported(dk, dv, dt == KDA_BF16) && tokens > 0)
-    e = kda::launch_fwd_tc_impl(a, s, 2000000000ull, 0, reinterpret_cast<int32_t*>(ws + L.order), ma);
-  else
-    e = kda::launch_fwd_simt(a, dt == KDA_BF16, s, ma);
+  cudaError_t e = cudaSuccess;
+  // Pass 1 (states only): the first segment of every sequence from its
+  // initial state, the middle ones as zero-start and transition runs; the
+  // segments form a packed batch of P sequences over the same token tensors.
+  if (n_seg > 1) {
+    kda::ModeArgs ma;
+    ma.mode = kda::MODE_SEG;
+    ma.seg_per_seq = n_seg;
+    ma.trans = tr;
+    kda::FwdArgs a{q, k, v, log_alpha, beta, init_state, nullptr, s0, seg_cu, P, tokens, H, dk, dv, status, nullptr};
+    e = tc ? kda::launch_fwd_tc_impl(a, s, 2000000000ull, 0, order, ma) : kda::launch_fwd_simt(a, bf16, s, ma);
+    if (e != cudaSuccess) return KDA_ERR_CUDA;
+  }
+  // Every segment's incoming state: S_in(0) = init, S_in(1) = the first
+  // segment's state, S_in(r+1) = S~_r + M_r S_in(r).
+  e = kda::launch_compose(tr, s0, init_state, s_in, nullptr, n_seg, B, H, dk, dv, 0, 1, 0, s);
   if (e != cudaSuccess) return KDA_ERR_CUDA;
-  e = kda::launch_compose(tr, s0, init_state, s_in, final_state, n_seg, B, H, dk, dv, 0, 1, s);
+  // Pass 2: the ordinary forward over all segments from their incoming states.
+  kda::FwdArgs a2{q, k, v, log_alpha, beta, s_in, out, final_state ? fin_seg : nullptr, seg_cu, P, tokens, H, dk, dv,
+                  status, nullptr};
+  e = tc ? kda::launch_fwd_tc_impl(a2, s, 2000000000ull, 0, order, kda::ModeArgs())
+         : kda::launch_fwd_simt(a2, bf16, s);
   if (e != cudaSuccess) return KDA_ERR_CUDA;
-  e = kda::launch_correct(o32, qhat, s_in, out, seg_cu, P, 0, tokens, H, dk, dv, dt == KDA_BF16, n_seg, s);
-  return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+  // The final state of each sequence is the one after its last segment.
+  if (final_state) {
+    const size_t head_states = (size_t)H * dk * dv * sizeof(float);
+    if (cudaMemcpy2DAsync(final_state, head_states, fin_seg + (size_t)(n_seg - 1) * H * dk * dv,
+                          head_states * n_seg, head_states, B, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+      return KDA_ERR_CUDA;
+  }
+  return KDA_OK;
 }
 
 // ---- test hooks (include/kda_testing.h) ----

@@ -55,7 +55,9 @@ __global__ void __launch_bounds__(DVB * 4)
   // MODE_SEG: a sequence's first segment runs from its initial state with
   // ordinary outputs and needs no transition run.
   const bool first = MODE == MODE_SEG && ma.seg_per_seq > 0 && n % ma.seg_per_seq == 0;
-  if (first && trans) return;
+  const bool last = MODE == MODE_SEG && ma.seg_per_seq > 0 && n % ma.seg_per_seq == ma.seg_per_seq - 1;
+  if ((first && trans) || (last && !first)) return;
+  float* const obuf = trans ? ma.qhat32 : ma.o32;  // MODE_SEG: null = states only
   if (MODE == MODE_SEG && !first) init = nullptr;
   int64_t t0, L;
   if (cu) {
@@ -165,10 +167,11 @@ __global__ void __launch_bounds__(DVB * 4)
     for (int e = tid; e < nt * DVB; e += NT) {
       const int r = e / DVB, c = e % DVB;
       const int64_t o = ((t0 + c0 + r) * H + h) * dv + blk * DVB + c;
-      if (MODE == MODE_SEG)
-        (trans ? ma.qhat32 : ma.o32)[o] = s_o[r][c];
-      else
+      if (MODE == MODE_SEG) {
+        if (obuf) obuf[o] = s_o[r][c];
+      } else {
         out[o] = from_f32<IO>(s_o[r][c]);
+      }
     }
   }
   if (fin) {

@@ -1193,7 +1193,9 @@ __device__ __forceinline__ void scan_group(const Ctx& x, const void* tmq, const 
     if constexpr (MODE == MODE_SEG) {
       // fp32 outputs straight from the registers: lane j writes channel j of
       // every valid token (a warp stores 128 contiguous bytes per token).
-      float* dst = (x.trans ? ma.qhat32 : ma.o32) + (tok0 * H + x.h) * D + j;
+      float* obuf = x.trans ? ma.qhat32 : ma.o32;
+      if (!obuf) return;  // states only
+      float* dst = obuf + (tok0 * H + x.h) * D + j;
       const int64_t st = (int64_t)H * D;
       const float sc = x.trans ? TRANS_UNSCALE : 1.f;
 #pragma unroll
@@ -1491,7 +1493,10 @@ __global__ void __launch_bounds__(NTHR, 1)
   int64_t ibase = ((int64_t)n * H + x.h) * D * D;  // initial state of this chain
   if constexpr (MODE == MODE_SEG) {
     x.first = ma.seg_per_seq > 0 && n % ma.seg_per_seq == 0;
-    if (x.first && x.trans) return;  // a first segment needs no transition (the whole block leaves)
+    const bool last = ma.seg_per_seq > 0 && n % ma.seg_per_seq == ma.seg_per_seq - 1;
+    // a first segment needs no transition and a last segment no pieces at all
+    // (the whole block leaves before it allocates anything)
+    if ((x.first && x.trans) || (last && !x.first)) return;
     if (x.first) ibase = ((int64_t)(n / ma.seg_per_seq) * H + x.h) * D * D;
   }
   if (cu) {

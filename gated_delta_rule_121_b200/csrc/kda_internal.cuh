@@ -77,8 +77,10 @@ struct ModeArgs {
   float* trans = nullptr;   // [N][H][dk][dk]
   int seg_per_seq = 0;      // > 0: the batch is N/seg_per_seq sequences cut into that many
                             // consecutive segments; the first segment of each runs from the
-                            // sequence's initial state (its fp32 outputs are final) and has
-                            // no transition run
+                            // sequence's initial state and has no transition run, and the
+                            // last segment of each is skipped (its pieces are not needed)
+                            // Outputs of MODE_SEG runs are written only when o32 / qhat32 are
+                            // set (kda_fwd_cp needs states only).
   // MODE_GATED
   const float* A_log = nullptr;  // [H] per-head log scale of the decay logits
   float g_min = -5.0f;           // lower bound of the log decay

@@ -51,7 +51,7 @@ template <int DK>
 __global__ void __launch_bounds__(256)
     compose_kernel(const float* __restrict__ trans, const float* __restrict__ s0, const float* __restrict__ init,
                    float* __restrict__ state_in, float* __restrict__ fin, int R, int N, int H, int dv,
-                   int rank_major, int first_from_init) {
+                   int rank_major, int first_from_init, int apply_last) {
   constexpr int RPT = DK / 8;  // rows per thread: warp w holds rows w, w + 8, ...
   extern __shared__ float cm[];
   float* s_m = cm;                        // [DK][DK + 4]
@@ -77,6 +77,12 @@ __global__ void __launch_bounds__(256)
     // first_from_init: piece 0 already ran from the initial state, so its
     // "zero-start" state is the state after it and it has no transition.
     const bool skip_m = first_from_init && r == 0;
+    if (r == R - 1 && !apply_last) {  // the last piece's incoming state is all that is wanted
+#pragma unroll
+      for (int u = 0; u < RPT; ++u)
+        if (col && state_in) state_in[ph * sd + (int64_t)(w + 8 * u) * dv + c] = cur[u];
+      break;
+    }
     const float* Mp = trans + ph * mm;
     if (!skip_m) {
       for (int e = threadIdx.x; e < DK * DK / 4; e += 256) {
@@ -104,7 +110,7 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
     for (int u = 0; u < RPT; ++u) cur[u] = acc[u];
   }
-  if (fin && col) {
+  if (fin && col && apply_last) {
 #pragma unroll
     for (int u = 0; u < RPT; ++u)
       fin[((int64_t)m * H + h) * sd + (int64_t)(w + 8 * u) * dv + c] = cur[u];
@@ -131,8 +137,9 @@ __device__ __forceinline__ int piece_of(const int32_t* cu, int P, int64_t t) {
   return lo;
 }
 
-// Persistent blocks walk 64-token tiles of one head at a time (tile index
-// i = head * ntiles + tile, strided by the grid), with a two-stage pipeline:
+// Persistent blocks walk 64-token tiles (tile index i = head * ntiles +
+// tile; block b takes a contiguous range of them, so consecutive tiles
+// usually share the head and the piece), with a two-stage pipeline:
 // while a tile is computed, the next tile's qhat rows and zero-start outputs
 // are already landing in shared memory (asynchronous copies).  The incoming
 // state S_in of a piece is staged once and kept while consecutive tiles stay
@@ -170,8 +177,10 @@ __global__ void __launch_bounds__(128)
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, g = lane >> 2, tq = lane & 3;
   const int64_t ntiles = (Ttot + TT - 1) / TT;
   const int64_t total = ntiles * H;
-  int64_t i = blockIdx.x;
-  if (i >= total) return;
+  const int64_t per = (total + gridDim.x - 1) / gridDim.x;
+  int64_t i = (int64_t)blockIdx.x * per;
+  const int64_t iend = i + per < total ? i + per : total;
+  if (i >= iend) return;
   int cur_p = -1, cur_h = -1;  // piece/head whose S_in is staged
   int buf = 0;
   {
@@ -179,7 +188,7 @@ __global__ void __launch_bounds__(128)
     const int64_t t0 = (i % ntiles) * TT;
     stage_tile<DK, DV>(s_q0, s_o0, qhat, o32, t0, (int)((Ttot - t0) < TT ? (Ttot - t0) : TT), h, H);
   }
-  for (; i < total; i += gridDim.x, buf ^= 1) {
+  for (; i < iend; ++i, buf ^= 1) {
     const int h = (int)(i / ntiles);
     const int64_t t0 = (i % ntiles) * TT;
     const int nt = (int)((Ttot - t0) < TT ? (Ttot - t0) : TT);
@@ -187,8 +196,8 @@ __global__ void __launch_bounds__(128)
     float* s_o = s_o0 + buf * TT * (DV + CPAD);
     // prefetch the next tile into the other buffer (its previous reader
     // finished at the barrier that ended the last iteration)
-    const int64_t inext = i + gridDim.x;
-    if (inext < total) {
+    const int64_t inext = i + 1;
+    if (inext < iend) {
       const int hn = (int)(inext / ntiles);
       const int64_t tn = (inext % ntiles) * TT;
       stage_tile<DK, DV>(s_q0 + (buf ^ 1) * TT * (DK + CPAD), s_o0 + (buf ^ 1) * TT * (DV + CPAD), qhat, o32, tn,
@@ -297,7 +306,7 @@ __global__ void segment_cu_kernel(const int32_t* __restrict__ cu, int64_t Tper, 
 
 template <int DK>
 cudaError_t compose_dk(const float* trans, const float* s0, const float* init, float* state_in, float* fin, int R,
-                       int N, int H, int dv, int rank_major, int first_from_init, cudaStream_t s) {
+                       int N, int H, int dv, int rank_major, int first_from_init, int apply_last, cudaStream_t s) {
   const int ncb = (dv + 31) / 32;
   const int64_t blocks = (int64_t)N * H * ncb;
   if (blocks == 0) return cudaSuccess;
@@ -305,7 +314,7 @@ cudaError_t compose_dk(const float* trans, const float* s0, const float* init, f
   cudaError_t e = cudaFuncSetAttribute(compose_kernel<DK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   compose_kernel<DK><<<(unsigned)blocks, 256, smem, s>>>(trans, s0, init, state_in, fin, R, N, H, dv, rank_major,
-                                                          first_from_init);
+                                                          first_from_init, apply_last);
   return cudaGetLastError();
 }
 
@@ -341,13 +350,13 @@ cudaError_t correct_dv(const float* o32, const float* qhat, const float* s_in, v
 }  // namespace
 
 cudaError_t launch_compose(const float* trans, const float* s0, const float* init, float* state_in, float* fin,
-                           int R, int N, int H, int dk, int dv, int rank_major, int first_from_init,
+                           int R, int N, int H, int dk, int dv, int rank_major, int first_from_init, int apply_last,
                            cudaStream_t s) {
   switch (dk) {
-    case 16: return compose_dk<16>(trans, s0, init, state_in, fin, R, N, H, dv, rank_major, first_from_init, s);
-    case 32: return compose_dk<32>(trans, s0, init, state_in, fin, R, N, H, dv, rank_major, first_from_init, s);
-    case 64: return compose_dk<64>(trans, s0, init, state_in, fin, R, N, H, dv, rank_major, first_from_init, s);
-    case 128: return compose_dk<128>(trans, s0, init, state_in, fin, R, N, H, dv, rank_major, first_from_init, s);
+    case 16: return compose_dk<16>(trans, s0, init, state_in, fin, R, N, H, dv, rank_major, first_from_init, apply_last, s);
+    case 32: return compose_dk<32>(trans, s0, init, state_in, fin, R, N, H, dv, rank_major, first_from_init, apply_last, s);
+    case 64: return compose_dk<64>(trans, s0, init, state_in, fin, R, N, H, dv, rank_major, first_from_init, apply_last, s);
+    case 128: return compose_dk<128>(trans, s0, init, state_in, fin, R, N, H, dv, rank_major, first_from_init, apply_last, s);
   }
   return cudaErrorInvalidValue;
 }

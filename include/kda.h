@@ -330,16 +330,23 @@ KDA_API kda_status_t kda_output_correct(const float *out_zero, const float *qhat
  *
  * Same arguments and results as kda_fwd, plus n_seg: every sequence is cut
  * into n_seg segments of near-equal length (at tokens start + floor(L r /
- * n_seg), anywhere inside a 64-token chunk).  One launch computes the pieces
- * of all segments (kda_segment_fwd), then kda_state_compose gives every
- * segment's incoming state and the final state, and kda_output_correct the
- * outputs.  Requires dk == dv.  n_seg = 1 is valid (one segment).
+ * n_seg), anywhere inside a 64-token chunk).  Three steps on `stream`:
+ *   1. a state pass over all segments at once: the first segment of each
+ *      sequence runs from its initial state, every middle segment as a
+ *      zero-start run (S~) and a transition run (M), the last segment not at
+ *      all; no outputs are written;
+ *   2. the composition S_in(r+1) = S~_r + M_r S_in(r) (kda_state_compose's
+ *      kernel) gives every segment's incoming state;
+ *   3. the ordinary forward (kda_fwd's kernel) over all segments from those
+ *      states, writing `out` and the final state.
+ * So the serial depth falls from L to about 2 L / n_seg tokens, at the price
+ * of about three times the forward work on the middle segments.
+ * Requires dk == dv.  n_seg = 1 is the plain forward.
  *   workspace  at least kda_fwd_cp_workspace_size(B, T_total, ..., n_seg)
- *              bytes, where T_total is the token count (B*T for batched
- *              inputs, T when packed); it holds the fp32 pieces: about
- *              T_total * H * (dk + dv) * 4 bytes plus 3 states per segment.
- * Worth it when 2 * N * H * n_seg blocks fit one wave on the device and the
- * chains are few (kda_cp_segments suggests n_seg).
+ *              bytes: four fp32 states per (segment, head) and the segment
+ *              offsets (T_total, the token count, is not needed for the size).
+ * Worth it when the chains are few: kda_cp_segments(N, L, H, sm_count) gives
+ * the largest n_seg whose passes fit one wave of blocks (1 when none does).
  */
 KDA_API size_t kda_fwd_cp_workspace_size(int B, int64_t T_total, int H, int dk, int dv, kda_dtype_t dt,
                                          int n_seg);

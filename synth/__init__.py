@@ -70,8 +70,11 @@ VARLEN = PrefillSpec("varlen_bf16_H32_T1048576_d128", 1, 1 << 20, 32, 128, 128, 
 STRESS = PrefillSpec("stress_bf16_B2_H16_T1024_d128_gmin5", 2, 1024, 16, 128, 128, torch.bfloat16, 5,
                      g_scale=5.0, init=True)
 DECODE = DecodeSpec("decode_bf16_B512_H96_d128", 512, 96, 128, 128, torch.bfloat16, 4, 256)
+# One tensor-parallel rank's share of the 64K prefill: 4 of the model's 96 heads
+# (24-way head split), the case where the chains are far fewer than the SMs.
+TP4 = PrefillSpec("tp4_bf16_B1_H4_T65536_d128", 1, 65536, 4, 128, 128, torch.bfloat16, 6)
 
-PREFILL_SPECS = {s.name: s for s in (TINY, MID, PRETRAIN, VARLEN, STRESS)}
+PREFILL_SPECS = {s.name: s for s in (TINY, MID, PRETRAIN, VARLEN, STRESS, TP4)}
 
 
 def varlen_lengths(total: int, lo: int, hi: int, seed: int) -> list[int]:

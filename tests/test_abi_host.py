@@ -141,8 +141,8 @@ def test_new_entry_points_reject_invalid_arguments_on_the_host():
     assert L.kda_fwd_cp(*fwd, 0, P(8192), 1 << 30) == kda.KDA_ERR_INVALID_ARG
     assert L.kda_fwd_cp(*cp, P(8192), 64) == kda.KDA_ERR_WORKSPACE
     need = L.kda_fwd_cp_workspace_size(1, 64, 2, 128, 128, kda.KDA_BF16, 2)
-    assert need >= 64 * 2 * 256 * 4
-    assert L.kda_cp_segments(2, 4096, 16, 148) == 2
+    assert need >= 2 * 2 * 4 * 128 * 128 * 4  # four states per (segment, head)
+    assert L.kda_cp_segments(2, 4096, 16, 148) == 3  # 32 chains: 3 x 32 blocks per pass
     assert L.kda_cp_segments(1, 65536, 96, 148) == 1
 
 
