@@ -309,6 +309,7 @@ def run_reference(args, d):
 TRAFFIC_PROFILES = {
     "kda_fwd_tc_kernel": ("kda_fwd_tc_prefill_h96_t4096_traffic.txt", "kda_fwd_tc.cu"),
     "kda_decode_kernel": ("kda_decode_b64_h96_traffic.txt", "kda_decode.cu"),
+    "kda_spec_kernel": ("kda_spec_b64_h96_w4_traffic.txt", "kda_spec.cu"),
 }
 FLUSH = {"mid": True, "stress": True, "prefill64k": False, "varlen": False, "tp4": False}
 
@@ -397,7 +398,7 @@ def bench_prefill(name, d, dev, stream, peaks, kda, synth, steps, warmup, with_t
                         "tensor_frac_of_bf16_peak": flops_alg / per_step / 1e12 / peaks["bf16_tflops"]},
            "gpu_launches": steps * launches, **extra}
     if variant == "cp":
-        res["roofline"]["kernel"] = "kda_fwd_tc_kernel (segment mode) + composition + correction"
+        res["roofline"]["kernel"] = "kda_fwd_tc_kernel state pass (segment mode) + composition + kda_fwd_tc_kernel from incoming states"
     del out, fin, ws
     return res, inp
 
@@ -537,10 +538,12 @@ def bench_spec(args, d, dev, stream, peaks, kda, synth, W=4, sweep=(1, 2, 4, 8))
             mean_acc = float(torch.stack(accs).float().mean())
             nbytes = B * H * (2 * dk * dv * 4 + (w + mean_acc) * (2 * (2 * dk + dv) + 4 * dk + 4) + w * 2 * dv)
             ach = nbytes / times[w] / 1e9
+            prof, src = TRAFFIC_PROFILES["kda_spec_kernel"]
+            traffic = scaled_traffic(prof, src, B * H, 0.0)
             res.update(value=job_throughput(d, B * H * w * args.steps, sec) / 1e6, unit=UNIT,
                        ms_per_step=times[w] * 1e3, mean_accepted=mean_acc, gpu_launches=args.steps,
                        roofline={"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                                 "frac": ach / peaks["hbm_gbs"], "traffic": None, "bytes_per_launch": nbytes,
+                                 "frac": ach / peaks["hbm_gbs"], "traffic": traffic, "bytes_per_launch": nbytes,
                                  "kernel": "kda_spec_kernel<128,128,bf16>"})
         del wins, accs, state, out
         torch.cuda.empty_cache()
@@ -577,6 +580,7 @@ CAPTURES = {
     "prefill_h96_t4096": "B=1 H=96 T=4096 d=128 bf16 prefill (the 64K workload's heads, 1/16 of its tokens)",
     "mid": "B=2 H=16 T=4096 d=128 bf16 prefill with initial states",
     "decode_b64_h96": "B=64 H=96 d=128 bf16 decode step (1/8 of the decode workload's sequences)",
+    "spec_b64_h96_w4": "B=64 H=96 d=128 bf16 speculative verification, windows of 4, accepted drafts 0..3",
 }
 
 
@@ -588,7 +592,15 @@ def run_capture(args):
     import synth
     dev = torch.device("cuda")
     n = max(1, args.steps)
-    if args.capture == "decode_b64_h96":
+    if args.capture == "spec_b64_h96_w4":
+        import numpy as np
+        spec, B, W = synth.DECODE, 64, 4
+        state = synth.make_decode_state(spec, dev, B=B)
+        wins = [synth.make_spec_window(spec, s, W, dev, B=B) for s in range(n + 1)]
+        acc = torch.tensor(np.random.default_rng(9).integers(0, W, B), dtype=torch.int32, device=dev)
+        for i in range(n):
+            kda.kda_decode_spec(wins[i], acc, wins[i + 1], state)
+    elif args.capture == "decode_b64_h96":
         spec = synth.DECODE
         state = synth.make_decode_state(spec, dev, B=64)
         x = synth.make_decode_step(spec, 0, dev, B=64)
