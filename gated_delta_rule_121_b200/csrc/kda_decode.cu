@@ -64,32 +64,27 @@ __global__ void __launch_bounds__(DecodeShape<DK, DV>::NT)
       s_a[i] = __expf(static_cast<const float*>(g)[bh * DK + i]);
   }
   __syncthreads();
-  if constexpr (GATED) {  // L2-normalise q and k in place (one warp), then the block uses them
-    __shared__ float s_sc[2];
-    if (tid < 32) {
-      float qq = 0.f, kk = 0.f;
-      for (int i = tid; i < DK; i += 32) {
-        qq += s_q[i] * s_q[i];
-        kk += s_k[i] * s_k[i];
-      }
+  // q.k, and for GATED the L2 norms of q and k: every warp reduces them itself
+  // (no further block barrier); the rows are scaled as they are used.
+  float fq = 1.f, fk = 1.f;
+  if constexpr (GATED) {
+    float qq = 0.f, kk = 0.f, qk = 0.f;
+    for (int i = tid & 31; i < DK; i += 32) {
+      const float a = s_q[i], b = s_k[i];
+      qq += a * a;
+      kk += b * b;
+      qk += a * b;
+    }
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        qq += __shfl_xor_sync(0xffffffffu, qq, o);
-        kk += __shfl_xor_sync(0xffffffffu, kk, o);
-      }
-      if (tid == 0) {
-        s_sc[0] = l2norm_scale(qq);
-        s_sc[1] = l2norm_scale(kk);
-      }
+    for (int o = 16; o > 0; o >>= 1) {
+      qq += __shfl_xor_sync(0xffffffffu, qq, o);
+      kk += __shfl_xor_sync(0xffffffffu, kk, o);
+      qk += __shfl_xor_sync(0xffffffffu, qk, o);
     }
-    __syncthreads();
-    for (int i = tid; i < DK; i += NT) {
-      s_q[i] *= s_sc[0];
-      s_k[i] *= s_sc[1];
-    }
-    __syncthreads();
-  }
-  if (tid < 32) {
+    fq = l2norm_scale(qq);
+    fk = l2norm_scale(kk);
+    if (tid == 0) s_qk = qk * fq * fk;
+  } else if (tid < 32) {
     float acc = 0.f;
     for (int i = tid; i < DK; i += 32) acc += s_q[i] * s_k[i];
 #pragma unroll
@@ -101,7 +96,7 @@ __global__ void __launch_bounds__(DecodeShape<DK, DV>::NT)
 #pragma unroll
   for (int m = 0; m < ROWS; ++m) {
     const int i = rg * ROWS + m;
-    const float a = s_a[i], ki = s_k[i], qi = s_q[i];
+    const float a = s_a[i], ki = s_k[i] * fk, qi = s_q[i] * fq;
     s[m].x *= a; s[m].y *= a; s[m].z *= a; s[m].w *= a;
     pu.x += s[m].x * ki; pu.y += s[m].y * ki; pu.z += s[m].z * ki; pu.w += s[m].w * ki;
     pp.x += s[m].x * qi; pp.y += s[m].y * qi; pp.z += s[m].z * qi; pp.w += s[m].w * qi;
@@ -125,7 +120,7 @@ __global__ void __launch_bounds__(DecodeShape<DK, DV>::NT)
   d.w = bt * (to_f32(vv[3]) - u.w);
 #pragma unroll
   for (int m = 0; m < ROWS; ++m) {
-    const float ki = s_k[rg * ROWS + m];
+    const float ki = s_k[rg * ROWS + m] * fk;
     s[m].x += ki * d.x; s[m].y += ki * d.y; s[m].z += ki * d.z; s[m].w += ki * d.w;
     __stcs(S + (rg * ROWS + m) * COLQ + cq, s[m]);
   }

@@ -111,7 +111,7 @@ constexpr uint32_t MS_GC = 768;      // [2][128] fp32: exp(G_C)
 constexpr uint32_t MS_RED = 1792;    // [8][128] fp32 log2 sums
 constexpr uint32_t MS_PAIRS = 5888;  // [64][8] fp32: P, A of the pairs inside 4-row groups (general chunks)
 constexpr uint32_t MS_RQK = 7936;    // [16][8] fp32: 1/|q_r|, 1/|k_r| of each row group's 4 rows (MODE_GATED)
-constexpr uint32_t MS_GATE = 8448;   // [2] fp32: -exp(A_h) log2(e), g_min log2(e) (MODE_GATED)
+constexpr uint32_t MS_GATE = 8448;   // [2] fp32: -exp(A_h) log2(e), g_min (MODE_GATED)
 constexpr uint32_t MS_END = 8464;
 static_assert(NUM_BARS * 8 <= MS_TMEM, "barrier area");
 static_assert(MS_END <= MISC_BYTES, "misc area");
@@ -270,51 +270,58 @@ struct Ctx {
   int64_t ckpt0;    // MODE_CKPT: checkpoint slot of this sequence's first interval
 };
 
-// MODE_GATED: per-token log2-decays of 8 channels from their bf16 decay
-// logits: g log2(e) = g_min log2(e) / (1 + 2^(-exp(A_h) log2(e) z)).
+// MODE_GATED: per-token log-decays of 8 channels from their bf16 decay
+// logits: g = g_min / (1 + 2^(-exp(A_h) log2(e) z)).  The prefix converts
+// them to log2 units like the plain path's inputs (keeping that one multiply
+// in both modes also keeps the front group's register allocation spill-free).
 __device__ __forceinline__ float rcp_approx(float x) {
   float y;
   asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
-__device__ __forceinline__ F8 gate_log2_8(uint4 u, float gz, float gmin2) {
+__device__ __forceinline__ F8 gate_8(uint4 u, float gz, float gmin) {
   F8 z = bf16x8_to_f32(u);
   float* e = &z.a.x;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) e[i] = gmin2 * rcp_approx(1.f + ex2(gz * e[i]));
+  for (int i = 0; i < 8; ++i) e[i] = gmin * rcp_approx(1.f + ex2(gz * e[i]));
   return z;
 }
 // MODE_GATED: 1/|x_r| for this thread's 4 rows of the raw q and k tiles (its 8
-// channels, summed over the 16 threads of the row group), stored in the row
-// group's entry of `tab` ([rg][0..3] = q, [rg][4..7] = k) for the group's
-// threads to read where they scale the rows (the values do not stay in
-// registers across the Gram).
+// channels), stored in the row group's entry of `tab` ([rg][0..3] = q,
+// [rg][4..7] = k) for the group's threads to read where they scale the rows
+// (the values do not stay in registers across the Gram).  The 8 partial sums
+// of the 16 threads of a row group are reduce-scattered by recursive halving
+// (offsets 8, 4, 2: lane pair l/2 ends with sum number l/2), then the pair
+// adds its two halves; 8 shuffles instead of 4 x 8.
 __device__ __forceinline__ void row_norms(const uint8_t* qb, const uint8_t* kb, int rg, int cc, float* tab) {
-  float rq[4], rk[4];
+  float v[8];
 #pragma unroll
   for (int m = 0; m < 4; ++m) {
     const uint32_t o = sw128_off(4 * rg + m, cc);
     const F8 a = bf16x8_to_f32(*reinterpret_cast<const uint4*>(qb + o));
     const F8 b = bf16x8_to_f32(*reinterpret_cast<const uint4*>(kb + o));
     const F8 a2 = mul8(a, a), b2 = mul8(b, b);
-    rq[m] = ((a2.a.x + a2.a.y) + (a2.a.z + a2.a.w)) + ((a2.b.x + a2.b.y) + (a2.b.z + a2.b.w));
-    rk[m] = ((b2.a.x + b2.a.y) + (b2.a.z + b2.a.w)) + ((b2.b.x + b2.b.y) + (b2.b.z + b2.b.w));
+    v[m] = ((a2.a.x + a2.a.y) + (a2.a.z + a2.a.w)) + ((a2.b.x + a2.b.y) + (a2.b.z + a2.b.w));
+    v[4 + m] = ((b2.a.x + b2.a.y) + (b2.a.z + b2.a.w)) + ((b2.b.x + b2.b.y) + (b2.b.z + b2.b.w));
   }
+  const int l = threadIdx.x & 15;
+  const bool b3 = l & 8, b2 = l & 4, b1 = l & 2;
+  float h4[4], h2[2];
 #pragma unroll
-  for (int o = 1; o < 16; o <<= 1) {
+  for (int j = 0; j < 4; ++j) h4[j] = (b3 ? v[j + 4] : v[j]) + __shfl_xor_sync(0xffffffffu, b3 ? v[j] : v[j + 4], 8);
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      rq[m] += __shfl_xor_sync(0xffffffffu, rq[m], o);
-      rk[m] += __shfl_xor_sync(0xffffffffu, rk[m], o);
-    }
-  }
-  if ((threadIdx.x & 15) == 0) {
-    *reinterpret_cast<float4*>(tab + rg * 8) =
-        make_float4(l2norm_scale(rq[0]), l2norm_scale(rq[1]), l2norm_scale(rq[2]), l2norm_scale(rq[3]));
-    *reinterpret_cast<float4*>(tab + rg * 8 + 4) =
-        make_float4(l2norm_scale(rk[0]), l2norm_scale(rk[1]), l2norm_scale(rk[2]), l2norm_scale(rk[3]));
-  }
+  for (int j = 0; j < 2; ++j) h2[j] = (b2 ? h4[j + 2] : h4[j]) + __shfl_xor_sync(0xffffffffu, b2 ? h4[j] : h4[j + 2], 4);
+  float h1 = (b1 ? h2[1] : h2[0]) + __shfl_xor_sync(0xffffffffu, b1 ? h2[0] : h2[1], 2);
+  h1 += __shfl_xor_sync(0xffffffffu, h1, 1);
+  if (!(l & 1)) tab[rg * 8 + (l >> 1)] = l2norm_scale(h1);
   __syncwarp();  // a row group is half a warp
+}
+// One factor of the table, read where it is used (a volatile shared load is
+// not hoisted, so the factors do not occupy registers across the pass).
+__device__ __forceinline__ float row_factor(const uint8_t* sm, int rg, int i) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(smem_u32(sm + SM_MISC + MS_RQK + (rg * 8 + i) * 4)));
+  return v;
 }
 // This row group's factors from the table.
 __device__ __forceinline__ void row_factors(const uint8_t* sm, int rg, float (&rq)[4], float (&rk)[4]) {
@@ -666,13 +673,13 @@ __device__ __forceinline__ void front_group(const Ctx& x, const float* __restric
     for (int m = 0; m < 4; ++m) {
       const int r = 4 * rg + m;
       if constexpr (MODE == MODE_GATED) {
-        // bf16 decay logits mapped to log2-decays at once; rows past the end
+        // bf16 decay logits mapped to log-decays at once; rows past the end
         // get -inf, whose gate is exactly 0
         const uint4 u = r < valid ? __ldg(reinterpret_cast<const uint4*>(
                                         reinterpret_cast<const __nv_bfloat16*>(g) + ((tok0 + r) * H + x.h) * D + ch0))
                                   : make_uint4(0xFF80FF80u, 0xFF80FF80u, 0xFF80FF80u, 0xFF80FF80u);
         const float* gc = reinterpret_cast<const float*>(x.sm + SM_MISC + MS_GATE);
-        gv[m] = gate_log2_8(u, gc[0], gc[1]);
+        gv[m] = gate_8(u, gc[0], gc[1]);
       } else {
         gv[m] = r < valid ? ldg8(g + ((tok0 + r) * H + x.h) * D + ch0, g32) : f8(0.f);
       }
@@ -712,7 +719,7 @@ __device__ __forceinline__ void front_group(const Ctx& x, const float* __restric
     const F8 l2e = f8(LOG2E);
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
-      if constexpr (MODE != MODE_GATED) gv[m] = mul8(gv[m], l2e);  // gated rows are in log2 units already
+      gv[m] = mul8(gv[m], l2e);
       acc = add8(acc, gv[m]);
     }
     F8 other;  // the other row group of this warp (lane ^ 16)
@@ -798,8 +805,6 @@ __device__ __forceinline__ void front_group(const Ctx& x, const float* __restric
     // fast chunks, 0 otherwise), H = e^{G_C - G_r}.  QE, KE and V (fp16) go
     // in place; KH goes to KX[b2] once the scan of chunk c-2 has released it.
     uint4 kraw[4];  // raw K rows, kept for KH
-    float rq[4] = {1.f, 1.f, 1.f, 1.f}, rk[4] = {1.f, 1.f, 1.f, 1.f};
-    if constexpr (MODE == MODE_GATED) row_factors(sm, rg, rq, rk);
     {
       F8 gr = f8(0.f);
 #pragma unroll
@@ -819,8 +824,8 @@ __device__ __forceinline__ void front_group(const Ctx& x, const float* __restric
           gr = add8(gr, gv[m]);
           const F8 fw = ex2_8(fast ? sub8(gr, tot) : gr);
           if constexpr (MODE == MODE_GATED) {
-            st_f16x8(qb + o, mul8(bf16x8_to_f32(qr[i]), mul8(fw, f8(rq[m]))));
-            st_f16x8(kb + o, mul8(bf16x8_to_f32(kraw[m]), mul8(fw, f8(rk[m]))));
+            st_f16x8(qb + o, mul8(bf16x8_to_f32(qr[i]), mul8(fw, f8(row_factor(sm, rg, m)))));
+            st_f16x8(kb + o, mul8(bf16x8_to_f32(kraw[m]), mul8(fw, f8(row_factor(sm, rg, 4 + m)))));
           } else {
             st_f16x8(qb + o, mul8(bf16x8_to_f32(qr[i]), fw));
             st_f16x8(kb + o, mul8(bf16x8_to_f32(kraw[m]), fw));
@@ -848,7 +853,7 @@ __device__ __forceinline__ void front_group(const Ctx& x, const float* __restric
         const uint32_t o = sw128_off(4 * rg + m, cc);
         gr = add8(gr, gv[m]);
         if constexpr (MODE == MODE_GATED)
-          st_f16x8(khb + o, mul8(bf16x8_to_f32(kraw[m]), mul8(ex2_8(sub8(tot, gr)), f8(rk[m]))));
+          st_f16x8(khb + o, mul8(bf16x8_to_f32(kraw[m]), mul8(ex2_8(sub8(tot, gr)), f8(row_factor(sm, rg, 4 + m)))));
         else
           st_f16x8(khb + o, mul8(bf16x8_to_f32(kraw[m]), ex2_8(sub8(tot, gr))));
       }
@@ -1512,7 +1517,7 @@ __global__ void __launch_bounds__(NTHR, 1)
     if (threadIdx.x == 0) {
       float* gc = reinterpret_cast<float*>(sm + SM_MISC + MS_GATE);
       gc[0] = -__expf(ma.A_log[x.h]) * LOG2E;
-      gc[1] = ma.g_min * LOG2E;
+      gc[1] = ma.g_min;
     }
   }
   if constexpr (MODE == MODE_CKPT)

@@ -23,15 +23,20 @@
 //   o_t = Y_t + sum_{s<=t} P_ts delta_s
 //   S_c = Diag(e^{G_c}) S0 + sum_{s<=c} (k_s * e^{G_c - G_s}) delta_s^T   (c: the bonus token)
 // So the state is read once into registers (ROWS x 4 values per thread) and
-// written once; what grows with the window is two dot products per token
-// against those registers plus an n x n triangular system, with no block
-// barrier in the token loop: a column group's RG row groups are lanes of one
-// warp, so the reductions over rows are shuffles.
+// written once, with the decode step's thread mapping: a warp holds whole rows
+// (for dv = 128, 16 consecutive rows x 128 columns per warp), so every state
+// load and store is 512 contiguous bytes per warp.  The products against the
+// state (X_t, Y_t) do not depend on delta, so they are formed for all tokens
+// together, four at a time, and the row groups' partial sums are added
+// through shared memory.  Only the n x n triangular system on dv-vectors
+// stays serial in t: one thread per value column, delta in registers.
 //
 // GATED: the inputs are the raw ones of the model's prologue (digest, KDA
 // section and "Bounded decay" section): q and k are L2-normalised per token
 // and head, and the decay is g = g_min * sigmoid(exp(A_h) * z) from the decay
 // logits z.
+#include <type_traits>
+
 #include "../../include/kda.h"
 #include "kda_gate.cuh"
 #include "kda_internal.cuh"
@@ -42,17 +47,25 @@ namespace {
 template <int DK, int DV>
 struct SpecShape {
   static constexpr int COLQ = DV / 4;                                  // float4 column groups
-  static constexpr int RG0 = (256 / COLQ) < DK ? (256 / COLQ) : DK;
-  static constexpr int RG = RG0 < 32 ? RG0 : 32;                       // row groups: lanes of one warp
-  static constexpr int ROWS = DK / RG;                                 // rows per thread
+  static constexpr int RG = (256 / COLQ) < DK ? (256 / COLQ) : DK;     // row groups
+  static constexpr int ROWS = DK / RG;                                 // consecutive rows per thread
   static constexpr int NT = COLQ * RG;                                 // threads per block
+  static constexpr int PART = RG * 4 * 2 * DV;                         // floats of partial X, Y sums
 };
 
-// Shared-memory floats of a block for chunks of up to `n` tokens.
+// Row stride (floats) of the channel-major operand arrays for chunks of n4
+// (a multiple of 4) tokens: an odd number of float4s, so the 16-byte reads of
+// eight consecutive channels hit eight different bank quads.
+__host__ __device__ constexpr int spec_ld(int n4) { return (n4 / 4) % 2 ? n4 : n4 + 4; }
+
+// Shared-memory floats of a block for chunks of up to `n` tokens (the
+// token-major arrays and the partial sums share one region).
 template <int DK, int DV>
 constexpr size_t spec_smem_floats(int n) {
   const size_t n4 = (size_t)((n + 3) & ~3);
-  return 3 * (size_t)n * DK + 2 * (size_t)n * DV + 2 * (size_t)n * n4 + n4 + DK;
+  const size_t tok = 3 * (size_t)n * DK, part = (size_t)SpecShape<DK, DV>::PART;
+  return (tok > part ? tok : part) + 2 * (size_t)n * DV + 2 * (size_t)n * n4 + n4 + DK +
+         3 * (size_t)DK * spec_ld((int)n4) + 2 * (size_t)n * DV;
 }
 
 struct SpecTok {  // where one token's inputs live
@@ -64,90 +77,108 @@ struct SpecTok {  // where one token's inputs live
 };
 
 template <int DK, int DV, typename IO, bool GATED>
-__global__ void __launch_bounds__(SpecShape<DK, DV>::NT)
+__global__ void __launch_bounds__(SpecShape<DK, DV>::NT, 2)
     kda_spec_kernel(SpecTok prev, SpecTok cur, const int32_t* __restrict__ n_accepted, float* __restrict__ state,
                     IO* __restrict__ out, int Wp, int W, int H, const float* __restrict__ A_log, float g_min) {
   using Sh = SpecShape<DK, DV>;
   constexpr int COLQ = Sh::COLQ, RG = Sh::RG, ROWS = Sh::ROWS, NT = Sh::NT;
   extern __shared__ float ssm[];
   const int b = blockIdx.x / H, h = blockIdx.x % H;
-  const int tid = threadIdx.x, rg = tid % RG, cq = tid / RG, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x, cq = tid % COLQ, rg = tid / COLQ, lane = tid & 31, warp = tid >> 5;
+
+  // ---- token loads first, for both windows whole (Wp + W <= 16 tokens), so
+  // that no address waits for n_accepted; the rejected drafts' rows are
+  // dropped when the chunk is laid out.  Then the state (ROWS consecutive
+  // rows x 4 columns per thread): its 64 KiB stream in while the chunk's own
+  // arithmetic runs.
+  const int NW = Wp + W;
+  auto row_of = [&](int tt) {  // token tt of the two windows -> its [b, t, h] row
+    return tt < Wp ? ((int64_t)b * Wp + tt) * H + h : ((int64_t)b * W + (tt - Wp)) * H + h;
+  };
+  constexpr int PK = (KDA_SPEC_MAX_TOKENS * DK + NT - 1) / NT, PV = (KDA_SPEC_MAX_TOKENS * DV + NT - 1) / NT;
+  float rk[PK], rq[PK], rg2[PK], rv[PV];
+#pragma unroll
+  for (int j = 0; j < PK; ++j) {
+    const int e = tid + j * NT;
+    if (e < NW * DK) {
+      const int tt = e / DK, i = e % DK;
+      const SpecTok& src = tt < Wp ? prev : cur;
+      const int64_t o = row_of(tt) * DK + i;
+      rk[j] = to_f32(static_cast<const IO*>(src.k)[o]);
+      rq[j] = to_f32(static_cast<const IO*>(src.q)[o]);
+      if constexpr (GATED)
+        rg2[j] = to_f32(static_cast<const IO*>(src.g)[o]);
+      else
+        rg2[j] = static_cast<const float*>(src.g)[o];
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < PV; ++j) {
+    const int e = tid + j * NT;
+    if (e < NW * DV) {
+      const int tt = e / DV, i = e % DV;
+      rv[j] = to_f32(static_cast<const IO*>((tt < Wp ? prev : cur).v)[row_of(tt) * DV + i]);
+    }
+  }
+  const float bt = tid < NW ? (tid < Wp ? prev : cur).beta[row_of(tid)] : 0.f;
   int na = n_accepted ? n_accepted[b] : 0;
   na = na < 0 ? 0 : (na > Wp ? Wp : na);
   const int n = na + W;               // tokens of the chunk
   const int c = W > 0 ? na : na - 1;  // the token after which the state is kept (-1: none, unchanged)
   if (c < 0) return;
   // shared layout (floats; every array starts on a multiple of 4 floats):
-  //   s_k, s_q, s_G [n][DK]  k, q, G; then e^G k, e^G q and k_t e^{G_c - G_t}
+  //   s_k, s_q, s_G [n][DK]  k, q, G (token-major; later the partial sums)
   //   s_v, s_d [n][DV]       values, delta
   //   s_A, s_P [n][n4]       pair sums;  s_b [n4] beta;  s_gc [DK] e^{G_c}
-  const int n4 = (n + 3) & ~3;
+  //   s_ek, s_eq, s_kc [DK][ld]  e^G k, e^G q, k e^{G_c - G}, channel-major (0 past the chunk)
+  //   s_xy [n][2 DV]         X_t, then Y_t
+  const int n4 = (n + 3) & ~3, ld = spec_ld(n4);
+  const int tok = 3 * n * DK > Sh::PART ? 3 * n * DK : Sh::PART;
   float* s_k = ssm;
   float* s_q = s_k + n * DK;
   float* s_G = s_q + n * DK;
-  float* s_v = s_G + n * DK;
+  float* s_part = ssm;
+  float* s_v = ssm + tok;
   float* s_d = s_v + n * DV;
   float* s_A = s_d + n * DV;
   float* s_P = s_A + n * n4;
   float* s_b = s_P + n * n4;
   float* s_gc = s_b + n4;
+  float* s_ek = s_gc + DK;
+  float* s_eq = s_ek + DK * ld;
+  float* s_kc = s_eq + DK * ld;
+  float* s_xy = s_kc + DK * ld;
 
-  float4* S = reinterpret_cast<float4*>(state + ((int64_t)b * H + h) * DK * DV);
-  float4 s[ROWS];  // rows m * RG + rg, columns 4 cq .. 4 cq + 3
-#pragma unroll
-  for (int m = 0; m < ROWS; ++m) s[m] = __ldcs(S + (m * RG + rg) * COLQ + cq);
-
-  // ---- stage the chunk: the replayed tokens, then the new window.  Every
-  // thread issues all of its loads before it uses any (the window is at most
-  // KDA_SPEC_MAX_TOKENS tokens), so their latencies overlap each other and
-  // the state loads above.
-  auto src_row = [&](int t) {
-    return t < na ? ((int64_t)b * Wp + t) * H + h : ((int64_t)b * W + (t - na)) * H + h;
-  };
+  // ---- lay out the chunk: prev[0, na) at 0 .. na-1, cur[0, W) at na ..
   {
-    constexpr int PK = (KDA_SPEC_MAX_TOKENS * DK + NT - 1) / NT, PV = (KDA_SPEC_MAX_TOKENS * DV + NT - 1) / NT;
-    float rk[PK], rq[PK], rg2[PK], rv[PV];
-#pragma unroll
-    for (int j = 0; j < PK; ++j) {
-      const int e = tid + j * NT;
-      if (e < n * DK) {
-        const int t = e / DK, i = e % DK;
-        const SpecTok& src = t < na ? prev : cur;
-        const int64_t o = src_row(t) * DK + i;
-        rk[j] = to_f32(static_cast<const IO*>(src.k)[o]);
-        rq[j] = to_f32(static_cast<const IO*>(src.q)[o]);
-        if constexpr (GATED)
-          rg2[j] = to_f32(static_cast<const IO*>(src.g)[o]);
-        else
-          rg2[j] = static_cast<const float*>(src.g)[o];
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < PV; ++j) {
-      const int e = tid + j * NT;
-      if (e < n * DV) {
-        const int t = e / DV, i = e % DV;
-        rv[j] = to_f32(static_cast<const IO*>((t < na ? prev : cur).v)[src_row(t) * DV + i]);
-      }
-    }
-    const float bt = tid < n ? (tid < na ? prev : cur).beta[src_row(tid)] : 0.f;
     const float Ah = GATED ? A_log[h] : 0.f;
+    auto pos = [&](int tt) { return tt < Wp ? (tt < na ? tt : -1) : na + (tt - Wp); };
 #pragma unroll
     for (int j = 0; j < PK; ++j) {
       const int e = tid + j * NT;
-      if (e < n * DK) {
-        s_k[e] = rk[j];
-        s_q[e] = rq[j];
-        s_G[e] = GATED ? gate_log_decay(rg2[j], Ah, g_min) : rg2[j];
+      if (e < NW * DK) {
+        const int p = pos(e / DK), i = e % DK;
+        if (p >= 0) {
+          s_k[p * DK + i] = rk[j];
+          s_q[p * DK + i] = rq[j];
+          s_G[p * DK + i] = GATED ? gate_log_decay(rg2[j], Ah, g_min) : rg2[j];
+        }
       }
     }
 #pragma unroll
     for (int j = 0; j < PV; ++j) {
       const int e = tid + j * NT;
-      if (e < n * DV) s_v[e] = rv[j];
+      if (e < NW * DV) {
+        const int p = pos(e / DV);
+        if (p >= 0) s_v[p * DV + e % DV] = rv[j];
+      }
     }
-    if (tid < n) s_b[tid] = bt;
+    if (tid < NW && pos(tid) >= 0) s_b[pos(tid)] = bt;
   }
+  float4* S = reinterpret_cast<float4*>(state + ((int64_t)b * H + h) * DK * DV);
+  float4 s[ROWS];  // rows rg * ROWS + m, columns 4 cq .. 4 cq + 3; first used by the X, Y products
+#pragma unroll
+  for (int m = 0; m < ROWS; ++m) s[m] = __ldcs(S + (rg * ROWS + m) * COLQ + cq);
   __syncthreads();
   if constexpr (GATED) {  // L2-normalise q and k per token, one warp per token
     for (int t = warp; t < n; t += NT / 32) {
@@ -169,7 +200,7 @@ __global__ void __launch_bounds__(SpecShape<DK, DV>::NT)
     }
     __syncthreads();
   }
-  // cumulative log-decay over the chunk, one thread per key channel
+  // ---- cumulative log-decay over the chunk, one thread per key channel
   for (int i = tid; i < DK; i += NT) {
     float acc = 0.f;
     for (int t = 0; t < n; ++t) {
@@ -178,99 +209,163 @@ __global__ void __launch_bounds__(SpecShape<DK, DV>::NT)
     }
   }
   __syncthreads();
-  // ---- pair sums, one warp per pair (t, s), s <= t
-  for (int p = warp; p < n * (n + 1) / 2; p += NT / 32) {
-    int t = 0;
-    while ((t + 1) * (t + 2) / 2 <= p) ++t;
-    const int s2 = p - t * (t + 1) / 2;
-    float pa = 0.f, pp = 0.f;
-    for (int i = lane; i < DK; i += 32) {
-      const float ke = s_k[s2 * DK + i] * __expf(s_G[t * DK + i] - s_G[s2 * DK + i]);  // decay s -> t, <= 1
-      pa += s_k[t * DK + i] * ke;
-      pp += s_q[t * DK + i] * ke;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      pa += __shfl_xor_sync(0xffffffffu, pa, o);
-      pp += __shfl_xor_sync(0xffffffffu, pp, o);
-    }
-    if (lane == 0) {
-      s_A[t * n4 + s2] = pa;
-      s_P[t * n4 + s2] = pp;
-    }
-  }
-  __syncthreads();
-  // ---- per-token operands in place: e^{G_t} k_t, e^{G_t} q_t, k_t e^{G_c - G_t} (t <= c)
+  // ---- per-token operands, channel-major, one thread per channel:
+  // e^{G_t} k_t, e^{G_t} q_t, k_t e^{G_c - G_t} (t <= c); zero for the tokens
+  // past the chunk (up to n4).  Then (no barrier: other arrays) the pair
+  // sums A_ts (s < t; the diagonal entry written is not used) and P_ts (s <= t).
   for (int i = tid; i < DK; i += NT) {
     const float gc = s_G[c * DK + i];
     s_gc[i] = __expf(gc);
-    for (int t = 0; t < n; ++t) {
-      const float G = s_G[t * DK + i], kk = s_k[t * DK + i];
-      const float eg = __expf(G);
-      s_k[t * DK + i] = eg * kk;
-      s_q[t * DK + i] *= eg;
-      s_G[t * DK + i] = t <= c ? kk * __expf(gc - G) : 0.f;
+#pragma unroll 4
+    for (int t = 0; t < n4; ++t) {
+      float ek = 0.f, eq = 0.f, kc = 0.f;
+      if (t < n) {
+        const float G = s_G[t * DK + i], kk = s_k[t * DK + i];
+        const float eg = __expf(G);
+        ek = eg * kk;
+        eq = eg * s_q[t * DK + i];
+        kc = t <= c ? kk * __expf(gc - G) : 0.f;
+      }
+      s_ek[i * ld + t] = ek;
+      s_eq[i * ld + t] = eq;
+      s_kc[i * ld + t] = kc;
+    }
+  }
+  // Four pairs per warp at a time (pairs in row order: p -> (t, s)): each
+  // lane sums its channels for the 8 values (A, P of 4 pairs), the warp
+  // reduce-scatters them (offsets 4, 2, 1: lane l keeps value l & 7), then
+  // adds across the remaining lane bits (offsets 8, 16).
+  const int npairs = n * (n + 1) / 2;
+  for (int p0 = warp * 4; p0 < npairs; p0 += NT / 32 * 4) {
+    int tq[4], sq[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int p = p0 + q < npairs ? p0 + q : 0;
+      int t = 0;
+      while ((t + 1) * (t + 2) / 2 <= p) ++t;
+      tq[q] = t;
+      sq[q] = p - t * (t + 1) / 2;
+    }
+    float v[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] = 0.f;
+    for (int i = lane; i < DK; i += 32) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int t = tq[q], s2 = sq[q];
+        const float ke = s_k[s2 * DK + i] * __expf(s_G[t * DK + i] - s_G[s2 * DK + i]);  // decay s -> t, <= 1
+        v[2 * q] += s_k[t * DK + i] * ke;
+        v[2 * q + 1] += s_q[t * DK + i] * ke;
+      }
+    }
+#pragma unroll
+    for (int o = 4; o >= 1; o >>= 1) {
+      const bool up = lane & o;
+#pragma unroll
+      for (int j = 0; j < o; ++j) v[j] = (up ? v[j + o] : v[j]) + __shfl_xor_sync(0xffffffffu, up ? v[j] : v[j + o], o);
+    }
+    v[0] += __shfl_xor_sync(0xffffffffu, v[0], 8);
+    v[0] += __shfl_xor_sync(0xffffffffu, v[0], 16);
+    const int q = (lane >> 1) & 3;
+    if (lane < 8 && p0 + q < npairs) (lane & 1 ? s_P : s_A)[tq[q] * n4 + sq[q]] = v[0];
+  }
+  __syncthreads();
+
+  // ---- X_t = S0^T ek_t and Y_t = S0^T eq_t, TB tokens at a time (groups of
+  // 4, the last one to three tokens in groups of 2 and 1): each thread's
+  // share over its rows, then the row groups' partial sums added through
+  // shared memory (the token-major arrays are no longer needed).
+  auto xy_group = [&](auto tb, int t0) {
+    constexpr int TB = decltype(tb)::value;
+#pragma unroll
+    for (int xy = 0; xy < 2; ++xy) {  // X from e^G k, then Y from e^G q (16 accumulators at a time)
+      const float* src = xy ? s_eq : s_ek;
+      float acc[TB][4];
+#pragma unroll
+      for (int u = 0; u < TB; ++u) acc[u][0] = acc[u][1] = acc[u][2] = acc[u][3] = 0.f;
+#pragma unroll
+      for (int m = 0; m < ROWS; ++m) {
+        const int i = rg * ROWS + m;
+        float ev[TB];
+        if constexpr (TB == 4) {
+          const float4 e4 = *reinterpret_cast<const float4*>(src + i * ld + t0);
+          ev[0] = e4.x; ev[1] = e4.y; ev[2] = e4.z; ev[3] = e4.w;
+        } else if constexpr (TB == 2) {
+          const float2 e2 = *reinterpret_cast<const float2*>(src + i * ld + t0);
+          ev[0] = e2.x; ev[1] = e2.y;
+        } else {
+          ev[0] = src[i * ld + t0];
+        }
+#pragma unroll
+        for (int u = 0; u < TB; ++u) {
+          acc[u][0] += s[m].x * ev[u]; acc[u][1] += s[m].y * ev[u];
+          acc[u][2] += s[m].z * ev[u]; acc[u][3] += s[m].w * ev[u];
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < TB; ++u)
+        *reinterpret_cast<float4*>(s_part + ((rg * TB + u) * 2 + xy) * DV + 4 * cq) =
+            make_float4(acc[u][0], acc[u][1], acc[u][2], acc[u][3]);
+    }
+    __syncthreads();
+    for (int e = tid; e < TB * 2 * DV; e += NT) {
+      float sum = 0.f;
+#pragma unroll 8
+      for (int r = 0; r < RG; ++r) sum += s_part[r * TB * 2 * DV + e];
+      s_xy[t0 * 2 * DV + e] = sum;  // token t0 + e / (2 DV), X or Y column e % (2 DV)
+    }
+    __syncthreads();  // the partial sums are read before the next group writes them
+  };
+  int t0 = 0;
+  for (; t0 + 4 <= n; t0 += 4) xy_group(std::integral_constant<int, 4>{}, t0);
+  if (n - t0 >= 2) {
+    xy_group(std::integral_constant<int, 2>{}, t0);
+    t0 += 2;
+  }
+  if (t0 < n) xy_group(std::integral_constant<int, 1>{}, t0);
+
+  // ---- delta_t by forward substitution and o_t, one thread per value column
+  IO* o_base = out + ((int64_t)b * W * H + h) * DV;
+  for (int j = tid; j < DV; j += NT) {
+    float dl[KDA_SPEC_MAX_TOKENS];
+#pragma unroll
+    for (int t = 0; t < KDA_SPEC_MAX_TOKENS; ++t) {
+      if (t < n) {
+        float d = s_v[t * DV + j] - s_xy[t * 2 * DV + j];
+#pragma unroll
+        for (int s2 = 0; s2 < t; ++s2) d -= s_A[t * n4 + s2] * dl[s2];
+        d *= s_b[t];
+        dl[t] = d;
+        s_d[t * DV + j] = d;
+        if (t >= na) {
+          float o = s_xy[t * 2 * DV + DV + j];
+#pragma unroll
+          for (int s2 = 0; s2 <= t; ++s2) o += s_P[t * n4 + s2] * dl[s2];
+          o_base[(int64_t)(t - na) * H * DV + j] = from_f32<IO>(o);
+        }
+      }
     }
   }
   __syncthreads();
 
-  // ---- token loop: X_t, Y_t by row-group shuffles, delta_t by substitution, o_t
-  IO* o_base = out + ((int64_t)b * W * H + h) * DV + 4 * cq;
-  for (int t = 0; t < n; ++t) {
-    float4 x = make_float4(0.f, 0.f, 0.f, 0.f), y = x;
-#pragma unroll
-    for (int m = 0; m < ROWS; ++m) {
-      const int i = m * RG + rg;
-      const float gk = s_k[t * DK + i], gq = s_q[t * DK + i];
-      x.x += s[m].x * gk; x.y += s[m].y * gk; x.z += s[m].z * gk; x.w += s[m].w * gk;
-      y.x += s[m].x * gq; y.y += s[m].y * gq; y.z += s[m].z * gq; y.w += s[m].w * gq;
-    }
-#pragma unroll
-    for (int o = 1; o < RG; o <<= 1) {
-      x.x += __shfl_xor_sync(0xffffffffu, x.x, o); x.y += __shfl_xor_sync(0xffffffffu, x.y, o);
-      x.z += __shfl_xor_sync(0xffffffffu, x.z, o); x.w += __shfl_xor_sync(0xffffffffu, x.w, o);
-      y.x += __shfl_xor_sync(0xffffffffu, y.x, o); y.y += __shfl_xor_sync(0xffffffffu, y.y, o);
-      y.z += __shfl_xor_sync(0xffffffffu, y.z, o); y.w += __shfl_xor_sync(0xffffffffu, y.w, o);
-    }
-    const float* vv = s_v + t * DV + 4 * cq;
-    float4 d = make_float4(vv[0] - x.x, vv[1] - x.y, vv[2] - x.z, vv[3] - x.w);
-    for (int s2 = 0; s2 < t; ++s2) {
-      const float a = s_A[t * n4 + s2];
-      const float4 ds = *reinterpret_cast<const float4*>(s_d + s2 * DV + 4 * cq);
-      d.x -= a * ds.x; d.y -= a * ds.y; d.z -= a * ds.z; d.w -= a * ds.w;
-    }
-    const float bt = s_b[t];
-    d.x *= bt; d.y *= bt; d.z *= bt; d.w *= bt;
-    if (rg == 0) *reinterpret_cast<float4*>(s_d + t * DV + 4 * cq) = d;
-    if (t >= na && rg == RG - 1) {  // another lane of the group writes the output
-      float4 o = y;
-      for (int s2 = 0; s2 < t; ++s2) {
-        const float pq = s_P[t * n4 + s2];
-        const float4 ds = *reinterpret_cast<const float4*>(s_d + s2 * DV + 4 * cq);
-        o.x += pq * ds.x; o.y += pq * ds.y; o.z += pq * ds.z; o.w += pq * ds.w;
-      }
-      const float pq = s_P[t * n4 + t];
-      o.x += pq * d.x; o.y += pq * d.y; o.z += pq * d.z; o.w += pq * d.w;
-      IO* dst = o_base + (int64_t)(t - na) * H * DV;
-      dst[0] = from_f32<IO>(o.x);
-      dst[1] = from_f32<IO>(o.y);
-      dst[2] = from_f32<IO>(o.z);
-      dst[3] = from_f32<IO>(o.w);
-    }
-    __syncwarp();  // delta_t is visible to the group's lanes for the next tokens
-  }
   // ---- the kept state: S_c = Diag(e^{G_c}) S0 + sum_{s<=c} (k_s e^{G_c - G_s}) delta_s^T
 #pragma unroll
   for (int m = 0; m < ROWS; ++m) {
-    const int i = m * RG + rg;
+    const int i = rg * ROWS + m;
     const float eg = s_gc[i];
     float4 a = make_float4(s[m].x * eg, s[m].y * eg, s[m].z * eg, s[m].w * eg);
-    for (int t = 0; t <= c; ++t) {
-      const float kc = s_G[t * DK + i];
-      const float4 ds = *reinterpret_cast<const float4*>(s_d + t * DV + 4 * cq);
-      a.x += kc * ds.x; a.y += kc * ds.y; a.z += kc * ds.z; a.w += kc * ds.w;
+    for (int t0 = 0; t0 <= c; t0 += 4) {
+      const float4 kq = *reinterpret_cast<const float4*>(s_kc + i * ld + t0);
+      const float kv[4] = {kq.x, kq.y, kq.z, kq.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (t0 + u <= c) {
+          const float4 ds = *reinterpret_cast<const float4*>(s_d + (t0 + u) * DV + 4 * cq);
+          a.x += kv[u] * ds.x; a.y += kv[u] * ds.y; a.z += kv[u] * ds.z; a.w += kv[u] * ds.w;
+        }
+      }
     }
-    __stcs(S + (m * RG + rg) * COLQ + cq, a);
+    __stcs(S + (rg * ROWS + m) * COLQ + cq, a);
   }
 }
 
