@@ -68,6 +68,62 @@ constexpr size_t spec_smem_floats(int n) {
          3 * (size_t)DK * spec_ld((int)n4) + 2 * (size_t)n * DV;
 }
 
+// One token array of both windows in 16-byte pieces (rows of D elements of T;
+// every pointer and row is 16-byte aligned): piece j of a thread is piece
+// tid + j * NT of the NW rows.
+template <typename T, int D, int NT>
+struct Pieces {
+  static constexpr int PER_ROW = D * (int)sizeof(T) / 16;                      // pieces per token row
+  static constexpr int EPP = 16 / (int)sizeof(T);                               // elements per piece
+  static constexpr int CNT = (KDA_SPEC_MAX_TOKENS * PER_ROW + NT - 1) / NT;  // pieces per thread, at most
+};
+
+template <typename T, int D, int NT>
+__device__ __forceinline__ void load_pieces(const void* prev, const void* cur, int NW, int Wp, int W, int b, int H,
+                                            int h, uint4 (&r)[Pieces<T, D, NT>::CNT]) {
+  using P = Pieces<T, D, NT>;
+#pragma unroll
+  for (int j = 0; j < P::CNT; ++j) {
+    const int pc = threadIdx.x + j * NT;
+    if (pc < NW * P::PER_ROW) {
+      const int tt = pc / P::PER_ROW, o = pc % P::PER_ROW;
+      const int64_t row = tt < Wp ? ((int64_t)b * Wp + tt) * H + h : ((int64_t)b * W + (tt - Wp)) * H + h;
+      r[j] = __ldg(reinterpret_cast<const uint4*>(static_cast<const T*>(tt < Wp ? prev : cur) + row * D) + o);
+    }
+  }
+}
+
+// The pieces as fp32 rows of dst at chunk position pos(tt) (rows with pos < 0
+// are dropped), each element passed through f.
+template <typename T, int D, int NT, typename Pos, typename F>
+__device__ __forceinline__ void store_pieces(const uint4 (&r)[Pieces<T, D, NT>::CNT], float* dst, int NW, Pos pos,
+                                             F f) {
+  using P = Pieces<T, D, NT>;
+#pragma unroll
+  for (int j = 0; j < P::CNT; ++j) {
+    const int pc = threadIdx.x + j * NT;
+    if (pc < NW * P::PER_ROW) {
+      const int p = pos(pc / P::PER_ROW), o = pc % P::PER_ROW;
+      if (p >= 0) {
+        const uint32_t w[4] = {r[j].x, r[j].y, r[j].z, r[j].w};
+        float e[P::EPP];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          if constexpr (sizeof(T) == 2) {  // bf16 pairs
+            e[2 * u] = f(__uint_as_float(w[u] << 16));
+            e[2 * u + 1] = f(__uint_as_float(w[u] & 0xffff0000u));
+          } else {
+            e[u] = f(__uint_as_float(w[u]));
+          }
+        }
+        float4* d4 = reinterpret_cast<float4*>(dst + p * D + o * P::EPP);
+#pragma unroll
+        for (int u = 0; u < P::EPP / 4; ++u) d4[u] = make_float4(e[4 * u], e[4 * u + 1], e[4 * u + 2], e[4 * u + 3]);
+      }
+    }
+  }
+}
+
 struct SpecTok {  // where one token's inputs live
   const void* q;
   const void* k;
@@ -92,35 +148,16 @@ __global__ void __launch_bounds__(SpecShape<DK, DV>::NT, 2)
   // rows x 4 columns per thread): its 64 KiB stream in while the chunk's own
   // arithmetic runs.
   const int NW = Wp + W;
-  auto row_of = [&](int tt) {  // token tt of the two windows -> its [b, t, h] row
-    return tt < Wp ? ((int64_t)b * Wp + tt) * H + h : ((int64_t)b * W + (tt - Wp)) * H + h;
-  };
-  constexpr int PK = (KDA_SPEC_MAX_TOKENS * DK + NT - 1) / NT, PV = (KDA_SPEC_MAX_TOKENS * DV + NT - 1) / NT;
-  float rk[PK], rq[PK], rg2[PK], rv[PV];
-#pragma unroll
-  for (int j = 0; j < PK; ++j) {
-    const int e = tid + j * NT;
-    if (e < NW * DK) {
-      const int tt = e / DK, i = e % DK;
-      const SpecTok& src = tt < Wp ? prev : cur;
-      const int64_t o = row_of(tt) * DK + i;
-      rk[j] = to_f32(static_cast<const IO*>(src.k)[o]);
-      rq[j] = to_f32(static_cast<const IO*>(src.q)[o]);
-      if constexpr (GATED)
-        rg2[j] = to_f32(static_cast<const IO*>(src.g)[o]);
-      else
-        rg2[j] = static_cast<const float*>(src.g)[o];
-    }
-  }
-#pragma unroll
-  for (int j = 0; j < PV; ++j) {
-    const int e = tid + j * NT;
-    if (e < NW * DV) {
-      const int tt = e / DV, i = e % DV;
-      rv[j] = to_f32(static_cast<const IO*>((tt < Wp ? prev : cur).v)[row_of(tt) * DV + i]);
-    }
-  }
-  const float bt = tid < NW ? (tid < Wp ? prev : cur).beta[row_of(tid)] : 0.f;
+  using GT = typename std::conditional<GATED, IO, float>::type;  // element type of the decay input
+  uint4 pk[Pieces<IO, DK, NT>::CNT], pq[Pieces<IO, DK, NT>::CNT], pg[Pieces<GT, DK, NT>::CNT],
+      pv[Pieces<IO, DV, NT>::CNT];
+  load_pieces<IO, DK, NT>(prev.k, cur.k, NW, Wp, W, b, H, h, pk);
+  load_pieces<IO, DK, NT>(prev.q, cur.q, NW, Wp, W, b, H, h, pq);
+  load_pieces<GT, DK, NT>(prev.g, cur.g, NW, Wp, W, b, H, h, pg);
+  load_pieces<IO, DV, NT>(prev.v, cur.v, NW, Wp, W, b, H, h, pv);
+  const float bt = tid < NW ? (tid < Wp ? prev.beta[((int64_t)b * Wp + tid) * H + h]
+                                        : cur.beta[((int64_t)b * W + (tid - Wp)) * H + h])
+                            : 0.f;
   int na = n_accepted ? n_accepted[b] : 0;
   na = na < 0 ? 0 : (na > Wp ? Wp : na);
   const int n = na + W;               // tokens of the chunk
@@ -130,7 +167,8 @@ __global__ void __launch_bounds__(SpecShape<DK, DV>::NT, 2)
   //   s_k, s_q, s_G [n][DK]  k, q, G (token-major; later the partial sums)
   //   s_v, s_d [n][DV]       values, delta
   //   s_A, s_P [n][n4]       pair sums;  s_b [n4] beta;  s_gc [DK] e^{G_c}
-  //   s_ek, s_eq, s_kc [DK][ld]  e^G k, e^G q, k e^{G_c - G}, channel-major (0 past the chunk)
+  //   s_ek, s_eq [DK][ld]    e^G k, e^G q, channel-major (0 past the chunk)
+  //   s_kc [n4][DK]          k e^{G_c - G}, token-major (0 past the kept token)
   //   s_xy [n][2 DV]         X_t, then Y_t
   const int n4 = (n + 3) & ~3, ld = spec_ld(n4);
   const int tok = 3 * n * DK > Sh::PART ? 3 * n * DK : Sh::PART;
@@ -153,33 +191,21 @@ __global__ void __launch_bounds__(SpecShape<DK, DV>::NT, 2)
   {
     const float Ah = GATED ? A_log[h] : 0.f;
     auto pos = [&](int tt) { return tt < Wp ? (tt < na ? tt : -1) : na + (tt - Wp); };
-#pragma unroll
-    for (int j = 0; j < PK; ++j) {
-      const int e = tid + j * NT;
-      if (e < NW * DK) {
-        const int p = pos(e / DK), i = e % DK;
-        if (p >= 0) {
-          s_k[p * DK + i] = rk[j];
-          s_q[p * DK + i] = rq[j];
-          s_G[p * DK + i] = GATED ? gate_log_decay(rg2[j], Ah, g_min) : rg2[j];
-        }
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < PV; ++j) {
-      const int e = tid + j * NT;
-      if (e < NW * DV) {
-        const int p = pos(e / DV);
-        if (p >= 0) s_v[p * DV + e % DV] = rv[j];
-      }
-    }
+    auto same = [](float x) { return x; };
+    store_pieces<IO, DK, NT>(pk, s_k, NW, pos, same);
+    store_pieces<IO, DK, NT>(pq, s_q, NW, pos, same);
+    if constexpr (GATED)
+      store_pieces<GT, DK, NT>(pg, s_G, NW, pos, [&](float z) { return gate_log_decay(z, Ah, g_min); });
+    else
+      store_pieces<GT, DK, NT>(pg, s_G, NW, pos, same);
+    store_pieces<IO, DV, NT>(pv, s_v, NW, pos, same);
     if (tid < NW && pos(tid) >= 0) s_b[pos(tid)] = bt;
   }
+  __syncthreads();
   float4* S = reinterpret_cast<float4*>(state + ((int64_t)b * H + h) * DK * DV);
   float4 s[ROWS];  // rows rg * ROWS + m, columns 4 cq .. 4 cq + 3; first used by the X, Y products
 #pragma unroll
   for (int m = 0; m < ROWS; ++m) s[m] = __ldcs(S + (rg * ROWS + m) * COLQ + cq);
-  __syncthreads();
   if constexpr (GATED) {  // L2-normalise q and k per token, one warp per token
     for (int t = warp; t < n; t += NT / 32) {
       float qq = 0.f, kk = 0.f;
@@ -228,7 +254,7 @@ __global__ void __launch_bounds__(SpecShape<DK, DV>::NT, 2)
       }
       s_ek[i * ld + t] = ek;
       s_eq[i * ld + t] = eq;
-      s_kc[i * ld + t] = kc;
+      s_kc[t * DK + i] = kc;
     }
   }
   // Four pairs per warp at a time (pairs in row order: p -> (t, s)): each
@@ -277,7 +303,7 @@ __global__ void __launch_bounds__(SpecShape<DK, DV>::NT, 2)
   // shared memory (the token-major arrays are no longer needed).
   auto xy_group = [&](auto tb, int t0) {
     constexpr int TB = decltype(tb)::value;
-#pragma unroll
+#pragma unroll 1
     for (int xy = 0; xy < 2; ++xy) {  // X from e^G k, then Y from e^G q (16 accumulators at a time)
       const float* src = xy ? s_eq : s_ek;
       float acc[TB][4];
@@ -348,24 +374,37 @@ __global__ void __launch_bounds__(SpecShape<DK, DV>::NT, 2)
   }
   __syncthreads();
 
-  // ---- the kept state: S_c = Diag(e^{G_c}) S0 + sum_{s<=c} (k_s e^{G_c - G_s}) delta_s^T
+  // ---- the kept state: S_c = Diag(e^{G_c}) S0 + sum_{s<=c} (k_s e^{G_c - G_s}) delta_s^T,
+  // updated in the state registers token by token (the thread's ROWS
+  // consecutive rows: its k e^{G_c - G} entries are contiguous).
+  {
+    const float* eg = s_gc + rg * ROWS;
 #pragma unroll
-  for (int m = 0; m < ROWS; ++m) {
-    const int i = rg * ROWS + m;
-    const float eg = s_gc[i];
-    float4 a = make_float4(s[m].x * eg, s[m].y * eg, s[m].z * eg, s[m].w * eg);
-    for (int t0 = 0; t0 <= c; t0 += 4) {
-      const float4 kq = *reinterpret_cast<const float4*>(s_kc + i * ld + t0);
-      const float kv[4] = {kq.x, kq.y, kq.z, kq.w};
+    for (int m = 0; m < ROWS; ++m) {
+      const float e = eg[m];
+      s[m].x *= e; s[m].y *= e; s[m].z *= e; s[m].w *= e;
+    }
+    for (int t = 0; t <= c; ++t) {
+      const float4 ds = *reinterpret_cast<const float4*>(s_d + t * DV + 4 * cq);
+      const float* kc = s_kc + t * DK + rg * ROWS;
+      float kv[ROWS];
+      if constexpr (ROWS % 4 == 0) {
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        if (t0 + u <= c) {
-          const float4 ds = *reinterpret_cast<const float4*>(s_d + (t0 + u) * DV + 4 * cq);
-          a.x += kv[u] * ds.x; a.y += kv[u] * ds.y; a.z += kv[u] * ds.z; a.w += kv[u] * ds.w;
+        for (int m = 0; m < ROWS; m += 4) {
+          const float4 k4 = *reinterpret_cast<const float4*>(kc + m);
+          kv[m] = k4.x; kv[m + 1] = k4.y; kv[m + 2] = k4.z; kv[m + 3] = k4.w;
         }
+      } else {
+#pragma unroll
+        for (int m = 0; m < ROWS; ++m) kv[m] = kc[m];
+      }
+#pragma unroll
+      for (int m = 0; m < ROWS; ++m) {
+        s[m].x += kv[m] * ds.x; s[m].y += kv[m] * ds.y; s[m].z += kv[m] * ds.z; s[m].w += kv[m] * ds.w;
       }
     }
-    __stcs(S + (rg * ROWS + m) * COLQ + cq, a);
+#pragma unroll
+    for (int m = 0; m < ROWS; ++m) __stcs(S + (rg * ROWS + m) * COLQ + cq, s[m]);
   }
 }
 
