@@ -53,19 +53,14 @@ struct SpecShape {
   static constexpr int PART = RG * 4 * 2 * DV;                         // floats of partial X, Y sums
 };
 
-// Row stride (floats) of the channel-major operand arrays for chunks of n4
-// (a multiple of 4) tokens: an odd number of float4s, so the 16-byte reads of
-// eight consecutive channels hit eight different bank quads.
-__host__ __device__ constexpr int spec_ld(int n4) { return (n4 / 4) % 2 ? n4 : n4 + 4; }
-
 // Shared-memory floats of a block for chunks of up to `n` tokens (the
 // token-major arrays and the partial sums share one region).
 template <int DK, int DV>
 constexpr size_t spec_smem_floats(int n) {
   const size_t n4 = (size_t)((n + 3) & ~3);
-  const size_t tok = 3 * (size_t)n * DK, part = (size_t)SpecShape<DK, DV>::PART;
-  return (tok > part ? tok : part) + 2 * (size_t)n * DV + 2 * (size_t)n * n4 + n4 + DK +
-         3 * (size_t)DK * spec_ld((int)n4) + 2 * (size_t)n * DV;
+  const size_t tok = 4 * (size_t)n * DK, part = (size_t)SpecShape<DK, DV>::PART;
+  return (tok > part ? tok : part) + 2 * (size_t)n * DV + 2 * (size_t)n * n4 + n4 + DK + 3 * n4 * DK +
+         2 * (size_t)n * DV;
 }
 
 // One token array of both windows in 16-byte pieces (rows of D elements of T;
@@ -164,17 +159,18 @@ __global__ void __launch_bounds__(SpecShape<DK, DV>::NT, 2)
   const int c = W > 0 ? na : na - 1;  // the token after which the state is kept (-1: none, unchanged)
   if (c < 0) return;
   // shared layout (floats; every array starts on a multiple of 4 floats):
-  //   s_k, s_q, s_G [n][DK]  k, q, G (token-major; later the partial sums)
+  //   s_k, s_q, s_G, s_al [n][DK]  k, q, G, e^{g} (later the partial sums)
   //   s_v, s_d [n][DV]       values, delta
   //   s_A, s_P [n][n4]       pair sums;  s_b [n4] beta;  s_gc [DK] e^{G_c}
-  //   s_ek, s_eq [DK][ld]    e^G k, e^G q, channel-major (0 past the chunk)
-  //   s_kc [n4][DK]          k e^{G_c - G}, token-major (0 past the kept token)
+  //   s_ek, s_eq, s_kc [n4][DK]  e^G k, e^G q, k e^{G_c - G} (0 past the chunk / the kept token)
   //   s_xy [n][2 DV]         X_t, then Y_t
-  const int n4 = (n + 3) & ~3, ld = spec_ld(n4);
-  const int tok = 3 * n * DK > Sh::PART ? 3 * n * DK : Sh::PART;
+  // (all token-major: a thread's ROWS consecutive rows of one token are contiguous)
+  const int n4 = (n + 3) & ~3;
+  const int tok = 4 * n * DK > Sh::PART ? 4 * n * DK : Sh::PART;
   float* s_k = ssm;
   float* s_q = s_k + n * DK;
   float* s_G = s_q + n * DK;
+  float* s_al = s_G + n * DK;
   float* s_part = ssm;
   float* s_v = ssm + tok;
   float* s_d = s_v + n * DV;
@@ -183,9 +179,9 @@ __global__ void __launch_bounds__(SpecShape<DK, DV>::NT, 2)
   float* s_b = s_P + n * n4;
   float* s_gc = s_b + n4;
   float* s_ek = s_gc + DK;
-  float* s_eq = s_ek + DK * ld;
-  float* s_kc = s_eq + DK * ld;
-  float* s_xy = s_kc + DK * ld;
+  float* s_eq = s_ek + n4 * DK;
+  float* s_kc = s_eq + n4 * DK;
+  float* s_xy = s_kc + n4 * DK;
 
   // ---- lay out the chunk: prev[0, na) at 0 .. na-1, cur[0, W) at na ..
   {
@@ -226,74 +222,94 @@ __global__ void __launch_bounds__(SpecShape<DK, DV>::NT, 2)
     }
     __syncthreads();
   }
-  // ---- cumulative log-decay over the chunk, one thread per key channel
+  // ---- cumulative log-decay over the chunk and the per-token decays
+  // alpha_t = e^{g_t}, one thread per key channel
   for (int i = tid; i < DK; i += NT) {
     float acc = 0.f;
     for (int t = 0; t < n; ++t) {
-      acc += s_G[t * DK + i];
+      const float g = s_G[t * DK + i];
+      acc += g;
       s_G[t * DK + i] = acc;
+      s_al[t * DK + i] = __expf(g);
     }
   }
   __syncthreads();
-  // ---- per-token operands, channel-major, one thread per channel:
-  // e^{G_t} k_t, e^{G_t} q_t, k_t e^{G_c - G_t} (t <= c); zero for the tokens
-  // past the chunk (up to n4).  Then (no barrier: other arrays) the pair
-  // sums A_ts (s < t; the diagonal entry written is not used) and P_ts (s <= t).
-  for (int i = tid; i < DK; i += NT) {
-    const float gc = s_G[c * DK + i];
-    s_gc[i] = __expf(gc);
-#pragma unroll 4
-    for (int t = 0; t < n4; ++t) {
-      float ek = 0.f, eq = 0.f, kc = 0.f;
-      if (t < n) {
-        const float G = s_G[t * DK + i], kk = s_k[t * DK + i];
-        const float eg = __expf(G);
-        ek = eg * kk;
-        eq = eg * s_q[t * DK + i];
-        kc = t <= c ? kk * __expf(gc - G) : 0.f;
-      }
-      s_ek[i * ld + t] = ek;
-      s_eq[i * ld + t] = eq;
-      s_kc[t * DK + i] = kc;
+  // ---- per-token operands, four channels per work item: e^{G_t} k_t,
+  // e^{G_t} q_t, k_t e^{G_c - G_t} (t <= c), zero past the chunk (up to n4),
+  // and e^{G_c}.  Then (no barrier: other arrays) the pair sums.
+  for (int w = tid; w < n4 * (DK / 4); w += NT) {
+    const int t = w / (DK / 4), i0 = 4 * (w % (DK / 4));
+    float4 ek = make_float4(0.f, 0.f, 0.f, 0.f), eq = ek, kc = ek;
+    if (t < n) {
+      const float4 G = *reinterpret_cast<const float4*>(s_G + t * DK + i0);
+      const float4 Gc = *reinterpret_cast<const float4*>(s_G + c * DK + i0);
+      const float4 kk = *reinterpret_cast<const float4*>(s_k + t * DK + i0);
+      const float4 qq = *reinterpret_cast<const float4*>(s_q + t * DK + i0);
+      const float4 e = make_float4(__expf(G.x), __expf(G.y), __expf(G.z), __expf(G.w));
+      ek = make_float4(e.x * kk.x, e.y * kk.y, e.z * kk.z, e.w * kk.w);
+      eq = make_float4(e.x * qq.x, e.y * qq.y, e.z * qq.z, e.w * qq.w);
+      if (t <= c)
+        kc = make_float4(kk.x * __expf(Gc.x - G.x), kk.y * __expf(Gc.y - G.y), kk.z * __expf(Gc.z - G.z),
+                         kk.w * __expf(Gc.w - G.w));
+      if (t == c) *reinterpret_cast<float4*>(s_gc + i0) = e;
     }
+    *reinterpret_cast<float4*>(s_ek + t * DK + i0) = ek;
+    *reinterpret_cast<float4*>(s_eq + t * DK + i0) = eq;
+    *reinterpret_cast<float4*>(s_kc + t * DK + i0) = kc;
   }
-  // Four pairs per warp at a time (pairs in row order: p -> (t, s)): each
-  // lane sums its channels for the 8 values (A, P of 4 pairs), the warp
-  // reduce-scatters them (offsets 4, 2, 1: lane l keeps value l & 7), then
-  // adds across the remaining lane bits (offsets 8, 16).
-  const int npairs = n * (n + 1) / 2;
-  for (int p0 = warp * 4; p0 < npairs; p0 += NT / 32 * 4) {
-    int tq[4], sq[4];
+  // Pair sums A_ts (s < t) and P_ts (s <= t), one warp per s (s = warp, then
+  // mirrored so that the warps' loads even out), four channels per lane: the
+  // decay e^{G_t - G_s} is the running product of alpha over s < u <= t
+  // (every factor <= 1).  The lane sums for t in an 8-token half are
+  // reduce-scattered over the warp (offsets 8, 4, 2, 1: lane l keeps value
+  // l & 15 = 2 (t - t_half) + {0: A, 1: P}), then added across offset 16.
+  {
+    constexpr int NWARP = NT / 32;
+    const bool lane_on = 4 * lane < DK;
+    const int i0 = lane_on ? 4 * lane : 0;
+    for (int r = 0; r * NWARP < n; ++r) {
+      const int s2 = (r & 1) ? (r + 1) * NWARP - 1 - warp : r * NWARP + warp;
+      if (s2 >= n) continue;
+      const float4 ks = lane_on ? *reinterpret_cast<const float4*>(s_k + s2 * DK + i0) : make_float4(0.f, 0.f, 0.f, 0.f);
+      float4 f = make_float4(1.f, 1.f, 1.f, 1.f);
+#pragma unroll 1
+      for (int th = (s2 / 8) * 8; th < n; th += 8) {  // 8-token halves of t that reach s
+        float v[16];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int p = p0 + q < npairs ? p0 + q : 0;
-      int t = 0;
-      while ((t + 1) * (t + 2) / 2 <= p) ++t;
-      tq[q] = t;
-      sq[q] = p - t * (t + 1) / 2;
-    }
-    float v[8];
+        for (int j = 0; j < 16; ++j) v[j] = 0.f;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) v[j] = 0.f;
-    for (int i = lane; i < DK; i += 32) {
+        for (int u = 0; u < 8; ++u) {
+          const int t = th + u;
+          if (t >= s2 && t < n) {
+            if (t > s2) {
+              const float4 al = *reinterpret_cast<const float4*>(s_al + t * DK + i0);
+              f.x *= al.x; f.y *= al.y; f.z *= al.z; f.w *= al.w;
+            }
+            const float4 ke = make_float4(ks.x * f.x, ks.y * f.y, ks.z * f.z, ks.w * f.w);
+            const float4 kt = *reinterpret_cast<const float4*>(s_k + t * DK + i0);
+            const float4 qt = *reinterpret_cast<const float4*>(s_q + t * DK + i0);
+            v[2 * u] = (kt.x * ke.x + kt.y * ke.y) + (kt.z * ke.z + kt.w * ke.w);
+            v[2 * u + 1] = (qt.x * ke.x + qt.y * ke.y) + (qt.z * ke.z + qt.w * ke.w);
+          }
+        }
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int t = tq[q], s2 = sq[q];
-        const float ke = s_k[s2 * DK + i] * __expf(s_G[t * DK + i] - s_G[s2 * DK + i]);  // decay s -> t, <= 1
-        v[2 * q] += s_k[t * DK + i] * ke;
-        v[2 * q + 1] += s_q[t * DK + i] * ke;
+        for (int o = 8; o >= 1; o >>= 1) {
+          const bool up = lane & o;
+#pragma unroll
+          for (int j = 0; j < o; ++j)
+            v[j] = (up ? v[j + o] : v[j]) + __shfl_xor_sync(0xffffffffu, up ? v[j] : v[j + o], o);
+        }
+        v[0] += __shfl_xor_sync(0xffffffffu, v[0], 16);
+        const int t = th + ((lane & 15) >> 1);
+        if (lane < 16 && t < n) {
+          if (lane & 1) {
+            if (t >= s2) s_P[t * n4 + s2] = v[0];
+          } else if (t > s2) {
+            s_A[t * n4 + s2] = v[0];
+          }
+        }
       }
     }
-#pragma unroll
-    for (int o = 4; o >= 1; o >>= 1) {
-      const bool up = lane & o;
-#pragma unroll
-      for (int j = 0; j < o; ++j) v[j] = (up ? v[j + o] : v[j]) + __shfl_xor_sync(0xffffffffu, up ? v[j] : v[j + o], o);
-    }
-    v[0] += __shfl_xor_sync(0xffffffffu, v[0], 8);
-    v[0] += __shfl_xor_sync(0xffffffffu, v[0], 16);
-    const int q = (lane >> 1) & 3;
-    if (lane < 8 && p0 + q < npairs) (lane & 1 ? s_P : s_A)[tq[q] * n4 + sq[q]] = v[0];
   }
   __syncthreads();
 
@@ -310,22 +326,23 @@ __global__ void __launch_bounds__(SpecShape<DK, DV>::NT, 2)
 #pragma unroll
       for (int u = 0; u < TB; ++u) acc[u][0] = acc[u][1] = acc[u][2] = acc[u][3] = 0.f;
 #pragma unroll
-      for (int m = 0; m < ROWS; ++m) {
-        const int i = rg * ROWS + m;
-        float ev[TB];
-        if constexpr (TB == 4) {
-          const float4 e4 = *reinterpret_cast<const float4*>(src + i * ld + t0);
-          ev[0] = e4.x; ev[1] = e4.y; ev[2] = e4.z; ev[3] = e4.w;
-        } else if constexpr (TB == 2) {
-          const float2 e2 = *reinterpret_cast<const float2*>(src + i * ld + t0);
-          ev[0] = e2.x; ev[1] = e2.y;
+      for (int u = 0; u < TB; ++u) {
+        const float* e = src + (t0 + u) * DK + rg * ROWS;  // this token's entries for the thread's rows
+        float ev[ROWS];
+        if constexpr (ROWS % 4 == 0) {
+#pragma unroll
+          for (int m = 0; m < ROWS; m += 4) {
+            const float4 e4 = *reinterpret_cast<const float4*>(e + m);
+            ev[m] = e4.x; ev[m + 1] = e4.y; ev[m + 2] = e4.z; ev[m + 3] = e4.w;
+          }
         } else {
-          ev[0] = src[i * ld + t0];
+#pragma unroll
+          for (int m = 0; m < ROWS; ++m) ev[m] = e[m];
         }
 #pragma unroll
-        for (int u = 0; u < TB; ++u) {
-          acc[u][0] += s[m].x * ev[u]; acc[u][1] += s[m].y * ev[u];
-          acc[u][2] += s[m].z * ev[u]; acc[u][3] += s[m].w * ev[u];
+        for (int m = 0; m < ROWS; ++m) {
+          acc[u][0] += s[m].x * ev[m]; acc[u][1] += s[m].y * ev[m];
+          acc[u][2] += s[m].z * ev[m]; acc[u][3] += s[m].w * ev[m];
         }
       }
 #pragma unroll
