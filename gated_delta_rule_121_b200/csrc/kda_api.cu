@@ -1,8 +1,11 @@
 // C ABI of libkda.so (declared in include/kda.h): host-side validation,
-// workspace layout and kernel dispatch.  No entry point allocates, frees or
-// synchronises, except kda_workspace_status which reads back a status word.
+// workspace layout and kernel dispatch.  No entry point allocates device
+// memory, frees or synchronises, except kda_workspace_status which reads back
+// a status word; kda_fwd_host makes two streams and a few events per device
+// on its first pipelined call and keeps them.
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "../../include/kda.h"
 #include "../../include/kda_testing.h"
@@ -25,6 +28,7 @@ int fwd_tc_debug_floats();
 namespace {
 
 constexpr size_t kStatusBytes = 256;  // DeviceStatus + reserve
+constexpr uint64_t kWaitNs = 2000000000ull;  // limit of every in-kernel wait (2 s)
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool dim_ok(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
@@ -74,7 +78,8 @@ static kda_status_t fwd_impl(const void* q, const void* k, const void* v, const 
                              const float* beta, const float* init_state, void* out, float* final_state, int B,
                              int64_t T, int H, int dk, int dv, const int32_t* cu_seqlens, void* stream,
                              kda_dtype_t dt, void* workspace, size_t workspace_bytes, float* dbg,
-                             uint64_t wait_ns, int inject_stuck, const kda::ModeArgs& ma = kda::ModeArgs()) {
+                             uint64_t wait_ns, int inject_stuck, const kda::ModeArgs& ma = kda::ModeArgs(),
+                             bool reset_status = true) {
   // Segment runs write fp32 outputs to their own buffers (out may be NULL).
   const void* out_chk = ma.mode == kda::MODE_SEG ? (const void*)(ma.o32 ? ma.o32 : final_state) : out;
   kda_status_t st = validate_fwd(q, k, v, log_alpha, beta, init_state, out_chk, final_state, B, T, H, dk, dv, dt);
@@ -86,7 +91,7 @@ static kda_status_t fwd_impl(const void* q, const void* k, const void* v, const 
   if ((cu_seqlens ? T : (int64_t)B * T) > (int64_t)INT32_MAX) return KDA_ERR_UNSUPPORTED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   kda::DeviceStatus* status = reinterpret_cast<kda::DeviceStatus*>(workspace);
-  if (cudaMemsetAsync(status, 0, sizeof(kda::DeviceStatus), s) != cudaSuccess) return KDA_ERR_CUDA;
+  if (reset_status && cudaMemsetAsync(status, 0, sizeof(kda::DeviceStatus), s) != cudaSuccess) return KDA_ERR_CUDA;
   if (B == 0) return KDA_OK;
   kda::FwdArgs a{q, k, v, log_alpha, beta, init_state, out, final_state, cu_seqlens, B, T, H, dk, dv, status, dbg};
   const bool bf16 = dt == KDA_BF16;
@@ -107,8 +112,67 @@ kda_status_t kda_fwd(const void* q, const void* k, const void* v, const float* l
                      int dv, const int32_t* cu_seqlens, void* stream, kda_dtype_t dt, void* workspace,
                      size_t workspace_bytes) {
   return fwd_impl(q, k, v, log_alpha, beta, init_state, out, final_state, B, T, H, dk, dv, cu_seqlens, stream,
-                  dt, workspace, workspace_bytes, nullptr, 2000000000ull, 0);
+                  dt, workspace, workspace_bytes, nullptr, kWaitNs, 0);
 }
+
+namespace {
+
+constexpr int kHostPieces = 8;  // pieces of a pipelined kda_fwd_host call, at most
+
+// Streams and events of the pipelined host path, one set per device, made on
+// first use and kept for the life of the process.
+struct HostPipe {
+  cudaStream_t in = nullptr, out = nullptr;
+  cudaEvent_t start = nullptr, done = nullptr, ev_in[kHostPieces], ev_comp[kHostPieces];
+};
+std::mutex g_pipe_mu;
+HostPipe g_pipe[64];
+bool g_pipe_ready[64];
+
+HostPipe* host_pipe(int dev) {  // call with g_pipe_mu held
+  if (dev < 0 || dev >= 64) return nullptr;
+  HostPipe& p = g_pipe[dev];
+  if (g_pipe_ready[dev]) return &p;
+  bool ok = cudaStreamCreateWithFlags(&p.in, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaStreamCreateWithFlags(&p.out, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaEventCreateWithFlags(&p.start, cudaEventDisableTiming) == cudaSuccess &&
+            cudaEventCreateWithFlags(&p.done, cudaEventDisableTiming) == cudaSuccess;
+  for (int i = 0; ok && i < kHostPieces; ++i)
+    ok = cudaEventCreateWithFlags(&p.ev_in[i], cudaEventDisableTiming) == cudaSuccess &&
+         cudaEventCreateWithFlags(&p.ev_comp[i], cudaEventDisableTiming) == cudaSuccess;
+  if (!ok) return nullptr;
+  g_pipe_ready[dev] = true;
+  return &p;
+}
+
+// Pieces of a batched (no cu_seqlens) kda_fwd_host call: whole sequences
+// [b0, b1) when B > 1, else token slices [t0, t1) of the one sequence whose
+// starts are multiples of the 64-token chunk (so every piece's chunks are the
+// unsliced call's chunks and the results are the same bits).
+struct Piece {
+  int b0, b1;
+  int64_t t0, t1;
+};
+int plan_pieces(int B, int64_t T, Piece* pc) {
+  if (B > 1) {
+    const int n = B < kHostPieces ? B : kHostPieces;
+    for (int i = 0; i < n; ++i) pc[i] = {(int)((int64_t)B * i / n), (int)((int64_t)B * (i + 1) / n), 0, T};
+    return n;
+  }
+  const int64_t chunks = (T + 63) / 64;
+  const int n = (int)(chunks < kHostPieces ? chunks : kHostPieces);
+  if (n <= 1) {
+    pc[0] = {0, B, 0, T};
+    return 1;
+  }
+  for (int i = 0; i < n; ++i) {
+    const int64_t c0 = chunks * i / n, c1 = chunks * (i + 1) / n;
+    pc[i] = {0, 1, 64 * c0, c1 == chunks ? T : 64 * c1};
+  }
+  return n;
+}
+
+}  // namespace
 
 kda_status_t kda_fwd_host(const kda_fwd_tensors_t* host, const kda_fwd_tensors_t* dev, int B, int64_t T, int H,
                           int dk, int dv, void* stream, kda_dtype_t dt, void* workspace, size_t workspace_bytes) {
@@ -117,39 +181,120 @@ kda_status_t kda_fwd_host(const kda_fwd_tensors_t* host, const kda_fwd_tensors_t
       (host->cu_seqlens == nullptr) != (dev->cu_seqlens == nullptr))
     return KDA_ERR_INVALID_ARG;
   if (B < 0 || T < 0 || H <= 0 || (dt != KDA_F32 && dt != KDA_BF16)) return KDA_ERR_INVALID_ARG;
+  kda_status_t st = validate_fwd(dev->q, dev->k, dev->v, dev->log_alpha, dev->beta, dev->init_state, dev->out,
+                                 dev->final_state, B, T, H, dk, dv, dt);
+  if (st != KDA_OK) return st;
   const bool packed = dev->cu_seqlens != nullptr;
   const int64_t tokens = packed ? T : (int64_t)B * T;
   const size_t esz = dt == KDA_BF16 ? 2 : 4;
   const size_t th = (size_t)tokens * H;
-  const size_t states = (size_t)B * H * dk * dv * sizeof(float);
+  const size_t state1 = (size_t)H * dk * dv * sizeof(float);  // one sequence's state
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  struct Copy {
-    void* dst;
-    const void* src;
-    size_t bytes;
+  const void* hin[] = {host->q, host->k, host->v, host->log_alpha, host->beta};
+  for (const void* p : hin)
+    if (th > 0 && !p) return KDA_ERR_INVALID_ARG;
+  Piece pc[kHostPieces];
+  // One piece (every copy, the forward, the copies back, in order on `stream`)
+  // for packed batches and where a token-sliced sequence has no final-state
+  // buffer to carry its state; otherwise pieces whose copies in, forward and
+  // copies out overlap across three streams.
+  int np = (packed || tokens == 0 || (B == 1 && !dev->final_state)) ? 1 : plan_pieces(B, T, pc);
+  for (int i = 0; i < np; ++i)  // beta rows are H floats: a piece must start on a 16-byte boundary
+    if ((((int64_t)pc[i].b0 * T + pc[i].t0) * H * 4) % 16 != 0) np = 1;
+  if (np == 1) pc[0] = {0, B, 0, T};
+  // Token tensors of a piece: rows [t0, t1) of sequences [b0, b1), one 2-D copy
+  // (a row per sequence) per tensor.
+  const size_t wq = (size_t)H * dk * esz, wv = (size_t)H * dv * esz, wg = (size_t)H * dk * 4, wb = (size_t)H * 4;
+  auto copy_tokens = [&](const Piece& p, cudaStream_t cs, bool in) -> bool {
+    const int64_t rows = packed ? 1 : p.b1 - p.b0;
+    const int64_t len = packed ? T : p.t1 - p.t0;
+    if (rows == 0 || len == 0) return true;
+    const int64_t first = packed ? 0 : (int64_t)p.b0 * T + p.t0;  // first token of the piece
+    struct C {
+      void* d;
+      const void* h;
+      size_t w;
+    };
+    if (in) {
+      const C cs_in[] = {{const_cast<void*>(dev->q), host->q, wq},
+                         {const_cast<void*>(dev->k), host->k, wq},
+                         {const_cast<void*>(dev->v), host->v, wv},
+                         {const_cast<float*>(dev->log_alpha), host->log_alpha, wg},
+                         {const_cast<float*>(dev->beta), host->beta, wb}};
+      for (const C& c : cs_in) {
+        char* d = static_cast<char*>(c.d) + first * c.w;
+        const char* h = static_cast<const char*>(c.h) + first * c.w;
+        if (cudaMemcpy2DAsync(d, T * c.w, h, T * c.w, len * c.w, rows, cudaMemcpyHostToDevice, cs) != cudaSuccess)
+          return false;
+      }
+    } else if (host->out) {
+      char* h = static_cast<char*>(host->out) + first * wv;
+      const char* d = static_cast<const char*>(dev->out) + first * wv;
+      if (cudaMemcpy2DAsync(h, T * wv, d, T * wv, len * wv, rows, cudaMemcpyDeviceToHost, cs) != cudaSuccess)
+        return false;
+    }
+    return true;
   };
-  const Copy in[] = {{const_cast<void*>(dev->q), host->q, th * dk * esz},
-                     {const_cast<void*>(dev->k), host->k, th * dk * esz},
-                     {const_cast<void*>(dev->v), host->v, th * dv * esz},
-                     {const_cast<float*>(dev->log_alpha), host->log_alpha, th * dk * sizeof(float)},
-                     {const_cast<float*>(dev->beta), host->beta, th * sizeof(float)},
-                     {const_cast<float*>(dev->init_state), host->init_state, dev->init_state ? states : 0},
-                     {const_cast<int32_t*>(dev->cu_seqlens), host->cu_seqlens,
-                      packed ? (size_t)(B + 1) * sizeof(int32_t) : 0}};
-  for (const Copy& c : in) {
-    if (c.bytes == 0) continue;
-    if (!c.dst || !c.src) return KDA_ERR_INVALID_ARG;
-    if (cudaMemcpyAsync(c.dst, c.src, c.bytes, cudaMemcpyHostToDevice, s) != cudaSuccess) return KDA_ERR_CUDA;
+  const size_t states = (size_t)B * state1;  // B sequences (packed: B = N)
+  if (np == 1) {  // everything in order on the caller's stream
+    if (!copy_tokens(pc[0], s, true)) return KDA_ERR_CUDA;
+    if (dev->init_state && states > 0 &&
+        cudaMemcpyAsync(const_cast<float*>(dev->init_state), host->init_state, states, cudaMemcpyHostToDevice, s) !=
+            cudaSuccess)
+      return KDA_ERR_CUDA;
+    if (packed && cudaMemcpyAsync(const_cast<int32_t*>(dev->cu_seqlens), host->cu_seqlens,
+                                  (size_t)(B + 1) * sizeof(int32_t), cudaMemcpyHostToDevice, s) != cudaSuccess)
+      return KDA_ERR_CUDA;
+    st = kda_fwd(dev->q, dev->k, dev->v, dev->log_alpha, dev->beta, dev->init_state, dev->out, dev->final_state, B,
+                 T, H, dk, dv, dev->cu_seqlens, stream, dt, workspace, workspace_bytes);
+    if (st != KDA_OK) return st;
+    if (th > 0 && !copy_tokens(pc[0], s, false)) return KDA_ERR_CUDA;
+    if (host->final_state && dev->final_state && states > 0 &&
+        cudaMemcpyAsync(host->final_state, dev->final_state, states, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+      return KDA_ERR_CUDA;
+    return KDA_OK;
   }
-  kda_status_t st = kda_fwd(dev->q, dev->k, dev->v, dev->log_alpha, dev->beta, dev->init_state, dev->out,
-                            dev->final_state, B, T, H, dk, dv, dev->cu_seqlens, stream, dt, workspace,
-                            workspace_bytes);
-  if (st != KDA_OK) return st;
-  if (host->out && th > 0 &&
-      cudaMemcpyAsync(host->out, dev->out, th * dv * esz, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+  if (!workspace || !aligned16(workspace) || workspace_bytes < kda_fwd_workspace_size(B, T, H, dk, dv, dt))
+    return KDA_ERR_WORKSPACE;
+  int devid = 0;
+  if (cudaGetDevice(&devid) != cudaSuccess) return KDA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_pipe_mu);
+  HostPipe* hp = host_pipe(devid);
+  if (!hp) return KDA_ERR_CUDA;
+  // The copy streams start after the work already on `stream` (which may
+  // still read the device buffers), and `stream` ends after the last copy out.
+  if (cudaEventRecord(hp->start, s) != cudaSuccess || cudaStreamWaitEvent(hp->in, hp->start, 0) != cudaSuccess ||
+      cudaStreamWaitEvent(hp->out, hp->start, 0) != cudaSuccess)
     return KDA_ERR_CUDA;
-  if (host->final_state && dev->final_state && states > 0 &&
-      cudaMemcpyAsync(host->final_state, dev->final_state, states, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+  if (dev->init_state && cudaMemcpyAsync(const_cast<float*>(dev->init_state), host->init_state, (size_t)B * state1,
+                                         cudaMemcpyHostToDevice, hp->in) != cudaSuccess)
+    return KDA_ERR_CUDA;
+  for (int i = 0; i < np; ++i) {
+    const Piece& p = pc[i];
+    if (!copy_tokens(p, hp->in, true) || cudaEventRecord(hp->ev_in[i], hp->in) != cudaSuccess ||
+        cudaStreamWaitEvent(s, hp->ev_in[i], 0) != cudaSuccess)
+      return KDA_ERR_CUDA;
+    const int Bp = p.b1 - p.b0;
+    const int64_t Tp = p.t1 - p.t0, first = (int64_t)p.b0 * T + p.t0;
+    // A token slice after the first continues from the state the previous
+    // slice left in final_state (read and overwritten in place).
+    const float* init = B == 1 ? (i == 0 ? dev->init_state : dev->final_state)
+                               : (dev->init_state ? dev->init_state + (size_t)p.b0 * state1 / 4 : nullptr);
+    float* fin = dev->final_state ? dev->final_state + (size_t)p.b0 * state1 / 4 : nullptr;
+    st = fwd_impl(static_cast<const char*>(dev->q) + first * wq, static_cast<const char*>(dev->k) + first * wq,
+                  static_cast<const char*>(dev->v) + first * wv, dev->log_alpha + first * H * dk,
+                  dev->beta + first * H, init, static_cast<char*>(dev->out) + first * wv, fin, Bp, Tp, H, dk, dv,
+                  nullptr, stream, dt, workspace, workspace_bytes, nullptr, kWaitNs, 0, kda::ModeArgs(), i == 0);
+    if (st != KDA_OK) return st;
+    if (cudaEventRecord(hp->ev_comp[i], s) != cudaSuccess || cudaStreamWaitEvent(hp->out, hp->ev_comp[i], 0) != cudaSuccess ||
+        !copy_tokens(p, hp->out, false))
+      return KDA_ERR_CUDA;
+  }
+  if (host->final_state && dev->final_state &&
+      cudaMemcpyAsync(host->final_state, dev->final_state, (size_t)B * state1, cudaMemcpyDeviceToHost, hp->out) !=
+          cudaSuccess)
+    return KDA_ERR_CUDA;
+  if (cudaEventRecord(hp->done, hp->out) != cudaSuccess || cudaStreamWaitEvent(s, hp->done, 0) != cudaSuccess)
     return KDA_ERR_CUDA;
   return KDA_OK;
 }
@@ -253,7 +398,7 @@ kda_status_t kda_fwd_gated(const void* q, const void* k, const void* v, const vo
   // The decay logits travel in the log-decay slot; validation checks them
   // as one more token tensor.
   return fwd_impl(q, k, v, static_cast<const float*>(z), beta, init_state, out, final_state, B, T, H, dk, dv,
-                  cu_seqlens, stream, dt, workspace, workspace_bytes, nullptr, 2000000000ull, 0, ma);
+                  cu_seqlens, stream, dt, workspace, workspace_bytes, nullptr, kWaitNs, 0, ma);
 }
 
 // ---- interval checkpoints (prefix-cache states) ----
@@ -289,7 +434,7 @@ kda_status_t kda_fwd_checkpoints(const void* q, const void* k, const void* v, co
     ma.ckpt_base = base;
   }
   return fwd_impl(q, k, v, log_alpha, beta, init_state, out, final_state, B, T, H, dk, dv, cu_seqlens, stream, dt,
-                  workspace, workspace_bytes, nullptr, 2000000000ull, 0, ma);
+                  workspace, workspace_bytes, nullptr, kWaitNs, 0, ma);
 }
 
 // ---- segment pieces, composition, correction (context parallelism) ----
@@ -310,7 +455,7 @@ kda_status_t kda_segment_fwd(const void* q, const void* k, const void* v, const 
   ma.qhat32 = qhat;
   ma.trans = transition;
   return fwd_impl(q, k, v, log_alpha, beta, nullptr, nullptr, state_zero, B, T, H, dk, dv, cu_seqlens, stream, dt,
-                  workspace, workspace_bytes, nullptr, 2000000000ull, 0, ma);
+                  workspace, workspace_bytes, nullptr, kWaitNs, 0, ma);
 }
 
 kda_status_t kda_state_compose(const float* transition, const float* state_zero, const float* init_state,
@@ -429,7 +574,7 @@ kda_status_t kda_fwd_cp(const void* q, const void* k, const void* v, const float
     ma.seg_per_seq = n_seg;
     ma.trans = tr;
     kda::FwdArgs a{q, k, v, log_alpha, beta, init_state, nullptr, s0, seg_cu, P, tokens, H, dk, dv, status, nullptr};
-    e = tc ? kda::launch_fwd_tc_impl(a, s, 2000000000ull, 0, order, ma) : kda::launch_fwd_simt(a, bf16, s, ma);
+    e = tc ? kda::launch_fwd_tc_impl(a, s, kWaitNs, 0, order, ma) : kda::launch_fwd_simt(a, bf16, s, ma);
     if (e != cudaSuccess) return KDA_ERR_CUDA;
   }
   // Every segment's incoming state: S_in(0) = init, S_in(1) = the first
@@ -439,7 +584,7 @@ kda_status_t kda_fwd_cp(const void* q, const void* k, const void* v, const float
   // Pass 2: the ordinary forward over all segments from their incoming states.
   kda::FwdArgs a2{q, k, v, log_alpha, beta, s_in, out, final_state ? fin_seg : nullptr, seg_cu, P, tokens, H, dk, dv,
                   status, nullptr};
-  e = tc ? kda::launch_fwd_tc_impl(a2, s, 2000000000ull, 0, order, kda::ModeArgs())
+  e = tc ? kda::launch_fwd_tc_impl(a2, s, kWaitNs, 0, order, kda::ModeArgs())
          : kda::launch_fwd_simt(a2, bf16, s);
   if (e != cudaSuccess) return KDA_ERR_CUDA;
   // The final state of each sequence is the one after its last segment.

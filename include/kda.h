@@ -178,14 +178,27 @@ typedef struct kda_fwd_tensors {
 } kda_fwd_tensors_t;
 
 /*
- * kda_fwd on host buffers: enqueues on `stream` the host-to-device copies of
- * every input in `host` (q, k, v, log_alpha, beta, and init_state /
- * cu_seqlens when set) into the caller's device buffers `dev`, the forward
- * on `dev`, and the device-to-host copies of out (and final_state when both
- * `host` and `dev` set it).  One cudaMemcpyAsync per tensor; page-locked host
- * memory makes the copies asynchronous.  Sizes and the other arguments are
- * those of kda_fwd; `host` and `dev` must set the same optional tensors.
- * Returns at once; synchronise `stream` before reading the host outputs.
+ * kda_fwd on host buffers: enqueues the host-to-device copies of every input
+ * in `host` (q, k, v, log_alpha, beta, and init_state / cu_seqlens when set)
+ * into the caller's device buffers `dev`, the forward on `dev`, and the
+ * device-to-host copies of out (and final_state when both `host` and `dev`
+ * set it).  Sizes and the other arguments are those of kda_fwd; `host` and
+ * `dev` must set the same optional tensors.  Host buffers should be
+ * page-locked (the copies are then asynchronous and overlap).
+ *
+ * Batched calls (no cu_seqlens) are split into up to 8 pieces — groups of
+ * whole sequences when B > 1, else token slices of the one sequence starting
+ * on 64-token chunk boundaries, carried through dev->final_state (which must
+ * then be set; without it the call runs in one piece) — and the pieces'
+ * copies in, forwards and copies out are overlapped: copies in on one
+ * internal stream, forwards on `stream`, copies out on another internal
+ * stream, ordered by events.  The results are the bits of one kda_fwd call.
+ * Packed batches run in one piece on `stream`.  The internal streams and
+ * events are made on the first pipelined call on a device and kept; calls
+ * from several host threads are serialised while they enqueue.  `stream`
+ * waits for everything the call enqueued: the call returns at once, and
+ * synchronising `stream` makes the host outputs readable.  A failure while
+ * enqueueing returns KDA_ERR_CUDA (work already enqueued still runs).
  * This is the end-to-end path a serving process without its own device
  * staging logic would call.
  */

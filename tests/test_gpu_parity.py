@@ -291,17 +291,30 @@ def test_fp16_range_overflow_is_reported(what):
     assert kda.kda_workspace_status(ws) == kda.KDA_OK
 
 
-@pytest.mark.parametrize("packed", [False, True])
-def test_host_buffer_entry_point_matches_device_call(packed):
+@pytest.mark.parametrize("case", ["batched_b2", "batched_b11", "one_sequence_sliced", "one_sequence_short",
+                                  "packed"])
+def test_host_buffer_entry_point_matches_device_call(case):
     """kda_fwd_host (host buffers, copies enqueued by the library) returns the
-    bits kda_fwd returns on device buffers."""
-    if packed:
+    bits kda_fwd returns on device buffers: in one piece (packed batches), in
+    pieces of whole sequences overlapping copies and compute (B > 1: 2 and 8
+    pieces), and in token slices of one sequence carried through the final
+    state (B = 1, 1000 tokens: 8 slices starting on chunk boundaries, the last
+    ragged), called twice on the same buffers."""
+    if case == "packed":
         inp = synth.make_prefill(synth.VARLEN, DEV, H=3, lengths=[70, 0, 129])
-    else:
+    elif case == "batched_b2":
         inp = synth.make_prefill(synth.MID, DEV, T=200, B=2, H=3)
+    elif case == "batched_b11":
+        inp = synth.make_prefill(synth.MID, DEV, T=130, B=11, H=2)
+    elif case == "one_sequence_sliced":
+        inp = synth.make_prefill(synth.MID, DEV, T=1000, B=1, H=3)
+    else:
+        inp = synth.make_prefill(synth.PRETRAIN, DEV, T=100, B=1, H=2)  # no initial state, 2 slices
     ref_out, ref_fin = run_gpu(inp)
     host = {n: (None if t is None else t.cpu().pin_memory()) for n, t in inp.items()}
-    out_h, fin_h, _ = kda.kda_fwd_host(host["q"], host["k"], host["v"], host["g"], host["beta"],
-                                       host["init_state"], host["cu_seqlens"], device=DEV)
-    torch.cuda.synchronize()
-    assert torch.equal(out_h, ref_out.cpu()) and torch.equal(fin_h, ref_fin.cpu())
+    bufs = None
+    for _ in range(2):
+        out_h, fin_h, bufs = kda.kda_fwd_host(host["q"], host["k"], host["v"], host["g"], host["beta"],
+                                              host["init_state"], host["cu_seqlens"], device=DEV, dev_buffers=bufs)
+        torch.cuda.synchronize()
+        assert torch.equal(out_h, ref_out.cpu()) and torch.equal(fin_h, ref_fin.cpu())
