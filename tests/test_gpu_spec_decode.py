@@ -60,13 +60,34 @@ def _spec_case(dtype, dk, dv, B, H, Wp, W, seed, prologue, steps):
 
 @pytest.mark.parametrize("dtype,dk,dv", [(torch.bfloat16, 128, 128), (torch.float32, 32, 64),
                                          (torch.bfloat16, 64, 16)])
-@pytest.mark.parametrize("W", [1, 4])
+@pytest.mark.parametrize("W", [1, 4, 8])
 @pytest.mark.parametrize("prologue", [False, True])
 def test_spec_decode_matches_oracle(dtype, dk, dv, W, prologue):
     state, ref, outs = _spec_case(dtype, dk, dv, B=5, H=3, Wp=W, W=W, seed=61 + W, prologue=prologue, steps=5)
     for i, (o, r) in enumerate(outs):
         assert_close(o, r, dtype, f"spec out step {i}")
     assert_close(state, ref, dtype, "spec committed state")
+
+
+@pytest.mark.parametrize("dtype,dk,dv", [(torch.bfloat16, 128, 128), (torch.float32, 16, 16),
+                                         (torch.bfloat16, 128, 16)])
+def test_spec_decode_longest_chunk(dtype, dk, dv):
+    """Every draft of an 8-token window accepted, then a new 8-token window:
+    chunks of the maximum 16 tokens (both 8-token halves of the pair sums)."""
+    spec = synth.DecodeSpec("sp16", 3, 2, dk, dv, dtype, 83, 2)
+    state = synth.make_decode_state(spec, DEV)
+    ref = state.double().cpu().numpy().copy()
+    prev = synth.make_spec_window(spec, 0, 8, DEV)
+    out0 = kda.kda_decode_spec(None, None, prev, state)
+    o0 = oracle.spec_decode(None, None, prev, ref)
+    na = torch.full((3,), 8, dtype=torch.int32, device=DEV)
+    cur = synth.make_spec_window(spec, 1, 8, DEV)
+    out1 = kda.kda_decode_spec(prev, na, cur, state)
+    o1 = oracle.spec_decode(prev, na.cpu(), cur, ref)
+    torch.cuda.synchronize()
+    assert_close(out0, o0, dtype, "first window")
+    assert_close(out1, o1, dtype, "16-token chunk")
+    assert_close(state, ref, dtype, "state after the 16-token chunk")
 
 
 def test_spec_decode_replay_only_and_full_accept():
