@@ -410,7 +410,9 @@ KDA_API kda_status_t kda_decode_step_gated(const void *q, const void *k, const v
  * The rejected drafts of the previous window are never applied; the new
  * drafts' states stay on chip.  The replayed and new tokens are taken as one
  * chunk (the chunkwise form of the recurrence, fp32), so the state is read
- * once and written once whatever the window.  Wp + W <= KDA_SPEC_MAX_TOKENS
+ * once and written once whatever the window (all Wp + W rows of both windows
+ * are read, the rejected drafts' too, so that no load waits for n_accepted;
+ * every pointer must be 16-byte aligned).  Wp + W <= KDA_SPEC_MAX_TOKENS
  * (else KDA_ERR_UNSUPPORTED).  W = 0 only replays (and keeps the state after
  * the accepted drafts).  No workspace.
  */
