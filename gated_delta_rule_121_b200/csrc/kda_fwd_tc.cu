@@ -891,6 +891,11 @@ __device__ __forceinline__ void front_group(const Ctx& x, const float* __restric
       store_pa(sm, b2, 32 * lq + lane, chh, s_beta, r0);
       tc_fence_before();
     }
+    // The next chunk's decay rows are requested after this chunk's last TMEM
+    // read and tile stores, so that their latency overlaps the barrier below
+    // (only named barriers follow until they are used).  The gated mode maps
+    // its logits to decays as they arrive, so it requests them at the end.
+    if constexpr (MODE != MODE_GATED) load_g(c + 1, gv, bv);
     fence_proxy_async_smem();  // P is read by the D2 UMMA
     if (dmp) {
       named_sync(GRP_FRONT, FRONT_T);
@@ -899,7 +904,7 @@ __device__ __forceinline__ void front_group(const Ctx& x, const float* __restric
     named_sync(GRP_FRONT, FRONT_T);  // the front's TMEM reads are done before the next G1
     mbar_arrive(&x.bars[B_FR0 + b2]);
     if (f == 0) tmark(x, c, 26);
-    load_g(c + 1, gv, bv);
+    if constexpr (MODE == MODE_GATED) load_g(c + 1, gv, bv);
   }
 }
 
