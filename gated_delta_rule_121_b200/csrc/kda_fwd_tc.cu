@@ -673,13 +673,13 @@ __device__ __forceinline__ void front_group(const Ctx& x, const float* __restric
     for (int m = 0; m < 4; ++m) {
       const int r = 4 * rg + m;
       if constexpr (MODE == MODE_GATED) {
-        // bf16 decay logits mapped to log-decays at once; rows past the end
-        // get -inf, whose gate is exactly 0
+        // the raw bf16 decay logits (their bits in the first half of the
+        // row); the prefix maps them to log-decays.  Rows past the end get
+        // -inf, whose gate is exactly 0.
         const uint4 u = r < valid ? __ldg(reinterpret_cast<const uint4*>(
                                         reinterpret_cast<const __nv_bfloat16*>(g) + ((tok0 + r) * H + x.h) * D + ch0))
                                   : make_uint4(0xFF80FF80u, 0xFF80FF80u, 0xFF80FF80u, 0xFF80FF80u);
-        const float* gc = reinterpret_cast<const float*>(x.sm + SM_MISC + MS_GATE);
-        gv[m] = gate_8(u, gc[0], gc[1]);
+        gv[m].a = make_float4(__uint_as_float(u.x), __uint_as_float(u.y), __uint_as_float(u.z), __uint_as_float(u.w));
       } else {
         gv[m] = r < valid ? ldg8(g + ((tok0 + r) * H + x.h) * D + ch0, g32) : f8(0.f);
       }
@@ -717,6 +717,14 @@ __device__ __forceinline__ void front_group(const Ctx& x, const float* __restric
     // groups and the chunk total G_C.
     F8 acc = f8(0.f);
     const F8 l2e = f8(LOG2E);
+    if constexpr (MODE == MODE_GATED) {
+      const float* gc = reinterpret_cast<const float*>(x.sm + SM_MISC + MS_GATE);
+      const float gz = gc[0], gmin = gc[1];
+#pragma unroll
+      for (int m = 0; m < 4; ++m)
+        gv[m] = gate_8(make_uint4(__float_as_uint(gv[m].a.x), __float_as_uint(gv[m].a.y),
+                                  __float_as_uint(gv[m].a.z), __float_as_uint(gv[m].a.w)), gz, gmin);
+    }
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
       gv[m] = mul8(gv[m], l2e);
@@ -893,9 +901,9 @@ __device__ __forceinline__ void front_group(const Ctx& x, const float* __restric
     }
     // The next chunk's decay rows are requested after this chunk's last TMEM
     // read and tile stores, so that their latency overlaps the barrier below
-    // (only named barriers follow until they are used).  The gated mode maps
-    // its logits to decays as they arrive, so it requests them at the end.
-    if constexpr (MODE != MODE_GATED) load_g(c + 1, gv, bv);
+    // (only named barriers follow until they are used; a wait on an mbarrier
+    // or a TMEM load with these loads in flight would stall until they land).
+    load_g(c + 1, gv, bv);
     fence_proxy_async_smem();  // P is read by the D2 UMMA
     if (dmp) {
       named_sync(GRP_FRONT, FRONT_T);
@@ -904,7 +912,6 @@ __device__ __forceinline__ void front_group(const Ctx& x, const float* __restric
     named_sync(GRP_FRONT, FRONT_T);  // the front's TMEM reads are done before the next G1
     mbar_arrive(&x.bars[B_FR0 + b2]);
     if (f == 0) tmark(x, c, 26);
-    if constexpr (MODE == MODE_GATED) load_g(c + 1, gv, bv);
   }
 }
 
