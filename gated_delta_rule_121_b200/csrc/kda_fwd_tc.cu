@@ -903,7 +903,10 @@ __device__ __forceinline__ void front_group(const Ctx& x, const float* __restric
     // read and tile stores, so that their latency overlaps the barrier below
     // (only named barriers follow until they are used; a wait on an mbarrier
     // or a TMEM load with these loads in flight would stall until they land).
-    load_g(c + 1, gv, bv);
+    // Measured faster for the plain and gated modes only (the checkpoint and
+    // segment builds lost 8-9 %), which request them at the end instead.
+    constexpr bool early_g = MODE == MODE_PLAIN || MODE == MODE_GATED;
+    if constexpr (early_g) load_g(c + 1, gv, bv);
     fence_proxy_async_smem();  // P is read by the D2 UMMA
     if (dmp) {
       named_sync(GRP_FRONT, FRONT_T);
@@ -912,6 +915,7 @@ __device__ __forceinline__ void front_group(const Ctx& x, const float* __restric
     named_sync(GRP_FRONT, FRONT_T);  // the front's TMEM reads are done before the next G1
     mbar_arrive(&x.bars[B_FR0 + b2]);
     if (f == 0) tmark(x, c, 26);
+    if constexpr (!early_g) load_g(c + 1, gv, bv);
   }
 }
 
