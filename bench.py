@@ -249,7 +249,7 @@ def job_throughput(d, units, seconds):
 def workload_spec(name):
     import synth
     return {"prefill64k": synth.PRETRAIN, "mid": synth.MID, "varlen": synth.VARLEN,
-            "stress": synth.STRESS, "tp4": synth.TP4}[name]
+            "stress": synth.STRESS, "tp4": synth.TP4, "prefill64k_model_range": synth.PRETRAIN_MODEL_RANGE}[name]
 
 
 # ----------------------------------------------------------------- oracle arm
@@ -311,7 +311,8 @@ TRAFFIC_PROFILES = {
     "kda_decode_kernel": ("kda_decode_b64_h96_traffic.txt", "kda_decode.cu"),
     "kda_spec_kernel": ("kda_spec_b64_h96_w4_traffic.txt", "kda_spec.cu"),
 }
-FLUSH = {"mid": True, "stress": True, "prefill64k": False, "varlen": False, "tp4": False}
+FLUSH = {"mid": True, "stress": True, "prefill64k": False, "varlen": False, "tp4": False,
+         "prefill64k_model_range": False}
 
 
 def bench_prefill(name, d, dev, stream, peaks, kda, synth, steps, warmup, with_traffic=False, variant=None):
@@ -446,6 +447,7 @@ def run_native(args, d):
         for key, name, steps, variant in (("mid", "mid", 50, None), ("mid_cp", "mid", 50, "cp"),
                                           ("tp4", "tp4", 10, None), ("tp4_cp", "tp4", 20, "cp"),
                                           ("varlen", "varlen", 8, None), ("stress", "stress", 50, None),
+                                          ("prefill64k_model_range", "prefill64k_model_range", 5, None),
                                           ("prefill64k_ckpt512", "prefill64k", 10, "ckpt512"),
                                           ("prefill64k_gated", "prefill64k", 10, "gated")):
             if name == args.workload and variant is None:
@@ -702,7 +704,8 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
-    ap.add_argument("--workload", choices=["prefill64k", "mid", "varlen", "stress", "tp4"], default="prefill64k")
+    ap.add_argument("--workload", choices=["prefill64k", "mid", "varlen", "stress", "tp4", "prefill64k_model_range"],
+                    default="prefill64k")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -74,7 +74,12 @@ DECODE = DecodeSpec("decode_bf16_B512_H96_d128", 512, 96, 128, 128, torch.bfloat
 # (24-way head split), the case where the chains are far fewer than the SMs.
 TP4 = PrefillSpec("tp4_bf16_B1_H4_T65536_d128", 1, 65536, 4, 128, 128, torch.bfloat16, 6)
 
-PREFILL_SPECS = {s.name: s for s in (TINY, MID, PRETRAIN, VARLEN, STRESS, TP4)}
+# The 64K prefill with decays in the model's whole range (g = -5 sigmoid(z)):
+# every chunk takes the bounded-decay (general) path.
+PRETRAIN_MODEL_RANGE = PrefillSpec("prefill_bf16_B1_H96_T65536_d128_gmin5", 1, 65536, 96, 128, 128, torch.bfloat16, 7,
+                                   g_scale=5.0)
+
+PREFILL_SPECS = {s.name: s for s in (TINY, MID, PRETRAIN, VARLEN, STRESS, TP4, PRETRAIN_MODEL_RANGE)}
 
 
 def varlen_lengths(total: int, lo: int, hi: int, seed: int) -> list[int]:
