@@ -468,14 +468,15 @@ def kda_decode_spec(prev, n_accepted, cur, state, A_log=None, g_min=G_MIN, out=N
 
 
 def kda_fwd_host(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None, device="cuda", stream=None,
-                 dev_buffers=None):
+                 dev_buffers=None, output_final_state=True):
     """kda_fwd on host tensors through the C entry point kda_fwd_host: one call
     enqueues the host-to-device copies of the inputs (pinned memory makes them
     asynchronous), the forward, and the copies of ``out`` and the final state
     back.  ``dev_buffers`` (a dict returned by a previous call) holds the
     device buffers and the pinned host outputs for repeated calls.  Returns
-    (out_host, final_host, dev_buffers); synchronise the stream before reading
-    the host outputs."""
+    (out_host, final_host, dev_buffers) (final_host None without
+    ``output_final_state``); synchronise the stream before reading the host
+    outputs."""
     s = stream if stream is not None else torch.cuda.current_stream(device)
     B, T, H, dk, dv, N = _shapes(q, v, cu_seqlens)
     host_in = dict(q=q, k=k, v=v, log_alpha=log_alpha, beta=beta, init_state=init_state, cu_seqlens=cu_seqlens)
@@ -492,12 +493,14 @@ def kda_fwd_host(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None, dev
         dev_buffers["ws"] = alloc_workspace(N, B * T, H, dk, dv, q.dtype, device)
         dev_buffers["out_h"] = torch.empty((B, T, H, dv), dtype=q.dtype, pin_memory=True)
         dev_buffers["fin_h"] = torch.empty((N, H, dk, dv), dtype=torch.float32, pin_memory=True)
-    host = dict(host_in, out=dev_buffers["out_h"], final_state=dev_buffers["fin_h"])
+    fin_h = dev_buffers["fin_h"] if output_final_state else None
+    host = dict(host_in, out=dev_buffers["out_h"], final_state=fin_h)
+    dev = dict(dev_buffers["dev"]) if output_final_state else dict(dev_buffers["dev"], final_state=None)
     for n, t in host_in.items():
         if t is not None and (t.device.type != "cpu" or not t.is_contiguous()):
             raise ValueError(f"{n}: expected a contiguous host tensor")
     ws = dev_buffers["ws"]
-    code = lib().kda_fwd_host(ctypes.byref(_tensors(host)), ctypes.byref(_tensors(dev_buffers["dev"])), N, T, H,
+    code = lib().kda_fwd_host(ctypes.byref(_tensors(host)), ctypes.byref(_tensors(dev)), N, T, H,
                               dk, dv, ctypes.c_void_p(s.cuda_stream), _DT[q.dtype], _ptr(ws), ws.numel())
     _check(code, "kda_fwd_host")
-    return dev_buffers["out_h"], dev_buffers["fin_h"], dev_buffers
+    return dev_buffers["out_h"], fin_h, dev_buffers

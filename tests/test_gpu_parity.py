@@ -292,14 +292,16 @@ def test_fp16_range_overflow_is_reported(what):
 
 
 @pytest.mark.parametrize("case", ["batched_b2", "batched_b11", "one_sequence_sliced", "one_sequence_short",
-                                  "packed"])
+                                  "packed", "batched_unaligned_beta", "one_sequence_no_final_state"])
 def test_host_buffer_entry_point_matches_device_call(case):
     """kda_fwd_host (host buffers, copies enqueued by the library) returns the
     bits kda_fwd returns on device buffers: in one piece (packed batches), in
     pieces of whole sequences overlapping copies and compute (B > 1: 2 and 8
     pieces), and in token slices of one sequence carried through the final
     state (B = 1, 1000 tokens: 8 slices starting on chunk boundaries, the last
-    ragged), called twice on the same buffers."""
+    ragged), called twice on the same buffers; in one piece where a piece's
+    beta rows would not start on 16 bytes (T H = 303) and for one sequence
+    without a final-state buffer."""
     if case == "packed":
         inp = synth.make_prefill(synth.VARLEN, DEV, H=3, lengths=[70, 0, 129])
     elif case == "batched_b2":
@@ -308,13 +310,20 @@ def test_host_buffer_entry_point_matches_device_call(case):
         inp = synth.make_prefill(synth.MID, DEV, T=130, B=11, H=2)
     elif case == "one_sequence_sliced":
         inp = synth.make_prefill(synth.MID, DEV, T=1000, B=1, H=3)
+    elif case == "batched_unaligned_beta":
+        inp = synth.make_prefill(synth.MID, DEV, T=101, B=3, H=3)
+    elif case == "one_sequence_no_final_state":
+        inp = synth.make_prefill(synth.MID, DEV, T=700, B=1, H=2)
     else:
         inp = synth.make_prefill(synth.PRETRAIN, DEV, T=100, B=1, H=2)  # no initial state, 2 slices
     ref_out, ref_fin = run_gpu(inp)
     host = {n: (None if t is None else t.cpu().pin_memory()) for n, t in inp.items()}
     bufs = None
+    want_final = case != "one_sequence_no_final_state"
     for _ in range(2):
         out_h, fin_h, bufs = kda.kda_fwd_host(host["q"], host["k"], host["v"], host["g"], host["beta"],
-                                              host["init_state"], host["cu_seqlens"], device=DEV, dev_buffers=bufs)
+                                              host["init_state"], host["cu_seqlens"], device=DEV, dev_buffers=bufs,
+                                              output_final_state=want_final)
         torch.cuda.synchronize()
-        assert torch.equal(out_h, ref_out.cpu()) and torch.equal(fin_h, ref_fin.cpu())
+        assert torch.equal(out_h, ref_out.cpu())
+        assert (fin_h is None) if not want_final else torch.equal(fin_h, ref_fin.cpu())
