@@ -119,6 +119,10 @@ __device__ __forceinline__ void store_pieces(const uint4 (&r)[Pieces<T, D, NT>::
   }
 }
 
+__device__ __forceinline__ float4 add4(float4 a, float4 b) {
+  return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
+}
+
 struct SpecTok {  // where one token's inputs live
   const void* q;
   const void* k;
@@ -190,10 +194,14 @@ __global__ void __launch_bounds__(SpecShape<DK, DV>::NT, 2)
     auto same = [](float x) { return x; };
     store_pieces<IO, DK, NT>(pk, s_k, NW, pos, same);
     store_pieces<IO, DK, NT>(pq, s_q, NW, pos, same);
-    if constexpr (GATED)
+    // the per-token log-decays g (s_G) and decays alpha = e^g (s_al)
+    if constexpr (GATED) {
       store_pieces<GT, DK, NT>(pg, s_G, NW, pos, [&](float z) { return gate_log_decay(z, Ah, g_min); });
-    else
+      store_pieces<GT, DK, NT>(pg, s_al, NW, pos, [&](float z) { return __expf(gate_log_decay(z, Ah, g_min)); });
+    } else {
       store_pieces<GT, DK, NT>(pg, s_G, NW, pos, same);
+      store_pieces<GT, DK, NT>(pg, s_al, NW, pos, [](float x) { return __expf(x); });
+    }
     store_pieces<IO, DV, NT>(pv, s_v, NW, pos, same);
     if (tid < NW && pos(tid) >= 0) s_b[pos(tid)] = bt;
   }
@@ -222,27 +230,22 @@ __global__ void __launch_bounds__(SpecShape<DK, DV>::NT, 2)
     }
     __syncthreads();
   }
-  // ---- cumulative log-decay over the chunk and the per-token decays
-  // alpha_t = e^{g_t}, one thread per key channel
-  for (int i = tid; i < DK; i += NT) {
-    float acc = 0.f;
-    for (int t = 0; t < n; ++t) {
-      const float g = s_G[t * DK + i];
-      acc += g;
-      s_G[t * DK + i] = acc;
-      s_al[t * DK + i] = __expf(g);
-    }
-  }
-  __syncthreads();
   // ---- per-token operands, four channels per work item: e^{G_t} k_t,
   // e^{G_t} q_t, k_t e^{G_c - G_t} (t <= c), zero past the chunk (up to n4),
-  // and e^{G_c}.  Then (no barrier: other arrays) the pair sums.
+  // and e^{G_c}; each item sums its own cumulative log-decays G_t and G_c
+  // over the tokens (at most 16).  Then (no barrier: other arrays) the pair
+  // sums.
   for (int w = tid; w < n4 * (DK / 4); w += NT) {
     const int t = w / (DK / 4), i0 = 4 * (w % (DK / 4));
     float4 ek = make_float4(0.f, 0.f, 0.f, 0.f), eq = ek, kc = ek;
     if (t < n) {
-      const float4 G = *reinterpret_cast<const float4*>(s_G + t * DK + i0);
-      const float4 Gc = *reinterpret_cast<const float4*>(s_G + c * DK + i0);
+      float4 G = make_float4(0.f, 0.f, 0.f, 0.f), Gc = G, acc = G;
+      const int last = t > c ? t : c;
+      for (int u = 0; u <= last; ++u) {
+        acc = add4(acc, *reinterpret_cast<const float4*>(s_G + u * DK + i0));
+        if (u == t) G = acc;
+        if (u == c) Gc = acc;
+      }
       const float4 kk = *reinterpret_cast<const float4*>(s_k + t * DK + i0);
       const float4 qq = *reinterpret_cast<const float4*>(s_q + t * DK + i0);
       const float4 e = make_float4(__expf(G.x), __expf(G.y), __expf(G.z), __expf(G.w));
