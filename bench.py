@@ -12,8 +12,14 @@ bf16 q/k/v/o with fp32 log-decay, beta and state (the 64K pretraining
 context with the model's 96 heads).  One step = one kda_fwd over that batch.
 The same run also times, each under its own key: the B=512, H=96
 single-token decode ("decode": one kda_decode_step per step, state updated
-in place) and the other prefill workloads ("workloads": the mid batch
-B=2 H=16 T=4096, the packed 1M-token batch, and the model-range decay case).
+in place; "decode_gated" on the raw prologue inputs), speculative
+verification ("decode_spec": windows of 4 with replay, and the step time for
+windows of 1, 2, 4 and 8), the same prefill end to end from pinned host
+buffers through kda_fwd_host ("e2e"), and the other prefill workloads
+("workloads": the mid batch B=2 H=16 T=4096 plain and through kda_fwd_cp,
+one tensor-parallel rank's 4 heads of the 64K prefill plain and through
+kda_fwd_cp, the packed 1M-token batch, the model-range decay cases, the 64K
+prefill with 512-token checkpoints and with the fused prologue).
 Inputs are synthetic (seeded) and resident in HBM before the timed region;
 workloads smaller than the 126 MB L2 (or close to it) get an L2 flush before
 every timed launch, the others are far larger than L2.
@@ -709,7 +715,8 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-workloads", action="store_true", help="skip the mid, varlen and stress objects")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the other workload objects (mid, tp4, varlen, stress, model range, checkpoints, gated)")
     ap.add_argument("--capture", choices=sorted(CAPTURES), default=None,
                     help="run --steps launches of a small case (for ncu), nothing else")
     ap.add_argument("--phases", action="store_true",
