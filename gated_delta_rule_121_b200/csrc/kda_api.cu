@@ -117,7 +117,7 @@ kda_status_t kda_fwd(const void* q, const void* k, const void* v, const float* l
 
 namespace {
 
-constexpr int kHostPieces = 8;  // pieces of a pipelined kda_fwd_host call, at most
+constexpr int kHostPieces = 16;  // pieces of a pipelined kda_fwd_host call, at most
 
 // Streams and events of the pipelined host path, one set per device, made on
 // first use and kept for the life of the process.

@@ -186,7 +186,7 @@ typedef struct kda_fwd_tensors {
  * `dev` must set the same optional tensors.  Host buffers should be
  * page-locked (the copies are then asynchronous and overlap).
  *
- * Batched calls (no cu_seqlens) are split into up to 8 pieces — groups of
+ * Batched calls (no cu_seqlens) are split into up to 16 pieces — groups of
  * whole sequences when B > 1, else token slices of the one sequence starting
  * on 64-token chunk boundaries, carried through dev->final_state (which must
  * then be set; without it the call runs in one piece) — and the pieces'

@@ -296,9 +296,9 @@ def test_fp16_range_overflow_is_reported(what):
 def test_host_buffer_entry_point_matches_device_call(case):
     """kda_fwd_host (host buffers, copies enqueued by the library) returns the
     bits kda_fwd returns on device buffers: in one piece (packed batches), in
-    pieces of whole sequences overlapping copies and compute (B > 1: 2 and 8
+    pieces of whole sequences overlapping copies and compute (B > 1: 2 and 11
     pieces), and in token slices of one sequence carried through the final
-    state (B = 1, 1000 tokens: 8 slices starting on chunk boundaries, the last
+    state (B = 1, 1000 tokens: 16 slices starting on chunk boundaries, the last
     ragged), called twice on the same buffers; in one piece where a piece's
     beta rows would not start on 16 bytes (T H = 303) and for one sequence
     without a final-state buffer."""
