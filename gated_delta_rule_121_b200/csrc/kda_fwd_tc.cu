@@ -331,6 +331,13 @@ __device__ __forceinline__ void row_factors(const uint8_t* sm, int rg, float (&r
   rk[0] = b.x; rk[1] = b.y; rk[2] = b.z; rk[3] = b.w;
 }
 
+// Which group converts a chunk's V tile to fp16 in place: the back group,
+// while it waits for the front's tiles (measured faster for the plain,
+// checkpoint and segment builds), or the front group in its scaling pass
+// (the fused-prologue build, whose front is the slower group).
+template <int MODE>
+constexpr bool V_IN_FRONT = MODE == MODE_GATED;
+
 // Phase timestamp (elected thread only) for the timing dump.
 __device__ __forceinline__ void tmark(const Ctx& x, int c, int ev) {
   if (x.tdbg && c < TIME_CHUNKS) x.tdbg[c * 32 + ev] = clock64() - x.tstart;
@@ -793,7 +800,7 @@ __device__ __forceinline__ void front_group(const Ctx& x, const float* __restric
           const uint32_t o = sw128_off(r, cc);
           *reinterpret_cast<uint4*>(qb + o) = make_uint4(0u, 0u, 0u, 0u);
           *reinterpret_cast<uint4*>(kb + o) = make_uint4(0u, 0u, 0u, 0u);
-          *reinterpret_cast<uint4*>(vb + o) = make_uint4(0u, 0u, 0u, 0u);
+          if constexpr (V_IN_FRONT<MODE>) *reinterpret_cast<uint4*>(vb + o) = make_uint4(0u, 0u, 0u, 0u);
         }
       }
     }
@@ -810,8 +817,9 @@ __device__ __forceinline__ void front_group(const Ctx& x, const float* __restric
     }
 
     // ---- (a2) operand scaling, row by row: E = e^{G_r - ref} (ref = G_C on
-    // fast chunks, 0 otherwise), H = e^{G_C - G_r}.  QE, KE and V (fp16) go
-    // in place; KH goes to KX[b2] once the scan of chunk c-2 has released it.
+    // fast chunks, 0 otherwise), H = e^{G_C - G_r}.  QE and KE (fp16) go in
+    // place (the back group converts V); KH goes to KX[b2] once the scan of
+    // chunk c-2 has released it.
     uint4 kraw[4];  // raw K rows, kept for KH
     {
       F8 gr = f8(0.f);
@@ -823,7 +831,7 @@ __device__ __forceinline__ void front_group(const Ctx& x, const float* __restric
           const uint32_t o = sw128_off(4 * rg + mb + i, cc);
           qr[i] = *reinterpret_cast<const uint4*>(qb + o);
           kraw[mb + i] = *reinterpret_cast<const uint4*>(kb + o);
-          vr[i] = *reinterpret_cast<const uint4*>(vb + o);
+          if constexpr (V_IN_FRONT<MODE>) vr[i] = *reinterpret_cast<const uint4*>(vb + o);
         }
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
@@ -838,11 +846,7 @@ __device__ __forceinline__ void front_group(const Ctx& x, const float* __restric
             st_f16x8(qb + o, mul8(bf16x8_to_f32(qr[i]), fw));
             st_f16x8(kb + o, mul8(bf16x8_to_f32(kraw[m]), fw));
           }
-          if constexpr (MODE == MODE_SEG) {  // a transition run takes every value as zero
-            st_f16x8(vb + o, x.trans ? f8(0.f) : bf16x8_to_f32(vr[i]));
-          } else {
-            st_f16x8(vb + o, bf16x8_to_f32(vr[i]));
-          }
+          if constexpr (V_IN_FRONT<MODE>) st_f16x8(vb + o, bf16x8_to_f32(vr[i]));
         }
       }
     }
@@ -919,6 +923,7 @@ __device__ __forceinline__ void front_group(const Ctx& x, const float* __restric
   }
 }
 
+template <int MODE>
 __device__ __forceinline__ void back_group(const Ctx& x) {
   const int k = threadIdx.x - BACK0;  // 0..127
   const int bw = k >> 5, lane = k & 31;
@@ -935,6 +940,22 @@ __device__ __forceinline__ void back_group(const Ctx& x) {
     const float* s_beta = reinterpret_cast<const float*>(sm + SM_MISC + MS_BETA) + b2 * 64;
 
     if (k == 0) tmark(x, c, 16);
+    // V of chunk c to fp16 in place for G3 (U^T = V^T T'^T) while the front
+    // forms this chunk's tiles: rows past the end of a sequence become zero,
+    // and so does every value of a transition run (segment mode).
+    if constexpr (!V_IN_FRONT<MODE>) {
+      if (!gwait(x, B_FULL0 + b2, (c >> 1) & 1, 25, GRP_BACK)) break;
+      const int valid = chunk_valid(x, c);
+      uint8_t* vbase = sm + b2 * STAGE_BYTES + OFF_V;
+#pragma unroll 4
+      for (int i = 0; i < 8; ++i) {  // 64 rows x 2 channel halves x 8 pieces of 8 channels
+        const int p = k + GRP * i, row = p >> 4;
+        uint8_t* ptr = vbase + ((p >> 3) & 1) * 8192 + sw128_off(row, 8 * (p & 7));
+        const uint4 raw = *reinterpret_cast<const uint4*>(ptr);
+        st_f16x8(ptr, (row < valid && !x.trans) ? bf16x8_to_f32(raw) : f8(0.f));
+      }
+      fence_proxy_async_smem();
+    }
     if (!gwait(x, B_FR0 + b2, (c >> 1) & 1, 21, GRP_BACK)) break;
     if (k == 0) tmark(x, c, 17);
 
@@ -1575,7 +1596,7 @@ __global__ void __launch_bounds__(NTHR, 1)
     front_group<MODE>(x, g, beta, &tm_g, cnt);
     if (tid == (int)FRONT0) { s_cnt[2] = cnt[0]; s_cnt[3] = cnt[1]; }
   } else {
-    back_group(x);
+    back_group<MODE>(x);
   }
 
   // Drain: every UMMA issued by a group's elected thread has completed, and
