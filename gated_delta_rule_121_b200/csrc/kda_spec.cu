@@ -316,21 +316,29 @@ __global__ void __launch_bounds__(SpecShape<DK, DV>::NT, 2)
   }
   __syncthreads();
 
-  // ---- X_t = S0^T ek_t and Y_t = S0^T eq_t, TB tokens at a time (groups of
-  // 4, the last one to three tokens in groups of 2 and 1): each thread's
-  // share over its rows, then the row groups' partial sums added through
-  // shared memory (the token-major arrays are no longer needed).
-  auto xy_group = [&](auto tb, int t0) {
-    constexpr int TB = decltype(tb)::value;
+  // ---- X_t = S0^T ek_t for every token and Y_t = S0^T eq_t for the new
+  // window's tokens (t >= na; the replayed ones have no outputs): a list of
+  // rows, the X rows first, taken eight at a time (two passes of four
+  // accumulators; the last one to seven rows in groups of 4, 2 and 1): each
+  // thread's share over its state rows, then the row groups' partial sums
+  // added through shared memory (the token-major arrays are no longer
+  // needed).
+  const int nrows = 2 * n - na;
+  // row r: its operand (this thread's entries) and where its sums go in s_xy
+  const float* s_eq_na = s_eq + rg * ROWS + (na - n) * DK;  // s_eq_na + r DK: token na + r - n
+  auto row_op = [&](int r) -> const float* { return r < n ? s_ek + rg * ROWS + r * DK : s_eq_na + r * DK; };
+  auto row_dst = [&](int r) { return r < n ? r * 2 * DV : (na + r - n) * 2 * DV + DV; };
+  auto xy_rows = [&](auto tb, int r0) {
+    constexpr int TB = decltype(tb)::value;  // rows of this group
+    constexpr int PB = TB < 4 ? TB : 4;      // rows per pass
 #pragma unroll 1
-    for (int xy = 0; xy < 2; ++xy) {  // X from e^G k, then Y from e^G q (16 accumulators at a time)
-      const float* src = xy ? s_eq : s_ek;
-      float acc[TB][4];
+    for (int pb = 0; pb < TB; pb += PB) {
+      float acc[PB][4];
 #pragma unroll
-      for (int u = 0; u < TB; ++u) acc[u][0] = acc[u][1] = acc[u][2] = acc[u][3] = 0.f;
+      for (int u = 0; u < PB; ++u) acc[u][0] = acc[u][1] = acc[u][2] = acc[u][3] = 0.f;
 #pragma unroll
-      for (int u = 0; u < TB; ++u) {
-        const float* e = src + (t0 + u) * DK + rg * ROWS;  // this token's entries for the thread's rows
+      for (int u = 0; u < PB; ++u) {
+        const float* e = row_op(r0 + pb + u);
         float ev[ROWS];
         if constexpr (ROWS % 4 == 0) {
 #pragma unroll
@@ -349,26 +357,31 @@ __global__ void __launch_bounds__(SpecShape<DK, DV>::NT, 2)
         }
       }
 #pragma unroll
-      for (int u = 0; u < TB; ++u)
-        *reinterpret_cast<float4*>(s_part + ((rg * TB + u) * 2 + xy) * DV + 4 * cq) =
+      for (int u = 0; u < PB; ++u)
+        *reinterpret_cast<float4*>(s_part + (rg * TB + pb + u) * DV + 4 * cq) =
             make_float4(acc[u][0], acc[u][1], acc[u][2], acc[u][3]);
     }
     __syncthreads();
-    for (int e = tid; e < TB * 2 * DV; e += NT) {
+    for (int e = tid; e < TB * DV; e += NT) {
+      const int row = e / DV, col = e % DV;
       float sum = 0.f;
 #pragma unroll 8
-      for (int r = 0; r < RG; ++r) sum += s_part[r * TB * 2 * DV + e];
-      s_xy[t0 * 2 * DV + e] = sum;  // token t0 + e / (2 DV), X or Y column e % (2 DV)
+      for (int r = 0; r < RG; ++r) sum += s_part[(r * TB + row) * DV + col];
+      s_xy[row_dst(r0 + row) + col] = sum;
     }
     __syncthreads();  // the partial sums are read before the next group writes them
   };
-  int t0 = 0;
-  for (; t0 + 4 <= n; t0 += 4) xy_group(std::integral_constant<int, 4>{}, t0);
-  if (n - t0 >= 2) {
-    xy_group(std::integral_constant<int, 2>{}, t0);
-    t0 += 2;
+  int r0 = 0;
+  for (; r0 + 8 <= nrows; r0 += 8) xy_rows(std::integral_constant<int, 8>{}, r0);
+  if (nrows - r0 >= 4) {
+    xy_rows(std::integral_constant<int, 4>{}, r0);
+    r0 += 4;
   }
-  if (t0 < n) xy_group(std::integral_constant<int, 1>{}, t0);
+  if (nrows - r0 >= 2) {
+    xy_rows(std::integral_constant<int, 2>{}, r0);
+    r0 += 2;
+  }
+  if (r0 < nrows) xy_rows(std::integral_constant<int, 1>{}, r0);
 
   // ---- delta_t by forward substitution and o_t, one thread per value column
   IO* o_base = out + ((int64_t)b * W * H + h) * DV;
