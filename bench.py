@@ -19,7 +19,8 @@ buffers through kda_fwd_host ("e2e"), and the other prefill workloads
 ("workloads": the mid batch B=2 H=16 T=4096 plain and through kda_fwd_cp,
 one tensor-parallel rank's 4 heads of the 64K prefill plain and through
 kda_fwd_cp, the packed 1M-token batch, the model-range decay cases, the 64K
-prefill with 512-token checkpoints and with the fused prologue).
+prefill with 512-token checkpoints and with the fused prologue, and one rank's
+compute of the 64K prefill split over 8 ranks by KCP).
 Inputs are synthetic (seeded) and resident in HBM before the timed region;
 workloads smaller than the 126 MB L2 (or close to it) get an L2 flush before
 every timed launch, the others are far larger than L2.
@@ -461,6 +462,8 @@ def run_native(args, d):
             res, _ = bench_prefill(name, d, dev, stream, peaks, kda, synth, steps, args.warmup, variant=variant)
             others[key] = res
             torch.cuda.empty_cache()
+        others["kcp8_rank"] = bench_kcp_rank(args, d, dev, stream, kda, synth, main["ms_per_step"])
+        torch.cuda.empty_cache()
         line["workloads"] = others
     if d.world == 1 and d.rank == 0 and not args.no_cpu_baseline:
         import oracle
@@ -511,6 +514,63 @@ def bench_decode(args, d, dev, stream, peaks, kda, synth, gated=False):
             "roofline": {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": ach / peaks["hbm_gbs"], "traffic": traffic, "bytes_per_launch": nbytes,
                          "kernel": "kda_decode_kernel<128,128,bf16>"}}
+
+
+def bench_kcp_rank(args, d, dev, stream, kda, synth, one_gpu_ms, R=8, steps=10):
+    """One rank's compute of KDA context parallelism across R ranks (KCP) for
+    the 64K prefill (B=1, H=96): the rank holds 65536 / R consecutive tokens
+    and runs its segment pieces (zero-start outputs and state, transformed
+    queries, transition), the composition of the R gathered pieces in rank
+    order and the correction of its outputs.  The all-gather of (M, S~)
+    between the pieces and the composition needs R GPUs and is not timed:
+    its bytes per rank are reported.  speedup_compute_only = the one-GPU
+    prefill's time over this rank's."""
+    import ctypes
+    import torch
+    spec = synth.PRETRAIN
+    T, H, dk, dv = spec.T // R, spec.H, spec.dk, spec.dv
+    inp = synth.make_prefill(spec, dev, T=T)
+    q, k, v, g, beta = inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"]
+    out_zero = torch.empty((1, T, H, dv), dtype=torch.float32, device=dev)
+    qhat = torch.empty((1, T, H, dk), dtype=torch.float32, device=dev)
+    s_zero = torch.empty((R, H, dk, dv), dtype=torch.float32, device=dev)  # this rank's piece + the gathered ones
+    trans = torch.empty((R, H, dk, dk), dtype=torch.float32, device=dev)
+    state_in = torch.empty_like(s_zero)
+    final = torch.empty((1, H, dk, dv), dtype=torch.float32, device=dev)
+    out = torch.empty((1, T, H, dv), dtype=spec.dtype, device=dev)
+    ws = kda.alloc_workspace(1, T, H, dk, dv, spec.dtype, dev)
+    lib, ptr, sp = kda.lib(), kda._ptr, kda._stream_ptr(stream)
+    rank = R // 2
+    # the other ranks' pieces stand in as copies of this one (the composition's
+    # cost does not depend on the values)
+    code = lib.kda_segment_fwd(ptr(q), ptr(k), ptr(v), ptr(g), ptr(beta), ptr(out_zero), ptr(s_zero[0]),
+                               ptr(qhat), ptr(trans[0]), 1, T, H, dk, dv, None, sp, kda._DT[q.dtype], ptr(ws),
+                               ws.numel())
+    kda._check(code, "kda_segment_fwd")
+    torch.cuda.synchronize()
+    s_zero[1:].copy_(s_zero[0].expand(R - 1, -1, -1, -1))
+    trans[1:].copy_(trans[0].expand(R - 1, -1, -1, -1))
+    s_mine, t_mine, s_in_mine = s_zero[rank], trans[rank], state_in[rank]
+
+    def step():
+        kda._check(lib.kda_segment_fwd(ptr(q), ptr(k), ptr(v), ptr(g), ptr(beta), ptr(out_zero), ptr(s_mine),
+                                       ptr(qhat), ptr(t_mine), 1, T, H, dk, dv, None, sp, kda._DT[q.dtype],
+                                       ptr(ws), ws.numel()), "kda_segment_fwd")
+        kda._check(lib.kda_state_compose(ptr(trans), ptr(s_zero), None, ptr(state_in), ptr(final), R, 1, H, dk, dv,
+                                         1, sp), "kda_state_compose")
+        kda._check(lib.kda_output_correct(ptr(out_zero), ptr(qhat), ptr(s_in_mine), ptr(out), 1, T, H, dk, dv, None,
+                                          sp, kda._DT[out.dtype]), "kda_output_correct")
+
+    sec = time_loop(step, steps, args.warmup, stream, d)
+    ms = d.max(sec) / steps * 1e3
+    gather_bytes = H * (dk * dk + dk * dv) * 4
+    res = {"workload": f"kcp_rank_of_{R}_prefill_bf16_B1_H{H}_T{spec.T}_d{dk}", "tokens_per_rank": T,
+           "value": job_throughput(d, T * H * steps, sec) / 1e6, "unit": UNIT, "ms_per_step": ms,
+           "gpu_launches": 3 * steps, "speedup_compute_only": one_gpu_ms / ms,
+           "allgather": {"bytes_sent_per_rank": gather_bytes, "bytes_received_per_rank": (R - 1) * gather_bytes,
+                         "timed": False, "why": "needs R GPUs; one here"}}
+    del inp, q, k, v, g, beta, out_zero, qhat, s_zero, trans, state_in, final, out, ws
+    return res
 
 
 def bench_spec(args, d, dev, stream, peaks, kda, synth, W=4, sweep=(1, 2, 4, 8)):
@@ -716,7 +776,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-workloads", action="store_true",
-                    help="skip the other workload objects (mid, tp4, varlen, stress, model range, checkpoints, gated)")
+                    help="skip the other workload objects (mid, tp4, varlen, stress, model range, checkpoints, gated, KCP rank)")
     ap.add_argument("--capture", choices=sorted(CAPTURES), default=None,
                     help="run --steps launches of a small case (for ncu), nothing else")
     ap.add_argument("--phases", action="store_true",
