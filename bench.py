@@ -525,7 +525,6 @@ def bench_kcp_rank(args, d, dev, stream, kda, synth, one_gpu_ms, R=8, steps=10):
     between the pieces and the composition needs R GPUs and is not timed:
     its bytes per rank are reported.  speedup_compute_only = the one-GPU
     prefill's time over this rank's."""
-    import ctypes
     import torch
     spec = synth.PRETRAIN
     T, H, dk, dv = spec.T // R, spec.H, spec.dk, spec.dv
